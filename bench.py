@@ -1,0 +1,480 @@
+#!/usr/bin/env python
+"""Benchmark: MoE FFN layer forward throughput on B200, one JSON line on rank 0.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config quartz] [--impl ours|reference]
+
+A step is one whole layer forward (route -> permute -> grouped expert GEMMs -> combine -> loss)
+over one batch of seeded synthetic tokens, inputs resident in HBM. With N > 1 (torchrun, one
+process per GPU) every rank runs its own batch of T tokens (weak scaling, data-parallel replicas);
+the only exchange is an NCCL all-reduce of the 2E per-expert statistics that the global
+load-balancing loss needs.
+
+Timing: W untimed warm-up steps; then K steps, each bracketed by CUDA events on the launching
+stream, with a 256 MiB write between steps (outside the events) to flush the 126 MB L2; a
+barrier and a device synchronise on both sides; the max over ranks. SM clocks are sampled with
+NVML during the timed region. A second pass of K steps with the library's per-kernel event
+profiler gives the per-kernel durations for the roofline figures; a third pass times the same
+steps end to end through the public API with pinned host buffers (x in, y and the loss out).
+
+--impl reference times the CPU oracle (the only other implementation of this path) on a bounded
+token sample of the same workload, on rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "MoE layer fwd tokens/s on 1 B200; grouped-GEMM % bf16 peak; permute % HBM BW"
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                  "sm_max_mhz": 1965.0}
+FLUSH_BYTES = 256 << 20
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as fh:
+            d = json.load(fh)
+        return d, "measured"
+    except Exception:
+        return dict(PEAKS_FALLBACK), "fallback"
+
+
+def workload_name(c) -> str:
+    parts = [f"{c.name}: T={c.T} d={c.d} E={c.E} top-{c.top_k} {c.score}"]
+    if c.expert == "swiglu":
+        parts.append(f"SwiGLU ffn {c.ffn}")
+    else:
+        parts.append(f"low-rank r={c.rank}")
+    parts.append(f"{c.n_shared} shared" + (f" (ffn {c.ffn_shared})" if c.n_shared else ""))
+    parts.append("dropless" if c.capacity_factor <= 0 else f"capacity factor {c.capacity_factor}")
+    parts.append(c.dtype)
+    return ", ".join(parts)
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x100: "display_clock_setting"}
+
+    def __init__(self, index: int):
+        self.samples = []
+        self.reasons = 0
+        self.ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.max_mhz = None
+        self._stop = threading.Event()
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                try:
+                    r = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                except Exception:
+                    r = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
+                self.reasons |= int(r)
+            except Exception:
+                pass
+            time.sleep(0.002)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        names = [n for b, n in self.REASONS.items() if self.reasons & b and b != 0x1]
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": names, "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------------ algorithmic work
+def algorithmic(c, n_kept: int):
+    """Per-launch algorithmic flops / bytes of each kernel kind (kept rows only, each input
+    read once, no tile padding)."""
+    T, d, E, k, S, fs = c.T, c.d, c.E, c.top_k, c.n_shared, c.ffn_shared
+    es = 2 if c.dtype == "bf16" else 4
+    out = {}
+    out["router"] = {"flops": 2.0 * T * d * E, "bytes": T * d * es + E * d * es + 8.0 * T * k}
+    out["router_prep"] = {"bytes": E * d * (es + 8.0)}
+    perm_bytes = T * d * es + n_kept * d * es + 16.0 * T * k
+    out["perm_scatter"] = {"bytes": perm_bytes}
+    if c.expert == "swiglu":
+        f = c.ffn
+        out["gemm_gateup"] = {"flops": 4.0 * d * f * n_kept + 4.0 * d * S * fs * T}
+        out["gemm_down"] = {"flops": 2.0 * d * f * n_kept + 2.0 * d * S * fs * T}
+    else:
+        r = c.rank
+        out["gemm_lowrank_v"] = {"flops": 2.0 * d * r * n_kept}
+        out["gemm_lowrank_u"] = {"flops": 2.0 * d * r * n_kept}
+        if S:
+            out["gemm_gateup"] = {"flops": 4.0 * d * S * fs * T}
+            out["gemm_down"] = {"flops": 2.0 * d * S * fs * T}
+    out["combine"] = {"bytes": n_kept * d * 4.0 + (T * d * 4.0 if S else 0) + 8.0 * T * k +
+                      T * d * 4.0}
+    return out
+
+
+def roofline_table(c, n_kept, prof, steps, peaks, src):
+    """Achieved vs peak per kernel kind from the profiler's per-launch averages."""
+    alg = algorithmic(c, n_kept)
+    fp64_peak = 148 * 64 * 2 * peaks.get("sm_max_mhz", 1965.0) * 1e6 / 1e12  # TFLOP/s, nominal
+    rows = {}
+    for name, (ms, n) in prof.items():
+        if n == 0:
+            continue
+        avg_ms = ms / n
+        a = alg.get(name, {})
+        row = {"launches": n, "avg_us": avg_ms * 1e3, "share": None}
+        if name.startswith("gemm"):
+            ach = a["flops"] / (avg_ms * 1e-3) / 1e12
+            row.update(bound="tensor", achieved=ach, peak=peaks["bf16_tflops"], unit="TFLOP/s",
+                       frac=ach / peaks["bf16_tflops"])
+        elif name == "router":
+            ach = a["flops"] / (avg_ms * 1e-3) / 1e12
+            row.update(bound="alu", achieved=ach, peak=fp64_peak, unit="TFLOP/s (fp64 FMA)",
+                       frac=ach / fp64_peak,
+                       hbm_gbs=a["bytes"] / (avg_ms * 1e-3) / 1e9)
+        elif "bytes" in a:
+            ach = a["bytes"] / (avg_ms * 1e-3) / 1e9
+            row.update(bound="hbm", achieved=ach, peak=peaks["hbm_gbs"], unit="GB/s",
+                       frac=ach / peaks["hbm_gbs"])
+        rows[name] = row
+    tot = sum(ms for ms, n in prof.values())
+    for name, (ms, n) in prof.items():
+        if name in rows:
+            rows[name]["share"] = ms / tot if tot else None
+    return rows
+
+
+# ------------------------------------------------------------------ our arm
+def run_ours(args, rank, world, local_rank):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    import fine_grained_mixture_moe_b200 as moe
+    from fine_grained_mixture_moe_b200 import binding as B
+    from fine_grained_mixture_moe_b200.layer import MoELayer, upload_weights
+    from moe_synth import get_config, make_inputs
+
+    from fine_grained_mixture_moe_b200 import build as _b
+    if rank == 0:
+        _b.build()
+    if world > 1:
+        dist.barrier()
+    moe.load()
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    c = get_config(args.config)
+    inp = make_inputs(c)
+    cfg = B.make_config(T=c.T, d=c.d, E=c.E, top_k=c.top_k, n_shared=c.n_shared, ffn=c.ffn,
+                        ffn_shared=c.ffn_shared, rank=c.rank, score=c.score, expert=c.expert,
+                        dtype=c.dtype, norm_topk=c.norm_topk, capacity_factor=c.capacity_factor,
+                        aux_alpha=c.aux_alpha)
+    weights = upload_weights(cfg, inp, dev)
+    layer = MoELayer(cfg, weights, dev)
+    dt = layer.dtype
+    x = torch.as_tensor(inp["x"]).to(dt).contiguous().to(dev)
+    y = torch.empty((c.T, c.d), dtype=torch.float32, device=dev)
+    aux = torch.empty((), dtype=torch.float32, device=dev)
+    cnt = torch.empty(c.E, dtype=torch.int32, device=dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    # multi-GPU: route -> all-reduce(count, prob_sum) -> rest, loss over all ranks' tokens
+    if world > 1:
+        T, k, E, d = c.T, c.top_k, c.E, c.d
+        idx = torch.empty((T, k), dtype=torch.int32, device=dev)
+        wts = torch.empty((T, k), dtype=torch.float32, device=dev)
+        stats = torch.empty(2 * E, dtype=torch.float32, device=dev)
+        cnt32 = torch.empty(E, dtype=torch.int32, device=dev)
+        prob = stats[E:]
+        offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
+        slot = torch.empty((T, k), dtype=torch.int32, device=dev)
+        src = torch.empty(T * k, dtype=torch.int32, device=dev)
+        xp = torch.empty((T * k, d), dtype=dt, device=dev)
+        yp = torch.empty((T * k, d), dtype=torch.float32, device=dev)
+        ysh = torch.empty((T, d), dtype=torch.float32, device=dev) if c.n_shared else None
+        gcfg = B.make_config(T=T * world, d=c.d, E=E, top_k=k, n_shared=c.n_shared, ffn=c.ffn,
+                             ffn_shared=c.ffn_shared, rank=c.rank, score=c.score,
+                             expert=c.expert, dtype=c.dtype, norm_topk=c.norm_topk,
+                             capacity_factor=c.capacity_factor, aux_alpha=c.aux_alpha)
+        gcnt = torch.empty(E, dtype=torch.int32, device=dev)
+
+        def step():
+            B.moe_route(cfg, x, layer.wstruct, idx, wts, cnt32, prob, layer.ws, layer.ws_bytes)
+            stats[:E].copy_(cnt32)                      # counts < 2^24: exact in fp32
+            dist.all_reduce(stats)
+            B.moe_permute(cfg, x, idx, offsets, slot, src, xp, layer.ws, layer.ws_bytes)
+            B.moe_expert_forward(cfg, xp, offsets, x, layer.wstruct, yp, ysh, layer.ws,
+                                 layer.ws_bytes)
+            B.moe_combine(cfg, yp, ysh, slot, wts, y)
+            gcnt.copy_(stats[:E])
+            B.moe_aux_loss(gcfg, gcnt, prob, aux)
+    else:
+        def step():
+            layer.forward(x, y, aux, cnt)
+
+    def timed(K, pre=None):
+        starts = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+        ends = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        for i in range(K):
+            flush.fill_(i & 0xff)
+            if pre:
+                pre(i)
+            starts[i].record(stream)
+            step()
+            ends[i].record(stream)
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        return [s.elapsed_time(e) for s, e in zip(starts, ends)]
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    st, info = B.moe_get_device_error()
+    if st != 0:
+        raise RuntimeError(f"device error after warm-up: {B.status_str(st)} info={info}")
+    n_kept = int(torch.as_tensor(cnt).sum()) if c.capacity_factor <= 0 else None
+    if n_kept is None or world > 1:
+        offs = torch.empty(c.E + 1, dtype=torch.int32, device=dev)
+        tmp_idx = torch.empty((c.T, c.top_k), dtype=torch.int32, device=dev)
+        tmp_w = torch.empty((c.T, c.top_k), dtype=torch.float32, device=dev)
+        tmp_c = torch.empty(c.E, dtype=torch.int32, device=dev)
+        tmp_p = torch.empty(c.E, dtype=torch.float32, device=dev)
+        B.moe_route(cfg, x, layer.wstruct, tmp_idx, tmp_w, tmp_c, tmp_p, layer.ws, layer.ws_bytes)
+        sl = torch.empty((c.T, c.top_k), dtype=torch.int32, device=dev)
+        sr = torch.empty(c.T * c.top_k, dtype=torch.int32, device=dev)
+        B.moe_permute(cfg, x, tmp_idx, offs, sl, sr, None, layer.ws, layer.ws_bytes)
+        torch.cuda.synchronize()
+        n_kept = int(offs[-1])
+        counts = tmp_c.cpu().numpy()
+    else:
+        counts = cnt.cpu().numpy()
+
+    # pass 1: the number
+    with ClockSampler(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ
+                      else local_rank) as clk:
+        times = timed(args.steps)
+    ms = statistics.fmean(times)
+    if world > 1:
+        t = torch.tensor([ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t)
+    st, info = B.moe_get_device_error()
+    if st != 0:
+        raise RuntimeError(f"device error in the timed region: {B.status_str(st)} info={info}")
+
+    # pass 2: per-kernel durations (library event profiler, same steps)
+    B.moe_debug_set(B.DEBUG_PROFILE, 1)
+    timed(args.steps)
+    prof = B.moe_profile_read()
+    B.moe_debug_set(B.DEBUG_PROFILE, 0)
+
+    # pass 3: end to end through the public API with pinned host buffers
+    x_host = torch.empty_like(x, device="cpu").pin_memory()
+    x_host.copy_(x.cpu())
+    y_host = torch.empty_like(y, device="cpu").pin_memory()
+    aux_host = torch.empty((), dtype=torch.float32).pin_memory()
+
+    def e2e_step():
+        x.copy_(x_host, non_blocking=True)
+        step()
+        y_host.copy_(y, non_blocking=True)
+        aux_host.copy_(aux, non_blocking=True)
+
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        flush.fill_(i & 0xff)
+        starts[i].record(stream)
+        e2e_step()
+        ends[i].record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = statistics.fmean(s.elapsed_time(e) for s, e in zip(starts, ends))
+    if world > 1:
+        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t)
+    h2d = x.numel() * x.element_size()
+    d2h = y.numel() * y.element_size() + 4
+
+    peaks, peak_src = load_peaks()
+    table = roofline_table(c, n_kept, prof, args.steps, peaks, peak_src)
+    dom = max(table, key=lambda n: table[n]["share"] or 0.0)
+    dr = table[dom]
+    launches_per_step = sum(n for _, n in prof.values()) / max(args.steps, 1)
+    tokens = c.T * world
+    result = {
+        "metric": METRIC,
+        "value": tokens / (ms * 1e-3),
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": c.dtype,
+        "data": "synthetic: seeded torch CPU generator, bf16-rounded N(0,1) tokens and "
+                "random-init weights of the configuration's shapes (no dataset, no checkpoint)",
+        "config": {
+            "workload": workload_name(c),
+            "tokens_per_gpu": c.T,
+            "l2": "flushed between timed steps (256 MiB write outside the events)",
+            "parallelism": f"dp{world} replicas" + (" + NCCL all-reduce of 2E expert stats"
+                                                     if world > 1 else ""),
+            "kept_pairs": n_kept,
+            "expert_rows_min_max": [int(counts.min()), int(counts.max())],
+            "dead_experts": int((counts == 0).sum()),
+            "kernels": {k: {kk: (round(vv, 4) if isinstance(vv, float) else vv)
+                            for kk, vv in v.items()} for k, v in table.items()},
+            "peaks": f"{peak_src} (MEASURED_PEAKS.json)" if peak_src == "measured" else
+                     "fallback pool figures",
+        },
+        "roofline": {"kernel": dom, "bound": dr.get("bound"), "achieved": dr.get("achieved"),
+                     "peak": dr.get("peak"), "unit": dr.get("unit"), "frac": dr.get("frac"),
+                     "traffic": None,
+                     "peak_kind": f"{peak_src} burst" if dr.get("bound") == "tensor" else peak_src},
+        "e2e": {"value": tokens / (e2e_ms * 1e-3), "unit": "tokens/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "gpu_launches": int(round(launches_per_step * args.steps)),
+        "clocks": clk.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        result["cpu_baseline"] = cpu_baseline(c, inp)
+    return result
+
+
+def _threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [p.get("num_threads", 1) for p in threadpool_info()]
+        return max(n) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(c, inp, T_sample=None):
+    """The oracle, as it stands, on a bounded token sample of the same workload."""
+    import oracle
+    T = c.T if T_sample is None else T_sample
+    sub = dict(inp)
+    sub["x"] = inp["x"][:T]
+    cs = c.with_(T=T)
+    t0 = time.perf_counter()
+    oracle.layer_forward(cs, sub)
+    dt = time.perf_counter() - t0
+    return {"value": T / dt, "unit": "tokens/s", "cores": _threads(), "kind": "oracle",
+            "sample": f"one layer forward over the first {T} tokens of the workload "
+                      f"({dt:.1f} s, fp64 numpy/OpenBLAS)"}
+
+
+# ------------------------------------------------------------------ reference arm (oracle)
+def run_reference(args):
+    from moe_synth import get_config, make_inputs
+    c = get_config(args.config)
+    inp = make_inputs(c)
+    # size the token sample so that all K + W steps take about two minutes
+    per_token_s = 11.0 / 4096 * (c.d * (3 * c.ffn * c.top_k + 3 * c.ffn_shared * c.n_shared +
+                                        c.E) + (2 * c.d * c.rank * c.top_k)) / (1024 * (3 * 640 * 8 + 24))
+    budget = 120.0 / max(args.steps + args.warmup, 1)
+    T_s = int(max(32, min(c.T, budget / max(per_token_s, 1e-9))) // 32 * 32) or 32
+    import oracle
+    sub = dict(inp)
+    sub["x"] = inp["x"][:T_s]
+    cs = c.with_(T=T_s)
+    for _ in range(args.warmup):
+        oracle.layer_forward(cs, sub)
+    times = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        oracle.layer_forward(cs, sub)
+        times.append(time.perf_counter() - t0)
+    ms = statistics.fmean(times) * 1e3
+    v = T_s / (ms * 1e-3)
+    return {
+        "impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": workload_name(c), "tokens_per_step": T_s},
+        "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": _threads(), "kind": "oracle",
+                         "sample": f"first {T_s} tokens of the workload per step"},
+        "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--config", default="quartz")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return
+    if world > 1:
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    try:
+        res = run_ours(args, rank, world, local_rank)
+        if rank == 0:
+            print(json.dumps(res), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,14 @@
+"""B200-native forward pass of a DeepSeek-style fine-grained mixture-of-experts FFN layer.
+
+The compute path is the sm_100a CUDA library ``lib/libmoe.so`` behind the C ABI in
+``include/moe.h``; :mod:`.binding` marshals arguments to it and :class:`MoELayer` holds device
+weights and a workspace. The library is loaded lazily and there is no fallback path: without
+the built library every call raises.
+"""
+from .binding import (DEBUG_FORCE_EXACT, DEBUG_PROFILE, DEBUG_WAIT_LIMIT_NS, EXPORTED,  # noqa: F401
+                      MoEConfig, MoEError, MoEWeights, load, make_config, make_weights,
+                      moe_aux_loss, moe_capacity, moe_combine, moe_debug_set,
+                      moe_debug_wait_timeout_probe, moe_expert_forward, moe_get_device_error,
+                      moe_layer_forward, moe_permute, moe_profile_read, moe_route,
+                      moe_workspace_size, status_str)
+from .layer import MoELayer, torch_dtype, upload_weights  # noqa: F401

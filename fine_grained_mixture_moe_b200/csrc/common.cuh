@@ -1,0 +1,117 @@
+// Shared device-side helpers of the MoE library (one translation unit: moe_lib.cu).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/moe.h"
+
+namespace moe {
+
+// ------------------------------------------------------------------ device error word
+// First error wins; the host reads and clears it with moe_get_device_error().
+__device__ int g_err_code = 0;
+__device__ long long g_err_info = 0;
+__device__ int g_force_exact = 0;
+__device__ unsigned long long g_wait_limit_ns = 2000000000ull;
+
+// detail codes stored in g_err_info
+enum : long long {
+  INFO_SIGMOID_UNRESOLVED = 1,
+  INFO_EXPANSION_OVERFLOW = 2,
+  INFO_WAIT_TMA_FULL = 10,
+  INFO_WAIT_MMA_EMPTY = 11,
+  INFO_WAIT_ACC_FULL = 12,
+  INFO_WAIT_ACC_EMPTY = 13,
+  INFO_WAIT_DRAIN = 14,
+  INFO_WAIT_PROBE = 20,
+};
+
+__device__ __forceinline__ void set_device_error(int code, long long info) {
+  if (atomicCAS(&g_err_code, 0, code) == 0) g_err_info = info;
+}
+
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// ------------------------------------------------------------------ element conversion
+template <typename T> struct Elem;
+template <> struct Elem<float> {
+  static __device__ __forceinline__ float to_f(float v) { return v; }
+  static __device__ __forceinline__ float from_f(float v) { return v; }
+};
+template <> struct Elem<__nv_bfloat16> {
+  static __device__ __forceinline__ float to_f(__nv_bfloat16 v) { return __bfloat162float(v); }
+  static __device__ __forceinline__ __nv_bfloat16 from_f(float v) { return __float2bfloat16_rn(v); }
+};
+
+// ------------------------------------------------------------------ warp helpers
+__device__ __forceinline__ unsigned lanemask_lt() {
+  unsigned m;
+  asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+  return m;
+}
+
+__device__ __forceinline__ float warp_sum_f(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+__device__ __forceinline__ float warp_max_f(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+__device__ __forceinline__ double warp_sum_d(double v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// Inclusive warp scan of ints.
+__device__ __forceinline__ int warp_incl_scan(int v) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    int n = __shfl_up_sync(0xffffffffu, v, o);
+    if (lane >= o) v += n;
+  }
+  return v;
+}
+
+// Exclusive scan of `n` ints in shared memory `a` (in place) by the whole block; returns total.
+// blockDim.x must be a multiple of 32. `tmp` needs blockDim.x/32 + 1 ints.
+__device__ int block_excl_scan_inplace(int *a, int n, int *tmp) {
+  const int tid = threadIdx.x, nt = blockDim.x;
+  const int per = (n + nt - 1) / nt;
+  const int lo = min(n, tid * per), hi = min(n, lo + per);
+  int s = 0;
+  for (int i = lo; i < hi; ++i) s += a[i];
+  int incl = warp_incl_scan(s);
+  const int warp = tid >> 5, lane = tid & 31;
+  if (lane == 31) tmp[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    int nw = nt >> 5;
+    int v = lane < nw ? tmp[lane] : 0;
+    int vi = warp_incl_scan(v);
+    if (lane < nw) tmp[lane] = vi - v;
+    if (lane == 31) tmp[nw] = vi;
+  }
+  __syncthreads();
+  int run = tmp[warp] + incl - s;
+  for (int i = lo; i < hi; ++i) {
+    int v = a[i];
+    a[i] = run;
+    run += v;
+  }
+  int total = tmp[nt >> 5];
+  __syncthreads();
+  return total;
+}
+
+}  // namespace moe

@@ -1,0 +1,381 @@
+// bf16 grouped expert GEMM on the 5th-generation tensor cores (sm_100a).
+//
+// One persistent CTA per SM walks a device-side tile list built from the group offsets
+// (Moonfrost's stacked (E, hidden, ffn) expert tensors, here indexed by expert on the device so
+// the host never sees a count). Per CTA: 6 warps.
+//   warp 0  TMA producer: A tile [128 x 64] and B tile(s) [BN x 64] per k-block into a STAGES-
+//           deep shared-memory ring (128-byte swizzle, K-major), completion on `full[s]`.
+//   warp 1  TMEM owner and MMA issuer: one thread issues tcgen05.mma (kind::f16, bf16 x bf16 ->
+//           fp32, M=128, N=BN, K=16) into one of two TMEM accumulators; tcgen05.commit frees the
+//           smem stage (`empty[s]`) and, per tile, publishes the accumulator (`acc_full[b]`).
+//   warps 2-5 epilogue: tcgen05.ld (32 lanes x 16 columns per load) -> SwiGLU / scale -> bf16
+//           (hidden activations, the next GEMM's operand) or fp32 (expert outputs) -> global;
+//           then `acc_empty[b]`, so the next tile's MMAs overlap this epilogue.
+// GATEUP keeps gate and up in two TMEM accumulators of the same columns (2 x 128 fp32 columns
+// per buffer, 512 with double buffering), so silu(gate) * up is fused without a weight repack.
+// Every wait is bounded (global timer); on expiry the CTA records MOE_ERR_TIMEOUT, drains what
+// it has in flight (again bounded), frees its TMEM and returns.
+#pragma once
+#include <cuda.h>
+#include "grouped.cuh"
+
+namespace moe {
+
+constexpr int TC_BM = 128;
+constexpr int TC_BK = 64;  // one 128-byte swizzle atom of bf16
+constexpr int TC_THREADS = 192;
+
+struct TcMaps {
+  CUtensorMap a_r, a_s, b0_r, b1_r, b0_s, b1_s;
+};
+
+struct TcParams {
+  TcMaps maps;
+  GroupedGemm p;
+};
+
+template <int MODE, int BN> struct TcCfg {
+  static constexpr int NB = (MODE == MODE_GATEUP) ? 2 : 1;        // B tiles per stage
+  static constexpr int A_BYTES = TC_BM * TC_BK * 2;               // 16 KB
+  static constexpr int B_BYTES = BN * TC_BK * 2;
+  static constexpr int STAGE_BYTES = A_BYTES + NB * B_BYTES;
+  static constexpr int STAGES = (192 * 1024) / STAGE_BYTES > 8 ? 8 : (192 * 1024) / STAGE_BYTES;
+  static constexpr int ACC_COLS = NB * BN;                        // fp32 columns per buffer
+  static constexpr int TMEM_COLS = (2 * ACC_COLS <= 32) ? 32 : (2 * ACC_COLS <= 64) ? 64
+                                   : (2 * ACC_COLS <= 128) ? 128 : (2 * ACC_COLS <= 256) ? 256 : 512;
+  static_assert(2 * ACC_COLS <= 512, "TMEM holds 512 columns");
+  static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "UMMA N for M=128");
+  // instruction descriptor: D fp32, A/B bf16, both K-major, N>>3 at bit 17, M>>4 at bit 24
+  static constexpr uint32_t IDESC = (1u << 4) | (1u << 7) | (1u << 10) |
+                                    ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(TC_BM >> 4) << 24);
+};
+
+// ---------------------------------------------------------------- PTX wrappers
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
+}
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Bounded wait: true when the phase of `parity` completed; false on timeout or abort.
+__device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int *abort_flag,
+                                       uint64_t limit_ns, long long info) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*abort_flag) return false;
+    if (globaltimer_ns() - t0 > limit_ns) {
+      set_device_error(MOE_ERR_TIMEOUT, info);
+      *abort_flag = 1;
+      return false;
+    }
+  }
+}
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int c0, int c1,
+                                            uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"((uint64_t)map), "r"(c0), "r"(c1), "r"(bar)
+      : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+               : "memory");
+}
+__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                       uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// Shared-memory matrix descriptor: K-major, 128-byte swizzle, 8-row core groups 1024 B apart.
+__device__ __forceinline__ uint64_t make_sdesc(uint32_t saddr) {
+  uint64_t d = (uint64_t)((saddr & 0x3FFFFu) >> 4);
+  d |= (uint64_t)1 << 16;             // leading byte offset (unused for swizzled K-major)
+  d |= (uint64_t)(1024 >> 4) << 32;   // stride byte offset
+  d |= (uint64_t)1 << 46;             // descriptor version (sm_100)
+  d |= (uint64_t)2 << 61;             // SWIZZLE_128B
+  return d;
+}
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,"
+      "%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_wait_ld() {
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+template <int MODE, int BN>
+__host__ __device__ constexpr size_t tc_smem_bytes(int G) {
+  using C = TcCfg<MODE, BN>;
+  return 1024 /*alignment slack*/ + (size_t)C::STAGES * C::STAGE_BYTES + 256 /*barriers*/ +
+         (size_t)(G + 1 + TC_THREADS / 32 + 1) * sizeof(int);
+}
+
+template <int MODE, int BN>
+__global__ void __launch_bounds__(TC_THREADS, 1) gemm_tc_kernel(const __grid_constant__ TcParams P) {
+  using C = TcCfg<MODE, BN>;
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  const GroupedGemm &p = P.p;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int G = p.E + p.has_shared;
+
+  // carve shared memory (stages must be 1024-byte aligned for the 128-byte swizzle)
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t pad = ((raw + 1023u) & ~1023u) - raw;
+  unsigned char *base = smem_raw + pad;
+  unsigned char *stages = base;
+  uint64_t *bars = (uint64_t *)(base + (size_t)C::STAGES * C::STAGE_BYTES);
+  // bars: full[STAGES], empty[STAGES], acc_full[2], acc_empty[2], drain
+  uint32_t *tmem_slot = (uint32_t *)(bars + 2 * C::STAGES + 5);
+  volatile int *abort_flag = (volatile int *)(tmem_slot + 1);
+  int *prefix = (int *)(base + (size_t)C::STAGES * C::STAGE_BYTES + 256);
+  int *scan_tmp = prefix + G + 1;
+
+  auto full_bar = [&](int s) { return smem_u32(bars + s); };
+  auto empty_bar = [&](int s) { return smem_u32(bars + C::STAGES + s); };
+  auto accf_bar = [&](int b) { return smem_u32(bars + 2 * C::STAGES + b); };
+  auto acce_bar = [&](int b) { return smem_u32(bars + 2 * C::STAGES + 2 + b); };
+  const uint32_t drain_bar = smem_u32(bars + 2 * C::STAGES + 4);
+
+  if (tid == 0) {
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(accf_bar(b), 1);
+      mbar_init(acce_bar(b), 4);
+    }
+    mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(tmem_slot)),
+                 "r"((uint32_t)C::TMEM_COLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  if (warp == 0 && lane == 0) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)&P.maps.a_r) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)&P.maps.b0_r) : "memory");
+  }
+  const int total = build_tile_prefix(p, TC_BM, BN, prefix, scan_tmp);  // contains __syncthreads
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const uint64_t limit = g_wait_limit_ns;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int issued_parity[8];
+      bool issued[8];
+      for (int s = 0; s < 8; ++s) { issued[s] = false; issued_parity[s] = 0; }
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+        const TileInfo ti = decode_tile(p, tile, prefix, TC_BM, BN);
+        const bool routed = ti.g < p.E;
+        const CUtensorMap *ma = routed ? &P.maps.a_r : &P.maps.a_s;
+        const CUtensorMap *mb0 = routed ? &P.maps.b0_r : &P.maps.b0_s;
+        const CUtensorMap *mb1 = routed ? &P.maps.b1_r : &P.maps.b1_s;
+        const int a_row = ti.a_row0 + ti.m0;
+        const int nk = ti.K / TC_BK;
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, limit, INFO_WAIT_MMA_EMPTY)) {
+            ok = false;
+            break;
+          }
+          const uint32_t sA = smem_u32(stages + (size_t)stage * C::STAGE_BYTES);
+          const uint32_t sB0 = sA + C::A_BYTES;
+          mbar_expect_tx(full_bar(stage), C::STAGE_BYTES);
+          const int kk = kb * TC_BK;
+          int b_row, b_col;
+          if (routed) {
+            b_row = ti.g * ti.N + ti.n0;
+            b_col = kk;
+          } else {
+            const int piece = kk / p.piece_k;
+            b_row = piece * p.piece_rows + ti.n0;
+            b_col = kk - piece * p.piece_k;
+          }
+          tma_load_2d(sA, ma, kk, a_row, full_bar(stage));
+          tma_load_2d(sB0, mb0, b_col, b_row, full_bar(stage));
+          if (C::NB == 2) tma_load_2d(sB0 + C::B_BYTES, mb1, b_col, b_row, full_bar(stage));
+          issued[stage] = true;
+          issued_parity[stage] = (int)phase;
+          if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
+        }
+      }
+      if (!ok) {
+        // drain: every issued load completes its barrier phase before shared memory goes away
+        for (int s = 0; s < C::STAGES; ++s)
+          if (issued[s]) {
+            volatile int never = 0;
+            mbar_wait(full_bar(s), (uint32_t)issued_parity[s], &never, limit, INFO_WAIT_DRAIN);
+          }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true, any = false;
+      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+        const TileInfo ti = decode_tile(p, tile, prefix, TC_BM, BN);
+        const int nk = ti.K / TC_BK;
+        if (!mbar_wait(acce_bar(acc), acc_phase ^ 1u, abort_flag, limit, INFO_WAIT_ACC_EMPTY)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d0 = tmem_base + (uint32_t)(acc * C::ACC_COLS);
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!mbar_wait(full_bar(stage), phase, abort_flag, limit, INFO_WAIT_TMA_FULL)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sA = smem_u32(stages + (size_t)stage * C::STAGE_BYTES);
+          const uint32_t sB0 = sA + C::A_BYTES;
+#pragma unroll
+          for (int k16 = 0; k16 < TC_BK / 16; ++k16) {
+            const uint64_t ad = make_sdesc(sA + k16 * 32);
+            const uint64_t bd0 = make_sdesc(sB0 + k16 * 32);
+            const uint32_t accum = (kb > 0 || k16 > 0) ? 1u : 0u;
+            tc_mma(d0, ad, bd0, C::IDESC, accum);
+            if (C::NB == 2) {
+              const uint64_t bd1 = make_sdesc(sB0 + C::B_BYTES + k16 * 32);
+              tc_mma(d0 + BN, ad, bd1, C::IDESC, accum);
+            }
+          }
+          any = true;
+          tc_commit(empty_bar(stage));
+          if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        tc_commit(accf_bar(acc));
+        if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+      }
+      if (!ok && any) {
+        // wait until every MMA issued so far has completed before TMEM is released
+        tc_commit(drain_bar);
+        volatile int never = 0;
+        mbar_wait(drain_bar, 0u, &never, limit, INFO_WAIT_DRAIN);
+      }
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue (warps 2..5)
+    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+      const TileInfo ti = decode_tile(p, tile, prefix, TC_BM, BN);
+      const bool routed = ti.g < p.E;
+      bool ok = true;
+      if (lane == 0)
+        ok = mbar_wait(accf_bar(acc), acc_phase, abort_flag, limit, INFO_WAIT_ACC_FULL);
+      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+      if (!ok) break;
+      tc_fence_after();
+      const int row = ti.m0 + q * 32 + lane;
+      const bool row_ok = row < ti.rows;
+      void *out = routed ? p.out_r : p.out_s;
+      const int ldo = routed ? p.ldo_r : p.ldo_s;
+      const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * C::ACC_COLS);
+#pragma unroll 1
+      for (int c = 0; c < BN; c += 16) {
+        uint32_t r0[16], r1[16];
+        tmem_ld16(tbase + c, r0);
+        if (C::NB == 2) tmem_ld16(tbase + BN + c, r1);
+        tmem_wait_ld();
+        const int col = ti.n0 + c;
+        if (row_ok && col < ti.N) {
+          float v[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const float g = __uint_as_float(r0[i]);
+            if (MODE == MODE_GATEUP) v[i] = silu_f(g) * __uint_as_float(r1[i]);
+            else if (MODE == MODE_SCALE) v[i] = g * __ldg(p.scale + (size_t)ti.g * ti.N + col + i);
+            else v[i] = g;
+          }
+          if (MODE == MODE_PLAIN) {
+            // expert outputs stay fp32 (combined in fp32 downstream)
+            float4 *dst = (float4 *)((float *)out + (size_t)(ti.a_row0 + row) * ldo + col);
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+          } else {
+            uint4 pk[2];
+            __nv_bfloat162 *h = (__nv_bfloat162 *)pk;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) h[i] = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
+            uint4 *dst = (uint4 *)((__nv_bfloat16 *)out + (size_t)(ti.a_row0 + row) * ldo + col);
+            dst[0] = pk[0];
+            dst[1] = pk[1];
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(acce_bar(acc));
+      if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                 "r"((uint32_t)C::TMEM_COLS)
+                 : "memory");
+  }
+}
+
+}  // namespace moe

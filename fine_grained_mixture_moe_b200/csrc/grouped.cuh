@@ -1,0 +1,92 @@
+// Grouped-GEMM problem description shared by the tensor-core (bf16) and SIMT (fp32) kernels.
+//
+// A launch covers up to E routed groups plus one shared group:
+//   routed group g < E : rows offsets[g]..offsets[g+1] of A_r / out_r, weight B*_r + g*N_r*K_r
+//                        ([N_r, K_r] row-major, i.e. K-major), read from device memory only
+//   shared group g = E : rows 0..T of A_s / out_s, weight B*_s. Its K may be split into pieces
+//                        of width piece_k whose rows sit piece_rows apart: element (n, kk) of
+//                        B*_s is at ((kk / piece_k) * piece_rows + n) * piece_k + kk % piece_k.
+//                        This reads the shared down projections [S, d, fs] as one [d, S*fs]
+//                        matrix, so S shared experts of width fs act as one of width S*fs.
+// Epilogue modes: GATEUP out = silu(A B0^T) * (A B1^T) (SwiGLU, gate and up fused);
+//                 PLAIN  out = A B0^T;   SCALE out = (A B0^T) * scale[g][n] (low-rank s).
+#pragma once
+#include "common.cuh"
+
+namespace moe {
+
+enum GemmMode { MODE_GATEUP = 0, MODE_PLAIN = 1, MODE_SCALE = 2 };
+
+struct GroupedGemm {
+  const int32_t *offsets;  // [E+1] device
+  int E;                   // routed groups in this launch (0: shared only)
+  const void *A_r;
+  int lda_r;
+  int rows_r;              // rows held by the A_r / out_r buffers (T*top_k): tensor-map extent
+  const void *B0_r, *B1_r;
+  int N_r, K_r;
+  void *out_r;
+  int ldo_r;
+  const float *scale;  // [E, N_r] for MODE_SCALE
+  int has_shared, T;
+  const void *A_s;
+  int lda_s;
+  const void *B0_s, *B1_s;
+  int N_s, K_s, piece_k, piece_rows;
+  int b_rows_s;            // rows of the shared weight viewed as [b_rows_s, piece_k]
+  void *out_s;
+  int ldo_s;
+};
+
+// Tile counts per group and their exclusive prefix in shared memory (all threads call).
+__device__ __forceinline__ int build_tile_prefix(const GroupedGemm &p, int BM, int BN,
+                                                 int *prefix, int *tmp) {
+  const int G = p.E + p.has_shared;
+  const int ntr = (p.N_r + BN - 1) / BN, nts = (p.N_s + BN - 1) / BN;
+  for (int g = threadIdx.x; g < G; g += blockDim.x) {
+    const int rows = g < p.E ? (p.offsets[g + 1] - p.offsets[g]) : p.T;
+    prefix[g] = ((rows + BM - 1) / BM) * (g < p.E ? ntr : nts);
+  }
+  __syncthreads();
+  const int total = block_excl_scan_inplace(prefix, G, tmp);
+  if (threadIdx.x == 0) prefix[G] = total;
+  __syncthreads();
+  return total;
+}
+
+struct TileInfo {
+  int g, rows, m0, n0, N, K;
+  int a_row0;  // first row of the group in A / out
+};
+
+__device__ __forceinline__ TileInfo decode_tile(const GroupedGemm &p, int tile,
+                                                const int *prefix, int BM, int BN) {
+  const int G = p.E + p.has_shared;
+  int lo = 0, hi = G - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (prefix[mid] <= tile) lo = mid;
+    else hi = mid - 1;
+  }
+  TileInfo ti;
+  ti.g = lo;
+  const bool routed = lo < p.E;
+  ti.N = routed ? p.N_r : p.N_s;
+  ti.K = routed ? p.K_r : p.K_s;
+  const int nt = (ti.N + BN - 1) / BN;
+  const int local = tile - prefix[lo];
+  ti.m0 = (local / nt) * BM;
+  ti.n0 = (local % nt) * BN;
+  if (routed) {
+    ti.a_row0 = p.offsets[lo];
+    ti.rows = p.offsets[lo + 1] - ti.a_row0;
+  } else {
+    ti.a_row0 = 0;
+    ti.rows = p.T;
+  }
+  return ti;
+}
+
+__device__ __forceinline__ float silu_f(float z) { return z / (1.0f + expf(-z)); }
+
+}  // namespace moe

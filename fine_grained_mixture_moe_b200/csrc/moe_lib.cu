@@ -1,0 +1,678 @@
+// C ABI of the MoE FFN layer: argument checks, workspace layout, tensor maps and launches.
+// All kernels live in this one translation unit (the .cuh files), so the device error word and
+// the debug switches are single symbols without relocatable device code.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/moe.h"
+#include "combine.cuh"
+#include "common.cuh"
+#include "gemm_simt.cuh"
+#include "gemm_tc.cuh"
+#include "permute.cuh"
+#include "router.cuh"
+
+using namespace moe;
+
+namespace {
+
+// ------------------------------------------------------------------ validation
+bool cfg_supported(const moe_config_t *c) {
+  if (!c) return false;
+  if (c->T < 0 || c->d <= 0 || c->E <= 0 || c->top_k <= 0 || c->n_shared < 0) return false;
+  if (c->E > 1024 || c->top_k > 8 || c->top_k > c->E || c->n_shared > 8) return false;
+  if (c->d % 64) return false;
+  if (c->score != MOE_SCORE_SOFTMAX && c->score != MOE_SCORE_SIGMOID) return false;
+  if (c->dtype != MOE_DTYPE_F32 && c->dtype != MOE_DTYPE_BF16) return false;
+  if (c->expert == MOE_EXPERT_SWIGLU) {
+    if (c->ffn <= 0 || c->ffn % 64) return false;
+  } else if (c->expert == MOE_EXPERT_LOWRANK) {
+    if (c->rank <= 0 || c->rank % 64 || c->rank > 256) return false;
+  } else {
+    return false;
+  }
+  if (c->n_shared > 0 && (c->ffn_shared <= 0 || c->ffn_shared % 64)) return false;
+  if (!std::isfinite(c->capacity_factor) || !std::isfinite(c->aux_alpha)) return false;
+  // 32-bit row indices inside the kernels
+  if ((long long)c->T * c->top_k * std::max(c->d, 256) >= (1ll << 31) * 64ll) return false;
+  if ((long long)c->T * c->top_k >= (1ll << 31)) return false;
+  return true;
+}
+
+inline bool aligned16(const void *p) { return p && ((uintptr_t)p & 15u) == 0; }
+// token-sized buffers may be NULL in an empty call (T == 0)
+inline bool tok16(const moe_config_t *c, const void *p) {
+  return (c->T == 0 && p == nullptr) || aligned16(p);
+}
+inline size_t esize(const moe_config_t *c) { return c->dtype == MOE_DTYPE_BF16 ? 2 : 4; }
+inline int ceil_div(long long a, long long b) { return (int)((a + b - 1) / b); }
+inline size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
+
+// exact ceil(cf * T * k / E) on the fp32 value of cf (cf = m * 2^ex, m a 24-bit integer)
+int32_t capacity_of(const moe_config_t *c) {
+  const float cf = c->capacity_factor;
+  if (!(cf > 0.0f)) return -1;
+  int ex;
+  const float fr = std::frexp(cf, &ex);                 // cf = fr * 2^ex, 0.5 <= fr < 1
+  const long long m = (long long)std::ldexp(fr, 24);    // exact 24-bit integer
+  ex -= 24;                                            // cf = m * 2^ex
+  __int128 num = (__int128)m * c->T * c->top_k;        // cf*T*k = num * 2^ex
+  __int128 den = c->E;
+  if (ex >= 0) {
+    if (ex > 60) return 0x7fffffff;
+    num <<= ex;
+  } else {
+    if (-ex > 100) return num > 0 ? 1 : 0;
+    den <<= -ex;
+  }
+  __int128 q = num / den;
+  if (q * den < num) q += 1;
+  if (q > 0x7fffffff) return 0x7fffffff;
+  return (int32_t)q;
+}
+
+// ------------------------------------------------------------------ workspace layout
+struct Layout {
+  size_t w64, wnorm, part_cnt, part_prob, rcounter;             // route
+  size_t chunk_count, chunk_base, ptotal, pcounter;             // permute
+  size_t hidden, hidden_sh;                                     // experts
+  size_t idx, wts, count, prob, offsets, slot_pos, src, x_perm, y_perm, y_shared, aux;  // layer
+  size_t total;
+};
+
+Layout layout_of(const moe_config_t *c) {
+  Layout L;
+  const size_t T = c->T, d = c->d, E = c->E, k = c->top_k, es = esize(c);
+  const size_t nblk = std::max<size_t>(1, ceil_div(c->T, RT_TM));
+  const size_t nch = std::max<size_t>(1, ceil_div(c->T, PM_CHUNK));
+  const size_t width = c->expert == MOE_EXPERT_SWIGLU ? (size_t)c->ffn : (size_t)c->rank;
+  size_t o = 0;
+  auto take = [&](size_t bytes) { size_t at = o; o = align256(o + std::max<size_t>(bytes, 1)); return at; };
+  L.w64 = take(E * d * 8);
+  L.wnorm = take(E * 8);
+  L.part_cnt = take(nblk * E * 4);
+  L.part_prob = take(nblk * E * 4);
+  L.rcounter = take(16);
+  L.chunk_count = take(nch * E * 4);
+  L.chunk_base = take(nch * E * 4);
+  L.ptotal = take(E * 4);
+  L.pcounter = take(16);
+  L.hidden = take(T * k * width * es);
+  L.hidden_sh = take(T * (size_t)c->n_shared * (size_t)c->ffn_shared * es);
+  L.idx = take(T * k * 4);
+  L.wts = take(T * k * 4);
+  L.count = take(E * 4);
+  L.prob = take(E * 4);
+  L.offsets = take((E + 1) * 4);
+  L.slot_pos = take(T * k * 4);
+  L.src = take(T * k * 4);
+  L.x_perm = take(T * k * d * es);
+  L.y_perm = take(T * k * d * 4);    // expert outputs are fp32 for every dtype
+  L.y_shared = take(T * d * 4);
+  L.aux = take(16);
+  L.total = o;
+  return L;
+}
+
+template <typename T> T *at(void *ws, size_t off) { return (T *)((char *)ws + off); }
+
+// ------------------------------------------------------------------ device properties
+struct DevInfo {
+  int sms = 0;
+  bool tc_attr[8] = {};
+};
+DevInfo g_dev[64];
+
+int current_device() {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  return dev;
+}
+int num_sms() {
+  const int dev = current_device();
+  if (dev >= 0 && dev < 64) {
+    if (!g_dev[dev].sms) cudaDeviceGetAttribute(&g_dev[dev].sms, cudaDevAttrMultiProcessorCount, dev);
+    return g_dev[dev].sms;
+  }
+  int s = 0;
+  cudaDeviceGetAttribute(&s, cudaDevAttrMultiProcessorCount, dev);
+  return s;
+}
+
+// ------------------------------------------------------------------ profiling (debug)
+enum KernelKind {
+  K_ROUTER_PREP, K_ROUTER, K_PERM_HIST, K_PERM_SCAN, K_PERM_SCATTER, K_GEMM_GATEUP, K_GEMM_DOWN,
+  K_GEMM_LR1, K_GEMM_LR2, K_COMBINE, K_AUX, K_COUNT
+};
+const char *kKindName[K_COUNT] = {"router_prep", "router", "perm_hist", "perm_scan",
+                                  "perm_scatter", "gemm_gateup", "gemm_down", "gemm_lowrank_v",
+                                  "gemm_lowrank_u", "combine", "aux_loss"};
+constexpr int PROF_SLOTS = 8192;
+struct Prof {
+  bool on = false;
+  cudaEvent_t ev[2 * PROF_SLOTS];
+  int kind[PROF_SLOTS];
+  int n = 0;
+  bool created = false;
+} g_prof;
+std::mutex g_prof_mu;
+
+struct ProfScope {
+  int slot = -1;
+  cudaStream_t st;
+  ProfScope(int kind, cudaStream_t s) : st(s) {
+    if (!g_prof.on) return;
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    if (g_prof.n >= PROF_SLOTS) return;
+    slot = g_prof.n++;
+    g_prof.kind[slot] = kind;
+    cudaEventRecord(g_prof.ev[2 * slot], st);
+  }
+  ~ProfScope() {
+    if (slot >= 0) cudaEventRecord(g_prof.ev[2 * slot + 1], st);
+  }
+};
+
+moe_status_t last_launch_status() {
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+// ------------------------------------------------------------------ tensor maps
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    cudaDriverEntryPointQueryResult q;
+    void *f = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = (PFN_cuTensorMapEncodeTiled_v12000)f;
+  });
+  return fn;
+}
+
+// 2-D bf16 map over a row-major [rows, cols] matrix; box [box_rows, 64 columns], 128B swizzle.
+bool make_map(CUtensorMap *m, const void *ptr, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  if (rows == 0 || ptr == nullptr) {  // never dereferenced: map a dummy 1-row extent
+    rows = 1;
+  }
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 2};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(ptr), dims, strides,
+                        box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// ------------------------------------------------------------------ grouped GEMM launches
+long long tile_bound(const GroupedGemm &g, int BM, int BN) {
+  long long t = 0;
+  if (g.E > 0) t += ((long long)ceil_div(g.rows_r, BM) + g.E) * ceil_div(g.N_r, BN);
+  if (g.has_shared) t += (long long)ceil_div(g.T, BM) * ceil_div(g.N_s, BN);
+  return t;
+}
+
+template <int MODE, int BN>
+moe_status_t launch_tc(const GroupedGemm &g, cudaStream_t st, int kind) {
+  TcParams P;
+  std::memset(&P, 0, sizeof(P));
+  P.p = g;
+  const void *any = g.E > 0 ? g.A_r : g.A_s;
+  bool ok = true;
+  // routed operands: A [rows_r, K_r], B [E*N_r, K_r]; shared: A [T, K_s], B [b_rows_s, piece_k]
+  ok &= make_map(&P.maps.a_r, g.E > 0 ? g.A_r : any, g.E > 0 ? g.rows_r : 1,
+                 g.E > 0 ? g.K_r : 64, TC_BM);
+  ok &= make_map(&P.maps.b0_r, g.E > 0 ? g.B0_r : any, g.E > 0 ? (uint64_t)g.E * g.N_r : 1,
+                 g.E > 0 ? g.K_r : 64, BN);
+  ok &= make_map(&P.maps.b1_r, (g.E > 0 && MODE == MODE_GATEUP) ? g.B1_r : any,
+                 (g.E > 0 && MODE == MODE_GATEUP) ? (uint64_t)g.E * g.N_r : 1,
+                 g.E > 0 ? g.K_r : 64, BN);
+  ok &= make_map(&P.maps.a_s, g.has_shared ? g.A_s : any, g.has_shared ? g.T : 1,
+                 g.has_shared ? g.K_s : 64, TC_BM);
+  ok &= make_map(&P.maps.b0_s, g.has_shared ? g.B0_s : any, g.has_shared ? g.b_rows_s : 1,
+                 g.has_shared ? g.piece_k : 64, BN);
+  ok &= make_map(&P.maps.b1_s, (g.has_shared && MODE == MODE_GATEUP) ? g.B1_s : any,
+                 (g.has_shared && MODE == MODE_GATEUP) ? g.b_rows_s : 1,
+                 g.has_shared ? g.piece_k : 64, BN);
+  if (!ok) return MOE_ERR_CUDA;
+  const int G = g.E + g.has_shared;
+  const size_t smem = tc_smem_bytes<MODE, BN>(G);
+  auto kern = gemm_tc_kernel<MODE, BN>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  const long long bound = tile_bound(g, TC_BM, BN);
+  if (bound == 0) return MOE_OK;
+  const int grid = (int)std::min<long long>(num_sms(), bound);
+  ProfScope ps(kind, st);
+  kern<<<grid, TC_THREADS, smem, st>>>(P);
+  return last_launch_status();
+}
+
+template <int MODE>
+moe_status_t launch_simt(const GroupedGemm &g, cudaStream_t st, int kind) {
+  const int G = g.E + g.has_shared;
+  const size_t smem = (size_t)(G + 1 + 256 / 32 + 1) * sizeof(int);
+  auto kern = gemm_simt_kernel<float, float, MODE>;
+  if (smem > 48 * 1024 &&
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  const long long bound = tile_bound(g, SM_BM, SM_BN);
+  if (bound == 0) return MOE_OK;
+  const int grid = (int)std::min<long long>((long long)num_sms() * 8, bound);
+  ProfScope ps(kind, st);
+  kern<<<grid, 256, smem, st>>>(g);
+  return last_launch_status();
+}
+
+template <int MODE>
+moe_status_t launch_gemm(const moe_config_t *c, const GroupedGemm &g, int bn_hint,
+                         cudaStream_t st, int kind) {
+  if (c->dtype == MOE_DTYPE_F32) return launch_simt<MODE>(g, st, kind);
+  if (MODE == MODE_GATEUP) return launch_tc<MODE_GATEUP, 128>(g, st, kind);
+  if (MODE == MODE_SCALE) return launch_tc<MODE_SCALE, 64>(g, st, kind);
+  if (bn_hint == 256) return launch_tc<MODE_PLAIN, 256>(g, st, kind);
+  return launch_tc<MODE_PLAIN, 128>(g, st, kind);
+}
+
+// ------------------------------------------------------------------ steps
+#define MOE_TRY(expr)                   \
+  do {                                  \
+    const moe_status_t _s = (expr);     \
+    if (_s != MOE_OK) return _s;        \
+  } while (0)
+
+template <typename Tin>
+moe_status_t route_impl(const moe_config_t *c, const void *x, const moe_weights_t *w,
+                        int32_t *idx, float *wts, int32_t *count, float *prob, void *ws,
+                        cudaStream_t st) {
+  const Layout L = layout_of(c);
+  if (c->T == 0) {
+    if (cudaMemsetAsync(count, 0, (size_t)c->E * 4, st) != cudaSuccess) return MOE_ERR_CUDA;
+    if (cudaMemsetAsync(prob, 0, (size_t)c->E * 4, st) != cudaSuccess) return MOE_ERR_CUDA;
+    return MOE_OK;
+  }
+  RouterArgs a;
+  a.x = x;
+  a.w64 = at<double>(ws, L.w64);
+  a.wnorm = at<double>(ws, L.wnorm);
+  a.off = w->logit_offset;
+  a.bias = c->score == MOE_SCORE_SIGMOID ? w->select_bias : nullptr;
+  a.T = c->T; a.d = c->d; a.E = c->E; a.k = c->top_k; a.score = c->score; a.norm = c->norm_topk;
+  a.idx = idx; a.wts = wts;
+  a.part_cnt = at<int32_t>(ws, L.part_cnt);
+  a.part_prob = at<float>(ws, L.part_prob);
+  a.count_out = count; a.prob_out = prob;
+  a.counter = at<unsigned>(ws, L.rcounter);
+  {
+    ProfScope ps(K_ROUTER_PREP, st);
+    router_prep_kernel<Tin><<<c->E, 256, 0, st>>>((const Tin *)w->w_router, c->E, c->d,
+                                                   (double *)a.w64, (double *)a.wnorm, a.counter);
+    MOE_TRY(last_launch_status());
+  }
+  const size_t smem = router_smem_bytes(c->E);
+  if (cudaFuncSetAttribute(router_kernel<Tin>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  ProfScope ps(K_ROUTER, st);
+  router_kernel<Tin><<<ceil_div(c->T, RT_TM), RT_THREADS, smem, st>>>(a);
+  return last_launch_status();
+}
+
+template <typename Tin>
+moe_status_t permute_impl(const moe_config_t *c, const void *x, const int32_t *idx,
+                          int32_t *offsets, int32_t *slot_pos, int32_t *src, void *x_perm,
+                          void *ws, cudaStream_t st) {
+  const Layout L = layout_of(c);
+  if (c->T == 0) {
+    return cudaMemsetAsync(offsets, 0, (size_t)(c->E + 1) * 4, st) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+  }
+  const int nch = ceil_div(c->T, PM_CHUNK);
+  const int C = capacity_of(c);
+  int32_t *cc = at<int32_t>(ws, L.chunk_count), *cb = at<int32_t>(ws, L.chunk_base);
+  unsigned *counter = at<unsigned>(ws, L.pcounter);
+  {
+    const size_t smem = (size_t)8 * c->E * 4;
+    if (cudaFuncSetAttribute(perm_hist_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    ProfScope ps(K_PERM_HIST, st);
+    perm_hist_kernel<<<ceil_div(nch, 8), 256, smem, st>>>(idx, c->T, c->top_k, c->E, cc, nch, counter);
+    MOE_TRY(last_launch_status());
+  }
+  {
+    const size_t smem = (size_t)(c->E + 256 / 32 + 1) * 4;
+    ProfScope ps(K_PERM_SCAN, st);
+    perm_scan_kernel<<<ceil_div(c->E, 8), 256, smem, st>>>(cc, cb, nch, c->E, C,
+                                                           at<int32_t>(ws, L.ptotal), offsets, counter);
+    MOE_TRY(last_launch_status());
+  }
+  {
+    ProfScope ps(K_PERM_SCATTER, st);
+    perm_scatter_kernel<Tin><<<nch, 256, (size_t)c->E * 4, st>>>(
+        idx, c->T, c->top_k, c->E, C, cb, offsets, slot_pos, src, (const Tin *)x, (Tin *)x_perm, c->d);
+    return last_launch_status();
+  }
+}
+
+moe_status_t experts_impl(const moe_config_t *c, const void *x_perm, const int32_t *offsets,
+                          const void *x, const moe_weights_t *w, void *y_perm, void *y_shared,
+                          void *ws, cudaStream_t st) {
+  if (c->T == 0) return MOE_OK;
+  const Layout L = layout_of(c);
+  const int T = c->T, d = c->d, E = c->E, k = c->top_k, S = c->n_shared, fs = c->ffn_shared;
+  void *H = at<char>(ws, L.hidden);
+  void *Hs = at<char>(ws, L.hidden_sh);
+  GroupedGemm g;
+  std::memset(&g, 0, sizeof(g));
+  g.offsets = offsets;
+  g.T = T;
+  g.rows_r = T * k;
+  const bool sh = S > 0;
+  const int bn_down = (d % 256 == 0) ? 256 : 128;
+  if (c->expert == MOE_EXPERT_SWIGLU) {
+    const int f = c->ffn;
+    GroupedGemm g1 = g;
+    g1.E = E; g1.A_r = x_perm; g1.lda_r = d; g1.B0_r = w->w_gate; g1.B1_r = w->w_up;
+    g1.N_r = f; g1.K_r = d; g1.out_r = H; g1.ldo_r = f;
+    g1.has_shared = sh;
+    if (sh) {
+      g1.A_s = x; g1.lda_s = d; g1.B0_s = w->ws_gate; g1.B1_s = w->ws_up;
+      g1.N_s = S * fs; g1.K_s = d; g1.piece_k = d; g1.piece_rows = 0; g1.b_rows_s = S * fs;
+      g1.out_s = Hs; g1.ldo_s = S * fs;
+    }
+    MOE_TRY(launch_gemm<MODE_GATEUP>(c, g1, 128, st, K_GEMM_GATEUP));
+    GroupedGemm g2 = g;
+    g2.E = E; g2.A_r = H; g2.lda_r = f; g2.B0_r = w->w_down; g2.N_r = d; g2.K_r = f;
+    g2.out_r = y_perm; g2.ldo_r = d;
+    g2.has_shared = sh;
+    if (sh) {
+      g2.A_s = Hs; g2.lda_s = S * fs; g2.B0_s = w->ws_down; g2.N_s = d; g2.K_s = S * fs;
+      g2.piece_k = fs; g2.piece_rows = d; g2.b_rows_s = S * d; g2.out_s = y_shared; g2.ldo_s = d;
+    }
+    return launch_gemm<MODE_PLAIN>(c, g2, bn_down, st, K_GEMM_DOWN);
+  }
+  // low-rank experts: Z = (X V^T) * s  (rounded to dtype), then Y = Z U^T
+  const int r = c->rank;
+  GroupedGemm g1 = g;
+  g1.E = E; g1.A_r = x_perm; g1.lda_r = d; g1.B0_r = w->lr_V; g1.N_r = r; g1.K_r = d;
+  g1.out_r = H; g1.ldo_r = r; g1.scale = w->lr_s;
+  MOE_TRY(launch_gemm<MODE_SCALE>(c, g1, 64, st, K_GEMM_LR1));
+  GroupedGemm g2 = g;
+  g2.E = E; g2.A_r = H; g2.lda_r = r; g2.B0_r = w->lr_U; g2.N_r = d; g2.K_r = r;
+  g2.out_r = y_perm; g2.ldo_r = d;
+  MOE_TRY(launch_gemm<MODE_PLAIN>(c, g2, bn_down, st, K_GEMM_LR2));
+  if (sh) {
+    GroupedGemm g3 = g;
+    g3.E = 0; g3.has_shared = 1;
+    g3.A_s = x; g3.lda_s = d; g3.B0_s = w->ws_gate; g3.B1_s = w->ws_up;
+    g3.N_s = S * fs; g3.K_s = d; g3.piece_k = d; g3.piece_rows = 0; g3.b_rows_s = S * fs;
+    g3.out_s = Hs; g3.ldo_s = S * fs;
+    MOE_TRY(launch_gemm<MODE_GATEUP>(c, g3, 128, st, K_GEMM_GATEUP));
+    GroupedGemm g4 = g;
+    g4.E = 0; g4.has_shared = 1;
+    g4.A_s = Hs; g4.lda_s = S * fs; g4.B0_s = w->ws_down; g4.N_s = d; g4.K_s = S * fs;
+    g4.piece_k = fs; g4.piece_rows = d; g4.b_rows_s = S * d; g4.out_s = y_shared; g4.ldo_s = d;
+    MOE_TRY(launch_gemm<MODE_PLAIN>(c, g4, bn_down, st, K_GEMM_DOWN));
+  }
+  return MOE_OK;
+}
+
+moe_status_t combine_impl(const moe_config_t *c, const void *y_perm, const void *y_shared,
+                          const int32_t *slot_pos, const float *wts, void *y, cudaStream_t st) {
+  if (c->T == 0) return MOE_OK;
+  ProfScope ps(K_COMBINE, st);
+  const float *ysh = c->n_shared > 0 ? (const float *)y_shared : nullptr;
+  combine_kernel<<<ceil_div(c->T, 8), 256, 0, st>>>((const float *)y_perm, ysh, slot_pos, wts,
+                                                    (float *)y, c->T, c->top_k, c->d);
+  return last_launch_status();
+}
+
+moe_status_t aux_impl(const moe_config_t *c, const int32_t *count, const float *prob, float *loss,
+                      cudaStream_t st) {
+  ProfScope ps(K_AUX, st);
+  aux_loss_kernel<<<1, 32, 0, st>>>(count, prob, c->E, c->T, c->top_k, c->aux_alpha, loss);
+  return last_launch_status();
+}
+
+// ------------------------------------------------------------------ argument checks
+moe_status_t check_cfg(const moe_config_t *c) {
+  if (!c) return MOE_ERR_INVALID_ARG;
+  return cfg_supported(c) ? MOE_OK : MOE_ERR_UNSUPPORTED;
+}
+moe_status_t check_ws(const moe_config_t *c, void *ws, size_t bytes) {
+  if (!aligned16(ws)) return MOE_ERR_INVALID_ARG;
+  return bytes >= layout_of(c).total ? MOE_OK : MOE_ERR_WORKSPACE;
+}
+moe_status_t check_weights(const moe_config_t *c, const moe_weights_t *w, bool router,
+                           bool experts) {
+  if (!w) return MOE_ERR_INVALID_ARG;
+  if (router && !aligned16(w->w_router)) return MOE_ERR_INVALID_ARG;
+  if (experts) {
+    if (c->expert == MOE_EXPERT_SWIGLU) {
+      if (!aligned16(w->w_gate) || !aligned16(w->w_up) || !aligned16(w->w_down)) return MOE_ERR_INVALID_ARG;
+    } else {
+      if (!aligned16(w->lr_V) || !aligned16(w->lr_U) || !aligned16(w->lr_s)) return MOE_ERR_INVALID_ARG;
+    }
+    if (c->n_shared > 0 && (!aligned16(w->ws_gate) || !aligned16(w->ws_up) || !aligned16(w->ws_down)))
+      return MOE_ERR_INVALID_ARG;
+  }
+  return MOE_OK;
+}
+
+#define MOE_REQUIRE(cond) \
+  do {                    \
+    if (!(cond)) return MOE_ERR_INVALID_ARG; \
+  } while (0)
+
+}  // namespace
+
+// ================================================================== C ABI
+extern "C" {
+
+size_t moe_workspace_size(const moe_config_t *cfg) {
+  if (check_cfg(cfg) != MOE_OK) return 0;
+  return layout_of(cfg).total;
+}
+
+int32_t moe_capacity(const moe_config_t *cfg) {
+  if (check_cfg(cfg) != MOE_OK) return -2;
+  return capacity_of(cfg);
+}
+
+moe_status_t moe_route(const moe_config_t *cfg, const void *x, const moe_weights_t *w,
+                       int32_t *topk_idx, float *topk_w, int32_t *expert_count, float *prob_sum,
+                       void *ws, size_t ws_bytes, void *stream) {
+  MOE_TRY(check_cfg(cfg));
+  MOE_TRY(check_weights(cfg, w, true, false));
+  MOE_REQUIRE(tok16(cfg, x) && tok16(cfg, topk_idx) && tok16(cfg, topk_w) &&
+              aligned16(expert_count) && aligned16(prob_sum));
+  MOE_TRY(check_ws(cfg, ws, ws_bytes));
+  cudaStream_t st = (cudaStream_t)stream;
+  if (cfg->dtype == MOE_DTYPE_BF16)
+    return route_impl<__nv_bfloat16>(cfg, x, w, topk_idx, topk_w, expert_count, prob_sum, ws, st);
+  return route_impl<float>(cfg, x, w, topk_idx, topk_w, expert_count, prob_sum, ws, st);
+}
+
+moe_status_t moe_permute(const moe_config_t *cfg, const void *x, const int32_t *topk_idx,
+                         int32_t *offsets, int32_t *slot_pos, int32_t *src_token, void *x_perm,
+                         void *ws, size_t ws_bytes, void *stream) {
+  MOE_TRY(check_cfg(cfg));
+  MOE_REQUIRE(tok16(cfg, x) && tok16(cfg, topk_idx) && aligned16(offsets) && tok16(cfg, slot_pos) &&
+              tok16(cfg, src_token) && (x_perm == nullptr || aligned16(x_perm)));
+  MOE_TRY(check_ws(cfg, ws, ws_bytes));
+  cudaStream_t st = (cudaStream_t)stream;
+  if (cfg->dtype == MOE_DTYPE_BF16)
+    return permute_impl<__nv_bfloat16>(cfg, x, topk_idx, offsets, slot_pos, src_token, x_perm, ws, st);
+  return permute_impl<float>(cfg, x, topk_idx, offsets, slot_pos, src_token, x_perm, ws, st);
+}
+
+moe_status_t moe_expert_forward(const moe_config_t *cfg, const void *x_perm,
+                                const int32_t *offsets, const void *x, const moe_weights_t *w,
+                                void *y_perm, void *y_shared, void *ws, size_t ws_bytes,
+                                void *stream) {
+  MOE_TRY(check_cfg(cfg));
+  MOE_TRY(check_weights(cfg, w, false, true));
+  MOE_REQUIRE(tok16(cfg, x_perm) && aligned16(offsets) && tok16(cfg, x) && tok16(cfg, y_perm));
+  MOE_REQUIRE(cfg->n_shared == 0 || tok16(cfg, y_shared));
+  MOE_TRY(check_ws(cfg, ws, ws_bytes));
+  return experts_impl(cfg, x_perm, offsets, x, w, y_perm, y_shared, ws, (cudaStream_t)stream);
+}
+
+moe_status_t moe_combine(const moe_config_t *cfg, const void *y_perm, const void *y_shared,
+                         const int32_t *slot_pos, const float *topk_w, void *y, void *stream) {
+  MOE_TRY(check_cfg(cfg));
+  MOE_REQUIRE(tok16(cfg, y_perm) && tok16(cfg, slot_pos) && tok16(cfg, topk_w) && tok16(cfg, y));
+  MOE_REQUIRE(cfg->n_shared == 0 || tok16(cfg, y_shared));
+  return combine_impl(cfg, y_perm, y_shared, slot_pos, topk_w, y, (cudaStream_t)stream);
+}
+
+moe_status_t moe_aux_loss(const moe_config_t *cfg, const int32_t *expert_count,
+                          const float *prob_sum, float *loss, void *stream) {
+  MOE_TRY(check_cfg(cfg));
+  MOE_REQUIRE(aligned16(expert_count) && aligned16(prob_sum) && loss != nullptr);
+  return aux_impl(cfg, expert_count, prob_sum, loss, (cudaStream_t)stream);
+}
+
+moe_status_t moe_layer_forward(const moe_config_t *cfg, const void *x, const moe_weights_t *w,
+                               void *y, float *aux_loss, int32_t *expert_count, void *ws,
+                               size_t ws_bytes, void *stream) {
+  MOE_TRY(check_cfg(cfg));
+  MOE_TRY(check_weights(cfg, w, true, true));
+  MOE_REQUIRE(tok16(cfg, x) && tok16(cfg, y));
+  MOE_REQUIRE(expert_count == nullptr || aligned16(expert_count));
+  MOE_TRY(check_ws(cfg, ws, ws_bytes));
+  const Layout L = layout_of(cfg);
+  cudaStream_t st = (cudaStream_t)stream;
+  int32_t *idx = at<int32_t>(ws, L.idx);
+  float *wts = at<float>(ws, L.wts);
+  int32_t *cnt = expert_count ? expert_count : at<int32_t>(ws, L.count);
+  float *prob = at<float>(ws, L.prob);
+  int32_t *offsets = at<int32_t>(ws, L.offsets);
+  int32_t *slot_pos = at<int32_t>(ws, L.slot_pos);
+  int32_t *src = at<int32_t>(ws, L.src);
+  void *x_perm = at<char>(ws, L.x_perm);
+  void *y_perm = at<char>(ws, L.y_perm);
+  void *y_sh = at<char>(ws, L.y_shared);
+  float *aux = aux_loss ? aux_loss : at<float>(ws, L.aux);
+  if (cfg->dtype == MOE_DTYPE_BF16) {
+    MOE_TRY(route_impl<__nv_bfloat16>(cfg, x, w, idx, wts, cnt, prob, ws, st));
+    MOE_TRY(permute_impl<__nv_bfloat16>(cfg, x, idx, offsets, slot_pos, src, x_perm, ws, st));
+  } else {
+    MOE_TRY(route_impl<float>(cfg, x, w, idx, wts, cnt, prob, ws, st));
+    MOE_TRY(permute_impl<float>(cfg, x, idx, offsets, slot_pos, src, x_perm, ws, st));
+  }
+  MOE_TRY(experts_impl(cfg, x_perm, offsets, x, w, y_perm, y_sh, ws, st));
+  MOE_TRY(combine_impl(cfg, y_perm, y_sh, slot_pos, wts, y, st));
+  return aux_impl(cfg, cnt, prob, aux, st);
+}
+
+const char *moe_status_str(moe_status_t s) {
+  switch (s) {
+    case MOE_OK: return "MOE_OK";
+    case MOE_ERR_INVALID_ARG: return "MOE_ERR_INVALID_ARG: null or misaligned pointer";
+    case MOE_ERR_UNSUPPORTED: return "MOE_ERR_UNSUPPORTED: shape or option outside the supported set";
+    case MOE_ERR_WORKSPACE: return "MOE_ERR_WORKSPACE: workspace smaller than moe_workspace_size()";
+    case MOE_ERR_CUDA: return "MOE_ERR_CUDA: a CUDA runtime call failed";
+    case MOE_ERR_TIMEOUT: return "MOE_ERR_TIMEOUT: a bounded device-side wait ran out";
+    case MOE_ERR_DEVICE_CHECK: return "MOE_ERR_DEVICE_CHECK: a device-side check failed";
+  }
+  return "unknown moe_status_t";
+}
+
+moe_status_t moe_get_device_error(void *stream, int64_t *info) {
+  if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return MOE_ERR_CUDA;
+  int code = 0;
+  long long inf = 0;
+  if (cudaMemcpyFromSymbol(&code, g_err_code, sizeof(int)) != cudaSuccess) return MOE_ERR_CUDA;
+  if (cudaMemcpyFromSymbol(&inf, g_err_info, sizeof(long long)) != cudaSuccess) return MOE_ERR_CUDA;
+  const int zero = 0;
+  const long long zero64 = 0;
+  cudaMemcpyToSymbol(g_err_code, &zero, sizeof(int));
+  cudaMemcpyToSymbol(g_err_info, &zero64, sizeof(long long));
+  if (info) *info = inf;
+  return (moe_status_t)code;
+}
+
+moe_status_t moe_debug_set(int32_t what, int64_t value) {
+  switch (what) {
+    case MOE_DEBUG_FORCE_EXACT: {
+      const int v = value ? 1 : 0;
+      return cudaMemcpyToSymbol(g_force_exact, &v, sizeof(int)) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+    }
+    case MOE_DEBUG_WAIT_LIMIT_NS: {
+      if (value <= 0) return MOE_ERR_INVALID_ARG;
+      const unsigned long long v = (unsigned long long)value;
+      return cudaMemcpyToSymbol(g_wait_limit_ns, &v, sizeof(v)) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+    }
+    case MOE_DEBUG_PROFILE: {
+      std::lock_guard<std::mutex> lk(g_prof_mu);
+      if (value && !g_prof.created) {
+        for (int i = 0; i < 2 * PROF_SLOTS; ++i)
+          if (cudaEventCreate(&g_prof.ev[i]) != cudaSuccess) return MOE_ERR_CUDA;
+        g_prof.created = true;
+      }
+      g_prof.on = value != 0;
+      g_prof.n = 0;
+      return MOE_OK;
+    }
+  }
+  return MOE_ERR_INVALID_ARG;
+}
+
+int32_t moe_profile_read(const char **names, double *total_ms, int64_t *launches, int32_t max) {
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  if (!g_prof.created) return 0;
+  cudaDeviceSynchronize();
+  double ms[K_COUNT] = {0};
+  long long n[K_COUNT] = {0};
+  for (int i = 0; i < g_prof.n; ++i) {
+    float t = 0.0f;
+    if (cudaEventElapsedTime(&t, g_prof.ev[2 * i], g_prof.ev[2 * i + 1]) == cudaSuccess) {
+      ms[g_prof.kind[i]] += t;
+      n[g_prof.kind[i]] += 1;
+    }
+  }
+  g_prof.n = 0;
+  int out = 0;
+  for (int k = 0; k < K_COUNT; ++k) {
+    if (!n[k]) continue;
+    if (out < max) {
+      if (names) names[out] = kKindName[k];
+      if (total_ms) total_ms[out] = ms[k];
+      if (launches) launches[out] = n[k];
+    }
+    ++out;
+  }
+  return out;
+}
+
+}  // extern "C"
+
+namespace moe {
+__global__ void wait_probe_kernel() {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bar), 1);
+    abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+  // nothing ever arrives on `bar`: the bounded wait must expire and record MOE_ERR_TIMEOUT
+  if (threadIdx.x == 0) mbar_wait(smem_u32(&bar), 0u, &abort_flag, g_wait_limit_ns, INFO_WAIT_PROBE);
+}
+}  // namespace moe
+
+extern "C" moe_status_t moe_debug_wait_timeout_probe(void *stream) {
+  moe::wait_probe_kernel<<<1, 32, 0, (cudaStream_t)stream>>>();
+  return last_launch_status();
+}

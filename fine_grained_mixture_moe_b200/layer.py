@@ -1,0 +1,64 @@
+"""A layer object over the C ABI: device weights, a workspace, and one forward call.
+
+torch supplies the device memory and the stream; every step of the forward pass runs in the
+CUDA library (``moe_layer_forward``). Nothing here computes any part of the layer.
+"""
+from __future__ import annotations
+
+from typing import Dict, Optional
+
+import torch
+
+from . import binding as B
+
+TORCH_DTYPE = {B.DTYPE["f32"]: torch.float32, B.DTYPE["bf16"]: torch.bfloat16}
+
+# tensors in the layer's dtype vs. always-fp32 tensors
+FP32_WEIGHTS = ("logit_offset", "select_bias", "lr_s")
+
+
+def torch_dtype(cfg: B.MoEConfig) -> torch.dtype:
+    return TORCH_DTYPE[cfg.dtype]
+
+
+def upload_weights(cfg: B.MoEConfig, host: Dict[str, object], device) -> Dict[str, torch.Tensor]:
+    """Copy host arrays (numpy or torch, values exact in the layer dtype) to the device."""
+    dt = torch_dtype(cfg)
+    out = {}
+    for name, _ in B.MoEWeights._fields_:
+        a = host.get(name)
+        if a is None:
+            continue
+        t = torch.as_tensor(a)
+        t = t.to(torch.float32 if name in FP32_WEIGHTS else dt)
+        out[name] = t.contiguous().to(device)
+    return out
+
+
+class MoELayer:
+    """Owns the device weights and the workspace of one MoE FFN layer configuration."""
+
+    def __init__(self, cfg: B.MoEConfig, weights: Dict[str, torch.Tensor], device=None):
+        self.cfg = cfg
+        self.device = torch.device(device if device is not None else "cuda")
+        self.weights = weights
+        self.wstruct = B.make_weights(weights)
+        self.ws_bytes = B.moe_workspace_size(cfg)
+        if self.ws_bytes == 0:
+            raise B.MoEError("moe_workspace_size", 2)
+        self.ws = torch.empty(self.ws_bytes, dtype=torch.uint8, device=self.device)
+        self.dtype = torch_dtype(cfg)
+
+    def forward(self, x: torch.Tensor, y: Optional[torch.Tensor] = None,
+                aux: Optional[torch.Tensor] = None, expert_count: Optional[torch.Tensor] = None,
+                stream=None):
+        T, d = self.cfg.T, self.cfg.d
+        if y is None:
+            y = torch.empty((T, d), dtype=torch.float32, device=self.device)
+        if aux is None:
+            aux = torch.empty((), dtype=torch.float32, device=self.device)
+        B.moe_layer_forward(self.cfg, x, self.wstruct, y, aux, expert_count, self.ws,
+                            self.ws_bytes, stream)
+        return y, aux
+
+    __call__ = forward

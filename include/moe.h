@@ -1,0 +1,188 @@
+/*
+ * moe.h - C ABI of the B200 fine-grained mixture-of-experts FFN layer (forward pass).
+ *
+ * The layer is the DeepSeek-style fine-grained MoE FFN that the source pages describe:
+ *   - Vertex AGI research page / quartz-micro-preview-base model card, "Architecture":
+ *     24 narrow routed experts (FFN 640) at hidden 1,024, top-6, 2 always-active shared experts,
+ *     a 0.01-weighted load-balancing loss;
+ *   - Moonfrost, expert card: 32 routed experts + 1 shared, top-3, experts held as three stacked
+ *     (E, hidden, ffn) tensors with capacity-based routing instead of a per-expert loop;
+ *   - Sutra-1.3B, "48 + 1 experts": top-4 by sigmoid score with bias-based load balancing;
+ *   - dormouse, "dropless MoE" and "TSCT low-rank experts": 1,024 experts U*diag(s)*V^T of
+ *     rank 64, top-2, dropless.
+ *
+ * Conventions for every call:
+ *   - Ownership: the caller allocates every buffer. The library allocates no device or host
+ *     memory; scratch comes from a caller-provided workspace of moe_workspace_size() bytes.
+ *   - Pointers are device pointers unless stated otherwise, 16-byte aligned, row-major and
+ *     densely packed. "dtype" below means fp32 for MOE_DTYPE_F32 and bf16 for MOE_DTYPE_BF16.
+ *   - Asynchrony: calls only enqueue work on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream) and return. Argument errors are detected on the host and returned at once,
+ *     with nothing enqueued. Faults detected on the device (a bounded wait that ran out, an
+ *     internal consistency check) set a device error word that moe_get_device_error() reads.
+ *     No call aborts, exits or traps.
+ *   - Determinism: every output is bitwise reproducible run to run (no floating-point atomics).
+ *   - Shapes: d, ffn, ffn_shared and rank must be multiples of 64; 1 <= top_k <= min(E, 8);
+ *     1 <= E <= 1024; n_shared <= 8. T may be 0. Other values return MOE_ERR_UNSUPPORTED.
+ *   - Inputs must be finite. Router logits of +-inf or NaN make the routing unspecified.
+ */
+#ifndef MOE_H
+#define MOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,   /* null pointer, negative size, misaligned pointer */
+  MOE_ERR_UNSUPPORTED = 2,   /* a shape or option outside the supported set */
+  MOE_ERR_WORKSPACE = 3,     /* ws_bytes smaller than moe_workspace_size() */
+  MOE_ERR_CUDA = 4,          /* a CUDA runtime call failed (launch error, no device) */
+  MOE_ERR_TIMEOUT = 5,       /* device: a bounded wait ran out; the kernel returned early */
+  MOE_ERR_DEVICE_CHECK = 6   /* device: an internal check failed (see moe_get_device_error) */
+} moe_status_t;
+
+typedef enum { MOE_SCORE_SOFTMAX = 0, MOE_SCORE_SIGMOID = 1 } moe_score_t;
+typedef enum { MOE_EXPERT_SWIGLU = 0, MOE_EXPERT_LOWRANK = 1 } moe_expert_t;
+typedef enum { MOE_DTYPE_F32 = 0, MOE_DTYPE_BF16 = 1 } moe_dtype_t;
+
+/* Problem statement of one layer call (the arguments the pages' architecture tables give:
+ * hidden size, routed experts, top-k, shared experts, expert FFN width, scoring, capacity). */
+typedef struct {
+  int32_t T;            /* tokens in the call (batch x sequence, flattened) */
+  int32_t d;            /* hidden size */
+  int32_t E;            /* routed experts */
+  int32_t top_k;        /* experts selected per token */
+  int32_t n_shared;     /* always-active shared experts (SwiGLU), 0 for none */
+  int32_t ffn;          /* routed SwiGLU expert width (ignored for low-rank experts) */
+  int32_t ffn_shared;   /* shared expert width */
+  int32_t rank;         /* low-rank expert rank r (ignored for SwiGLU experts) */
+  int32_t score;        /* moe_score_t */
+  int32_t expert;       /* moe_expert_t */
+  int32_t dtype;        /* moe_dtype_t: activations and weights */
+  int32_t norm_topk;    /* 1: divide the k selected weights by their sum */
+  float capacity_factor;/* <= 0: dropless; else C = ceil(cf*T*top_k/E), exact on this fp32 */
+  float aux_alpha;      /* load-balancing loss weight (0.01 on the Quartz pages) */
+} moe_config_t;
+
+/* Weights, all device pointers in dtype unless noted; [a,b,c] = row-major shape. */
+typedef struct {
+  const void *w_router;      /* [E, d] */
+  const float *logit_offset; /* [E] fp32 added to the logit before rounding, or NULL */
+  const float *select_bias;  /* [E] fp32 selection-only bias (sigmoid scoring), or NULL */
+  const void *w_gate;        /* SwiGLU: [E, ffn, d] */
+  const void *w_up;          /* SwiGLU: [E, ffn, d] */
+  const void *w_down;        /* SwiGLU: [E, d, ffn] */
+  const void *lr_V;          /* low-rank: [E, rank, d]  (V^T of each expert) */
+  const void *lr_U;          /* low-rank: [E, d, rank] */
+  const float *lr_s;         /* low-rank: [E, rank] fp32 */
+  const void *ws_gate;       /* shared: [n_shared, ffn_shared, d] */
+  const void *ws_up;         /* shared: [n_shared, ffn_shared, d] */
+  const void *ws_down;       /* shared: [n_shared, d, ffn_shared] */
+} moe_weights_t;
+
+/* Bytes of workspace that every call below needs for `cfg` (the largest, moe_layer_forward).
+ * Returns 0 for an invalid or unsupported configuration. */
+size_t moe_workspace_size(const moe_config_t *cfg);
+
+/* Per-expert capacity C of this configuration, or -1 for dropless, or -2 if cfg is invalid.
+ * C = ceil(capacity_factor * T * top_k / E) evaluated exactly on the fp32 capacity_factor
+ * (Moonfrost expert card: capacity-based routing; the bound is taken over the call's T). */
+int32_t moe_capacity(const moe_config_t *cfg);
+
+/* Router: logits, scoring, top-k, combine weights and the per-expert statistics.
+ * (Quartz "Router: top-6 of 24"; Moonfrost "a router picks the top 3"; Sutra "top-4 routing
+ * with sigmoid scoring and bias-based load balancing".)
+ *   l[t,e] = RN32(sum_i x[t,i]*w_router[e,i] + logit_offset[e])  - exact sum, rounded once
+ *   key    = l (softmax) or RN32(sigmoid(l) + select_bias[e]) (sigmoid), exact, rounded once
+ *   topk_idx[t,j]  [T, top_k] int32: experts by descending key, equal keys -> lower index
+ *   topk_w[t,j]    [T, top_k] fp32: softmax over all E of l (or sigmoid(l)) of the selected
+ *                  expert, divided by the sum over the selected k when norm_topk is set
+ *   expert_count[e][E] int32: number of tokens that selected e (before capacity)
+ *   prob_sum[e]    [E] fp32: sum over tokens of the token's probability of e (softmax; for
+ *                  sigmoid scoring, sigmoids normalised over all E), fixed-order sums */
+moe_status_t moe_route(const moe_config_t *cfg, const void *x /*[T,d]*/,
+                       const moe_weights_t *w, int32_t *topk_idx, float *topk_w,
+                       int32_t *expert_count, float *prob_sum,
+                       void *ws, size_t ws_bytes, void *stream);
+
+/* Token permutation grouped by expert (the stacked-expert layout of the Moonfrost card).
+ * Per expert, routed (token, slot) pairs are ranked by ascending token; rank >= C is dropped.
+ *   offsets  [E+1] int32: exclusive scan of kept counts; offsets[E] = N kept pairs
+ *   slot_pos [T, top_k] int32: row of pair (t,j) in the grouped order, -1 if dropped
+ *   src_token[T*top_k] int32: token of each grouped row (first N entries valid)
+ *   x_perm   [T*top_k, d] dtype: x_perm[r] = x[src_token[r]] (first N rows valid); may be
+ *            NULL to skip the copy. */
+moe_status_t moe_permute(const moe_config_t *cfg, const void *x, const int32_t *topk_idx,
+                         int32_t *offsets, int32_t *slot_pos, int32_t *src_token,
+                         void *x_perm, void *ws, size_t ws_bytes, void *stream);
+
+/* Grouped expert GEMMs on the grouped rows, and the shared experts on all tokens.
+ *   SwiGLU expert e on row r (offsets[e] <= r < offsets[e+1]):
+ *     y_perm[r] = W_down[e] (silu(W_gate[e] x_perm[r]) * (W_up[e] x_perm[r]))
+ *   low-rank expert: y_perm[r] = U[e] (s[e] * (V[e] x_perm[r]))
+ *   y_shared[t] = sum over shared experts of their SwiGLU output on x[t]
+ * Intermediates (the SwiGLU hidden activations, the low-rank projections) are rounded to
+ * dtype, since they are the next tensor-core product's operand; accumulation is fp32.
+ * y_perm: [T*top_k, d] fp32 (first offsets[E] rows written); y_shared: [T, d] fp32, may be
+ * NULL when n_shared = 0. Expert outputs stay fp32 for every dtype: one bf16 rounding of them
+ * or of y costs up to 2^-8 * max|y| / rms(y), the whole 2e-2 error budget of the layer. */
+moe_status_t moe_expert_forward(const moe_config_t *cfg, const void *x_perm,
+                                const int32_t *offsets, const void *x,
+                                const moe_weights_t *w, void *y_perm, void *y_shared,
+                                void *ws, size_t ws_bytes, void *stream);
+
+/* Weighted un-permute: y[t] = y_shared[t] + sum_j [slot_pos[t,j] >= 0] topk_w[t,j] *
+ * y_perm[slot_pos[t,j]], summed in fp32 in slot order. y_perm, y_shared and y are fp32 [.., d].
+ * No atomics. y_shared may be NULL (no shared experts). */
+moe_status_t moe_combine(const moe_config_t *cfg, const void *y_perm, const void *y_shared,
+                         const int32_t *slot_pos, const float *topk_w, void *y, void *stream);
+
+/* Load-balancing loss (Quartz: "0.01-weighted load-balancing loss"):
+ *   loss = aux_alpha * E * sum_i (expert_count[i] / (T*top_k)) * (prob_sum[i] / T)
+ * written to the device scalar `loss` (fp32); 0 when T = 0. */
+moe_status_t moe_aux_loss(const moe_config_t *cfg, const int32_t *expert_count,
+                          const float *prob_sum, float *loss, void *stream);
+
+/* The whole layer: route -> permute -> experts -> combine -> loss, no host synchronisation.
+ *   y [T, d] fp32; aux_loss: device fp32 scalar (may be NULL); expert_count: optional [E]
+ *   int32 output of the router's per-expert selection counts (may be NULL). */
+moe_status_t moe_layer_forward(const moe_config_t *cfg, const void *x, const moe_weights_t *w,
+                               void *y, float *aux_loss, int32_t *expert_count,
+                               void *ws, size_t ws_bytes, void *stream);
+
+/* Human-readable name of a status. Never NULL. */
+const char *moe_status_str(moe_status_t s);
+
+/* Synchronises `stream`, then returns and clears the device error word of the current device
+ * (MOE_OK if no device-side fault was recorded). *info (may be NULL) receives a detail code. */
+moe_status_t moe_get_device_error(void *stream, int64_t *info);
+
+/* Test and measurement controls (synchronous, current device):
+ *   MOE_DEBUG_FORCE_EXACT: 1 = route every logit and sigmoid key through the exact fallback
+ *     path instead of only the ones the fp64 screen cannot decide (for parity tests);
+ *   MOE_DEBUG_WAIT_LIMIT_NS: upper bound on any device-side wait (default 2e9 ns);
+ *   MOE_DEBUG_PROFILE: 1 = record a CUDA event pair around every kernel the library launches,
+ *     per kernel kind, read with moe_profile_read(). */
+typedef enum { MOE_DEBUG_FORCE_EXACT = 1, MOE_DEBUG_WAIT_LIMIT_NS = 2, MOE_DEBUG_PROFILE = 3 }
+    moe_debug_t;
+moe_status_t moe_debug_set(int32_t what, int64_t value);
+
+/* Kernel-level timing collected while MOE_DEBUG_PROFILE is on. Synchronises the device.
+ * Fills up to `max` entries: names[i] (static strings), total_ms[i] and launches[i]; returns
+ * the number of kernel kinds with at least one launch, and resets the accumulators. */
+int32_t moe_profile_read(const char **names, double *total_ms, int64_t *launches, int32_t max);
+
+/* Test hook for failure detection: launches one tiny kernel that waits on a shared-memory
+ * barrier nothing will complete, bounded by MOE_DEBUG_WAIT_LIMIT_NS; the kernel then records
+ * MOE_ERR_TIMEOUT in the device error word and returns. Returns the launch status. */
+moe_status_t moe_debug_wait_timeout_probe(void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOE_H */

@@ -1,0 +1,93 @@
+"""Helpers for the GPU parity tests: run the C ABI on seeded inputs and compare with the oracle."""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+from fine_grained_mixture_moe_b200 import binding as B
+from fine_grained_mixture_moe_b200.layer import torch_dtype, upload_weights
+
+
+def to_cfg(c, T=None) -> B.MoEConfig:
+    return B.make_config(T=c.T if T is None else T, d=c.d, E=c.E, top_k=c.top_k,
+                         n_shared=c.n_shared, ffn=c.ffn, ffn_shared=c.ffn_shared, rank=c.rank,
+                         score=c.score, expert=c.expert, dtype=c.dtype, norm_topk=c.norm_topk,
+                         capacity_factor=c.capacity_factor, aux_alpha=c.aux_alpha)
+
+
+def tol_of(c) -> float:
+    """max|y - y_oracle| / rms(y_oracle) bound: 2e-2 for bf16, 1e-4 for fp32."""
+    return 2e-2 if c.dtype == "bf16" else 1e-4
+
+
+def rel_err(got, ref) -> float:
+    ref = np.asarray(ref, np.float64)
+    got = np.asarray(got, np.float64)
+    rms = np.sqrt(np.mean(ref ** 2)) if ref.size else 1.0
+    if ref.size == 0:
+        return 0.0
+    return float(np.max(np.abs(got - ref)) / max(rms, 1e-30))
+
+
+def np_(t: torch.Tensor) -> np.ndarray:
+    if t.dtype == torch.bfloat16:
+        t = t.float()
+    return t.detach().cpu().numpy()
+
+
+class GpuRun:
+    """Device copies of one configuration's inputs plus every step's outputs."""
+
+    def __init__(self, c, inp, device="cuda:0"):
+        self.c = c
+        self.inp = inp
+        self.cfg = to_cfg(c, T=inp["x"].shape[0])
+        self.dev = torch.device(device)
+        self.dt = torch_dtype(self.cfg)
+        self.w = upload_weights(self.cfg, inp, self.dev)
+        self.ws_struct = B.make_weights(self.w)
+        self.x = torch.as_tensor(inp["x"]).to(self.dt).contiguous().to(self.dev)
+        self.ws_bytes = B.moe_workspace_size(self.cfg)
+        assert self.ws_bytes > 0
+        self.ws = torch.empty(self.ws_bytes, dtype=torch.uint8, device=self.dev)
+
+    def steps(self):
+        c, T, k, E, d = self.c, self.cfg.T, self.cfg.top_k, self.cfg.E, self.cfg.d
+        dev, dt = self.dev, self.dt
+        o = {}
+        o["idx"] = torch.empty((T, k), dtype=torch.int32, device=dev)
+        o["w"] = torch.empty((T, k), dtype=torch.float32, device=dev)
+        o["count"] = torch.empty(E, dtype=torch.int32, device=dev)
+        o["prob"] = torch.empty(E, dtype=torch.float32, device=dev)
+        B.moe_route(self.cfg, self.x, self.ws_struct, o["idx"], o["w"], o["count"], o["prob"],
+                    self.ws, self.ws_bytes)
+        o["offsets"] = torch.empty(E + 1, dtype=torch.int32, device=dev)
+        o["slot_pos"] = torch.empty((T, k), dtype=torch.int32, device=dev)
+        o["src"] = torch.empty(max(T * k, 1), dtype=torch.int32, device=dev)
+        o["x_perm"] = torch.empty((max(T * k, 1), d), dtype=dt, device=dev)
+        B.moe_permute(self.cfg, self.x, o["idx"], o["offsets"], o["slot_pos"], o["src"],
+                      o["x_perm"], self.ws, self.ws_bytes)
+        o["y_perm"] = torch.empty((max(T * k, 1), d), dtype=torch.float32, device=dev)
+        o["y_shared"] = torch.empty((max(T, 1), d), dtype=torch.float32, device=dev) if c.n_shared else None
+        B.moe_expert_forward(self.cfg, o["x_perm"], o["offsets"], self.x, self.ws_struct,
+                             o["y_perm"], o["y_shared"], self.ws, self.ws_bytes)
+        o["y"] = torch.empty((max(T, 1), d), dtype=torch.float32, device=dev)
+        B.moe_combine(self.cfg, o["y_perm"], o["y_shared"], o["slot_pos"], o["w"], o["y"])
+        o["aux"] = torch.empty((), dtype=torch.float32, device=dev)
+        B.moe_aux_loss(self.cfg, o["count"], o["prob"], o["aux"])
+        torch.cuda.synchronize()
+        st, info = B.moe_get_device_error()
+        assert st == 0, (B.status_str(st), info)
+        return o
+
+    def layer(self, y=None, aux=None, count=None):
+        T, d = self.cfg.T, self.cfg.d
+        y = torch.empty((max(T, 1), d), dtype=torch.float32, device=self.dev) if y is None else y
+        aux = torch.empty((), dtype=torch.float32, device=self.dev) if aux is None else aux
+        count = torch.empty(self.cfg.E, dtype=torch.int32, device=self.dev) if count is None else count
+        B.moe_layer_forward(self.cfg, self.x, self.ws_struct, y, aux, count, self.ws,
+                            self.ws_bytes)
+        torch.cuda.synchronize()
+        st, info = B.moe_get_device_error()
+        assert st == 0, (B.status_str(st), info)
+        return y, aux, count

@@ -1,0 +1,129 @@
+"""Host-side tests of the C ABI: the library loads, exports what include/moe.h declares, sizes
+its workspace, computes the capacity exactly, and rejects bad arguments before touching a GPU."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import fine_grained_mixture_moe_b200 as moe
+from fine_grained_mixture_moe_b200 import binding as B
+from moe_synth import CONFIGS
+import oracle
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from fine_grained_mixture_moe_b200 import build
+    build.build()
+    return B.load()
+
+
+def header_functions():
+    src = open(os.path.join(ROOT, "include", "moe.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(moe_[a-z_0-9]+)\s*\(", src)))
+
+
+def test_header_declares_the_six_steps():
+    fns = header_functions()
+    for f in ("moe_route", "moe_permute", "moe_expert_forward", "moe_combine", "moe_aux_loss",
+              "moe_layer_forward"):
+        assert f in fns
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for f in header_functions():
+        assert hasattr(lib, f), f
+    assert sorted(B.EXPORTED) == header_functions()
+
+
+def cfg_of(c, **kw):
+    d = dict(T=c.T, d=c.d, E=c.E, top_k=c.top_k, n_shared=c.n_shared, ffn=c.ffn,
+             ffn_shared=c.ffn_shared, rank=c.rank, score=c.score, expert=c.expert,
+             dtype=c.dtype, norm_topk=c.norm_topk, capacity_factor=c.capacity_factor,
+             aux_alpha=c.aux_alpha)
+    d.update(kw)
+    return B.make_config(**d)
+
+
+@pytest.mark.parametrize("name", sorted(CONFIGS))
+def test_workspace_size_and_capacity(lib, name):
+    c = CONFIGS[name]
+    cfg = cfg_of(c)
+    ws = B.moe_workspace_size(cfg)
+    es = 2 if c.dtype == "bf16" else 4
+    assert ws >= c.T * c.top_k * c.d * es * 2      # permuted activations and expert outputs
+    cap = B.moe_capacity(cfg)
+    ref = oracle.capacity(c.T, c.top_k, c.E, c.capacity_factor)
+    assert cap == (-1 if ref is None else ref)
+
+
+@pytest.mark.parametrize("T,k,E,cf", [(16384, 3, 32, 1.25), (10, 3, 3, 1.1), (7, 2, 5, 0.3),
+                                      (1000, 8, 1024, 2.0), (3, 1, 7, 1e-6), (0, 2, 4, 1.0),
+                                      (12345, 6, 24, 0.9999999), (5, 1, 1, 100.0)])
+def test_capacity_matches_oracle(lib, T, k, E, cf):
+    cfg = B.make_config(T=max(T, 0), d=64, E=E, top_k=min(k, E), ffn=64, capacity_factor=cf)
+    assert B.moe_capacity(cfg) == oracle.capacity(T, min(k, E), E, cf)
+
+
+@pytest.mark.parametrize("bad", [dict(d=100), dict(E=0), dict(E=2000), dict(top_k=9),
+                                 dict(top_k=30, E=24), dict(ffn=100), dict(T=-1),
+                                 dict(score=7), dict(dtype=5), dict(expert=3),
+                                 dict(n_shared=1, ffn_shared=0), dict(expert="lowrank", rank=32)])
+def test_unsupported_configs_are_rejected(lib, bad):
+    base = dict(T=16, d=128, E=8, top_k=2, ffn=64)
+    for key in ("score", "dtype", "expert"):
+        if isinstance(bad.get(key), int):
+            base[key] = "softmax" if key == "score" else ("bf16" if key == "dtype" else "swiglu")
+    base.update({k: v for k, v in bad.items() if not isinstance(v, int) or k not in
+                 ("score", "dtype", "expert")})
+    cfg = B.make_config(**base)
+    for key in ("score", "dtype", "expert"):
+        if isinstance(bad.get(key), int):
+            setattr(cfg, key, bad[key])
+    assert B.moe_workspace_size(cfg) == 0
+    w = B.MoEWeights()
+    st = lib.moe_route(ctypes.byref(cfg), 16, ctypes.byref(w), 16, 16, 16, 16, 16, 1 << 30, None)
+    assert st == 2  # MOE_ERR_UNSUPPORTED
+
+
+def test_bad_pointers_and_workspace_are_rejected_on_the_host(lib):
+    cfg = B.make_config(T=16, d=128, E=8, top_k=2, ffn=64)
+    w = B.MoEWeights()
+    w.w_router = 4096
+    need = B.moe_workspace_size(cfg)
+    P = ctypes.byref
+    # null x
+    assert lib.moe_route(P(cfg), None, P(w), 16, 16, 16, 16, 16, need, None) == 1
+    # misaligned output
+    assert lib.moe_route(P(cfg), 16, P(w), 24, 16, 16, 16, 16, need, None) == 1
+    # workspace too small
+    assert lib.moe_route(P(cfg), 16, P(w), 16, 16, 16, 16, 16, need - 1, None) == 3
+    # null weights struct / config
+    assert lib.moe_route(P(cfg), 16, None, 16, 16, 16, 16, 16, need, None) == 1
+    assert lib.moe_route(None, 16, P(w), 16, 16, 16, 16, 16, need, None) == 1
+    # expert weights missing
+    assert lib.moe_expert_forward(P(cfg), 16, 16, 16, P(w), 16, 16, 16, need, None) == 1
+    assert lib.moe_layer_forward(P(cfg), 16, P(w), 16, None, None, 16, need, None) == 1
+    assert lib.moe_combine(P(cfg), 16, 16, 16, 16, 8, None) == 1
+    assert lib.moe_aux_loss(P(cfg), 16, 16, None, None) == 1
+
+
+def test_status_strings(lib):
+    for s in range(7):
+        assert B.status_str(s).startswith(B.STATUS_NAMES[s])
+    assert lib.moe_status_str(99) == b"unknown moe_status_t"
+
+
+def test_package_fails_loudly_without_library(tmp_path):
+    with pytest.raises(RuntimeError, match="not built"):
+        B._lib_saved = B._lib
+        try:
+            B._lib = None
+            B.load(str(tmp_path / "missing.so"))
+        finally:
+            B._lib = B._lib_saved

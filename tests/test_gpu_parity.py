@@ -1,0 +1,198 @@
+"""GPU parity: every step of the CUDA path, through the C ABI, against the CPU oracle.
+
+Integer outputs (expert indices, counts, offsets, slot positions, source tokens, the permuted
+copy of x) must match bit for bit. Floating outputs must satisfy
+max|y - y_oracle| / rms(y_oracle) <= 2e-2 (bf16) or 1e-4 (fp32); combine weights and the
+per-expert probability sums 1e-5 relative; the load-balancing loss 1e-5 relative.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from fine_grained_mixture_moe_b200 import binding as B
+from moe_synth import CONFIGS, MoEConfig, get_config, make_inputs
+from tests.gpu_helpers import GpuRun, np_, rel_err, tol_of
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    from fine_grained_mixture_moe_b200 import build
+    build.build()
+    B.load()
+    yield
+    B.moe_debug_set(B.DEBUG_FORCE_EXACT, 0)
+
+
+# Reduced-T versions of the five configurations: several M tiles per expert, several N and K
+# blocks, and a ragged tail (T not a multiple of 32 or 128).
+SMALL = {
+    "tiny_f32": get_config("tiny_f32"),
+    "quartz_s": get_config("quartz", T=515),
+    "capacity_s": get_config("capacity", T=1037),
+    "sigmoid_s": get_config("sigmoid", T=611),
+    "lowrank_s": get_config("lowrank", T=1500, E=256),
+}
+
+EDGE = {
+    "T1": get_config("quartz", T=1),
+    "T33": get_config("quartz", T=33),
+    "E1k1": MoEConfig(name="E1k1", T=77, d=128, E=1, top_k=1, n_shared=1, ffn=64, ffn_shared=64),
+    "k_eq_E": MoEConfig(name="kE", T=90, d=64, E=3, top_k=3, n_shared=0, ffn=128, ffn_shared=0),
+    "heavy_drops": get_config("capacity", T=700, capacity_factor=0.25),
+    "norm_softmax": get_config("quartz", T=200, norm_topk=True),
+    "sigmoid_nobias": get_config("sigmoid", T=150, bias=()),
+    "three_shared": MoEConfig(name="s3", T=160, d=256, E=8, top_k=2, n_shared=3, ffn=128,
+                              ffn_shared=64, offset=("normal", 0.5)),
+    "lowrank_shared": MoEConfig(name="lrs", T=300, d=256, E=16, top_k=2, n_shared=1, ffn=0,
+                                ffn_shared=128, rank=64, expert="lowrank", offset=("zipf", 1.1)),
+    "f32_sigmoid_cap": MoEConfig(name="f32sc", T=130, d=128, E=8, top_k=3, n_shared=1, ffn=64,
+                                 ffn_shared=64, dtype="f32", score="sigmoid", norm_topk=True,
+                                 bias=("uniform", 0.1), capacity_factor=0.8),
+}
+
+
+def check_steps(c, inp, run=None, exact_only=False):
+    run = run or GpuRun(c, inp)
+    ref = oracle.layer_forward(c, inp, with_outputs=not exact_only)
+    o = run.steps()
+    r, pm = ref["route"], ref["perm"]
+    T = inp["x"].shape[0]
+    N = int(pm["offsets"][-1])
+    # routing: bit-exact indices, weights 1e-5
+    assert np.array_equal(np_(o["idx"])[:T], r["idx"]), "expert indices differ"
+    np.testing.assert_allclose(np_(o["w"])[:T], r["w"], rtol=1e-5, atol=1e-7)
+    assert np.array_equal(np_(o["count"]), r["count"])
+    np.testing.assert_allclose(np_(o["prob"]), r["prob_sum"], rtol=1e-5, atol=1e-6)
+    # permutation: bit-exact
+    assert np.array_equal(np_(o["offsets"]), pm["offsets"])
+    assert np.array_equal(np_(o["slot_pos"])[:T], pm["slot_pos"])
+    assert np.array_equal(np_(o["src"])[:N], pm["src"])
+    xp = np_(o["x_perm"])[:N]
+    assert np.array_equal(xp, inp["x"][pm["src"]]), "x_perm is not an exact copy"
+    if exact_only:
+        return o, ref
+    tol = tol_of(c)
+    ef = ref["experts"]
+    assert rel_err(np_(o["y_perm"])[:N], ef["y_perm"]) <= tol
+    if c.n_shared:
+        assert rel_err(np_(o["y_shared"])[:T], ef["y_shared"]) <= tol
+    assert rel_err(np_(o["y"])[:T], ref["y"]) <= tol
+    assert float(o["aux"]) == pytest.approx(ref["aux"], rel=1e-5, abs=1e-9)
+    # the fused call gives bitwise the same result as the steps
+    y, aux, cnt = run.layer()
+    assert torch.equal(y[:T], o["y"][:T])
+    assert float(aux) == float(o["aux"])
+    assert torch.equal(cnt, o["count"])
+    return o, ref
+
+
+@pytest.mark.parametrize("name", sorted(SMALL))
+def test_small_configs(name):
+    c = SMALL[name]
+    check_steps(c, make_inputs(c))
+
+
+@pytest.mark.parametrize("name", sorted(EDGE))
+def test_edge_cases(name):
+    c = EDGE[name]
+    check_steps(c, make_inputs(c))
+
+
+@pytest.mark.parametrize("name", ["tiny_f32", "quartz_s", "sigmoid_s"])
+def test_forced_exact_router_paths(name):
+    """Every logit through the expansion sum and every sigmoid key through double-double."""
+    c = SMALL[name]
+    if c.T > 300:
+        c = c.with_(T=300)
+    inp = make_inputs(c)
+    B.moe_debug_set(B.DEBUG_FORCE_EXACT, 1)
+    try:
+        check_steps(c, inp, exact_only=True)
+    finally:
+        B.moe_debug_set(B.DEBUG_FORCE_EXACT, 0)
+
+
+def test_logits_on_rounding_midpoints():
+    """Exact sums on and next to fp32 rounding boundaries: a plain fp64 dot product rounded to
+    fp32 would tie experts 0, 1 and 2; the exact rounding ranks expert 2 first."""
+    c = MoEConfig(name="mid", T=3, d=64, E=4, top_k=3, n_shared=0, ffn=64, ffn_shared=0)
+    inp = make_inputs(c)
+    x = np.zeros((3, 64), np.float32)
+    x[:, 0] = 1.0
+    x[:, 1] = 2.0 ** -24
+    x[:, 2] = 2.0 ** -60
+    x[1, 2] = -2.0 ** -60
+    W = np.zeros((4, 64), np.float32)
+    W[0, :2] = 1.0
+    W[1, 0] = 1.0
+    W[2, :3] = 1.0
+    W[3, 0] = 0.5
+    inp["x"], inp["w_router"] = x, W
+    o, ref = check_steps(c, inp, exact_only=True)
+    assert ref["route"]["idx"][0].tolist() == [2, 0, 1]
+    assert ref["route"]["idx"][1].tolist() == [0, 1, 2]
+
+
+def test_empty_call():
+    c = get_config("quartz", T=0)
+    run = GpuRun(c, make_inputs(c, T=0))
+    y, aux, cnt = run.layer()
+    assert float(aux) == 0.0
+    assert int(cnt.abs().sum()) == 0
+
+
+def test_bitwise_determinism():
+    c = SMALL["quartz_s"]
+    run = GpuRun(c, make_inputs(c))
+    y1, a1, _ = run.layer()
+    y1 = y1.clone()
+    y2, a2, _ = run.layer()
+    assert torch.equal(y1, y2) and float(a1) == float(a2)
+
+
+def test_bounded_wait_times_out_cleanly():
+    """A wait on a barrier that nothing completes ends with MOE_ERR_TIMEOUT; the context stays
+    usable for the next call."""
+    B.moe_get_device_error()
+    B.moe_debug_set(B.DEBUG_WAIT_LIMIT_NS, 2_000_000)
+    try:
+        B.moe_debug_wait_timeout_probe()
+        st, info = B.moe_get_device_error()
+        assert st == 5 and info == 20
+    finally:
+        B.moe_debug_set(B.DEBUG_WAIT_LIMIT_NS, 2_000_000_000)
+    c = EDGE["E1k1"]
+    check_steps(c, make_inputs(c))
+
+
+# ------------------------------------------------------------------ full-size configurations
+@pytest.mark.parametrize("name", sorted(CONFIGS))
+def test_full_size(name):
+    """Every token's routing and permutation bit-exact; y on sampled tokens vs the per-token
+    definition; the loss. Launch configuration as the benchmark runs it (moe_layer_forward)."""
+    c = get_config(name)
+    inp = make_inputs(c)
+    run = GpuRun(c, inp)
+    o = run.steps()
+    ref = oracle.layer_forward(c, inp, with_outputs=False)
+    r, pm = ref["route"], ref["perm"]
+    assert np.array_equal(np_(o["idx"]), r["idx"])
+    np.testing.assert_allclose(np_(o["w"]), r["w"], rtol=1e-5, atol=1e-7)
+    assert np.array_equal(np_(o["count"]), r["count"])
+    np.testing.assert_allclose(np_(o["prob"]), r["prob_sum"], rtol=1e-5, atol=1e-5)
+    assert np.array_equal(np_(o["offsets"]), pm["offsets"])
+    assert np.array_equal(np_(o["slot_pos"]), pm["slot_pos"])
+    N = int(pm["offsets"][-1])
+    assert np.array_equal(np_(o["src"])[:N], pm["src"])
+    assert float(o["aux"]) == pytest.approx(ref["aux"], rel=1e-5)
+    y, aux, cnt = run.layer()
+    assert torch.equal(y, o["y"])
+    rng = np.random.default_rng(123)
+    sample = np.unique(np.concatenate([[0, c.T - 1], rng.choice(c.T, 94, replace=False)]))
+    yg = np_(y)[sample]
+    yr = np.stack([oracle.token_output(c, inp, int(t), r["idx"][t], r["w"][t],
+                                       pm["slot_pos"][t] >= 0) for t in sample])
+    assert rel_err(yg, yr) <= tol_of(c)
