@@ -84,6 +84,8 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
         "moe_profile_read": (c_int32, [P(ctypes.c_char_p), P(ctypes.c_double), P(c_int64),
                                        c_int32]),
         "moe_debug_wait_timeout_probe": (c_int32, [c_void_p]),
+        "moe_route_noalloc": (c_int32, [P(MoEConfig), c_void_p, P(MoEWeights), c_void_p,
+                                        c_void_p, c_void_p, c_void_p, c_void_p]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -96,7 +98,7 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
 EXPORTED = ("moe_workspace_size", "moe_capacity", "moe_route", "moe_permute",
             "moe_expert_forward", "moe_combine", "moe_aux_loss", "moe_layer_forward",
             "moe_status_str", "moe_get_device_error", "moe_debug_set", "moe_profile_read",
-            "moe_debug_wait_timeout_probe")
+            "moe_debug_wait_timeout_probe", "moe_route_noalloc")
 
 
 def _ptr(t) -> Optional[int]:
@@ -215,3 +217,15 @@ def moe_profile_read(max_kinds: int = 32):
 
 def moe_debug_wait_timeout_probe(stream=None) -> None:
     _check("moe_debug_wait_timeout_probe", load().moe_debug_wait_timeout_probe(_stream(stream)))
+
+
+ROUTE_NOALLOC_SCRATCH_BYTES = 4 << 20
+
+
+def moe_route_noalloc(cfg, x, w: MoEWeights, topk_idx, topk_w, expert_count, prob_sum,
+                      stream=None) -> None:
+    """moe_route with its scratch in the library's fixed device array (no workspace)."""
+    _check("moe_route_noalloc",
+           load().moe_route_noalloc(ctypes.byref(cfg), _ptr(x), ctypes.byref(w), _ptr(topk_idx),
+                                    _ptr(topk_w), _ptr(expert_count), _ptr(prob_sum),
+                                    _stream(stream)))

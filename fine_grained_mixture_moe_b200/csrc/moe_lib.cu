@@ -676,3 +676,105 @@ extern "C" moe_status_t moe_debug_wait_timeout_probe(void *stream) {
   moe::wait_probe_kernel<<<1, 32, 0, (cudaStream_t)stream>>>();
   return last_launch_status();
 }
+
+// ================================================================== moe_route_noalloc
+// The router's scratch (fp64 router weight, row norms, per-CTA partial statistics and the
+// completion counter) placed in a fixed array of the library's own device memory instead of a
+// caller workspace. Host code must not use the array's name as a device pointer: it is a host
+// stand-in for the symbol, so its device address is looked up once per device below.
+namespace {
+
+static __device__ __align__(256) unsigned char g_route_scratch[MOE_ROUTE_NOALLOC_SCRATCH_BYTES];
+
+void *g_route_scratch_dev[64];
+std::mutex g_route_scratch_mu;
+
+// Device address of g_route_scratch on the current device (looked up on the first call there).
+moe_status_t route_scratch_address(void **out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
+  if (dev < 0 || dev >= 64) return MOE_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lk(g_route_scratch_mu);
+  if (g_route_scratch_dev[dev] == nullptr) {
+    void *p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_route_scratch);
+    if (e != cudaSuccess || p == nullptr) return MOE_ERR_CUDA;
+    g_route_scratch_dev[dev] = p;
+  }
+  *out = g_route_scratch_dev[dev];
+  return MOE_OK;
+}
+
+struct RouteScratch {
+  size_t w64, wnorm, part_cnt, part_prob, counter, total;
+};
+
+RouteScratch route_scratch_layout(const moe_config_t *c) {
+  RouteScratch L;
+  const size_t E = c->E, d = c->d;
+  const size_t nblk = std::max<size_t>(1, ceil_div(c->T, RT_TM));
+  size_t o = 0;
+  auto take = [&](size_t bytes) { size_t at = o; o = align256(o + std::max<size_t>(bytes, 1)); return at; };
+  L.w64 = take(E * d * 8);
+  L.wnorm = take(E * 8);
+  L.part_cnt = take(nblk * E * 4);
+  L.part_prob = take(nblk * E * 4);
+  L.counter = take(16);
+  L.total = o;
+  return L;
+}
+
+template <typename Tin>
+moe_status_t route_noalloc_impl(const moe_config_t *c, const void *x, const moe_weights_t *w,
+                                int32_t *idx, float *wts, int32_t *count, float *prob,
+                                char *scratch, cudaStream_t st) {
+  const RouteScratch L = route_scratch_layout(c);
+  if (c->T == 0) {
+    if (cudaMemsetAsync(count, 0, (size_t)c->E * 4, st) != cudaSuccess) return MOE_ERR_CUDA;
+    if (cudaMemsetAsync(prob, 0, (size_t)c->E * 4, st) != cudaSuccess) return MOE_ERR_CUDA;
+    return MOE_OK;
+  }
+  RouterArgs a;
+  a.x = x;
+  a.w64 = (const double *)(scratch + L.w64);
+  a.wnorm = (const double *)(scratch + L.wnorm);
+  a.off = w->logit_offset;
+  a.bias = c->score == MOE_SCORE_SIGMOID ? w->select_bias : nullptr;
+  a.T = c->T; a.d = c->d; a.E = c->E; a.k = c->top_k; a.score = c->score; a.norm = c->norm_topk;
+  a.idx = idx; a.wts = wts;
+  a.part_cnt = (int32_t *)(scratch + L.part_cnt);
+  a.part_prob = (float *)(scratch + L.part_prob);
+  a.count_out = count; a.prob_out = prob;
+  a.counter = (unsigned *)(scratch + L.counter);
+  // router_prep_kernel rewrites the fp64 weight and the norms and clears the completion
+  // counter on every call, so nothing left in the array by an earlier call is read.
+  router_prep_kernel<Tin><<<c->E, 256, 0, st>>>((const Tin *)w->w_router, c->E, c->d,
+                                                 (double *)a.w64, (double *)a.wnorm, a.counter);
+  MOE_TRY(last_launch_status());
+  const size_t smem = router_smem_bytes(c->E);
+  if (cudaFuncSetAttribute(router_kernel<Tin>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  router_kernel<Tin><<<ceil_div(c->T, RT_TM), RT_THREADS, smem, st>>>(a);
+  return last_launch_status();
+}
+
+}  // namespace
+
+extern "C" moe_status_t moe_route_noalloc(const moe_config_t *cfg, const void *x,
+                                          const moe_weights_t *w, int32_t *topk_idx,
+                                          float *topk_w, int32_t *expert_count, float *prob_sum,
+                                          void *stream) {
+  MOE_TRY(check_cfg(cfg));
+  MOE_TRY(check_weights(cfg, w, true, false));
+  MOE_REQUIRE(tok16(cfg, x) && tok16(cfg, topk_idx) && tok16(cfg, topk_w) &&
+              aligned16(expert_count) && aligned16(prob_sum));
+  if (route_scratch_layout(cfg).total > MOE_ROUTE_NOALLOC_SCRATCH_BYTES) return MOE_ERR_WORKSPACE;
+  void *scratch = nullptr;
+  MOE_TRY(route_scratch_address(&scratch));
+  cudaStream_t st = (cudaStream_t)stream;
+  if (cfg->dtype == MOE_DTYPE_BF16)
+    return route_noalloc_impl<__nv_bfloat16>(cfg, x, w, topk_idx, topk_w, expert_count, prob_sum,
+                                             (char *)scratch, st);
+  return route_noalloc_impl<float>(cfg, x, w, topk_idx, topk_w, expert_count, prob_sum,
+                                   (char *)scratch, st);
+}

@@ -155,6 +155,26 @@ moe_status_t moe_layer_forward(const moe_config_t *cfg, const void *x, const moe
                                void *y, float *aux_loss, int32_t *expert_count,
                                void *ws, size_t ws_bytes, void *stream);
 
+/* moe_route without a workspace, for callers that cannot allocate device memory.
+ * The source pages have no counterpart to this entry point; it serves integration needs only.
+ * Some callers cannot call cudaMalloc or hand out a workspace: for example a plugin that runs
+ * inside a host framework whose allocator owns all device memory, or a latency-critical loop
+ * where cudaMalloc's implicit device-wide synchronisation is not acceptable. This variant
+ * computes exactly what moe_route computes (same kernels, same outputs), but its scratch lives
+ * in a fixed array of MOE_ROUTE_NOALLOC_SCRATCH_BYTES in the library's own device memory, which
+ * every GPU that loads the library holds until the process exits. The caller still passes x,
+ * the weights and all outputs.
+ *   - Limit: the scratch needed is about 8*E*d + 8*E*ceil(T/32) bytes; configurations that need
+ *     more than MOE_ROUTE_NOALLOC_SCRATCH_BYTES return MOE_ERR_WORKSPACE with nothing enqueued.
+ *   - Set-up: the first call on each device looks up the array's device address (with that
+ *     device current); make that first call before any stream capture begins.
+ *   - Sharing: every call on a device uses the same array. Calls whose work overlaps on the GPU
+ *     (other streams, other host threads) race on it and must be serialised by the caller. */
+#define MOE_ROUTE_NOALLOC_SCRATCH_BYTES (4u << 20)
+moe_status_t moe_route_noalloc(const moe_config_t *cfg, const void *x, const moe_weights_t *w,
+                               int32_t *topk_idx, float *topk_w, int32_t *expert_count,
+                               float *prob_sum, void *stream);
+
 /* Human-readable name of a status. Never NULL. */
 const char *moe_status_str(moe_status_t s);
 
