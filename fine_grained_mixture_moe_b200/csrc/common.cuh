@@ -13,7 +13,7 @@ namespace moe {
 // First error wins; the host reads and clears it with moe_get_device_error().
 __device__ int g_err_code = 0;
 __device__ long long g_err_info = 0;
-__device__ int g_force_exact = 0;
+__device__ int g_force_exact = 0;  // 0 off; 1 every logit/key via the exact paths; 2 also skip the integer path
 __device__ unsigned long long g_wait_limit_ns = 2000000000ull;
 
 // detail codes stored in g_err_info

@@ -292,6 +292,31 @@ moe_status_t launch_gemm(const moe_config_t *c, const GroupedGemm &g, int bn_hin
     if (_s != MOE_OK) return _s;        \
   } while (0)
 
+template <typename Tin, int RE>
+moe_status_t launch_router_re(const RouterArgs &a, cudaStream_t st) {
+  const size_t smem = router_smem_bytes(a.E, RE);
+  if (cudaFuncSetAttribute(router_kernel<Tin, RE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)smem) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  router_kernel<Tin, RE><<<ceil_div(a.T, RT_TM), RT_THREADS, smem, st>>>(a);
+  return last_launch_status();
+}
+
+template <typename Tin>
+moe_status_t launch_router(const RouterArgs &a, cudaStream_t st) {
+  moe_status_t s;
+  switch (router_re_for(a.E)) {
+    case 2: s = launch_router_re<Tin, 2>(a, st); break;
+    case 4: s = launch_router_re<Tin, 4>(a, st); break;
+    case 6: s = launch_router_re<Tin, 6>(a, st); break;
+    default: s = launch_router_re<Tin, 8>(a, st); break;
+  }
+  if (s != MOE_OK) return s;
+  router_reduce_kernel<<<a.E, 128, 0, st>>>(a.part_cnt, a.part_prob, ceil_div(a.T, RT_TM), a.E,
+                                           a.count_out, a.prob_out);
+  return last_launch_status();
+}
+
 template <typename Tin>
 moe_status_t route_impl(const moe_config_t *c, const void *x, const moe_weights_t *w,
                         int32_t *idx, float *wts, int32_t *count, float *prob, void *ws,
@@ -320,12 +345,8 @@ moe_status_t route_impl(const moe_config_t *c, const void *x, const moe_weights_
                                                    (double *)a.w64, (double *)a.wnorm, a.counter);
     MOE_TRY(last_launch_status());
   }
-  const size_t smem = router_smem_bytes(c->E);
-  if (cudaFuncSetAttribute(router_kernel<Tin>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-    return MOE_ERR_CUDA;
   ProfScope ps(K_ROUTER, st);
-  router_kernel<Tin><<<ceil_div(c->T, RT_TM), RT_THREADS, smem, st>>>(a);
-  return last_launch_status();
+  return launch_router<Tin>(a, st);
 }
 
 template <typename Tin>
@@ -605,7 +626,8 @@ moe_status_t moe_get_device_error(void *stream, int64_t *info) {
 moe_status_t moe_debug_set(int32_t what, int64_t value) {
   switch (what) {
     case MOE_DEBUG_FORCE_EXACT: {
-      const int v = value ? 1 : 0;
+      if (value < 0 || value > 2) return MOE_ERR_INVALID_ARG;
+      const int v = (int)value;
       return cudaMemcpyToSymbol(g_force_exact, &v, sizeof(int)) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
     }
     case MOE_DEBUG_WAIT_LIMIT_NS: {
@@ -751,11 +773,7 @@ moe_status_t route_noalloc_impl(const moe_config_t *c, const void *x, const moe_
   router_prep_kernel<Tin><<<c->E, 256, 0, st>>>((const Tin *)w->w_router, c->E, c->d,
                                                  (double *)a.w64, (double *)a.wnorm, a.counter);
   MOE_TRY(last_launch_status());
-  const size_t smem = router_smem_bytes(c->E);
-  if (cudaFuncSetAttribute(router_kernel<Tin>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-    return MOE_ERR_CUDA;
-  router_kernel<Tin><<<ceil_div(c->T, RT_TM), RT_THREADS, smem, st>>>(a);
-  return last_launch_status();
+  return launch_router<Tin>(a, st);
 }
 
 }  // namespace

@@ -10,9 +10,14 @@
 // How: the dot products run on the fp64 FMA pipe. bf16 and fp32 inputs multiply exactly in
 // fp64, so the only error is the summation, bounded by (d+2) 2^-52 (|x|_2 |W_e|_2 + |off|).
 // When that enclosure holds no fp32 rounding boundary, RN32 of the fp64 value *is* the exact
-// rounding. Otherwise (about 1 logit in 10^5 at these sizes) the thread recomputes the sum
-// exactly as a non-overlapping floating-point expansion (Shewchuk's Grow-Expansion with zero
-// elimination) and decides the rounding from its sign against the boundary. Sigmoid keys are
+// rounding. Otherwise the logit is marked and, after the main pass, a whole warp decides it
+// exactly: bf16 products carry at most 16 significant bits, so the exact sum of a row is a
+// multiple of a small power of two and lands exactly on an fp32 rounding boundary for about
+// 0.4% of logits - genuine ties that no error bound can settle. The warp scales every exact
+// product to an integer multiple of the smallest power of two present and sums them in int64,
+// exactly, then compares with the boundaries. Only when the exponent span exceeds 50 bits (or
+// in a forced test mode) does one thread sum the products as a non-overlapping floating-point
+// expansion (Shewchuk's Grow-Expansion with zero elimination) and decide from its sign. Sigmoid keys are
 // screened the same way (fp64 exp, documented 1-ulp) and resolved in double-double arithmetic.
 // So the integer routing decisions are exact, not merely tolerant.
 #pragma once
@@ -20,11 +25,23 @@
 
 namespace moe {
 
-constexpr int RT_TM = 32;       // tokens per CTA (one per lane)
-constexpr int RT_THREADS = 256; // 8 warps
-constexpr int RT_KC = 128;      // k-chunk of x staged in fp64
-constexpr int RT_EWMAX = 8;     // experts per warp per round
+constexpr int RT_TM = 16;          // tokens per CTA
+constexpr int RT_THREADS = 256;    // 8 warps, each a slice of the K dimension
+constexpr int RT_KC = 32;          // k-chunk staged (fp64) in a warp's shared-memory slot
+constexpr int RT_LD = RT_KC + 2;   // padded row: 68 words = 4 (mod 32), conflict-free 16 B loads
 constexpr int EXPANSION_MAX = 40;
+constexpr int RT_FIX_CAP = 256;   // flagged logits per CTA kept with their fp64 sums
+
+// Experts per thread in one round (a round covers 4*RE experts): the RE in {8,6,4,2} that wastes
+// the fewest padded expert slots over all rounds, larger RE on ties.
+inline int router_re_for(int E) {
+  int best = 8, waste = 1 << 30;
+  for (int re : {8, 6, 4, 2}) {
+    const int eb = 4 * re, w = ((E + eb - 1) / eb) * eb - E;
+    if (w < waste) { waste = w; best = re; }
+  }
+  return best;
+}
 
 struct RouterArgs {
   const void *x;
@@ -160,6 +177,119 @@ __device__ __forceinline__ dd dd_div(dd a, dd b) {
   return dd_add(q, {q3, 0.0});
 }
 
+// Exponent of the leading bit and of the lowest set bit of a nonzero, normal double.
+__device__ __forceinline__ void dbl_bit_range(double v, int &lead, int &lsb) {
+  const unsigned long long b = (unsigned long long)__double_as_longlong(v);
+  const int ef = (int)((b >> 52) & 0x7ff);
+  const unsigned long long M = (b & 0xFFFFFFFFFFFFFull) | (1ull << 52);
+  lead = ef - 1075 + 52;
+  lsb = ef - 1075 + (__ffsll((long long)M) - 1);
+}
+
+// Warp-cooperative exact comparison of S = sum_i x_i W_i + off with two dyadic thresholds.
+// Every product is exact in fp64 and so is a multiple of 2^lsb(p); with q the smallest such
+// exponent over all terms and thresholds, every term is an integer multiple of 2^q and, when
+// the exponent span is at most 50 bits, below 2^51, so their sum (at most d + 3 terms) is exact
+// in int64. Returns false (caller falls back) when the span is wider or a term is subnormal.
+// Eight consecutive elements of x (bf16 or fp32) as doubles, from a 16-byte aligned address.
+__device__ __forceinline__ void load8(const __nv_bfloat16 *p, double *v) {
+  const uint4 q = *(const uint4 *)p;
+  const __nv_bfloat162 *h = (const __nv_bfloat162 *)&q;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 f = __bfloat1622float2(h[i]);
+    v[2 * i] = f.x;
+    v[2 * i + 1] = f.y;
+  }
+}
+__device__ __forceinline__ void load8(const float *p, double *v) {
+  const float4 a = *(const float4 *)p, b = *(const float4 *)(p + 4);
+  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+  v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+__device__ __forceinline__ void load8(const double *p, double *v) {
+#pragma unroll
+  for (int i = 0; i < 8; i += 2) {
+    const double2 q = *(const double2 *)(p + i);
+    v[i] = q.x;
+    v[i + 1] = q.y;
+  }
+}
+
+template <typename Tin>
+__device__ bool warp_exact_signs(const Tin *xrow, const double *wrow, int d, double off,
+                                 double mh, double ml, int &c_hi, int &c_lo) {
+  const int lane = threadIdx.x & 31;
+  int qmin = 0x7fffffff, emax = -0x7fffffff;
+  bool bad = false;
+  auto scan = [&](double v) {
+    if (v == 0.0) return;
+    if (fabs(v) < 0x1p-1020) { bad = true; return; }
+    int lead, lsb;
+    dbl_bit_range(v, lead, lsb);
+    qmin = min(qmin, lsb);
+    emax = max(emax, lead);
+  };
+  // lane covers elements [8*lane + 256*j, +8): d is a multiple of 64, so a chunk never straddles d
+  for (int i = 8 * lane; i < d; i += 256) {
+    double xv[8], wv[8];
+    load8(xrow + i, xv);
+    load8(wrow + i, wv);
+#pragma unroll
+    for (int u = 0; u < 8; ++u) scan(__dmul_rn(xv[u], wv[u]));
+  }
+  if (lane == 0) {
+    scan(off);
+    scan(mh);
+    scan(ml);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    qmin = min(qmin, __shfl_xor_sync(0xffffffffu, qmin, o));
+    emax = max(emax, __shfl_xor_sync(0xffffffffu, emax, o));
+  }
+  bad = __any_sync(0xffffffffu, bad);
+  if (bad || emax - qmin > 50) return false;
+  long long acc = 0;
+  for (int i = 8 * lane; i < d; i += 256) {
+    double xv[8], wv[8];
+    load8(xrow + i, xv);
+    load8(wrow + i, wv);
+#pragma unroll
+    for (int u = 0; u < 8; ++u) acc += (long long)ldexp(__dmul_rn(xv[u], wv[u]), -qmin);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+  acc += (long long)ldexp(off, -qmin);
+  const long long h = (long long)ldexp(mh, -qmin), l = (long long)ldexp(ml, -qmin);
+  c_hi = acc > h ? 1 : (acc < h ? -1 : 0);
+  c_lo = acc > l ? 1 : (acc < l ? -1 : 0);
+  return true;
+}
+
+// Warp-cooperative resolution of one logit whose fp64 screen was undecided (or every logit in
+// the forced test modes). Every lane calls it with the same arguments and gets the same result.
+// `approx` is the fp64 sum of the main pass, within (d+16) 2^-52 |x||W_e| of the exact value -
+// far below an fp32 step - so RN32 of the exact value is r = RN32(approx) or a neighbour; the
+// exact integer comparison against the two rounding boundaries around r decides which, ties to
+// even. force_level 2 skips the integer path and sends the logit to the single-thread
+// expansion, to test that path too.
+template <typename Tin>
+__device__ __noinline__ float resolve_logit(const Tin *xrow, const double *wrow, int d, double off,
+                                            double approx, int force_level) {
+  const int lane = threadIdx.x & 31;
+  float r, up, dn;
+  double mh, ml;
+  rn32_certain(approx, 0.0, r, up, dn, mh, ml);
+  int c_hi, c_lo;
+  if (force_level < 2 && fabs((double)r) < 0x1p126 &&
+      warp_exact_signs<Tin>(xrow, wrow, d, off, mh, ml, c_hi, c_lo))
+    return rn32_from_signs(r, up, dn, c_hi, c_lo);
+  float l = 0.0f;
+  if (lane == 0) l = exact_logit<Tin>(xrow, wrow, d, off, approx);
+  return __shfl_sync(0xffffffffu, l, 0);
+}
+
 // e^y in double-double: y = n ln2 + r, e^r by its Taylor series on r/2^10, squared 10 times.
 // ln 2 to 106 bits as a double-double (hi = ln 2 rounded to double, lo = the remainder).
 __device__ dd dd_exp(double y) {
@@ -242,33 +372,47 @@ __global__ void __launch_bounds__(256) router_prep_kernel(const Tin *__restrict_
   }
 }
 
-__host__ __device__ inline size_t router_smem_bytes(int E) {
-  size_t b = (size_t)RT_TM * (RT_KC + 1) * sizeof(double);  // x chunk (fp64)
+__host__ __device__ inline size_t router_smem_bytes(int E, int RE) {
+  size_t b = (size_t)(RT_THREADS / 32) * (RT_TM + 4 * RE) * RT_LD * sizeof(double);  // staging
   b += (size_t)RT_TM * E * sizeof(float);                  // logits / probabilities
   b += (size_t)(RT_THREADS / 32) * E * sizeof(float);      // per-warp sigmoid keys
   b += (size_t)E * sizeof(int);                             // selection counts
+  b += (size_t)RT_TM * ((E + 31) / 32) * sizeof(unsigned);  // undecided-logit flags
   b = (b + 15) & ~(size_t)15;
   b += RT_TM * sizeof(double);                              // token norms
+  b += (size_t)RT_FIX_CAP * sizeof(double);                 // fp64 sums of flagged logits
   return b;
 }
 
-template <typename Tin>
-__global__ void __launch_bounds__(RT_THREADS) router_kernel(RouterArgs a) {
+template <typename Tin, int RE>
+__global__ void __launch_bounds__(RT_THREADS, 2) router_kernel(RouterArgs a) {
+  constexpr int EB = 4 * RE;  // experts per round
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   const int E = a.E, d = a.d, k = a.k;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int lt = lane >> 2, le = lane & 3;  // thread tile: tokens {lt, lt+8} x experts {le+4j}
   const int t0 = blockIdx.x * RT_TM;
   const int ntok = min(RT_TM, a.T - t0);
   const Tin *__restrict__ x = (const Tin *)a.x;
-  const bool force = g_force_exact != 0;
+  const int force_level = g_force_exact;
+  const bool force = force_level != 0;
 
-  double *xs = (double *)smem_raw;
-  float *lg = (float *)(xs + RT_TM * (RT_KC + 1));
+  double *stage = (double *)smem_raw;
+  double *xs = stage + warp * (RT_TM + EB) * RT_LD;  // this warp's [16][RT_LD] x chunk
+  double *wsm = xs + RT_TM * RT_LD;                  // this warp's [EB][RT_LD] W chunk
+  double *part = stage;                              // reused: [8 warps][16][EB] partial sums
+  float *lg = (float *)(stage + (RT_THREADS / 32) * (RT_TM + EB) * RT_LD);
   float *keys = lg + RT_TM * E;
   int *cnt = (int *)(keys + (RT_THREADS / 32) * E);
-  double *xnorm = (double *)(((uintptr_t)(cnt + E) + 15) & ~(uintptr_t)15);
+  const int nfw = (E + 31) / 32;
+  unsigned *flags = (unsigned *)(cnt + E);  // [RT_TM][nfw] undecided logits
+  double *xnorm = (double *)(((uintptr_t)(flags + RT_TM * nfw) + 15) & ~(uintptr_t)15);
+  double *fix_s = xnorm + RT_TM;  // fp64 sums of the first RT_FIX_CAP flagged logits
+  __shared__ int s_nfix;
 
   for (int e = tid; e < E; e += RT_THREADS) cnt[e] = 0;
+  for (int i = tid; i < RT_TM * nfw; i += RT_THREADS) flags[i] = 0u;
+  if (tid == 0) s_nfix = 0;
   for (int tt = warp; tt < RT_TM; tt += RT_THREADS / 32) {
     double s = 0.0;
     if (tt < ntok) {
@@ -282,57 +426,119 @@ __global__ void __launch_bounds__(RT_THREADS) router_kernel(RouterArgs a) {
     if (lane == 0) xnorm[tt] = sqrt(s);
   }
 
-  // ---- logits: warp w owns experts [e0, e0+ne) of each round, lane owns token t0+lane
-  const int ew = min(RT_EWMAX, (E + 7) / 8);
-  const int per_round = 8 * ew;
-  for (int eb = 0; eb < E; eb += per_round) {
-    double acc[RT_EWMAX];
+  // ---- logits. Warp w sums the k-chunks w, w+8, ... of every (token, expert) of the round;
+  // the eight partial sums are then added in warp order. Both operands sit in shared memory
+  // as fp64: one 16-byte load of x serves 4 lanes and one of W serves 8, so a warp issues one
+  // wavefront per load and 2*RE fp64 FMAs per pair of loads.
+  const int nchunk = d / RT_KC;
+  for (int eb = 0; eb < E; eb += EB) {
+    double acc[2][RE];
 #pragma unroll
-    for (int j = 0; j < RT_EWMAX; ++j) acc[j] = 0.0;
-    const int e0 = eb + warp * ew;
-    const int ne = max(0, min(ew, E - e0));
-    for (int kc = 0; kc < d; kc += RT_KC) {
-      const int kn = min(RT_KC, d - kc);
-      __syncthreads();
-      for (int i = tid; i < RT_TM * kn; i += RT_THREADS) {
-        const int r = i / kn, c = i - r * kn;
-        double v = 0.0;
-        if (r < ntok) v = (double)Elem<Tin>::to_f(x[(size_t)(t0 + r) * d + kc + c]);
-        xs[r * (RT_KC + 1) + c] = v;
+    for (int j = 0; j < RE; ++j) acc[0][j] = acc[1][j] = 0.0;
+    for (int c = warp; c < nchunk; c += RT_THREADS / 32) {
+      const int k0 = c * RT_KC;
+      {  // x chunk: lane -> token lane/2, 16 consecutive k
+        const int tt = lane >> 1, h = (lane & 1) * 16;
+        double *dst = xs + tt * RT_LD + h;
+        if (tt < ntok) {
+          const Tin *src = x + (size_t)(t0 + tt) * d + k0 + h;
+#pragma unroll
+          for (int i = 0; i < 16; i += 2)
+            *(double2 *)(dst + i) = make_double2((double)Elem<Tin>::to_f(src[i]),
+                                                 (double)Elem<Tin>::to_f(src[i + 1]));
+        } else {
+#pragma unroll
+          for (int i = 0; i < 16; i += 2) *(double2 *)(dst + i) = make_double2(0.0, 0.0);
+        }
       }
-      __syncthreads();
-      if (ne > 0) {
-        const double *xrow = xs + lane * (RT_KC + 1);
-        const double *wbase = a.w64 + (size_t)e0 * d + kc;
-        for (int c = 0; c < kn; c += 2) {
-          const double x0 = xrow[c], x1 = xrow[c + 1];
+      for (int i = lane; i < EB * (RT_KC / 2); i += 32) {  // W chunk from the fp64 copy
+        const int e = i / (RT_KC / 2), kp = (i % (RT_KC / 2)) * 2;
+        double2 wv = make_double2(0.0, 0.0);
+        if (eb + e < E) wv = *(const double2 *)(a.w64 + (size_t)(eb + e) * d + k0 + kp);
+        *(double2 *)(wsm + e * RT_LD + kp) = wv;
+      }
+      __syncwarp();
+#pragma unroll 4
+      for (int kk = 0; kk < RT_KC; kk += 2) {
+        const double2 x0 = *(const double2 *)(xs + lt * RT_LD + kk);
+        const double2 x1 = *(const double2 *)(xs + (lt + 8) * RT_LD + kk);
 #pragma unroll
-          for (int j = 0; j < RT_EWMAX; ++j) {
-            if (j < ne) {
-              const double2 wv = *(const double2 *)(wbase + (size_t)j * d + c);
-              acc[j] = fma(x0, wv.x, acc[j]);
-              acc[j] = fma(x1, wv.y, acc[j]);
-            }
+        for (int j = 0; j < RE; ++j) {
+          const double2 wv = *(const double2 *)(wsm + (le + 4 * j) * RT_LD + kk);
+          acc[0][j] = fma(x0.x, wv.x, acc[0][j]);
+          acc[0][j] = fma(x0.y, wv.y, acc[0][j]);
+          acc[1][j] = fma(x1.x, wv.x, acc[1][j]);
+          acc[1][j] = fma(x1.y, wv.y, acc[1][j]);
+        }
+      }
+      __syncwarp();
+    }
+    __syncthreads();  // staging slots become the partial-sum buffer
+#pragma unroll
+    for (int j = 0; j < RE; ++j) {
+      part[(warp * RT_TM + lt) * EB + le + 4 * j] = acc[0][j];
+      part[(warp * RT_TM + lt + 8) * EB + le + 4 * j] = acc[1][j];
+    }
+    __syncthreads();
+    for (int q = tid; q < RT_TM * EB; q += RT_THREADS) {
+      const int tt = q / EB, e = eb + q % EB;
+      if (tt < ntok && e < E) {
+        double s = 0.0;
+#pragma unroll
+        for (int w = 0; w < RT_THREADS / 32; ++w) s += part[(w * RT_TM + tt) * EB + q % EB];
+        const double o = a.off ? (double)a.off[e] : 0.0;
+        s += o;
+        // any summation order over d products plus 8 partials and the offset:
+        // |error| <= gamma_{d+16} (sum |x_i W_i| + |off|) <= (d+16) 2^-52 (|x|_2 |W_e|_2 + |off|)
+        const double B = (double)(d + 16) * 0x1p-52 * (xnorm[tt] * a.wnorm[e] + fabs(o));
+        float r, up, dn;
+        double mh, ml;
+        float l;
+        if (rn32_certain(s, B, r, up, dn, mh, ml) && !force) {
+          l = r;
+        } else {
+          // undecided: resolved exactly by the fixup pass below, which needs the fp64 sum
+          const int slot = atomicAdd(&s_nfix, 1);
+          if (slot < RT_FIX_CAP) {
+            fix_s[slot] = s;
+            l = __int_as_float(slot);  // the slot index rides in the logit until resolved
+            atomicOr(&flags[tt * nfw + (e >> 5)], 1u << (e & 31));
+          } else {
+            // overflow (forced test modes only): the fixup recomputes the fp64 sum
+            l = __int_as_float(-1);
+            atomicOr(&flags[tt * nfw + (e >> 5)], 1u << (e & 31));
           }
         }
+        lg[tt * E + e] = l;
       }
     }
-    if (lane < ntok) {
-#pragma unroll
-      for (int j = 0; j < RT_EWMAX; ++j) {
-        if (j < ne) {
-          const int e = e0 + j;
-          const double o = a.off ? (double)a.off[e] : 0.0;
-          const double s = acc[j] + o;
-          const double B = (double)(d + 2) * 0x1p-52 * (xnorm[lane] * a.wnorm[e] + fabs(o));
-          float r, up, dn;
-          double mh, ml;
-          float l;
-          if (rn32_certain(s, B, r, up, dn, mh, ml) && !force) l = r;
-          else l = exact_logit<Tin>(x + (size_t)(t0 + lane) * d, a.w64 + (size_t)e * d, d, o, s);
-          lg[lane * E + e] = l;
-        }
+    __syncthreads();  // the partial-sum buffer is the next round's staging area
+  }
+
+  // ---- fixup of undecided logits: flag words dealt round-robin to the warps; one warp decides
+  // one logit exactly (see resolve_logit)
+  for (int wi = warp; wi < ntok * nfw; wi += RT_THREADS / 32) {
+    unsigned m = flags[wi];
+    const int tt = wi / nfw, e0 = (wi % nfw) * 32;
+    while (m) {
+      const int ee = e0 + __ffs(m) - 1;
+      m &= m - 1;
+      const int slot = __float_as_int(lg[tt * E + ee]);
+      const Tin *xrow = x + (size_t)(t0 + tt) * d;
+      const double *wrow = a.w64 + (size_t)ee * d;
+      const double o = a.off ? (double)a.off[ee] : 0.0;
+      double approx;
+      if (slot >= 0 && slot < RT_FIX_CAP) {
+        approx = fix_s[slot];
+      } else {
+        double s = 0.0;
+        for (int i = lane; i < d; i += 32) s = fma((double)Elem<Tin>::to_f(xrow[i]), wrow[i], s);
+        approx = warp_sum_d(s) + o;
       }
+      const float l = resolve_logit<Tin>(xrow, wrow, d, o, approx, force_level);
+      __syncwarp();
+      if (lane == 0) lg[tt * E + ee] = l;
+      __syncwarp();
     }
   }
   __syncthreads();
@@ -422,25 +628,38 @@ __global__ void __launch_bounds__(RT_THREADS) router_kernel(RouterArgs a) {
     a.part_cnt[(size_t)blockIdx.x * E + e] = cnt[e];
     a.part_prob[(size_t)blockIdx.x * E + e] = ps;
   }
-  __threadfence();
+}
+
+// Per-expert totals of the per-CTA selection counts and probability sums: one block per
+// expert; thread t adds the CTAs t, t+128, ... in order, then a fixed-shape tree combines the
+// 128 partial sums, so prob_sum is bitwise reproducible.
+__global__ void __launch_bounds__(128) router_reduce_kernel(const int32_t *__restrict__ part_cnt,
+                                                            const float *__restrict__ part_prob,
+                                                            int nblk, int E,
+                                                            int32_t *__restrict__ count_out,
+                                                            float *__restrict__ prob_out) {
+  const int e = blockIdx.x, tid = threadIdx.x;
+  int c = 0;
+  float p = 0.0f;
+  for (int b = tid; b < nblk; b += 128) {
+    c += part_cnt[(size_t)b * E + e];
+    p += part_prob[(size_t)b * E + e];
+  }
+  __shared__ int sc[4];
+  __shared__ float sp[4];
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    c += __shfl_xor_sync(0xffffffffu, c, o);
+    p += __shfl_xor_sync(0xffffffffu, p, o);
+  }
+  if ((tid & 31) == 0) {
+    sc[tid >> 5] = c;
+    sp[tid >> 5] = p;
+  }
   __syncthreads();
-  __shared__ int s_last;
-  if (tid == 0) s_last = (atomicAdd(a.counter, 1u) == gridDim.x - 1);
-  __syncthreads();
-  if (s_last) {
-    __threadfence();
-    const int nb = gridDim.x;
-    for (int e = tid; e < E; e += RT_THREADS) {
-      int c = 0;
-      float p = 0.0f;
-      for (int b = 0; b < nb; ++b) {
-        c += __ldcg(a.part_cnt + (size_t)b * E + e);
-        p += __ldcg(a.part_prob + (size_t)b * E + e);
-      }
-      a.count_out[e] = c;
-      a.prob_out[e] = p;
-    }
-    if (tid == 0) *a.counter = 0u;
+  if (tid == 0) {
+    count_out[e] = (sc[0] + sc[1]) + (sc[2] + sc[3]);
+    prob_out[e] = (sp[0] + sp[1]) + (sp[2] + sp[3]);
   }
 }
 

@@ -164,7 +164,7 @@ moe_status_t moe_layer_forward(const moe_config_t *cfg, const void *x, const moe
  * in a fixed array of MOE_ROUTE_NOALLOC_SCRATCH_BYTES in the library's own device memory, which
  * every GPU that loads the library holds until the process exits. The caller still passes x,
  * the weights and all outputs.
- *   - Limit: the scratch needed is about 8*E*d + 8*E*ceil(T/32) bytes; configurations that need
+ *   - Limit: the scratch needed is about 8*E*d + 8*E*ceil(T/16) bytes; configurations that need
  *     more than MOE_ROUTE_NOALLOC_SCRATCH_BYTES return MOE_ERR_WORKSPACE with nothing enqueued.
  *   - Set-up: the first call on each device looks up the array's device address (with that
  *     device current); make that first call before any stream capture begins.
@@ -183,8 +183,9 @@ const char *moe_status_str(moe_status_t s);
 moe_status_t moe_get_device_error(void *stream, int64_t *info);
 
 /* Test and measurement controls (synchronous, current device):
- *   MOE_DEBUG_FORCE_EXACT: 1 = route every logit and sigmoid key through the exact fallback
- *     path instead of only the ones the fp64 screen cannot decide (for parity tests);
+ *   MOE_DEBUG_FORCE_EXACT: 1 = route every logit and sigmoid key through the exact paths
+ *     instead of only the ones the fp64 screen cannot decide; 2 = the same, with logits sent to
+ *     the floating-point expansion rather than the exact integer sum (for parity tests);
  *   MOE_DEBUG_WAIT_LIMIT_NS: upper bound on any device-side wait (default 2e9 ns);
  *   MOE_DEBUG_PROFILE: 1 = record a CUDA event pair around every kernel the library launches,
  *     per kernel kind, read with moe_profile_read(). */

@@ -101,14 +101,16 @@ def test_edge_cases(name):
     check_steps(c, make_inputs(c))
 
 
+@pytest.mark.parametrize("level", [1, 2])
 @pytest.mark.parametrize("name", ["tiny_f32", "quartz_s", "sigmoid_s"])
-def test_forced_exact_router_paths(name):
-    """Every logit through the expansion sum and every sigmoid key through double-double."""
+def test_forced_exact_router_paths(name, level):
+    """Every logit through the exact integer sum (level 1) or the floating-point expansion
+    (level 2), and every sigmoid key through double-double."""
     c = SMALL[name]
     if c.T > 300:
-        c = c.with_(T=300)
+        c = c.with_(T=300 if level == 1 else 96)
     inp = make_inputs(c)
-    B.moe_debug_set(B.DEBUG_FORCE_EXACT, 1)
+    B.moe_debug_set(B.DEBUG_FORCE_EXACT, level)
     try:
         check_steps(c, inp, exact_only=True)
     finally:
