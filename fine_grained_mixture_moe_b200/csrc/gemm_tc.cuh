@@ -8,11 +8,13 @@
 //   warp 1  TMEM owner and MMA issuer: one thread issues tcgen05.mma (kind::f16, bf16 x bf16 ->
 //           fp32, M=128, N=BN, K=16) into one of two TMEM accumulators; tcgen05.commit frees the
 //           smem stage (`empty[s]`) and, per tile, publishes the accumulator (`acc_full[b]`).
-//   warps 2-5 epilogue: tcgen05.ld (32 lanes x 16 columns per load) -> SwiGLU / scale -> bf16
-//           (hidden activations, the next GEMM's operand) or fp32 (expert outputs) -> global;
-//           then `acc_empty[b]`, so the next tile's MMAs overlap this epilogue.
-// GATEUP keeps gate and up in two TMEM accumulators of the same columns (2 x 128 fp32 columns
-// per buffer, 512 with double buffering), so silu(gate) * up is fused without a weight repack.
+//   warps 2-9 epilogue: two warps per TMEM lane quarter, each taking half of the tile's columns;
+//           tcgen05.ld (32 lanes x 32 columns per load) -> SwiGLU / scale -> bf16 (hidden
+//           activations, the next GEMM's operand) or fp32 (expert outputs) -> global; then
+//           `acc_empty[b]`, so the next tile's MMAs overlap this epilogue.
+// GATEUP stages the gate and up weight tiles back to back, so one N=256 MMA fills 128 gate and
+// 128 up accumulator columns (256 fp32 columns per buffer, 512 with double buffering) and
+// silu(gate) * up is fused without a weight repack.
 // Every wait is bounded (global timer); on expiry the CTA records MOE_ERR_TIMEOUT, drains what
 // it has in flight (again bounded), frees its TMEM and returns.
 #pragma once
@@ -23,7 +25,8 @@ namespace moe {
 
 constexpr int TC_BM = 128;
 constexpr int TC_BK = 64;  // one 128-byte swizzle atom of bf16
-constexpr int TC_THREADS = 192;
+constexpr int TC_EPI_WARPS = 8;  // two per TMEM lane quarter, each taking half the columns
+constexpr int TC_THREADS = 64 + 32 * TC_EPI_WARPS;
 
 struct TcMaps {
   CUtensorMap a_r, a_s, b0_r, b1_r, b0_s, b1_s;
@@ -39,15 +42,22 @@ template <int MODE, int BN> struct TcCfg {
   static constexpr int A_BYTES = TC_BM * TC_BK * 2;               // 16 KB
   static constexpr int B_BYTES = BN * TC_BK * 2;
   static constexpr int STAGE_BYTES = A_BYTES + NB * B_BYTES;
-  static constexpr int STAGES = (192 * 1024) / STAGE_BYTES > 8 ? 8 : (192 * 1024) / STAGE_BYTES;
+  static constexpr int STG_BYTES = MODE == MODE_PLAIN ? TC_EPI_WARPS * 4096 : 0;  // fp32 staging
+  static constexpr int STAGES = (200 * 1024 - STG_BYTES) / STAGE_BYTES > 8
+                                    ? 8 : (200 * 1024 - STG_BYTES) / STAGE_BYTES;
   static constexpr int ACC_COLS = NB * BN;                        // fp32 columns per buffer
   static constexpr int TMEM_COLS = (2 * ACC_COLS <= 32) ? 32 : (2 * ACC_COLS <= 64) ? 64
                                    : (2 * ACC_COLS <= 128) ? 128 : (2 * ACC_COLS <= 256) ? 256 : 512;
   static_assert(2 * ACC_COLS <= 512, "TMEM holds 512 columns");
-  static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "UMMA N for M=128");
+  static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "UMMA N for M=128, epilogue in 32s");
+  // one MMA covers N = NB*BN columns: for GATEUP the gate and up tiles sit back to back in
+  // shared memory, so they form one [2*BN, 64] B operand whose first BN accumulator columns are
+  // the gate and the next BN the up projection
+  static constexpr int MMA_N = NB * BN;
+  static_assert(MMA_N <= 256, "UMMA N <= 256");
   // instruction descriptor: D fp32, A/B bf16, both K-major, N>>3 at bit 17, M>>4 at bit 24
   static constexpr uint32_t IDESC = (1u << 4) | (1u << 7) | (1u << 10) |
-                                    ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(TC_BM >> 4) << 24);
+                                    ((uint32_t)(MMA_N >> 3) << 17) | ((uint32_t)(TC_BM >> 4) << 24);
 };
 
 // ---------------------------------------------------------------- PTX wrappers
@@ -135,6 +145,17 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
         "=r"(r[14]), "=r"(r[15])
       : "r"(taddr));
 }
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,"
+      "%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+}
 __device__ __forceinline__ void tmem_wait_ld() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
@@ -142,8 +163,8 @@ __device__ __forceinline__ void tmem_wait_ld() {
 template <int MODE, int BN>
 __host__ __device__ constexpr size_t tc_smem_bytes(int G) {
   using C = TcCfg<MODE, BN>;
-  return 1024 /*alignment slack*/ + (size_t)C::STAGES * C::STAGE_BYTES + 256 /*barriers*/ +
-         (size_t)(G + 1 + TC_THREADS / 32 + 1) * sizeof(int);
+  return 1024 /*alignment slack*/ + (size_t)C::STAGES * C::STAGE_BYTES + C::STG_BYTES +
+         256 /*barriers*/ + (size_t)(G + 1 + TC_THREADS / 32 + 1) * sizeof(int);
 }
 
 template <int MODE, int BN>
@@ -159,11 +180,12 @@ __global__ void __launch_bounds__(TC_THREADS, 1) gemm_tc_kernel(const __grid_con
   const uint32_t pad = ((raw + 1023u) & ~1023u) - raw;
   unsigned char *base = smem_raw + pad;
   unsigned char *stages = base;
-  uint64_t *bars = (uint64_t *)(base + (size_t)C::STAGES * C::STAGE_BYTES);
+  unsigned char *stg_all = base + (size_t)C::STAGES * C::STAGE_BYTES;  // [8 warps][4 KB]
+  uint64_t *bars = (uint64_t *)(stg_all + C::STG_BYTES);
   // bars: full[STAGES], empty[STAGES], acc_full[2], acc_empty[2], drain
   uint32_t *tmem_slot = (uint32_t *)(bars + 2 * C::STAGES + 5);
   volatile int *abort_flag = (volatile int *)(tmem_slot + 1);
-  int *prefix = (int *)(base + (size_t)C::STAGES * C::STAGE_BYTES + 256);
+  int *prefix = (int *)(stg_all + C::STG_BYTES + 256);
   int *scan_tmp = prefix + G + 1;
 
   auto full_bar = [&](int s) { return smem_u32(bars + s); };
@@ -179,7 +201,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) gemm_tc_kernel(const __grid_con
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(accf_bar(b), 1);
-      mbar_init(acce_bar(b), 4);
+      mbar_init(acce_bar(b), TC_EPI_WARPS);
     }
     mbar_init(drain_bar, 1);
     *abort_flag = 0;
@@ -288,10 +310,6 @@ __global__ void __launch_bounds__(TC_THREADS, 1) gemm_tc_kernel(const __grid_con
             const uint64_t bd0 = make_sdesc(sB0 + k16 * 32);
             const uint32_t accum = (kb > 0 || k16 > 0) ? 1u : 0u;
             tc_mma(d0, ad, bd0, C::IDESC, accum);
-            if (C::NB == 2) {
-              const uint64_t bd1 = make_sdesc(sB0 + C::B_BYTES + k16 * 32);
-              tc_mma(d0 + BN, ad, bd1, C::IDESC, accum);
-            }
           }
           any = true;
           tc_commit(empty_bar(stage));
@@ -310,8 +328,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1) gemm_tc_kernel(const __grid_con
     }
     __syncwarp();
   } else {
-    // ------------------------------------------------------------ epilogue (warps 2..5)
-    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    // ------------------------------------------------------------ epilogue (warps 2..9)
+    const int q = warp & 3;                            // TMEM lane quarter this warp may access
+    const int half = (warp - 2) >> 2;                  // which half of the tile's columns
+    const int cbeg = half * (BN / 2), cend = cbeg + BN / 2;
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
@@ -328,38 +348,70 @@ __global__ void __launch_bounds__(TC_THREADS, 1) gemm_tc_kernel(const __grid_con
       void *out = routed ? p.out_r : p.out_s;
       const int ldo = routed ? p.ldo_r : p.ldo_s;
       const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * C::ACC_COLS);
+      // fp32 outputs (expert outputs) use a staged write-back: the warp's 32 rows x 32 columns
+      // go to a private 4 KB buffer (16-byte chunk j of row r stored at chunk j ^ (r & 7), so
+      // both the row-wise writes and the column-wise reads are conflict-free), then leave as 32
+      // row stores of 128 contiguous bytes each instead of 32-row scattered 16-byte stores.
+      unsigned char *stg = stg_all + (warp - 2) * 4096;
+      constexpr int SUB = (MODE == MODE_PLAIN) ? 1 : 2;  // 32-column TMEM loads per block
 #pragma unroll 1
-      for (int c = 0; c < BN; c += 16) {
-        uint32_t r0[16], r1[16];
-        tmem_ld16(tbase + c, r0);
-        if (C::NB == 2) tmem_ld16(tbase + BN + c, r1);
-        tmem_wait_ld();
-        const int col = ti.n0 + c;
-        if (row_ok && col < ti.N) {
-          float v[16];
+      for (int c = cbeg; c < cend; c += 32 * SUB) {
+        if (MODE != MODE_PLAIN) {
+          // bf16 outputs (SwiGLU hidden, low-rank projection): each lane already writes 64
+          // contiguous bytes of its row, so they go out directly
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const float g = __uint_as_float(r0[i]);
-            if (MODE == MODE_GATEUP) v[i] = silu_f(g) * __uint_as_float(r1[i]);
-            else if (MODE == MODE_SCALE) v[i] = g * __ldg(p.scale + (size_t)ti.g * ti.N + col + i);
-            else v[i] = g;
+          for (int sub = 0; sub < SUB; ++sub) {
+            uint32_t r0[32], r1[32];
+            tmem_ld32(tbase + c + 32 * sub, r0);
+            if (C::NB == 2) tmem_ld32(tbase + BN + c + 32 * sub, r1);
+            tmem_wait_ld();
+            const int col = ti.n0 + c + 32 * sub;
+            if (row_ok && col < ti.N) {
+              uint4 pk[4];
+              __nv_bfloat162 *h = (__nv_bfloat162 *)pk;
+#pragma unroll
+              for (int i = 0; i < 16; ++i) {
+                const float g0 = __uint_as_float(r0[2 * i]), g1 = __uint_as_float(r0[2 * i + 1]);
+                float v0, v1;
+                if (MODE == MODE_GATEUP) {
+                  v0 = __fdividef(g0, 1.0f + __expf(-g0)) * __uint_as_float(r1[2 * i]);
+                  v1 = __fdividef(g1, 1.0f + __expf(-g1)) * __uint_as_float(r1[2 * i + 1]);
+                } else {
+                  v0 = g0 * __ldg(p.scale + (size_t)ti.g * ti.N + col + 2 * i);
+                  v1 = g1 * __ldg(p.scale + (size_t)ti.g * ti.N + col + 2 * i + 1);
+                }
+                h[i] = __floats2bfloat162_rn(v0, v1);
+              }
+              uint4 *dst = (uint4 *)((__nv_bfloat16 *)out + (size_t)(ti.a_row0 + row) * ldo + col);
+#pragma unroll
+              for (int i = 0; i < 4; ++i) dst[i] = pk[i];
+            }
           }
-          if (MODE == MODE_PLAIN) {
-            // expert outputs stay fp32 (combined in fp32 downstream)
-            float4 *dst = (float4 *)((float *)out + (size_t)(ti.a_row0 + row) * ldo + col);
+          continue;
+        }
+        {
+          uint32_t r0[32];
+          tmem_ld32(tbase + c, r0);
+          tmem_wait_ld();
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
-              dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
-          } else {
-            uint4 pk[2];
-            __nv_bfloat162 *h = (__nv_bfloat162 *)pk;
-#pragma unroll
-            for (int i = 0; i < 8; ++i) h[i] = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
-            uint4 *dst = (uint4 *)((__nv_bfloat16 *)out + (size_t)(ti.a_row0 + row) * ldo + col);
-            dst[0] = pk[0];
-            dst[1] = pk[1];
+          for (int i = 0; i < 8; ++i)
+            *(uint4 *)(stg + lane * 128 + ((i ^ (lane & 7)) << 4)) =
+                make_uint4(r0[4 * i], r0[4 * i + 1], r0[4 * i + 2], r0[4 * i + 3]);
+        }
+        __syncwarp();
+        const int col = ti.n0 + c;
+        if (col < ti.N) {
+          const int rbase = ti.m0 + q * 32;
+          const int nrows = min(32, ti.rows - rbase);
+          unsigned char *obase = (unsigned char *)out + ((size_t)(ti.a_row0 + rbase) * ldo + col) * 4;
+          const size_t row_bytes = (size_t)ldo * 4;
+          for (int rr = 0; rr < nrows; ++rr) {
+            const uint32_t v = *(const uint32_t *)(stg + rr * 128 + (((lane >> 2) ^ (rr & 7)) << 4) +
+                                                   ((lane & 3) << 2));
+            *(uint32_t *)(obase + rr * row_bytes + lane * 4) = v;
           }
         }
+        __syncwarp();
       }
       tc_fence_before();
       __syncwarp();

@@ -17,8 +17,11 @@
 #include "gemm_tc.cuh"
 #include "permute.cuh"
 #include "router.cuh"
+#include "stats.cuh"
 
 using namespace moe;
+
+static_assert(RT_TM == PM_CHUNK, "the router CTA is the permutation chunk");
 
 namespace {
 
@@ -79,8 +82,8 @@ int32_t capacity_of(const moe_config_t *c) {
 
 // ------------------------------------------------------------------ workspace layout
 struct Layout {
-  size_t w64, wnorm, part_cnt, part_prob, rcounter;             // route
-  size_t chunk_count, chunk_base, ptotal, pcounter;             // permute
+  size_t part_cnt, part_prob, chunk_base, kept, scounter;       // route / statistics
+  size_t chunk_count;                                           // moe_permute's own histogram
   size_t hidden, hidden_sh;                                     // experts
   size_t idx, wts, count, prob, offsets, slot_pos, src, x_perm, y_perm, y_shared, aux;  // layer
   size_t total;
@@ -89,20 +92,16 @@ struct Layout {
 Layout layout_of(const moe_config_t *c) {
   Layout L;
   const size_t T = c->T, d = c->d, E = c->E, k = c->top_k, es = esize(c);
-  const size_t nblk = std::max<size_t>(1, ceil_div(c->T, RT_TM));
-  const size_t nch = std::max<size_t>(1, ceil_div(c->T, PM_CHUNK));
+  const size_t nch = std::max<size_t>(1, ceil_div(c->T, RT_TM));
   const size_t width = c->expert == MOE_EXPERT_SWIGLU ? (size_t)c->ffn : (size_t)c->rank;
   size_t o = 0;
   auto take = [&](size_t bytes) { size_t at = o; o = align256(o + std::max<size_t>(bytes, 1)); return at; };
-  L.w64 = take(E * d * 8);
-  L.wnorm = take(E * 8);
-  L.part_cnt = take(nblk * E * 4);
-  L.part_prob = take(nblk * E * 4);
-  L.rcounter = take(16);
-  L.chunk_count = take(nch * E * 4);
+  L.part_cnt = take(nch * E * 4);
+  L.part_prob = take(nch * E * 4);
   L.chunk_base = take(nch * E * 4);
-  L.ptotal = take(E * 4);
-  L.pcounter = take(16);
+  L.kept = take(E * 4);
+  L.scounter = take(16);
+  L.chunk_count = take(nch * E * 4);
   L.hidden = take(T * k * width * es);
   L.hidden_sh = take(T * (size_t)c->n_shared * (size_t)c->ffn_shared * es);
   L.idx = take(T * k * 4);
@@ -147,12 +146,12 @@ int num_sms() {
 
 // ------------------------------------------------------------------ profiling (debug)
 enum KernelKind {
-  K_ROUTER_PREP, K_ROUTER, K_PERM_HIST, K_PERM_SCAN, K_PERM_SCATTER, K_GEMM_GATEUP, K_GEMM_DOWN,
-  K_GEMM_LR1, K_GEMM_LR2, K_COMBINE, K_AUX, K_COUNT
+  K_ROUTER, K_STATS, K_PERM_HIST, K_PERM_SCATTER, K_GEMM_GATEUP, K_GEMM_DOWN, K_GEMM_LR1,
+  K_GEMM_LR2, K_COMBINE, K_AUX, K_COUNT
 };
-const char *kKindName[K_COUNT] = {"router_prep", "router", "perm_hist", "perm_scan",
-                                  "perm_scatter", "gemm_gateup", "gemm_down", "gemm_lowrank_v",
-                                  "gemm_lowrank_u", "combine", "aux_loss"};
+const char *kKindName[K_COUNT] = {"router", "stats", "perm_hist", "perm_scatter", "gemm_gateup",
+                                  "gemm_down", "gemm_lowrank_v", "gemm_lowrank_u", "combine",
+                                  "aux_loss"};
 constexpr int PROF_SLOTS = 8192;
 struct Prof {
   bool on = false;
@@ -292,29 +291,63 @@ moe_status_t launch_gemm(const moe_config_t *c, const GroupedGemm &g, int bn_hin
     if (_s != MOE_OK) return _s;        \
   } while (0)
 
-template <typename Tin, int RE>
-moe_status_t launch_router_re(const RouterArgs &a, cudaStream_t st) {
-  const size_t smem = router_smem_bytes(a.E, RE);
-  if (cudaFuncSetAttribute(router_kernel<Tin, RE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+template <typename Tin, int NT>
+moe_status_t launch_router_nt(const RouterArgs &a, cudaStream_t st) {
+  const size_t smem = router_smem(a.E, a.d, NT, (int)sizeof(Tin), a.score == MOE_SCORE_SIGMOID).total;
+  if (smem > 227 * 1024) return MOE_ERR_UNSUPPORTED;
+  if (cudaFuncSetAttribute(router_kernel<Tin, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)smem) != cudaSuccess)
     return MOE_ERR_CUDA;
-  router_kernel<Tin, RE><<<ceil_div(a.T, RT_TM), RT_THREADS, smem, st>>>(a);
+  router_kernel<Tin, NT><<<ceil_div(a.T, RT_TM), RT_THREADS, smem, st>>>(a);
   return last_launch_status();
 }
 
 template <typename Tin>
 moe_status_t launch_router(const RouterArgs &a, cudaStream_t st) {
-  moe_status_t s;
-  switch (router_re_for(a.E)) {
-    case 2: s = launch_router_re<Tin, 2>(a, st); break;
-    case 4: s = launch_router_re<Tin, 4>(a, st); break;
-    case 6: s = launch_router_re<Tin, 6>(a, st); break;
-    default: s = launch_router_re<Tin, 8>(a, st); break;
+  ProfScope ps(K_ROUTER, st);
+  switch (router_nt_for(a.E)) {
+    case 1: return launch_router_nt<Tin, 1>(a, st);
+    case 2: return launch_router_nt<Tin, 2>(a, st);
+    case 3: return launch_router_nt<Tin, 3>(a, st);
+    default: return launch_router_nt<Tin, 4>(a, st);
   }
-  if (s != MOE_OK) return s;
-  router_reduce_kernel<<<a.E, 128, 0, st>>>(a.part_cnt, a.part_prob, ceil_div(a.T, RT_TM), a.E,
-                                           a.count_out, a.prob_out);
+}
+
+moe_status_t launch_stats(const StatsArgs &sa, cudaStream_t st) {
+  ProfScope ps(K_STATS, st);
+  moe_stats_kernel<<<sa.E, ST_THREADS, 0, st>>>(sa);
   return last_launch_status();
+}
+
+template <typename Tin>
+moe_status_t router_only(const moe_config_t *c, const void *x, const moe_weights_t *w,
+                         int32_t *idx, float *wts, int32_t *part_cnt, float *part_prob,
+                         unsigned *counter, cudaStream_t st) {
+  RouterArgs a;
+  a.x = x;
+  a.w = w->w_router;
+  a.off = w->logit_offset;
+  a.bias = c->score == MOE_SCORE_SIGMOID ? w->select_bias : nullptr;
+  a.T = c->T; a.d = c->d; a.E = c->E; a.k = c->top_k; a.score = c->score; a.norm = c->norm_topk;
+  a.idx = idx; a.wts = wts;
+  a.part_cnt = part_cnt;
+  a.part_prob = part_prob;
+  a.counter = counter;
+  return launch_router<Tin>(a, st);
+}
+
+StatsArgs stats_args(const moe_config_t *c, const int32_t *chunk_cnt, const float *chunk_prob,
+                     unsigned *counter) {
+  StatsArgs sa;
+  std::memset(&sa, 0, sizeof(sa));
+  sa.chunk_cnt = chunk_cnt;
+  sa.chunk_prob = chunk_prob;
+  sa.nchunk = ceil_div(c->T, RT_TM);
+  sa.E = c->E; sa.T = c->T; sa.k = c->top_k;
+  sa.C = capacity_of(c);
+  sa.alpha = c->aux_alpha;
+  sa.counter = counter;
+  return sa;
 }
 
 template <typename Tin>
@@ -327,26 +360,25 @@ moe_status_t route_impl(const moe_config_t *c, const void *x, const moe_weights_
     if (cudaMemsetAsync(prob, 0, (size_t)c->E * 4, st) != cudaSuccess) return MOE_ERR_CUDA;
     return MOE_OK;
   }
-  RouterArgs a;
-  a.x = x;
-  a.w64 = at<double>(ws, L.w64);
-  a.wnorm = at<double>(ws, L.wnorm);
-  a.off = w->logit_offset;
-  a.bias = c->score == MOE_SCORE_SIGMOID ? w->select_bias : nullptr;
-  a.T = c->T; a.d = c->d; a.E = c->E; a.k = c->top_k; a.score = c->score; a.norm = c->norm_topk;
-  a.idx = idx; a.wts = wts;
-  a.part_cnt = at<int32_t>(ws, L.part_cnt);
-  a.part_prob = at<float>(ws, L.part_prob);
-  a.count_out = count; a.prob_out = prob;
-  a.counter = at<unsigned>(ws, L.rcounter);
-  {
-    ProfScope ps(K_ROUTER_PREP, st);
-    router_prep_kernel<Tin><<<c->E, 256, 0, st>>>((const Tin *)w->w_router, c->E, c->d,
-                                                   (double *)a.w64, (double *)a.wnorm, a.counter);
-    MOE_TRY(last_launch_status());
-  }
-  ProfScope ps(K_ROUTER, st);
-  return launch_router<Tin>(a, st);
+  int32_t *pc = at<int32_t>(ws, L.part_cnt);
+  float *pp = at<float>(ws, L.part_prob);
+  unsigned *ctr = at<unsigned>(ws, L.scounter);
+  MOE_TRY(router_only<Tin>(c, x, w, idx, wts, pc, pp, ctr, st));
+  StatsArgs sa = stats_args(c, pc, pp, ctr);
+  sa.count_out = count;
+  sa.prob_out = prob;
+  return launch_stats(sa, st);
+}
+
+template <typename Tin>
+moe_status_t scatter_impl(const moe_config_t *c, const void *x, const int32_t *idx,
+                          const int32_t *chunk_base, const int32_t *offsets, int32_t *slot_pos,
+                          int32_t *src, void *x_perm, cudaStream_t st) {
+  ProfScope ps(K_PERM_SCATTER, st);
+  perm_scatter_kernel<Tin><<<ceil_div(c->T, PM_CHUNK), 256, (size_t)c->E * 4, st>>>(
+      idx, c->T, c->top_k, c->E, capacity_of(c), chunk_base, offsets, slot_pos, src,
+      (const Tin *)x, (Tin *)x_perm, c->d);
+  return last_launch_status();
 }
 
 template <typename Tin>
@@ -358,30 +390,22 @@ moe_status_t permute_impl(const moe_config_t *c, const void *x, const int32_t *i
     return cudaMemsetAsync(offsets, 0, (size_t)(c->E + 1) * 4, st) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
   }
   const int nch = ceil_div(c->T, PM_CHUNK);
-  const int C = capacity_of(c);
   int32_t *cc = at<int32_t>(ws, L.chunk_count), *cb = at<int32_t>(ws, L.chunk_base);
-  unsigned *counter = at<unsigned>(ws, L.pcounter);
+  unsigned *ctr = at<unsigned>(ws, L.scounter);
   {
     const size_t smem = (size_t)8 * c->E * 4;
     if (cudaFuncSetAttribute(perm_hist_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
       return MOE_ERR_CUDA;
     ProfScope ps(K_PERM_HIST, st);
-    perm_hist_kernel<<<ceil_div(nch, 8), 256, smem, st>>>(idx, c->T, c->top_k, c->E, cc, nch, counter);
+    perm_hist_kernel<<<ceil_div(nch, 8), 256, smem, st>>>(idx, c->T, c->top_k, c->E, cc, nch, ctr);
     MOE_TRY(last_launch_status());
   }
-  {
-    const size_t smem = (size_t)(c->E + 256 / 32 + 1) * 4;
-    ProfScope ps(K_PERM_SCAN, st);
-    perm_scan_kernel<<<ceil_div(c->E, 8), 256, smem, st>>>(cc, cb, nch, c->E, C,
-                                                           at<int32_t>(ws, L.ptotal), offsets, counter);
-    MOE_TRY(last_launch_status());
-  }
-  {
-    ProfScope ps(K_PERM_SCATTER, st);
-    perm_scatter_kernel<Tin><<<nch, 256, (size_t)c->E * 4, st>>>(
-        idx, c->T, c->top_k, c->E, C, cb, offsets, slot_pos, src, (const Tin *)x, (Tin *)x_perm, c->d);
-    return last_launch_status();
-  }
+  StatsArgs sa = stats_args(c, cc, nullptr, ctr);
+  sa.chunk_base = cb;
+  sa.kept = at<int32_t>(ws, L.kept);
+  sa.offsets = offsets;
+  MOE_TRY(launch_stats(sa, st));
+  return scatter_impl<Tin>(c, x, idx, cb, offsets, slot_pos, src, x_perm, st);
 }
 
 moe_status_t experts_impl(const moe_config_t *c, const void *x_perm, const int32_t *offsets,
@@ -584,16 +608,33 @@ moe_status_t moe_layer_forward(const moe_config_t *cfg, const void *x, const moe
   void *y_perm = at<char>(ws, L.y_perm);
   void *y_sh = at<char>(ws, L.y_shared);
   float *aux = aux_loss ? aux_loss : at<float>(ws, L.aux);
-  if (cfg->dtype == MOE_DTYPE_BF16) {
-    MOE_TRY(route_impl<__nv_bfloat16>(cfg, x, w, idx, wts, cnt, prob, ws, st));
-    MOE_TRY(permute_impl<__nv_bfloat16>(cfg, x, idx, offsets, slot_pos, src, x_perm, ws, st));
-  } else {
-    MOE_TRY(route_impl<float>(cfg, x, w, idx, wts, cnt, prob, ws, st));
-    MOE_TRY(permute_impl<float>(cfg, x, idx, offsets, slot_pos, src, x_perm, ws, st));
+  if (cfg->T == 0) {
+    if (cudaMemsetAsync(cnt, 0, (size_t)cfg->E * 4, st) != cudaSuccess) return MOE_ERR_CUDA;
+    return cudaMemsetAsync(aux, 0, 4, st) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
   }
+  // route -> statistics (counts, probability sums, chunk scans, offsets, loss) -> scatter
+  int32_t *pc = at<int32_t>(ws, L.part_cnt);
+  float *pp = at<float>(ws, L.part_prob);
+  int32_t *cb = at<int32_t>(ws, L.chunk_base);
+  unsigned *ctr = at<unsigned>(ws, L.scounter);
+  if (cfg->dtype == MOE_DTYPE_BF16)
+    MOE_TRY(router_only<__nv_bfloat16>(cfg, x, w, idx, wts, pc, pp, ctr, st));
+  else
+    MOE_TRY(router_only<float>(cfg, x, w, idx, wts, pc, pp, ctr, st));
+  StatsArgs sa = stats_args(cfg, pc, pp, ctr);
+  sa.count_out = cnt;
+  sa.prob_out = prob;
+  sa.chunk_base = cb;
+  sa.kept = at<int32_t>(ws, L.kept);
+  sa.offsets = offsets;
+  sa.aux = aux;
+  MOE_TRY(launch_stats(sa, st));
+  if (cfg->dtype == MOE_DTYPE_BF16)
+    MOE_TRY(scatter_impl<__nv_bfloat16>(cfg, x, idx, cb, offsets, slot_pos, src, x_perm, st));
+  else
+    MOE_TRY(scatter_impl<float>(cfg, x, idx, cb, offsets, slot_pos, src, x_perm, st));
   MOE_TRY(experts_impl(cfg, x_perm, offsets, x, w, y_perm, y_sh, ws, st));
-  MOE_TRY(combine_impl(cfg, y_perm, y_sh, slot_pos, wts, y, st));
-  return aux_impl(cfg, cnt, prob, aux, st);
+  return combine_impl(cfg, y_perm, y_sh, slot_pos, wts, y, st);
 }
 
 const char *moe_status_str(moe_status_t s) {
@@ -728,17 +769,15 @@ moe_status_t route_scratch_address(void **out) {
 }
 
 struct RouteScratch {
-  size_t w64, wnorm, part_cnt, part_prob, counter, total;
+  size_t part_cnt, part_prob, counter, total;
 };
 
 RouteScratch route_scratch_layout(const moe_config_t *c) {
   RouteScratch L;
-  const size_t E = c->E, d = c->d;
+  const size_t E = c->E;
   const size_t nblk = std::max<size_t>(1, ceil_div(c->T, RT_TM));
   size_t o = 0;
   auto take = [&](size_t bytes) { size_t at = o; o = align256(o + std::max<size_t>(bytes, 1)); return at; };
-  L.w64 = take(E * d * 8);
-  L.wnorm = take(E * 8);
   L.part_cnt = take(nblk * E * 4);
   L.part_prob = take(nblk * E * 4);
   L.counter = take(16);
@@ -756,24 +795,16 @@ moe_status_t route_noalloc_impl(const moe_config_t *c, const void *x, const moe_
     if (cudaMemsetAsync(prob, 0, (size_t)c->E * 4, st) != cudaSuccess) return MOE_ERR_CUDA;
     return MOE_OK;
   }
-  RouterArgs a;
-  a.x = x;
-  a.w64 = (const double *)(scratch + L.w64);
-  a.wnorm = (const double *)(scratch + L.wnorm);
-  a.off = w->logit_offset;
-  a.bias = c->score == MOE_SCORE_SIGMOID ? w->select_bias : nullptr;
-  a.T = c->T; a.d = c->d; a.E = c->E; a.k = c->top_k; a.score = c->score; a.norm = c->norm_topk;
-  a.idx = idx; a.wts = wts;
-  a.part_cnt = (int32_t *)(scratch + L.part_cnt);
-  a.part_prob = (float *)(scratch + L.part_prob);
-  a.count_out = count; a.prob_out = prob;
-  a.counter = (unsigned *)(scratch + L.counter);
-  // router_prep_kernel rewrites the fp64 weight and the norms and clears the completion
-  // counter on every call, so nothing left in the array by an earlier call is read.
-  router_prep_kernel<Tin><<<c->E, 256, 0, st>>>((const Tin *)w->w_router, c->E, c->d,
-                                                 (double *)a.w64, (double *)a.wnorm, a.counter);
-  MOE_TRY(last_launch_status());
-  return launch_router<Tin>(a, st);
+  // every call rewrites the per-CTA partials before reading them, and the router clears the
+  // counter, so nothing left in the array by an earlier call is read
+  int32_t *pc = (int32_t *)(scratch + L.part_cnt);
+  float *pp = (float *)(scratch + L.part_prob);
+  unsigned *ctr = (unsigned *)(scratch + L.counter);
+  MOE_TRY(router_only<Tin>(c, x, w, idx, wts, pc, pp, ctr, st));
+  StatsArgs sa = stats_args(c, pc, pp, ctr);
+  sa.count_out = count;
+  sa.prob_out = prob;
+  return launch_stats(sa, st);
 }
 
 }  // namespace

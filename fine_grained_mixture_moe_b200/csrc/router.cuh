@@ -27,26 +27,35 @@ namespace moe {
 
 constexpr int RT_TM = 16;          // tokens per CTA
 constexpr int RT_THREADS = 256;    // 8 warps, each a slice of the K dimension
-constexpr int RT_KC = 32;          // k-chunk staged (fp64) in a warp's shared-memory slot
-constexpr int RT_LD = RT_KC + 2;   // padded row: 68 words = 4 (mod 32), conflict-free 16 B loads
+constexpr int RT_KB = 16;          // k block: lane (row r, column c) of a fragment reads the 4
+                                   // consecutive elements 4c..4c+3 of the block with one load
+constexpr int RT_SEL_THREAD_MAX_E = 64;  // up to this many experts, one thread selects per token
 constexpr int EXPANSION_MAX = 40;
 constexpr int RT_FIX_CAP = 256;   // flagged logits per CTA kept with their fp64 sums
 
-// Experts per thread in one round (a round covers 4*RE experts): the RE in {8,6,4,2} that wastes
-// the fewest padded expert slots over all rounds, larger RE on ties.
-inline int router_re_for(int E) {
-  int best = 8, waste = 1 << 30;
-  for (int re : {8, 6, 4, 2}) {
-    const int eb = 4 * re, w = ((E + eb - 1) / eb) * eb - E;
-    if (w < waste) { waste = w; best = re; }
+// Expert tiles of 8 per round (a round covers 8*NT experts): the NT in {4,3,2,1} that wastes the
+// fewest padded expert slots over all rounds, larger NT on ties.
+inline int router_nt_for(int E) {
+  int best = 4, waste = 1 << 30;
+  for (int nt : {4, 3, 2, 1}) {
+    const int eb = 8 * nt, w = ((E + eb - 1) / eb) * eb - E;
+    if (w < waste) { waste = w; best = nt; }
   }
   return best;
 }
 
+// D(8x8) += A(8x4) B(4x8) in fp64 on the tensor cores. Fragments: lane l holds A[l/4][l%4],
+// B[l%4][l/4] and D[l/4][2(l%4) + {0,1}]. Every product of bf16 or fp32 inputs is exact in fp64
+// and each accumulation is an fp64 rounding, so the summation error bound below still holds.
+__device__ __forceinline__ void dmma_8x8x4(double (&d)[2], double a, double b) {
+  asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0, %1}, {%2}, {%3}, {%0, %1};"
+               : "+d"(d[0]), "+d"(d[1])
+               : "d"(a), "d"(b));
+}
+
 struct RouterArgs {
   const void *x;
-  const double *w64;    // [E, d] router weight in fp64 (prep kernel)
-  const double *wnorm;  // [E] l2 norms
+  const void *w;        // [E, d] router weight in the input dtype
   const float *off;     // [E] or null
   const float *bias;    // [E] or null
   int T, d, E, k, score, norm;
@@ -56,7 +65,7 @@ struct RouterArgs {
   float *part_prob;     // [nblk, E]
   int32_t *count_out;   // [E]
   float *prob_out;      // [E]
-  unsigned int *counter;
+  unsigned int *counter; // completion counter of the statistics kernel, cleared here
 };
 
 // ------------------------------------------------------------------ exact expansion sums
@@ -115,7 +124,7 @@ __device__ __forceinline__ bool rn32_certain(double v, double B, float &r, float
 }
 
 template <typename Tin>
-__device__ __noinline__ float exact_logit(const Tin *xrow, const double *wrow, int d, double off,
+__device__ __noinline__ float exact_logit(const Tin *xrow, const Tin *wrow, int d, double off,
                                           double approx) {
   float r, up, dn;
   double mh, ml;
@@ -124,7 +133,7 @@ __device__ __noinline__ float exact_logit(const Tin *xrow, const double *wrow, i
   X.n = 0;
   X.overflow = false;
   for (int i = 0; i < d; ++i) {
-    const double p = __dmul_rn((double)Elem<Tin>::to_f(xrow[i]), wrow[i]);  // exact
+    const double p = __dmul_rn((double)Elem<Tin>::to_f(xrow[i]), (double)Elem<Tin>::to_f(wrow[i]));  // exact
     if (p != 0.0) expansion_add(X, p);
   }
   if (off != 0.0) expansion_add(X, off);
@@ -217,7 +226,7 @@ __device__ __forceinline__ void load8(const double *p, double *v) {
 }
 
 template <typename Tin>
-__device__ bool warp_exact_signs(const Tin *xrow, const double *wrow, int d, double off,
+__device__ bool warp_exact_signs(const Tin *xrow, const Tin *wrow, int d, double off,
                                  double mh, double ml, int &c_hi, int &c_lo) {
   const int lane = threadIdx.x & 31;
   int qmin = 0x7fffffff, emax = -0x7fffffff;
@@ -275,7 +284,7 @@ __device__ bool warp_exact_signs(const Tin *xrow, const double *wrow, int d, dou
 // even. force_level 2 skips the integer path and sends the logit to the single-thread
 // expansion, to test that path too.
 template <typename Tin>
-__device__ __noinline__ float resolve_logit(const Tin *xrow, const double *wrow, int d, double off,
+__device__ __noinline__ float resolve_logit(const Tin *xrow, const Tin *wrow, int d, double off,
                                             double approx, int force_level) {
   const int lane = threadIdx.x & 31;
   float r, up, dn;
@@ -347,138 +356,152 @@ __device__ float sigmoid_key(float l, float b, bool force) {
 }
 
 // ------------------------------------------------------------------ kernels
-// fp64 copy of the router weight and its row norms; also clears the completion counter.
-template <typename Tin>
-__global__ void __launch_bounds__(256) router_prep_kernel(const Tin *__restrict__ w, int E, int d,
-                                                          double *__restrict__ w64,
-                                                          double *__restrict__ wnorm,
-                                                          unsigned *counter) {
-  const int e = blockIdx.x;
-  double s = 0.0;
-  for (int i = threadIdx.x; i < d; i += blockDim.x) {
-    const double v = (double)Elem<Tin>::to_f(w[(size_t)e * d + i]);
-    w64[(size_t)e * d + i] = v;
-    s = fma(v, v, s);
-  }
-  __shared__ double red[8];
-  s = warp_sum_d(s);
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = s;
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    double t = 0.0;
-    for (int i = 0; i < (int)(blockDim.x >> 5); ++i) t += red[i];
-    wnorm[e] = sqrt(t);
-    if (e == 0) *counter = 0u;
-  }
+// Shared-memory layout of the router kernel (byte offsets), shared by host and device.
+struct RouterSmem {
+  size_t xs, wsb, part, lg, pb, keys, sel_e, sel_p, wn, cnt, flags, xnorm, fix, total;
+  int ldx;  // padded row length of xs / wsb in elements: (ldx * esize) = 32 (mod 128)
+};
+__host__ __device__ inline RouterSmem router_smem(int E, int d, int NT, int esize, bool sigmoid) {
+  RouterSmem L;
+  const int EB = 8 * NT;
+  L.ldx = d + 32 / esize;
+  size_t o = 0;
+  auto take = [&](size_t bytes) { size_t at = o; o = (o + bytes + 15) & ~(size_t)15; return at; };
+  L.xs = take((size_t)RT_TM * L.ldx * esize);
+  L.wsb = take((size_t)EB * L.ldx * esize);
+  L.part = take((size_t)(RT_THREADS / 32) * RT_TM * EB * sizeof(double));
+  L.lg = take((size_t)RT_TM * E * sizeof(float));
+  const bool rank_sel = E <= RT_SEL_THREAD_MAX_E;
+  L.pb = take(rank_sel ? (size_t)RT_TM * E * sizeof(float) : 0);
+  // sigmoid keys: [16][E] for the rank selection; the warp selection keeps [8][E] in wsb
+  L.keys = take(sigmoid && rank_sel ? (size_t)RT_TM * E * sizeof(float) : 0);
+  L.sel_e = take((size_t)RT_TM * 8 * sizeof(int));
+  L.sel_p = take((size_t)RT_TM * 8 * sizeof(float));
+  L.wn = take((size_t)EB * sizeof(double));
+  L.cnt = take((size_t)E * sizeof(int));
+  L.flags = take((size_t)RT_TM * ((E + 31) / 32) * sizeof(unsigned));
+  L.xnorm = take(RT_TM * sizeof(double));
+  L.fix = take(RT_FIX_CAP * sizeof(double));
+  L.total = o;
+  return L;
 }
 
-__host__ __device__ inline size_t router_smem_bytes(int E, int RE) {
-  size_t b = (size_t)(RT_THREADS / 32) * (RT_TM + 4 * RE) * RT_LD * sizeof(double);  // staging
-  b += (size_t)RT_TM * E * sizeof(float);                  // logits / probabilities
-  b += (size_t)(RT_THREADS / 32) * E * sizeof(float);      // per-warp sigmoid keys
-  b += (size_t)E * sizeof(int);                             // selection counts
-  b += (size_t)RT_TM * ((E + 31) / 32) * sizeof(unsigned);  // undecided-logit flags
-  b = (b + 15) & ~(size_t)15;
-  b += RT_TM * sizeof(double);                              // token norms
-  b += (size_t)RT_FIX_CAP * sizeof(double);                 // fp64 sums of flagged logits
-  return b;
+// Four consecutive inputs as fp64 (bf16: one 8-byte load; fp32: one 16-byte load).
+__device__ __forceinline__ void load4d(const __nv_bfloat16 *p, double (&v)[4]) {
+  const uint2 q = *(const uint2 *)p;
+  const __nv_bfloat162 *h = (const __nv_bfloat162 *)&q;
+  const float2 f0 = __bfloat1622float2(h[0]), f1 = __bfloat1622float2(h[1]);
+  v[0] = f0.x; v[1] = f0.y; v[2] = f1.x; v[3] = f1.y;
+}
+__device__ __forceinline__ void load4d(const float *p, double (&v)[4]) {
+  const float4 q = *(const float4 *)p;
+  v[0] = q.x; v[1] = q.y; v[2] = q.z; v[3] = q.w;
 }
 
-template <typename Tin, int RE>
+template <typename Tin, int NT>
 __global__ void __launch_bounds__(RT_THREADS, 2) router_kernel(RouterArgs a) {
-  constexpr int EB = 4 * RE;  // experts per round
+  constexpr int EB = 8 * NT;  // experts per round
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   const int E = a.E, d = a.d, k = a.k;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int lt = lane >> 2, le = lane & 3;  // thread tile: tokens {lt, lt+8} x experts {le+4j}
+  const int fr = lane >> 2, fc = lane & 3;  // fragment row / column of this lane
   const int t0 = blockIdx.x * RT_TM;
   const int ntok = min(RT_TM, a.T - t0);
   const Tin *__restrict__ x = (const Tin *)a.x;
+  const Tin *__restrict__ wr = (const Tin *)a.w;
   const int force_level = g_force_exact;
   const bool force = force_level != 0;
-
-  double *stage = (double *)smem_raw;
-  double *xs = stage + warp * (RT_TM + EB) * RT_LD;  // this warp's [16][RT_LD] x chunk
-  double *wsm = xs + RT_TM * RT_LD;                  // this warp's [EB][RT_LD] W chunk
-  double *part = stage;                              // reused: [8 warps][16][EB] partial sums
-  float *lg = (float *)(stage + (RT_THREADS / 32) * (RT_TM + EB) * RT_LD);
-  float *keys = lg + RT_TM * E;
-  int *cnt = (int *)(keys + (RT_THREADS / 32) * E);
+  const bool sigmoid = a.score == MOE_SCORE_SIGMOID;
+  const RouterSmem SL = router_smem(E, d, NT, (int)sizeof(Tin), sigmoid);
+  const int ldx = SL.ldx;
+  Tin *xs = (Tin *)(smem_raw + SL.xs);    // [16][ldx] the CTA's tokens
+  Tin *wsb = (Tin *)(smem_raw + SL.wsb);  // [EB][ldx] the round's router rows
+  double *part = (double *)(smem_raw + SL.part);
+  float *lg = (float *)(smem_raw + SL.lg);
+  float *keys = (float *)(smem_raw + (E <= RT_SEL_THREAD_MAX_E ? SL.keys : SL.wsb));
+  const bool rank_sel = E <= RT_SEL_THREAD_MAX_E;
+  float *pb = rank_sel ? (float *)(smem_raw + SL.pb) : lg;
+  int *sel_e = (int *)(smem_raw + SL.sel_e);
+  float *sel_p = (float *)(smem_raw + SL.sel_p);
+  double *wn = (double *)(smem_raw + SL.wn);  // [EB] norms of the round's rows
+  int *cnt = (int *)(smem_raw + SL.cnt);
   const int nfw = (E + 31) / 32;
-  unsigned *flags = (unsigned *)(cnt + E);  // [RT_TM][nfw] undecided logits
-  double *xnorm = (double *)(((uintptr_t)(flags + RT_TM * nfw) + 15) & ~(uintptr_t)15);
-  double *fix_s = xnorm + RT_TM;  // fp64 sums of the first RT_FIX_CAP flagged logits
+  unsigned *flags = (unsigned *)(smem_raw + SL.flags);  // [RT_TM][nfw] undecided logits
+  double *xnorm = (double *)(smem_raw + SL.xnorm);
+  double *fix_s = (double *)(smem_raw + SL.fix);  // fp64 sums of the first RT_FIX_CAP flagged
   __shared__ int s_nfix;
 
   for (int e = tid; e < E; e += RT_THREADS) cnt[e] = 0;
   for (int i = tid; i < RT_TM * nfw; i += RT_THREADS) flags[i] = 0u;
   if (tid == 0) s_nfix = 0;
+  if (blockIdx.x == 0 && tid == 0) *a.counter = 0u;
+  const int rvec = d * (int)sizeof(Tin) / 16;  // 16-byte vectors per row
+  for (int i = tid; i < RT_TM * rvec; i += RT_THREADS) {
+    const int r = i / rvec, v = i - r * rvec;
+    uint4 q = make_uint4(0u, 0u, 0u, 0u);
+    if (r < ntok) q = *(const uint4 *)(x + (size_t)(t0 + r) * d + v * (16 / (int)sizeof(Tin)));
+    *(uint4 *)(xs + r * ldx + v * (16 / (int)sizeof(Tin))) = q;
+  }
+  __syncthreads();
   for (int tt = warp; tt < RT_TM; tt += RT_THREADS / 32) {
     double s = 0.0;
-    if (tt < ntok) {
-      const Tin *row = x + (size_t)(t0 + tt) * d;
-      for (int i = lane; i < d; i += 32) {
-        const double v = (double)Elem<Tin>::to_f(row[i]);
-        s = fma(v, v, s);
-      }
+    for (int i = lane; i < d; i += 32) {
+      const double v = (double)Elem<Tin>::to_f(xs[tt * ldx + i]);
+      s = fma(v, v, s);
     }
     s = warp_sum_d(s);
     if (lane == 0) xnorm[tt] = sqrt(s);
   }
 
-  // ---- logits. Warp w sums the k-chunks w, w+8, ... of every (token, expert) of the round;
-  // the eight partial sums are then added in warp order. Both operands sit in shared memory
-  // as fp64: one 16-byte load of x serves 4 lanes and one of W serves 8, so a warp issues one
-  // wavefront per load and 2*RE fp64 FMAs per pair of loads.
-  const int nchunk = d / RT_KC;
+  // ---- logits on the fp64 tensor cores. Each round stages 8*NT router rows; warp w takes the
+  // 16-k blocks w, w+8, ... For a block, the lane at fragment (row r, column c) loads elements
+  // 4c..4c+3 of its token row and of its expert row, and MMA step i uses element 4c+i: a
+  // permutation of k inside the block, identical for both operands. The eight per-warp partial
+  // sums are then added in warp order.
+  const int nkb = d / RT_KB;
   for (int eb = 0; eb < E; eb += EB) {
-    double acc[2][RE];
-#pragma unroll
-    for (int j = 0; j < RE; ++j) acc[0][j] = acc[1][j] = 0.0;
-    for (int c = warp; c < nchunk; c += RT_THREADS / 32) {
-      const int k0 = c * RT_KC;
-      {  // x chunk: lane -> token lane/2, 16 consecutive k
-        const int tt = lane >> 1, h = (lane & 1) * 16;
-        double *dst = xs + tt * RT_LD + h;
-        if (tt < ntok) {
-          const Tin *src = x + (size_t)(t0 + tt) * d + k0 + h;
-#pragma unroll
-          for (int i = 0; i < 16; i += 2)
-            *(double2 *)(dst + i) = make_double2((double)Elem<Tin>::to_f(src[i]),
-                                                 (double)Elem<Tin>::to_f(src[i + 1]));
-        } else {
-#pragma unroll
-          for (int i = 0; i < 16; i += 2) *(double2 *)(dst + i) = make_double2(0.0, 0.0);
-        }
-      }
-      for (int i = lane; i < EB * (RT_KC / 2); i += 32) {  // W chunk from the fp64 copy
-        const int e = i / (RT_KC / 2), kp = (i % (RT_KC / 2)) * 2;
-        double2 wv = make_double2(0.0, 0.0);
-        if (eb + e < E) wv = *(const double2 *)(a.w64 + (size_t)(eb + e) * d + k0 + kp);
-        *(double2 *)(wsm + e * RT_LD + kp) = wv;
-      }
-      __syncwarp();
-#pragma unroll 4
-      for (int kk = 0; kk < RT_KC; kk += 2) {
-        const double2 x0 = *(const double2 *)(xs + lt * RT_LD + kk);
-        const double2 x1 = *(const double2 *)(xs + (lt + 8) * RT_LD + kk);
-#pragma unroll
-        for (int j = 0; j < RE; ++j) {
-          const double2 wv = *(const double2 *)(wsm + (le + 4 * j) * RT_LD + kk);
-          acc[0][j] = fma(x0.x, wv.x, acc[0][j]);
-          acc[0][j] = fma(x0.y, wv.y, acc[0][j]);
-          acc[1][j] = fma(x1.x, wv.x, acc[1][j]);
-          acc[1][j] = fma(x1.y, wv.y, acc[1][j]);
-        }
-      }
-      __syncwarp();
+    __syncthreads();  // the previous round is done with wsb and part
+    for (int i = tid; i < EB * rvec; i += RT_THREADS) {
+      const int r = i / rvec, v = i - r * rvec;
+      uint4 q = make_uint4(0u, 0u, 0u, 0u);
+      if (eb + r < E) q = *(const uint4 *)(wr + (size_t)(eb + r) * d + v * (16 / (int)sizeof(Tin)));
+      *(uint4 *)(wsb + r * ldx + v * (16 / (int)sizeof(Tin))) = q;
     }
-    __syncthreads();  // staging slots become the partial-sum buffer
-#pragma unroll
-    for (int j = 0; j < RE; ++j) {
-      part[(warp * RT_TM + lt) * EB + le + 4 * j] = acc[0][j];
-      part[(warp * RT_TM + lt + 8) * EB + le + 4 * j] = acc[1][j];
+    __syncthreads();
+    for (int r = warp; r < EB; r += RT_THREADS / 32) {  // |W_e|_2 of the round's rows
+      double s = 0.0;
+      for (int i = lane; i < d; i += 32) {
+        const double v = (double)Elem<Tin>::to_f(wsb[r * ldx + i]);
+        s = fma(v, v, s);
+      }
+      s = warp_sum_d(s);
+      if (lane == 0) wn[r] = sqrt(s);
     }
+    double acc[2][NT][2];
+#pragma unroll
+    for (int j = 0; j < NT; ++j) acc[0][j][0] = acc[0][j][1] = acc[1][j][0] = acc[1][j][1] = 0.0;
+    for (int kb = warp; kb < nkb; kb += RT_THREADS / 32) {
+      const int kk = kb * RT_KB + 4 * fc;
+      double a0[4], a1[4], bw[NT][4];
+      load4d(xs + fr * ldx + kk, a0);
+      load4d(xs + (8 + fr) * ldx + kk, a1);
+#pragma unroll
+      for (int j = 0; j < NT; ++j) load4d(wsb + (8 * j + fr) * ldx + kk, bw[j]);
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < NT; ++j) {
+          dmma_8x8x4(acc[0][j], a0[i], bw[j][i]);
+          dmma_8x8x4(acc[1][j], a1[i], bw[j][i]);
+        }
+    }
+#pragma unroll
+    for (int j = 0; j < NT; ++j)
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        part[(warp * RT_TM + fr) * EB + 8 * j + 2 * fc + h] = acc[0][j][h];
+        part[(warp * RT_TM + 8 + fr) * EB + 8 * j + 2 * fc + h] = acc[1][j][h];
+      }
     __syncthreads();
     for (int q = tid; q < RT_TM * EB; q += RT_THREADS) {
       const int tt = q / EB, e = eb + q % EB;
@@ -490,7 +513,7 @@ __global__ void __launch_bounds__(RT_THREADS, 2) router_kernel(RouterArgs a) {
         s += o;
         // any summation order over d products plus 8 partials and the offset:
         // |error| <= gamma_{d+16} (sum |x_i W_i| + |off|) <= (d+16) 2^-52 (|x|_2 |W_e|_2 + |off|)
-        const double B = (double)(d + 16) * 0x1p-52 * (xnorm[tt] * a.wnorm[e] + fabs(o));
+        const double B = (double)(d + 16) * 0x1p-52 * (xnorm[tt] * wn[q % EB] + fabs(o));
         float r, up, dn;
         double mh, ml;
         float l;
@@ -502,18 +525,16 @@ __global__ void __launch_bounds__(RT_THREADS, 2) router_kernel(RouterArgs a) {
           if (slot < RT_FIX_CAP) {
             fix_s[slot] = s;
             l = __int_as_float(slot);  // the slot index rides in the logit until resolved
-            atomicOr(&flags[tt * nfw + (e >> 5)], 1u << (e & 31));
           } else {
-            // overflow (forced test modes only): the fixup recomputes the fp64 sum
-            l = __int_as_float(-1);
-            atomicOr(&flags[tt * nfw + (e >> 5)], 1u << (e & 31));
+            l = __int_as_float(-1);    // overflow (forced test modes): the fixup recomputes
           }
+          atomicOr(&flags[tt * nfw + (e >> 5)], 1u << (e & 31));
         }
         lg[tt * E + e] = l;
       }
     }
-    __syncthreads();  // the partial-sum buffer is the next round's staging area
   }
+  __syncthreads();
 
   // ---- fixup of undecided logits: flag words dealt round-robin to the warps; one warp decides
   // one logit exactly (see resolve_logit)
@@ -524,15 +545,16 @@ __global__ void __launch_bounds__(RT_THREADS, 2) router_kernel(RouterArgs a) {
       const int ee = e0 + __ffs(m) - 1;
       m &= m - 1;
       const int slot = __float_as_int(lg[tt * E + ee]);
-      const Tin *xrow = x + (size_t)(t0 + tt) * d;
-      const double *wrow = a.w64 + (size_t)ee * d;
+      const Tin *xrow = xs + tt * ldx;  // the staged copy (16-byte aligned rows)
+      const Tin *wrow = wr + (size_t)ee * d;
       const double o = a.off ? (double)a.off[ee] : 0.0;
       double approx;
       if (slot >= 0 && slot < RT_FIX_CAP) {
         approx = fix_s[slot];
       } else {
         double s = 0.0;
-        for (int i = lane; i < d; i += 32) s = fma((double)Elem<Tin>::to_f(xrow[i]), wrow[i], s);
+        for (int i = lane; i < d; i += 32)
+          s = fma((double)Elem<Tin>::to_f(xrow[i]), (double)Elem<Tin>::to_f(wrow[i]), s);
         approx = warp_sum_d(s) + o;
       }
       const float l = resolve_logit<Tin>(xrow, wrow, d, o, approx, force_level);
@@ -543,7 +565,65 @@ __global__ void __launch_bounds__(RT_THREADS, 2) router_kernel(RouterArgs a) {
   }
   __syncthreads();
 
-  // ---- selection, one warp per token
+  // ---- selection
+  if (rank_sel) {
+    // up to 64 experts: every (token, expert) pair finds its own rank among the token's keys
+    if (sigmoid)
+      for (int q = tid; q < ntok * E; q += RT_THREADS)
+        keys[q] = sigmoid_key(lg[q], a.bias ? a.bias[q % E] : 0.0f, force);
+    __syncthreads();
+    for (int q = tid; q < ntok * E; q += RT_THREADS) {
+      const int tt = q / E, e = q - tt * E;
+      const float *krow = (sigmoid ? keys : lg) + tt * E;
+      const float *lrow = lg + tt * E;
+      float v = krow[e];
+      if (v != v) v = -INFINITY;
+      int rank = 0;
+      float m = -INFINITY;
+      for (int e2 = 0; e2 < E; ++e2) {
+        float v2 = krow[e2];
+        if (v2 != v2) v2 = -INFINITY;
+        rank += (v2 > v || (v2 == v && e2 < e)) ? 1 : 0;
+        m = fmaxf(m, lrow[e2]);
+      }
+      // the token's normaliser, summed in expert order by each of its threads alike
+      float ssum = 0.0f;
+      if (!sigmoid)
+        for (int e2 = 0; e2 < E; ++e2) ssum += expf(lrow[e2] - m);
+      else
+        for (int e2 = 0; e2 < E; ++e2) ssum += 1.0f / (1.0f + expf(-lrow[e2]));
+      const float inv = 1.0f / ssum;
+      const float l = lrow[e];
+      float p, pbasis;
+      if (!sigmoid) {
+        p = expf(l - m) * inv;
+        pbasis = p;
+      } else {
+        p = 1.0f / (1.0f + expf(-l));
+        pbasis = p * inv;
+      }
+      pb[q] = pbasis;
+      if (rank < k) {
+        sel_e[tt * 8 + rank] = e;
+        sel_p[tt * 8 + rank] = p;
+      }
+    }
+    __syncthreads();
+    if (tid < ntok) {
+      const int t = t0 + tid;
+      float psel = 0.0f;
+      for (int j = 0; j < k; ++j) psel += sel_p[tid * 8 + j];
+      for (int j = 0; j < k; ++j) {
+        const int e = sel_e[tid * 8 + j];
+        const float pj = sel_p[tid * 8 + j];
+        a.idx[(size_t)t * k + j] = e;
+        a.wts[(size_t)t * k + j] = a.norm ? pj / psel : pj;
+        atomicAdd(&cnt[e], 1);
+      }
+    }
+    __syncthreads();
+  } else {
+    // one warp per token
   for (int tt = warp; tt < ntok; tt += RT_THREADS / 32) {
     const int t = t0 + tt;
     float *lrow = lg + tt * E;
@@ -620,46 +700,14 @@ __global__ void __launch_bounds__(RT_THREADS, 2) router_kernel(RouterArgs a) {
     __syncwarp();
   }
   __syncthreads();
+  }
 
   // ---- per-CTA statistics (fixed token order), then the last CTA reduces in CTA order
   for (int e = tid; e < E; e += RT_THREADS) {
     float ps = 0.0f;
-    for (int tt = 0; tt < ntok; ++tt) ps += lg[tt * E + e];
+    for (int tt = 0; tt < ntok; ++tt) ps += pb[tt * E + e];
     a.part_cnt[(size_t)blockIdx.x * E + e] = cnt[e];
     a.part_prob[(size_t)blockIdx.x * E + e] = ps;
-  }
-}
-
-// Per-expert totals of the per-CTA selection counts and probability sums: one block per
-// expert; thread t adds the CTAs t, t+128, ... in order, then a fixed-shape tree combines the
-// 128 partial sums, so prob_sum is bitwise reproducible.
-__global__ void __launch_bounds__(128) router_reduce_kernel(const int32_t *__restrict__ part_cnt,
-                                                            const float *__restrict__ part_prob,
-                                                            int nblk, int E,
-                                                            int32_t *__restrict__ count_out,
-                                                            float *__restrict__ prob_out) {
-  const int e = blockIdx.x, tid = threadIdx.x;
-  int c = 0;
-  float p = 0.0f;
-  for (int b = tid; b < nblk; b += 128) {
-    c += part_cnt[(size_t)b * E + e];
-    p += part_prob[(size_t)b * E + e];
-  }
-  __shared__ int sc[4];
-  __shared__ float sp[4];
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    c += __shfl_xor_sync(0xffffffffu, c, o);
-    p += __shfl_xor_sync(0xffffffffu, p, o);
-  }
-  if ((tid & 31) == 0) {
-    sc[tid >> 5] = c;
-    sp[tid >> 5] = p;
-  }
-  __syncthreads();
-  if (tid == 0) {
-    count_out[e] = (sc[0] + sc[1]) + (sc[2] + sc[3]);
-    prob_out[e] = (sp[0] + sp[1]) + (sp[2] + sp[3]);
   }
 }
 

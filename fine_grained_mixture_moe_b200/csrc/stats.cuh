@@ -1,0 +1,121 @@
+// Per-expert statistics over token chunks, in one launch:
+//   count[e]          = sum over chunks of the chunk's selections of e (before capacity)
+//   prob_sum[e]       = sum over chunks of the chunk's probability mass on e, fixed order
+//   chunk_base[c][e]  = exclusive scan over chunks of the selections of e (token order)
+//   offsets[0..E]     = exclusive scan over experts of kept_e = min(count_e, C) (dropless: count_e)
+//   aux               = alpha * E * sum_e (count_e / (T k)) * (prob_sum_e / T)
+// One block per expert does the first three; the block that finishes last does the scan over
+// experts and the loss (Moonfrost expert card: capacity-based routing over stacked experts;
+// Quartz: 0.01-weighted load-balancing loss). Chunks are RT_TM = 16 tokens, the router's CTA,
+// so the router's per-CTA counts are the permutation's histogram. Every sum has a fixed order.
+#pragma once
+#include "common.cuh"
+
+namespace moe {
+
+constexpr int ST_THREADS = 256;
+
+struct StatsArgs {
+  const int32_t *chunk_cnt;  // [nchunk][E]
+  const float *chunk_prob;   // [nchunk][E] or null
+  int nchunk, E, T, k, C;    // C < 0: dropless
+  int32_t *count_out;        // [E] or null
+  float *prob_out;           // [E] or null (needs chunk_prob)
+  int32_t *chunk_base;       // [nchunk][E] or null
+  int32_t *kept;             // [E] scratch, needed with offsets
+  int32_t *offsets;          // [E+1] or null
+  float *aux;                // scalar or null (needs chunk_prob)
+  float alpha;
+  unsigned *counter;         // cleared before the launch; reset to 0 by the last block
+};
+
+__global__ void __launch_bounds__(ST_THREADS) moe_stats_kernel(StatsArgs a) {
+  const int e = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int E = a.E;
+  __shared__ int s_wc[ST_THREADS / 32 + 1];
+  __shared__ float s_wp[ST_THREADS / 32];
+  __shared__ int s_run;
+  // totals: thread t adds chunks t, t+256, ... then a fixed tree
+  int c = 0;
+  float p = 0.0f;
+  for (int b = tid; b < a.nchunk; b += ST_THREADS) {
+    c += a.chunk_cnt[(size_t)b * E + e];
+    if (a.chunk_prob) p += a.chunk_prob[(size_t)b * E + e];
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    c += __shfl_xor_sync(0xffffffffu, c, o);
+    p += __shfl_xor_sync(0xffffffffu, p, o);
+  }
+  if (lane == 0) { s_wc[warp] = c; s_wp[warp] = p; }
+  __syncthreads();
+  int total = 0;
+  float psum = 0.0f;
+#pragma unroll
+  for (int w = 0; w < ST_THREADS / 32; ++w) { total += s_wc[w]; psum += s_wp[w]; }
+  if (tid == 0) {
+    if (a.count_out) a.count_out[e] = total;
+    if (a.prob_out) a.prob_out[e] = psum;
+    if (a.kept) a.kept[e] = a.C < 0 ? total : min(total, a.C);
+  }
+  // exclusive scan over chunks, 256 chunks per pass
+  if (a.chunk_base) {
+    if (tid == 0) s_run = 0;
+    __syncthreads();
+    for (int b0 = 0; b0 < a.nchunk; b0 += ST_THREADS) {
+      const int b = b0 + tid;
+      const int v = b < a.nchunk ? a.chunk_cnt[(size_t)b * E + e] : 0;
+      const int incl = warp_incl_scan(v);
+      __syncthreads();
+      if (lane == 31) s_wc[warp] = incl;
+      __syncthreads();
+      if (warp == 0) {
+        const int wv = lane < ST_THREADS / 32 ? s_wc[lane] : 0;
+        const int wi = warp_incl_scan(wv);
+        if (lane < ST_THREADS / 32) s_wc[lane] = wi - wv;
+        if (lane == ST_THREADS / 32 - 1) s_wc[ST_THREADS / 32] = wi;
+      }
+      __syncthreads();
+      if (b < a.nchunk) a.chunk_base[(size_t)b * E + e] = s_run + s_wc[warp] + incl - v;
+      __syncthreads();
+      if (tid == 0) s_run += s_wc[ST_THREADS / 32];
+      __syncthreads();
+    }
+  }
+  if (!a.offsets && !a.aux) return;
+  // the last block to finish scans the kept counts over experts and forms the loss
+  __threadfence();
+  __syncthreads();
+  __shared__ int s_last;
+  if (tid == 0) s_last = (atomicAdd(a.counter, 1u) == gridDim.x - 1);
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  if (a.offsets) {
+    __shared__ int s_scan[1024 + ST_THREADS / 32 + 1];
+    for (int i = tid; i < E; i += ST_THREADS) s_scan[i] = __ldcg(a.kept + i);
+    __syncthreads();
+    const int tot = block_excl_scan_inplace(s_scan, E, s_scan + 1024);
+    for (int i = tid; i < E; i += ST_THREADS) a.offsets[i] = s_scan[i];
+    if (tid == 0) a.offsets[E] = tot;
+  }
+  if (a.aux) {
+    double s = 0.0;
+    for (int i = tid; i < E; i += ST_THREADS)
+      s += (double)__ldcg(a.count_out + i) * (double)__ldcg(a.prob_out + i);
+    s = warp_sum_d(s);
+    __shared__ double s_d[ST_THREADS / 32];
+    if (lane == 0) s_d[warp] = s;
+    __syncthreads();
+    if (tid == 0) {
+      double t = 0.0;
+      for (int w = 0; w < ST_THREADS / 32; ++w) t += s_d[w];
+      double L = 0.0;
+      if (a.T > 0) L = (double)a.alpha * (double)E * t / ((double)a.T * (double)a.k * (double)a.T);
+      *a.aux = (float)L;
+    }
+  }
+  if (tid == 0) *a.counter = 0u;
+}
+
+}  // namespace moe
