@@ -51,6 +51,33 @@ def load_peaks():
         return dict(PEAKS_FALLBACK), "fallback"
 
 
+def kernel_sources_sha256() -> str:
+    import glob
+    import hashlib
+    h = hashlib.sha256()
+    for f in sorted(glob.glob(os.path.join(ROOT, "fine_grained_mixture_moe_b200", "csrc", "*"))):
+        with open(f, "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def captured_traffic(config_name: str, kernel: str):
+    """DRAM bytes per launch from a committed ncu capture, or None when the kernels changed."""
+    path = os.path.join(ROOT, "profiles", f"traffic_{config_name}.txt")
+    try:
+        vals = {}
+        with open(path) as fh:
+            for line in fh:
+                if line.strip() and not line.startswith("#"):
+                    k, v = line.split()
+                    vals[k] = v
+    except (OSError, ValueError):
+        return None
+    if vals.get("sources_sha256") != kernel_sources_sha256():
+        return None
+    return int(vals[kernel]) if kernel in vals else None
+
+
 def workload_name(c) -> str:
     parts = [f"{c.name}: T={c.T} d={c.d} E={c.E} top-{c.top_k} {c.score}"]
     if c.expert == "swiglu":
@@ -373,7 +400,8 @@ def run_ours(args, rank, world, local_rank):
         },
         "roofline": {"kernel": dom, "bound": dr.get("bound"), "achieved": dr.get("achieved"),
                      "peak": dr.get("peak"), "unit": dr.get("unit"), "frac": dr.get("frac"),
-                     "traffic": None,
+                     "traffic": captured_traffic(c.name, dom),
+                     "traffic_source": "profiles/gemm_tc_quartz.md (ncu dram bytes read+write, one launch)",
                      "peak_kind": f"{peak_src} burst" if dr.get("bound") == "tensor" else peak_src},
         "e2e": {"value": tokens / (e2e_ms * 1e-3), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
