@@ -68,23 +68,38 @@ __global__ void __launch_bounds__(256) combine_kernel(const float *__restrict__ 
     pos[j] = __shfl_sync(0xffffffffu, pos_l, j);
     wj[j] = __shfl_sync(0xffffffffu, w_l, j);
   }
-  for (int c = lane * V; c < d; c += 32 * V) {
-    float acc[V];
-    if (y_shared) Vec16<Tio>::load(y_shared + (size_t)t * d + c, acc);
-    else {
+  // two vectors per lane per pass, all loads of a pass issued before the sums
+#pragma unroll 1
+  for (int c0 = lane * V; c0 < d; c0 += 64 * V) {
+    float acc[2][V];
+    float v[2][8][V];
 #pragma unroll
-      for (int i = 0; i < V; ++i) acc[i] = 0.0f;
-    }
+    for (int h = 0; h < 2; ++h) {
+      const int c = c0 + h * 32 * V;
+      if (c < d) {
+        if (y_shared) Vec16<Tio>::load(y_shared + (size_t)t * d + c, acc[h]);
+        else {
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      if (j < k && pos[j] >= 0) {
-        float v[V];
-        Vec16<Tio>::load(y_perm + (size_t)pos[j] * d + c, v);
+          for (int i = 0; i < V; ++i) acc[h][i] = 0.0f;
+        }
 #pragma unroll
-        for (int i = 0; i < V; ++i) acc[i] = fmaf(wj[j], v[i], acc[i]);
+        for (int j = 0; j < 8; ++j)
+          if (j < k && pos[j] >= 0) Vec16<Tio>::load(y_perm + (size_t)pos[j] * d + c, v[h][j]);
       }
     }
-    Vec16<Tio>::store(y + (size_t)t * d + c, acc);
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int c = c0 + h * 32 * V;
+      if (c < d) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          if (j < k && pos[j] >= 0) {
+#pragma unroll
+            for (int i = 0; i < V; ++i) acc[h][i] = fmaf(wj[j], v[h][j][i], acc[h][i]);
+          }
+        __stcs((float4 *)(y + (size_t)t * d + c), make_float4(acc[h][0], acc[h][1], acc[h][2], acc[h][3]));
+      }
+    }
   }
 }
 

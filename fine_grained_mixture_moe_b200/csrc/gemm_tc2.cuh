@@ -1,0 +1,331 @@
+// bf16 grouped expert GEMM on CTA pairs (tcgen05 .cta_group::2, sm_100a).
+//
+// Same grouped problem, tile list and epilogues as gemm_tc.cuh, but each tile is 256 rows and is
+// computed by a cluster of two CTAs on two SMs: CTA r loads rows [128r, 128r+128) of the A tile
+// and half of the B tile (GATEUP: CTA 0 the gate rows, CTA 1 the up rows of the same 128 output
+// columns; PLAIN: rows [128r, 128r+128) of a 256-column weight tile) into its own shared memory.
+// The leader (CTA 0) issues one M=256, N=256, K=16 MMA per step that reads both CTAs' tiles
+// and leaves rows [128r, 128r+128) of the fp32 accumulator in CTA r's TMEM. So each SM ingests
+// 32 KB per 64-wide k-block instead of 48 KB for the same tensor work.
+// Synchronisation: both CTAs' TMA loads complete on the leader's `full` barrier (the leader
+// expects both CTAs' bytes); the leader's commits multicast to both CTAs' `empty` and
+// `acc_full` barriers; all sixteen epilogue warps arrive on the leader's `acc_empty`. No TMA
+// multicast is used. All waits are bounded as in gemm_tc.cuh.
+#pragma once
+#include "gemm_tc.cuh"
+
+namespace moe {
+
+constexpr int TC2_BM = 256;  // rows per tile (128 per CTA)
+
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.aligned;\n\tbarrier.cluster.wait.aligned;" ::: "memory");
+}
+// TMA load into this CTA's shared memory whose completion is counted on the leader CTA's barrier
+// (same shared-memory offset in CTA 0: the CTA-rank bit of the cluster address cleared).
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap *map, int c0,
+                                                 int c1, uint32_t bar_local) {
+  const uint32_t bar0 = bar_local & 0xFEFFFFFFu;
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"((uint64_t)map), "r"(c0), "r"(c1), "r"(bar0)
+      : "memory");
+}
+__device__ __forceinline__ void tc2_mma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                        uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// Arrive once on the barrier at this shared offset in both CTAs of the pair when all prior
+// tcgen05 operations of the issuing thread complete.
+__device__ __forceinline__ void tc2_commit_both(uint32_t bar) {
+  const uint16_t mask = 0x3;
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+      " [%0], %1;" ::"r"(bar),
+      "h"(mask)
+      : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_cta0(uint32_t bar_local) {
+  asm volatile(
+      "{\n\t.reg .b32 ra;\n\t"
+      "mapa.shared::cluster.u32 ra, %0, 0;\n\t"
+      "mbarrier.arrive.release.cluster.shared::cluster.b64 _, [ra];\n\t}" ::"r"(bar_local)
+      : "memory");
+}
+
+template <int MODE> struct Tc2Cfg {
+  static_assert(MODE == MODE_GATEUP || MODE == MODE_PLAIN, "pair kernel modes");
+  static constexpr int BN = MODE == MODE_GATEUP ? 128 : 256;  // output columns per tile
+  static constexpr int MMA_N = 256;                           // accumulator columns
+  static constexpr int A_BYTES = 128 * TC_BK * 2;             // this CTA's 128 rows
+  static constexpr int B_BYTES = 128 * TC_BK * 2;             // this CTA's half of B
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;       // 32 KB
+  static constexpr int STG_BYTES = MODE == MODE_PLAIN ? TC_EPI_WARPS * 4096 : 0;
+  static constexpr int STAGES = (200 * 1024 - STG_BYTES) / STAGE_BYTES > 8
+                                    ? 8 : (200 * 1024 - STG_BYTES) / STAGE_BYTES;
+  static constexpr int ACC_COLS = MMA_N;
+  static constexpr int TMEM_COLS = 512;
+  static constexpr uint32_t IDESC = (1u << 4) | (1u << 7) | (1u << 10) |
+                                    ((uint32_t)(MMA_N >> 3) << 17) |
+                                    ((uint32_t)(TC2_BM >> 4) << 24);
+};
+
+template <int MODE>
+__host__ __device__ constexpr size_t tc2_smem_bytes(int G) {
+  using C = Tc2Cfg<MODE>;
+  return 1024 + (size_t)C::STAGES * C::STAGE_BYTES + C::STG_BYTES + 256 +
+         (size_t)(G + 1 + TC_THREADS / 32 + 1) * sizeof(int);
+}
+
+template <int MODE>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TC_THREADS, 1)
+    gemm_tc2_kernel(const __grid_constant__ TcParams P) {
+  using C = Tc2Cfg<MODE>;
+  constexpr int BN = C::BN;
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  const GroupedGemm &p = P.p;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int G = p.E + p.has_shared;
+  const uint32_t rank = cluster_ctarank();
+  const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t pad = ((raw + 1023u) & ~1023u) - raw;
+  unsigned char *base = smem_raw + pad;
+  unsigned char *stages = base;
+  unsigned char *stg_all = base + (size_t)C::STAGES * C::STAGE_BYTES;
+  uint64_t *bars = (uint64_t *)(stg_all + C::STG_BYTES);
+  uint32_t *tmem_slot = (uint32_t *)(bars + 2 * C::STAGES + 5);
+  volatile int *abort_flag = (volatile int *)(tmem_slot + 1);
+  int *prefix = (int *)(stg_all + C::STG_BYTES + 256);
+  int *scan_tmp = prefix + G + 1;
+
+  auto full_bar = [&](int s) { return smem_u32(bars + s); };
+  auto empty_bar = [&](int s) { return smem_u32(bars + C::STAGES + s); };
+  auto accf_bar = [&](int b) { return smem_u32(bars + 2 * C::STAGES + b); };
+  auto acce_bar = [&](int b) { return smem_u32(bars + 2 * C::STAGES + 2 + b); };
+  const uint32_t drain_bar = smem_u32(bars + 2 * C::STAGES + 4);
+
+  if (tid == 0) {
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(accf_bar(b), 1);
+      mbar_init(acce_bar(b), 2 * TC_EPI_WARPS);
+    }
+    mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(tmem_slot)),
+                 "r"((uint32_t)C::TMEM_COLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+  }
+  const int total = build_tile_prefix(p, TC2_BM, BN, prefix, scan_tmp);
+  tc_fence_before();
+  cluster_sync_all();  // barriers of both CTAs initialised, TMEM allocated in both
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const uint64_t limit = g_wait_limit_ns;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer (both CTAs)
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      int issued_parity[8];
+      bool issued[8];
+      for (int s = 0; s < 8; ++s) { issued[s] = false; issued_parity[s] = 0; }
+      for (int tile = pair; tile < total && ok; tile += npairs) {
+        const TileInfo ti = decode_tile(p, tile, prefix, TC2_BM, BN);
+        const bool routed = ti.g < p.E;
+        const CUtensorMap *ma = routed ? &P.maps.a_r : &P.maps.a_s;
+        const CUtensorMap *mb = (MODE == MODE_GATEUP && rank == 1)
+                                    ? (routed ? &P.maps.b1_r : &P.maps.b1_s)
+                                    : (routed ? &P.maps.b0_r : &P.maps.b0_s);
+        const int a_row = ti.a_row0 + ti.m0 + (int)rank * 128;
+        const int n_off = MODE == MODE_GATEUP ? 0 : (int)rank * 128;
+        const int nk = ti.K / TC_BK;
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, limit, INFO_WAIT_MMA_EMPTY)) {
+            ok = false;
+            break;
+          }
+          const uint32_t sA = smem_u32(stages + (size_t)stage * C::STAGE_BYTES);
+          const uint32_t sB = sA + C::A_BYTES;
+          if (rank == 0) mbar_expect_tx(full_bar(stage), 2 * C::STAGE_BYTES);
+          const int kk = kb * TC_BK;
+          int b_row, b_col;
+          if (routed) {
+            b_row = ti.g * ti.N + ti.n0 + n_off;
+            b_col = kk;
+          } else {
+            const int piece = kk / p.piece_k;
+            b_row = piece * p.piece_rows + ti.n0 + n_off;
+            b_col = kk - piece * p.piece_k;
+          }
+          tma_load_2d_pair(sA, ma, kk, a_row, full_bar(stage));
+          tma_load_2d_pair(sB, mb, b_col, b_row, full_bar(stage));
+          issued[stage] = true;
+          issued_parity[stage] = (int)phase;
+          if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
+        }
+      }
+      if (!ok && rank == 0) {
+        for (int s = 0; s < C::STAGES; ++s)
+          if (issued[s]) {
+            volatile int never = 0;
+            mbar_wait(full_bar(s), (uint32_t)issued_parity[s], &never, limit, INFO_WAIT_DRAIN);
+          }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer (leader only)
+    if (rank == 0 && lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true, any = false;
+      for (int tile = pair; tile < total && ok; tile += npairs) {
+        const TileInfo ti = decode_tile(p, tile, prefix, TC2_BM, BN);
+        const int nk = ti.K / TC_BK;
+        if (!mbar_wait(acce_bar(acc), acc_phase ^ 1u, abort_flag, limit, INFO_WAIT_ACC_EMPTY)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d0 = tmem_base + (uint32_t)(acc * C::ACC_COLS);
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!mbar_wait(full_bar(stage), phase, abort_flag, limit, INFO_WAIT_TMA_FULL)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sA = smem_u32(stages + (size_t)stage * C::STAGE_BYTES);
+          const uint32_t sB = sA + C::A_BYTES;
+#pragma unroll
+          for (int k16 = 0; k16 < TC_BK / 16; ++k16) {
+            const uint32_t accum = (kb > 0 || k16 > 0) ? 1u : 0u;
+            tc2_mma(d0, make_sdesc(sA + k16 * 32), make_sdesc(sB + k16 * 32), C::IDESC, accum);
+          }
+          any = true;
+          tc2_commit_both(empty_bar(stage));
+          if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        tc2_commit_both(accf_bar(acc));
+        if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+      }
+      if (!ok && any) {
+        tc2_commit_both(drain_bar);
+        volatile int never = 0;
+        mbar_wait(drain_bar, 0u, &never, limit, INFO_WAIT_DRAIN);
+      }
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue (warps 2..9)
+    const int q = warp & 3;
+    const int half = (warp - 2) >> 2;
+    const int cbeg = half * (BN / 2), cend = cbeg + BN / 2;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int tile = pair; tile < total; tile += npairs) {
+      const TileInfo ti = decode_tile(p, tile, prefix, TC2_BM, BN);
+      const bool routed = ti.g < p.E;
+      bool ok = true;
+      if (lane == 0)
+        ok = mbar_wait(accf_bar(acc), acc_phase, abort_flag, limit, INFO_WAIT_ACC_FULL);
+      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+      if (!ok) break;
+      tc_fence_after();
+      const int rbase = ti.m0 + (int)rank * 128 + q * 32;  // first row of this warp's block
+      const int row = rbase + lane;
+      const bool row_ok = row < ti.rows;
+      void *out = routed ? p.out_r : p.out_s;
+      const int ldo = routed ? p.ldo_r : p.ldo_s;
+      const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * C::ACC_COLS);
+      unsigned char *stg = stg_all + (warp - 2) * 4096;
+#pragma unroll 1
+      for (int c = cbeg; c < cend; c += 32) {
+        if (MODE == MODE_GATEUP) {
+          uint32_t r0[32], r1[32];
+          tmem_ld32(tbase + c, r0);
+          tmem_ld32(tbase + BN + c, r1);
+          tmem_wait_ld();
+          const int col = ti.n0 + c;
+          if (row_ok && col < ti.N) {
+            uint4 pk[4];
+            __nv_bfloat162 *h = (__nv_bfloat162 *)pk;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const float g0 = __uint_as_float(r0[2 * i]), g1 = __uint_as_float(r0[2 * i + 1]);
+              h[i] = __floats2bfloat162_rn(__fdividef(g0, 1.0f + __expf(-g0)) * __uint_as_float(r1[2 * i]),
+                                           __fdividef(g1, 1.0f + __expf(-g1)) * __uint_as_float(r1[2 * i + 1]));
+            }
+            uint4 *dst = (uint4 *)((__nv_bfloat16 *)out + (size_t)(ti.a_row0 + row) * ldo + col);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) dst[i] = pk[i];
+          }
+        } else {
+          uint32_t r0[32];
+          tmem_ld32(tbase + c, r0);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            *(uint4 *)(stg + lane * 128 + ((i ^ (lane & 7)) << 4)) =
+                make_uint4(r0[4 * i], r0[4 * i + 1], r0[4 * i + 2], r0[4 * i + 3]);
+          __syncwarp();
+          const int col = ti.n0 + c;
+          if (col < ti.N) {
+            const int nrows = min(32, ti.rows - rbase);
+            unsigned char *obase = (unsigned char *)out + ((size_t)(ti.a_row0 + rbase) * ldo + col) * 4;
+            const size_t row_bytes = (size_t)ldo * 4;
+            for (int rr = 0; rr < nrows; ++rr) {
+              const uint32_t v = *(const uint32_t *)(stg + rr * 128 +
+                                                     (((lane >> 2) ^ (rr & 7)) << 4) + ((lane & 3) << 2));
+              *(uint32_t *)(obase + rr * row_bytes + lane * 4) = v;
+            }
+          }
+          __syncwarp();
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cta0(acce_bar(acc));
+      if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();  // no CTA leaves while its peer may still read its smem or TMEM
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                 "r"((uint32_t)C::TMEM_COLS)
+                 : "memory");
+  }
+}
+
+}  // namespace moe

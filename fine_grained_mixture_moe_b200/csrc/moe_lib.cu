@@ -15,6 +15,7 @@
 #include "common.cuh"
 #include "gemm_simt.cuh"
 #include "gemm_tc.cuh"
+#include "gemm_tc2.cuh"
 #include "permute.cuh"
 #include "router.cuh"
 #include "stats.cuh"
@@ -222,29 +223,31 @@ long long tile_bound(const GroupedGemm &g, int BM, int BN) {
   return t;
 }
 
+// Tensor maps of one grouped launch: A boxes of 128 rows, B boxes of `b_box` rows.
+// routed operands: A [rows_r, K_r], B [E*N_r, K_r]; shared: A [T, K_s], B [b_rows_s, piece_k]
+bool build_maps(const GroupedGemm &g, bool two_b, uint32_t b_box, TcMaps *m) {
+  const void *any = g.E > 0 ? g.A_r : g.A_s;
+  bool ok = true;
+  ok &= make_map(&m->a_r, g.E > 0 ? g.A_r : any, g.E > 0 ? g.rows_r : 1, g.E > 0 ? g.K_r : 64, 128);
+  ok &= make_map(&m->b0_r, g.E > 0 ? g.B0_r : any, g.E > 0 ? (uint64_t)g.E * g.N_r : 1,
+                 g.E > 0 ? g.K_r : 64, b_box);
+  ok &= make_map(&m->b1_r, (g.E > 0 && two_b) ? g.B1_r : any,
+                 (g.E > 0 && two_b) ? (uint64_t)g.E * g.N_r : 1, g.E > 0 ? g.K_r : 64, b_box);
+  ok &= make_map(&m->a_s, g.has_shared ? g.A_s : any, g.has_shared ? g.T : 1,
+                 g.has_shared ? g.K_s : 64, 128);
+  ok &= make_map(&m->b0_s, g.has_shared ? g.B0_s : any, g.has_shared ? g.b_rows_s : 1,
+                 g.has_shared ? g.piece_k : 64, b_box);
+  ok &= make_map(&m->b1_s, (g.has_shared && two_b) ? g.B1_s : any,
+                 (g.has_shared && two_b) ? g.b_rows_s : 1, g.has_shared ? g.piece_k : 64, b_box);
+  return ok;
+}
+
 template <int MODE, int BN>
 moe_status_t launch_tc(const GroupedGemm &g, cudaStream_t st, int kind) {
   TcParams P;
   std::memset(&P, 0, sizeof(P));
   P.p = g;
-  const void *any = g.E > 0 ? g.A_r : g.A_s;
-  bool ok = true;
-  // routed operands: A [rows_r, K_r], B [E*N_r, K_r]; shared: A [T, K_s], B [b_rows_s, piece_k]
-  ok &= make_map(&P.maps.a_r, g.E > 0 ? g.A_r : any, g.E > 0 ? g.rows_r : 1,
-                 g.E > 0 ? g.K_r : 64, TC_BM);
-  ok &= make_map(&P.maps.b0_r, g.E > 0 ? g.B0_r : any, g.E > 0 ? (uint64_t)g.E * g.N_r : 1,
-                 g.E > 0 ? g.K_r : 64, BN);
-  ok &= make_map(&P.maps.b1_r, (g.E > 0 && MODE == MODE_GATEUP) ? g.B1_r : any,
-                 (g.E > 0 && MODE == MODE_GATEUP) ? (uint64_t)g.E * g.N_r : 1,
-                 g.E > 0 ? g.K_r : 64, BN);
-  ok &= make_map(&P.maps.a_s, g.has_shared ? g.A_s : any, g.has_shared ? g.T : 1,
-                 g.has_shared ? g.K_s : 64, TC_BM);
-  ok &= make_map(&P.maps.b0_s, g.has_shared ? g.B0_s : any, g.has_shared ? g.b_rows_s : 1,
-                 g.has_shared ? g.piece_k : 64, BN);
-  ok &= make_map(&P.maps.b1_s, (g.has_shared && MODE == MODE_GATEUP) ? g.B1_s : any,
-                 (g.has_shared && MODE == MODE_GATEUP) ? g.b_rows_s : 1,
-                 g.has_shared ? g.piece_k : 64, BN);
-  if (!ok) return MOE_ERR_CUDA;
+  if (!build_maps(g, MODE == MODE_GATEUP, BN, &P.maps)) return MOE_ERR_CUDA;
   const int G = g.E + g.has_shared;
   const size_t smem = tc_smem_bytes<MODE, BN>(G);
   auto kern = gemm_tc_kernel<MODE, BN>;
@@ -255,6 +258,27 @@ moe_status_t launch_tc(const GroupedGemm &g, cudaStream_t st, int kind) {
   const int grid = (int)std::min<long long>(num_sms(), bound);
   ProfScope ps(kind, st);
   kern<<<grid, TC_THREADS, smem, st>>>(P);
+  return last_launch_status();
+}
+
+// CTA-pair form (two SMs per 256-row tile); each CTA loads 128-row halves of A and B.
+template <int MODE>
+moe_status_t launch_tc2(const GroupedGemm &g, cudaStream_t st, int kind) {
+  using C = Tc2Cfg<MODE>;
+  TcParams P;
+  std::memset(&P, 0, sizeof(P));
+  P.p = g;
+  if (!build_maps(g, MODE == MODE_GATEUP, 128, &P.maps)) return MOE_ERR_CUDA;
+  const int G = g.E + g.has_shared;
+  const size_t smem = tc2_smem_bytes<MODE>(G);
+  auto kern = gemm_tc2_kernel<MODE>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  const long long bound = tile_bound(g, TC2_BM, C::BN);
+  if (bound == 0) return MOE_OK;
+  const int pairs = (int)std::min<long long>(num_sms() / 2, bound);
+  ProfScope ps(kind, st);
+  kern<<<2 * pairs, TC_THREADS, smem, st>>>(P);
   return last_launch_status();
 }
 
@@ -278,9 +302,9 @@ template <int MODE>
 moe_status_t launch_gemm(const moe_config_t *c, const GroupedGemm &g, int bn_hint,
                          cudaStream_t st, int kind) {
   if (c->dtype == MOE_DTYPE_F32) return launch_simt<MODE>(g, st, kind);
-  if (MODE == MODE_GATEUP) return launch_tc<MODE_GATEUP, 128>(g, st, kind);
+  if (MODE == MODE_GATEUP) return launch_tc2<MODE_GATEUP>(g, st, kind);
   if (MODE == MODE_SCALE) return launch_tc<MODE_SCALE, 64>(g, st, kind);
-  if (bn_hint == 256) return launch_tc<MODE_PLAIN, 256>(g, st, kind);
+  if (bn_hint == 256) return launch_tc2<MODE_PLAIN>(g, st, kind);
   return launch_tc<MODE_PLAIN, 128>(g, st, kind);
 }
 
@@ -375,7 +399,7 @@ moe_status_t scatter_impl(const moe_config_t *c, const void *x, const int32_t *i
                           const int32_t *chunk_base, const int32_t *offsets, int32_t *slot_pos,
                           int32_t *src, void *x_perm, cudaStream_t st) {
   ProfScope ps(K_PERM_SCATTER, st);
-  perm_scatter_kernel<Tin><<<ceil_div(c->T, PM_CHUNK), 256, (size_t)c->E * 4, st>>>(
+  perm_scatter_kernel<Tin><<<ceil_div(c->T, PM_CHUNK) * PM_SPLIT, 256, (size_t)c->E * 4, st>>>(
       idx, c->T, c->top_k, c->E, capacity_of(c), chunk_base, offsets, slot_pos, src,
       (const Tin *)x, (Tin *)x_perm, c->d);
   return last_launch_status();

@@ -17,6 +17,7 @@
 namespace moe {
 
 constexpr int PM_CHUNK = 16;
+constexpr int PM_SPLIT = 4;  // CTAs per chunk in the scatter
 
 __global__ void __launch_bounds__(256) perm_hist_kernel(const int32_t *__restrict__ idx, int T,
                                                         int k, int E,
@@ -53,7 +54,7 @@ __global__ void __launch_bounds__(256) perm_scatter_kernel(
   __shared__ int s_tok[PM_CHUNK * 8];
   const bool active = (threadIdx.x & 31) < PM_CHUNK;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int chunk = blockIdx.x;
+  const int chunk = blockIdx.x / PM_SPLIT, part = blockIdx.x % PM_SPLIT;
   const int t = chunk * PM_CHUNK + lane;
   if (warp == 0) {
     for (int e = lane; e < E; e += 32) smask[e] = 0u;
@@ -81,8 +82,10 @@ __global__ void __launch_bounds__(256) perm_scatter_kernel(
         if (e >= 0) {
           const int rank = chunk_base[(size_t)chunk * E + e] + __popc(smask[e] & lt);
           if (C < 0 || rank < C) pos = offsets[e] + rank;
-          slot_pos[(size_t)t * k + j] = pos;
-          if (pos >= 0) src[pos] = t;
+          if (part == 0) {
+            slot_pos[(size_t)t * k + j] = pos;
+            if (pos >= 0) src[pos] = t;
+          }
         }
         if (active) {
           s_pos[lane * k + j] = pos;
@@ -93,12 +96,15 @@ __global__ void __launch_bounds__(256) perm_scatter_kernel(
   }
   __syncthreads();
   if (x_perm == nullptr) return;
+  // the chunk's rows are shared by PM_SPLIT CTAs (slots part, part + PM_SPLIT, ...), so more
+  // copies are in flight per SM than 16-token chunks alone would give
   const int nvec = d * (int)sizeof(Tin) / 16;
-  for (int s = warp; s < PM_CHUNK * k; s += 8) {
+  for (int s = part + PM_SPLIT * warp; s < PM_CHUNK * k; s += PM_SPLIT * 8) {
     const int pos = s_pos[s];
     if (pos < 0) continue;
     const uint4 *srow = (const uint4 *)(x + (size_t)s_tok[s] * d);
     uint4 *drow = (uint4 *)(x_perm + (size_t)pos * d);
+#pragma unroll 4
     for (int v = lane; v < nvec; v += 32) drow[v] = __ldg(srow + v);
   }
 }
