@@ -4,7 +4,7 @@
 //
 // Stable counting sort of the (token, slot) pairs by expert, with the capacity mask:
 //   rank(t, e) = #{t' < t : e in topk(t')};   kept iff rank < C;   row = offsets[e] + rank.
-// Tokens are cut into chunks of 16 (the router's CTA). Steps:
+// Tokens are cut into chunks of 8 (the router's CTA). Steps:
 //   hist    per-chunk expert histogram -> chunk_count[chunk][E] (inside the layer call the
 //           router's per-CTA counts already are this histogram, so it is only launched by
 //           moe_permute on its own)
@@ -16,8 +16,8 @@
 
 namespace moe {
 
-constexpr int PM_CHUNK = 16;
-constexpr int PM_SPLIT = 4;  // CTAs per chunk in the scatter
+constexpr int PM_CHUNK = 8;
+constexpr int PM_SPLIT = 2;  // CTAs per chunk in the scatter
 
 __global__ void __launch_bounds__(256) perm_hist_kernel(const int32_t *__restrict__ idx, int T,
                                                         int k, int E,

@@ -25,8 +25,9 @@
 
 namespace moe {
 
-constexpr int RT_TM = 16;          // tokens per CTA
-constexpr int RT_THREADS = 256;    // 8 warps, each a slice of the K dimension
+constexpr int RT_TM = 8;           // tokens per CTA (one fp64 MMA row tile)
+constexpr int RT_WARPS = 4;        // each a slice of the K dimension
+constexpr int RT_THREADS = 32 * RT_WARPS;
 constexpr int RT_KB = 16;          // k block: lane (row r, column c) of a fragment reads the 4
                                    // consecutive elements 4c..4c+3 of the block with one load
 constexpr int RT_SEL_THREAD_MAX_E = 64;  // up to this many experts, one thread selects per token
@@ -358,49 +359,87 @@ __device__ float sigmoid_key(float l, float b, bool force) {
 // ------------------------------------------------------------------ kernels
 // Shared-memory layout of the router kernel (byte offsets), shared by host and device.
 struct RouterSmem {
-  size_t xs, wsb, part, lg, pb, keys, sel_e, sel_p, wn, cnt, flags, xnorm, fix, total;
-  int ldx;  // padded row length of xs / wsb in elements: (ldx * esize) = 32 (mod 128)
+  size_t part, sq, ex, lg, pb, keys, sel_e, sel_p, wn, wexp, cnt, flags, xnorm, xexp, fix, total;
 };
-__host__ __device__ inline RouterSmem router_smem(int E, int d, int NT, int esize, bool sigmoid) {
+__host__ __device__ inline RouterSmem router_smem(int E, int NT, bool sigmoid) {
   RouterSmem L;
   const int EB = 8 * NT;
-  L.ldx = d + 32 / esize;
   size_t o = 0;
   auto take = [&](size_t bytes) { size_t at = o; o = (o + bytes + 15) & ~(size_t)15; return at; };
-  L.xs = take((size_t)RT_TM * L.ldx * esize);
-  L.wsb = take((size_t)EB * L.ldx * esize);
-  L.part = take((size_t)(RT_THREADS / 32) * RT_TM * EB * sizeof(double));
+  L.part = take((size_t)RT_WARPS * RT_TM * EB * sizeof(double));   // per-warp partial sums
+  L.sq = take((size_t)RT_WARPS * (EB + RT_TM) * sizeof(double));   // per-warp sums of squares
+  L.ex = take((size_t)RT_WARPS * (EB + RT_TM) * 2 * sizeof(int));  // per-warp exponent ranges
   L.lg = take((size_t)RT_TM * E * sizeof(float));
   const bool rank_sel = E <= RT_SEL_THREAD_MAX_E;
   L.pb = take(rank_sel ? (size_t)RT_TM * E * sizeof(float) : 0);
-  // sigmoid keys: [16][E] for the rank selection; the warp selection keeps [8][E] in wsb
-  L.keys = take(sigmoid && rank_sel ? (size_t)RT_TM * E * sizeof(float) : 0);
+  L.keys = take(sigmoid ? (size_t)(rank_sel ? RT_TM : RT_WARPS) * E * sizeof(float) : 0);
   L.sel_e = take((size_t)RT_TM * 8 * sizeof(int));
   L.sel_p = take((size_t)RT_TM * 8 * sizeof(float));
   L.wn = take((size_t)EB * sizeof(double));
+  L.wexp = take((size_t)EB * 2 * sizeof(int));
   L.cnt = take((size_t)E * sizeof(int));
   L.flags = take((size_t)RT_TM * ((E + 31) / 32) * sizeof(unsigned));
   L.xnorm = take(RT_TM * sizeof(double));
+  L.xexp = take(RT_TM * 2 * sizeof(int));
   L.fix = take(RT_FIX_CAP * sizeof(double));
   L.total = o;
   return L;
 }
 
-// Four consecutive inputs as fp64 (bf16: one 8-byte load; fp32: one 16-byte load).
-__device__ __forceinline__ void load4d(const __nv_bfloat16 *p, double (&v)[4]) {
-  const uint2 q = *(const uint2 *)p;
-  const __nv_bfloat162 *h = (const __nv_bfloat162 *)&q;
-  const float2 f0 = __bfloat1622float2(h[0]), f1 = __bfloat1622float2(h[1]);
-  v[0] = f0.x; v[1] = f0.y; v[2] = f1.x; v[3] = f1.y;
-}
-__device__ __forceinline__ void load4d(const float *p, double (&v)[4]) {
-  const float4 q = *(const float4 *)p;
-  v[0] = q.x; v[1] = q.y; v[2] = q.z; v[3] = q.w;
-}
+// Raw 4-element fragment loads (bf16: 8 bytes; fp32: 16 bytes) and their conversion to fp64.
+template <typename Tin> struct Frag4;
+template <> struct Frag4<__nv_bfloat16> {
+  using raw_t = uint2;
+  static __device__ __forceinline__ raw_t load(const __nv_bfloat16 *p) { return __ldg((const uint2 *)p); }
+  static __device__ __forceinline__ raw_t zero() { return make_uint2(0u, 0u); }
+  static __device__ __forceinline__ void cvt(raw_t q, double (&v)[4]) {
+    const __nv_bfloat162 *h = (const __nv_bfloat162 *)&q;
+    const float2 f0 = __bfloat1622float2(h[0]), f1 = __bfloat1622float2(h[1]);
+    v[0] = f0.x; v[1] = f0.y; v[2] = f1.x; v[3] = f1.y;
+  }
+  static constexpr int MANT = 7;  // fraction bits
+  // min / max biased exponent over the nonzero elements (subnormals count as exponent 0)
+  static __device__ __forceinline__ void exps(raw_t q, int &mn, int &mx) {
+    const uint32_t w[2] = {q.x, q.y};
+#pragma unroll
+    for (int i = 0; i < 2; ++i)
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const uint32_t b = (w[i] >> (16 * h)) & 0xFFFFu;
+        if (b & 0x7FFFu) {
+          const int e = (int)((b >> 7) & 0xFFu);
+          mn = min(mn, e);
+          mx = max(mx, e);
+        }
+      }
+  }
+};
+template <> struct Frag4<float> {
+  using raw_t = float4;
+  static __device__ __forceinline__ raw_t load(const float *p) { return __ldg((const float4 *)p); }
+  static __device__ __forceinline__ raw_t zero() { return make_float4(0.f, 0.f, 0.f, 0.f); }
+  static __device__ __forceinline__ void cvt(raw_t q, double (&v)[4]) {
+    v[0] = q.x; v[1] = q.y; v[2] = q.z; v[3] = q.w;
+  }
+  static constexpr int MANT = 23;
+  static __device__ __forceinline__ void exps(raw_t q, int &mn, int &mx) {
+    const float f[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint32_t b = __float_as_uint(f[i]);
+      if (b & 0x7FFFFFFFu) {
+        const int e = (int)((b >> 23) & 0xFFu);
+        mn = min(mn, e);
+        mx = max(mx, e);
+      }
+    }
+  }
+};
 
 template <typename Tin, int NT>
-__global__ void __launch_bounds__(RT_THREADS, 2) router_kernel(RouterArgs a) {
+__global__ void __launch_bounds__(RT_THREADS, 4) router_kernel(RouterArgs a) {
   constexpr int EB = 8 * NT;  // experts per round
+  using F = Frag4<Tin>;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   const int E = a.E, d = a.d, k = a.k;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -412,13 +451,14 @@ __global__ void __launch_bounds__(RT_THREADS, 2) router_kernel(RouterArgs a) {
   const int force_level = g_force_exact;
   const bool force = force_level != 0;
   const bool sigmoid = a.score == MOE_SCORE_SIGMOID;
-  const RouterSmem SL = router_smem(E, d, NT, (int)sizeof(Tin), sigmoid);
-  const int ldx = SL.ldx;
-  Tin *xs = (Tin *)(smem_raw + SL.xs);    // [16][ldx] the CTA's tokens
-  Tin *wsb = (Tin *)(smem_raw + SL.wsb);  // [EB][ldx] the round's router rows
-  double *part = (double *)(smem_raw + SL.part);
+  const RouterSmem SL = router_smem(E, NT, sigmoid);
+  double *part = (double *)(smem_raw + SL.part);  // [RT_WARPS][RT_TM][EB]
+  double *sq = (double *)(smem_raw + SL.sq);      // [RT_WARPS][EB + RT_TM]
+  int *exr = (int *)(smem_raw + SL.ex);            // [RT_WARPS][EB + RT_TM][min, max]
+  int *wexp = (int *)(smem_raw + SL.wexp);         // [EB][min, max] of the round's rows
+  int *xexp = (int *)(smem_raw + SL.xexp);         // [RT_TM][min, max]
   float *lg = (float *)(smem_raw + SL.lg);
-  float *keys = (float *)(smem_raw + (E <= RT_SEL_THREAD_MAX_E ? SL.keys : SL.wsb));
+  float *keys = (float *)(smem_raw + SL.keys);
   const bool rank_sel = E <= RT_SEL_THREAD_MAX_E;
   float *pb = rank_sel ? (float *)(smem_raw + SL.pb) : lg;
   int *sel_e = (int *)(smem_raw + SL.sel_e);
@@ -435,89 +475,157 @@ __global__ void __launch_bounds__(RT_THREADS, 2) router_kernel(RouterArgs a) {
   for (int i = tid; i < RT_TM * nfw; i += RT_THREADS) flags[i] = 0u;
   if (tid == 0) s_nfix = 0;
   if (blockIdx.x == 0 && tid == 0) *a.counter = 0u;
-  const int rvec = d * (int)sizeof(Tin) / 16;  // 16-byte vectors per row
-  for (int i = tid; i < RT_TM * rvec; i += RT_THREADS) {
-    const int r = i / rvec, v = i - r * rvec;
-    uint4 q = make_uint4(0u, 0u, 0u, 0u);
-    if (r < ntok) q = *(const uint4 *)(x + (size_t)(t0 + r) * d + v * (16 / (int)sizeof(Tin)));
-    *(uint4 *)(xs + r * ldx + v * (16 / (int)sizeof(Tin))) = q;
-  }
-  __syncthreads();
-  for (int tt = warp; tt < RT_TM; tt += RT_THREADS / 32) {
-    double s = 0.0;
-    for (int i = lane; i < d; i += 32) {
-      const double v = (double)Elem<Tin>::to_f(xs[tt * ldx + i]);
-      s = fma(v, v, s);
-    }
-    s = warp_sum_d(s);
-    if (lane == 0) xnorm[tt] = sqrt(s);
-  }
 
-  // ---- logits on the fp64 tensor cores. Each round stages 8*NT router rows; warp w takes the
-  // 16-k blocks w, w+8, ... For a block, the lane at fragment (row r, column c) loads elements
-  // 4c..4c+3 of its token row and of its expert row, and MMA step i uses element 4c+i: a
-  // permutation of k inside the block, identical for both operands. The eight per-warp partial
-  // sums are then added in warp order.
+  // ---- logits on the fp64 tensor cores, one round per 8*NT experts. Warp w takes the 16-k
+  // blocks w, w+4, ... of the d dimension. For a block, the lane at fragment (row r, column c)
+  // loads elements 4c..4c+3 of token row r and of expert row r of each column tile, straight
+  // from global memory (L1/L2), and MMA step i uses element 4c+i: a permutation of k inside the
+  // block, identical for both operands. Every element of the CTA's token rows and of the
+  // round's expert rows is loaded exactly once per round, so the sums of squares of the loaded
+  // values give |x_t| and |W_e| for the rounding bound. The four per-warp partial sums are then
+  // added in warp order.
   const int nkb = d / RT_KB;
+  const bool tok_ok = fr < ntok;
+  const Tin *xrow_f = x + (size_t)(t0 + (tok_ok ? fr : 0)) * d + 4 * fc;
   for (int eb = 0; eb < E; eb += EB) {
-    __syncthreads();  // the previous round is done with wsb and part
-    for (int i = tid; i < EB * rvec; i += RT_THREADS) {
-      const int r = i / rvec, v = i - r * rvec;
-      uint4 q = make_uint4(0u, 0u, 0u, 0u);
-      if (eb + r < E) q = *(const uint4 *)(wr + (size_t)(eb + r) * d + v * (16 / (int)sizeof(Tin)));
-      *(uint4 *)(wsb + r * ldx + v * (16 / (int)sizeof(Tin))) = q;
+    double acc[NT][2], wsq[NT];
+    double xsq = 0.0;
+    int xmn = 255, xmx = -1, wmn[NT], wmx[NT];
+    const Tin *wrow_f[NT];
+    bool e_ok[NT];
+#pragma unroll
+    for (int j = 0; j < NT; ++j) {
+      acc[j][0] = acc[j][1] = 0.0;
+      wsq[j] = 0.0;
+      wmn[j] = 255;
+      wmx[j] = -1;
+      const int e = eb + 8 * j + fr;
+      e_ok[j] = e < E;
+      wrow_f[j] = wr + (size_t)(e_ok[j] ? e : 0) * d + 4 * fc;
     }
-    __syncthreads();
-    for (int r = warp; r < EB; r += RT_THREADS / 32) {  // |W_e|_2 of the round's rows
-      double s = 0.0;
-      for (int i = lane; i < d; i += 32) {
-        const double v = (double)Elem<Tin>::to_f(wsb[r * ldx + i]);
-        s = fma(v, v, s);
+    // one-block-ahead prefetch of the raw fragments
+    typename F::raw_t ra = F::zero(), rb[NT];
+#pragma unroll
+    for (int j = 0; j < NT; ++j) rb[j] = F::zero();
+    int kb = warp;
+    if (kb < nkb) {
+      if (tok_ok) ra = F::load(xrow_f + kb * RT_KB);
+#pragma unroll
+      for (int j = 0; j < NT; ++j) if (e_ok[j]) rb[j] = F::load(wrow_f[j] + kb * RT_KB);
+    }
+    for (; kb < nkb; kb += RT_WARPS) {
+      double av[4], bv[NT][4];
+      F::cvt(ra, av);
+      F::exps(ra, xmn, xmx);
+#pragma unroll
+      for (int j = 0; j < NT; ++j) {
+        F::cvt(rb[j], bv[j]);
+        F::exps(rb[j], wmn[j], wmx[j]);
       }
-      s = warp_sum_d(s);
-      if (lane == 0) wn[r] = sqrt(s);
-    }
-    double acc[2][NT][2];
+      const int kn = kb + RT_WARPS;
+      if (kn < nkb) {
+        ra = tok_ok ? F::load(xrow_f + kn * RT_KB) : F::zero();
 #pragma unroll
-    for (int j = 0; j < NT; ++j) acc[0][j][0] = acc[0][j][1] = acc[1][j][0] = acc[1][j][1] = 0.0;
-    for (int kb = warp; kb < nkb; kb += RT_THREADS / 32) {
-      const int kk = kb * RT_KB + 4 * fc;
-      double a0[4], a1[4], bw[NT][4];
-      load4d(xs + fr * ldx + kk, a0);
-      load4d(xs + (8 + fr) * ldx + kk, a1);
+        for (int j = 0; j < NT; ++j) rb[j] = e_ok[j] ? F::load(wrow_f[j] + kn * RT_KB) : F::zero();
+      }
 #pragma unroll
-      for (int j = 0; j < NT; ++j) load4d(wsb + (8 * j + fr) * ldx + kk, bw[j]);
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
+      for (int i = 0; i < 4; ++i) {
+        xsq = fma(av[i], av[i], xsq);
 #pragma unroll
         for (int j = 0; j < NT; ++j) {
-          dmma_8x8x4(acc[0][j], a0[i], bw[j][i]);
-          dmma_8x8x4(acc[1][j], a1[i], bw[j][i]);
+          wsq[j] = fma(bv[j][i], bv[j][i], wsq[j]);
+          dmma_8x8x4(acc[j], av[i], bv[j][i]);
         }
+      }
+    }
+    // per-warp row sums of squares (lanes of one fragment row differ in fc = lane bits 0-1)
+#pragma unroll
+    for (int o = 1; o < 4; o <<= 1) {
+      xsq += __shfl_xor_sync(0xffffffffu, xsq, o);
+      xmn = min(xmn, __shfl_xor_sync(0xffffffffu, xmn, o));
+      xmx = max(xmx, __shfl_xor_sync(0xffffffffu, xmx, o));
+#pragma unroll
+      for (int j = 0; j < NT; ++j) {
+        wsq[j] += __shfl_xor_sync(0xffffffffu, wsq[j], o);
+        wmn[j] = min(wmn[j], __shfl_xor_sync(0xffffffffu, wmn[j], o));
+        wmx[j] = max(wmx[j], __shfl_xor_sync(0xffffffffu, wmx[j], o));
+      }
+    }
+    if (fc == 0) {
+#pragma unroll
+      for (int j = 0; j < NT; ++j) {
+        sq[warp * (EB + RT_TM) + 8 * j + fr] = wsq[j];
+        exr[2 * (warp * (EB + RT_TM) + 8 * j + fr)] = wmn[j];
+        exr[2 * (warp * (EB + RT_TM) + 8 * j + fr) + 1] = wmx[j];
+      }
+      sq[warp * (EB + RT_TM) + EB + fr] = xsq;
+      exr[2 * (warp * (EB + RT_TM) + EB + fr)] = xmn;
+      exr[2 * (warp * (EB + RT_TM) + EB + fr) + 1] = xmx;
     }
 #pragma unroll
     for (int j = 0; j < NT; ++j)
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        part[(warp * RT_TM + fr) * EB + 8 * j + 2 * fc + h] = acc[0][j][h];
-        part[(warp * RT_TM + 8 + fr) * EB + 8 * j + 2 * fc + h] = acc[1][j][h];
+      for (int h = 0; h < 2; ++h) part[(warp * RT_TM + fr) * EB + 8 * j + 2 * fc + h] = acc[j][h];
+    __syncthreads();
+    for (int q = tid; q < EB + RT_TM; q += RT_THREADS) {
+      double t = 0.0;
+      int mn = 255, mx = -1;
+#pragma unroll
+      for (int w = 0; w < RT_WARPS; ++w) {
+        t += sq[w * (EB + RT_TM) + q];
+        mn = min(mn, exr[2 * (w * (EB + RT_TM) + q)]);
+        mx = max(mx, exr[2 * (w * (EB + RT_TM) + q) + 1]);
       }
+      if (q < EB) {
+        wn[q] = sqrt(t);
+        wexp[2 * q] = mn;
+        wexp[2 * q + 1] = mx;
+      } else if (eb == 0) {
+        xnorm[q - EB] = sqrt(t);
+        xexp[2 * (q - EB)] = mn;
+        xexp[2 * (q - EB) + 1] = mx;
+      }
+    }
     __syncthreads();
     for (int q = tid; q < RT_TM * EB; q += RT_THREADS) {
       const int tt = q / EB, e = eb + q % EB;
       if (tt < ntok && e < E) {
         double s = 0.0;
 #pragma unroll
-        for (int w = 0; w < RT_THREADS / 32; ++w) s += part[(w * RT_TM + tt) * EB + q % EB];
+        for (int w = 0; w < RT_WARPS; ++w) s += part[(w * RT_TM + tt) * EB + q % EB];
         const double o = a.off ? (double)a.off[e] : 0.0;
         s += o;
-        // any summation order over d products plus 8 partials and the offset:
+        // any summation order over d products plus the partials and the offset:
         // |error| <= gamma_{d+16} (sum |x_i W_i| + |off|) <= (d+16) 2^-52 (|x|_2 |W_e|_2 + |off|)
         const double B = (double)(d + 16) * 0x1p-52 * (xnorm[tt] * wn[q % EB] + fabs(o));
+        // Exactness certificate. With biased exponents of at least xmin and wmin (all normal),
+        // every product is an integer multiple of 2^qq, qq = xmin + wmin - 254 - 2 MANT, and so is
+        // the offset when its own quantum is folded in. Every partial sum, in any order, is
+        // bounded by sum |x_i W_i| + |off| <= |x|_2 |W_e|_2 + |off| (Cauchy-Schwarz); the computed
+        // norms are within (d + 8) 2^-50 of that relatively. Below 2^(qq + 53) every partial sum
+        // is an fp64 value, so s is the exact sum and its round-to-nearest-even to fp32 is the
+        // canonical logit, exact ties included.
+        bool exact;
+        {
+          const int xmn_ = xexp[2 * tt], xmx_ = xexp[2 * tt + 1];
+          const int wmn_ = wexp[2 * (q % EB)], wmx_ = wexp[2 * (q % EB) + 1];
+          int qq = 1 << 20;
+          if (xmx_ >= 0 && wmx_ >= 0) qq = xmn_ + wmn_ - 254 - 2 * F::MANT;
+          bool ok = (xmx_ < 0 || wmx_ < 0 || (xmn_ > 0 && wmn_ > 0)) && xmx_ < 255 && wmx_ < 255;
+          if (o != 0.0) {
+            const int eo = (int)((__float_as_uint((float)o) >> 23) & 0xFFu);
+            ok = ok && eo > 0 && eo < 255;
+            qq = min(qq, eo - 150);
+          }
+          const double S = (xnorm[tt] * wn[q % EB] + fabs(o)) * (1.0 + (double)(d + 8) * 0x1p-50);
+          exact = ok && S <= ldexp(1.0, min(qq + 53, 1023));
+        }
         float r, up, dn;
         double mh, ml;
         float l;
-        if (rn32_certain(s, B, r, up, dn, mh, ml) && !force) {
+        if (exact && !force) {
+          l = __double2float_rn(s);
+        } else if (rn32_certain(s, B, r, up, dn, mh, ml) && !force) {
           l = r;
         } else {
           // undecided: resolved exactly by the fixup pass below, which needs the fp64 sum
@@ -533,8 +641,8 @@ __global__ void __launch_bounds__(RT_THREADS, 2) router_kernel(RouterArgs a) {
         lg[tt * E + e] = l;
       }
     }
+    __syncthreads();  // part, sq and wn are rewritten by the next round
   }
-  __syncthreads();
 
   // ---- fixup of undecided logits: flag words dealt round-robin to the warps; one warp decides
   // one logit exactly (see resolve_logit)
@@ -545,7 +653,7 @@ __global__ void __launch_bounds__(RT_THREADS, 2) router_kernel(RouterArgs a) {
       const int ee = e0 + __ffs(m) - 1;
       m &= m - 1;
       const int slot = __float_as_int(lg[tt * E + ee]);
-      const Tin *xrow = xs + tt * ldx;  // the staged copy (16-byte aligned rows)
+      const Tin *xrow = x + (size_t)(t0 + tt) * d;
       const Tin *wrow = wr + (size_t)ee * d;
       const double o = a.off ? (double)a.off[ee] : 0.0;
       double approx;

@@ -138,6 +138,28 @@ def test_logits_on_rounding_midpoints():
     assert ref["route"]["idx"][1].tolist() == [0, 1, 2]
 
 
+def test_certified_ties_round_to_even():
+    """Sums exactly on fp32 midpoints with a narrow exponent span: the fp64 sum is exact, so it
+    decides the tie by round-to-nearest-even without the exact pass. Expert 0 gets 1 + 2^-24
+    (rounds down to 1) for token 0 and 1 + 3 2^-24 (rounds up to 1 + 2^-22) for token 1; either
+    rounding the other way changes the top-2 set."""
+    c = MoEConfig(name="tie", T=2, d=64, E=3, top_k=2, n_shared=0, ffn=64, ffn_shared=0)
+    inp = make_inputs(c)
+    x = np.zeros((2, 64), np.float32)
+    x[:, 0] = 1.0
+    x[0, 1] = 2.0 ** -24
+    x[1, 1] = 3 * 2.0 ** -24
+    x[1, 2] = 2.0 ** -22
+    W = np.zeros((3, 64), np.float32)
+    W[0, :2] = 1.0
+    W[1, 0], W[1, 1] = 1.0, 2.0
+    W[2, 0], W[2, 2] = 1.0, 1.0
+    inp["x"], inp["w_router"] = x, W
+    o, ref = check_steps(c, inp, exact_only=True)
+    assert ref["route"]["idx"][0].tolist() == [1, 0]
+    assert ref["route"]["idx"][1].tolist() == [1, 0]
+
+
 def test_empty_call():
     c = get_config("quartz", T=0)
     run = GpuRun(c, make_inputs(c, T=0))
