@@ -212,6 +212,7 @@ def run_ours(args, rank, world, local_rank):
 
     import fine_grained_mixture_moe_b200 as moe
     from fine_grained_mixture_moe_b200 import binding as B
+    from fine_grained_mixture_moe_b200 import dist as D
     from fine_grained_mixture_moe_b200.layer import MoELayer, upload_weights
     from moe_synth import get_config, make_inputs
 
@@ -244,31 +245,24 @@ def run_ours(args, rank, world, local_rank):
         T, k, E, d = c.T, c.top_k, c.E, c.d
         idx = torch.empty((T, k), dtype=torch.int32, device=dev)
         wts = torch.empty((T, k), dtype=torch.float32, device=dev)
-        stats = torch.empty(2 * E, dtype=torch.float32, device=dev)
-        cnt32 = torch.empty(E, dtype=torch.int32, device=dev)
-        prob = stats[E:]
+        packed = torch.empty(2 * E, dtype=torch.float32, device=dev)
+        prob = torch.empty(E, dtype=torch.float32, device=dev)
         offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
         slot = torch.empty((T, k), dtype=torch.int32, device=dev)
         src = torch.empty(T * k, dtype=torch.int32, device=dev)
         xp = torch.empty((T * k, d), dtype=dt, device=dev)
         yp = torch.empty((T * k, d), dtype=torch.float32, device=dev)
         ysh = torch.empty((T, d), dtype=torch.float32, device=dev) if c.n_shared else None
-        gcfg = B.make_config(T=T * world, d=c.d, E=E, top_k=k, n_shared=c.n_shared, ffn=c.ffn,
-                             ffn_shared=c.ffn_shared, rank=c.rank, score=c.score,
-                             expert=c.expert, dtype=c.dtype, norm_topk=c.norm_topk,
-                             capacity_factor=c.capacity_factor, aux_alpha=c.aux_alpha)
-        gcnt = torch.empty(E, dtype=torch.int32, device=dev)
+        gcfg = D.loss_config(cfg, world)
 
         def step():
-            B.moe_route(cfg, x, layer.wstruct, idx, wts, cnt32, prob, layer.ws, layer.ws_bytes)
-            stats[:E].copy_(cnt32)                      # counts < 2^24: exact in fp32
-            dist.all_reduce(stats)
+            B.moe_route(cfg, x, layer.wstruct, idx, wts, cnt, prob, layer.ws, layer.ws_bytes)
+            gcnt, gprob = D.allreduce_route_stats(cnt, prob, T * world * k, packed=packed)
             B.moe_permute(cfg, x, idx, offsets, slot, src, xp, layer.ws, layer.ws_bytes)
             B.moe_expert_forward(cfg, xp, offsets, x, layer.wstruct, yp, ysh, layer.ws,
                                  layer.ws_bytes)
             B.moe_combine(cfg, yp, ysh, slot, wts, y)
-            gcnt.copy_(stats[:E])
-            B.moe_aux_loss(gcfg, gcnt, prob, aux)
+            B.moe_aux_loss(gcfg, gcnt, gprob, aux)
     else:
         def step():
             layer.forward(x, y, aux, cnt)
