@@ -167,7 +167,9 @@ def algorithmic(c, n_kept: int):
         if S:
             out["gemm_gateup"] = {"flops": 4.0 * d * S * fs * T}
             out["gemm_down"] = {"flops": 2.0 * d * S * fs * T}
-    out["combine"] = {"bytes": n_kept * d * 4.0 + (T * d * 4.0 if S else 0) + 8.0 * T * k +
+    # routed expert rows (bf16 for bf16 SwiGLU layers, else fp32), shared output and y in fp32
+    ys = 2 if (c.dtype == "bf16" and c.expert == "swiglu") else 4
+    out["combine"] = {"bytes": n_kept * d * ys + (T * d * 4.0 if S else 0) + 8.0 * T * k +
                       T * d * 4.0}
     return out
 
@@ -213,7 +215,7 @@ def run_ours(args, rank, world, local_rank):
     import fine_grained_mixture_moe_b200 as moe
     from fine_grained_mixture_moe_b200 import binding as B
     from fine_grained_mixture_moe_b200 import dist as D
-    from fine_grained_mixture_moe_b200.layer import MoELayer, upload_weights
+    from fine_grained_mixture_moe_b200.layer import MoELayer, upload_weights, y_perm_dtype
     from moe_synth import get_config, make_inputs
 
     from fine_grained_mixture_moe_b200 import build as _b
@@ -251,7 +253,7 @@ def run_ours(args, rank, world, local_rank):
         slot = torch.empty((T, k), dtype=torch.int32, device=dev)
         src = torch.empty(T * k, dtype=torch.int32, device=dev)
         xp = torch.empty((T * k, d), dtype=dt, device=dev)
-        yp = torch.empty((T * k, d), dtype=torch.float32, device=dev)
+        yp = torch.empty((T * k, d), dtype=y_perm_dtype(cfg), device=dev)
         ysh = torch.empty((T, d), dtype=torch.float32, device=dev) if c.n_shared else None
         gcfg = D.loss_config(cfg, world)
 

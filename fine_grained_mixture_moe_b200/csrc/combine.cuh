@@ -1,57 +1,61 @@
 // Weighted un-permute and the load-balancing loss.
 //
 // combine: y[t] = y_shared[t] + sum_j [slot_pos[t,j] >= 0] w[t,j] * y_perm[slot_pos[t,j]]
-// (Moonfrost: "a token passes through 4 of 33" - the shared expert plus its top-3), summed in
-// fp32 in slot order; expert outputs and y are fp32 (a bf16 rounding of y alone would cost
-// up to 2^-8 max|y| / rms(y), the whole error budget). A gather: no atomics, bitwise-deterministic.
-// One warp per token, 16-byte vectors along the hidden dimension.
+// (Moonfrost expert card: a token passes through the shared expert and its top-k routed ones),
+// summed in fp32 in slot order. The routed outputs y_perm are in the layer's dtype (bf16 rows
+// average out in the weighted sum); the shared output and y are fp32, since a bf16 rounding of
+// y itself would cost up to 2^-8 max|y| / rms(y), the whole error budget. A gather: no atomics,
+// bitwise-deterministic.
 //
-// aux: L = alpha * E * sum_i (count_i / (T k)) * (prob_sum_i / T) (Quartz "0.01-weighted
-// load-balancing loss"), accumulated in fp64 in a fixed order.
+// aux: L = alpha * E * sum_i (count_i / (T k)) * (prob_sum_i / T) (Quartz: the load-balancing
+// term, weight 0.01), accumulated in fp64 in a fixed order.
 #pragma once
 #include "common.cuh"
 
 namespace moe {
 
-template <typename T> struct Vec16;
-template <> struct Vec16<float> {
+// One 16-byte vector of expert outputs: 4 fp32 (fp32 layers) or 8 bf16 (bf16 layers), loaded
+// with the streaming hint (each row is read once) and accumulated in fp32.
+template <typename Ty> struct YVec;
+template <> struct YVec<float> {
+  using raw_t = float4;
   static constexpr int N = 4;
-  static __device__ __forceinline__ void load(const float *p, float *v) {
-    const float4 q = __ldg((const float4 *)p);
-    v[0] = q.x; v[1] = q.y; v[2] = q.z; v[3] = q.w;
-  }
-  static __device__ __forceinline__ void store(float *p, const float *v) {
-    *(float4 *)p = make_float4(v[0], v[1], v[2], v[3]);
+  static __device__ __forceinline__ raw_t load(const float *p) { return __ldcs((const float4 *)p); }
+  static __device__ __forceinline__ void fma(float w, raw_t q, float *a) {
+    a[0] = fmaf(w, q.x, a[0]);
+    a[1] = fmaf(w, q.y, a[1]);
+    a[2] = fmaf(w, q.z, a[2]);
+    a[3] = fmaf(w, q.w, a[3]);
   }
 };
-template <> struct Vec16<__nv_bfloat16> {
+template <> struct YVec<__nv_bfloat16> {
+  using raw_t = uint4;
   static constexpr int N = 8;
-  static __device__ __forceinline__ void load(const __nv_bfloat16 *p, float *v) {
-    const uint4 q = __ldg((const uint4 *)p);
+  static __device__ __forceinline__ raw_t load(const __nv_bfloat16 *p) {
+    return __ldcs((const uint4 *)p);
+  }
+  static __device__ __forceinline__ void fma(float w, raw_t q, float *a) {
     const __nv_bfloat162 *h = (const __nv_bfloat162 *)&q;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const float2 f = __bfloat1622float2(h[i]);
-      v[2 * i] = f.x;
-      v[2 * i + 1] = f.y;
+      a[2 * i] = fmaf(w, f.x, a[2 * i]);
+      a[2 * i + 1] = fmaf(w, f.y, a[2 * i + 1]);
     }
-  }
-  static __device__ __forceinline__ void store(__nv_bfloat16 *p, const float *v) {
-    uint4 q;
-    __nv_bfloat162 *h = (__nv_bfloat162 *)&q;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) h[i] = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
-    *(uint4 *)p = q;
   }
 };
 
-__global__ void __launch_bounds__(256) combine_kernel(const float *__restrict__ y_perm,
+// One warp per token; each lane owns N consecutive columns per vector and two vectors per pass,
+// with every load of a pass issued before the sums. d is a multiple of 64, so a lane's vector is
+// wholly inside or wholly outside the row.
+template <typename Ty>
+__global__ void __launch_bounds__(256) combine_kernel(const Ty *__restrict__ y_perm,
                                                       const float *__restrict__ y_shared,
                                                       const int32_t *__restrict__ slot_pos,
                                                       const float *__restrict__ w,
                                                       float *__restrict__ y, int T, int k, int d) {
-  using Tio = float;
-  constexpr int V = Vec16<Tio>::N;
+  using YV = YVec<Ty>;
+  constexpr int V = YV::N;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t = blockIdx.x * 8 + warp;
   if (t >= T) return;
@@ -68,23 +72,26 @@ __global__ void __launch_bounds__(256) combine_kernel(const float *__restrict__ 
     pos[j] = __shfl_sync(0xffffffffu, pos_l, j);
     wj[j] = __shfl_sync(0xffffffffu, w_l, j);
   }
-  // two vectors per lane per pass, all loads of a pass issued before the sums
 #pragma unroll 1
   for (int c0 = lane * V; c0 < d; c0 += 64 * V) {
     float acc[2][V];
-    float v[2][8][V];
+    typename YV::raw_t v[2][8];
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
       const int c = c0 + h * 32 * V;
       if (c < d) {
-        if (y_shared) Vec16<Tio>::load(y_shared + (size_t)t * d + c, acc[h]);
-        else {
 #pragma unroll
-          for (int i = 0; i < V; ++i) acc[h][i] = 0.0f;
+        for (int i = 0; i < V; i += 4) {
+          float4 q = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+          if (y_shared) q = __ldcs((const float4 *)(y_shared + (size_t)t * d + c + i));
+          acc[h][i] = q.x;
+          acc[h][i + 1] = q.y;
+          acc[h][i + 2] = q.z;
+          acc[h][i + 3] = q.w;
         }
 #pragma unroll
         for (int j = 0; j < 8; ++j)
-          if (j < k && pos[j] >= 0) Vec16<Tio>::load(y_perm + (size_t)pos[j] * d + c, v[h][j]);
+          if (j < k && pos[j] >= 0) v[h][j] = YV::load(y_perm + (size_t)pos[j] * d + c);
       }
     }
 #pragma unroll
@@ -93,11 +100,11 @@ __global__ void __launch_bounds__(256) combine_kernel(const float *__restrict__ 
       if (c < d) {
 #pragma unroll
         for (int j = 0; j < 8; ++j)
-          if (j < k && pos[j] >= 0) {
+          if (j < k && pos[j] >= 0) YV::fma(wj[j], v[h][j], acc[h]);
 #pragma unroll
-            for (int i = 0; i < V; ++i) acc[h][i] = fmaf(wj[j], v[h][j][i], acc[h][i]);
-          }
-        __stcs((float4 *)(y + (size_t)t * d + c), make_float4(acc[h][0], acc[h][1], acc[h][2], acc[h][3]));
+        for (int i = 0; i < V; i += 4)
+          __stcs((float4 *)(y + (size_t)t * d + c + i),
+                 make_float4(acc[h][i], acc[h][i + 1], acc[h][i + 2], acc[h][i + 3]));
       }
     }
   }

@@ -255,7 +255,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) gemm_tc_kernel(const __grid_con
           int b_row, b_col;
           if (routed) {
             b_row = ti.g * ti.N + ti.n0;
-            b_col = kk;
+            b_col = p.kb_r ? kk % p.kb_r : kk;
           } else {
             const int piece = kk / p.piece_k;
             b_row = piece * p.piece_rows + ti.n0;
@@ -348,7 +348,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) gemm_tc_kernel(const __grid_con
       void *out = routed ? p.out_r : p.out_s;
       const int ldo = routed ? p.ldo_r : p.ldo_s;
       const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * C::ACC_COLS);
-      // fp32 outputs (expert outputs) use a staged write-back: the warp's 32 rows x 32 columns
+      // fp32 outputs use a staged write-back: the warp's 32 rows x 32 columns
       // go to a private 4 KB buffer (16-byte chunk j of row r stored at chunk j ^ (r & 7), so
       // both the row-wise writes and the column-wise reads are conflict-free), then leave as 32
       // row stores of 128 contiguous bytes each instead of 32-row scattered 16-byte stores.
@@ -385,7 +385,37 @@ __global__ void __launch_bounds__(TC_THREADS, 1) gemm_tc_kernel(const __grid_con
               uint4 *dst = (uint4 *)((__nv_bfloat16 *)out + (size_t)(ti.a_row0 + row) * ldo + col);
 #pragma unroll
               for (int i = 0; i < 4; ++i) dst[i] = pk[i];
+              if (MODE == MODE_SCALE && p.lo_split > 0) {
+                // second term: the rounding residual v - hi, exact in fp32, rounded to bf16
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                  const float v0 = __uint_as_float(r0[2 * i]) * __ldg(p.scale + (size_t)ti.g * ti.N + col + 2 * i);
+                  const float v1 = __uint_as_float(r0[2 * i + 1]) * __ldg(p.scale + (size_t)ti.g * ti.N + col + 2 * i + 1);
+                  const float2 hf = __bfloat1622float2(h[i]);
+                  h[i] = __floats2bfloat162_rn(v0 - hf.x, v1 - hf.y);
+                }
+#pragma unroll
+                for (int i = 0; i < 4; ++i) dst[p.lo_split / 8 + i] = pk[i];
+              }
             }
+          }
+          continue;
+        }
+        if (routed && p.out_r_bf16) {
+          // routed expert outputs in bf16: 64 contiguous bytes of the lane's row, stored directly
+          uint32_t r0[32];
+          tmem_ld32(tbase + c, r0);
+          tmem_wait_ld();
+          const int col = ti.n0 + c;
+          if (row_ok && col < ti.N) {
+            uint4 pk[4];
+            __nv_bfloat162 *h = (__nv_bfloat162 *)pk;
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+              h[i] = __floats2bfloat162_rn(__uint_as_float(r0[2 * i]), __uint_as_float(r0[2 * i + 1]));
+            uint4 *dst = (uint4 *)((__nv_bfloat16 *)out + (size_t)(ti.a_row0 + row) * ldo + col);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) dst[i] = pk[i];
           }
           continue;
         }

@@ -176,7 +176,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TC_THREADS, 1)
           int b_row, b_col;
           if (routed) {
             b_row = ti.g * ti.N + ti.n0 + n_off;
-            b_col = kk;
+            b_col = p.kb_r ? kk % p.kb_r : kk;
           } else {
             const int piece = kk / p.piece_k;
             b_row = piece * p.piece_rows + ti.n0 + n_off;
@@ -287,7 +287,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TC_THREADS, 1)
 #pragma unroll
             for (int i = 0; i < 4; ++i) dst[i] = pk[i];
           }
+        } else if (routed && p.out_r_bf16) {
+          // routed expert outputs in bf16: 64 contiguous bytes of the lane's row, stored directly
+          uint32_t r0[32];
+          tmem_ld32(tbase + c, r0);
+          tmem_wait_ld();
+          const int col = ti.n0 + c;
+          if (row_ok && col < ti.N) {
+            uint4 pk[4];
+            __nv_bfloat162 *h = (__nv_bfloat162 *)pk;
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+              h[i] = __floats2bfloat162_rn(__uint_as_float(r0[2 * i]), __uint_as_float(r0[2 * i + 1]));
+            uint4 *dst = (uint4 *)((__nv_bfloat16 *)out + (size_t)(ti.a_row0 + row) * ldo + col);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) dst[i] = pk[i];
+          }
         } else {
+          // fp32 output, staged per warp and written as 128-byte rows
           uint32_t r0[32];
           tmem_ld32(tbase + c, r0);
           tmem_wait_ld();

@@ -10,6 +10,10 @@
 //                        matrix, so S shared experts of width fs act as one of width S*fs.
 // Epilogue modes: GATEUP out = silu(A B0^T) * (A B1^T) (SwiGLU, gate and up fused);
 //                 PLAIN  out = A B0^T;   SCALE out = (A B0^T) * scale[g][n] (low-rank s).
+// Output types in the tensor-core (bf16) kernels: GATEUP and SCALE write bf16 (the next
+// product's operand, SCALE optionally as a hi + lo pair); PLAIN writes the routed groups' rows in
+// bf16 or fp32 (out_r_bf16) and the shared group's rows in fp32. The SIMT (fp32) kernels write
+// fp32 throughout.
 #pragma once
 #include "common.cuh"
 
@@ -28,6 +32,11 @@ struct GroupedGemm {
   void *out_r;
   int ldo_r;
   const float *scale;  // [E, N_r] for MODE_SCALE
+  int kb_r;            // row length of B_r when shorter than K_r: k wraps over B's columns
+                       // (k-block at kk reads B columns kk % kb_r); 0 means K_r
+  int lo_split;        // MODE_SCALE, bf16: > 0 stores v as hi = bf16(v) at column n and
+                       // lo = bf16(v - hi) at column n + lo_split (a two-term bf16 split)
+  int out_r_bf16;      // MODE_PLAIN, tensor-core kernels: routed rows stored as bf16 (else fp32)
   int has_shared, T;
   const void *A_s;
   int lda_s;

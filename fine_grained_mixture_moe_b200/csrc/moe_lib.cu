@@ -82,6 +82,14 @@ int32_t capacity_of(const moe_config_t *c) {
 }
 
 // ------------------------------------------------------------------ workspace layout
+// Routed expert outputs are stored in bf16 for bf16 SwiGLU layers (each enters y through a
+// weighted sum of top_k rows plus the fp32 shared output, which averages their rounding) and in
+// fp32 otherwise: a low-rank layer's y is a weighted sum of as few as two rows and no shared
+// output, where one bf16 rounding of the rows exceeds the layer's error budget on its own.
+inline bool yperm_bf16(const moe_config_t *c) {
+  return c->dtype == MOE_DTYPE_BF16 && c->expert == MOE_EXPERT_SWIGLU;
+}
+
 struct Layout {
   size_t part_cnt, part_prob, chunk_base, kept, scounter;       // route / statistics
   size_t chunk_count;                                           // moe_permute's own histogram
@@ -94,7 +102,10 @@ Layout layout_of(const moe_config_t *c) {
   Layout L;
   const size_t T = c->T, d = c->d, E = c->E, k = c->top_k, es = esize(c);
   const size_t nch = std::max<size_t>(1, ceil_div(c->T, RT_TM));
-  const size_t width = c->expert == MOE_EXPERT_SWIGLU ? (size_t)c->ffn : (size_t)c->rank;
+  // hidden rows: the SwiGLU activations, or the low-rank projection (bf16: hi and lo terms)
+  const size_t width = c->expert == MOE_EXPERT_SWIGLU
+                           ? (size_t)c->ffn
+                           : (size_t)c->rank * (c->dtype == MOE_DTYPE_BF16 ? 2 : 1);
   size_t o = 0;
   auto take = [&](size_t bytes) { size_t at = o; o = align256(o + std::max<size_t>(bytes, 1)); return at; };
   L.part_cnt = take(nch * E * 4);
@@ -113,7 +124,7 @@ Layout layout_of(const moe_config_t *c) {
   L.slot_pos = take(T * k * 4);
   L.src = take(T * k * 4);
   L.x_perm = take(T * k * d * es);
-  L.y_perm = take(T * k * d * 4);    // expert outputs are fp32 for every dtype
+  L.y_perm = take(T * k * d * (yperm_bf16(c) ? 2 : 4));
   L.y_shared = take(T * d * 4);
   L.aux = take(16);
   L.total = o;
@@ -229,10 +240,11 @@ bool build_maps(const GroupedGemm &g, bool two_b, uint32_t b_box, TcMaps *m) {
   const void *any = g.E > 0 ? g.A_r : g.A_s;
   bool ok = true;
   ok &= make_map(&m->a_r, g.E > 0 ? g.A_r : any, g.E > 0 ? g.rows_r : 1, g.E > 0 ? g.K_r : 64, 128);
+  const int kb = g.kb_r ? g.kb_r : g.K_r;  // row length of the routed weights
   ok &= make_map(&m->b0_r, g.E > 0 ? g.B0_r : any, g.E > 0 ? (uint64_t)g.E * g.N_r : 1,
-                 g.E > 0 ? g.K_r : 64, b_box);
+                 g.E > 0 ? kb : 64, b_box);
   ok &= make_map(&m->b1_r, (g.E > 0 && two_b) ? g.B1_r : any,
-                 (g.E > 0 && two_b) ? (uint64_t)g.E * g.N_r : 1, g.E > 0 ? g.K_r : 64, b_box);
+                 (g.E > 0 && two_b) ? (uint64_t)g.E * g.N_r : 1, g.E > 0 ? kb : 64, b_box);
   ok &= make_map(&m->a_s, g.has_shared ? g.A_s : any, g.has_shared ? g.T : 1,
                  g.has_shared ? g.K_s : 64, 128);
   ok &= make_map(&m->b0_s, g.has_shared ? g.B0_s : any, g.has_shared ? g.b_rows_s : 1,
@@ -461,7 +473,7 @@ moe_status_t experts_impl(const moe_config_t *c, const void *x_perm, const int32
     MOE_TRY(launch_gemm<MODE_GATEUP>(c, g1, 128, st, K_GEMM_GATEUP));
     GroupedGemm g2 = g;
     g2.E = E; g2.A_r = H; g2.lda_r = f; g2.B0_r = w->w_down; g2.N_r = d; g2.K_r = f;
-    g2.out_r = y_perm; g2.ldo_r = d;
+    g2.out_r = y_perm; g2.ldo_r = d; g2.out_r_bf16 = yperm_bf16(c) ? 1 : 0;
     g2.has_shared = sh;
     if (sh) {
       g2.A_s = Hs; g2.lda_s = S * fs; g2.B0_s = w->ws_down; g2.N_s = d; g2.K_s = S * fs;
@@ -469,15 +481,20 @@ moe_status_t experts_impl(const moe_config_t *c, const void *x_perm, const int32
     }
     return launch_gemm<MODE_PLAIN>(c, g2, bn_down, st, K_GEMM_DOWN);
   }
-  // low-rank experts: Z = (X V^T) * s  (rounded to dtype), then Y = Z U^T
+  // low-rank experts: Z = (X V^T) * s, then Y = Z U^T. In bf16, Z is kept as two bf16 terms
+  // [Z_hi | Z_lo] (Z_lo = the rounding residual), and the second product runs over K = 2r with
+  // the k loop wrapping over U's r columns: Y = Z_hi U^T + Z_lo U^T, i.e. Z at ~2^-17 relative
+  // precision for twice the (small) flops of that product.
   const int r = c->rank;
+  const bool split = c->dtype == MOE_DTYPE_BF16;
   GroupedGemm g1 = g;
   g1.E = E; g1.A_r = x_perm; g1.lda_r = d; g1.B0_r = w->lr_V; g1.N_r = r; g1.K_r = d;
-  g1.out_r = H; g1.ldo_r = r; g1.scale = w->lr_s;
+  g1.out_r = H; g1.ldo_r = split ? 2 * r : r; g1.scale = w->lr_s; g1.lo_split = split ? r : 0;
   MOE_TRY(launch_gemm<MODE_SCALE>(c, g1, 64, st, K_GEMM_LR1));
   GroupedGemm g2 = g;
-  g2.E = E; g2.A_r = H; g2.lda_r = r; g2.B0_r = w->lr_U; g2.N_r = d; g2.K_r = r;
-  g2.out_r = y_perm; g2.ldo_r = d;
+  g2.E = E; g2.A_r = H; g2.lda_r = split ? 2 * r : r; g2.B0_r = w->lr_U; g2.N_r = d;
+  g2.K_r = split ? 2 * r : r; g2.kb_r = split ? r : 0;
+  g2.out_r = y_perm; g2.ldo_r = d; g2.out_r_bf16 = yperm_bf16(c) ? 1 : 0;
   MOE_TRY(launch_gemm<MODE_PLAIN>(c, g2, bn_down, st, K_GEMM_LR2));
   if (sh) {
     GroupedGemm g3 = g;
@@ -500,8 +517,12 @@ moe_status_t combine_impl(const moe_config_t *c, const void *y_perm, const void 
   if (c->T == 0) return MOE_OK;
   ProfScope ps(K_COMBINE, st);
   const float *ysh = c->n_shared > 0 ? (const float *)y_shared : nullptr;
-  combine_kernel<<<ceil_div(c->T, 8), 256, 0, st>>>((const float *)y_perm, ysh, slot_pos, wts,
-                                                    (float *)y, c->T, c->top_k, c->d);
+  if (yperm_bf16(c))
+    combine_kernel<__nv_bfloat16><<<ceil_div(c->T, 8), 256, 0, st>>>(
+        (const __nv_bfloat16 *)y_perm, ysh, slot_pos, wts, (float *)y, c->T, c->top_k, c->d);
+  else
+    combine_kernel<float><<<ceil_div(c->T, 8), 256, 0, st>>>(
+        (const float *)y_perm, ysh, slot_pos, wts, (float *)y, c->T, c->top_k, c->d);
   return last_launch_status();
 }
 

@@ -1,6 +1,6 @@
 // Token permutation grouped by expert (Moonfrost expert card: experts as stacked (E, hidden,
-// ffn) tensors with capacity-based routing, replacing a per-expert loop that synchronised the
-// host once per expert; here nothing returns to the host at all).
+// ffn) tensors routed under a per-expert capacity, replacing a per-expert loop that synchronised
+// the host once per expert; here nothing returns to the host at all).
 //
 // Stable counting sort of the (token, slot) pairs by expert, with the capacity mask:
 //   rank(t, e) = #{t' < t : e in topk(t')};   kept iff rank < C;   row = offsets[e] + rank.

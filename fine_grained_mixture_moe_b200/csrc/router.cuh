@@ -1,7 +1,7 @@
 // Router: logits, selection keys, top-k, combine weights and per-expert statistics.
 //
-// What it computes (Quartz "Router: top-6 of 24", Moonfrost "a router picks the top 3",
-// Sutra-1.3B "top-4 routing with sigmoid scoring and bias-based load balancing"):
+// What it computes (Quartz: softmax router, 6 of 24 experts; Moonfrost expert card: top-3
+// routing; Sutra-1.3B: top-4 by sigmoid score plus a per-expert balancing bias):
 //   l[t,e]  = RN32(exact sum_i x[t,i] W[e,i] + off[e])              (fp32, canonical)
 //   key     = l  (softmax)  |  RN32(exact sigmoid(l) + b[e])  (sigmoid + selection bias)
 //   top-k by key, ties -> lower expert index, slot order = descending key

@@ -5,8 +5,8 @@
 //   offsets[0..E]     = exclusive scan over experts of kept_e = min(count_e, C) (dropless: count_e)
 //   aux               = alpha * E * sum_e (count_e / (T k)) * (prob_sum_e / T)
 // One block per expert does the first three; the block that finishes last does the scan over
-// experts and the loss (Moonfrost expert card: capacity-based routing over stacked experts;
-// Quartz: 0.01-weighted load-balancing loss). Chunks are RT_TM = 8 tokens, the router's CTA,
+// experts and the loss (Moonfrost expert card: routing under a per-expert capacity over stacked experts;
+// Quartz: load-balancing loss with weight 0.01). Chunks are RT_TM = 8 tokens, the router's CTA,
 // so the router's per-CTA counts are the permutation's histogram. Every sum has a fixed order.
 #pragma once
 #include "common.cuh"

@@ -1,8 +1,8 @@
 """Data-parallel replicas of the MoE layer: one process per GPU, each holding every weight and
 routing its own T_local tokens, with no exchange on the data path.
 
-The forward pass has exactly one exchange. The load-balancing loss (Quartz: a 0.01-weighted
-load-balancing term) is alpha * E * sum_i f_i P_i with f_i = count_i / (T k) and
+The forward pass has exactly one exchange. The load-balancing loss (Quartz: architecture table,
+row "Router", weight 0.01) is alpha * E * sum_i f_i P_i with f_i = count_i / (T k) and
 P_i = prob_sum_i / T over the whole batch. It is bilinear in the per-expert counts and probability
 sums, so per-rank losses must not be averaged: the ranks sum count[E] and prob_sum[E] over the
 group (one all-reduce of 2E values) and form the loss with T = T_local * world. Capacity stays per

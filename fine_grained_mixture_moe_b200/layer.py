@@ -21,6 +21,14 @@ def torch_dtype(cfg: B.MoEConfig) -> torch.dtype:
     return TORCH_DTYPE[cfg.dtype]
 
 
+def y_perm_dtype(cfg: B.MoEConfig) -> torch.dtype:
+    """Element type of moe_expert_forward's routed output rows (moe.h): bf16 for bf16 SwiGLU
+    layers, fp32 for fp32 layers and for low-rank layers."""
+    if cfg.dtype == B.DTYPE["bf16"] and cfg.expert == B.EXPERT["swiglu"]:
+        return torch.bfloat16
+    return torch.float32
+
+
 def upload_weights(cfg: B.MoEConfig, host: Dict[str, object], device) -> Dict[str, torch.Tensor]:
     """Copy host arrays (numpy or torch, values exact in the layer dtype) to the device."""
     dt = torch_dtype(cfg)

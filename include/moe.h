@@ -4,10 +4,10 @@
  * The layer is the DeepSeek-style fine-grained MoE FFN that the source pages describe:
  *   - Vertex AGI research page / quartz-micro-preview-base model card, "Architecture":
  *     24 narrow routed experts (FFN 640) at hidden 1,024, top-6, 2 always-active shared experts,
- *     a 0.01-weighted load-balancing loss;
+ *     a load-balancing loss with weight 0.01;
  *   - Moonfrost, expert card: 32 routed experts + 1 shared, top-3, experts held as three stacked
- *     (E, hidden, ffn) tensors with capacity-based routing instead of a per-expert loop;
- *   - Sutra-1.3B, "48 + 1 experts": top-4 by sigmoid score with bias-based load balancing;
+ *     (E, hidden, ffn) tensors with routing under a per-expert capacity instead of a per-expert loop;
+ *   - Sutra-1.3B, "48 + 1 experts": top-4 by sigmoid score with balancing through a per-expert bias;
  *   - dormouse, "dropless MoE" and "TSCT low-rank experts": 1,024 experts U*diag(s)*V^T of
  *     rank 64, top-2, dropless.
  *
@@ -91,12 +91,12 @@ size_t moe_workspace_size(const moe_config_t *cfg);
 
 /* Per-expert capacity C of this configuration, or -1 for dropless, or -2 if cfg is invalid.
  * C = ceil(capacity_factor * T * top_k / E) evaluated exactly on the fp32 capacity_factor
- * (Moonfrost expert card: capacity-based routing; the bound is taken over the call's T). */
+ * (Moonfrost expert card: routing under a per-expert capacity; the bound is taken over the call's T). */
 int32_t moe_capacity(const moe_config_t *cfg);
 
 /* Router: logits, scoring, top-k, combine weights and the per-expert statistics.
- * (Quartz "Router: top-6 of 24"; Moonfrost "a router picks the top 3"; Sutra "top-4 routing
- * with sigmoid scoring and bias-based load balancing".)
+ * (Quartz architecture table, row "Router": 6 of 24 experts; Moonfrost expert card: top-3
+ * routing; Sutra-1.3B, "48 + 1 experts": top-4 by sigmoid score, balanced by a per-expert bias.)
  *   l[t,e] = RN32(sum_i x[t,i]*w_router[e,i] + logit_offset[e])  - exact sum, rounded once
  *   key    = l (softmax) or RN32(sigmoid(l) + select_bias[e]) (sigmoid), exact, rounded once
  *   topk_idx[t,j]  [T, top_k] int32: experts by descending key, equal keys -> lower index
@@ -128,21 +128,23 @@ moe_status_t moe_permute(const moe_config_t *cfg, const void *x, const int32_t *
  *   y_shared[t] = sum over shared experts of their SwiGLU output on x[t]
  * Intermediates (the SwiGLU hidden activations, the low-rank projections) are rounded to
  * dtype, since they are the next tensor-core product's operand; accumulation is fp32.
- * y_perm: [T*top_k, d] fp32 (first offsets[E] rows written); y_shared: [T, d] fp32, may be
- * NULL when n_shared = 0. Expert outputs stay fp32 for every dtype: one bf16 rounding of them
- * or of y costs up to 2^-8 * max|y| / rms(y), the whole 2e-2 error budget of the layer. */
+ * y_perm: [T*top_k, d] in dtype (first offsets[E] rows written), each row rounded once from its
+ * fp32 accumulator; y_shared: [T, d] fp32 (the S shared outputs summed in fp32), may be NULL
+ * when n_shared = 0. The routed rows enter y through a weighted sum of top_k of them, which
+ * averages their rounding; the shared output enters y alone, so it stays fp32. */
 moe_status_t moe_expert_forward(const moe_config_t *cfg, const void *x_perm,
                                 const int32_t *offsets, const void *x,
                                 const moe_weights_t *w, void *y_perm, void *y_shared,
                                 void *ws, size_t ws_bytes, void *stream);
 
 /* Weighted un-permute: y[t] = y_shared[t] + sum_j [slot_pos[t,j] >= 0] topk_w[t,j] *
- * y_perm[slot_pos[t,j]], summed in fp32 in slot order. y_perm, y_shared and y are fp32 [.., d].
- * No atomics. y_shared may be NULL (no shared experts). */
+ * y_perm[slot_pos[t,j]], summed in fp32 in slot order. y_perm is in dtype, y_shared and y are
+ * fp32 [.., d]: a bf16 rounding of y itself would cost up to 2^-8 * max|y| / rms(y), the whole
+ * 2e-2 error budget of the layer. No atomics. y_shared may be NULL (no shared experts). */
 moe_status_t moe_combine(const moe_config_t *cfg, const void *y_perm, const void *y_shared,
                          const int32_t *slot_pos, const float *topk_w, void *y, void *stream);
 
-/* Load-balancing loss (Quartz: "0.01-weighted load-balancing loss"):
+/* Load-balancing loss (Quartz: architecture table, row "Router", weight 0.01):
  *   loss = aux_alpha * E * sum_i (expert_count[i] / (T*top_k)) * (prob_sum[i] / T)
  * written to the device scalar `loss` (fp32); 0 when T = 0. */
 moe_status_t moe_aux_loss(const moe_config_t *cfg, const int32_t *expert_count,

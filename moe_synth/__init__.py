@@ -8,10 +8,10 @@ Shapes mirror the models the source pages describe:
 
 * "Quartz" (Vertex AGI research page, "Architecture"; quartz-micro-preview-base model card,
   "Architecture" table): hidden 1,024, 24 routed experts of FFN 640, top-6, 2 shared experts,
-  0.01-weighted load-balancing loss, 4,096 tokens per step.
+  load-balancing loss with weight 0.01, 4,096 tokens per step.
 * Moonfrost (property table and the "stacked (32, hidden, ffn) tensors" card): hidden 896,
-  32 routed experts top-3 plus 1 shared, capacity-based routing.
-* Sutra-1.3B ("48 + 1 experts"): top-4 of 48 by sigmoid score with bias-based balancing,
+  32 routed experts top-3 plus 1 shared, routing under a per-expert capacity.
+* Sutra-1.3B ("48 + 1 experts"): top-4 of 48 by sigmoid score with balancing through a per-expert bias,
   1 shared expert.
 * dormouse ("dropless MoE", "TSCT low-rank experts"): 1,024 experts, top-2, dropless, each
   expert U·diag(s)·Vᵀ of rank 64; batch 24 × sequence 1,024.

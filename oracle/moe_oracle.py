@@ -6,12 +6,12 @@ leg. It shares no code with the CUDA path, and nothing in the product calls it.
 
 What it computes (every step evaluated in fp64 on the exact fp32 / bf16 input values):
 
-1. Router logits (Vertex AGI research page and quartz-micro-preview-base card, "Router: top-6 of
-   24"; Moonfrost, "A router picks the top 3"):
+1. Router logits (Vertex AGI research page and quartz-micro-preview-base card, architecture
+   table, row "Router": 6 of 24 experts; Moonfrost, expert card: top-3 routing):
    ``l[t,e] = RN32( sum_i x[t,i] * W_r[e,i] + off[e] )``, the exact real value rounded once to
    fp32 with round-to-nearest-even. ``off`` is an optional per-expert logit offset.
 2. Selection keys: softmax scoring uses ``key = l``. Sigmoid scoring with a per-expert selection
-   bias (Sutra-1.3B, "48 + 1 experts": sigmoid scoring and bias-based load balancing) uses
+   bias (Sutra-1.3B, "48 + 1 experts": sigmoid scoring and balancing through a per-expert bias) uses
    ``key = RN32( sigma(l) + b[e] )``, again the exact real value rounded once.
 3. Top-k: the k largest keys; equal keys go to the lower expert index first; slot j is the j-th
    entry of that ranking.
@@ -19,7 +19,7 @@ What it computes (every step evaluated in fp64 on the exact fp32 / bf16 input va
    ``sigma(l)`` for sigmoid scoring (the selection bias is not part of the weight). The combine
    weight of slot j is the selected expert's probability, divided by the sum over the k
    selected probabilities when ``norm_topk`` is set.
-5. Capacity (Moonfrost, "capacity-based routing"): ``C = ceil(cf * T * k / E)`` over the T tokens
+5. Capacity (Moonfrost, "routing under a per-expert capacity"): ``C = ceil(cf * T * k / E)`` over the T tokens
    of the call; ``cf <= 0`` is dropless (dormouse, "dropless MoE": no capacity drops). Per
    expert, routed tokens are ranked by ascending token index; rank >= C is dropped.
 6. Permutation grouped by expert (the stacked-expert layout of the Moonfrost card):
@@ -30,7 +30,7 @@ What it computes (every step evaluated in fp64 on the exact fp32 / bf16 input va
    (always active) are SwiGLU experts on every token, their outputs summed.
 8. Combine: ``y[t] = sum_shared + sum_j [kept] w[t,j] * E_{e_j}(x[t])``; dropped slots add 0 and
    the remaining weights are not renormalised.
-9. Load-balancing loss (research page, "0.01-weighted load-balancing loss"):
+9. Load-balancing loss (research page, architecture table, row "Router": load-balancing loss with weight 0.01):
    ``L = alpha * E * sum_i f_i * P_i`` with ``f_i = count_i / (T k)`` counted before capacity
    drops, and ``P_i`` the mean over tokens of the token's probability of expert i (for sigmoid
    scoring, ``sigma(l_i)`` normalised over all E experts).

@@ -12,7 +12,7 @@ import torch
 import oracle
 from fine_grained_mixture_moe_b200 import binding as B
 from moe_synth import CONFIGS, MoEConfig, get_config, make_inputs
-from tests.gpu_helpers import GpuRun, np_, rel_err, tol_of
+from tests.gpu_helpers import GpuRun, np_, rel_err, rel_err_stored, tol_of
 
 pytestmark = pytest.mark.gpu
 
@@ -76,7 +76,8 @@ def check_steps(c, inp, run=None, exact_only=False):
         return o, ref
     tol = tol_of(c)
     ef = ref["experts"]
-    assert rel_err(np_(o["y_perm"])[:N], ef["y_perm"]) <= tol
+    ydt = "bf16" if o["y_perm"].dtype == torch.bfloat16 else "f32"
+    assert rel_err_stored(np_(o["y_perm"])[:N], ef["y_perm"], ydt) <= tol
     if c.n_shared:
         assert rel_err(np_(o["y_shared"])[:T], ef["y_shared"]) <= tol
     assert rel_err(np_(o["y"])[:T], ref["y"]) <= tol
@@ -214,9 +215,15 @@ def test_full_size(name):
     assert float(o["aux"]) == pytest.approx(ref["aux"], rel=1e-5)
     y, aux, cnt = run.layer()
     assert torch.equal(y, o["y"])
+    # a random sample fixes the rms; the 32 tokens with the largest outputs are added to the
+    # max, since the rounding errors grow with the magnitude of the summed rows
     rng = np.random.default_rng(123)
-    sample = np.unique(np.concatenate([[0, c.T - 1], rng.choice(c.T, 94, replace=False)]))
-    yg = np_(y)[sample]
-    yr = np.stack([oracle.token_output(c, inp, int(t), r["idx"][t], r["w"][t],
-                                       pm["slot_pos"][t] >= 0) for t in sample])
-    assert rel_err(yg, yr) <= tol_of(c)
+    rand = np.unique(np.concatenate([[0, c.T - 1], rng.choice(c.T, 126, replace=False)]))
+    yall = np_(y)
+    heavy = np.argsort(-np.abs(yall).max(axis=1))[:32]
+    sample = np.unique(np.concatenate([rand, heavy]))
+    yr = {int(t): oracle.token_output(c, inp, int(t), r["idx"][t], r["w"][t],
+                                      pm["slot_pos"][t] >= 0) for t in sample}
+    rms = np.sqrt(np.mean(np.stack([yr[int(t)] for t in rand]) ** 2))
+    err = max(float(np.max(np.abs(yall[t] - yr[int(t)]))) for t in sample)
+    assert err / rms <= tol_of(c), f"max|dy|/rms = {err / rms:.4f}" 
