@@ -329,7 +329,7 @@ moe_status_t launch_gemm(const moe_config_t *c, const GroupedGemm &g, int bn_hin
 
 template <typename Tin, int NT>
 moe_status_t launch_router_nt(const RouterArgs &a, cudaStream_t st) {
-  const size_t smem = router_smem(a.E, NT, a.score == MOE_SCORE_SIGMOID).total;
+  const size_t smem = router_smem(a.E, NT, a.score == MOE_SCORE_SIGMOID, a.d, (int)sizeof(Tin)).total;
   if (smem > 227 * 1024) return MOE_ERR_UNSUPPORTED;
   if (cudaFuncSetAttribute(router_kernel<Tin, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)smem) != cudaSuccess)

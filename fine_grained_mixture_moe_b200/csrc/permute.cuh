@@ -4,20 +4,21 @@
 //
 // Stable counting sort of the (token, slot) pairs by expert, with the capacity mask:
 //   rank(t, e) = #{t' < t : e in topk(t')};   kept iff rank < C;   row = offsets[e] + rank.
-// Tokens are cut into chunks of 8 (the router's CTA). Steps:
+// Tokens are cut into chunks of 16 (the router's CTA). Steps:
 //   hist    per-chunk expert histogram -> chunk_count[chunk][E] (inside the layer call the
 //           router's per-CTA counts already are this histogram, so it is only launched by
 //           moe_permute on its own)
 //   stats   per-expert exclusive scan over chunks -> chunk_base; offsets[E+1] (stats.cuh)
-//   scatter per-chunk ranks from a per-expert lane bitmask, slot_pos / src_token, then the
-//           CTA's eight warps copy the chunk's x rows to x_perm with 16-byte loads and stores.
+//   scatter per-chunk ranks from a per-expert lane bitmask, slot_pos / src_token, then
+//           PM_SPLIT CTAs of eight warps copy the chunk's x rows to x_perm with 16-byte loads
+//           and stores.
 #pragma once
 #include "common.cuh"
 
 namespace moe {
 
-constexpr int PM_CHUNK = 8;
-constexpr int PM_SPLIT = 2;  // CTAs per chunk in the scatter
+constexpr int PM_CHUNK = 16;
+constexpr int PM_SPLIT = 4;  // CTAs per chunk in the scatter
 
 __global__ void __launch_bounds__(256) perm_hist_kernel(const int32_t *__restrict__ idx, int T,
                                                         int k, int E,

@@ -25,8 +25,9 @@
 
 namespace moe {
 
-constexpr int RT_TM = 8;           // tokens per CTA (one fp64 MMA row tile)
-constexpr int RT_WARPS = 4;        // each a slice of the K dimension
+constexpr int RT_TM = 16;          // tokens per CTA
+constexpr int RT_MT = RT_TM / 8;   // fp64 MMA row tiles per warp (each W fragment feeds all)
+constexpr int RT_WARPS = 8;        // each a slice of the K dimension
 constexpr int RT_THREADS = 32 * RT_WARPS;
 constexpr int RT_KB = 16;          // k block: lane (row r, column c) of a fragment reads the 4
                                    // consecutive elements 4c..4c+3 of the block with one load
@@ -359,13 +360,18 @@ __device__ float sigmoid_key(float l, float b, bool force) {
 // ------------------------------------------------------------------ kernels
 // Shared-memory layout of the router kernel (byte offsets), shared by host and device.
 struct RouterSmem {
-  size_t part, sq, ex, lg, pb, keys, sel_e, sel_p, wn, wexp, cnt, flags, xnorm, xexp, fix, total;
+  size_t xs, xs_stride, part, sq, ex, lg, pb, keys, sel_e, sel_p, wn, wexp, cnt, flags, xnorm,
+      xexp, fix, total;
 };
-__host__ __device__ inline RouterSmem router_smem(int E, int NT, bool sigmoid) {
+__host__ __device__ inline RouterSmem router_smem(int E, int NT, bool sigmoid, int d, int esize) {
   RouterSmem L;
   const int EB = 8 * NT;
   size_t o = 0;
   auto take = [&](size_t bytes) { size_t at = o; o = (o + bytes + 15) & ~(size_t)15; return at; };
+  // the CTA's token rows, each padded by 32 bytes so that the 8 rows of an MMA fragment fall
+  // on distinct bank pairs
+  L.xs_stride = (size_t)d * esize + 32;
+  L.xs = take((size_t)RT_TM * L.xs_stride);
   L.part = take((size_t)RT_WARPS * RT_TM * EB * sizeof(double));   // per-warp partial sums
   L.sq = take((size_t)RT_WARPS * (EB + RT_TM) * sizeof(double));   // per-warp sums of squares
   L.ex = take((size_t)RT_WARPS * (EB + RT_TM) * 2 * sizeof(int));  // per-warp exponent ranges
@@ -387,57 +393,66 @@ __host__ __device__ inline RouterSmem router_smem(int E, int NT, bool sigmoid) {
 }
 
 // Raw 4-element fragment loads (bf16: 8 bytes; fp32: 16 bytes) and their conversion to fp64.
+// Fragment digest: the four raw elements a lane loads per 16-k block become (1) fp64 MMA
+// operands (a bf16 widens exactly to fp32 by a shift, then to fp64 by the conversion
+// instruction), (2) an fp32 running sum of squares for the norm bound, (3) the running min / max
+// magnitude key (the element's bits without the sign: key >> MANT is the biased exponent) over
+// the nonzero elements, for the exactness certificate.
 template <typename Tin> struct Frag4;
 template <> struct Frag4<__nv_bfloat16> {
   using raw_t = uint2;
-  static __device__ __forceinline__ raw_t load(const __nv_bfloat16 *p) { return __ldg((const uint2 *)p); }
-  static __device__ __forceinline__ raw_t zero() { return make_uint2(0u, 0u); }
-  static __device__ __forceinline__ void cvt(raw_t q, double (&v)[4]) {
-    const __nv_bfloat162 *h = (const __nv_bfloat162 *)&q;
-    const float2 f0 = __bfloat1622float2(h[0]), f1 = __bfloat1622float2(h[1]);
-    v[0] = f0.x; v[1] = f0.y; v[2] = f1.x; v[3] = f1.y;
-  }
   static constexpr int MANT = 7;  // fraction bits
-  // min / max biased exponent over the nonzero elements (subnormals count as exponent 0)
-  static __device__ __forceinline__ void exps(raw_t q, int &mn, int &mx) {
+  static __device__ __forceinline__ raw_t load(const __nv_bfloat16 *p) { return __ldg((const uint2 *)p); }
+  static __device__ __forceinline__ raw_t load_s(const __nv_bfloat16 *p) { return *(const uint2 *)p; }
+  static __device__ __forceinline__ raw_t zero() { return make_uint2(0u, 0u); }
+  static __device__ __forceinline__ void digest(raw_t q, double (&v)[4], float &sq, uint32_t &mn,
+                                                uint32_t &mx) {
     const uint32_t w[2] = {q.x, q.y};
 #pragma unroll
     for (int i = 0; i < 2; ++i)
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
-        const uint32_t b = (w[i] >> (16 * h)) & 0xFFFFu;
-        if (b & 0x7FFFu) {
-          const int e = (int)((b >> 7) & 0xFFu);
-          mn = min(mn, e);
-          mx = max(mx, e);
-        }
+        const uint32_t b = h ? (w[i] >> 16) : (w[i] & 0xFFFFu);
+        const uint32_t m = b & 0x7FFFu;
+        const float f = __uint_as_float(b << 16);
+        sq = fmaf(f, f, sq);
+        mn = min(mn, m ? m : 0xFFFFFFFFu);
+        mx = max(mx, m);
+        v[2 * i + h] = (double)f;
       }
   }
 };
 template <> struct Frag4<float> {
   using raw_t = float4;
-  static __device__ __forceinline__ raw_t load(const float *p) { return __ldg((const float4 *)p); }
-  static __device__ __forceinline__ raw_t zero() { return make_float4(0.f, 0.f, 0.f, 0.f); }
-  static __device__ __forceinline__ void cvt(raw_t q, double (&v)[4]) {
-    v[0] = q.x; v[1] = q.y; v[2] = q.z; v[3] = q.w;
-  }
   static constexpr int MANT = 23;
-  static __device__ __forceinline__ void exps(raw_t q, int &mn, int &mx) {
+  static __device__ __forceinline__ raw_t load(const float *p) { return __ldg((const float4 *)p); }
+  static __device__ __forceinline__ raw_t load_s(const float *p) { return *(const float4 *)p; }
+  static __device__ __forceinline__ raw_t zero() { return make_float4(0.f, 0.f, 0.f, 0.f); }
+  static __device__ __forceinline__ void digest(raw_t q, double (&v)[4], float &sq, uint32_t &mn,
+                                                uint32_t &mx) {
     const float f[4] = {q.x, q.y, q.z, q.w};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      const uint32_t b = __float_as_uint(f[i]);
-      if (b & 0x7FFFFFFFu) {
-        const int e = (int)((b >> 23) & 0xFFu);
-        mn = min(mn, e);
-        mx = max(mx, e);
-      }
+      v[i] = f[i];
+      sq = fmaf(f[i], f[i], sq);
+      const uint32_t m = __float_as_uint(f[i]) & 0x7FFFFFFFu;
+      mn = min(mn, m ? m : 0xFFFFFFFFu);
+      mx = max(mx, m);
     }
   }
 };
 
+// Upper bound on sqrt(sum of squares) from an fp32 accumulation of at most n = d + 16 fused
+// multiply-adds and additions: each step rounds with relative error <= 2^-24 or, in the
+// subnormal range, absolute error <= 2^-150, so the exact sum is at most
+// (computed + n 2^-149) (1 + n 2^-23) while n 2^-24 is small. Infinite or NaN input stays so.
+__device__ __forceinline__ double norm_upper(double computed, int d) {
+  const double n = (double)(d + 16);
+  return sqrt((computed + n * 0x1p-149) * (1.0 + n * 0x1p-23));
+}
+
 template <typename Tin, int NT>
-__global__ void __launch_bounds__(RT_THREADS, 4) router_kernel(RouterArgs a) {
+__global__ void __launch_bounds__(RT_THREADS, 2) router_kernel(RouterArgs a) {
   constexpr int EB = 8 * NT;  // experts per round
   using F = Frag4<Tin>;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -451,10 +466,10 @@ __global__ void __launch_bounds__(RT_THREADS, 4) router_kernel(RouterArgs a) {
   const int force_level = g_force_exact;
   const bool force = force_level != 0;
   const bool sigmoid = a.score == MOE_SCORE_SIGMOID;
-  const RouterSmem SL = router_smem(E, NT, sigmoid);
+  const RouterSmem SL = router_smem(E, NT, sigmoid, d, (int)sizeof(Tin));
   double *part = (double *)(smem_raw + SL.part);  // [RT_WARPS][RT_TM][EB]
   double *sq = (double *)(smem_raw + SL.sq);      // [RT_WARPS][EB + RT_TM]
-  int *exr = (int *)(smem_raw + SL.ex);            // [RT_WARPS][EB + RT_TM][min, max]
+  uint32_t *exr = (uint32_t *)(smem_raw + SL.ex);  // [RT_WARPS][EB + RT_TM][min, max] keys
   int *wexp = (int *)(smem_raw + SL.wexp);         // [EB][min, max] of the round's rows
   int *xexp = (int *)(smem_raw + SL.xexp);         // [RT_TM][min, max]
   float *lg = (float *)(smem_raw + SL.lg);
@@ -471,79 +486,119 @@ __global__ void __launch_bounds__(RT_THREADS, 4) router_kernel(RouterArgs a) {
   double *fix_s = (double *)(smem_raw + SL.fix);  // fp64 sums of the first RT_FIX_CAP flagged
   __shared__ int s_nfix;
 
+  // ---- the CTA's token rows -> shared memory: one bulk copy per row, all in flight at once
+  unsigned char *xs = smem_raw + SL.xs;
+  const size_t xs_stride = SL.xs_stride;
+  const uint32_t row_bytes = (uint32_t)d * (uint32_t)sizeof(Tin);
+  __shared__ __align__(8) uint64_t s_xbar;
+  __shared__ volatile int s_xabort;
+  const uint32_t xbar = smem_u32(&s_xbar);
+  if (tid == 0) {
+    mbar_init(xbar, 1);
+    s_xabort = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+  if (tid == 0) {
+    mbar_expect_tx(xbar, (uint32_t)ntok * row_bytes);
+    for (int r = 0; r < ntok; ++r)
+      bulk_load_1d(smem_u32(xs + (size_t)r * xs_stride), x + (size_t)(t0 + r) * d, row_bytes, xbar);
+  }
+  for (int r = ntok; r < RT_TM; ++r)  // rows past the last token read as zeros
+    for (uint32_t i = tid; i < row_bytes / 16; i += RT_THREADS)
+      ((uint4 *)(xs + (size_t)r * xs_stride))[i] = make_uint4(0u, 0u, 0u, 0u);
   for (int e = tid; e < E; e += RT_THREADS) cnt[e] = 0;
   for (int i = tid; i < RT_TM * nfw; i += RT_THREADS) flags[i] = 0u;
   if (tid == 0) s_nfix = 0;
   if (blockIdx.x == 0 && tid == 0) *a.counter = 0u;
+  mbar_wait(xbar, 0u, (volatile int *)&s_xabort, g_wait_limit_ns, INFO_WAIT_ROUTER_X);
+  __syncthreads();
+  if (s_xabort) {  // the copies did not land in time: error recorded; let them drain, then leave
+    if (tid == 0) {
+      volatile int never = 0;
+      mbar_wait(xbar, 0u, &never, g_wait_limit_ns, INFO_WAIT_DRAIN);
+    }
+    __syncthreads();
+    return;
+  }
 
   // ---- logits on the fp64 tensor cores, one round per 8*NT experts. Warp w takes the 16-k
-  // blocks w, w+4, ... of the d dimension. For a block, the lane at fragment (row r, column c)
-  // loads elements 4c..4c+3 of token row r and of expert row r of each column tile, straight
-  // from global memory (L1/L2), and MMA step i uses element 4c+i: a permutation of k inside the
-  // block, identical for both operands. Every element of the CTA's token rows and of the
+  // blocks w, w+RT_WARPS, ... of the d dimension. For a block, the lane at fragment (row r, column c)
+  // loads elements 4c..4c+3 of token rows r, r+8 (shared memory) and of expert row r of each
+  // column tile (global memory, L2), and MMA step i uses element 4c+i: a permutation of k inside
+  // the block, identical for both operands. Every element of the CTA's token rows and of the
   // round's expert rows is loaded exactly once per round, so the sums of squares of the loaded
-  // values give |x_t| and |W_e| for the rounding bound. The four per-warp partial sums are then
+  // values give |x_t| and |W_e| for the rounding bound. The per-warp partial sums are then
   // added in warp order.
   const int nkb = d / RT_KB;
-  const bool tok_ok = fr < ntok;
-  const Tin *xrow_f = x + (size_t)(t0 + (tok_ok ? fr : 0)) * d + 4 * fc;
+  const Tin *xs_f[RT_MT];
+#pragma unroll
+  for (int mt = 0; mt < RT_MT; ++mt) xs_f[mt] = (const Tin *)(xs + (size_t)(fr + 8 * mt) * xs_stride) + 4 * fc;
   for (int eb = 0; eb < E; eb += EB) {
-    double acc[NT][2], wsq[NT];
-    double xsq = 0.0;
-    int xmn = 255, xmx = -1, wmn[NT], wmx[NT];
+    double acc[RT_MT][NT][2];
+    float xsq[RT_MT], wsq[NT];
+    uint32_t xmn[RT_MT], xmx[RT_MT], wmn[NT], wmx[NT];
     const Tin *wrow_f[NT];
     bool e_ok[NT];
 #pragma unroll
+    for (int mt = 0; mt < RT_MT; ++mt) {
+      xsq[mt] = 0.0f;
+      xmn[mt] = 0xFFFFFFFFu;
+      xmx[mt] = 0u;
+#pragma unroll
+      for (int j = 0; j < NT; ++j) acc[mt][j][0] = acc[mt][j][1] = 0.0;
+    }
+#pragma unroll
     for (int j = 0; j < NT; ++j) {
-      acc[j][0] = acc[j][1] = 0.0;
-      wsq[j] = 0.0;
-      wmn[j] = 255;
-      wmx[j] = -1;
+      wsq[j] = 0.0f;
+      wmn[j] = 0xFFFFFFFFu;
+      wmx[j] = 0u;
       const int e = eb + 8 * j + fr;
       e_ok[j] = e < E;
       wrow_f[j] = wr + (size_t)(e_ok[j] ? e : 0) * d + 4 * fc;
     }
     // one-block-ahead prefetch of the raw fragments
-    typename F::raw_t ra = F::zero(), rb[NT];
+    typename F::raw_t ra[RT_MT], rb[NT];
+#pragma unroll
+    for (int mt = 0; mt < RT_MT; ++mt) ra[mt] = F::zero();
 #pragma unroll
     for (int j = 0; j < NT; ++j) rb[j] = F::zero();
     int kb = warp;
     if (kb < nkb) {
-      if (tok_ok) ra = F::load(xrow_f + kb * RT_KB);
+#pragma unroll
+      for (int mt = 0; mt < RT_MT; ++mt) ra[mt] = F::load_s(xs_f[mt] + kb * RT_KB);
 #pragma unroll
       for (int j = 0; j < NT; ++j) if (e_ok[j]) rb[j] = F::load(wrow_f[j] + kb * RT_KB);
     }
     for (; kb < nkb; kb += RT_WARPS) {
-      double av[4], bv[NT][4];
-      F::cvt(ra, av);
-      F::exps(ra, xmn, xmx);
+      double av[RT_MT][4], bv[NT][4];
 #pragma unroll
-      for (int j = 0; j < NT; ++j) {
-        F::cvt(rb[j], bv[j]);
-        F::exps(rb[j], wmn[j], wmx[j]);
-      }
+      for (int mt = 0; mt < RT_MT; ++mt) F::digest(ra[mt], av[mt], xsq[mt], xmn[mt], xmx[mt]);
+#pragma unroll
+      for (int j = 0; j < NT; ++j) F::digest(rb[j], bv[j], wsq[j], wmn[j], wmx[j]);
       const int kn = kb + RT_WARPS;
       if (kn < nkb) {
-        ra = tok_ok ? F::load(xrow_f + kn * RT_KB) : F::zero();
+#pragma unroll
+        for (int mt = 0; mt < RT_MT; ++mt) ra[mt] = F::load_s(xs_f[mt] + kn * RT_KB);
 #pragma unroll
         for (int j = 0; j < NT; ++j) rb[j] = e_ok[j] ? F::load(wrow_f[j] + kn * RT_KB) : F::zero();
       }
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        xsq = fma(av[i], av[i], xsq);
+      for (int i = 0; i < 4; ++i)
 #pragma unroll
-        for (int j = 0; j < NT; ++j) {
-          wsq[j] = fma(bv[j][i], bv[j][i], wsq[j]);
-          dmma_8x8x4(acc[j], av[i], bv[j][i]);
-        }
-      }
+        for (int j = 0; j < NT; ++j)
+#pragma unroll
+          for (int mt = 0; mt < RT_MT; ++mt) dmma_8x8x4(acc[mt][j], av[mt][i], bv[j][i]);
     }
     // per-warp row sums of squares (lanes of one fragment row differ in fc = lane bits 0-1)
 #pragma unroll
     for (int o = 1; o < 4; o <<= 1) {
-      xsq += __shfl_xor_sync(0xffffffffu, xsq, o);
-      xmn = min(xmn, __shfl_xor_sync(0xffffffffu, xmn, o));
-      xmx = max(xmx, __shfl_xor_sync(0xffffffffu, xmx, o));
+#pragma unroll
+      for (int mt = 0; mt < RT_MT; ++mt) {
+        xsq[mt] += __shfl_xor_sync(0xffffffffu, xsq[mt], o);
+        xmn[mt] = min(xmn[mt], __shfl_xor_sync(0xffffffffu, xmn[mt], o));
+        xmx[mt] = max(xmx[mt], __shfl_xor_sync(0xffffffffu, xmx[mt], o));
+      }
 #pragma unroll
       for (int j = 0; j < NT; ++j) {
         wsq[j] += __shfl_xor_sync(0xffffffffu, wsq[j], o);
@@ -558,32 +613,40 @@ __global__ void __launch_bounds__(RT_THREADS, 4) router_kernel(RouterArgs a) {
         exr[2 * (warp * (EB + RT_TM) + 8 * j + fr)] = wmn[j];
         exr[2 * (warp * (EB + RT_TM) + 8 * j + fr) + 1] = wmx[j];
       }
-      sq[warp * (EB + RT_TM) + EB + fr] = xsq;
-      exr[2 * (warp * (EB + RT_TM) + EB + fr)] = xmn;
-      exr[2 * (warp * (EB + RT_TM) + EB + fr) + 1] = xmx;
+#pragma unroll
+      for (int mt = 0; mt < RT_MT; ++mt) {
+        sq[warp * (EB + RT_TM) + EB + fr + 8 * mt] = xsq[mt];
+        exr[2 * (warp * (EB + RT_TM) + EB + fr + 8 * mt)] = xmn[mt];
+        exr[2 * (warp * (EB + RT_TM) + EB + fr + 8 * mt) + 1] = xmx[mt];
+      }
     }
 #pragma unroll
-    for (int j = 0; j < NT; ++j)
+    for (int mt = 0; mt < RT_MT; ++mt)
 #pragma unroll
-      for (int h = 0; h < 2; ++h) part[(warp * RT_TM + fr) * EB + 8 * j + 2 * fc + h] = acc[j][h];
+      for (int j = 0; j < NT; ++j)
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+          part[(warp * RT_TM + fr + 8 * mt) * EB + 8 * j + 2 * fc + h] = acc[mt][j][h];
     __syncthreads();
     for (int q = tid; q < EB + RT_TM; q += RT_THREADS) {
       double t = 0.0;
-      int mn = 255, mx = -1;
+      uint32_t mn = 0xFFFFFFFFu, mx = 0u;
 #pragma unroll
       for (int w = 0; w < RT_WARPS; ++w) {
         t += sq[w * (EB + RT_TM) + q];
         mn = min(mn, exr[2 * (w * (EB + RT_TM) + q)]);
         mx = max(mx, exr[2 * (w * (EB + RT_TM) + q) + 1]);
       }
+      // biased exponents of the smallest and largest nonzero magnitude; (255, -1): all zero
+      const int emn = mx ? (int)(mn >> F::MANT) : 255, emx = mx ? (int)(mx >> F::MANT) : -1;
       if (q < EB) {
-        wn[q] = sqrt(t);
-        wexp[2 * q] = mn;
-        wexp[2 * q + 1] = mx;
+        wn[q] = norm_upper(t, d);
+        wexp[2 * q] = emn;
+        wexp[2 * q + 1] = emx;
       } else if (eb == 0) {
-        xnorm[q - EB] = sqrt(t);
-        xexp[2 * (q - EB)] = mn;
-        xexp[2 * (q - EB) + 1] = mx;
+        xnorm[q - EB] = norm_upper(t, d);
+        xexp[2 * (q - EB)] = emn;
+        xexp[2 * (q - EB) + 1] = emx;
       }
     }
     __syncthreads();
@@ -601,8 +664,9 @@ __global__ void __launch_bounds__(RT_THREADS, 4) router_kernel(RouterArgs a) {
         // Exactness certificate. With biased exponents of at least xmin and wmin (all normal),
         // every product is an integer multiple of 2^qq, qq = xmin + wmin - 254 - 2 MANT, and so is
         // the offset when its own quantum is folded in. Every partial sum, in any order, is
-        // bounded by sum |x_i W_i| + |off| <= |x|_2 |W_e|_2 + |off| (Cauchy-Schwarz); the computed
-        // norms are within (d + 8) 2^-50 of that relatively. Below 2^(qq + 53) every partial sum
+        // bounded by sum |x_i W_i| + |off| <= |x|_2 |W_e|_2 + |off| (Cauchy-Schwarz); xnorm and wn
+        // are upper bounds of the norms and the factor covers this line's own rounding. Below
+        // 2^(qq + 53) every partial sum
         // is an fp64 value, so s is the exact sum and its round-to-nearest-even to fp32 is the
         // canonical logit, exact ties included.
         bool exact;
@@ -680,31 +744,41 @@ __global__ void __launch_bounds__(RT_THREADS, 4) router_kernel(RouterArgs a) {
       for (int q = tid; q < ntok * E; q += RT_THREADS)
         keys[q] = sigmoid_key(lg[q], a.bias ? a.bias[q % E] : 0.0f, force);
     __syncthreads();
+    // the token's max logit and normaliser, once per token (one warp per token, fixed order)
+    __shared__ float s_tok_m[RT_TM], s_tok_inv[RT_TM];
+    for (int tt = warp; tt < ntok; tt += RT_THREADS / 32) {
+      const float *lrow = lg + tt * E;
+      float m = -INFINITY;
+      for (int e = lane; e < E; e += 32) m = fmaxf(m, lrow[e]);
+      m = warp_max_f(m);
+      float ssum = 0.0f;
+      if (!sigmoid)
+        for (int e = lane; e < E; e += 32) ssum += expf(lrow[e] - m);
+      else
+        for (int e = lane; e < E; e += 32) ssum += 1.0f / (1.0f + expf(-lrow[e]));
+      ssum = warp_sum_f(ssum);
+      if (lane == 0) {
+        s_tok_m[tt] = m;
+        s_tok_inv[tt] = 1.0f / ssum;
+      }
+    }
+    __syncthreads();
     for (int q = tid; q < ntok * E; q += RT_THREADS) {
       const int tt = q / E, e = q - tt * E;
       const float *krow = (sigmoid ? keys : lg) + tt * E;
-      const float *lrow = lg + tt * E;
       float v = krow[e];
       if (v != v) v = -INFINITY;
       int rank = 0;
-      float m = -INFINITY;
       for (int e2 = 0; e2 < E; ++e2) {
         float v2 = krow[e2];
         if (v2 != v2) v2 = -INFINITY;
         rank += (v2 > v || (v2 == v && e2 < e)) ? 1 : 0;
-        m = fmaxf(m, lrow[e2]);
       }
-      // the token's normaliser, summed in expert order by each of its threads alike
-      float ssum = 0.0f;
-      if (!sigmoid)
-        for (int e2 = 0; e2 < E; ++e2) ssum += expf(lrow[e2] - m);
-      else
-        for (int e2 = 0; e2 < E; ++e2) ssum += 1.0f / (1.0f + expf(-lrow[e2]));
-      const float inv = 1.0f / ssum;
-      const float l = lrow[e];
+      const float inv = s_tok_inv[tt];
+      const float l = lg[tt * E + e];
       float p, pbasis;
       if (!sigmoid) {
-        p = expf(l - m) * inv;
+        p = expf(l - s_tok_m[tt]) * inv;
         pbasis = p;
       } else {
         p = 1.0f / (1.0f + expf(-l));

@@ -6,7 +6,7 @@
 //   aux               = alpha * E * sum_e (count_e / (T k)) * (prob_sum_e / T)
 // One block per expert does the first three; the block that finishes last does the scan over
 // experts and the loss (Moonfrost expert card: routing under a per-expert capacity over stacked experts;
-// Quartz: load-balancing loss with weight 0.01). Chunks are RT_TM = 8 tokens, the router's CTA,
+// Quartz: load-balancing loss with weight 0.01). Chunks are RT_TM tokens, the router's CTA,
 // so the router's per-CTA counts are the permutation's histogram. Every sum has a fixed order.
 #pragma once
 #include "common.cuh"

@@ -166,7 +166,7 @@ moe_status_t moe_layer_forward(const moe_config_t *cfg, const void *x, const moe
  * in a fixed array of MOE_ROUTE_NOALLOC_SCRATCH_BYTES in the library's own device memory, which
  * every GPU that loads the library holds until the process exits. The caller still passes x,
  * the weights and all outputs.
- *   - Limit: the scratch needed is about 8*E*ceil(T/8) bytes; configurations that need
+ *   - Limit: the scratch needed is about 8*E*ceil(T/16) bytes; configurations that need
  *     more than MOE_ROUTE_NOALLOC_SCRATCH_BYTES return MOE_ERR_WORKSPACE with nothing enqueued.
  *   - Set-up: the first call on each device looks up the array's device address (with that
  *     device current); make that first call before any stream capture begins.
