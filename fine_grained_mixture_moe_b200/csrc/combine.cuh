@@ -45,15 +45,17 @@ template <> struct YVec<__nv_bfloat16> {
   }
 };
 
-// One warp per token; each lane owns N consecutive columns per vector and two vectors per pass,
-// with every load of a pass issued before the sums. d is a multiple of 64, so a lane's vector is
-// wholly inside or wholly outside the row.
+// One warp per token; each lane owns one 16-byte vector of expert outputs (N columns) per pass,
+// with the pass's k row loads and the shared-output load issued before the sums. About 60
+// registers, so 4 CTAs (32 warps) fit per SM and a Quartz-sized call is one wave. d is a
+// multiple of 64, so a lane's vector is wholly inside or wholly outside the row.
 template <typename Ty>
-__global__ void __launch_bounds__(256) combine_kernel(const Ty *__restrict__ y_perm,
-                                                      const float *__restrict__ y_shared,
-                                                      const int32_t *__restrict__ slot_pos,
-                                                      const float *__restrict__ w,
-                                                      float *__restrict__ y, int T, int k, int d) {
+__global__ void __launch_bounds__(256, sizeof(Ty) == 2 ? 4 : 3) combine_kernel(const Ty *__restrict__ y_perm,
+                                                         const float *__restrict__ y_shared,
+                                                         const int32_t *__restrict__ slot_pos,
+                                                         const float *__restrict__ w,
+                                                         float *__restrict__ y, int T, int k,
+                                                         int d) {
   using YV = YVec<Ty>;
   constexpr int V = YV::N;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -73,40 +75,28 @@ __global__ void __launch_bounds__(256) combine_kernel(const Ty *__restrict__ y_p
     wj[j] = __shfl_sync(0xffffffffu, w_l, j);
   }
 #pragma unroll 1
-  for (int c0 = lane * V; c0 < d; c0 += 64 * V) {
-    float acc[2][V];
-    typename YV::raw_t v[2][8];
+  for (int c = lane * V; c < d; c += 32 * V) {
+    float acc[V];
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const int c = c0 + h * 32 * V;
-      if (c < d) {
-#pragma unroll
-        for (int i = 0; i < V; i += 4) {
-          float4 q = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-          if (y_shared) q = __ldcs((const float4 *)(y_shared + (size_t)t * d + c + i));
-          acc[h][i] = q.x;
-          acc[h][i + 1] = q.y;
-          acc[h][i + 2] = q.z;
-          acc[h][i + 3] = q.w;
-        }
-#pragma unroll
-        for (int j = 0; j < 8; ++j)
-          if (j < k && pos[j] >= 0) v[h][j] = YV::load(y_perm + (size_t)pos[j] * d + c);
-      }
+    for (int i = 0; i < V; i += 4) {
+      float4 q = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+      if (y_shared) q = __ldcs((const float4 *)(y_shared + (size_t)t * d + c + i));
+      acc[i] = q.x;
+      acc[i + 1] = q.y;
+      acc[i + 2] = q.z;
+      acc[i + 3] = q.w;
     }
+    typename YV::raw_t v[8];
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const int c = c0 + h * 32 * V;
-      if (c < d) {
+    for (int j = 0; j < 8; ++j)
+      if (j < k && pos[j] >= 0) v[j] = YV::load(y_perm + (size_t)pos[j] * d + c);
 #pragma unroll
-        for (int j = 0; j < 8; ++j)
-          if (j < k && pos[j] >= 0) YV::fma(wj[j], v[h][j], acc[h]);
+    for (int j = 0; j < 8; ++j)
+      if (j < k && pos[j] >= 0) YV::fma(wj[j], v[j], acc);
 #pragma unroll
-        for (int i = 0; i < V; i += 4)
-          __stcs((float4 *)(y + (size_t)t * d + c + i),
-                 make_float4(acc[h][i], acc[h][i + 1], acc[h][i + 2], acc[h][i + 3]));
-      }
-    }
+    for (int i = 0; i < V; i += 4)
+      __stcs((float4 *)(y + (size_t)t * d + c + i),
+             make_float4(acc[i], acc[i + 1], acc[i + 2], acc[i + 3]));
   }
 }
 

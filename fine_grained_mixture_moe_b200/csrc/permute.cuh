@@ -9,9 +9,9 @@
 //           router's per-CTA counts already are this histogram, so it is only launched by
 //           moe_permute on its own)
 //   stats   per-expert exclusive scan over chunks -> chunk_base; offsets[E+1] (stats.cuh)
-//   scatter per-chunk ranks from a per-expert lane bitmask, slot_pos / src_token, then
-//           PM_SPLIT CTAs of eight warps copy the chunk's x rows to x_perm with 16-byte loads
-//           and stores.
+//   scatter per-chunk ranks from a per-expert lane bitmask, slot_pos / src_token; PM_SPLIT
+//           CTAs per chunk each copy 4 of its x rows to their k destinations in x_perm with
+//           16-byte loads and stores (each row read once).
 #pragma once
 #include "common.cuh"
 
@@ -44,6 +44,15 @@ __global__ void __launch_bounds__(256) perm_hist_kernel(const int32_t *__restric
   for (int e = lane; e < E; e += 32) chunk_count[(size_t)chunk * E + e] = c[e];
 }
 
+// Scatter. CTA (chunk, part) owns tokens chunk*16 + part*TPC .. +TPC (TPC = 16 / PM_SPLIT): two
+// warps per token, one half of the row each. Each warp loads its half-row into registers first
+// (these loads do not depend on the routing, so they overlap the index work), warp 0 meanwhile
+// ranks the chunk's (token, slot) pairs, and after one barrier every warp stores its half-row to
+// the token's kept destinations: x is read once and written k times.
+constexpr int PM_TPC = PM_CHUNK / PM_SPLIT;        // tokens per scatter CTA
+constexpr int PM_VMAX = 4;                          // 16-byte vectors per lane held at once
+static_assert(PM_TPC * 2 == 8, "two warps per token, eight warps per CTA");
+
 template <typename Tin>
 __global__ void __launch_bounds__(256) perm_scatter_kernel(
     const int32_t *__restrict__ idx, int T, int k, int E, int C,
@@ -52,12 +61,28 @@ __global__ void __launch_bounds__(256) perm_scatter_kernel(
     Tin *__restrict__ x_perm, int d) {
   extern __shared__ unsigned smask[];  // [E]
   __shared__ int s_pos[PM_CHUNK * 8];
-  __shared__ int s_tok[PM_CHUNK * 8];
   const bool active = (threadIdx.x & 31) < PM_CHUNK;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int chunk = blockIdx.x / PM_SPLIT, part = blockIdx.x % PM_SPLIT;
-  const int t = chunk * PM_CHUNK + lane;
+  // this warp's token and half-row
+  const int tl = part * PM_TPC + (warp >> 1);  // token within the chunk
+  const int tw = chunk * PM_CHUNK + tl;
+  const int nvec = d * (int)sizeof(Tin) / 16;   // 16-byte vectors per row
+  const int hv = (nvec + 1) / 2;
+  const int vbeg = (warp & 1) * hv, vend = min(nvec, vbeg + hv);
+  const uint4 *srow = (const uint4 *)(x + (size_t)(tw < T ? tw : 0) * d);
+  const bool copy = x_perm != nullptr && tw < T;
+  uint4 held[PM_VMAX];
+  int v0 = vbeg;
+  if (copy) {
+#pragma unroll
+    for (int i = 0; i < PM_VMAX; ++i) {
+      const int v = v0 + lane + 32 * i;
+      if (v < vend) held[i] = __ldg(srow + v);
+    }
+  }
   if (warp == 0) {
+    const int t = chunk * PM_CHUNK + lane;
     for (int e = lane; e < E; e += 32) smask[e] = 0u;
     __syncwarp();
     const bool valid = active && t < T;
@@ -88,25 +113,31 @@ __global__ void __launch_bounds__(256) perm_scatter_kernel(
             if (pos >= 0) src[pos] = t;
           }
         }
-        if (active) {
-          s_pos[lane * k + j] = pos;
-          s_tok[lane * k + j] = t;
-        }
+        if (active) s_pos[lane * k + j] = pos;
       }
     }
   }
   __syncthreads();
-  if (x_perm == nullptr) return;
-  // the chunk's rows are shared by PM_SPLIT CTAs (slots part, part + PM_SPLIT, ...), so more
-  // copies are in flight per SM than 16-token chunks alone would give
-  const int nvec = d * (int)sizeof(Tin) / 16;
-  for (int s = part + PM_SPLIT * warp; s < PM_CHUNK * k; s += PM_SPLIT * 8) {
-    const int pos = s_pos[s];
-    if (pos < 0) continue;
-    const uint4 *srow = (const uint4 *)(x + (size_t)s_tok[s] * d);
-    uint4 *drow = (uint4 *)(x_perm + (size_t)pos * d);
-#pragma unroll 4
-    for (int v = lane; v < nvec; v += 32) drow[v] = __ldg(srow + v);
+  if (!copy) return;
+  for (;;) {
+    for (int j = 0; j < k; ++j) {
+      const int pos = s_pos[tl * k + j];
+      if (pos < 0) continue;
+      uint4 *drow = (uint4 *)(x_perm + (size_t)pos * d);
+#pragma unroll
+      for (int i = 0; i < PM_VMAX; ++i) {
+        const int v = v0 + lane + 32 * i;
+        if (v < vend) drow[v] = held[i];
+      }
+    }
+    // rows longer than 2 * 32 * PM_VMAX vectors: the next slice of the half-row
+    v0 += 32 * PM_VMAX;
+    if (v0 >= vend) break;
+#pragma unroll
+    for (int i = 0; i < PM_VMAX; ++i) {
+      const int v = v0 + lane + 32 * i;
+      if (v < vend) held[i] = __ldg(srow + v);
+    }
   }
 }
 
