@@ -56,6 +56,8 @@ __global__ void __launch_bounds__(256, sizeof(Ty) == 2 ? 4 : 3) combine_kernel(c
                                                          const float *__restrict__ w,
                                                          float *__restrict__ y, int T, int k,
                                                          int d) {
+  griddep_wait();
+  griddep_launch();
   using YV = YVec<Ty>;
   constexpr int V = YV::N;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -102,6 +104,8 @@ __global__ void __launch_bounds__(256, sizeof(Ty) == 2 ? 4 : 3) combine_kernel(c
 
 __global__ void aux_loss_kernel(const int32_t *__restrict__ count, const float *__restrict__ prob,
                                 int E, int T, int k, float alpha, float *__restrict__ loss) {
+  griddep_wait();
+  griddep_launch();
   double s = 0.0;
   for (int e = threadIdx.x; e < E; e += 32) s += (double)count[e] * (double)prob[e];
   s = warp_sum_d(s);

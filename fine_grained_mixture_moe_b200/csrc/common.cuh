@@ -115,6 +115,18 @@ __device__ int block_excl_scan_inplace(int *a, int n, int *tmp) {
   return total;
 }
 
+// ---------------------------------------------------------------- programmatic dependent launch
+// The library launches its kernels with programmatic stream serialisation: a kernel may be
+// scheduled while the previous kernel of the stream is still finishing. griddep_wait() returns
+// once that kernel has completed and its memory operations are visible; every kernel calls it
+// before its first access to global memory that an earlier kernel may write or read (set-up of
+// shared memory, barriers and TMEM may precede it). griddep_launch() allows the next kernel to
+// be scheduled. Both are no-ops for a kernel launched without the attribute.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---------------------------------------------------------------- mbarriers (shared memory)
 // 1-D bulk copy global -> this CTA's shared memory, counted on an mbarrier (complete_tx).
 // dst, src 16-byte aligned; bytes a multiple of 16.

@@ -195,6 +195,27 @@ moe_status_t last_launch_status() {
   return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
+// Every layer kernel is launched with programmatic stream serialisation, so its CTAs may be
+// scheduled (and set up shared memory, barriers and TMEM) while the previous kernel finishes;
+// each kernel's griddep_wait() orders its memory accesses after that kernel (common.cuh).
+template <typename... KArgs, typename... Args>
+moe_status_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                        cudaStream_t st, Args... args) {
+  cudaLaunchConfig_t cfg;
+  std::memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+  return e == cudaSuccess ? last_launch_status() : MOE_ERR_CUDA;
+}
+
 // ------------------------------------------------------------------ tensor maps
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
@@ -269,8 +290,7 @@ moe_status_t launch_tc(const GroupedGemm &g, cudaStream_t st, int kind) {
   if (bound == 0) return MOE_OK;
   const int grid = (int)std::min<long long>(num_sms(), bound);
   ProfScope ps(kind, st);
-  kern<<<grid, TC_THREADS, smem, st>>>(P);
-  return last_launch_status();
+  return launch_pdl(kern, dim3(grid), dim3(TC_THREADS), smem, st, P);
 }
 
 // CTA-pair form (two SMs per 256-row tile); each CTA loads 128-row halves of A and B.
@@ -290,8 +310,7 @@ moe_status_t launch_tc2(const GroupedGemm &g, cudaStream_t st, int kind) {
   if (bound == 0) return MOE_OK;
   const int pairs = (int)std::min<long long>(num_sms() / 2, bound);
   ProfScope ps(kind, st);
-  kern<<<2 * pairs, TC_THREADS, smem, st>>>(P);
-  return last_launch_status();
+  return launch_pdl(kern, dim3(2 * pairs), dim3(TC_THREADS), smem, st, P);
 }
 
 template <int MODE>
@@ -306,8 +325,7 @@ moe_status_t launch_simt(const GroupedGemm &g, cudaStream_t st, int kind) {
   if (bound == 0) return MOE_OK;
   const int grid = (int)std::min<long long>((long long)num_sms() * 8, bound);
   ProfScope ps(kind, st);
-  kern<<<grid, 256, smem, st>>>(g);
-  return last_launch_status();
+  return launch_pdl(kern, dim3(grid), dim3(256), smem, st, g);
 }
 
 template <int MODE>
@@ -334,8 +352,7 @@ moe_status_t launch_router_nt(const RouterArgs &a, cudaStream_t st) {
   if (cudaFuncSetAttribute(router_kernel<Tin, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)smem) != cudaSuccess)
     return MOE_ERR_CUDA;
-  router_kernel<Tin, NT><<<ceil_div(a.T, RT_TM), RT_THREADS, smem, st>>>(a);
-  return last_launch_status();
+  return launch_pdl(router_kernel<Tin, NT>, dim3(ceil_div(a.T, RT_TM)), dim3(RT_THREADS), smem, st, a);
 }
 
 template <typename Tin>
@@ -351,8 +368,7 @@ moe_status_t launch_router(const RouterArgs &a, cudaStream_t st) {
 
 moe_status_t launch_stats(const StatsArgs &sa, cudaStream_t st) {
   ProfScope ps(K_STATS, st);
-  moe_stats_kernel<<<sa.E, ST_THREADS, 0, st>>>(sa);
-  return last_launch_status();
+  return launch_pdl(moe_stats_kernel, dim3(sa.E), dim3(ST_THREADS), 0, st, sa);
 }
 
 template <typename Tin>
@@ -411,10 +427,9 @@ moe_status_t scatter_impl(const moe_config_t *c, const void *x, const int32_t *i
                           const int32_t *chunk_base, const int32_t *offsets, int32_t *slot_pos,
                           int32_t *src, void *x_perm, cudaStream_t st) {
   ProfScope ps(K_PERM_SCATTER, st);
-  perm_scatter_kernel<Tin><<<ceil_div(c->T, PM_CHUNK) * PM_SPLIT, 256, (size_t)c->E * 4, st>>>(
-      idx, c->T, c->top_k, c->E, capacity_of(c), chunk_base, offsets, slot_pos, src,
-      (const Tin *)x, (Tin *)x_perm, c->d);
-  return last_launch_status();
+  return launch_pdl(perm_scatter_kernel<Tin>, dim3(ceil_div(c->T, PM_CHUNK) * PM_SPLIT), dim3(256),
+                    (size_t)c->E * 4, st, idx, c->T, c->top_k, c->E, capacity_of(c), chunk_base,
+                    offsets, slot_pos, src, (const Tin *)x, (Tin *)x_perm, c->d);
 }
 
 template <typename Tin>
@@ -433,8 +448,8 @@ moe_status_t permute_impl(const moe_config_t *c, const void *x, const int32_t *i
     if (cudaFuncSetAttribute(perm_hist_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
       return MOE_ERR_CUDA;
     ProfScope ps(K_PERM_HIST, st);
-    perm_hist_kernel<<<ceil_div(nch, 8), 256, smem, st>>>(idx, c->T, c->top_k, c->E, cc, nch, ctr);
-    MOE_TRY(last_launch_status());
+    MOE_TRY(launch_pdl(perm_hist_kernel, dim3(ceil_div(nch, 8)), dim3(256), smem, st, idx, c->T,
+                       c->top_k, c->E, cc, nch, ctr));
   }
   StatsArgs sa = stats_args(c, cc, nullptr, ctr);
   sa.chunk_base = cb;
@@ -518,19 +533,18 @@ moe_status_t combine_impl(const moe_config_t *c, const void *y_perm, const void 
   ProfScope ps(K_COMBINE, st);
   const float *ysh = c->n_shared > 0 ? (const float *)y_shared : nullptr;
   if (yperm_bf16(c))
-    combine_kernel<__nv_bfloat16><<<ceil_div(c->T, 8), 256, 0, st>>>(
-        (const __nv_bfloat16 *)y_perm, ysh, slot_pos, wts, (float *)y, c->T, c->top_k, c->d);
-  else
-    combine_kernel<float><<<ceil_div(c->T, 8), 256, 0, st>>>(
-        (const float *)y_perm, ysh, slot_pos, wts, (float *)y, c->T, c->top_k, c->d);
-  return last_launch_status();
+    return launch_pdl(combine_kernel<__nv_bfloat16>, dim3(ceil_div(c->T, 8)), dim3(256), 0, st,
+                      (const __nv_bfloat16 *)y_perm, ysh, slot_pos, wts, (float *)y, c->T,
+                      c->top_k, c->d);
+  return launch_pdl(combine_kernel<float>, dim3(ceil_div(c->T, 8)), dim3(256), 0, st,
+                    (const float *)y_perm, ysh, slot_pos, wts, (float *)y, c->T, c->top_k, c->d);
 }
 
 moe_status_t aux_impl(const moe_config_t *c, const int32_t *count, const float *prob, float *loss,
                       cudaStream_t st) {
   ProfScope ps(K_AUX, st);
-  aux_loss_kernel<<<1, 32, 0, st>>>(count, prob, c->E, c->T, c->top_k, c->aux_alpha, loss);
-  return last_launch_status();
+  return launch_pdl(aux_loss_kernel, dim3(1), dim3(32), 0, st, count, prob, c->E, c->T, c->top_k,
+                    c->aux_alpha, loss);
 }
 
 // ------------------------------------------------------------------ argument checks

@@ -24,6 +24,8 @@ __global__ void __launch_bounds__(256) perm_hist_kernel(const int32_t *__restric
                                                         int k, int E,
                                                         int32_t *__restrict__ chunk_count,
                                                         int nchunks, unsigned *stats_counter) {
+  griddep_wait();
+  griddep_launch();
   extern __shared__ int sh_cnt[];  // [8][E]
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   int *c = sh_cnt + warp * E;
@@ -59,6 +61,8 @@ __global__ void __launch_bounds__(256) perm_scatter_kernel(
     const int32_t *__restrict__ chunk_base, const int32_t *__restrict__ offsets,
     int32_t *__restrict__ slot_pos, int32_t *__restrict__ src, const Tin *__restrict__ x,
     Tin *__restrict__ x_perm, int d) {
+  griddep_wait();
+  griddep_launch();
   extern __shared__ unsigned smask[];  // [E]
   __shared__ int s_pos[PM_CHUNK * 8];
   const bool active = (threadIdx.x & 31) < PM_CHUNK;

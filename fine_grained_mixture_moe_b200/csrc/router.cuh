@@ -486,6 +486,8 @@ __global__ void __launch_bounds__(RT_THREADS, 2) router_kernel(RouterArgs a) {
   double *fix_s = (double *)(smem_raw + SL.fix);  // fp64 sums of the first RT_FIX_CAP flagged
   __shared__ int s_nfix;
 
+  griddep_wait();
+  griddep_launch();
   // ---- the CTA's token rows -> shared memory: one bulk copy per row, all in flight at once
   unsigned char *xs = smem_raw + SL.xs;
   const size_t xs_stride = SL.xs_stride;

@@ -30,6 +30,8 @@ struct StatsArgs {
 };
 
 __global__ void __launch_bounds__(ST_THREADS) moe_stats_kernel(StatsArgs a) {
+  griddep_wait();
+  griddep_launch();
   const int e = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int E = a.E;
   __shared__ int s_wc[ST_THREADS / 32 + 1];
