@@ -36,56 +36,44 @@ __global__ void __launch_bounds__(ST_THREADS) moe_stats_kernel(StatsArgs a) {
   const int E = a.E;
   __shared__ int s_wc[ST_THREADS / 32 + 1];
   __shared__ float s_wp[ST_THREADS / 32];
-  __shared__ int s_run;
-  // totals: thread t adds chunks t, t+256, ... then a fixed tree
-  int c = 0;
+  // One pass over the chunks, ST_THREADS at a time: the exclusive scan in chunk order gives
+  // chunk_base and the count total; thread t adds the probability sums of chunks t, t+256, ...
+  int run = 0;
   float p = 0.0f;
-  for (int b = tid; b < a.nchunk; b += ST_THREADS) {
-    c += a.chunk_cnt[(size_t)b * E + e];
-    if (a.chunk_prob) p += a.chunk_prob[(size_t)b * E + e];
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    c += __shfl_xor_sync(0xffffffffu, c, o);
-    p += __shfl_xor_sync(0xffffffffu, p, o);
-  }
-  if (lane == 0) { s_wc[warp] = c; s_wp[warp] = p; }
-  __syncthreads();
-  int total = 0;
-  float psum = 0.0f;
-#pragma unroll
-  for (int w = 0; w < ST_THREADS / 32; ++w) { total += s_wc[w]; psum += s_wp[w]; }
-  if (tid == 0) {
-    if (a.count_out) a.count_out[e] = total;
-    if (a.prob_out) a.prob_out[e] = psum;
-    if (a.kept) a.kept[e] = a.C < 0 ? total : min(total, a.C);
-  }
-  // exclusive scan over chunks, 256 chunks per pass
-  if (a.chunk_base) {
-    if (tid == 0) s_run = 0;
+  for (int b0 = 0; b0 < a.nchunk; b0 += ST_THREADS) {
+    const int b = b0 + tid;
+    const int v = b < a.nchunk ? a.chunk_cnt[(size_t)b * E + e] : 0;
+    if (a.chunk_prob && b < a.nchunk) p += a.chunk_prob[(size_t)b * E + e];
+    const int incl = warp_incl_scan(v);
+    if (lane == 31) s_wc[warp] = incl;
     __syncthreads();
-    for (int b0 = 0; b0 < a.nchunk; b0 += ST_THREADS) {
-      const int b = b0 + tid;
-      const int v = b < a.nchunk ? a.chunk_cnt[(size_t)b * E + e] : 0;
-      const int incl = warp_incl_scan(v);
-      __syncthreads();
-      if (lane == 31) s_wc[warp] = incl;
-      __syncthreads();
-      if (warp == 0) {
-        const int wv = lane < ST_THREADS / 32 ? s_wc[lane] : 0;
-        const int wi = warp_incl_scan(wv);
-        if (lane < ST_THREADS / 32) s_wc[lane] = wi - wv;
-        if (lane == ST_THREADS / 32 - 1) s_wc[ST_THREADS / 32] = wi;
-      }
-      __syncthreads();
-      if (b < a.nchunk) a.chunk_base[(size_t)b * E + e] = s_run + s_wc[warp] + incl - v;
-      __syncthreads();
-      if (tid == 0) s_run += s_wc[ST_THREADS / 32];
-      __syncthreads();
+    if (warp == 0) {
+      const int wv = lane < ST_THREADS / 32 ? s_wc[lane] : 0;
+      const int wi = warp_incl_scan(wv);
+      if (lane < ST_THREADS / 32) s_wc[lane] = wi - wv;
+      if (lane == ST_THREADS / 32 - 1) s_wc[ST_THREADS / 32] = wi;
     }
+    __syncthreads();
+    if (a.chunk_base && b < a.nchunk) a.chunk_base[(size_t)b * E + e] = run + s_wc[warp] + incl - v;
+    run += s_wc[ST_THREADS / 32];
+    __syncthreads();
+  }
+  // probability total in a fixed tree: lanes, then warps in order
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) p += __shfl_xor_sync(0xffffffffu, p, o);
+  if (lane == 0) s_wp[warp] = p;
+  __syncthreads();
+  if (tid == 0) {
+    float psum = 0.0f;
+#pragma unroll
+    for (int w = 0; w < ST_THREADS / 32; ++w) psum += s_wp[w];
+    if (a.count_out) a.count_out[e] = run;
+    if (a.prob_out) a.prob_out[e] = psum;
+    if (a.kept) a.kept[e] = a.C < 0 ? run : min(run, a.C);
   }
   if (!a.offsets && !a.aux) return;
-  // the last block to finish scans the kept counts over experts and forms the loss
+  // the last block to finish scans the kept counts over experts and forms the loss; all of its
+  // loads are issued together
   __threadfence();
   __syncthreads();
   __shared__ int s_last;
@@ -93,18 +81,19 @@ __global__ void __launch_bounds__(ST_THREADS) moe_stats_kernel(StatsArgs a) {
   __syncthreads();
   if (!s_last) return;
   __threadfence();
+  __shared__ int s_scan[1024 + ST_THREADS / 32 + 1];
+  double s = 0.0;
+  for (int i = tid; i < E; i += ST_THREADS) {
+    if (a.offsets) s_scan[i] = __ldcg(a.kept + i);
+    if (a.aux) s += (double)__ldcg(a.count_out + i) * (double)__ldcg(a.prob_out + i);
+  }
+  __syncthreads();
   if (a.offsets) {
-    __shared__ int s_scan[1024 + ST_THREADS / 32 + 1];
-    for (int i = tid; i < E; i += ST_THREADS) s_scan[i] = __ldcg(a.kept + i);
-    __syncthreads();
     const int tot = block_excl_scan_inplace(s_scan, E, s_scan + 1024);
     for (int i = tid; i < E; i += ST_THREADS) a.offsets[i] = s_scan[i];
     if (tid == 0) a.offsets[E] = tot;
   }
   if (a.aux) {
-    double s = 0.0;
-    for (int i = tid; i < E; i += ST_THREADS)
-      s += (double)__ldcg(a.count_out + i) * (double)__ldcg(a.prob_out + i);
     s = warp_sum_d(s);
     __shared__ double s_d[ST_THREADS / 32];
     if (lane == 0) s_d[warp] = s;
