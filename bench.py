@@ -112,18 +112,24 @@ class ClockSampler:
             self.max_mhz = None
         self._stop = threading.Event()
 
-    def _run(self):
+    def sample(self):
+        """One reading of the SM clock and the active clock-event reasons."""
+        if not self.ok:
+            return
         nv = self.nv
-        while not self._stop.is_set():
+        try:
+            self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
             try:
-                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
-                try:
-                    r = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
-                except Exception:
-                    r = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
-                self.reasons |= int(r)
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
             except Exception:
-                pass
+                r = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
+            self.reasons |= int(r)
+        except Exception:
+            pass
+
+    def _run(self):
+        while not self._stop.is_set():
+            self.sample()
             time.sleep(0.002)
 
     def __enter__(self):
@@ -269,7 +275,7 @@ def run_ours(args, rank, world, local_rank):
         def step():
             layer.forward(x, y, aux, cnt)
 
-    def timed(K, pre=None):
+    def timed(K, pre=None, tick=None):
         starts = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
         ends = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
         if world > 1:
@@ -282,6 +288,8 @@ def run_ours(args, rank, world, local_rank):
             starts[i].record(stream)
             step()
             ends[i].record(stream)
+            if tick:
+                tick()  # the GPU is still working through the queued steps
         torch.cuda.synchronize()
         if world > 1:
             dist.barrier()
@@ -313,7 +321,7 @@ def run_ours(args, rank, world, local_rank):
     # pass 1: the number
     with ClockSampler(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ
                       else local_rank) as clk:
-        times = timed(args.steps)
+        times = timed(args.steps, tick=clk.sample)
     ms = statistics.fmean(times)
     if world > 1:
         t = torch.tensor([ms], dtype=torch.float64, device=dev)

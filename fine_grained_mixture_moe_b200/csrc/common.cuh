@@ -115,6 +115,23 @@ __device__ int block_excl_scan_inplace(int *a, int n, int *tmp) {
   return total;
 }
 
+// ---------------------------------------------------------------- clusters
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// All threads of every CTA in the cluster; release / acquire ordering of shared-memory writes.
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.aligned;\n\tbarrier.cluster.wait.aligned;" ::: "memory");
+}
+// Generic address of the same shared-memory object in CTA `rank` of this cluster.
+template <typename T> __device__ __forceinline__ T *cluster_map(T *p, uint32_t rank) {
+  uint64_t out;
+  asm volatile("mapa.u64 %0, %1, %2;" : "=l"(out) : "l"((uint64_t)p), "r"(rank));
+  return (T *)out;
+}
+
 // ---------------------------------------------------------------- programmatic dependent launch
 // The library launches its kernels with programmatic stream serialisation: a kernel may be
 // scheduled while the previous kernel of the stream is still finishing. griddep_wait() returns

@@ -18,14 +18,6 @@ namespace moe {
 
 constexpr int TC2_BM = 256;  // rows per tile (128 per CTA)
 
-__device__ __forceinline__ uint32_t cluster_ctarank() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-  return r;
-}
-__device__ __forceinline__ void cluster_sync_all() {
-  asm volatile("barrier.cluster.arrive.aligned;\n\tbarrier.cluster.wait.aligned;" ::: "memory");
-}
 // TMA load into this CTA's shared memory whose completion is counted on the leader CTA's barrier
 // (same shared-memory offset in CTA 0: the CTA-rank bit of the cluster address cleared).
 __device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap *map, int c0,
