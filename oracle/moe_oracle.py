@@ -19,7 +19,7 @@ What it computes (every step evaluated in fp64 on the exact fp32 / bf16 input va
    ``sigma(l)`` for sigmoid scoring (the selection bias is not part of the weight). The combine
    weight of slot j is the selected expert's probability, divided by the sum over the k
    selected probabilities when ``norm_topk`` is set.
-5. Capacity (Moonfrost, "routing under a per-expert capacity"): ``C = ceil(cf * T * k / E)`` over the T tokens
+5. Capacity (Moonfrost, expert card: routing under a per-expert capacity): ``C = ceil(cf * T * k / E)`` over the T tokens
    of the call; ``cf <= 0`` is dropless (dormouse, "dropless MoE": no capacity drops). Per
    expert, routed tokens are ranked by ascending token index; rank >= C is dropped.
 6. Permutation grouped by expert (the stacked-expert layout of the Moonfrost card):
@@ -34,6 +34,10 @@ What it computes (every step evaluated in fp64 on the exact fp32 / bf16 input va
    ``L = alpha * E * sum_i f_i * P_i`` with ``f_i = count_i / (T k)`` counted before capacity
    drops, and ``P_i`` the mean over tokens of the token's probability of expert i (for sigmoid
    scoring, ``sigma(l_i)`` normalised over all E experts).
+10. Loss-free balancing (dormouse, "dropless MoE": a bias on the router balances the load instead
+    of an auxiliary loss, after arXiv 2408.15664): ``b_i <- RN32(b_i + u * sign(mean - count_i))``
+    with mean = sum(count) / E, compared exactly on integers; u is the caller's step size (the
+    pages give none).
 
 Exactness of steps 1-2: the fp64 evaluation is screened with a rigorous error bound; only the
 entries whose enclosure contains an fp32 rounding boundary are recomputed exactly (integer
@@ -57,7 +61,7 @@ __all__ = [
     "rn32_dyadic", "rn32_fraction", "router_logits", "selection_keys", "topk",
     "probabilities", "aux_probabilities", "combine_weights", "capacity", "route",
     "permute", "swiglu", "lowrank", "expert_forward", "combine", "aux_loss",
-    "layer_forward", "token_output",
+    "layer_forward", "token_output", "bias_update",
 ]
 
 _U64 = 2.0 ** -53
@@ -395,6 +399,24 @@ def combine(y_perm: np.ndarray, y_shared: Optional[np.ndarray], slot_pos: np.nda
         kept = slot_pos[:, j] >= 0
         y[kept] += w[kept, j][:, None] * y_perm[slot_pos[kept, j]]
     return y
+
+
+def bias_update(count: np.ndarray, bias: np.ndarray, u: float) -> np.ndarray:
+    """Loss-free balancing step on the per-expert selection bias (dormouse, "dropless MoE":
+    balancing by a bias on the router instead of an auxiliary loss, after arXiv 2408.15664):
+    ``b_i <- b_i + u * sign(mean_load - load_i)`` with load_i = count_i and mean_load =
+    sum(count) / E. The comparison is made exactly on integers (sign(sum(count) - E count_i));
+    the new fp32 bias is the exact real b_i + u*s rounded once to fp32 (nearest even).
+    """
+    count = np.asarray(count, np.int64)
+    E = count.shape[0]
+    total = int(count.sum())
+    u32 = Fraction(float(np.float32(u)))
+    out = np.empty(E, np.float32)
+    for i in range(E):
+        s = (total > E * int(count[i])) - (total < E * int(count[i]))
+        out[i] = rn32_fraction(Fraction(float(np.float32(bias[i]))) + u32 * s)
+    return out
 
 
 def aux_loss(count: np.ndarray, prob_sum: np.ndarray, T: int, k: int, alpha: float) -> float:

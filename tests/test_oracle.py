@@ -359,3 +359,41 @@ def test_config_table_capacity_and_shapes():
     assert oracle.capacity(cfg.T, cfg.top_k, cfg.E, cfg.capacity_factor) == 1920
     q = get_config("quartz")
     assert (q.d, q.E, q.top_k, q.n_shared, q.ffn) == (1024, 24, 6, 2, 640)
+
+
+# ------------------------------------------------------------------ loss-free balancing
+def test_bias_update_signs_and_balance():
+    """Overloaded experts lose u, underloaded gain u, experts at the mean keep their bias;
+    perfectly balanced counts change nothing."""
+    b = np.array([0.5, 0.5, 0.5, 0.5], np.float32)
+    out = oracle.bias_update(np.array([3, 1, 2, 2]), b, 0.25)
+    assert out.tolist() == [0.25, 0.75, 0.5, 0.5]
+    assert np.array_equal(oracle.bias_update(np.array([7, 7, 7]), b[:3], 0.1), b[:3])
+    # mean 1.5 is between the counts: no expert sits on it
+    assert oracle.bias_update(np.array([1, 2]), np.zeros(2, np.float32), 1.0).tolist() == [1.0, -1.0]
+    # scaling every count by the same factor keeps every sign
+    c = np.array([5, 0, 9, 2, 2])
+    bb = np.linspace(-1, 1, 5).astype(np.float32)
+    assert np.array_equal(oracle.bias_update(c, bb, 0.01), oracle.bias_update(3 * c, bb, 0.01))
+
+
+def test_bias_update_rounds_once_to_nearest_even():
+    """1 + 2^-24 is a midpoint between fp32 neighbours and rounds to 1 (even); 1 - 2^-24 is an
+    fp32 value; a step below half an ulp leaves the bias unchanged."""
+    out = oracle.bias_update(np.array([4, 0]), np.array([1.0, 1.0], np.float32), 2.0 ** -24)
+    assert out[0] == np.float32(1.0 - 2.0 ** -24) and out[1] == np.float32(1.0)
+    out = oracle.bias_update(np.array([0, 4]), np.array([3.0, 3.0], np.float32), 2.0 ** -30)
+    assert out.tolist() == [3.0, 3.0]
+
+
+def test_bias_update_matches_ieee_fp32_addition():
+    """Against numpy's fp32 addition (IEEE, correctly rounded) of b and +-u, on random cases."""
+    rng = np.random.default_rng(7)
+    for _ in range(200):
+        E = int(rng.integers(1, 40))
+        c = rng.integers(0, 50, E)
+        b = (rng.standard_normal(E) * 10.0 ** rng.integers(-8, 3)).astype(np.float32)
+        u = np.float32(10.0 ** rng.uniform(-9, 0))
+        s = np.sign(c.sum() - E * c).astype(np.float32)
+        ref = b + (u * s).astype(np.float32)  # float32 + float32 in numpy: one IEEE rounding
+        assert np.array_equal(oracle.bias_update(c, b, float(u)), ref)
