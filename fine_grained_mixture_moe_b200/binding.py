@@ -76,6 +76,7 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
         "moe_combine": (c_int32, [P(MoEConfig), c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                                   c_void_p]),
         "moe_aux_loss": (c_int32, [P(MoEConfig), c_void_p, c_void_p, c_void_p, c_void_p]),
+        "moe_bias_update": (c_int32, [P(MoEConfig), c_void_p, c_void_p, ctypes.c_float, c_void_p]),
         "moe_layer_forward": (c_int32, [P(MoEConfig), c_void_p, P(MoEWeights), c_void_p,
                                         c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
         "moe_status_str": (ctypes.c_char_p, [c_int32]),
@@ -96,7 +97,8 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
 
 
 EXPORTED = ("moe_workspace_size", "moe_capacity", "moe_route", "moe_permute",
-            "moe_expert_forward", "moe_combine", "moe_aux_loss", "moe_layer_forward",
+            "moe_expert_forward", "moe_combine", "moe_aux_loss", "moe_bias_update",
+            "moe_layer_forward",
             "moe_status_str", "moe_get_device_error", "moe_debug_set", "moe_profile_read",
             "moe_debug_wait_timeout_probe", "moe_route_noalloc")
 
@@ -187,6 +189,12 @@ def moe_combine(cfg, y_perm, y_shared, slot_pos, topk_w, y, stream=None) -> None
 def moe_aux_loss(cfg, expert_count, prob_sum, loss, stream=None) -> None:
     _check("moe_aux_loss", load().moe_aux_loss(ctypes.byref(cfg), _ptr(expert_count),
                                                _ptr(prob_sum), _ptr(loss), _stream(stream)))
+
+
+def moe_bias_update(cfg, expert_count, select_bias, u: float, stream=None) -> None:
+    _check("moe_bias_update", load().moe_bias_update(ctypes.byref(cfg), _ptr(expert_count),
+                                                     _ptr(select_bias), ctypes.c_float(u),
+                                                     _stream(stream)))
 
 
 def moe_layer_forward(cfg, x, w: MoEWeights, y, aux_loss, expert_count, ws, ws_bytes,

@@ -646,6 +646,14 @@ moe_status_t moe_aux_loss(const moe_config_t *cfg, const int32_t *expert_count,
   return aux_impl(cfg, expert_count, prob_sum, loss, (cudaStream_t)stream);
 }
 
+moe_status_t moe_bias_update(const moe_config_t *cfg, const int32_t *expert_count,
+                             float *select_bias, float u, void *stream) {
+  MOE_TRY(check_cfg(cfg));
+  MOE_REQUIRE(aligned16(expert_count) && aligned16(select_bias) && std::isfinite(u));
+  return launch_pdl(bias_update_kernel, dim3(1), dim3(256), 0, (cudaStream_t)stream,
+                    expert_count, select_bias, cfg->E, u);
+}
+
 moe_status_t moe_layer_forward(const moe_config_t *cfg, const void *x, const moe_weights_t *w,
                                void *y, float *aux_loss, int32_t *expert_count, void *ws,
                                size_t ws_bytes, void *stream) {

@@ -109,4 +109,31 @@ __global__ void __launch_bounds__(ST_THREADS) moe_stats_kernel(StatsArgs a) {
   if (tid == 0) *a.counter = 0u;
 }
 
+// Loss-free balancing step (dormouse pages: a router bias balances the load in place of the
+// auxiliary loss, after arXiv 2408.15664): b_i <- b_i + u * sign(mean - count_i) with
+// mean = sum(count) / E. The sign compares sum(count) with E * count_i exactly in int64; u * s is
+// exact (s in {-1, 0, 1}), so the fp32 add is the only rounding.
+__global__ void __launch_bounds__(256) bias_update_kernel(const int32_t *__restrict__ count,
+                                                          float *__restrict__ bias, int E,
+                                                          float u) {
+  griddep_wait();
+  griddep_launch();
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  __shared__ long long s_part[8];
+  long long t = 0;
+  for (int i = tid; i < E; i += 256) t += count[i];
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+  if (lane == 0) s_part[warp] = t;
+  __syncthreads();
+  long long total = 0;
+#pragma unroll
+  for (int w = 0; w < 8; ++w) total += s_part[w];
+  for (int i = tid; i < E; i += 256) {
+    const long long ec = (long long)E * count[i];
+    const float sgn = total > ec ? 1.0f : (total < ec ? -1.0f : 0.0f);
+    bias[i] = __fadd_rn(bias[i], u * sgn);
+  }
+}
+
 }  // namespace moe

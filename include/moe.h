@@ -150,6 +150,19 @@ moe_status_t moe_combine(const moe_config_t *cfg, const void *y_perm, const void
 moe_status_t moe_aux_loss(const moe_config_t *cfg, const int32_t *expert_count,
                           const float *prob_sum, float *loss, void *stream);
 
+/* Loss-free balancing step (dormouse, "dropless MoE": a bias on the router balances the load in
+ * place of an auxiliary loss, after arXiv 2408.15664). For every expert i:
+ *   select_bias[i] <- RN32(select_bias[i] + u * sign(mean - expert_count[i])),
+ *   mean = sum_j expert_count[j] / E,
+ * the sign decided exactly on integers (sign(0) = 0), one fp32 rounding (nearest even).
+ * expert_count: [E] int32 on the device, the per-expert selection counts before capacity drops
+ * (as moe_route and moe_layer_forward return them); select_bias: [E] fp32 on the device,
+ * updated in place and read by the next sigmoid-scored routing call; u: the step size (the
+ * pages give none). Only cfg->E of the configuration is used, but the whole configuration is
+ * validated. Asynchronous on `stream`; bad arguments return MOE_ERR_INVALID_ARG. */
+moe_status_t moe_bias_update(const moe_config_t *cfg, const int32_t *expert_count,
+                             float *select_bias, float u, void *stream);
+
 /* The whole layer: route -> permute -> experts -> combine -> loss, no host synchronisation.
  *   y [T, d] fp32; aux_loss: device fp32 scalar (may be NULL); expert_count: optional [E]
  *   int32 output of the router's per-expert selection counts (may be NULL). */

@@ -111,6 +111,10 @@ def test_bad_pointers_and_workspace_are_rejected_on_the_host(lib):
     assert lib.moe_layer_forward(P(cfg), 16, P(w), 16, None, None, 16, need, None) == 1
     assert lib.moe_combine(P(cfg), 16, 16, 16, 16, 8, None) == 1
     assert lib.moe_aux_loss(P(cfg), 16, 16, None, None) == 1
+    # bias update: null counts, misaligned bias, non-finite step
+    assert lib.moe_bias_update(P(cfg), None, 16, ctypes.c_float(0.1), None) == 1
+    assert lib.moe_bias_update(P(cfg), 16, 20, ctypes.c_float(0.1), None) == 1
+    assert lib.moe_bias_update(P(cfg), 16, 16, ctypes.c_float(float("nan")), None) == 1
 
 
 def test_status_strings(lib):

@@ -161,6 +161,35 @@ def test_certified_ties_round_to_even():
     assert ref["route"]["idx"][1].tolist() == [1, 0]
 
 
+def test_bias_update_bitwise():
+    """Loss-free balancing step on the routed counts of the sigmoid configuration, then the next
+    routing call with the updated bias: the bias bit-exact against the oracle, the new routing
+    bit-exact as well. Balanced counts and a single expert leave the bias unchanged."""
+    c = SMALL["sigmoid_s"]
+    inp = make_inputs(c)
+    run = GpuRun(c, inp)
+    o = run.steps()
+    bias0 = np.asarray(inp["select_bias"], np.float32)
+    for u in (1e-3, 2.0 ** -24, 0.05):
+        bd = torch.tensor(bias0, device="cuda")
+        B.moe_bias_update(run.cfg, o["count"], bd, u)
+        assert np.array_equal(np_(bd), oracle.bias_update(np_(o["count"]), bias0, u))
+    # route again with the updated bias: selections follow it exactly
+    inp2 = dict(inp)
+    inp2["select_bias"] = np_(bd)
+    check_steps(c, inp2, exact_only=True)
+    # balanced counts and E = 1: no change
+    cfg = run.cfg
+    flat = torch.full((c.E,), 7, dtype=torch.int32, device="cuda")
+    bd = torch.tensor(bias0, device="cuda")
+    B.moe_bias_update(cfg, flat, bd, 0.5)
+    assert np.array_equal(np_(bd), bias0)
+    one = B.make_config(T=16, d=64, E=1, top_k=1, ffn=64)
+    b1 = torch.tensor([0.25], device="cuda")
+    B.moe_bias_update(one, torch.tensor([16], dtype=torch.int32, device="cuda"), b1, 0.5)
+    assert float(b1) == 0.25
+
+
 def test_empty_call():
     c = get_config("quartz", T=0)
     run = GpuRun(c, make_inputs(c, T=0))
