@@ -51,6 +51,13 @@ EDGE = {
     "f32_sigmoid_cap": MoEConfig(name="f32sc", T=130, d=128, E=8, top_k=3, n_shared=1, ffn=64,
                                  ffn_shared=64, dtype="f32", score="sigmoid", norm_topk=True,
                                  bias=("uniform", 0.1), capacity_factor=0.8),
+    # the largest top_k, on both sides of the switch from per-pair rank selection (E <= 64) to
+    # per-token warp selection
+    "k8_E64": MoEConfig(name="k8e64", T=97, d=128, E=64, top_k=8, n_shared=1, ffn=64,
+                        ffn_shared=64, offset=("normal", 0.5)),
+    "k8_E65_sigmoid": MoEConfig(name="k8e65", T=97, d=128, E=65, top_k=8, n_shared=0, ffn=64,
+                                ffn_shared=0, score="sigmoid", norm_topk=True,
+                                bias=("uniform", 0.1)),
 }
 
 
@@ -196,6 +203,37 @@ def test_empty_call():
     y, aux, cnt = run.layer()
     assert float(aux) == 0.0
     assert int(cnt.abs().sum()) == 0
+
+
+def test_back_to_back_calls_on_one_workspace():
+    """Four layer calls queued without synchronisation on one workspace and stream, each on
+    different tokens, must give exactly what each gives alone: every kernel orders its memory
+    accesses after the previous one (programmatic dependent launch), including reuse of the
+    workspace by the next call."""
+    c = SMALL["quartz_s"]
+    inp = make_inputs(c)
+    run = GpuRun(c, inp)
+    rng = np.random.default_rng(11)
+    xs = [torch.as_tensor(rng.standard_normal(inp["x"].shape).astype(np.float32)).to(run.dt)
+          .contiguous().to(run.dev) for _ in range(4)]
+    alone = []
+    for xb in xs:
+        run.x = xb
+        y, aux, cnt = run.layer()
+        torch.cuda.synchronize()
+        alone.append((y.clone(), float(aux), cnt.clone()))
+    outs = []
+    for xb in xs:  # queued back to back, no host synchronisation in between
+        y = torch.empty_like(alone[0][0])
+        aux = torch.empty((), dtype=torch.float32, device=run.dev)
+        cnt = torch.empty_like(alone[0][2])
+        B.moe_layer_forward(run.cfg, xb, run.ws_struct, y, aux, cnt, run.ws, run.ws_bytes)
+        outs.append((y, aux, cnt))
+    torch.cuda.synchronize()
+    st, info = B.moe_get_device_error()
+    assert st == 0, (B.status_str(st), info)
+    for (ya, aa, ca), (yb, ab, cb) in zip(alone, outs):
+        assert torch.equal(ya, yb) and aa == float(ab) and torch.equal(ca, cb)
 
 
 def test_bitwise_determinism():
