@@ -43,6 +43,10 @@ bool cfg_supported(const moe_config_t *c) {
   }
   if (c->n_shared > 0 && (c->ffn_shared <= 0 || c->ffn_shared % 64)) return false;
   if (!std::isfinite(c->capacity_factor) || !std::isfinite(c->aux_alpha)) return false;
+  // the router stages its 16 token rows and the logits in shared memory (227 KB per CTA)
+  if (router_smem(c->E, router_nt_for(c->E), c->score == MOE_SCORE_SIGMOID, c->d,
+                  c->dtype == MOE_DTYPE_BF16 ? 2 : 4).total > 227 * 1024)
+    return false;
   // 32-bit row indices inside the kernels
   if ((long long)c->T * c->top_k * std::max(c->d, 256) >= (1ll << 31) * 64ll) return false;
   if ((long long)c->T * c->top_k >= (1ll << 31)) return false;

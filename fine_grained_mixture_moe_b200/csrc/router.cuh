@@ -7,19 +7,23 @@
 //   top-k by key, ties -> lower expert index, slot order = descending key
 //   weights = softmax over all E (or sigmoid) of the selected experts, optional renormalise
 //
-// How: the dot products run on the fp64 FMA pipe. bf16 and fp32 inputs multiply exactly in
-// fp64, so the only error is the summation, bounded by (d+2) 2^-52 (|x|_2 |W_e|_2 + |off|).
-// When that enclosure holds no fp32 rounding boundary, RN32 of the fp64 value *is* the exact
-// rounding. Otherwise the logit is marked and, after the main pass, a whole warp decides it
-// exactly: bf16 products carry at most 16 significant bits, so the exact sum of a row is a
-// multiple of a small power of two and lands exactly on an fp32 rounding boundary for about
-// 0.4% of logits - genuine ties that no error bound can settle. The warp scales every exact
-// product to an integer multiple of the smallest power of two present and sums them in int64,
-// exactly, then compares with the boundaries. Only when the exponent span exceeds 50 bits (or
-// in a forced test mode) does one thread sum the products as a non-overlapping floating-point
-// expansion (Shewchuk's Grow-Expansion with zero elimination) and decide from its sign. Sigmoid keys are
-// screened the same way (fp64 exp, documented 1-ulp) and resolved in double-double arithmetic.
-// So the integer routing decisions are exact, not merely tolerant.
+// How: the dot products run on the fp64 tensor pipe (mma.sync m8n8k4). bf16 and fp32 inputs
+// multiply exactly in fp64, so the only error is the summation. Each logit is then decided one
+// of three ways, all exact:
+//   1. certificate: when every product is a multiple of 2^q (from the rows' smallest exponents)
+//      and the Cauchy-Schwarz bound on every partial sum is below 2^(q+53), the fp64 sum *is*
+//      the exact sum and its round-to-nearest-even is the logit. This covers the exact ties that
+//      bf16 data produce often (~0.8% of logits land exactly on an fp32 rounding midpoint);
+//   2. enclosure: the error bound (d+16) 2^-52 (|x|_2 |W_e|_2 + |off|) leaves no fp32 rounding
+//      boundary inside the interval, so RN32 of the fp64 value is the exact rounding;
+//   3. otherwise (2 in 98,304 Quartz logits) a whole warp decides it after the main pass: it
+//      scales every exact product to an integer multiple of the smallest power of two present,
+//      sums them in int64, exactly, and compares with the boundaries. Only when the exponent span
+//      exceeds 50 bits (or in a forced test mode) does one thread sum the products as a
+//      non-overlapping floating-point expansion (Shewchuk's Grow-Expansion with zero
+//      elimination) and decide from its sign.
+// Sigmoid keys are screened the same way (fp64 exp within its documented error) and resolved
+// in double-double arithmetic. So the integer routing decisions are exact, not merely tolerant.
 #pragma once
 #include "common.cuh"
 
@@ -31,7 +35,8 @@ constexpr int RT_WARPS = 8;        // each a slice of the K dimension
 constexpr int RT_THREADS = 32 * RT_WARPS;
 constexpr int RT_KB = 16;          // k block: lane (row r, column c) of a fragment reads the 4
                                    // consecutive elements 4c..4c+3 of the block with one load
-constexpr int RT_SEL_THREAD_MAX_E = 64;  // up to this many experts, one thread selects per token
+constexpr int RT_SEL_THREAD_MAX_E = 64;  // up to this many experts: one thread per (token,
+                                         // expert) finds its rank; above, a warp per token
 constexpr int EXPANSION_MAX = 40;
 constexpr int RT_FIX_CAP = 256;   // flagged logits per CTA kept with their fp64 sums
 
