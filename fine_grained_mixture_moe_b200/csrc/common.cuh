@@ -26,6 +26,7 @@ enum : long long {
   INFO_WAIT_ACC_EMPTY = 13,
   INFO_WAIT_DRAIN = 14,
   INFO_WAIT_ROUTER_X = 15,
+  INFO_WAIT_SCATTER = 16,
   INFO_WAIT_PROBE = 20,
 };
 
@@ -145,6 +146,17 @@ __device__ __forceinline__ void griddep_launch() {
 }
 
 // ---------------------------------------------------------------- mbarriers (shared memory)
+// 1-D bulk copy shared -> global, tracked by the issuing thread's bulk group. src, dst 16-byte
+// aligned; bytes a multiple of 16. bulk_store_commit_wait_read() returns when every store the
+// thread issued has finished reading shared memory (the buffer may then be reused).
+__device__ __forceinline__ void bulk_store_1d(void *dst, uint32_t src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst), "r"(src),
+               "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_store_commit_wait_read() {
+  asm volatile("cp.async.bulk.commit_group;\n\tcp.async.bulk.wait_group.read 0;" ::: "memory");
+}
 // 1-D bulk copy global -> this CTA's shared memory, counted on an mbarrier (complete_tx).
 // dst, src 16-byte aligned; bytes a multiple of 16.
 __device__ __forceinline__ void bulk_load_1d(uint32_t dst, const void *src, uint32_t bytes,

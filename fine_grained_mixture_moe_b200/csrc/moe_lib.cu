@@ -431,9 +431,15 @@ moe_status_t scatter_impl(const moe_config_t *c, const void *x, const int32_t *i
                           const int32_t *chunk_base, const int32_t *offsets, int32_t *slot_pos,
                           int32_t *src, void *x_perm, cudaStream_t st) {
   ProfScope ps(K_PERM_SCATTER, st);
+  // shared memory: the CTA's PM_TPC token rows, then the per-expert lane masks
+  const size_t smem = (size_t)PM_TPC * c->d * sizeof(Tin) + (size_t)c->E * 4;
+  if (smem > 48 * 1024 &&
+      cudaFuncSetAttribute(perm_scatter_kernel<Tin>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)smem) != cudaSuccess)
+    return MOE_ERR_CUDA;
   return launch_pdl(perm_scatter_kernel<Tin>, dim3(ceil_div(c->T, PM_CHUNK) * PM_SPLIT), dim3(256),
-                    (size_t)c->E * 4, st, idx, c->T, c->top_k, c->E, capacity_of(c), chunk_base,
-                    offsets, slot_pos, src, (const Tin *)x, (Tin *)x_perm, c->d);
+                    smem, st, idx, c->T, c->top_k, c->E, capacity_of(c), chunk_base, offsets,
+                    slot_pos, src, (const Tin *)x, (Tin *)x_perm, c->d);
 }
 
 template <typename Tin>

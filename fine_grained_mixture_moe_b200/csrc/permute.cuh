@@ -10,8 +10,8 @@
 //           moe_permute on its own)
 //   stats   per-expert exclusive scan over chunks -> chunk_base; offsets[E+1] (stats.cuh)
 //   scatter per-chunk ranks from a per-expert lane bitmask, slot_pos / src_token; PM_SPLIT
-//           CTAs per chunk each copy 4 of its x rows to their k destinations in x_perm with
-//           16-byte loads and stores (each row read once).
+//           CTAs per chunk each bring 4 of its x rows into shared memory and store each to its
+//           k destinations in x_perm with 1-D bulk copies (each row read once).
 #pragma once
 #include "common.cuh"
 
@@ -46,14 +46,12 @@ __global__ void __launch_bounds__(256) perm_hist_kernel(const int32_t *__restric
   for (int e = lane; e < E; e += 32) chunk_count[(size_t)chunk * E + e] = c[e];
 }
 
-// Scatter. CTA (chunk, part) owns tokens chunk*16 + part*TPC .. +TPC (TPC = 16 / PM_SPLIT): two
-// warps per token, one half of the row each. Each warp loads its half-row into registers first
-// (these loads do not depend on the routing, so they overlap the index work), warp 0 meanwhile
-// ranks the chunk's (token, slot) pairs, and after one barrier every warp stores its half-row to
-// the token's kept destinations: x is read once and written k times.
+// Scatter. CTA (chunk, part) owns tokens chunk*16 + part*TPC .. +TPC (TPC = 16 / PM_SPLIT).
+// Thread 0 brings the CTA's token rows into shared memory with 1-D bulk copies (they do not
+// depend on the routing, so they overlap the index work) while warp 0 ranks the chunk's
+// (token, slot) pairs; then one thread per kept pair stores the whole row to its x_perm row with
+// a single shared -> global bulk copy. x is read once and written k times by the copy engine.
 constexpr int PM_TPC = PM_CHUNK / PM_SPLIT;        // tokens per scatter CTA
-constexpr int PM_VMAX = 4;                          // 16-byte vectors per lane held at once
-static_assert(PM_TPC * 2 == 8, "two warps per token, eight warps per CTA");
 
 template <typename Tin>
 __global__ void __launch_bounds__(256) perm_scatter_kernel(
@@ -63,27 +61,31 @@ __global__ void __launch_bounds__(256) perm_scatter_kernel(
     Tin *__restrict__ x_perm, int d) {
   griddep_wait();
   griddep_launch();
-  extern __shared__ unsigned smask[];  // [E]
+  extern __shared__ __align__(128) unsigned char sm_raw[];  // [PM_TPC rows][row_bytes] | [E]
   __shared__ int s_pos[PM_CHUNK * 8];
+  __shared__ __align__(8) uint64_t s_bar;
+  __shared__ volatile int s_abort;
   const bool active = (threadIdx.x & 31) < PM_CHUNK;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int chunk = blockIdx.x / PM_SPLIT, part = blockIdx.x % PM_SPLIT;
-  // this warp's token and half-row
-  const int tl = part * PM_TPC + (warp >> 1);  // token within the chunk
-  const int tw = chunk * PM_CHUNK + tl;
-  const int nvec = d * (int)sizeof(Tin) / 16;   // 16-byte vectors per row
-  const int hv = (nvec + 1) / 2;
-  const int vbeg = (warp & 1) * hv, vend = min(nvec, vbeg + hv);
-  const uint4 *srow = (const uint4 *)(x + (size_t)(tw < T ? tw : 0) * d);
-  const bool copy = x_perm != nullptr && tw < T;
-  uint4 held[PM_VMAX];
-  int v0 = vbeg;
-  if (copy) {
-#pragma unroll
-    for (int i = 0; i < PM_VMAX; ++i) {
-      const int v = v0 + lane + 32 * i;
-      if (v < vend) held[i] = __ldg(srow + v);
-    }
+  const uint32_t row_bytes = (uint32_t)d * (uint32_t)sizeof(Tin);
+  unsigned char *rows = sm_raw;
+  unsigned *smask = (unsigned *)(sm_raw + (size_t)PM_TPC * row_bytes);
+  const int tfirst = chunk * PM_CHUNK + part * PM_TPC;
+  const int nrows = max(0, min(PM_TPC, T - tfirst));
+  const bool copy = x_perm != nullptr && nrows > 0;
+  const uint32_t bar = smem_u32(&s_bar);
+  if (tid == 0) {
+    s_abort = 0;
+    mbar_init(bar, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();  // the barrier is initialised before anyone waits on it
+  if (tid == 0 && copy) {
+    mbar_expect_tx(bar, (uint32_t)nrows * row_bytes);
+    for (int r = 0; r < nrows; ++r)
+      bulk_load_1d(smem_u32(rows + (size_t)r * row_bytes), x + (size_t)(tfirst + r) * d,
+                   row_bytes, bar);
   }
   if (warp == 0) {
     const int t = chunk * PM_CHUNK + lane;
@@ -121,26 +123,23 @@ __global__ void __launch_bounds__(256) perm_scatter_kernel(
       }
     }
   }
-  __syncthreads();
-  if (!copy) return;
-  for (;;) {
-    for (int j = 0; j < k; ++j) {
-      const int pos = s_pos[tl * k + j];
-      if (pos < 0) continue;
-      uint4 *drow = (uint4 *)(x_perm + (size_t)pos * d);
-#pragma unroll
-      for (int i = 0; i < PM_VMAX; ++i) {
-        const int v = v0 + lane + 32 * i;
-        if (v < vend) drow[v] = held[i];
-      }
+  if (!copy) return;  // uniform over the CTA
+  // rows landed (bounded wait; on expiry the error is recorded and the copies drain)
+  mbar_wait(bar, 0u, &s_abort, g_wait_limit_ns, INFO_WAIT_SCATTER);
+  __syncthreads();  // s_pos ready; every thread has seen the rows land or the abort
+  if (s_abort) {
+    if (tid == 0) {
+      volatile int never = 0;
+      mbar_wait(bar, 0u, &never, g_wait_limit_ns, INFO_WAIT_DRAIN);
     }
-    // rows longer than 2 * 32 * PM_VMAX vectors: the next slice of the half-row
-    v0 += 32 * PM_VMAX;
-    if (v0 >= vend) break;
-#pragma unroll
-    for (int i = 0; i < PM_VMAX; ++i) {
-      const int v = v0 + lane + 32 * i;
-      if (v < vend) held[i] = __ldg(srow + v);
+    return;
+  }
+  if (tid < nrows * k) {
+    const int r = tid / k, j = tid - r * k;
+    const int pos = s_pos[(part * PM_TPC + r) * k + j];
+    if (pos >= 0) {
+      bulk_store_1d(x_perm + (size_t)pos * d, smem_u32(rows + (size_t)r * row_bytes), row_bytes);
+      bulk_store_commit_wait_read();  // the rows stay in shared memory until read
     }
   }
 }
