@@ -1,20 +1,21 @@
-// bf16 grouped expert GEMM on the 5th-generation tensor cores (sm_100a).
+// bf16 grouped expert GEMM on the 5th-generation tensor cores (sm_100a), single-SM form.
+//
+// It serves the low-rank V projection (SCALE) and down projections whose width is not a multiple
+// of 256 (PLAIN). The SwiGLU gate/up product and the other down projections run on CTA pairs
+// (gemm_tc2.cuh), which share this file's PTX wrappers, tensor maps and epilogue conventions.
 //
 // One persistent CTA per SM walks a device-side tile list built from the group offsets
 // (Moonfrost's stacked (E, hidden, ffn) expert tensors, here indexed by expert on the device so
-// the host never sees a count). Per CTA: 6 warps.
-//   warp 0  TMA producer: A tile [128 x 64] and B tile(s) [BN x 64] per k-block into a STAGES-
-//           deep shared-memory ring (128-byte swizzle, K-major), completion on `full[s]`.
+// the host never sees a count). Per CTA: 10 warps.
+//   warp 0  TMA producer: A tile [128 x 64] and B tile [BN x 64] per k-block into a STAGES-deep
+//           shared-memory ring (128-byte swizzle, K-major), completion on `full[s]`.
 //   warp 1  TMEM owner and MMA issuer: one thread issues tcgen05.mma (kind::f16, bf16 x bf16 ->
 //           fp32, M=128, N=BN, K=16) into one of two TMEM accumulators; tcgen05.commit frees the
 //           smem stage (`empty[s]`) and, per tile, publishes the accumulator (`acc_full[b]`).
 //   warps 2-9 epilogue: two warps per TMEM lane quarter, each taking half of the tile's columns;
-//           tcgen05.ld (32 lanes x 32 columns per load) -> SwiGLU / scale -> bf16 (hidden
-//           activations, the next GEMM's operand) or fp32 (expert outputs) -> global; then
+//           tcgen05.ld (32 lanes x 32 columns per load) -> scale -> bf16 (the low-rank
+//           projection, the next GEMM's operand) or bf16 / fp32 expert outputs -> global; then
 //           `acc_empty[b]`, so the next tile's MMAs overlap this epilogue.
-// GATEUP stages the gate and up weight tiles back to back, so one N=256 MMA fills 128 gate and
-// 128 up accumulator columns (256 fp32 columns per buffer, 512 with double buffering) and
-// silu(gate) * up is fused without a weight repack.
 // Every wait is bounded (global timer); on expiry the CTA records MOE_ERR_TIMEOUT, drains what
 // it has in flight (again bounded), frees its TMEM and returns.
 #pragma once
@@ -38,7 +39,9 @@ struct TcParams {
 };
 
 template <int MODE, int BN> struct TcCfg {
-  static constexpr int NB = (MODE == MODE_GATEUP) ? 2 : 1;        // B tiles per stage
+  static_assert(MODE == MODE_PLAIN || MODE == MODE_SCALE,
+                "single-SM form: down and low-rank products (gate/up runs on CTA pairs)");
+  static constexpr int NB = 1;                                    // B tiles per stage
   static constexpr int A_BYTES = TC_BM * TC_BK * 2;               // 16 KB
   static constexpr int B_BYTES = BN * TC_BK * 2;
   static constexpr int STAGE_BYTES = A_BYTES + NB * B_BYTES;
@@ -50,9 +53,6 @@ template <int MODE, int BN> struct TcCfg {
                                    : (2 * ACC_COLS <= 128) ? 128 : (2 * ACC_COLS <= 256) ? 256 : 512;
   static_assert(2 * ACC_COLS <= 512, "TMEM holds 512 columns");
   static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "UMMA N for M=128, epilogue in 32s");
-  // one MMA covers N = NB*BN columns: for GATEUP the gate and up tiles sit back to back in
-  // shared memory, so they form one [2*BN, 64] B operand whose first BN accumulator columns are
-  // the gate and the next BN the up projection
   static constexpr int MMA_N = NB * BN;
   static_assert(MMA_N <= 256, "UMMA N <= 256");
   // instruction descriptor: D fp32, A/B bf16, both K-major, N>>3 at bit 17, M>>4 at bit 24
@@ -203,7 +203,6 @@ __global__ void __launch_bounds__(TC_THREADS, 1) gemm_tc_kernel(const __grid_con
         const bool routed = ti.g < p.E;
         const CUtensorMap *ma = routed ? &P.maps.a_r : &P.maps.a_s;
         const CUtensorMap *mb0 = routed ? &P.maps.b0_r : &P.maps.b0_s;
-        const CUtensorMap *mb1 = routed ? &P.maps.b1_r : &P.maps.b1_s;
         const int a_row = ti.a_row0 + ti.m0;
         const int nk = ti.K / TC_BK;
         for (int kb = 0; kb < nk; ++kb) {
@@ -226,7 +225,6 @@ __global__ void __launch_bounds__(TC_THREADS, 1) gemm_tc_kernel(const __grid_con
           }
           tma_load_2d(sA, ma, kk, a_row, full_bar(stage));
           tma_load_2d(sB0, mb0, b_col, b_row, full_bar(stage));
-          if (C::NB == 2) tma_load_2d(sB0 + C::B_BYTES, mb1, b_col, b_row, full_bar(stage));
           issued[stage] = true;
           issued_parity[stage] = (int)phase;
           if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
@@ -319,14 +317,13 @@ __global__ void __launch_bounds__(TC_THREADS, 1) gemm_tc_kernel(const __grid_con
       constexpr int SUB = (MODE == MODE_PLAIN) ? 1 : 2;  // 32-column TMEM loads per block
 #pragma unroll 1
       for (int c = cbeg; c < cend; c += 32 * SUB) {
-        if (MODE != MODE_PLAIN) {
-          // bf16 outputs (SwiGLU hidden, low-rank projection): each lane already writes 64
-          // contiguous bytes of its row, so they go out directly
+        if (MODE == MODE_SCALE) {
+          // bf16 low-rank projection: each lane already writes 64 contiguous bytes of its row, so
+          // they go out directly
 #pragma unroll
           for (int sub = 0; sub < SUB; ++sub) {
-            uint32_t r0[32], r1[32];
+            uint32_t r0[32];
             tmem_ld32(tbase + c + 32 * sub, r0);
-            if (C::NB == 2) tmem_ld32(tbase + BN + c + 32 * sub, r1);
             tmem_wait_ld();
             const int col = ti.n0 + c + 32 * sub;
             if (row_ok && col < ti.N) {
@@ -335,14 +332,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1) gemm_tc_kernel(const __grid_con
 #pragma unroll
               for (int i = 0; i < 16; ++i) {
                 const float g0 = __uint_as_float(r0[2 * i]), g1 = __uint_as_float(r0[2 * i + 1]);
-                float v0, v1;
-                if (MODE == MODE_GATEUP) {
-                  v0 = __fdividef(g0, 1.0f + __expf(-g0)) * __uint_as_float(r1[2 * i]);
-                  v1 = __fdividef(g1, 1.0f + __expf(-g1)) * __uint_as_float(r1[2 * i + 1]);
-                } else {
-                  v0 = g0 * __ldg(p.scale + (size_t)ti.g * ti.N + col + 2 * i);
-                  v1 = g1 * __ldg(p.scale + (size_t)ti.g * ti.N + col + 2 * i + 1);
-                }
+                const float v0 = g0 * __ldg(p.scale + (size_t)ti.g * ti.N + col + 2 * i);
+                const float v1 = g1 * __ldg(p.scale + (size_t)ti.g * ti.N + col + 2 * i + 1);
                 h[i] = __floats2bfloat162_rn(v0, v1);
               }
               uint4 *dst = (uint4 *)((__nv_bfloat16 *)out + (size_t)(ti.a_row0 + row) * ldo + col);
