@@ -58,6 +58,9 @@ EDGE = {
     "k8_E65_sigmoid": MoEConfig(name="k8e65", T=97, d=128, E=65, top_k=8, n_shared=0, ffn=64,
                                 ffn_shared=0, score="sigmoid", norm_topk=True,
                                 bias=("uniform", 0.1)),
+    # a wide hidden size: 16 staged token rows of 8 KB in the router, K = 4096 in gate/up
+    "d4096": MoEConfig(name="d4096", T=45, d=4096, E=8, top_k=2, n_shared=1, ffn=128,
+                       ffn_shared=128, offset=("normal", 0.5)),
 }
 
 
