@@ -331,14 +331,11 @@ __device__ dd dd_exp(double y) {
   return {ldexp(s.hi, ni), ldexp(s.lo, ni)};
 }
 
-// RN32(sigmoid(l) + b), exact. fp64 screen first unless forced.
-__device__ float sigmoid_key(float l, float b, bool force) {
-  const double s = 1.0 / (1.0 + exp(-(double)l));
-  const double v = s + (double)b;
-  const double B = 0x1p-48 * s + 0x1p-52 * fabs(v) + 1e-300;
-  float r, up, dn;
-  double mh, ml;
-  if (rn32_certain(v, B, r, up, dn, mh, ml) && !force) return r;
+// The exact decision for a sigmoid key the fp64 screen could not settle (rare, kept out of line
+// so it does not occupy the instruction cache of the hot loop): double-double sigmoid, compared
+// with the fp32 rounding midpoints mh / ml around the candidate r.
+__device__ __noinline__ float sigmoid_key_exact(float l, float b, float r, float up, float dn,
+                                                double mh, double ml) {
   int c_hi, c_lo;
   if (l == 0.0f) {  // sigmoid(0) = 1/2 exactly
     const dd vv = two_sum(0.5, (double)b);
@@ -358,8 +355,18 @@ __device__ float sigmoid_key(float l, float b, bool force) {
     set_device_error(MOE_ERR_DEVICE_CHECK, INFO_SIGMOID_UNRESOLVED);
   c_hi = a.hi > 0 ? 1 : (a.hi < 0 ? -1 : 0);
   c_lo = c.hi > 0 ? 1 : (c.hi < 0 ? -1 : 0);
-  // recompute the candidate around the dd value in case the screen's r was a neighbour off
   return rn32_from_signs(r, up, dn, c_hi, c_lo);
+}
+
+// RN32(sigmoid(l) + b), exact. fp64 screen first unless forced.
+__device__ __forceinline__ float sigmoid_key(float l, float b, bool force) {
+  const double s = 1.0 / (1.0 + exp(-(double)l));
+  const double v = s + (double)b;
+  const double B = 0x1p-48 * s + 0x1p-52 * fabs(v) + 1e-300;
+  float r, up, dn;
+  double mh, ml;
+  if (rn32_certain(v, B, r, up, dn, mh, ml) && !force) return r;
+  return sigmoid_key_exact(l, b, r, up, dn, mh, ml);
 }
 
 // ------------------------------------------------------------------ kernels
