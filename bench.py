@@ -97,15 +97,25 @@ class ClockSampler:
                0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
                0x100: "display_clock_setting"}
 
-    def __init__(self, index: int):
+    def __init__(self, device):
+        """`device`: the torch CUDA device index of this rank. NVML numbers devices physically,
+        so the handle is found by the device's UUID (CUDA_VISIBLE_DEVICES may reorder or name
+        devices), falling back to the index."""
         self.samples = []
         self.reasons = 0
         self.ok = False
         try:
             import pynvml
+            import torch
             pynvml.nvmlInit()
             self.nv = pynvml
-            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.h = None
+            try:
+                uuid = str(torch.cuda.get_device_properties(device).uuid)
+                self.h = pynvml.nvmlDeviceGetHandleByUUID(
+                    uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+            except Exception:
+                self.h = pynvml.nvmlDeviceGetHandleByIndex(device)
             self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
             self.ok = True
         except Exception:
@@ -319,8 +329,7 @@ def run_ours(args, rank, world, local_rank):
         counts = cnt.cpu().numpy()
 
     # pass 1: the number
-    with ClockSampler(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ
-                      else local_rank) as clk:
+    with ClockSampler(torch.cuda.current_device()) as clk:
         times = timed(args.steps, tick=clk.sample)
     ms = statistics.fmean(times)
     if world > 1:
