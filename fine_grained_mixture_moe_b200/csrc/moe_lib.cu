@@ -566,10 +566,13 @@ moe_status_t check_ws(const moe_config_t *c, void *ws, size_t bytes) {
   if (!aligned16(ws)) return MOE_ERR_INVALID_ARG;
   return bytes >= layout_of(c).total ? MOE_OK : MOE_ERR_WORKSPACE;
 }
+inline bool aligned4_or_null(const void *p) { return ((uintptr_t)p & 3u) == 0; }
 moe_status_t check_weights(const moe_config_t *c, const moe_weights_t *w, bool router,
                            bool experts) {
   if (!w) return MOE_ERR_INVALID_ARG;
   if (router && !aligned16(w->w_router)) return MOE_ERR_INVALID_ARG;
+  if (router && (!aligned4_or_null(w->logit_offset) || !aligned4_or_null(w->select_bias)))
+    return MOE_ERR_INVALID_ARG;
   if (experts) {
     if (c->expert == MOE_EXPERT_SWIGLU) {
       if (!aligned16(w->w_gate) || !aligned16(w->w_up) || !aligned16(w->w_down)) return MOE_ERR_INVALID_ARG;

@@ -128,21 +128,26 @@ moe_status_t moe_permute(const moe_config_t *cfg, const void *x, const int32_t *
  *     y_perm[r] = W_down[e] (silu(W_gate[e] x_perm[r]) * (W_up[e] x_perm[r]))
  *   low-rank expert: y_perm[r] = U[e] (s[e] * (V[e] x_perm[r]))
  *   y_shared[t] = sum over shared experts of their SwiGLU output on x[t]
- * Intermediates (the SwiGLU hidden activations, the low-rank projections) are rounded to
- * dtype, since they are the next tensor-core product's operand; accumulation is fp32.
- * y_perm: [T*top_k, d] in dtype (first offsets[E] rows written), each row rounded once from its
- * fp32 accumulator; y_shared: [T, d] fp32 (the S shared outputs summed in fp32), may be NULL
- * when n_shared = 0. The routed rows enter y through a weighted sum of top_k of them, which
- * averages their rounding; the shared output enters y alone, so it stays fp32. */
+ * The SwiGLU hidden activations are rounded to dtype, since they are the next tensor-core
+ * product's operand; a bf16 low-rank projection is kept as two bf16 terms (its value and its
+ * rounding residual); accumulation is fp32.
+ * y_perm: [T*top_k, d] (first offsets[E] rows written), each row rounded once from its fp32
+ * accumulator: bf16 for bf16 SwiGLU layers, fp32 for fp32 layers and for low-rank layers. A
+ * SwiGLU row enters y through a weighted sum of top_k rows plus the shared output, which
+ * averages its rounding; a low-rank layer's y can be a sum of as few as two rows with no shared
+ * output, where one bf16 rounding alone exceeds the error budget.
+ * y_shared: [T, d] fp32 (the S shared outputs summed in fp32), may be NULL when n_shared = 0;
+ * it enters y alone, so it stays fp32. */
 moe_status_t moe_expert_forward(const moe_config_t *cfg, const void *x_perm,
                                 const int32_t *offsets, const void *x,
                                 const moe_weights_t *w, void *y_perm, void *y_shared,
                                 void *ws, size_t ws_bytes, void *stream);
 
 /* Weighted un-permute: y[t] = y_shared[t] + sum_j [slot_pos[t,j] >= 0] topk_w[t,j] *
- * y_perm[slot_pos[t,j]], summed in fp32 in slot order. y_perm is in dtype, y_shared and y are
- * fp32 [.., d]: a bf16 rounding of y itself would cost up to 2^-8 * max|y| / rms(y), the whole
- * 2e-2 error budget of the layer. No atomics. y_shared may be NULL (no shared experts). */
+ * y_perm[slot_pos[t,j]], summed in fp32 in slot order. y_perm as moe_expert_forward writes it
+ * (bf16 for bf16 SwiGLU layers, else fp32); y_shared and y are fp32 [.., d]: a bf16 rounding of
+ * y itself would cost up to 2^-8 * max|y| / rms(y), the whole 2e-2 error budget of the layer.
+ * No atomics. y_shared may be NULL (no shared experts). */
 moe_status_t moe_combine(const moe_config_t *cfg, const void *y_perm, const void *y_shared,
                          const int32_t *slot_pos, const float *topk_w, void *y, void *stream);
 
