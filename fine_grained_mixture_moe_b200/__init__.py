@@ -7,8 +7,8 @@ the built library every call raises.
 """
 from .binding import (DEBUG_FORCE_EXACT, DEBUG_PROFILE, DEBUG_WAIT_LIMIT_NS, EXPORTED,  # noqa: F401
                       MoEConfig, MoEError, MoEWeights, load, make_config, make_weights,
-                      moe_aux_loss, moe_capacity, moe_combine, moe_debug_set,
+                      moe_aux_loss, moe_bias_update, moe_capacity, moe_combine, moe_debug_set,
                       moe_debug_wait_timeout_probe, moe_expert_forward, moe_get_device_error,
                       moe_layer_forward, moe_permute, moe_profile_read, moe_route,
-                      moe_workspace_size, status_str)
-from .layer import MoELayer, torch_dtype, upload_weights  # noqa: F401
+                      moe_route_noalloc, moe_workspace_size, status_str)
+from .layer import MoELayer, torch_dtype, upload_weights, y_perm_dtype  # noqa: F401

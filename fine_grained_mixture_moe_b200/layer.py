@@ -69,4 +69,12 @@ class MoELayer:
                             self.ws_bytes, stream)
         return y, aux
 
+    def update_bias(self, expert_count: torch.Tensor, u: float, stream=None) -> None:
+        """Loss-free balancing step (moe_bias_update) on this layer's selection bias, from the
+        expert counts a forward call returned; the next sigmoid-scored call routes with it."""
+        bias = self.weights.get("select_bias")
+        if bias is None:
+            raise ValueError("the layer has no select_bias weight to update")
+        B.moe_bias_update(self.cfg, expert_count, bias, u, stream)
+
     __call__ = forward
