@@ -431,8 +431,9 @@ moe_status_t scatter_impl(const moe_config_t *c, const void *x, const int32_t *i
                           const int32_t *chunk_base, const int32_t *offsets, int32_t *slot_pos,
                           int32_t *src, void *x_perm, cudaStream_t st) {
   ProfScope ps(K_PERM_SCATTER, st);
-  // shared memory: the CTA's PM_TPC token rows, then the per-expert lane masks
-  const size_t smem = (size_t)PM_TPC * c->d * sizeof(Tin) + (size_t)c->E * 4;
+  // shared memory: the CTA's PM_TPC token rows, then per expert the lane mask, the chunk's
+  // base rank and the offset
+  const size_t smem = (size_t)PM_TPC * c->d * sizeof(Tin) + (size_t)c->E * 12;
   if (smem > 48 * 1024 &&
       cudaFuncSetAttribute(perm_scatter_kernel<Tin>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)smem) != cudaSuccess)

@@ -47,10 +47,11 @@ __global__ void __launch_bounds__(256) perm_hist_kernel(const int32_t *__restric
 }
 
 // Scatter. CTA (chunk, part) owns tokens chunk*16 + part*TPC .. +TPC (TPC = 16 / PM_SPLIT).
-// Thread 0 brings the CTA's token rows into shared memory with 1-D bulk copies (they do not
-// depend on the routing, so they overlap the index work) while warp 0 ranks the chunk's
-// (token, slot) pairs; then one thread per kept pair stores the whole row to its x_perm row with
-// a single shared -> global bulk copy. x is read once and written k times by the copy engine.
+// Thread 0 first starts 1-D bulk copies of the CTA's token rows into shared memory (they do not
+// depend on the routing); the chunk's routing, its per-expert base ranks and the expert offsets
+// are read together; warp 0 then ranks the chunk's (token, slot) pairs, and one thread per kept
+// pair stores the whole row to its x_perm row with a single shared -> global bulk copy. x is read
+// once and written k times by the copy engine.
 constexpr int PM_TPC = PM_CHUNK / PM_SPLIT;        // tokens per scatter CTA
 
 template <typename Tin>
@@ -61,7 +62,8 @@ __global__ void __launch_bounds__(256) perm_scatter_kernel(
     Tin *__restrict__ x_perm, int d) {
   griddep_wait();
   griddep_launch();
-  extern __shared__ __align__(128) unsigned char sm_raw[];  // [PM_TPC rows][row_bytes] | [E]
+  // [PM_TPC rows][row_bytes] | lane masks [E] | chunk base [E] | offsets [E]
+  extern __shared__ __align__(128) unsigned char sm_raw[];
   __shared__ int s_pos[PM_CHUNK * 8];
   __shared__ __align__(8) uint64_t s_bar;
   __shared__ volatile int s_abort;
@@ -71,39 +73,47 @@ __global__ void __launch_bounds__(256) perm_scatter_kernel(
   const uint32_t row_bytes = (uint32_t)d * (uint32_t)sizeof(Tin);
   unsigned char *rows = sm_raw;
   unsigned *smask = (unsigned *)(sm_raw + (size_t)PM_TPC * row_bytes);
+  int *s_base = (int *)(smask + E);  // this chunk's per-expert base rank and the expert offsets,
+  int *s_off = s_base + E;           // loaded alongside the routing, not after it
   const int tfirst = chunk * PM_CHUNK + part * PM_TPC;
   const int nrows = max(0, min(PM_TPC, T - tfirst));
   const bool copy = x_perm != nullptr && nrows > 0;
   const uint32_t bar = smem_u32(&s_bar);
-  if (tid == 0) {
+  if (tid == 0) {  // the rows do not depend on the routing: their copies go out first
     s_abort = 0;
     mbar_init(bar, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    if (copy) {
+      mbar_expect_tx(bar, (uint32_t)nrows * row_bytes);
+      for (int r = 0; r < nrows; ++r)
+        bulk_load_1d(smem_u32(rows + (size_t)r * row_bytes), x + (size_t)(tfirst + r) * d,
+                     row_bytes, bar);
+    }
   }
-  __syncthreads();  // the barrier is initialised before anyone waits on it
-  if (tid == 0 && copy) {
-    mbar_expect_tx(bar, (uint32_t)nrows * row_bytes);
-    for (int r = 0; r < nrows; ++r)
-      bulk_load_1d(smem_u32(rows + (size_t)r * row_bytes), x + (size_t)(tfirst + r) * d,
-                   row_bytes, bar);
-  }
+  // warp 0 reads the chunk's routing while the other warps read the bases and offsets
+  const int t = chunk * PM_CHUNK + lane;
+  int ev[8];
   if (warp == 0) {
-    const int t = chunk * PM_CHUNK + lane;
-    for (int e = lane; e < E; e += 32) smask[e] = 0u;
-    __syncwarp();
     const bool valid = active && t < T;
-    int ev[8];
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
       ev[j] = -1;
       if (j < k && valid) {
         const int e = idx[(size_t)t * k + j];
-        if (e >= 0 && e < E) {
-          ev[j] = e;
-          atomicOr(&smask[e], 1u << lane);
-        }
+        if (e >= 0 && e < E) ev[j] = e;
       }
     }
+  }
+  for (int e = tid; e < E; e += blockDim.x) {
+    smask[e] = 0u;
+    s_base[e] = chunk_base[(size_t)chunk * E + e];
+    s_off[e] = offsets[e];
+  }
+  __syncthreads();  // the barrier is initialised, masks cleared, bases and offsets in place
+  if (warp == 0) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      if (ev[j] >= 0) atomicOr(&smask[ev[j]], 1u << lane);
     __syncwarp();
     const unsigned lt = lanemask_lt();
 #pragma unroll
@@ -112,8 +122,8 @@ __global__ void __launch_bounds__(256) perm_scatter_kernel(
         int pos = -1;
         const int e = ev[j];
         if (e >= 0) {
-          const int rank = chunk_base[(size_t)chunk * E + e] + __popc(smask[e] & lt);
-          if (C < 0 || rank < C) pos = offsets[e] + rank;
+          const int rank = s_base[e] + __popc(smask[e] & lt);
+          if (C < 0 || rank < C) pos = s_off[e] + rank;
           if (part == 0) {
             slot_pos[(size_t)t * k + j] = pos;
             if (pos >= 0) src[pos] = t;
