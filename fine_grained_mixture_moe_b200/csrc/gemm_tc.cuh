@@ -36,6 +36,7 @@ struct TcMaps {
 struct TcParams {
   TcMaps maps;
   GroupedGemm p;
+  int stages;  // CTA-pair kernel: operand pipeline depth chosen from the group count
 };
 
 template <int MODE, int BN> struct TcCfg {

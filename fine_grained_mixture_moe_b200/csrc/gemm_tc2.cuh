@@ -63,9 +63,8 @@ template <int MODE> struct Tc2Cfg {
   static constexpr int A_BYTES = 128 * TC_BK * 2;             // this CTA's 128 rows
   static constexpr int B_BYTES = 128 * TC_BK * 2;             // this CTA's half of B
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;       // 32 KB
-  static constexpr int STG_BYTES = MODE == MODE_PLAIN ? TC_EPI_WARPS * 4096 : 0;
-  static constexpr int STAGES = (200 * 1024 - STG_BYTES) / STAGE_BYTES > 8
-                                    ? 8 : (200 * 1024 - STG_BYTES) / STAGE_BYTES;
+  static constexpr int STG_BYTES = TC_EPI_WARPS * 4096;  // per-warp epilogue staging
+  static constexpr int MAX_STAGES = 8;
   static constexpr int ACC_COLS = MMA_N;
   static constexpr int TMEM_COLS = 512;
   static constexpr uint32_t IDESC = (1u << 4) | (1u << 7) | (1u << 10) |
@@ -73,11 +72,20 @@ template <int MODE> struct Tc2Cfg {
                                     ((uint32_t)(TC2_BM >> 4) << 24);
 };
 
-template <int MODE>
-__host__ __device__ constexpr size_t tc2_smem_bytes(int G) {
-  using C = Tc2Cfg<MODE>;
-  return 1024 + (size_t)C::STAGES * C::STAGE_BYTES + C::STG_BYTES + 256 +
+// Shared memory beside the operand stages: alignment pad, staging, barriers, tile list.
+template <int MODE> constexpr size_t tc2_fixed_bytes(int G) {
+  return 1024 + (size_t)Tc2Cfg<MODE>::STG_BYTES + 256 +
          (size_t)(G + 1 + TC_THREADS / 32 + 1) * sizeof(int);
+}
+// Operand stages that fit in the 227 KB a CTA may hold (at most MAX_STAGES; < 2 means the tile
+// list of G groups leaves no room for double buffering).
+template <int MODE> constexpr int tc2_stages(int G) {
+  const long long room = 227LL * 1024 - (long long)tc2_fixed_bytes<MODE>(G);
+  const long long n = room < 0 ? 0 : room / Tc2Cfg<MODE>::STAGE_BYTES;
+  return n > Tc2Cfg<MODE>::MAX_STAGES ? Tc2Cfg<MODE>::MAX_STAGES : (int)n;
+}
+template <int MODE> constexpr size_t tc2_smem_bytes(int G) {
+  return tc2_fixed_bytes<MODE>(G) + (size_t)tc2_stages<MODE>(G) * Tc2Cfg<MODE>::STAGE_BYTES;
 }
 
 template <int MODE>
@@ -91,26 +99,27 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TC_THREADS, 1)
   const int G = p.E + p.has_shared;
   const uint32_t rank = cluster_ctarank();
   const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+  const int NST = P.stages;  // operand stages (2..MAX_STAGES), fixed by the host from G
 
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t pad = ((raw + 1023u) & ~1023u) - raw;
   unsigned char *base = smem_raw + pad;
   unsigned char *stages = base;
-  unsigned char *stg_all = base + (size_t)C::STAGES * C::STAGE_BYTES;
+  unsigned char *stg_all = base + (size_t)NST * C::STAGE_BYTES;
   uint64_t *bars = (uint64_t *)(stg_all + C::STG_BYTES);
-  uint32_t *tmem_slot = (uint32_t *)(bars + 2 * C::STAGES + 5);
+  uint32_t *tmem_slot = (uint32_t *)(bars + 2 * NST + 5);
   volatile int *abort_flag = (volatile int *)(tmem_slot + 1);
   int *prefix = (int *)(stg_all + C::STG_BYTES + 256);
   int *scan_tmp = prefix + G + 1;
 
   auto full_bar = [&](int s) { return smem_u32(bars + s); };
-  auto empty_bar = [&](int s) { return smem_u32(bars + C::STAGES + s); };
-  auto accf_bar = [&](int b) { return smem_u32(bars + 2 * C::STAGES + b); };
-  auto acce_bar = [&](int b) { return smem_u32(bars + 2 * C::STAGES + 2 + b); };
-  const uint32_t drain_bar = smem_u32(bars + 2 * C::STAGES + 4);
+  auto empty_bar = [&](int s) { return smem_u32(bars + NST + s); };
+  auto accf_bar = [&](int b) { return smem_u32(bars + 2 * NST + b); };
+  auto acce_bar = [&](int b) { return smem_u32(bars + 2 * NST + 2 + b); };
+  const uint32_t drain_bar = smem_u32(bars + 2 * NST + 4);
 
   if (tid == 0) {
-    for (int s = 0; s < C::STAGES; ++s) {
+    for (int s = 0; s < NST; ++s) {
       mbar_init(full_bar(s), 1);
       mbar_init(empty_bar(s), 1);
     }
@@ -145,9 +154,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TC_THREADS, 1)
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
-      int issued_parity[8];
-      bool issued[8];
-      for (int s = 0; s < 8; ++s) { issued[s] = false; issued_parity[s] = 0; }
+      int issued_parity[C::MAX_STAGES];
+      bool issued[C::MAX_STAGES];
+      for (int s = 0; s < C::MAX_STAGES; ++s) { issued[s] = false; issued_parity[s] = 0; }
       for (int tile = pair; tile < total && ok; tile += npairs) {
         const TileInfo ti = decode_tile(p, tile, prefix, TC2_BM, BN);
         const bool routed = ti.g < p.E;
@@ -180,11 +189,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TC_THREADS, 1)
           tma_load_2d_pair(sB, mb, b_col, b_row, full_bar(stage));
           issued[stage] = true;
           issued_parity[stage] = (int)phase;
-          if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
+          if (++stage == NST) { stage = 0; phase ^= 1u; }
         }
       }
       if (!ok && rank == 0) {
-        for (int s = 0; s < C::STAGES; ++s)
+        for (int s = 0; s < NST; ++s)
           if (issued[s]) {
             volatile int never = 0;
             mbar_wait(full_bar(s), (uint32_t)issued_parity[s], &never, limit, INFO_WAIT_DRAIN);
@@ -224,7 +233,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TC_THREADS, 1)
           }
           any = true;
           tc2_commit_both(empty_bar(stage));
-          if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
+          if (++stage == NST) { stage = 0; phase ^= 1u; }
         }
         if (!ok) break;
         tc2_commit_both(accf_bar(acc));
@@ -263,40 +272,75 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TC_THREADS, 1)
 #pragma unroll 1
       for (int c = cbeg; c < cend; c += 32) {
         if (MODE == MODE_GATEUP) {
-          uint32_t r0[32], r1[32];
-          tmem_ld32(tbase + c, r0);
-          tmem_ld32(tbase + BN + c, r1);
-          tmem_wait_ld();
-          const int col = ti.n0 + c;
-          if (row_ok && col < ti.N) {
-            uint4 pk[4];
-            __nv_bfloat162 *h = (__nv_bfloat162 *)pk;
+          // silu(gate) * up in bf16, 64 columns (128 bytes of each row) at a time: both 32-column
+          // halves are packed, staged per warp and written as 32 coalesced 128-byte row stores
+          if ((c - cbeg) & 32) continue;  // the odd 32-column steps were taken with the even ones
+          uint32_t pk[32];
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh) {
+            uint32_t r0[32], r1[32];
+            tmem_ld32(tbase + c + 32 * hh, r0);
+            tmem_ld32(tbase + BN + c + 32 * hh, r1);
+            tmem_wait_ld();
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
               const float g0 = __uint_as_float(r0[2 * i]), g1 = __uint_as_float(r0[2 * i + 1]);
-              h[i] = __floats2bfloat162_rn(__fdividef(g0, 1.0f + __expf(-g0)) * __uint_as_float(r1[2 * i]),
-                                           __fdividef(g1, 1.0f + __expf(-g1)) * __uint_as_float(r1[2 * i + 1]));
+              __nv_bfloat162 h = __floats2bfloat162_rn(
+                  __fdividef(g0, 1.0f + __expf(-g0)) * __uint_as_float(r1[2 * i]),
+                  __fdividef(g1, 1.0f + __expf(-g1)) * __uint_as_float(r1[2 * i + 1]));
+              pk[16 * hh + i] = *(uint32_t *)&h;
             }
-            uint4 *dst = (uint4 *)((__nv_bfloat16 *)out + (size_t)(ti.a_row0 + row) * ldo + col);
-#pragma unroll
-            for (int i = 0; i < 4; ++i) dst[i] = pk[i];
           }
-        } else if (routed && p.out_r_bf16) {
-          // routed expert outputs in bf16: 64 contiguous bytes of the lane's row, stored directly
-          uint32_t r0[32];
-          tmem_ld32(tbase + c, r0);
-          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            *(uint4 *)(stg + lane * 128 + ((i ^ (lane & 7)) << 4)) =
+                make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+          __syncwarp();
           const int col = ti.n0 + c;
-          if (row_ok && col < ti.N) {
-            uint4 pk[4];
-            __nv_bfloat162 *h = (__nv_bfloat162 *)pk;
-#pragma unroll
-            for (int i = 0; i < 16; ++i)
-              h[i] = __floats2bfloat162_rn(__uint_as_float(r0[2 * i]), __uint_as_float(r0[2 * i + 1]));
-            uint4 *dst = (uint4 *)((__nv_bfloat16 *)out + (size_t)(ti.a_row0 + row) * ldo + col);
-#pragma unroll
-            for (int i = 0; i < 4; ++i) dst[i] = pk[i];
+          if (col < ti.N) {
+            const int nrows = min(32, ti.rows - rbase);
+            unsigned char *obase = (unsigned char *)out + ((size_t)(ti.a_row0 + rbase) * ldo + col) * 2;
+            const size_t row_bytes = (size_t)ldo * 2;
+            for (int rr = 0; rr < nrows; ++rr) {
+              const uint32_t v = *(const uint32_t *)(stg + rr * 128 +
+                                                     (((lane >> 2) ^ (rr & 7)) << 4) + ((lane & 3) << 2));
+              *(uint32_t *)(obase + rr * row_bytes + lane * 4) = v;
+            }
           }
+          __syncwarp();
+        } else if (routed && p.out_r_bf16) {
+          // routed expert outputs in bf16, 64 columns (128 bytes of each row) at a time: staged
+          // per warp like the fp32 path and written as 32 coalesced 128-byte row stores
+          if ((c - cbeg) & 32) continue;  // the odd 32-column steps were taken with the even ones
+          uint32_t r0[32], r1[32];
+          tmem_ld32(tbase + c, r0);
+          tmem_ld32(tbase + c + 32, r1);
+          tmem_wait_ld();
+          uint32_t pk[32];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            __nv_bfloat162 a = __floats2bfloat162_rn(__uint_as_float(r0[2 * i]), __uint_as_float(r0[2 * i + 1]));
+            __nv_bfloat162 b = __floats2bfloat162_rn(__uint_as_float(r1[2 * i]), __uint_as_float(r1[2 * i + 1]));
+            pk[i] = *(uint32_t *)&a;
+            pk[16 + i] = *(uint32_t *)&b;
+          }
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            *(uint4 *)(stg + lane * 128 + ((i ^ (lane & 7)) << 4)) =
+                make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+          __syncwarp();
+          const int col = ti.n0 + c;
+          if (col < ti.N) {
+            const int nrows = min(32, ti.rows - rbase);
+            unsigned char *obase = (unsigned char *)out + ((size_t)(ti.a_row0 + rbase) * ldo + col) * 2;
+            const size_t row_bytes = (size_t)ldo * 2;
+            for (int rr = 0; rr < nrows; ++rr) {
+              const uint32_t v = *(const uint32_t *)(stg + rr * 128 +
+                                                     (((lane >> 2) ^ (rr & 7)) << 4) + ((lane & 3) << 2));
+              *(uint32_t *)(obase + rr * row_bytes + lane * 4) = v;
+            }
+          }
+          __syncwarp();
         } else {
           // fp32 output, staged per warp and written as 128-byte rows
           uint32_t r0[32];

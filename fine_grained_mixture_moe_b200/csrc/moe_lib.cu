@@ -306,6 +306,9 @@ moe_status_t launch_tc2(const GroupedGemm &g, cudaStream_t st, int kind) {
   P.p = g;
   if (!build_maps(g, MODE == MODE_GATEUP, 128, &P.maps)) return MOE_ERR_CUDA;
   const int G = g.E + g.has_shared;
+  static_assert(tc2_stages<MODE>(1024 + 1) >= 2, "tile list of 1024 experts leaves no room");
+  P.stages = tc2_stages<MODE>(G);
+  if (P.stages < 2) return MOE_ERR_UNSUPPORTED;
   const size_t smem = tc2_smem_bytes<MODE>(G);
   auto kern = gemm_tc2_kernel<MODE>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
