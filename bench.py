@@ -169,7 +169,6 @@ def algorithmic(c, n_kept: int):
     es = 2 if c.dtype == "bf16" else 4
     out = {}
     out["router"] = {"flops": 2.0 * T * d * E, "bytes": T * d * es + E * d * es + 8.0 * T * k}
-    out["router_prep"] = {"bytes": E * d * (es + 8.0)}
     perm_bytes = T * d * es + n_kept * d * es + 16.0 * T * k
     out["perm_scatter"] = {"bytes": perm_bytes}
     if c.expert == "swiglu":
@@ -193,7 +192,8 @@ def algorithmic(c, n_kept: int):
 def roofline_table(c, n_kept, prof, steps, peaks, src):
     """Achieved vs peak per kernel kind from the profiler's per-launch averages."""
     alg = algorithmic(c, n_kept)
-    fp64_peak = 148 * 64 * 2 * peaks.get("sm_max_mhz", 1965.0) * 1e6 / 1e12  # TFLOP/s, nominal
+    # fp32 FMA on the CUDA cores: 148 SMs x 128 lanes x 2 flops at the maximum SM clock
+    fp32_peak = 148 * 128 * 2 * peaks.get("sm_max_mhz", 1965.0) * 1e6 / 1e12  # TFLOP/s, nominal
     rows = {}
     for name, (ms, n) in prof.items():
         if n == 0:
@@ -207,8 +207,8 @@ def roofline_table(c, n_kept, prof, steps, peaks, src):
                        frac=ach / peaks["bf16_tflops"])
         elif name == "router":
             ach = a["flops"] / (avg_ms * 1e-3) / 1e12
-            row.update(bound="alu", achieved=ach, peak=fp64_peak, unit="TFLOP/s (fp64 FMA)",
-                       frac=ach / fp64_peak,
+            row.update(bound="alu", achieved=ach, peak=fp32_peak, unit="TFLOP/s (fp32 FMA)",
+                       frac=ach / fp32_peak,
                        hbm_gbs=a["bytes"] / (avg_ms * 1e-3) / 1e9)
         elif "bytes" in a:
             ach = a["bytes"] / (avg_ms * 1e-3) / 1e9

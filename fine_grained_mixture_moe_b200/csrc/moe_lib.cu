@@ -44,7 +44,7 @@ bool cfg_supported(const moe_config_t *c) {
   if (c->n_shared > 0 && (c->ffn_shared <= 0 || c->ffn_shared % 64)) return false;
   if (!std::isfinite(c->capacity_factor) || !std::isfinite(c->aux_alpha)) return false;
   // the router stages its 16 token rows and the logits in shared memory (227 KB per CTA)
-  if (router_smem(c->E, router_nt_for(c->E), c->score == MOE_SCORE_SIGMOID, c->d,
+  if (router_smem(c->E, c->score == MOE_SCORE_SIGMOID, c->d,
                   c->dtype == MOE_DTYPE_BF16 ? 2 : 4).total > 227 * 1024)
     return false;
   // 32-bit row indices inside the kernels
@@ -352,25 +352,15 @@ moe_status_t launch_gemm(const moe_config_t *c, const GroupedGemm &g, int bn_hin
     if (_s != MOE_OK) return _s;        \
   } while (0)
 
-template <typename Tin, int NT>
-moe_status_t launch_router_nt(const RouterArgs &a, cudaStream_t st) {
-  const size_t smem = router_smem(a.E, NT, a.score == MOE_SCORE_SIGMOID, a.d, (int)sizeof(Tin)).total;
-  if (smem > 227 * 1024) return MOE_ERR_UNSUPPORTED;
-  if (cudaFuncSetAttribute(router_kernel<Tin, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)smem) != cudaSuccess)
-    return MOE_ERR_CUDA;
-  return launch_pdl(router_kernel<Tin, NT>, dim3(ceil_div(a.T, RT_TM)), dim3(RT_THREADS), smem, st, a);
-}
-
 template <typename Tin>
 moe_status_t launch_router(const RouterArgs &a, cudaStream_t st) {
   ProfScope ps(K_ROUTER, st);
-  switch (router_nt_for(a.E)) {
-    case 1: return launch_router_nt<Tin, 1>(a, st);
-    case 2: return launch_router_nt<Tin, 2>(a, st);
-    case 3: return launch_router_nt<Tin, 3>(a, st);
-    default: return launch_router_nt<Tin, 4>(a, st);
-  }
+  const size_t smem = router_smem(a.E, a.score == MOE_SCORE_SIGMOID, a.d, (int)sizeof(Tin)).total;
+  if (smem > 227 * 1024) return MOE_ERR_UNSUPPORTED;
+  if (cudaFuncSetAttribute(router_kernel<Tin>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)smem) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  return launch_pdl(router_kernel<Tin>, dim3(ceil_div(a.T, RT_TM)), dim3(RT_THREADS), smem, st, a);
 }
 
 moe_status_t launch_stats(const StatsArgs &sa, cudaStream_t st) {

@@ -7,58 +7,42 @@
 //   top-k by key, ties -> lower expert index, slot order = descending key
 //   weights = softmax over all E (or sigmoid) of the selected experts, optional renormalise
 //
-// How: the dot products run on the fp64 tensor pipe (mma.sync m8n8k4). bf16 and fp32 inputs
-// multiply exactly in fp64, so the only error is the summation. Each logit is then decided one
-// of three ways, all exact:
-//   1. certificate: when every product is a multiple of 2^q (from the rows' smallest exponents)
-//      and the Cauchy-Schwarz bound on every partial sum is below 2^(q+53), the fp64 sum *is*
-//      the exact sum and its round-to-nearest-even is the logit. This covers the exact ties that
-//      bf16 data produce often (~0.8% of logits land exactly on an fp32 rounding midpoint);
-//   2. enclosure: the error bound (d+16) 2^-52 (|x|_2 |W_e|_2 + |off|) leaves no fp32 rounding
-//      boundary inside the interval, so RN32 of the fp64 value is the exact rounding;
-//   3. otherwise (2 in 98,304 Quartz logits) a whole warp decides it after the main pass: it
-//      scales every exact product to an integer multiple of the smallest power of two present,
-//      sums them in int64, exactly, and compares with the boundaries. Only when the exponent span
-//      exceeds 50 bits (or in a forced test mode) does one thread sum the products as a
-//      non-overlapping floating-point expansion (Shewchuk's Grow-Expansion with zero
-//      elimination) and decide from its sign.
-// Sigmoid keys are screened the same way (fp64 exp within its documented error) and resolved
-// in double-double arithmetic. So the integer routing decisions are exact, not merely tolerant.
+// How. The integer results (which experts, in which slot order) depend only on the order of the
+// k+1 largest canonical keys, so the kernel computes every logit approximately and proves the
+// order, falling back to exact arithmetic only where the proof fails:
+//   1. screen: fp32 dot products on the CUDA cores with packed two-lane fused multiply-adds.
+//      A product is exact inside its FMA, so each term passes through at most
+//      m = 4 ceil(d/128) + 10 roundings and |l~ - l| <= gamma_m (|x_t|_2 max_e |W_e|_2 + max|off|)
+//      =: B_t for every expert of token t (norms from fp32 sums of squares, bounded above);
+//   2. proof: if each of the k gaps between consecutive keys of the approximate top k+1 exceeds
+//      twice the key bound plus two fp32 steps, the canonical keys of those k+1 experts lie in
+//      the same strict order and above every other expert's, so the approximate selection is
+//      the exact one;
+//   3. otherwise (about 1% of Quartz tokens) every expert whose key could still reach the top k
+//      (within that margin of the (k+1)-th key) gets its canonical logit: an fp64 sum of the exact
+//      products (error <= (d+16) 2^-52 (|x||W_e| + |off|)) rounded directly when no fp32 rounding
+//      boundary lies inside the error, else decided by an exact integer comparison with the
+//      boundaries (or, for exponent spans beyond 50 bits, a floating-point expansion). The other
+//      experts provably stay below the k-th canonical key, and selection reruns on the mix.
+// Sigmoid keys are screened from the approximate logit (sigmoid is 1/4-Lipschitz) and, for the
+// candidates of step 3, resolved exactly in double-double. Combine weights and probability sums
+// use the logits as computed: within B_t of canonical, far inside their tolerance.
 #pragma once
 #include "common.cuh"
 
 namespace moe {
 
 constexpr int RT_TM = 16;          // tokens per CTA
-constexpr int RT_MT = RT_TM / 8;   // fp64 MMA row tiles per warp (each W fragment feeds all)
-constexpr int RT_WARPS = 8;        // each a slice of the K dimension
+constexpr int RT_WARPS = 8;        // each takes every 8th slice of the d dimension
 constexpr int RT_THREADS = 32 * RT_WARPS;
-constexpr int RT_KB = 16;          // k block: lane (row r, column c) of a fragment reads the 4
-                                   // consecutive elements 4c..4c+3 of the block with one load
+// Screen tiling. Lane = ks + 2 (eg + 8 tg): tg in {0,1} picks tokens tg, tg+2, ..., tg+14;
+// eg in 0..7 picks experts eg, eg+8, eg+16 of the round; ks in {0,1} halves the warp's d slice.
+constexpr int RT_TPT = 8;          // tokens per thread
+constexpr int RT_EPT = 3;          // experts per thread
+constexpr int RT_EB = 8 * RT_EPT;  // experts per round
 constexpr int RT_SEL_THREAD_MAX_E = 64;  // up to this many experts: one thread per (token,
-                                         // expert) finds its rank; above, a warp per token
+                                         // expert) ranks; above, a warp per token
 constexpr int EXPANSION_MAX = 40;
-constexpr int RT_FIX_CAP = 256;   // flagged logits per CTA kept with their fp64 sums
-
-// Expert tiles of 8 per round (a round covers 8*NT experts): the NT in {4,3,2,1} that wastes the
-// fewest padded expert slots over all rounds, larger NT on ties.
-inline int router_nt_for(int E) {
-  int best = 4, waste = 1 << 30;
-  for (int nt : {4, 3, 2, 1}) {
-    const int eb = 8 * nt, w = ((E + eb - 1) / eb) * eb - E;
-    if (w < waste) { waste = w; best = nt; }
-  }
-  return best;
-}
-
-// D(8x8) += A(8x4) B(4x8) in fp64 on the tensor cores. Fragments: lane l holds A[l/4][l%4],
-// B[l%4][l/4] and D[l/4][2(l%4) + {0,1}]. Every product of bf16 or fp32 inputs is exact in fp64
-// and each accumulation is an fp64 rounding, so the summation error bound below still holds.
-__device__ __forceinline__ void dmma_8x8x4(double (&d)[2], double a, double b) {
-  asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0, %1}, {%2}, {%3}, {%0, %1};"
-               : "+d"(d[0]), "+d"(d[1])
-               : "d"(a), "d"(b));
-}
 
 struct RouterArgs {
   const void *x;
@@ -73,6 +57,46 @@ struct RouterArgs {
   int32_t *count_out;   // [E]
   float *prob_out;      // [E]
   unsigned int *counter; // completion counter of the statistics kernel, cleared here
+};
+
+// Eight consecutive elements (bf16: 16 bytes; fp32: 32 bytes) and their pairs as fp32.
+template <typename Tin> struct Chunk8;
+template <> struct Chunk8<__nv_bfloat16> {
+  static constexpr int PARTS = 1;  // 16-byte parts
+  uint4 q;
+  __device__ __forceinline__ void ld_s(const __nv_bfloat16 *p) { q = *(const uint4 *)p; }
+  __device__ __forceinline__ void ld(const __nv_bfloat16 *p) { q = *(const uint4 *)p; }  // any space
+  __device__ __forceinline__ void ld_g(const __nv_bfloat16 *p) { q = __ldg((const uint4 *)p); }
+  __device__ __forceinline__ void zero() { q = make_uint4(0u, 0u, 0u, 0u); }
+  // parts `stride` uint4s apart (the ring layout)
+  __device__ __forceinline__ void ld_ring(const uint4 *p, int) { q = *p; }
+  // elements 2i and 2i+1, widened exactly (a bf16 is the upper half of an fp32)
+  __device__ __forceinline__ float2 pair(int i) const {
+    const uint32_t w = i == 0 ? q.x : (i == 1 ? q.y : (i == 2 ? q.z : q.w));
+    return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+  }
+};
+template <> struct Chunk8<float> {
+  static constexpr int PARTS = 2;
+  float4 a, b;
+  __device__ __forceinline__ void ld_s(const float *p) {
+    a = ((const float4 *)p)[0];
+    b = ((const float4 *)p)[1];
+  }
+  __device__ __forceinline__ void ld(const float *p) { ld_s(p); }  // any space
+  __device__ __forceinline__ void ld_g(const float *p) {
+    a = __ldg((const float4 *)p);
+    b = __ldg((const float4 *)p + 1);
+  }
+  __device__ __forceinline__ void zero() { a = b = make_float4(0.f, 0.f, 0.f, 0.f); }
+  __device__ __forceinline__ void ld_ring(const uint4 *p, int stride) {
+    a = *(const float4 *)p;
+    b = *(const float4 *)(p + stride);
+  }
+  __device__ __forceinline__ float2 pair(int i) const {
+    return i == 0 ? make_float2(a.x, a.y)
+                  : (i == 1 ? make_float2(a.z, a.w) : (i == 2 ? make_float2(b.x, b.y) : make_float2(b.z, b.w)));
+  }
 };
 
 // ------------------------------------------------------------------ exact expansion sums
@@ -246,14 +270,33 @@ __device__ bool warp_exact_signs(const Tin *xrow, const Tin *wrow, int d, double
     qmin = min(qmin, lsb);
     emax = max(emax, lead);
   };
-  // lane covers elements [8*lane + 256*j, +8): d is a multiple of 64, so a chunk never straddles d
-  for (int i = 8 * lane; i < d; i += 256) {
-    double xv[8], wv[8];
-    load8(xrow + i, xv);
-    load8(wrow + i, wv);
+  // lane covers elements [8*lane + 256*j, +8): d is a multiple of 64, so a chunk never straddles
+  // d. Four chunks of each row are requested together; the products of bf16 or fp32 values are
+  // exact in fp64.
+  auto for_products = [&](auto &&fn) {
+    for (int i0 = 8 * lane; i0 < d; i0 += 4 * 256) {
+      Chunk8<Tin> xq[4], wq[4];
 #pragma unroll
-    for (int u = 0; u < 8; ++u) scan(__dmul_rn(xv[u], wv[u]));
-  }
+      for (int u = 0; u < 4; ++u) {
+        if (i0 + 256 * u < d) {
+          xq[u].ld(xrow + i0 + 256 * u);
+          wq[u].ld(wrow + i0 + 256 * u);
+        } else {
+          xq[u].zero();
+          wq[u].zero();
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+#pragma unroll
+        for (int p = 0; p < 4; ++p) {
+          const float2 xf = xq[u].pair(p), wf = wq[u].pair(p);
+          fn(__dmul_rn((double)xf.x, (double)wf.x));
+          fn(__dmul_rn((double)xf.y, (double)wf.y));
+        }
+    }
+  };
+  for_products(scan);
   if (lane == 0) {
     scan(off);
     scan(mh);
@@ -267,13 +310,7 @@ __device__ bool warp_exact_signs(const Tin *xrow, const Tin *wrow, int d, double
   bad = __any_sync(0xffffffffu, bad);
   if (bad || emax - qmin > 50) return false;
   long long acc = 0;
-  for (int i = 8 * lane; i < d; i += 256) {
-    double xv[8], wv[8];
-    load8(xrow + i, xv);
-    load8(wrow + i, wv);
-#pragma unroll
-    for (int u = 0; u < 8; ++u) acc += (long long)ldexp(__dmul_rn(xv[u], wv[u]), -qmin);
-  }
+  for_products([&](double v) { acc += (long long)ldexp(v, -qmin); });
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
   acc += (long long)ldexp(off, -qmin);
@@ -369,90 +406,37 @@ __device__ __forceinline__ float sigmoid_key(float l, float b, bool force) {
   return sigmoid_key_exact(l, b, r, up, dn, mh, ml);
 }
 
-// ------------------------------------------------------------------ kernels
+// ------------------------------------------------------------------ kernel
+constexpr int RT_WD = 4;  // W chunks in flight per lane pair (cp.async ring)
+
 // Shared-memory layout of the router kernel (byte offsets), shared by host and device.
 struct RouterSmem {
-  size_t xs, xs_stride, part, sq, ex, lg, pb, keys, sel_e, sel_p, wn, wexp, cnt, flags, xnorm,
-      xexp, fix, total;
+  size_t xs, xs_stride, ring, part, wsq, wn, off, lg, keys, byrank, cnt, xnorm, cmask, total;
 };
-__host__ __device__ inline RouterSmem router_smem(int E, int NT, bool sigmoid, int d, int esize) {
+__host__ __device__ inline RouterSmem router_smem(int E, bool sigmoid, int d, int esize) {
   RouterSmem L;
-  const int EB = 8 * NT;
   size_t o = 0;
   auto take = [&](size_t bytes) { size_t at = o; o = (o + bytes + 15) & ~(size_t)15; return at; };
-  // the CTA's token rows, each padded by 32 bytes so that the 8 rows of an MMA fragment fall
-  // on distinct bank pairs
+  // the CTA's token rows, each padded by 32 bytes: the rows tg, tg+2, ... that a warp reads in
+  // one instruction then start 32 bytes apart in the banks
   L.xs_stride = (size_t)d * esize + 32;
   L.xs = take((size_t)RT_TM * L.xs_stride);
-  L.part = take((size_t)RT_WARPS * RT_TM * EB * sizeof(double));   // per-warp partial sums
-  L.sq = take((size_t)RT_WARPS * (EB + RT_TM) * sizeof(double));   // per-warp sums of squares
-  L.ex = take((size_t)RT_WARPS * (EB + RT_TM) * 2 * sizeof(int));  // per-warp exponent ranges
+  // rings of W chunks, one per lane pair (lanes tg = 0, 1 use the same chunks):
+  // [slot][expert][16-byte part][pair]
+  L.ring = take((size_t)RT_WD * RT_EPT * (RT_THREADS / 2) * 8 * esize);
+  L.part = take((size_t)RT_WARPS * RT_TM * RT_EB * sizeof(float));  // per-warp partial logits
+  L.wsq = take((size_t)RT_WARPS * RT_EB * sizeof(float));           // per-warp W sums of squares
+  L.wn = take((size_t)E * sizeof(double));
+  L.off = take((size_t)E * sizeof(float));
   L.lg = take((size_t)RT_TM * E * sizeof(float));
-  const bool rank_sel = E <= RT_SEL_THREAD_MAX_E;
-  L.pb = take(rank_sel ? (size_t)RT_TM * E * sizeof(float) : 0);
-  L.keys = take(sigmoid ? (size_t)(rank_sel ? RT_TM : RT_WARPS) * E * sizeof(float) : 0);
-  L.sel_e = take((size_t)RT_TM * 8 * sizeof(int));
-  L.sel_p = take((size_t)RT_TM * 8 * sizeof(float));
-  L.wn = take((size_t)EB * sizeof(double));
-  L.wexp = take((size_t)EB * 2 * sizeof(int));
+  L.keys = take(sigmoid ? (size_t)RT_TM * E * sizeof(float) : 0);
+  L.byrank = take((size_t)RT_WARPS * 9 * sizeof(int));
   L.cnt = take((size_t)E * sizeof(int));
-  L.flags = take((size_t)RT_TM * ((E + 31) / 32) * sizeof(unsigned));
   L.xnorm = take(RT_TM * sizeof(double));
-  L.xexp = take(RT_TM * 2 * sizeof(int));
-  L.fix = take(RT_FIX_CAP * sizeof(double));
+  L.cmask = take((size_t)RT_TM * ((E + 31) / 32) * sizeof(unsigned));  // candidates per listed token
   L.total = o;
   return L;
 }
-
-// Raw 4-element fragment loads (bf16: 8 bytes; fp32: 16 bytes) and their conversion to fp64.
-// Fragment digest: the four raw elements a lane loads per 16-k block become (1) fp64 MMA
-// operands (a bf16 widens exactly to fp32 by a shift, then to fp64 by the conversion
-// instruction), (2) an fp32 running sum of squares for the norm bound, (3) the running min / max
-// magnitude key (the element's bits without the sign: key >> MANT is the biased exponent) over
-// the nonzero elements, for the exactness certificate.
-template <typename Tin> struct Frag4;
-template <> struct Frag4<__nv_bfloat16> {
-  using raw_t = uint2;
-  static constexpr int MANT = 7;  // fraction bits
-  static __device__ __forceinline__ raw_t load(const __nv_bfloat16 *p) { return __ldg((const uint2 *)p); }
-  static __device__ __forceinline__ raw_t load_s(const __nv_bfloat16 *p) { return *(const uint2 *)p; }
-  static __device__ __forceinline__ raw_t zero() { return make_uint2(0u, 0u); }
-  static __device__ __forceinline__ void digest(raw_t q, double (&v)[4], float &sq, uint32_t &mn,
-                                                uint32_t &mx) {
-    const uint32_t w[2] = {q.x, q.y};
-#pragma unroll
-    for (int i = 0; i < 2; ++i)
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const uint32_t b = h ? (w[i] >> 16) : (w[i] & 0xFFFFu);
-        const uint32_t m = b & 0x7FFFu;
-        const float f = __uint_as_float(b << 16);
-        sq = fmaf(f, f, sq);
-        mn = min(mn, m ? m : 0xFFFFFFFFu);
-        mx = max(mx, m);
-        v[2 * i + h] = (double)f;
-      }
-  }
-};
-template <> struct Frag4<float> {
-  using raw_t = float4;
-  static constexpr int MANT = 23;
-  static __device__ __forceinline__ raw_t load(const float *p) { return __ldg((const float4 *)p); }
-  static __device__ __forceinline__ raw_t load_s(const float *p) { return *(const float4 *)p; }
-  static __device__ __forceinline__ raw_t zero() { return make_float4(0.f, 0.f, 0.f, 0.f); }
-  static __device__ __forceinline__ void digest(raw_t q, double (&v)[4], float &sq, uint32_t &mn,
-                                                uint32_t &mx) {
-    const float f[4] = {q.x, q.y, q.z, q.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      v[i] = f[i];
-      sq = fmaf(f[i], f[i], sq);
-      const uint32_t m = __float_as_uint(f[i]) & 0x7FFFFFFFu;
-      mn = min(mn, m ? m : 0xFFFFFFFFu);
-      mx = max(mx, m);
-    }
-  }
-};
 
 // Upper bound on sqrt(sum of squares) from an fp32 accumulation of at most n = d + 16 fused
 // multiply-adds and additions: each step rounds with relative error <= 2^-24 or, in the
@@ -463,14 +447,85 @@ __device__ __forceinline__ double norm_upper(double computed, int d) {
   return sqrt((computed + n * 0x1p-149) * (1.0 + n * 0x1p-23));
 }
 
-template <typename Tin, int NT>
+__device__ __forceinline__ double sigmoid64(float l) { return 1.0 / (1.0 + exp(-(double)l)); }
+
+// The n largest keys of a row (NaN as -infinity; equal keys: lower index first) into sel[0..n).
+__device__ __forceinline__ void warp_topn(const float *krow, int E, int n, int (&sel)[9]) {
+  const int lane = threadIdx.x & 31;
+  unsigned selmask = 0u;
+#pragma unroll
+  for (int j = 0; j < 9; ++j) {
+    sel[j] = 0;
+    if (j < n) {
+      float bk = -INFINITY;
+      int be = 0x7fffffff;
+      for (int i = 0, e = lane; e < E; ++i, e += 32) {
+        if ((selmask >> i) & 1u) continue;
+        float kv = krow[e];
+        if (kv != kv) kv = -INFINITY;
+        if (be == 0x7fffffff || kv > bk) { bk = kv; be = e; }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const float ok = __shfl_xor_sync(0xffffffffu, bk, o);
+        const int oe = __shfl_xor_sync(0xffffffffu, be, o);
+        if (oe != 0x7fffffff && (be == 0x7fffffff || ok > bk || (ok == bk && oe < be))) {
+          bk = ok;
+          be = oe;
+        }
+      }
+      sel[j] = be;
+      if ((be & 31) == lane) selmask |= 1u << (be >> 5);
+    }
+  }
+}
+
+// Experts of rank 0..n-1 of a row (descending key, NaN as -infinity, ties to the lower index)
+// into br[0..n), one warp. Up to 64 experts every lane counts the rank of its own experts.
+__device__ __forceinline__ void warp_rank_into(const float *krow, int E, int n, int *br) {
+  const int lane = threadIdx.x & 31;
+  if (E <= RT_SEL_THREAD_MAX_E) {
+    for (int e = lane; e < E; e += 32) {
+      float v = krow[e];
+      if (v != v) v = -INFINITY;
+      int rank = 0;
+      for (int e2 = 0; e2 < E; ++e2) {
+        float v2 = krow[e2];
+        if (v2 != v2) v2 = -INFINITY;
+        rank += (v2 > v || (v2 == v && e2 < e)) ? 1 : 0;
+      }
+      if (rank < n) br[rank] = e;
+    }
+  } else {
+    int sel[9];
+    warp_topn(krow, E, n, sel);
+#pragma unroll
+    for (int j = 0; j < 9; ++j)
+      if (j < n && lane == 0) br[j] = sel[j];
+  }
+}
+
+// Canonical logit from the fp64 sum s of the exact products plus the offset (every lane holds
+// the same s): |s - S| <= gamma_{d+16} (sum |x_i W_i| + |off|) <= (d+16) 2^-52 (|x||W_e| + |off|).
+// When no fp32 rounding boundary lies within that distance, RN32(s) is the canonical logit;
+// otherwise resolve_logit decides exactly (warp-cooperative).
+template <typename Tin>
+__device__ float finish_logit(double s, const Tin *xrow, const Tin *wrow, int d, double off,
+                              double xn, double wne, int force_level) {
+  if (!isfinite(s)) return (float)s;  // an infinite or NaN input: the sum is that, exactly
+  const double B = (double)(d + 16) * 0x1p-52 * (xn * wne + fabs(off));
+  float r, up, dn;
+  double mh, ml;
+  if (force_level == 0 && rn32_certain(s, B, r, up, dn, mh, ml)) return r;
+  return resolve_logit<Tin>(xrow, wrow, d, off, s, force_level);
+}
+
+template <typename Tin>
 __global__ void __launch_bounds__(RT_THREADS, 2) router_kernel(RouterArgs a) {
-  constexpr int EB = 8 * NT;  // experts per round
-  using F = Frag4<Tin>;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
+  using CH = Chunk8<Tin>;
   const int E = a.E, d = a.d, k = a.k;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int fr = lane >> 2, fc = lane & 3;  // fragment row / column of this lane
   const int t0 = blockIdx.x * RT_TM;
   const int ntok = min(RT_TM, a.T - t0);
   const Tin *__restrict__ x = (const Tin *)a.x;
@@ -478,25 +533,21 @@ __global__ void __launch_bounds__(RT_THREADS, 2) router_kernel(RouterArgs a) {
   const int force_level = g_force_exact;
   const bool force = force_level != 0;
   const bool sigmoid = a.score == MOE_SCORE_SIGMOID;
-  const RouterSmem SL = router_smem(E, NT, sigmoid, d, (int)sizeof(Tin));
-  double *part = (double *)(smem_raw + SL.part);  // [RT_WARPS][RT_TM][EB]
-  double *sq = (double *)(smem_raw + SL.sq);      // [RT_WARPS][EB + RT_TM]
-  uint32_t *exr = (uint32_t *)(smem_raw + SL.ex);  // [RT_WARPS][EB + RT_TM][min, max] keys
-  int *wexp = (int *)(smem_raw + SL.wexp);         // [EB][min, max] of the round's rows
-  int *xexp = (int *)(smem_raw + SL.xexp);         // [RT_TM][min, max]
-  float *lg = (float *)(smem_raw + SL.lg);
-  float *keys = (float *)(smem_raw + SL.keys);
-  const bool rank_sel = E <= RT_SEL_THREAD_MAX_E;
-  float *pb = rank_sel ? (float *)(smem_raw + SL.pb) : lg;
-  int *sel_e = (int *)(smem_raw + SL.sel_e);
-  float *sel_p = (float *)(smem_raw + SL.sel_p);
-  double *wn = (double *)(smem_raw + SL.wn);  // [EB] norms of the round's rows
+  const RouterSmem SL = router_smem(E, sigmoid, d, (int)sizeof(Tin));
+  uint4 *ring = (uint4 *)(smem_raw + SL.ring);   // [RT_WD][RT_EPT][PARTS][RT_THREADS / 2]
+  float *off_s = (float *)(smem_raw + SL.off);   // [E] logit offsets (zeros without)
+  float *part = (float *)(smem_raw + SL.part);   // [RT_WARPS][RT_TM][RT_EB]
+  float *wsq_s = (float *)(smem_raw + SL.wsq);   // [RT_WARPS][RT_EB]
+  double *wn = (double *)(smem_raw + SL.wn);     // [E] upper bounds of |W_e|_2
+  float *lg = (float *)(smem_raw + SL.lg);       // [RT_TM][E] logits, then probabilities
+  float *keys = (float *)(smem_raw + SL.keys);   // [RT_TM][E] sigmoid keys
+  int *brw = (int *)(smem_raw + SL.byrank) + warp * 9;  // this warp's experts by rank
   int *cnt = (int *)(smem_raw + SL.cnt);
-  const int nfw = (E + 31) / 32;
-  unsigned *flags = (unsigned *)(smem_raw + SL.flags);  // [RT_TM][nfw] undecided logits
   double *xnorm = (double *)(smem_raw + SL.xnorm);
-  double *fix_s = (double *)(smem_raw + SL.fix);  // fp64 sums of the first RT_FIX_CAP flagged
-  __shared__ int s_nfix;
+  unsigned *cmask = (unsigned *)(smem_raw + SL.cmask);  // [listed token][E/32]
+  __shared__ int s_nflag, s_flag[RT_TM];
+  __shared__ unsigned long long s_wnmax;  // bits of nonnegative doubles / floats order as integers
+  __shared__ int s_offmax, s_bmax;
 
   griddep_wait();
   griddep_launch();
@@ -510,6 +561,10 @@ __global__ void __launch_bounds__(RT_THREADS, 2) router_kernel(RouterArgs a) {
   if (tid == 0) {
     mbar_init(xbar, 1);
     s_xabort = 0;
+    s_wnmax = 0ull;
+    s_offmax = 0;
+    s_bmax = 0;
+    s_nflag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   __syncthreads();
@@ -518,12 +573,57 @@ __global__ void __launch_bounds__(RT_THREADS, 2) router_kernel(RouterArgs a) {
     for (int r = 0; r < ntok; ++r)
       bulk_load_1d(smem_u32(xs + (size_t)r * xs_stride), x + (size_t)(t0 + r) * d, row_bytes, xbar);
   }
+
+  // ---- screen tiling (see the header): this lane's chunks of d and its W ring
+  const int nch = d >> 3;  // 8-element chunks per row (d is a multiple of 64)
+  const int ks = lane & 1, eg = (lane >> 1) & 7, tg = lane >> 4;
+  const int c0 = 2 * warp + ks;
+  const int nmine = c0 < nch ? (nch - c0 + 2 * RT_WARPS - 1) / (2 * RT_WARPS) : 0;
+  const int pr = warp * 16 + (lane & 15);  // the lane pair
+  constexpr int NP = RT_THREADS / 2;
+  auto slot_ptr = [&](int s, int j) { return ring + ((size_t)(s * RT_EPT + j) * CH::PARTS) * NP + pr; };
+  // copies of chunk n of the pair's expert rows of the round at eb into slot n % RT_WD, the
+  // 16-byte parts q = j PARTS + u dealt to the two lanes by q % 2 = tg; one commit group per
+  // call, empty or not, so that the group count stays uniform
+  auto ring_issue = [&](int eb, int n) {
+    if (n < nmine) {
+      const int c = c0 + 2 * RT_WARPS * n;
+#pragma unroll
+      for (int j = 0; j < RT_EPT; ++j) {
+        const int e = eb + eg + 8 * j;
+#pragma unroll
+        for (int u = 0; u < CH::PARTS; ++u)
+          if (((j * CH::PARTS + u) & 1) == tg && e < E)
+            cp_async16(smem_u32(slot_ptr(n % RT_WD, j) + u * NP),
+                       (const unsigned char *)(wr + (size_t)e * d + 8 * c) + 16 * u);
+      }
+    }
+    cp_async_commit();
+  };
+  // the first chunks of a round; parts of experts past E are zeroed (never copied into)
+  auto ring_prologue = [&](int eb) {
+#pragma unroll
+    for (int j = 0; j < RT_EPT; ++j)
+#pragma unroll
+      for (int u = 0; u < CH::PARTS; ++u)
+        if (((j * CH::PARTS + u) & 1) == tg && eb + eg + 8 * j >= E)
+          for (int s = 0; s < RT_WD; ++s) slot_ptr(s, j)[u * NP] = make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+    for (int n = 0; n < RT_WD; ++n) ring_issue(eb, n);
+  };
+  ring_prologue(0);  // W does not depend on x: its first chunks travel with the token rows
+
   for (int r = ntok; r < RT_TM; ++r)  // rows past the last token read as zeros
     for (uint32_t i = tid; i < row_bytes / 16; i += RT_THREADS)
       ((uint4 *)(xs + (size_t)r * xs_stride))[i] = make_uint4(0u, 0u, 0u, 0u);
-  for (int e = tid; e < E; e += RT_THREADS) cnt[e] = 0;
-  for (int i = tid; i < RT_TM * nfw; i += RT_THREADS) flags[i] = 0u;
-  if (tid == 0) s_nfix = 0;
+  for (int e = tid; e < E; e += RT_THREADS) {
+    cnt[e] = 0;
+    const float o = a.off ? a.off[e] : 0.0f;
+    off_s[e] = o;
+    // largest |offset| and |bias| (NaN orders above infinity and poisons the bound, as it should)
+    atomicMax(&s_offmax, __float_as_int(fabsf(o)));
+    if (a.bias) atomicMax(&s_bmax, __float_as_int(fabsf(a.bias[e])));
+  }
   if (blockIdx.x == 0 && tid == 0) *a.counter = 0u;
   mbar_wait(xbar, 0u, (volatile int *)&s_xabort, g_wait_limit_ns, INFO_WAIT_ROUTER_X);
   __syncthreads();
@@ -532,376 +632,330 @@ __global__ void __launch_bounds__(RT_THREADS, 2) router_kernel(RouterArgs a) {
       volatile int never = 0;
       mbar_wait(xbar, 0u, &never, g_wait_limit_ns, INFO_WAIT_DRAIN);
     }
+    cp_async_wait<0>();
     __syncthreads();
     return;
   }
 
-  // ---- logits on the fp64 tensor cores, one round per 8*NT experts. Warp w takes the 16-k
-  // blocks w, w+RT_WARPS, ... of the d dimension. For a block, the lane at fragment (row r, column c)
-  // loads elements 4c..4c+3 of token rows r, r+8 (shared memory) and of expert row r of each
-  // column tile (global memory, L2), and MMA step i uses element 4c+i: a permutation of k inside
-  // the block, identical for both operands. Every element of the CTA's token rows and of the
-  // round's expert rows is loaded exactly once per round, so the sums of squares of the loaded
-  // values give |x_t| and |W_e| for the rounding bound. The per-warp partial sums are then
-  // added in warp order.
-  const int nkb = d / RT_KB;
-  const Tin *xs_f[RT_MT];
+  // ---- |x_t|_2 bounds: 16 threads per row, fp32 sums of squares, fixed tree
+  {
+    const int tt = tid >> 4, q16 = tid & 15;
+    const Tin *row = (const Tin *)(xs + (size_t)tt * xs_stride);
+    float s = 0.0f;
+    for (int c = q16; c < nch; c += 16) {
+      CH q;
+      q.ld_s(row + 8 * c);
 #pragma unroll
-  for (int mt = 0; mt < RT_MT; ++mt) xs_f[mt] = (const Tin *)(xs + (size_t)(fr + 8 * mt) * xs_stride) + 4 * fc;
-  for (int eb = 0; eb < E; eb += EB) {
-    double acc[RT_MT][NT][2];
-    float xsq[RT_MT], wsq[NT];
-    uint32_t xmn[RT_MT], xmx[RT_MT], wmn[NT], wmx[NT];
-    const Tin *wrow_f[NT];
-    bool e_ok[NT];
-#pragma unroll
-    for (int mt = 0; mt < RT_MT; ++mt) {
-      xsq[mt] = 0.0f;
-      xmn[mt] = 0xFFFFFFFFu;
-      xmx[mt] = 0u;
-#pragma unroll
-      for (int j = 0; j < NT; ++j) acc[mt][j][0] = acc[mt][j][1] = 0.0;
-    }
-#pragma unroll
-    for (int j = 0; j < NT; ++j) {
-      wsq[j] = 0.0f;
-      wmn[j] = 0xFFFFFFFFu;
-      wmx[j] = 0u;
-      const int e = eb + 8 * j + fr;
-      e_ok[j] = e < E;
-      wrow_f[j] = wr + (size_t)(e_ok[j] ? e : 0) * d + 4 * fc;
-    }
-    // one-block-ahead prefetch of the raw fragments
-    typename F::raw_t ra[RT_MT], rb[NT];
-#pragma unroll
-    for (int mt = 0; mt < RT_MT; ++mt) ra[mt] = F::zero();
-#pragma unroll
-    for (int j = 0; j < NT; ++j) rb[j] = F::zero();
-    int kb = warp;
-    if (kb < nkb) {
-#pragma unroll
-      for (int mt = 0; mt < RT_MT; ++mt) ra[mt] = F::load_s(xs_f[mt] + kb * RT_KB);
-#pragma unroll
-      for (int j = 0; j < NT; ++j) if (e_ok[j]) rb[j] = F::load(wrow_f[j] + kb * RT_KB);
-    }
-    for (; kb < nkb; kb += RT_WARPS) {
-      double av[RT_MT][4], bv[NT][4];
-#pragma unroll
-      for (int mt = 0; mt < RT_MT; ++mt) F::digest(ra[mt], av[mt], xsq[mt], xmn[mt], xmx[mt]);
-#pragma unroll
-      for (int j = 0; j < NT; ++j) F::digest(rb[j], bv[j], wsq[j], wmn[j], wmx[j]);
-      const int kn = kb + RT_WARPS;
-      if (kn < nkb) {
-#pragma unroll
-        for (int mt = 0; mt < RT_MT; ++mt) ra[mt] = F::load_s(xs_f[mt] + kn * RT_KB);
-#pragma unroll
-        for (int j = 0; j < NT; ++j) rb[j] = e_ok[j] ? F::load(wrow_f[j] + kn * RT_KB) : F::zero();
-      }
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < NT; ++j)
-#pragma unroll
-          for (int mt = 0; mt < RT_MT; ++mt) dmma_8x8x4(acc[mt][j], av[mt][i], bv[j][i]);
-    }
-    // per-warp row sums of squares (lanes of one fragment row differ in fc = lane bits 0-1)
-#pragma unroll
-    for (int o = 1; o < 4; o <<= 1) {
-#pragma unroll
-      for (int mt = 0; mt < RT_MT; ++mt) {
-        xsq[mt] += __shfl_xor_sync(0xffffffffu, xsq[mt], o);
-        xmn[mt] = min(xmn[mt], __shfl_xor_sync(0xffffffffu, xmn[mt], o));
-        xmx[mt] = max(xmx[mt], __shfl_xor_sync(0xffffffffu, xmx[mt], o));
-      }
-#pragma unroll
-      for (int j = 0; j < NT; ++j) {
-        wsq[j] += __shfl_xor_sync(0xffffffffu, wsq[j], o);
-        wmn[j] = min(wmn[j], __shfl_xor_sync(0xffffffffu, wmn[j], o));
-        wmx[j] = max(wmx[j], __shfl_xor_sync(0xffffffffu, wmx[j], o));
-      }
-    }
-    if (fc == 0) {
-#pragma unroll
-      for (int j = 0; j < NT; ++j) {
-        sq[warp * (EB + RT_TM) + 8 * j + fr] = wsq[j];
-        exr[2 * (warp * (EB + RT_TM) + 8 * j + fr)] = wmn[j];
-        exr[2 * (warp * (EB + RT_TM) + 8 * j + fr) + 1] = wmx[j];
-      }
-#pragma unroll
-      for (int mt = 0; mt < RT_MT; ++mt) {
-        sq[warp * (EB + RT_TM) + EB + fr + 8 * mt] = xsq[mt];
-        exr[2 * (warp * (EB + RT_TM) + EB + fr + 8 * mt)] = xmn[mt];
-        exr[2 * (warp * (EB + RT_TM) + EB + fr + 8 * mt) + 1] = xmx[mt];
+      for (int i = 0; i < 4; ++i) {
+        const float2 p = q.pair(i);
+        s = fmaf(p.x, p.x, s);
+        s = fmaf(p.y, p.y, s);
       }
     }
 #pragma unroll
-    for (int mt = 0; mt < RT_MT; ++mt)
+    for (int o = 8; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    if (q16 == 0) xnorm[tt] = norm_upper((double)s, d);
+  }
+
+  // ---- screen: approximate logits in fp32, RT_EB experts per round. Warp w takes the chunks
+  // 2w + ks + 16n of d; per chunk a thread takes its 3 expert chunks from its ring (filled
+  // RT_WD chunks ahead) and its 8 token chunks from the staged rows, and accumulates 24 (token,
+  // expert) pairs as two-lane packed FMAs (even and odd elements in the two lanes of a pair).
+  // The sums of squares of the W rows ride along: lane tg squares pairs 2tg, 2tg+1 of a chunk.
+  const size_t xs_es = xs_stride / sizeof(Tin);  // row stride in elements
+  const Tin *xrow0 = (const Tin *)(xs + (size_t)tg * xs_stride);
+  for (int eb = 0; eb < E; eb += RT_EB) {
+    float2 acc[RT_TPT][RT_EPT], wsq[RT_EPT];
 #pragma unroll
-      for (int j = 0; j < NT; ++j)
+    for (int j = 0; j < RT_EPT; ++j) {
+      wsq[j] = make_float2(0.f, 0.f);
 #pragma unroll
-        for (int h = 0; h < 2; ++h)
-          part[(warp * RT_TM + fr + 8 * mt) * EB + 8 * j + 2 * fc + h] = acc[mt][j][h];
-    __syncthreads();
-    for (int q = tid; q < EB + RT_TM; q += RT_THREADS) {
-      double t = 0.0;
-      uint32_t mn = 0xFFFFFFFFu, mx = 0u;
+      for (int tj = 0; tj < RT_TPT; ++tj) acc[tj][j] = make_float2(0.f, 0.f);
+    }
+    for (int n = 0; n < nmine; ++n) {
+      const int c = c0 + 2 * RT_WARPS * n;
+      // both lanes of the pair are done with slot (n-1) % RT_WD: it refills with chunk
+      // n-1+RT_WD; then chunk n (RT_WD groups back) is complete in both lanes and visible
+      __syncwarp();
+      if (n > 0) ring_issue(eb, n - 1 + RT_WD);
+      else cp_async_commit();
+      cp_async_wait<RT_WD>();
+      __syncwarp();
+      float2 w2[RT_EPT][4];
 #pragma unroll
-      for (int w = 0; w < RT_WARPS; ++w) {
-        t += sq[w * (EB + RT_TM) + q];
-        mn = min(mn, exr[2 * (w * (EB + RT_TM) + q)]);
-        mx = max(mx, exr[2 * (w * (EB + RT_TM) + q) + 1]);
+      for (int j = 0; j < RT_EPT; ++j) {
+        CH wc;
+        wc.ld_ring(slot_ptr(n % RT_WD, j), NP);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) w2[j][i] = wc.pair(i);
+        const float2 p0 = tg ? w2[j][2] : w2[j][0], p1 = tg ? w2[j][3] : w2[j][1];
+        wsq[j] = __ffma2_rn(p0, p0, wsq[j]);
+        wsq[j] = __ffma2_rn(p1, p1, wsq[j]);
       }
-      // biased exponents of the smallest and largest nonzero magnitude; (255, -1): all zero
-      const int emn = mx ? (int)(mn >> F::MANT) : 255, emx = mx ? (int)(mx >> F::MANT) : -1;
-      if (q < EB) {
-        wn[q] = norm_upper(t, d);
-        wexp[2 * q] = emn;
-        wexp[2 * q + 1] = emx;
-      } else if (eb == 0) {
-        xnorm[q - EB] = norm_upper(t, d);
-        xexp[2 * (q - EB)] = emn;
-        xexp[2 * (q - EB) + 1] = emx;
+#pragma unroll
+      for (int tj = 0; tj < RT_TPT; ++tj) {
+        CH xc;
+        xc.ld_s(xrow0 + (size_t)(2 * tj) * xs_es + 8 * c);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float2 x2 = xc.pair(i);
+#pragma unroll
+          for (int j = 0; j < RT_EPT; ++j) acc[tj][j] = __ffma2_rn(x2, w2[j][i], acc[tj][j]);
+        }
       }
+    }
+    cp_async_wait<0>();
+    __syncwarp();  // both lanes done with the ring before the next round's copies
+    if (eb + RT_EB < E) ring_prologue(eb + RT_EB);  // the next round's W, during this reduction
+    // fold the two lanes of each pair, then the two k halves (lanes ks = 0, 1); lane ks = 0
+    // stores tokens tg + 2tj for tj < 4, lane ks = 1 the rest
+    float *pw = part + (size_t)warp * RT_TM * RT_EB;
+#pragma unroll
+    for (int tj = 0; tj < RT_TPT; ++tj)
+#pragma unroll
+      for (int j = 0; j < RT_EPT; ++j) {
+        float v = __fadd_rn(acc[tj][j].x, acc[tj][j].y);
+        v = __fadd_rn(v, __shfl_xor_sync(0xffffffffu, v, 1));
+        if ((tj >> 2) == ks) pw[(tg + 2 * tj) * RT_EB + eg + 8 * j] = v;
+      }
+#pragma unroll
+    for (int j = 0; j < RT_EPT; ++j) {
+      float s = __fadd_rn(wsq[j].x, wsq[j].y);
+      s = __fadd_rn(s, __shfl_xor_sync(0xffffffffu, s, 16));
+      s = __fadd_rn(s, __shfl_xor_sync(0xffffffffu, s, 1));
+      if (tg == 0 && ks == 0) wsq_s[warp * RT_EB + eg + 8 * j] = s;
     }
     __syncthreads();
-    for (int q = tid; q < RT_TM * EB; q += RT_THREADS) {
-      const int tt = q / EB, e = eb + q % EB;
+    // per-warp partials added in warp order, then the offset: every product passes through at
+    // most 4 ceil(d/128) (its chain) + 1 + 1 + 7 + 1 roundings
+    for (int q = tid; q < RT_TM * RT_EB; q += RT_THREADS) {
+      const int tt = q / RT_EB, el = q - tt * RT_EB, e = eb + el;
       if (tt < ntok && e < E) {
-        double s = 0.0;
+        float s = part[tt * RT_EB + el];
 #pragma unroll
-        for (int w = 0; w < RT_WARPS; ++w) s += part[(w * RT_TM + tt) * EB + q % EB];
-        const double o = a.off ? (double)a.off[e] : 0.0;
-        s += o;
-        // any summation order over d products plus the partials and the offset:
-        // |error| <= gamma_{d+16} (sum |x_i W_i| + |off|) <= (d+16) 2^-52 (|x|_2 |W_e|_2 + |off|)
-        const double B = (double)(d + 16) * 0x1p-52 * (xnorm[tt] * wn[q % EB] + fabs(o));
-        // Exactness certificate. With biased exponents of at least xmin and wmin (all normal),
-        // every product is an integer multiple of 2^qq, qq = xmin + wmin - 254 - 2 MANT, and so is
-        // the offset when its own quantum is folded in. Every partial sum, in any order, is
-        // bounded by sum |x_i W_i| + |off| <= |x|_2 |W_e|_2 + |off| (Cauchy-Schwarz); xnorm and wn
-        // are upper bounds of the norms and the factor covers this line's own rounding. Below
-        // 2^(qq + 53) every partial sum
-        // is an fp64 value, so s is the exact sum and its round-to-nearest-even to fp32 is the
-        // canonical logit, exact ties included.
-        bool exact;
-        {
-          const int xmn_ = xexp[2 * tt], xmx_ = xexp[2 * tt + 1];
-          const int wmn_ = wexp[2 * (q % EB)], wmx_ = wexp[2 * (q % EB) + 1];
-          int qq = 1 << 20;
-          if (xmx_ >= 0 && wmx_ >= 0) qq = xmn_ + wmn_ - 254 - 2 * F::MANT;
-          bool ok = (xmx_ < 0 || wmx_ < 0 || (xmn_ > 0 && wmn_ > 0)) && xmx_ < 255 && wmx_ < 255;
-          if (o != 0.0) {
-            const int eo = (int)((__float_as_uint((float)o) >> 23) & 0xFFu);
-            ok = ok && eo > 0 && eo < 255;
-            qq = min(qq, eo - 150);
-          }
-          const double S = (xnorm[tt] * wn[q % EB] + fabs(o)) * (1.0 + (double)(d + 8) * 0x1p-50);
-          exact = ok && S <= ldexp(1.0, min(qq + 53, 1023));
-        }
-        float r, up, dn;
-        double mh, ml;
-        float l;
-        if (exact && !force) {
-          l = __double2float_rn(s);
-        } else if (rn32_certain(s, B, r, up, dn, mh, ml) && !force) {
-          l = r;
-        } else {
-          // undecided: resolved exactly by the fixup pass below, which needs the fp64 sum
-          const int slot = atomicAdd(&s_nfix, 1);
-          if (slot < RT_FIX_CAP) {
-            fix_s[slot] = s;
-            l = __int_as_float(slot);  // the slot index rides in the logit until resolved
-          } else {
-            l = __int_as_float(-1);    // overflow (forced test modes): the fixup recomputes
-          }
-          atomicOr(&flags[tt * nfw + (e >> 5)], 1u << (e & 31));
-        }
-        lg[tt * E + e] = l;
+        for (int w = 1; w < RT_WARPS; ++w) s = __fadd_rn(s, part[(w * RT_TM + tt) * RT_EB + el]);
+        if (a.off) s = __fadd_rn(s, off_s[e]);
+        lg[tt * E + e] = s;
       }
     }
-    __syncthreads();  // part, sq and wn are rewritten by the next round
+    if (tid < RT_EB && eb + tid < E) {
+      float s = wsq_s[tid];
+#pragma unroll
+      for (int w = 1; w < RT_WARPS; ++w) s = __fadd_rn(s, wsq_s[w * RT_EB + tid]);
+      const double nrm = norm_upper((double)s, d);
+      wn[eb + tid] = nrm;
+      atomicMax(&s_wnmax, (unsigned long long)__double_as_longlong(nrm));
+    }
+    __syncthreads();  // part and wsq_s are rewritten by the next round
   }
 
-  // ---- fixup of undecided logits: flag words dealt round-robin to the warps; one warp decides
-  // one logit exactly (see resolve_logit)
-  for (int wi = warp; wi < ntok * nfw; wi += RT_THREADS / 32) {
-    unsigned m = flags[wi];
-    const int tt = wi / nfw, e0 = (wi % nfw) * 32;
-    while (m) {
-      const int ee = e0 + __ffs(m) - 1;
-      m &= m - 1;
-      const int slot = __float_as_int(lg[tt * E + ee]);
-      const Tin *xrow = x + (size_t)(t0 + tt) * d;
-      const Tin *wrow = wr + (size_t)ee * d;
-      const double o = a.off ? (double)a.off[ee] : 0.0;
-      double approx;
-      if (slot >= 0 && slot < RT_FIX_CAP) {
-        approx = fix_s[slot];
-      } else {
-        double s = 0.0;
-        for (int i = lane; i < d; i += 32)
-          s = fma((double)Elem<Tin>::to_f(xrow[i]), (double)Elem<Tin>::to_f(wrow[i]), s);
-        approx = warp_sum_d(s) + o;
-      }
-      const float l = resolve_logit<Tin>(xrow, wrow, d, o, approx, force_level);
-      __syncwarp();
-      if (lane == 0) lg[tt * E + ee] = l;
-      __syncwarp();
-    }
-  }
-  __syncthreads();
-
-  // ---- selection
-  if (rank_sel) {
-    // up to 64 experts: every (token, expert) pair finds its own rank among the token's keys
-    if (sigmoid)
-      for (int q = tid; q < ntok * E; q += RT_THREADS)
-        keys[q] = sigmoid_key(lg[q], a.bias ? a.bias[q % E] : 0.0f, force);
-    __syncthreads();
-    // the token's max logit and normaliser, once per token (one warp per token, fixed order)
-    __shared__ float s_tok_m[RT_TM], s_tok_inv[RT_TM];
-    for (int tt = warp; tt < ntok; tt += RT_THREADS / 32) {
-      const float *lrow = lg + tt * E;
-      float m = -INFINITY;
-      for (int e = lane; e < E; e += 32) m = fmaxf(m, lrow[e]);
-      m = warp_max_f(m);
-      float ssum = 0.0f;
-      if (!sigmoid)
-        for (int e = lane; e < E; e += 32) ssum += expf(lrow[e] - m);
-      else
-        for (int e = lane; e < E; e += 32) ssum += 1.0f / (1.0f + expf(-lrow[e]));
-      ssum = warp_sum_f(ssum);
-      if (lane == 0) {
-        s_tok_m[tt] = m;
-        s_tok_inv[tt] = 1.0f / ssum;
-      }
-    }
-    __syncthreads();
-    for (int q = tid; q < ntok * E; q += RT_THREADS) {
-      const int tt = q / E, e = q - tt * E;
-      const float *krow = (sigmoid ? keys : lg) + tt * E;
-      float v = krow[e];
-      if (v != v) v = -INFINITY;
-      int rank = 0;
-      for (int e2 = 0; e2 < E; ++e2) {
-        float v2 = krow[e2];
-        if (v2 != v2) v2 = -INFINITY;
-        rank += (v2 > v || (v2 == v && e2 < e)) ? 1 : 0;
-      }
-      const float inv = s_tok_inv[tt];
-      const float l = lg[tt * E + e];
-      float p, pbasis;
-      if (!sigmoid) {
-        p = expf(l - s_tok_m[tt]) * inv;
-        pbasis = p;
-      } else {
-        p = 1.0f / (1.0f + expf(-l));
-        pbasis = p * inv;
-      }
-      pb[q] = pbasis;
-      if (rank < k) {
-        sel_e[tt * 8 + rank] = e;
-        sel_p[tt * 8 + rank] = p;
-      }
-    }
-    __syncthreads();
-    if (tid < ntok) {
-      const int t = t0 + tid;
-      float psel = 0.0f;
-      for (int j = 0; j < k; ++j) psel += sel_p[tid * 8 + j];
-      for (int j = 0; j < k; ++j) {
-        const int e = sel_e[tid * 8 + j];
-        const float pj = sel_p[tid * 8 + j];
-        a.idx[(size_t)t * k + j] = e;
-        a.wts[(size_t)t * k + j] = a.norm ? pj / psel : pj;
-        atomicAdd(&cnt[e], 1);
-      }
-    }
-    __syncthreads();
-  } else {
-    // one warp per token
-  for (int tt = warp; tt < ntok; tt += RT_THREADS / 32) {
+  // key of expert e of token tt as the screen sees it (fp64, before any fp32 rounding)
+  auto key_of = [&](int tt, int e) -> double {
+    const float l = lg[tt * E + e];
+    if (!sigmoid) return (double)l;
+    return sigmoid64(l) + (a.bias ? (double)a.bias[e] : 0.0);
+  };
+  // Probabilities, weights and outputs of token tt from its logits and its experts by rank
+  // (one warp, fixed-order trees); the logits row becomes the probability basis of the
+  // load-balancing statistics.
+  auto finish_token = [&](int tt) {
     const int t = t0 + tt;
     float *lrow = lg + tt * E;
-    const float *krow = lrow;
-    if (a.score == MOE_SCORE_SIGMOID) {
-      float *kw = keys + warp * E;
-      for (int e = lane; e < E; e += 32) kw[e] = sigmoid_key(lrow[e], a.bias ? a.bias[e] : 0.0f, force);
-      __syncwarp();
-      krow = kw;
-    }
-    unsigned selmask = 0u;
-    int sel[8];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      sel[j] = 0;
-      if (j < k) {
-        float bk = -INFINITY;
-        int be = 0x7fffffff;
-        for (int i = 0, e = lane; e < E; ++i, e += 32) {
-          if ((selmask >> i) & 1u) continue;
-          float kv = krow[e];
-          if (kv != kv) kv = -INFINITY;
-          if (be == 0x7fffffff || kv > bk) { bk = kv; be = e; }
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-          const float ok = __shfl_xor_sync(0xffffffffu, bk, o);
-          const int oe = __shfl_xor_sync(0xffffffffu, be, o);
-          if (oe != 0x7fffffff &&
-              (be == 0x7fffffff || ok > bk || (ok == bk && oe < be))) { bk = ok; be = oe; }
-        }
-        sel[j] = be;
-        if ((be & 31) == lane) selmask |= 1u << (be >> 5);
-      }
-    }
-    // probabilities
-    float pj = 0.0f;
-    if (a.score == MOE_SCORE_SOFTMAX) {
-      float m = -INFINITY;
+    float m = -INFINITY, s = 0.0f;
+    if (!sigmoid) {
       for (int e = lane; e < E; e += 32) m = fmaxf(m, lrow[e]);
       m = warp_max_f(m);
-      float s = 0.0f;
       for (int e = lane; e < E; e += 32) s += expf(lrow[e] - m);
-      s = warp_sum_f(s);
-#pragma unroll
-      for (int j = 0; j < 8; ++j)
-        if (j < k && lane == j) pj = expf(lrow[sel[j]] - m) / s;
-      __syncwarp();
-      for (int e = lane; e < E; e += 32) lrow[e] = expf(lrow[e] - m) / s;
     } else {
-      float s = 0.0f;
       for (int e = lane; e < E; e += 32) s += 1.0f / (1.0f + expf(-lrow[e]));
-      s = warp_sum_f(s);
-#pragma unroll
-      for (int j = 0; j < 8; ++j)
-        if (j < k && lane == j) pj = 1.0f / (1.0f + expf(-lrow[sel[j]]));
-      __syncwarp();
-      for (int e = lane; e < E; e += 32) lrow[e] = (1.0f / (1.0f + expf(-lrow[e]))) / s;
     }
-    float psel = 0.0f;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const float v = __shfl_sync(0xffffffffu, pj, j);
-      if (j < k) psel += v;
-    }
+    s = warp_sum_f(s);
+    int ej = 0;
+    float pj = 0.0f;
     if (lane < k) {
-      int e_out = 0;
-#pragma unroll
-      for (int j = 0; j < 8; ++j) if (j == lane) e_out = sel[j];
-      a.idx[(size_t)t * k + lane] = e_out;
+      ej = brw[lane];
+      pj = !sigmoid ? expf(lrow[ej] - m) / s : 1.0f / (1.0f + expf(-lrow[ej]));
+    }
+    const float psel = warp_sum_f(pj);
+    __syncwarp();
+    for (int e = lane; e < E; e += 32)
+      lrow[e] = !sigmoid ? expf(lrow[e] - m) / s : (1.0f / (1.0f + expf(-lrow[e]))) / s;
+    if (lane < k) {
+      a.idx[(size_t)t * k + lane] = ej;
       a.wts[(size_t)t * k + lane] = a.norm ? pj / psel : pj;
-      atomicAdd(&cnt[e_out], 1);
+      atomicAdd(&cnt[ej], 1);
+    }
+    __syncwarp();
+  };
+
+  // ---- selection, one warp per token. Tokens whose order the screen proves are finished here;
+  // the others are listed with their candidate experts, settled by the whole CTA below.
+  const double mg = (double)(4 * ((nch + 15) / 16) + 10);  // roundings per term of the screen
+  const double gam = mg * 0x1p-24 / (1.0 - mg * 0x1p-24);
+  const double wmax = __longlong_as_double((long long)s_wnmax);
+  const double omax = (double)__int_as_float(s_offmax), bmax = (double)__int_as_float(s_bmax);
+  const int nmw = (E + 31) >> 5;  // candidate mask words per token
+  for (int tt = warp; tt < ntok; tt += RT_WARPS) {
+    float *lrow = lg + tt * E;
+    float *krow = sigmoid ? keys + tt * E : lrow;
+    bool bad = false;
+    float lmax = 0.0f;
+    for (int e = lane; e < E; e += 32) {
+      const float l = lrow[e];
+      bad |= !isfinite(l);
+      lmax = fmaxf(lmax, fabsf(l));
+      if (sigmoid) krow[e] = (float)key_of(tt, e);
+    }
+    bad = __any_sync(0xffffffffu, bad);
+    lmax = warp_max_f(lmax);
+    // Bound of the token's keys. Screen: |l~ - S| <= gamma_m (|x_t| max_e |W_e| + max |off|) for
+    // the exact sum S of every expert (m roundings per term, plus m 2^-149 for underflow).
+    // Sigmoid: the key comes from the canonical (rounded) logit, within that plus half an fp32
+    // step of l~; sigmoid is 1/4-Lipschitz, and its fp64 evaluation plus the bias add err by less
+    // than 2^-47 + 2^-51 |b|.
+    double Bk = gam * (xnorm[tt] * wmax + omax) * (1.0 + 0x1p-40) + mg * 0x1p-149;
+    if (sigmoid) Bk = 0.25 * (Bk + 0x1p-24 * ((double)lmax + Bk) + 0x1p-149) + 0x1p-47 + 0x1p-51 * bmax;
+    __syncwarp();
+    warp_rank_into(krow, E, min(k + 1, E), brw);
+    __syncwarp();
+    // the proof: each of the J gaps between consecutive approximate ranks exceeds twice the key
+    // bound plus two fp32 steps at that magnitude (lane j checks gap j)
+    const int J = min(k, E - 1);
+    bool ok = true;
+    if (lane < J) {
+      const double prev = key_of(tt, brw[lane]), cur = key_of(tt, brw[lane + 1]);
+      ok = prev - cur > 2.0 * Bk + 0x1p-22 * (fmax(fabs(prev), fabs(cur)) + Bk) + 0x1p-148;
+    }
+    const bool proven = __all_sync(0xffffffffu, ok) && !bad && !force && Bk < INFINITY;
+    if (proven) {
+      finish_token(tt);
+      continue;
+    }
+    // candidates: every expert whose key is not provably below the (k+1)-th approximate key
+    // (all of them when the bound is unusable or k = E)
+    const bool all = force || bad || E <= k || !(Bk < INFINITY);
+    double cut = -INFINITY;
+    if (!all) {
+      const double vk = key_of(tt, brw[k]);
+      cut = vk - 2.0 * Bk - 0x1p-22 * (fabs(vk) + Bk) - 0x1p-148;
+    }
+    int f = 0;
+    if (lane == 0) f = atomicAdd(&s_nflag, 1);
+    f = __shfl_sync(0xffffffffu, f, 0);
+    if (lane == 0) s_flag[f] = tt;
+    for (int w0 = 0; w0 < nmw; ++w0) {
+      const int e = 32 * w0 + lane;
+      const unsigned m = __ballot_sync(0xffffffffu, e < E && (all || key_of(tt, e) >= cut));
+      if (lane == 0) cmask[f * nmw + w0] = m;
     }
     __syncwarp();
   }
   __syncthreads();
+
+  // ---- exact settlement of the listed tokens: their candidates dealt round-robin to the warps,
+  // one warp per candidate (fp64 sum of the exact products, then finish_logit)
+  const int nflag = s_nflag;
+  if (nflag > 0) {
+    int ci = 0;
+    for (int f = 0; f < nflag; ++f) {
+      const int tt = s_flag[f];
+      const Tin *xrow = (const Tin *)(xs + (size_t)tt * xs_stride);
+      for (int w0 = 0; w0 < nmw; ++w0) {
+        unsigned m = cmask[f * nmw + w0];
+        while (m) {
+          const int ee = 32 * w0 + __ffs(m) - 1;
+          m &= m - 1;
+          if ((ci++ % RT_WARPS) != warp) continue;
+          const Tin *wrow = wr + (size_t)ee * d;
+          double acc = 0.0;
+          uint32_t xmn = 0xFFFFFFFFu, wmn = 0xFFFFFFFFu, emx = 0u;  // fp32 magnitude bits
+          auto note = [&](float xv, float wv) {
+            const uint32_t bx = __float_as_uint(xv) & 0x7FFFFFFFu, bw = __float_as_uint(wv) & 0x7FFFFFFFu;
+            xmn = min(xmn, bx ? bx : 0xFFFFFFFFu);
+            wmn = min(wmn, bw ? bw : 0xFFFFFFFFu);
+            emx = max(emx, max(bx, bw));
+          };
+          for (int i0 = 8 * lane; i0 < d; i0 += 4 * 256) {
+            CH wq[4], xq[4];  // four chunks of the lane requested together
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const int i = i0 + 256 * u;
+              if (i < d) {
+                wq[u].ld_g(wrow + i);
+                xq[u].ld_s(xrow + i);
+              } else {
+                wq[u].zero();
+                xq[u].zero();
+              }
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+#pragma unroll
+              for (int p = 0; p < 4; ++p) {
+                const float2 xf = xq[u].pair(p), wf = wq[u].pair(p);
+                acc = fma((double)xf.x, (double)wf.x, acc);
+                acc = fma((double)xf.y, (double)wf.y, acc);
+                note(xf.x, wf.x);
+                note(xf.y, wf.y);
+              }
+          }
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) {
+            xmn = min(xmn, __shfl_xor_sync(0xffffffffu, xmn, o));
+            wmn = min(wmn, __shfl_xor_sync(0xffffffffu, wmn, o));
+            emx = max(emx, __shfl_xor_sync(0xffffffffu, emx, o));
+          }
+          const float of = off_s[ee];
+          const double o = (double)of;
+          const double sum = warp_sum_d(acc) + o;
+          // Exactness certificate: with all elements normal and finite (biased exponents
+          // >= xe, we), every product is an integer multiple of 2^q, q = xe + we - 254 - 2 MANT
+          // (MANT fraction bits of the input type), and so is the offset with its own quantum.
+          // Every partial sum, in any order, is at most |x||W_e| + |off| (Cauchy-Schwarz); below
+          // 2^(q+53) all of them are fp64 values, so `sum` is the exact sum and its fp32
+          // rounding the canonical logit, ties to even included.
+          constexpr int MANT = sizeof(Tin) == 2 ? 7 : 23;
+          bool exact = false;
+          if (xmn != 0xFFFFFFFFu && wmn != 0xFFFFFFFFu) {
+            const int xe = (int)(xmn >> 23), we = (int)(wmn >> 23);
+            int q = xe + we - 254 - 2 * MANT;
+            bool okc = xe > 0 && we > 0 && (emx >> 23) < 255u;
+            if (of != 0.0f) {
+              const int eo = (int)((__float_as_uint(of) >> 23) & 0xFFu);
+              okc = okc && eo > 0 && eo < 255;
+              q = min(q, eo - 150);
+            }
+            const double S = (xnorm[tt] * wn[ee] + fabs(o)) * (1.0 + (double)(d + 8) * 0x1p-50);
+            exact = okc && S <= ldexp(1.0, min(q + 53, 1023));
+          } else if (xmn == 0xFFFFFFFFu || wmn == 0xFFFFFFFFu) {
+            exact = (emx >> 23) < 255u;  // one row all zeros: the sum is the offset, exactly
+          }
+          const float l = exact && !force
+                              ? __double2float_rn(sum)
+                              : finish_logit<Tin>(sum, xrow, wrow, d, o, xnorm[tt], wn[ee], force_level);
+          if (lane == 0) {
+            lg[tt * E + ee] = l;
+            if (sigmoid) keys[tt * E + ee] = sigmoid_key(l, a.bias ? a.bias[ee] : 0.0f, force);
+          }
+          __syncwarp();
+        }
+      }
+    }
+    __syncthreads();
+    // the listed tokens, ranked again on their canonical candidate keys, then finished
+    for (int f = warp; f < nflag; f += RT_WARPS) {
+      const int tt = s_flag[f];
+      warp_rank_into((sigmoid ? keys : lg) + tt * E, E, k, brw);
+      __syncwarp();
+      finish_token(tt);
+    }
   }
+  __syncthreads();
 
   // ---- per-CTA statistics (fixed token order), then the last CTA reduces in CTA order
   for (int e = tid; e < E; e += RT_THREADS) {
     float ps = 0.0f;
-    for (int tt = 0; tt < ntok; ++tt) ps += pb[tt * E + e];
+    for (int tt = 0; tt < ntok; ++tt) ps += lg[tt * E + e];
     a.part_cnt[(size_t)blockIdx.x * E + e] = cnt[e];
     a.part_prob[(size_t)blockIdx.x * E + e] = ps;
   }
