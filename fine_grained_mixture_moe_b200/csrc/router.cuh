@@ -482,7 +482,7 @@ __device__ __forceinline__ void warp_topn(const float *krow, int E, int n, int (
 
 // Experts of rank 0..n-1 of a row (descending key, NaN as -infinity, ties to the lower index)
 // into br[0..n), one warp. Up to 64 experts every lane counts the rank of its own experts.
-__device__ __forceinline__ void warp_rank_into(const float *krow, int E, int n, int *br) {
+__device__ __noinline__ void warp_rank_into(const float *krow, int E, int n, int *br) {
   const int lane = threadIdx.x & 31;
   if (E <= RT_SEL_THREAD_MAX_E) {
     for (int e = lane; e < E; e += 32) {
@@ -518,6 +518,41 @@ __device__ float finish_logit(double s, const Tin *xrow, const Tin *wrow, int d,
   double mh, ml;
   if (force_level == 0 && rn32_certain(s, B, r, up, dn, mh, ml)) return r;
   return resolve_logit<Tin>(xrow, wrow, d, off, s, force_level);
+}
+
+// Probabilities, weights and outputs of token t (row lrow of logits, experts by rank in br), one
+// warp, fixed-order trees; the logits row becomes the probability basis of the load-balancing
+// statistics. One out-of-line copy serves the proven tokens and the settled ones.
+__device__ __noinline__ void finish_token(const RouterArgs &a, float *lrow, const int *br, int t,
+                                          int *cnt) {
+  const int lane = threadIdx.x & 31;
+  const int E = a.E, k = a.k;
+  const bool sigmoid = a.score == MOE_SCORE_SIGMOID;
+  float m = -INFINITY, s = 0.0f;
+  if (!sigmoid) {
+    for (int e = lane; e < E; e += 32) m = fmaxf(m, lrow[e]);
+    m = warp_max_f(m);
+    for (int e = lane; e < E; e += 32) s += expf(lrow[e] - m);
+  } else {
+    for (int e = lane; e < E; e += 32) s += 1.0f / (1.0f + expf(-lrow[e]));
+  }
+  s = warp_sum_f(s);
+  int ej = 0;
+  float pj = 0.0f;
+  if (lane < k) {
+    ej = br[lane];
+    pj = !sigmoid ? expf(lrow[ej] - m) / s : 1.0f / (1.0f + expf(-lrow[ej]));
+  }
+  const float psel = warp_sum_f(pj);
+  __syncwarp();
+  for (int e = lane; e < E; e += 32)
+    lrow[e] = !sigmoid ? expf(lrow[e] - m) / s : (1.0f / (1.0f + expf(-lrow[e]))) / s;
+  if (lane < k) {
+    a.idx[(size_t)t * k + lane] = ej;
+    a.wts[(size_t)t * k + lane] = a.norm ? pj / psel : pj;
+    atomicAdd(&cnt[ej], 1);
+  }
+  __syncwarp();
 }
 
 template <typename Tin>
@@ -755,39 +790,6 @@ __global__ void __launch_bounds__(RT_THREADS, 2) router_kernel(RouterArgs a) {
     if (!sigmoid) return (double)l;
     return sigmoid64(l) + (a.bias ? (double)a.bias[e] : 0.0);
   };
-  // Probabilities, weights and outputs of token tt from its logits and its experts by rank
-  // (one warp, fixed-order trees); the logits row becomes the probability basis of the
-  // load-balancing statistics.
-  auto finish_token = [&](int tt) {
-    const int t = t0 + tt;
-    float *lrow = lg + tt * E;
-    float m = -INFINITY, s = 0.0f;
-    if (!sigmoid) {
-      for (int e = lane; e < E; e += 32) m = fmaxf(m, lrow[e]);
-      m = warp_max_f(m);
-      for (int e = lane; e < E; e += 32) s += expf(lrow[e] - m);
-    } else {
-      for (int e = lane; e < E; e += 32) s += 1.0f / (1.0f + expf(-lrow[e]));
-    }
-    s = warp_sum_f(s);
-    int ej = 0;
-    float pj = 0.0f;
-    if (lane < k) {
-      ej = brw[lane];
-      pj = !sigmoid ? expf(lrow[ej] - m) / s : 1.0f / (1.0f + expf(-lrow[ej]));
-    }
-    const float psel = warp_sum_f(pj);
-    __syncwarp();
-    for (int e = lane; e < E; e += 32)
-      lrow[e] = !sigmoid ? expf(lrow[e] - m) / s : (1.0f / (1.0f + expf(-lrow[e]))) / s;
-    if (lane < k) {
-      a.idx[(size_t)t * k + lane] = ej;
-      a.wts[(size_t)t * k + lane] = a.norm ? pj / psel : pj;
-      atomicAdd(&cnt[ej], 1);
-    }
-    __syncwarp();
-  };
-
   // ---- selection, one warp per token. Tokens whose order the screen proves are finished here;
   // the others are listed with their candidate experts, settled by the whole CTA below.
   const double mg = (double)(4 * ((nch + 15) / 16) + 10);  // roundings per term of the screen
@@ -828,7 +830,7 @@ __global__ void __launch_bounds__(RT_THREADS, 2) router_kernel(RouterArgs a) {
     }
     const bool proven = __all_sync(0xffffffffu, ok) && !bad && !force && Bk < INFINITY;
     if (proven) {
-      finish_token(tt);
+      finish_token(a, lrow, brw, t0 + tt, cnt);
       continue;
     }
     // candidates: every expert whose key is not provably below the (k+1)-th approximate key
@@ -947,7 +949,7 @@ __global__ void __launch_bounds__(RT_THREADS, 2) router_kernel(RouterArgs a) {
       const int tt = s_flag[f];
       warp_rank_into((sigmoid ? keys : lg) + tt * E, E, k, brw);
       __syncwarp();
-      finish_token(tt);
+      finish_token(a, lg + tt * E, brw, t0 + tt, cnt);
     }
   }
   __syncthreads();
