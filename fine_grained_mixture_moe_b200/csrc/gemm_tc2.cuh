@@ -48,11 +48,15 @@ __device__ __forceinline__ void tc2_commit_both(uint32_t bar) {
       "h"(mask)
       : "memory");
 }
+// Relaxed: the arrival only has to follow this thread's completed TMEM reads (tcgen05.wait::ld
+// precedes it in program order, and the MMA that may overwrite those columns is issued only after
+// the arrival is observed). A release here would also wait for every global store the epilogue
+// warp has in flight.
 __device__ __forceinline__ void mbar_arrive_cta0(uint32_t bar_local) {
   asm volatile(
       "{\n\t.reg .b32 ra;\n\t"
       "mapa.shared::cluster.u32 ra, %0, 0;\n\t"
-      "mbarrier.arrive.release.cluster.shared::cluster.b64 _, [ra];\n\t}" ::"r"(bar_local)
+      "mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [ra];\n\t}" ::"r"(bar_local)
       : "memory");
 }
 
