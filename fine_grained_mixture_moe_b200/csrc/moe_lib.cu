@@ -95,7 +95,7 @@ inline bool yperm_bf16(const moe_config_t *c) {
 }
 
 struct Layout {
-  size_t part_cnt, part_prob, chunk_base, kept, scounter;       // route / statistics
+  size_t part_cnt, part_prob, chunk_base, kept;                 // route / statistics
   size_t chunk_count;                                           // moe_permute's own histogram
   size_t hidden, hidden_sh;                                     // experts
   size_t idx, wts, count, prob, offsets, slot_pos, src, x_perm, y_perm, y_shared, aux;  // layer
@@ -116,7 +116,6 @@ Layout layout_of(const moe_config_t *c) {
   L.part_prob = take(nch * E * 4);
   L.chunk_base = take(nch * E * 4);
   L.kept = take(E * 4);
-  L.scounter = take(16);
   L.chunk_count = take(nch * E * 4);
   L.hidden = take(T * k * width * es);
   L.hidden_sh = take(T * (size_t)c->n_shared * (size_t)c->ffn_shared * es);
@@ -371,7 +370,7 @@ moe_status_t launch_stats(const StatsArgs &sa, cudaStream_t st) {
 template <typename Tin>
 moe_status_t router_only(const moe_config_t *c, const void *x, const moe_weights_t *w,
                          int32_t *idx, float *wts, int32_t *part_cnt, float *part_prob,
-                         unsigned *counter, cudaStream_t st) {
+                         cudaStream_t st) {
   RouterArgs a;
   a.x = x;
   a.w = w->w_router;
@@ -381,21 +380,17 @@ moe_status_t router_only(const moe_config_t *c, const void *x, const moe_weights
   a.idx = idx; a.wts = wts;
   a.part_cnt = part_cnt;
   a.part_prob = part_prob;
-  a.counter = counter;
   return launch_router<Tin>(a, st);
 }
 
-StatsArgs stats_args(const moe_config_t *c, const int32_t *chunk_cnt, const float *chunk_prob,
-                     unsigned *counter) {
+StatsArgs stats_args(const moe_config_t *c, const int32_t *chunk_cnt, const float *chunk_prob) {
   StatsArgs sa;
   std::memset(&sa, 0, sizeof(sa));
   sa.chunk_cnt = chunk_cnt;
   sa.chunk_prob = chunk_prob;
   sa.nchunk = ceil_div(c->T, RT_TM);
-  sa.E = c->E; sa.T = c->T; sa.k = c->top_k;
+  sa.E = c->E;
   sa.C = capacity_of(c);
-  sa.alpha = c->aux_alpha;
-  sa.counter = counter;
   return sa;
 }
 
@@ -411,9 +406,8 @@ moe_status_t route_impl(const moe_config_t *c, const void *x, const moe_weights_
   }
   int32_t *pc = at<int32_t>(ws, L.part_cnt);
   float *pp = at<float>(ws, L.part_prob);
-  unsigned *ctr = at<unsigned>(ws, L.scounter);
-  MOE_TRY(router_only<Tin>(c, x, w, idx, wts, pc, pp, ctr, st));
-  StatsArgs sa = stats_args(c, pc, pp, ctr);
+  MOE_TRY(router_only<Tin>(c, x, w, idx, wts, pc, pp, st));
+  StatsArgs sa = stats_args(c, pc, pp);
   sa.count_out = count;
   sa.prob_out = prob;
   return launch_stats(sa, st);
@@ -421,8 +415,9 @@ moe_status_t route_impl(const moe_config_t *c, const void *x, const moe_weights_
 
 template <typename Tin>
 moe_status_t scatter_impl(const moe_config_t *c, const void *x, const int32_t *idx,
-                          const int32_t *chunk_base, const int32_t *offsets, int32_t *slot_pos,
-                          int32_t *src, void *x_perm, cudaStream_t st) {
+                          const int32_t *chunk_base, const int32_t *kept, int32_t *offsets,
+                          int32_t *slot_pos, int32_t *src, void *x_perm, const int32_t *count,
+                          const float *prob, float *aux, cudaStream_t st) {
   ProfScope ps(K_PERM_SCATTER, st);
   // shared memory: the CTA's PM_TPC token rows, then per expert the lane mask, the chunk's
   // base rank and the offset
@@ -432,8 +427,9 @@ moe_status_t scatter_impl(const moe_config_t *c, const void *x, const int32_t *i
                            (int)smem) != cudaSuccess)
     return MOE_ERR_CUDA;
   return launch_pdl(perm_scatter_kernel<Tin>, dim3(ceil_div(c->T, PM_CHUNK) * PM_SPLIT), dim3(256),
-                    smem, st, idx, c->T, c->top_k, c->E, capacity_of(c), chunk_base, offsets,
-                    slot_pos, src, (const Tin *)x, (Tin *)x_perm, c->d);
+                    smem, st, idx, c->T, c->top_k, c->E, capacity_of(c), chunk_base, kept, offsets,
+                    slot_pos, src, (const Tin *)x, (Tin *)x_perm, c->d, count, prob, c->aux_alpha,
+                    aux);
 }
 
 template <typename Tin>
@@ -446,21 +442,20 @@ moe_status_t permute_impl(const moe_config_t *c, const void *x, const int32_t *i
   }
   const int nch = ceil_div(c->T, PM_CHUNK);
   int32_t *cc = at<int32_t>(ws, L.chunk_count), *cb = at<int32_t>(ws, L.chunk_base);
-  unsigned *ctr = at<unsigned>(ws, L.scounter);
   {
     const size_t smem = (size_t)8 * c->E * 4;
     if (cudaFuncSetAttribute(perm_hist_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
       return MOE_ERR_CUDA;
     ProfScope ps(K_PERM_HIST, st);
     MOE_TRY(launch_pdl(perm_hist_kernel, dim3(ceil_div(nch, 8)), dim3(256), smem, st, idx, c->T,
-                       c->top_k, c->E, cc, nch, ctr));
+                       c->top_k, c->E, cc, nch));
   }
-  StatsArgs sa = stats_args(c, cc, nullptr, ctr);
+  StatsArgs sa = stats_args(c, cc, nullptr);
   sa.chunk_base = cb;
   sa.kept = at<int32_t>(ws, L.kept);
-  sa.offsets = offsets;
   MOE_TRY(launch_stats(sa, st));
-  return scatter_impl<Tin>(c, x, idx, cb, offsets, slot_pos, src, x_perm, st);
+  return scatter_impl<Tin>(c, x, idx, cb, sa.kept, offsets, slot_pos, src, x_perm, nullptr,
+                           nullptr, nullptr, st);
 }
 
 moe_status_t experts_impl(const moe_config_t *c, const void *x_perm, const int32_t *offsets,
@@ -686,27 +681,27 @@ moe_status_t moe_layer_forward(const moe_config_t *cfg, const void *x, const moe
     if (cudaMemsetAsync(cnt, 0, (size_t)cfg->E * 4, st) != cudaSuccess) return MOE_ERR_CUDA;
     return cudaMemsetAsync(aux, 0, 4, st) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
   }
-  // route -> statistics (counts, probability sums, chunk scans, offsets, loss) -> scatter
+  // route -> statistics (counts, probability sums, chunk scans, kept counts) -> scatter
+  // (offsets, loss, positions, rows)
   int32_t *pc = at<int32_t>(ws, L.part_cnt);
   float *pp = at<float>(ws, L.part_prob);
   int32_t *cb = at<int32_t>(ws, L.chunk_base);
-  unsigned *ctr = at<unsigned>(ws, L.scounter);
   if (cfg->dtype == MOE_DTYPE_BF16)
-    MOE_TRY(router_only<__nv_bfloat16>(cfg, x, w, idx, wts, pc, pp, ctr, st));
+    MOE_TRY(router_only<__nv_bfloat16>(cfg, x, w, idx, wts, pc, pp, st));
   else
-    MOE_TRY(router_only<float>(cfg, x, w, idx, wts, pc, pp, ctr, st));
-  StatsArgs sa = stats_args(cfg, pc, pp, ctr);
+    MOE_TRY(router_only<float>(cfg, x, w, idx, wts, pc, pp, st));
+  StatsArgs sa = stats_args(cfg, pc, pp);
   sa.count_out = cnt;
   sa.prob_out = prob;
   sa.chunk_base = cb;
   sa.kept = at<int32_t>(ws, L.kept);
-  sa.offsets = offsets;
-  sa.aux = aux;
   MOE_TRY(launch_stats(sa, st));
   if (cfg->dtype == MOE_DTYPE_BF16)
-    MOE_TRY(scatter_impl<__nv_bfloat16>(cfg, x, idx, cb, offsets, slot_pos, src, x_perm, st));
+    MOE_TRY(scatter_impl<__nv_bfloat16>(cfg, x, idx, cb, sa.kept, offsets, slot_pos, src, x_perm,
+                                        cnt, prob, aux, st));
   else
-    MOE_TRY(scatter_impl<float>(cfg, x, idx, cb, offsets, slot_pos, src, x_perm, st));
+    MOE_TRY(scatter_impl<float>(cfg, x, idx, cb, sa.kept, offsets, slot_pos, src, x_perm, cnt,
+                                prob, aux, st));
   MOE_TRY(experts_impl(cfg, x_perm, offsets, x, w, y_perm, y_sh, ws, st));
   return combine_impl(cfg, y_perm, y_sh, slot_pos, wts, y, st);
 }
@@ -815,9 +810,8 @@ extern "C" moe_status_t moe_debug_wait_timeout_probe(void *stream) {
 }
 
 // ================================================================== moe_route_noalloc
-// The router's scratch (fp64 router weight, row norms, per-CTA partial statistics and the
-// completion counter) placed in a fixed array of the library's own device memory instead of a
-// caller workspace. Host code must not use the array's name as a device pointer: it is a host
+// The router's scratch (the per-CTA partial statistics) placed in a fixed array of the library's
+// own device memory instead of a caller workspace. Host code must not use the array's name as a device pointer: it is a host
 // stand-in for the symbol, so its device address is looked up once per device below.
 namespace {
 
@@ -843,7 +837,7 @@ moe_status_t route_scratch_address(void **out) {
 }
 
 struct RouteScratch {
-  size_t part_cnt, part_prob, counter, total;
+  size_t part_cnt, part_prob, total;
 };
 
 RouteScratch route_scratch_layout(const moe_config_t *c) {
@@ -854,7 +848,6 @@ RouteScratch route_scratch_layout(const moe_config_t *c) {
   auto take = [&](size_t bytes) { size_t at = o; o = align256(o + std::max<size_t>(bytes, 1)); return at; };
   L.part_cnt = take(nblk * E * 4);
   L.part_prob = take(nblk * E * 4);
-  L.counter = take(16);
   L.total = o;
   return L;
 }
@@ -869,13 +862,12 @@ moe_status_t route_noalloc_impl(const moe_config_t *c, const void *x, const moe_
     if (cudaMemsetAsync(prob, 0, (size_t)c->E * 4, st) != cudaSuccess) return MOE_ERR_CUDA;
     return MOE_OK;
   }
-  // every call rewrites the per-CTA partials before reading them, and the router clears the
-  // counter, so nothing left in the array by an earlier call is read
+  // every call rewrites the per-CTA partials before reading them, so nothing left in the
+  // array by an earlier call is read
   int32_t *pc = (int32_t *)(scratch + L.part_cnt);
   float *pp = (float *)(scratch + L.part_prob);
-  unsigned *ctr = (unsigned *)(scratch + L.counter);
-  MOE_TRY(router_only<Tin>(c, x, w, idx, wts, pc, pp, ctr, st));
-  StatsArgs sa = stats_args(c, pc, pp, ctr);
+  MOE_TRY(router_only<Tin>(c, x, w, idx, wts, pc, pp, st));
+  StatsArgs sa = stats_args(c, pc, pp);
   sa.count_out = count;
   sa.prob_out = prob;
   return launch_stats(sa, st);

@@ -8,10 +8,12 @@
 //   hist    per-chunk expert histogram -> chunk_count[chunk][E] (inside the layer call the
 //           router's per-CTA counts already are this histogram, so it is only launched by
 //           moe_permute on its own)
-//   stats   per-expert exclusive scan over chunks -> chunk_base; offsets[E+1] (stats.cuh)
-//   scatter per-chunk ranks from a per-expert lane bitmask, slot_pos / src_token; PM_SPLIT
-//           CTAs per chunk each bring 4 of its x rows into shared memory and store each to its
-//           k destinations in x_perm with 1-D bulk copies (each row read once).
+//   stats   per-expert exclusive scan over chunks -> chunk_base; kept counts (stats.cuh)
+//   scatter offsets[E+1] = exclusive scan of the kept counts (every CTA, in shared memory; block
+//           0 writes them out, with the load-balancing loss); per-chunk ranks from a
+//           per-expert lane bitmask, slot_pos / src_token; PM_SPLIT CTAs per chunk each bring 4
+//           of its x rows into shared memory and store each to its k destinations in x_perm
+//           with 1-D bulk copies (each row read once).
 #pragma once
 #include "common.cuh"
 
@@ -23,7 +25,7 @@ constexpr int PM_SPLIT = 4;  // CTAs per chunk in the scatter
 __global__ void __launch_bounds__(256) perm_hist_kernel(const int32_t *__restrict__ idx, int T,
                                                         int k, int E,
                                                         int32_t *__restrict__ chunk_count,
-                                                        int nchunks, unsigned *stats_counter) {
+                                                        int nchunks) {
   griddep_wait();
   griddep_launch();
   extern __shared__ int sh_cnt[];  // [8][E]
@@ -32,7 +34,6 @@ __global__ void __launch_bounds__(256) perm_hist_kernel(const int32_t *__restric
   for (int e = lane; e < E; e += 32) c[e] = 0;
   __syncwarp();
   const int chunk = blockIdx.x * 8 + warp;
-  if (blockIdx.x == 0 && threadIdx.x == 0) *stats_counter = 0u;  // consumed by moe_stats_kernel
   if (chunk >= nchunks) return;
   const int t = chunk * PM_CHUNK + lane;
   if (lane < PM_CHUNK && t < T) {
@@ -48,23 +49,28 @@ __global__ void __launch_bounds__(256) perm_hist_kernel(const int32_t *__restric
 
 // Scatter. CTA (chunk, part) owns tokens chunk*16 + part*TPC .. +TPC (TPC = 16 / PM_SPLIT).
 // Thread 0 first starts 1-D bulk copies of the CTA's token rows into shared memory (they do not
-// depend on the routing); the chunk's routing, its per-expert base ranks and the expert offsets
-// are read together; warp 0 then ranks the chunk's (token, slot) pairs, and one thread per kept
-// pair stores the whole row to its x_perm row with a single shared -> global bulk copy. x is read
-// once and written k times by the copy engine.
+// depend on the routing); the chunk's routing, its per-expert base ranks and the kept counts are
+// read together and the kept counts scanned into the expert offsets; warp 0 then ranks the
+// chunk's (token, slot) pairs, and one thread per kept pair stores the whole row to its x_perm
+// row with a single shared -> global bulk copy. x is read once and written k times by the copy
+// engine. Block 0 also writes offsets[0..E] and, when `aux` is set, the load-balancing loss
+// alpha E sum_e (count_e / (T k)) (prob_e / T) (Quartz: weight 0.01), in the order of
+// aux_loss_kernel, so that the fused layer and the separate call agree bit for bit.
 constexpr int PM_TPC = PM_CHUNK / PM_SPLIT;        // tokens per scatter CTA
 
 template <typename Tin>
 __global__ void __launch_bounds__(256) perm_scatter_kernel(
     const int32_t *__restrict__ idx, int T, int k, int E, int C,
-    const int32_t *__restrict__ chunk_base, const int32_t *__restrict__ offsets,
-    int32_t *__restrict__ slot_pos, int32_t *__restrict__ src, const Tin *__restrict__ x,
-    Tin *__restrict__ x_perm, int d) {
+    const int32_t *__restrict__ chunk_base, const int32_t *__restrict__ kept,
+    int32_t *__restrict__ offsets, int32_t *__restrict__ slot_pos, int32_t *__restrict__ src,
+    const Tin *__restrict__ x, Tin *__restrict__ x_perm, int d, const int32_t *__restrict__ count,
+    const float *__restrict__ prob, float alpha, float *__restrict__ aux) {
   griddep_wait();
   griddep_launch();
   // [PM_TPC rows][row_bytes] | lane masks [E] | chunk base [E] | offsets [E]
   extern __shared__ __align__(128) unsigned char sm_raw[];
   __shared__ int s_pos[PM_CHUNK * 8];
+  __shared__ int s_scan[256 / 32 + 1];
   __shared__ __align__(8) uint64_t s_bar;
   __shared__ volatile int s_abort;
   const bool active = (threadIdx.x & 31) < PM_CHUNK;
@@ -73,8 +79,8 @@ __global__ void __launch_bounds__(256) perm_scatter_kernel(
   const uint32_t row_bytes = (uint32_t)d * (uint32_t)sizeof(Tin);
   unsigned char *rows = sm_raw;
   unsigned *smask = (unsigned *)(sm_raw + (size_t)PM_TPC * row_bytes);
-  int *s_base = (int *)(smask + E);  // this chunk's per-expert base rank and the expert offsets,
-  int *s_off = s_base + E;           // loaded alongside the routing, not after it
+  int *s_base = (int *)(smask + E);  // this chunk's per-expert base rank and the expert offsets
+  int *s_off = s_base + E;           // (from the kept counts), read alongside the routing
   const int tfirst = chunk * PM_CHUNK + part * PM_TPC;
   const int nrows = max(0, min(PM_TPC, T - tfirst));
   const bool copy = x_perm != nullptr && nrows > 0;
@@ -90,7 +96,7 @@ __global__ void __launch_bounds__(256) perm_scatter_kernel(
                      row_bytes, bar);
     }
   }
-  // warp 0 reads the chunk's routing while the other warps read the bases and offsets
+  // warp 0 reads the chunk's routing while the other warps read the bases and kept counts
   const int t = chunk * PM_CHUNK + lane;
   int ev[8];
   if (warp == 0) {
@@ -107,9 +113,24 @@ __global__ void __launch_bounds__(256) perm_scatter_kernel(
   for (int e = tid; e < E; e += blockDim.x) {
     smask[e] = 0u;
     s_base[e] = chunk_base[(size_t)chunk * E + e];
-    s_off[e] = offsets[e];
+    s_off[e] = kept[e];
   }
-  __syncthreads();  // the barrier is initialised, masks cleared, bases and offsets in place
+  __syncthreads();  // the barrier is initialised, masks cleared, bases and kept counts in place
+  const int n_kept = block_excl_scan_inplace(s_off, E, s_scan);  // -> expert offsets
+  if (blockIdx.x == 0) {
+    for (int e = tid; e < E; e += blockDim.x) offsets[e] = s_off[e];
+    if (tid == 0) offsets[E] = n_kept;
+    if (aux != nullptr && warp == 0) {
+      double sd = 0.0;
+      for (int e = lane; e < E; e += 32) sd += (double)count[e] * (double)prob[e];
+      sd = warp_sum_d(sd);
+      if (lane == 0) {
+        double L = 0.0;
+        if (T > 0) L = (double)alpha * (double)E * sd / ((double)T * (double)k * (double)T);
+        *aux = (float)L;
+      }
+    }
+  }
   if (warp == 0) {
 #pragma unroll
     for (int j = 0; j < 8; ++j)

@@ -56,7 +56,6 @@ struct RouterArgs {
   float *part_prob;     // [nblk, E]
   int32_t *count_out;   // [E]
   float *prob_out;      // [E]
-  unsigned int *counter; // completion counter of the statistics kernel, cleared here
 };
 
 // Eight consecutive elements (bf16: 16 bytes; fp32: 32 bytes) and their pairs as fp32.
@@ -659,7 +658,6 @@ __global__ void __launch_bounds__(RT_THREADS, 2) router_kernel(RouterArgs a) {
     atomicMax(&s_offmax, __float_as_int(fabsf(o)));
     if (a.bias) atomicMax(&s_bmax, __float_as_int(fabsf(a.bias[e])));
   }
-  if (blockIdx.x == 0 && tid == 0) *a.counter = 0u;
   mbar_wait(xbar, 0u, (volatile int *)&s_xabort, g_wait_limit_ns, INFO_WAIT_ROUTER_X);
   __syncthreads();
   if (s_xabort) {  // the copies did not land in time: error recorded; let them drain, then leave

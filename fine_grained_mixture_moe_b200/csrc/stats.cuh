@@ -2,12 +2,12 @@
 //   count[e]          = sum over chunks of the chunk's selections of e (before capacity)
 //   prob_sum[e]       = sum over chunks of the chunk's probability mass on e, fixed order
 //   chunk_base[c][e]  = exclusive scan over chunks of the selections of e (token order)
-//   offsets[0..E]     = exclusive scan over experts of kept_e = min(count_e, C) (dropless: count_e)
-//   aux               = alpha * E * sum_e (count_e / (T k)) * (prob_sum_e / T)
-// One block per expert does the first three; the block that finishes last does the scan over
-// experts and the loss (Moonfrost expert card: routing under a per-expert capacity over stacked experts;
-// Quartz: load-balancing loss with weight 0.01). Chunks are RT_TM tokens, the router's CTA,
-// so the router's per-CTA counts are the permutation's histogram. Every sum has a fixed order.
+//   kept[e]           = min(count_e, C) (dropless: count_e)
+// One block per expert, no atomics. The scan over experts (offsets) and the load-balancing loss
+// (Quartz: weight 0.01) are formed by the scatter kernel that follows, which needs the offsets
+// anyway (permute.cuh). Chunks are RT_TM tokens, the router's CTA, so the router's per-CTA
+// counts are the permutation's histogram (Moonfrost expert card: routing under a per-expert
+// capacity over stacked experts). Every sum has a fixed order.
 #pragma once
 #include "common.cuh"
 
@@ -18,15 +18,11 @@ constexpr int ST_THREADS = 256;
 struct StatsArgs {
   const int32_t *chunk_cnt;  // [nchunk][E]
   const float *chunk_prob;   // [nchunk][E] or null
-  int nchunk, E, T, k, C;    // C < 0: dropless
+  int nchunk, E, C;          // C < 0: dropless
   int32_t *count_out;        // [E] or null
   float *prob_out;           // [E] or null (needs chunk_prob)
   int32_t *chunk_base;       // [nchunk][E] or null
-  int32_t *kept;             // [E] scratch, needed with offsets
-  int32_t *offsets;          // [E+1] or null
-  float *aux;                // scalar or null (needs chunk_prob)
-  float alpha;
-  unsigned *counter;         // cleared before the launch; reset to 0 by the last block
+  int32_t *kept;             // [E] or null
 };
 
 __global__ void __launch_bounds__(ST_THREADS) moe_stats_kernel(StatsArgs a) {
@@ -71,42 +67,6 @@ __global__ void __launch_bounds__(ST_THREADS) moe_stats_kernel(StatsArgs a) {
     if (a.prob_out) a.prob_out[e] = psum;
     if (a.kept) a.kept[e] = a.C < 0 ? run : min(run, a.C);
   }
-  if (!a.offsets && !a.aux) return;
-  // the last block to finish scans the kept counts over experts and forms the loss; all of its
-  // loads are issued together
-  __threadfence();
-  __syncthreads();
-  __shared__ int s_last;
-  if (tid == 0) s_last = (atomicAdd(a.counter, 1u) == gridDim.x - 1);
-  __syncthreads();
-  if (!s_last) return;
-  __threadfence();
-  __shared__ int s_scan[1024 + ST_THREADS / 32 + 1];
-  double s = 0.0;
-  for (int i = tid; i < E; i += ST_THREADS) {
-    if (a.offsets) s_scan[i] = __ldcg(a.kept + i);
-    if (a.aux) s += (double)__ldcg(a.count_out + i) * (double)__ldcg(a.prob_out + i);
-  }
-  __syncthreads();
-  if (a.offsets) {
-    const int tot = block_excl_scan_inplace(s_scan, E, s_scan + 1024);
-    for (int i = tid; i < E; i += ST_THREADS) a.offsets[i] = s_scan[i];
-    if (tid == 0) a.offsets[E] = tot;
-  }
-  if (a.aux) {
-    s = warp_sum_d(s);
-    __shared__ double s_d[ST_THREADS / 32];
-    if (lane == 0) s_d[warp] = s;
-    __syncthreads();
-    if (tid == 0) {
-      double t = 0.0;
-      for (int w = 0; w < ST_THREADS / 32; ++w) t += s_d[w];
-      double L = 0.0;
-      if (a.T > 0) L = (double)a.alpha * (double)E * t / ((double)a.T * (double)a.k * (double)a.T);
-      *a.aux = (float)L;
-    }
-  }
-  if (tid == 0) *a.counter = 0u;
 }
 
 // Loss-free balancing step (dormouse pages: a router bias balances the load in place of the
