@@ -171,6 +171,34 @@ def test_certified_ties_round_to_even():
     assert ref["route"]["idx"][1].tolist() == [1, 0]
 
 
+@pytest.mark.parametrize("name", ["quartz", "sigmoid"])
+def test_near_ties_settled_exactly(name):
+    """Router rows 0 and 1 are equal except in element 0 (2^-20 against 2^-20 (1 + 2^-7)), and a
+    common offset (softmax) or bias (sigmoid) puts both at the top of every token: their logits
+    differ by x[t,0] 2^-27, far inside the fp32 screen's bound, so every token's order is settled
+    by the exact path without forcing it. Exact sums that land in one fp32 rounding cell tie and
+    go to the lower index; the others are ordered by value. Bit-exact against the oracle."""
+    c = get_config(name, T=300)
+    inp = make_inputs(c)
+    W = inp["w_router"].copy()
+    W[1] = W[0]
+    W[0, 0] = 2.0 ** -20
+    W[1, 0] = 2.0 ** -20 * (1.0 + 2.0 ** -7)
+    inp["w_router"] = W
+    if c.score == "softmax":
+        off = inp["logit_offset"].copy()
+        off[0] = off[1] = 8.0
+        inp["logit_offset"] = off
+    else:
+        b = inp["select_bias"].copy()
+        b[0] = b[1] = 2.0
+        inp["select_bias"] = b
+    o, ref = check_steps(c, inp, exact_only=True)
+    idx = ref["route"]["idx"]
+    assert np.array_equal(np.sort(idx[:, :2], axis=1), np.tile([0, 1], (idx.shape[0], 1)))
+    assert (idx[:, 0] == 0).any() and (idx[:, 0] == 1).any()  # both orders occur
+
+
 def test_bias_update_bitwise():
     """Loss-free balancing step on the routed counts of the sigmoid configuration, then the next
     routing call with the updated bias: the bias bit-exact against the oracle, the new routing
