@@ -91,6 +91,17 @@ def test_unsupported_configs_are_rejected(lib, bad):
     assert st == 2  # MOE_ERR_UNSUPPORTED
 
 
+@pytest.mark.parametrize("dtype,d_max", [("bf16", 6016), ("f32", 2624)])
+def test_hidden_size_limit_of_the_router_tile(lib, dtype, d_max):
+    """The router stages 16 token rows of d elements, a ring of router-row chunks and the logits
+    in one CTA's shared memory (227 KB): the largest d (multiple of 64) with E = 8 is d_max, as
+    the header states (about 6,000 bf16, 2,600 fp32)."""
+    ok = B.make_config(T=16, d=d_max, E=8, top_k=2, ffn=64, dtype=dtype)
+    too_big = B.make_config(T=16, d=d_max + 64, E=8, top_k=2, ffn=64, dtype=dtype)
+    assert B.moe_workspace_size(ok) > 0
+    assert B.moe_workspace_size(too_big) == 0
+
+
 def test_bad_pointers_and_workspace_are_rejected_on_the_host(lib):
     cfg = B.make_config(T=16, d=128, E=8, top_k=2, ffn=64)
     w = B.MoEWeights()
