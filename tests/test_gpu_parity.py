@@ -228,6 +228,23 @@ def test_bias_update_bitwise():
     assert float(b1) == 0.25
 
 
+def test_permute_without_the_copy():
+    """moe_permute with x_perm = NULL computes the same offsets, slot positions and source tokens
+    and copies nothing (the header allows skipping the copy)."""
+    c = SMALL["capacity_s"]
+    run = GpuRun(c, make_inputs(c))
+    o = run.steps()
+    offs = torch.empty_like(o["offsets"])
+    sl = torch.empty_like(o["slot_pos"])
+    sr = torch.full_like(o["src"], -7)
+    B.moe_permute(run.cfg, run.x, o["idx"], offs, sl, sr, None, run.ws, run.ws_bytes)
+    torch.cuda.synchronize()
+    N = int(o["offsets"][-1])
+    assert torch.equal(offs, o["offsets"])
+    assert torch.equal(sl, o["slot_pos"])
+    assert torch.equal(sr[:N], o["src"][:N])
+
+
 def test_empty_call():
     c = get_config("quartz", T=0)
     run = GpuRun(c, make_inputs(c, T=0))
