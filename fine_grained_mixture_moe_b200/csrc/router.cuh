@@ -230,31 +230,6 @@ __device__ __forceinline__ void dbl_bit_range(double v, int &lead, int &lsb) {
 // exponent over all terms and thresholds, every term is an integer multiple of 2^q and, when
 // the exponent span is at most 50 bits, below 2^51, so their sum (at most d + 3 terms) is exact
 // in int64. Returns false (caller falls back) when the span is wider or a term is subnormal.
-// Eight consecutive elements of x (bf16 or fp32) as doubles, from a 16-byte aligned address.
-__device__ __forceinline__ void load8(const __nv_bfloat16 *p, double *v) {
-  const uint4 q = *(const uint4 *)p;
-  const __nv_bfloat162 *h = (const __nv_bfloat162 *)&q;
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const float2 f = __bfloat1622float2(h[i]);
-    v[2 * i] = f.x;
-    v[2 * i + 1] = f.y;
-  }
-}
-__device__ __forceinline__ void load8(const float *p, double *v) {
-  const float4 a = *(const float4 *)p, b = *(const float4 *)(p + 4);
-  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
-  v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
-}
-__device__ __forceinline__ void load8(const double *p, double *v) {
-#pragma unroll
-  for (int i = 0; i < 8; i += 2) {
-    const double2 q = *(const double2 *)(p + i);
-    v[i] = q.x;
-    v[i + 1] = q.y;
-  }
-}
-
 template <typename Tin>
 __device__ bool warp_exact_signs(const Tin *xrow, const Tin *wrow, int d, double off,
                                  double mh, double ml, int &c_hi, int &c_lo) {
