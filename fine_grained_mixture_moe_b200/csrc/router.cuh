@@ -153,12 +153,11 @@ __device__ __forceinline__ bool rn32_certain(double v, double B, float &r, float
   return (v + B < mid_hi) && (v - B > mid_lo) && fabs((double)r) < 0x1p126;
 }
 
+// RN32 of S = sum_i x_i W_i + off by one thread: S as an exact non-overlapping expansion; its top
+// component is within an fp64 step of S, so RN32(S) is the fp32 value r nearest to it or a
+// neighbour, and the signs of S minus the two rounding midpoints around r decide which.
 template <typename Tin>
-__device__ __noinline__ float exact_logit(const Tin *xrow, const Tin *wrow, int d, double off,
-                                          double approx) {
-  float r, up, dn;
-  double mh, ml;
-  rn32_certain(approx, 0.0, r, up, dn, mh, ml);
+__device__ __noinline__ float exact_logit(const Tin *xrow, const Tin *wrow, int d, double off) {
   Expansion X;
   X.n = 0;
   X.overflow = false;
@@ -167,11 +166,15 @@ __device__ __noinline__ float exact_logit(const Tin *xrow, const Tin *wrow, int 
     if (p != 0.0) expansion_add(X, p);
   }
   if (off != 0.0) expansion_add(X, off);
+  if (X.overflow) set_device_error(MOE_ERR_DEVICE_CHECK, INFO_EXPANSION_OVERFLOW);
+  if (X.n == 0) return 0.0f;
+  float r, up, dn;
+  double mh, ml;
+  rn32_certain(X.h[X.n - 1], 0.0, r, up, dn, mh, ml);
   expansion_add(X, -mh);                    // X = S - mid_hi
   const int c_hi = expansion_sign(X);
   expansion_add(X, mh - ml);                // X = S - mid_lo (difference exact)
   const int c_lo = expansion_sign(X);
-  if (X.overflow) set_device_error(MOE_ERR_DEVICE_CHECK, INFO_EXPANSION_OVERFLOW);
   return rn32_from_signs(r, up, dn, c_hi, c_lo);
 }
 
@@ -225,14 +228,37 @@ __device__ __forceinline__ void dbl_bit_range(double v, int &lead, int &lsb) {
   lsb = ef - 1075 + (__ffsll((long long)M) - 1);
 }
 
-// Warp-cooperative exact comparison of S = sum_i x_i W_i + off with two dyadic thresholds.
-// Every product is exact in fp64 and so is a multiple of 2^lsb(p); with q the smallest such
-// exponent over all terms and thresholds, every term is an integer multiple of 2^q and, when
-// the exponent span is at most 50 bits, below 2^51, so their sum (at most d + 3 terms) is exact
-// in int64. Returns false (caller falls back) when the span is wider or a term is subnormal.
+// RN32(a 2^q), exactly: round to nearest even on the integer at the fp32 quantum of the value's
+// binade (2^(E-23), or 2^-149 below 2^-126), then scale by a power of two, which is exact.
+__device__ __forceinline__ float rn32_scaled_int(long long a, int q) {
+  if (a == 0) return 0.0f;
+  const bool neg = a < 0;
+  const unsigned long long m = neg ? 0ull - (unsigned long long)a : (unsigned long long)a;
+  const int E = (63 - __clzll((long long)m)) + q;  // 2^E <= |a 2^q| < 2^(E+1)
+  if (E > 127) return neg ? -INFINITY : INFINITY;
+  const int qexp = E >= -126 ? E - 23 : -149;
+  const int sh = qexp - q;  // bits of m below the quantum
+  unsigned long long t;
+  if (sh <= 0) {
+    t = m << (-sh);  // already a multiple of the quantum: t < 2^24
+  } else if (sh >= 64) {
+    t = 0ull;        // m < 2^63 <= half a quantum
+  } else {
+    t = m >> sh;
+    const unsigned long long rem = m & ((1ull << sh) - 1ull), half = 1ull << (sh - 1);
+    if (rem > half || (rem == half && (t & 1ull))) ++t;
+  }
+  const float r = ldexpf((float)t, qexp);  // t <= 2^24: exact, or the correct overflow to infinity
+  return neg ? -r : r;
+}
+
+// Warp-cooperative exact rounding of S = sum_i x_i W_i + off. Every product is exact in fp64 and
+// so is a multiple of 2^lsb(p); with q the smallest such exponent over all terms, every term is
+// an integer multiple of 2^q below 2^(span+1), span = top exponent - q. When span + 1 +
+// ceil(log2(d + 3)) <= 62 the integer sum of the terms is exact in int64, and S is that integer
+// times 2^q. Returns false (caller falls back) when the span is wider or a term is subnormal.
 template <typename Tin>
-__device__ bool warp_exact_signs(const Tin *xrow, const Tin *wrow, int d, double off,
-                                 double mh, double ml, int &c_hi, int &c_lo) {
+__device__ bool warp_exact_round(const Tin *xrow, const Tin *wrow, int d, double off, float &out) {
   const int lane = threadIdx.x & 31;
   int qmin = 0x7fffffff, emax = -0x7fffffff;
   bool bad = false;
@@ -271,49 +297,37 @@ __device__ bool warp_exact_signs(const Tin *xrow, const Tin *wrow, int d, double
     }
   };
   for_products(scan);
-  if (lane == 0) {
-    scan(off);
-    scan(mh);
-    scan(ml);
-  }
+  if (lane == 0) scan(off);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
     qmin = min(qmin, __shfl_xor_sync(0xffffffffu, qmin, o));
     emax = max(emax, __shfl_xor_sync(0xffffffffu, emax, o));
   }
   bad = __any_sync(0xffffffffu, bad);
-  if (bad || emax - qmin > 50) return false;
+  const int span_max = 61 - (32 - __clz(d + 2));  // 61 - ceil(log2(d + 3))
+  if (bad || emax - qmin > span_max) return false;
   long long acc = 0;
   for_products([&](double v) { acc += (long long)ldexp(v, -qmin); });
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
   acc += (long long)ldexp(off, -qmin);
-  const long long h = (long long)ldexp(mh, -qmin), l = (long long)ldexp(ml, -qmin);
-  c_hi = acc > h ? 1 : (acc < h ? -1 : 0);
-  c_lo = acc > l ? 1 : (acc < l ? -1 : 0);
+  out = rn32_scaled_int(acc, qmin);
   return true;
 }
 
-// Warp-cooperative resolution of one logit whose fp64 screen was undecided (or every logit in
-// the forced test modes). Every lane calls it with the same arguments and gets the same result.
-// `approx` is the fp64 sum of the main pass, within (d+16) 2^-52 |x||W_e| of the exact value -
-// far below an fp32 step - so RN32 of the exact value is r = RN32(approx) or a neighbour; the
-// exact integer comparison against the two rounding boundaries around r decides which, ties to
-// even. force_level 2 skips the integer path and sends the logit to the single-thread
-// expansion, to test that path too.
+// Warp-cooperative exact RN32 of one logit whose fp64 evaluation could not settle it (or every
+// logit in the forced test modes). Every lane calls it with the same arguments and gets the same
+// result: the exact integer sum when the terms' exponent span allows, else the single-thread
+// expansion. Neither depends on the fp64 sum, so a sum that cancels below its own error bound is
+// rounded exactly too. force_level 2 skips the integer path, to test the expansion as well.
 template <typename Tin>
 __device__ __noinline__ float resolve_logit(const Tin *xrow, const Tin *wrow, int d, double off,
-                                            double approx, int force_level) {
+                                            int force_level) {
   const int lane = threadIdx.x & 31;
-  float r, up, dn;
-  double mh, ml;
-  rn32_certain(approx, 0.0, r, up, dn, mh, ml);
-  int c_hi, c_lo;
-  if (force_level < 2 && fabs((double)r) < 0x1p126 &&
-      warp_exact_signs<Tin>(xrow, wrow, d, off, mh, ml, c_hi, c_lo))
-    return rn32_from_signs(r, up, dn, c_hi, c_lo);
-  float l = 0.0f;
-  if (lane == 0) l = exact_logit<Tin>(xrow, wrow, d, off, approx);
+  float l;
+  if (force_level < 2 && warp_exact_round<Tin>(xrow, wrow, d, off, l)) return l;
+  l = 0.0f;
+  if (lane == 0) l = exact_logit<Tin>(xrow, wrow, d, off);
   return __shfl_sync(0xffffffffu, l, 0);
 }
 
@@ -491,7 +505,7 @@ __device__ float finish_logit(double s, const Tin *xrow, const Tin *wrow, int d,
   float r, up, dn;
   double mh, ml;
   if (force_level == 0 && rn32_certain(s, B, r, up, dn, mh, ml)) return r;
-  return resolve_logit<Tin>(xrow, wrow, d, off, s, force_level);
+  return resolve_logit<Tin>(xrow, wrow, d, off, force_level);
 }
 
 // Probabilities, weights and outputs of token t (row lrow of logits, experts by rank in br), one

@@ -171,6 +171,26 @@ def test_certified_ties_round_to_even():
     assert ref["route"]["idx"][1].tolist() == [1, 0]
 
 
+def test_cancelling_sums_rounded_exactly():
+    """Logits whose fp64 sums cancel below their own error bound: 1 + 2^-53 - 1 (an fp64 chain
+    gives 0; the exact sum 2^-53 is decided by the integer path) and 1 + 2^-60 - 1 (an exponent
+    span of 60 bits: the expansion path), against plain logits 2^-70 and 2^-100. The exact order
+    of the top three is experts 0, 2, 3; rounding near the fp64 sums would put 0 and 2 last."""
+    c = MoEConfig(name="cancel", T=2, d=64, E=4, top_k=3, n_shared=0, ffn=64, ffn_shared=0)
+    inp = make_inputs(c)
+    x = np.zeros((2, 64), np.float32)
+    x[:, :3] = 1.0
+    W = np.zeros((4, 64), np.float32)
+    W[0, :3] = [1.0, 2.0 ** -53, -1.0]
+    W[1, 0] = 2.0 ** -100
+    W[2, :3] = [1.0, 2.0 ** -60, -1.0]
+    W[3, 0] = 2.0 ** -70
+    inp["x"], inp["w_router"] = x, W
+    o, ref = check_steps(c, inp, exact_only=True)
+    assert ref["route"]["idx"][0].tolist() == [0, 2, 3]
+    assert ref["route"]["idx"][1].tolist() == [0, 2, 3]
+
+
 @pytest.mark.parametrize("name", ["quartz", "sigmoid"])
 def test_near_ties_settled_exactly(name):
     """Router rows 0 and 1 are equal except in element 0 (2^-20 against 2^-20 (1 + 2^-7)), and a
