@@ -49,7 +49,7 @@ def np_(t: torch.Tensor) -> np.ndarray:
     return t.detach().cpu().numpy()
 
 
-class GpuRun:
+class LayerOnGpu:
     """Device copies of one configuration's inputs plus every step's outputs."""
 
     def __init__(self, c, inp, device="cuda:0"):

@@ -12,7 +12,7 @@ import torch
 import oracle
 from fine_grained_mixture_moe_b200 import binding as B
 from moe_synth import CONFIGS, MoEConfig, get_config, make_inputs
-from tests.gpu_helpers import GpuRun, np_, rel_err, rel_err_stored, tol_of
+from tests.gpu_helpers import LayerOnGpu, np_, rel_err, rel_err_stored, tol_of
 
 pytestmark = pytest.mark.gpu
 
@@ -65,7 +65,7 @@ EDGE = {
 
 
 def check_steps(c, inp, run=None, exact_only=False):
-    run = run or GpuRun(c, inp)
+    run = run or LayerOnGpu(c, inp)
     ref = oracle.layer_forward(c, inp, with_outputs=not exact_only)
     o = run.steps()
     r, pm = ref["route"], ref["perm"]
@@ -225,7 +225,7 @@ def test_bias_update_bitwise():
     bit-exact as well. Balanced counts and a single expert leave the bias unchanged."""
     c = SMALL["sigmoid_s"]
     inp = make_inputs(c)
-    run = GpuRun(c, inp)
+    run = LayerOnGpu(c, inp)
     o = run.steps()
     bias0 = np.asarray(inp["select_bias"], np.float32)
     for u in (1e-3, 2.0 ** -24, 0.05):
@@ -252,7 +252,7 @@ def test_permute_without_the_copy():
     """moe_permute with x_perm = NULL computes the same offsets, slot positions and source tokens
     and copies nothing (the header allows skipping the copy)."""
     c = SMALL["capacity_s"]
-    run = GpuRun(c, make_inputs(c))
+    run = LayerOnGpu(c, make_inputs(c))
     o = run.steps()
     offs = torch.empty_like(o["offsets"])
     sl = torch.empty_like(o["slot_pos"])
@@ -267,7 +267,7 @@ def test_permute_without_the_copy():
 
 def test_empty_call():
     c = get_config("quartz", T=0)
-    run = GpuRun(c, make_inputs(c, T=0))
+    run = LayerOnGpu(c, make_inputs(c, T=0))
     y, aux, cnt = run.layer()
     assert float(aux) == 0.0
     assert int(cnt.abs().sum()) == 0
@@ -280,7 +280,7 @@ def test_back_to_back_calls_on_one_workspace():
     workspace by the next call."""
     c = SMALL["quartz_s"]
     inp = make_inputs(c)
-    run = GpuRun(c, inp)
+    run = LayerOnGpu(c, inp)
     rng = np.random.default_rng(11)
     xs = [torch.as_tensor(rng.standard_normal(inp["x"].shape).astype(np.float32)).to(run.dt)
           .contiguous().to(run.dev) for _ in range(4)]
@@ -306,7 +306,7 @@ def test_back_to_back_calls_on_one_workspace():
 
 def test_bitwise_determinism():
     c = SMALL["quartz_s"]
-    run = GpuRun(c, make_inputs(c))
+    run = LayerOnGpu(c, make_inputs(c))
     y1, a1, _ = run.layer()
     y1 = y1.clone()
     y2, a2, _ = run.layer()
@@ -335,7 +335,7 @@ def test_full_size(name):
     definition; the loss. Launch configuration as the benchmark runs it (moe_layer_forward)."""
     c = get_config(name)
     inp = make_inputs(c)
-    run = GpuRun(c, inp)
+    run = LayerOnGpu(c, inp)
     o = run.steps()
     ref = oracle.layer_forward(c, inp, with_outputs=False)
     r, pm = ref["route"], ref["perm"]

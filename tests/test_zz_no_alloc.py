@@ -14,7 +14,7 @@ import torch
 
 from fine_grained_mixture_moe_b200 import binding as B
 from moe_synth import get_config, make_inputs
-from tests.gpu_helpers import GpuRun, np_
+from tests.gpu_helpers import LayerOnGpu, np_
 
 pytestmark = pytest.mark.gpu
 
@@ -27,7 +27,7 @@ def _lib():
 
 
 def _route_both(c):
-    run = GpuRun(c, make_inputs(c))
+    run = LayerOnGpu(c, make_inputs(c))
     T, k, E, dev = run.cfg.T, run.cfg.top_k, run.cfg.E, run.dev
     outs = []
     for noalloc in (False, True):
