@@ -40,8 +40,8 @@ constexpr int RT_THREADS = 32 * RT_WARPS;
 constexpr int RT_TPT = 8;          // tokens per thread
 constexpr int RT_EPT = 3;          // experts per thread
 constexpr int RT_EB = 8 * RT_EPT;  // experts per round
-constexpr int RT_SEL_THREAD_MAX_E = 64;  // up to this many experts: one thread per (token,
-                                         // expert) ranks; above, a warp per token
+constexpr int RT_SEL_THREAD_MAX_E = 64;  // ranking: up to this many experts each lane counts
+                                         // the rank of its own; above, iterative warp argmax
 constexpr int EXPANSION_MAX = 40;
 
 struct RouterArgs {
