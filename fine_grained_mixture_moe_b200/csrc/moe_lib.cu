@@ -44,8 +44,9 @@ bool cfg_supported(const moe_config_t *c) {
   if (c->n_shared > 0 && (c->ffn_shared <= 0 || c->ffn_shared % 64)) return false;
   if (!std::isfinite(c->capacity_factor) || !std::isfinite(c->aux_alpha)) return false;
   // the router stages its 16 token rows and the logits in shared memory (227 KB per CTA)
-  if (router_smem(c->E, c->score == MOE_SCORE_SIGMOID, c->d,
-                  c->dtype == MOE_DTYPE_BF16 ? 2 : 4).total > 227 * 1024)
+  const bool sig = c->score == MOE_SCORE_SIGMOID;
+  const int es = c->dtype == MOE_DTYPE_BF16 ? 2 : 4;
+  if (router_smem(c->E, sig, c->d, es, router_ept(c->E, sig, c->d, es)).total > 227 * 1024)
     return false;
   // 32-bit row indices inside the kernels
   if ((long long)c->T * c->top_k * std::max(c->d, 256) >= (1ll << 31) * 64ll) return false;
@@ -351,15 +352,24 @@ moe_status_t launch_gemm(const moe_config_t *c, const GroupedGemm &g, int bn_hin
     if (_s != MOE_OK) return _s;        \
   } while (0)
 
+template <typename Tin, int EPT>
+moe_status_t launch_router_ept(const RouterArgs &a, cudaStream_t st) {
+  const size_t smem =
+      router_smem(a.E, a.score == MOE_SCORE_SIGMOID, a.d, (int)sizeof(Tin), EPT).total;
+  if (smem > 227 * 1024) return MOE_ERR_UNSUPPORTED;
+  if (cudaFuncSetAttribute(router_kernel<Tin, EPT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)smem) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  return launch_pdl(router_kernel<Tin, EPT>, dim3(ceil_div(a.T, RT_TM)), dim3(RT_THREADS), smem,
+                    st, a);
+}
+
 template <typename Tin>
 moe_status_t launch_router(const RouterArgs &a, cudaStream_t st) {
   ProfScope ps(K_ROUTER, st);
-  const size_t smem = router_smem(a.E, a.score == MOE_SCORE_SIGMOID, a.d, (int)sizeof(Tin)).total;
-  if (smem > 227 * 1024) return MOE_ERR_UNSUPPORTED;
-  if (cudaFuncSetAttribute(router_kernel<Tin>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)smem) != cudaSuccess)
-    return MOE_ERR_CUDA;
-  return launch_pdl(router_kernel<Tin>, dim3(ceil_div(a.T, RT_TM)), dim3(RT_THREADS), smem, st, a);
+  if (router_ept(a.E, a.score == MOE_SCORE_SIGMOID, a.d, (int)sizeof(Tin)) == RT_EPT_WIDE)
+    return launch_router_ept<Tin, RT_EPT_WIDE>(a, st);
+  return launch_router_ept<Tin, RT_EPT>(a, st);
 }
 
 moe_status_t launch_stats(const StatsArgs &sa, cudaStream_t st) {

@@ -36,10 +36,11 @@ constexpr int RT_TM = 16;          // tokens per CTA
 constexpr int RT_WARPS = 8;        // each takes every 8th slice of the d dimension
 constexpr int RT_THREADS = 32 * RT_WARPS;
 // Screen tiling. Lane = ks + 2 (eg + 8 tg): tg in {0,1} picks tokens tg, tg+2, ..., tg+14;
-// eg in 0..7 picks experts eg, eg+8, eg+16 of the round; ks in {0,1} halves the warp's d slice.
+// eg in 0..7 picks experts eg, eg+8, ... of the round; ks in {0,1} halves the warp's d slice.
 constexpr int RT_TPT = 8;          // tokens per thread
-constexpr int RT_EPT = 3;          // experts per thread
-constexpr int RT_EB = 8 * RT_EPT;  // experts per round
+constexpr int RT_EPT = 3;          // experts per thread (6 in the wide form for many experts)
+constexpr int RT_EPT_WIDE = 6;
+constexpr int RT_WIDE_MIN_E = 97;  // the wide form from this many experts, when it fits
 constexpr int RT_SEL_THREAD_MAX_E = 64;  // ranking: up to this many experts each lane counts
                                          // the rank of its own; above, iterative warp argmax
 constexpr int EXPANSION_MAX = 40;
@@ -401,7 +402,7 @@ constexpr int RT_WD = 4;  // W chunks in flight per lane pair (cp.async ring)
 struct RouterSmem {
   size_t xs, xs_stride, ring, part, wsq, wn, off, lg, keys, byrank, cnt, xnorm, cmask, total;
 };
-__host__ __device__ inline RouterSmem router_smem(int E, bool sigmoid, int d, int esize) {
+__host__ __device__ inline RouterSmem router_smem(int E, bool sigmoid, int d, int esize, int ept) {
   RouterSmem L;
   size_t o = 0;
   auto take = [&](size_t bytes) { size_t at = o; o = (o + bytes + 15) & ~(size_t)15; return at; };
@@ -411,9 +412,9 @@ __host__ __device__ inline RouterSmem router_smem(int E, bool sigmoid, int d, in
   L.xs = take((size_t)RT_TM * L.xs_stride);
   // rings of W chunks, one per lane pair (lanes tg = 0, 1 use the same chunks):
   // [slot][expert][16-byte part][pair]
-  L.ring = take((size_t)RT_WD * RT_EPT * (RT_THREADS / 2) * 8 * esize);
-  L.part = take((size_t)RT_WARPS * RT_TM * RT_EB * sizeof(float));  // per-warp partial logits
-  L.wsq = take((size_t)RT_WARPS * RT_EB * sizeof(float));           // per-warp W sums of squares
+  L.ring = take((size_t)RT_WD * ept * (RT_THREADS / 2) * 8 * esize);
+  L.part = take((size_t)RT_WARPS * RT_TM * 8 * ept * sizeof(float));  // per-warp partial logits
+  L.wsq = take((size_t)RT_WARPS * 8 * ept * sizeof(float));           // per-warp W sums of squares
   L.wn = take((size_t)E * sizeof(double));
   L.off = take((size_t)E * sizeof(float));
   L.lg = take((size_t)RT_TM * E * sizeof(float));
@@ -424,6 +425,14 @@ __host__ __device__ inline RouterSmem router_smem(int E, bool sigmoid, int d, in
   L.cmask = take((size_t)RT_TM * ((E + 31) / 32) * sizeof(unsigned));  // candidates per listed token
   L.total = o;
   return L;
+}
+
+// Experts per thread of a launch: the wide tile from RT_WIDE_MIN_E experts when its shared memory
+// fits, else the narrow one.
+__host__ __device__ inline int router_ept(int E, bool sigmoid, int d, int esize) {
+  if (E >= RT_WIDE_MIN_E && router_smem(E, sigmoid, d, esize, RT_EPT_WIDE).total <= 227 * 1024)
+    return RT_EPT_WIDE;
+  return RT_EPT;
 }
 
 // Upper bound on sqrt(sum of squares) from an fp32 accumulation of at most n = d + 16 fused
@@ -543,8 +552,11 @@ __device__ __noinline__ void finish_token(const RouterArgs &a, float *lrow, cons
   __syncwarp();
 }
 
-template <typename Tin>
-__global__ void __launch_bounds__(RT_THREADS, 2) router_kernel(RouterArgs a) {
+// EPT experts per thread (a round covers 8 EPT experts): 3 for up to 96 experts (two CTAs per SM),
+// 6 above, where the logit rows already hold one CTA per SM and the wider tile halves the rounds.
+template <typename Tin, int EPT>
+__global__ void __launch_bounds__(RT_THREADS, EPT == RT_EPT ? 2 : 1) router_kernel(RouterArgs a) {
+  constexpr int EB = 8 * EPT;  // experts per round
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   using CH = Chunk8<Tin>;
   const int E = a.E, d = a.d, k = a.k;
@@ -556,11 +568,11 @@ __global__ void __launch_bounds__(RT_THREADS, 2) router_kernel(RouterArgs a) {
   const int force_level = g_force_exact;
   const bool force = force_level != 0;
   const bool sigmoid = a.score == MOE_SCORE_SIGMOID;
-  const RouterSmem SL = router_smem(E, sigmoid, d, (int)sizeof(Tin));
-  uint4 *ring = (uint4 *)(smem_raw + SL.ring);   // [RT_WD][RT_EPT][PARTS][RT_THREADS / 2]
+  const RouterSmem SL = router_smem(E, sigmoid, d, (int)sizeof(Tin), EPT);
+  uint4 *ring = (uint4 *)(smem_raw + SL.ring);   // [RT_WD][EPT][PARTS][RT_THREADS / 2]
   float *off_s = (float *)(smem_raw + SL.off);   // [E] logit offsets (zeros without)
-  float *part = (float *)(smem_raw + SL.part);   // [RT_WARPS][RT_TM][RT_EB]
-  float *wsq_s = (float *)(smem_raw + SL.wsq);   // [RT_WARPS][RT_EB]
+  float *part = (float *)(smem_raw + SL.part);   // [RT_WARPS][RT_TM][EB]
+  float *wsq_s = (float *)(smem_raw + SL.wsq);   // [RT_WARPS][EB]
   double *wn = (double *)(smem_raw + SL.wn);     // [E] upper bounds of |W_e|_2
   float *lg = (float *)(smem_raw + SL.lg);       // [RT_TM][E] logits, then probabilities
   float *keys = (float *)(smem_raw + SL.keys);   // [RT_TM][E] sigmoid keys
@@ -604,7 +616,7 @@ __global__ void __launch_bounds__(RT_THREADS, 2) router_kernel(RouterArgs a) {
   const int nmine = c0 < nch ? (nch - c0 + 2 * RT_WARPS - 1) / (2 * RT_WARPS) : 0;
   const int pr = warp * 16 + (lane & 15);  // the lane pair
   constexpr int NP = RT_THREADS / 2;
-  auto slot_ptr = [&](int s, int j) { return ring + ((size_t)(s * RT_EPT + j) * CH::PARTS) * NP + pr; };
+  auto slot_ptr = [&](int s, int j) { return ring + ((size_t)(s * EPT + j) * CH::PARTS) * NP + pr; };
   // copies of chunk n of the pair's expert rows of the round at eb into slot n % RT_WD, the
   // 16-byte parts q = j PARTS + u dealt to the two lanes by q % 2 = tg; one commit group per
   // call, empty or not, so that the group count stays uniform
@@ -612,7 +624,7 @@ __global__ void __launch_bounds__(RT_THREADS, 2) router_kernel(RouterArgs a) {
     if (n < nmine) {
       const int c = c0 + 2 * RT_WARPS * n;
 #pragma unroll
-      for (int j = 0; j < RT_EPT; ++j) {
+      for (int j = 0; j < EPT; ++j) {
         const int e = eb + eg + 8 * j;
 #pragma unroll
         for (int u = 0; u < CH::PARTS; ++u)
@@ -626,7 +638,7 @@ __global__ void __launch_bounds__(RT_THREADS, 2) router_kernel(RouterArgs a) {
   // the first chunks of a round; parts of experts past E are zeroed (never copied into)
   auto ring_prologue = [&](int eb) {
 #pragma unroll
-    for (int j = 0; j < RT_EPT; ++j)
+    for (int j = 0; j < EPT; ++j)
 #pragma unroll
       for (int u = 0; u < CH::PARTS; ++u)
         if (((j * CH::PARTS + u) & 1) == tg && eb + eg + 8 * j >= E)
@@ -679,17 +691,17 @@ __global__ void __launch_bounds__(RT_THREADS, 2) router_kernel(RouterArgs a) {
     if (q16 == 0) xnorm[tt] = norm_upper((double)s, d);
   }
 
-  // ---- screen: approximate logits in fp32, RT_EB experts per round. Warp w takes the chunks
-  // 2w + ks + 16n of d; per chunk a thread takes its 3 expert chunks from its ring (filled
-  // RT_WD chunks ahead) and its 8 token chunks from the staged rows, and accumulates 24 (token,
-  // expert) pairs as two-lane packed FMAs (even and odd elements in the two lanes of a pair).
+  // ---- screen: approximate logits in fp32, EB experts per round. Warp w takes the chunks
+  // 2w + ks + 16n of d; per chunk a thread takes its EPT expert chunks from its ring (filled
+  // RT_WD chunks ahead) and its 8 token chunks from the staged rows, and accumulates 8 EPT
+  // (token, expert) pairs as two-lane packed FMAs (even and odd elements in the two lanes).
   // The sums of squares of the W rows ride along: lane tg squares pairs 2tg, 2tg+1 of a chunk.
   const size_t xs_es = xs_stride / sizeof(Tin);  // row stride in elements
   const Tin *xrow0 = (const Tin *)(xs + (size_t)tg * xs_stride);
-  for (int eb = 0; eb < E; eb += RT_EB) {
-    float2 acc[RT_TPT][RT_EPT], wsq[RT_EPT];
+  for (int eb = 0; eb < E; eb += EB) {
+    float2 acc[RT_TPT][EPT], wsq[EPT];
 #pragma unroll
-    for (int j = 0; j < RT_EPT; ++j) {
+    for (int j = 0; j < EPT; ++j) {
       wsq[j] = make_float2(0.f, 0.f);
 #pragma unroll
       for (int tj = 0; tj < RT_TPT; ++tj) acc[tj][j] = make_float2(0.f, 0.f);
@@ -703,9 +715,9 @@ __global__ void __launch_bounds__(RT_THREADS, 2) router_kernel(RouterArgs a) {
       else cp_async_commit();
       cp_async_wait<RT_WD>();
       __syncwarp();
-      float2 w2[RT_EPT][4];
+      float2 w2[EPT][4];
 #pragma unroll
-      for (int j = 0; j < RT_EPT; ++j) {
+      for (int j = 0; j < EPT; ++j) {
         CH wc;
         wc.ld_ring(slot_ptr(n % RT_WD, j), NP);
 #pragma unroll
@@ -722,48 +734,48 @@ __global__ void __launch_bounds__(RT_THREADS, 2) router_kernel(RouterArgs a) {
         for (int i = 0; i < 4; ++i) {
           const float2 x2 = xc.pair(i);
 #pragma unroll
-          for (int j = 0; j < RT_EPT; ++j) acc[tj][j] = __ffma2_rn(x2, w2[j][i], acc[tj][j]);
+          for (int j = 0; j < EPT; ++j) acc[tj][j] = __ffma2_rn(x2, w2[j][i], acc[tj][j]);
         }
       }
     }
     cp_async_wait<0>();
     __syncwarp();  // both lanes done with the ring before the next round's copies
-    if (eb + RT_EB < E) ring_prologue(eb + RT_EB);  // the next round's W, during this reduction
+    if (eb + EB < E) ring_prologue(eb + EB);  // the next round's W, during this reduction
     // fold the two lanes of each pair, then the two k halves (lanes ks = 0, 1); lane ks = 0
     // stores tokens tg + 2tj for tj < 4, lane ks = 1 the rest
-    float *pw = part + (size_t)warp * RT_TM * RT_EB;
+    float *pw = part + (size_t)warp * RT_TM * EB;
 #pragma unroll
     for (int tj = 0; tj < RT_TPT; ++tj)
 #pragma unroll
-      for (int j = 0; j < RT_EPT; ++j) {
+      for (int j = 0; j < EPT; ++j) {
         float v = __fadd_rn(acc[tj][j].x, acc[tj][j].y);
         v = __fadd_rn(v, __shfl_xor_sync(0xffffffffu, v, 1));
-        if ((tj >> 2) == ks) pw[(tg + 2 * tj) * RT_EB + eg + 8 * j] = v;
+        if ((tj >> 2) == ks) pw[(tg + 2 * tj) * EB + eg + 8 * j] = v;
       }
 #pragma unroll
-    for (int j = 0; j < RT_EPT; ++j) {
+    for (int j = 0; j < EPT; ++j) {
       float s = __fadd_rn(wsq[j].x, wsq[j].y);
       s = __fadd_rn(s, __shfl_xor_sync(0xffffffffu, s, 16));
       s = __fadd_rn(s, __shfl_xor_sync(0xffffffffu, s, 1));
-      if (tg == 0 && ks == 0) wsq_s[warp * RT_EB + eg + 8 * j] = s;
+      if (tg == 0 && ks == 0) wsq_s[warp * EB + eg + 8 * j] = s;
     }
     __syncthreads();
     // per-warp partials added in warp order, then the offset: every product passes through at
     // most 4 ceil(d/128) (its chain) + 1 + 1 + 7 + 1 roundings
-    for (int q = tid; q < RT_TM * RT_EB; q += RT_THREADS) {
-      const int tt = q / RT_EB, el = q - tt * RT_EB, e = eb + el;
+    for (int q = tid; q < RT_TM * EB; q += RT_THREADS) {
+      const int tt = q / EB, el = q - tt * EB, e = eb + el;
       if (tt < ntok && e < E) {
-        float s = part[tt * RT_EB + el];
+        float s = part[tt * EB + el];
 #pragma unroll
-        for (int w = 1; w < RT_WARPS; ++w) s = __fadd_rn(s, part[(w * RT_TM + tt) * RT_EB + el]);
+        for (int w = 1; w < RT_WARPS; ++w) s = __fadd_rn(s, part[(w * RT_TM + tt) * EB + el]);
         if (a.off) s = __fadd_rn(s, off_s[e]);
         lg[tt * E + e] = s;
       }
     }
-    if (tid < RT_EB && eb + tid < E) {
+    if (tid < EB && eb + tid < E) {
       float s = wsq_s[tid];
 #pragma unroll
-      for (int w = 1; w < RT_WARPS; ++w) s = __fadd_rn(s, wsq_s[w * RT_EB + tid]);
+      for (int w = 1; w < RT_WARPS; ++w) s = __fadd_rn(s, wsq_s[w * EB + tid]);
       const double nrm = norm_upper((double)s, d);
       wn[eb + tid] = nrm;
       atomicMax(&s_wnmax, (unsigned long long)__double_as_longlong(nrm));
