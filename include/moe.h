@@ -25,7 +25,8 @@
  *   - Shapes: d, ffn, ffn_shared and rank must be multiples of 64; 1 <= top_k <= min(E, 8);
  *     1 <= E <= 1024; n_shared <= 8; rank <= 256; the router's per-CTA tile (16 token rows of
  *     d elements, the staging ring of the router rows and 16 x E logits) must fit in 227 KB of
- *     shared memory, so d up to about 6,000 (bf16) or 2,600 (fp32) for small E. T may be 0.
+ *     shared memory, so d up to about 6,000 (bf16) or 2,600 (fp32) for small E, and at
+ *     d = 1536 with sigmoid keys E up to 991. T may be 0.
  *     Other values return MOE_ERR_UNSUPPORTED.
  *   - Inputs must be finite. Router logits of +-inf or NaN make the routing unspecified.
  */

@@ -102,6 +102,17 @@ def test_hidden_size_limit_of_the_router_tile(lib, dtype, d_max):
     assert B.moe_workspace_size(too_big) == 0
 
 
+def test_expert_limit_falls_back_to_the_narrow_router_tile(lib):
+    """From 97 experts the router keeps six experts per thread when that tile's shared memory
+    fits, else three. At d = 1536 with sigmoid keys the wide tile holds up to 733 experts and the
+    narrow one up to 991: every E up to 991 must be accepted, 992 refused."""
+    def cfg(E):
+        return B.make_config(T=16, d=1536, E=E, top_k=4, ffn=64, score="sigmoid")
+    for E in (97, 733, 734, 991):
+        assert B.moe_workspace_size(cfg(E)) > 0, E
+    assert B.moe_workspace_size(cfg(992)) == 0
+
+
 def test_bad_pointers_and_workspace_are_rejected_on_the_host(lib):
     cfg = B.make_config(T=16, d=128, E=8, top_k=2, ffn=64)
     w = B.MoEWeights()

@@ -58,6 +58,10 @@ EDGE = {
     "k8_E65_sigmoid": MoEConfig(name="k8e65", T=97, d=128, E=65, top_k=8, n_shared=0, ffn=64,
                                 ffn_shared=0, score="sigmoid", norm_topk=True,
                                 bias=("uniform", 0.1)),
+    # the first expert count of the six-experts-per-thread router tile: its second round of 48
+    # experts is full, the third holds one expert
+    "k8_E97": MoEConfig(name="k8e97", T=131, d=192, E=97, top_k=8, n_shared=1, ffn=64,
+                        ffn_shared=64, offset=("normal", 0.5)),
     # a wide hidden size: 16 staged token rows of 8 KB in the router, K = 4096 in gate/up
     "d4096": MoEConfig(name="d4096", T=45, d=4096, E=8, top_k=2, n_shared=1, ffn=128,
                        ffn_shared=128, offset=("normal", 0.5)),
