@@ -169,6 +169,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TC_THREADS, 1)
                                     ? (routed ? &P.maps.b1_r : &P.maps.b1_s)
                                     : (routed ? &P.maps.b0_r : &P.maps.b0_s);
         const int a_row = ti.a_row0 + ti.m0 + (int)rank * 128;
+        // CTA 1's half of a group's last tile can hold no row of the group (an expert's tail of
+        // at most 128 rows): its A rows are never stored, so they are not loaded. The MMA reads
+        // what that stage last held there and the epilogue masks those rows; the leader expects
+        // the smaller byte count. Both CTAs decide it from the same tile record.
+        const bool a1_void = ti.m0 + 128 >= ti.rows;
+        const uint32_t stage_tx = 2 * C::STAGE_BYTES - (a1_void ? C::A_BYTES : 0);
         const int n_off = MODE == MODE_GATEUP ? 0 : (int)rank * 128;
         const int nk = ti.K / TC_BK;
         for (int kb = 0; kb < nk; ++kb) {
@@ -178,7 +184,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TC_THREADS, 1)
           }
           const uint32_t sA = smem_u32(stages + (size_t)stage * C::STAGE_BYTES);
           const uint32_t sB = sA + C::A_BYTES;
-          if (rank == 0) mbar_expect_tx(full_bar(stage), 2 * C::STAGE_BYTES);
+          if (rank == 0) mbar_expect_tx(full_bar(stage), stage_tx);
           const int kk = kb * TC_BK;
           int b_row, b_col;
           if (routed) {
@@ -189,7 +195,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TC_THREADS, 1)
             b_row = piece * p.piece_rows + ti.n0 + n_off;
             b_col = kk - piece * p.piece_k;
           }
-          tma_load_2d_pair(sA, ma, kk, a_row, full_bar(stage));
+          if (rank == 0 || !a1_void) tma_load_2d_pair(sA, ma, kk, a_row, full_bar(stage));
           tma_load_2d_pair(sB, mb, b_col, b_row, full_bar(stage));
           issued[stage] = true;
           issued_parity[stage] = (int)phase;
@@ -273,8 +279,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TC_THREADS, 1)
       const int ldo = routed ? p.ldo_r : p.ldo_s;
       const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * C::ACC_COLS);
       unsigned char *stg = stg_all + (warp - 2) * 4096;
+      const int cstop = rbase < ti.rows ? cend : cbeg;  // a warp of padding rows only: nothing to store
 #pragma unroll 1
-      for (int c = cbeg; c < cend; c += 32) {
+      for (int c = cbeg; c < cstop; c += 32) {
         if (MODE == MODE_GATEUP) {
           // silu(gate) * up in bf16, 64 columns (128 bytes of each row) at a time: both 32-column
           // halves are packed, staged per warp and written as 32 coalesced 128-byte row stores
