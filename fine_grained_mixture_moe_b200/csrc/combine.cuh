@@ -49,26 +49,31 @@ template <> struct YVec<__nv_bfloat16> {
 // with the pass's k row loads and the shared-output load issued before the sums. About 60
 // registers, so 4 CTAs (32 warps) fit per SM and a Quartz-sized call is one wave. d is a
 // multiple of 64, so a lane's vector is wholly inside or wholly outside the row.
+// early: slot_pos and w were written at least two kernels before this one in the stream (inside
+// the layer, the expert GEMMs lie between the scatter and the combine). The kernel just before
+// lets this one start only after its own griddep_wait, so they are final at entry and are read
+// (through L2) before griddep_wait; only y_perm and y_shared wait for it.
 template <typename Ty>
 __global__ void __launch_bounds__(256, sizeof(Ty) == 2 ? 4 : 3) combine_kernel(const Ty *__restrict__ y_perm,
                                                          const float *__restrict__ y_shared,
                                                          const int32_t *__restrict__ slot_pos,
                                                          const float *__restrict__ w,
                                                          float *__restrict__ y, int T, int k,
-                                                         int d) {
-  griddep_wait();
-  griddep_launch();
+                                                         int d, bool early) {
   using YV = YVec<Ty>;
   constexpr int V = YV::N;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t = blockIdx.x * 8 + warp;
-  if (t >= T) return;
+  if (!early) griddep_wait();
   int pos_l = -1;
   float w_l = 0.0f;
-  if (lane < k) {
-    pos_l = slot_pos[(size_t)t * k + lane];
-    w_l = w[(size_t)t * k + lane];
+  if (t < T && lane < k) {
+    pos_l = __ldcg(slot_pos + (size_t)t * k + lane);
+    w_l = __ldcg(w + (size_t)t * k + lane);
   }
+  if (early) griddep_wait();
+  griddep_launch();
+  if (t >= T) return;
   int pos[8];
   float wj[8];
 #pragma unroll

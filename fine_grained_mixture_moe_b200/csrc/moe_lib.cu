@@ -536,17 +536,20 @@ moe_status_t experts_impl(const moe_config_t *c, const void *x_perm, const int32
   return MOE_OK;
 }
 
+// early: slot_pos and wts were written at least two kernels back in the stream (combine.cuh).
 moe_status_t combine_impl(const moe_config_t *c, const void *y_perm, const void *y_shared,
-                          const int32_t *slot_pos, const float *wts, void *y, cudaStream_t st) {
+                          const int32_t *slot_pos, const float *wts, void *y, cudaStream_t st,
+                          bool early) {
   if (c->T == 0) return MOE_OK;
   ProfScope ps(K_COMBINE, st);
   const float *ysh = c->n_shared > 0 ? (const float *)y_shared : nullptr;
   if (yperm_bf16(c))
     return launch_pdl(combine_kernel<__nv_bfloat16>, dim3(ceil_div(c->T, 8)), dim3(256), 0, st,
                       (const __nv_bfloat16 *)y_perm, ysh, slot_pos, wts, (float *)y, c->T,
-                      c->top_k, c->d);
+                      c->top_k, c->d, early);
   return launch_pdl(combine_kernel<float>, dim3(ceil_div(c->T, 8)), dim3(256), 0, st,
-                    (const float *)y_perm, ysh, slot_pos, wts, (float *)y, c->T, c->top_k, c->d);
+                    (const float *)y_perm, ysh, slot_pos, wts, (float *)y, c->T, c->top_k, c->d,
+                    early);
 }
 
 moe_status_t aux_impl(const moe_config_t *c, const int32_t *count, const float *prob, float *loss,
@@ -648,7 +651,7 @@ moe_status_t moe_combine(const moe_config_t *cfg, const void *y_perm, const void
   MOE_TRY(check_cfg(cfg));
   MOE_REQUIRE(tok16(cfg, y_perm) && tok16(cfg, slot_pos) && tok16(cfg, topk_w) && tok16(cfg, y));
   MOE_REQUIRE(cfg->n_shared == 0 || tok16(cfg, y_shared));
-  return combine_impl(cfg, y_perm, y_shared, slot_pos, topk_w, y, (cudaStream_t)stream);
+  return combine_impl(cfg, y_perm, y_shared, slot_pos, topk_w, y, (cudaStream_t)stream, false);
 }
 
 moe_status_t moe_aux_loss(const moe_config_t *cfg, const int32_t *expert_count,
@@ -712,8 +715,9 @@ moe_status_t moe_layer_forward(const moe_config_t *cfg, const void *x, const moe
   else
     MOE_TRY(scatter_impl<float>(cfg, x, idx, cb, sa.kept, offsets, slot_pos, src, x_perm, cnt,
                                 prob, aux, st));
+  // T > 0 here: the expert forward launched at least two kernels after the scatter
   MOE_TRY(experts_impl(cfg, x_perm, offsets, x, w, y_perm, y_sh, ws, st));
-  return combine_impl(cfg, y_perm, y_sh, slot_pos, wts, y, st);
+  return combine_impl(cfg, y_perm, y_sh, slot_pos, wts, y, st, true);
 }
 
 const char *moe_status_str(moe_status_t s) {

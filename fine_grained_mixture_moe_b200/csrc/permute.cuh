@@ -65,8 +65,6 @@ __global__ void __launch_bounds__(256) perm_scatter_kernel(
     int32_t *__restrict__ offsets, int32_t *__restrict__ slot_pos, int32_t *__restrict__ src,
     const Tin *__restrict__ x, Tin *__restrict__ x_perm, int d, const int32_t *__restrict__ count,
     const float *__restrict__ prob, float alpha, float *__restrict__ aux) {
-  griddep_wait();
-  griddep_launch();
   // [PM_TPC rows][row_bytes] | lane masks [E] | chunk base [E] | offsets [E]
   extern __shared__ __align__(128) unsigned char sm_raw[];
   __shared__ int s_pos[PM_CHUNK * 8];
@@ -85,6 +83,11 @@ __global__ void __launch_bounds__(256) perm_scatter_kernel(
   const int nrows = max(0, min(PM_TPC, T - tfirst));
   const bool copy = x_perm != nullptr && nrows > 0;
   const uint32_t bar = smem_u32(&s_bar);
+  // Before griddep_wait: this kernel always follows the statistics kernel, whose CTAs allow it
+  // to start only after their own griddep_wait, i.e. once the kernel before the statistics (the
+  // router or the histogram) has completed and flushed. So x (an input of the call) and the
+  // routing are final here; only the statistics' outputs (chunk bases, kept counts) wait. The
+  // routing is read through L2 (ld.global.cg).
   if (tid == 0) {  // the rows do not depend on the routing: their copies go out first
     s_abort = 0;
     mbar_init(bar, 1);
@@ -105,11 +108,13 @@ __global__ void __launch_bounds__(256) perm_scatter_kernel(
     for (int j = 0; j < 8; ++j) {
       ev[j] = -1;
       if (j < k && valid) {
-        const int e = idx[(size_t)t * k + j];
+        const int e = __ldcg(idx + (size_t)t * k + j);
         if (e >= 0 && e < E) ev[j] = e;
       }
     }
   }
+  griddep_wait();
+  griddep_launch();
   for (int e = tid; e < E; e += blockDim.x) {
     smask[e] = 0u;
     s_base[e] = chunk_base[(size_t)chunk * E + e];
