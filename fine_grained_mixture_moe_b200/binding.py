@@ -76,6 +76,11 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
         "moe_combine": (c_int32, [P(MoEConfig), c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                                   c_void_p]),
         "moe_aux_loss": (c_int32, [P(MoEConfig), c_void_p, c_void_p, c_void_p, c_void_p]),
+        "moe_combine_backward": (c_int32, [P(MoEConfig), c_void_p, c_void_p, c_void_p, c_void_p,
+                                           c_void_p, c_void_p, c_void_p]),
+        "moe_route_backward": (c_int32, [P(MoEConfig), c_void_p, P(MoEWeights), c_void_p,
+                                         c_void_p, c_void_p, ctypes.c_float, c_void_p, c_void_p,
+                                         c_void_p, c_void_p]),
         "moe_bias_update": (c_int32, [P(MoEConfig), c_void_p, c_void_p, ctypes.c_float, c_void_p]),
         "moe_layer_forward": (c_int32, [P(MoEConfig), c_void_p, P(MoEWeights), c_void_p,
                                         c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
@@ -98,6 +103,7 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
 
 EXPORTED = ("moe_workspace_size", "moe_capacity", "moe_route", "moe_permute",
             "moe_expert_forward", "moe_combine", "moe_aux_loss", "moe_bias_update",
+            "moe_combine_backward", "moe_route_backward",
             "moe_layer_forward",
             "moe_status_str", "moe_get_device_error", "moe_debug_set", "moe_profile_read",
             "moe_debug_wait_timeout_probe", "moe_route_noalloc")
@@ -184,6 +190,23 @@ def moe_combine(cfg, y_perm, y_shared, slot_pos, topk_w, y, stream=None) -> None
     _check("moe_combine", load().moe_combine(ctypes.byref(cfg), _ptr(y_perm), _ptr(y_shared),
                                              _ptr(slot_pos), _ptr(topk_w), _ptr(y),
                                              _stream(stream)))
+
+
+def moe_combine_backward(cfg, dy, y_perm, slot_pos, topk_w, dy_perm, d_topk_w,
+                         stream=None) -> None:
+    _check("moe_combine_backward",
+           load().moe_combine_backward(ctypes.byref(cfg), _ptr(dy), _ptr(y_perm), _ptr(slot_pos),
+                                       _ptr(topk_w), _ptr(dy_perm), _ptr(d_topk_w),
+                                       _stream(stream)))
+
+
+def moe_route_backward(cfg, x, w: MoEWeights, topk_idx, expert_count, d_topk_w, d_loss: float,
+                       d_logits, d_w_router, dx, stream=None) -> None:
+    _check("moe_route_backward",
+           load().moe_route_backward(ctypes.byref(cfg), _ptr(x), ctypes.byref(w), _ptr(topk_idx),
+                                     _ptr(expert_count), _ptr(d_topk_w), ctypes.c_float(d_loss),
+                                     _ptr(d_logits), _ptr(d_w_router), _ptr(dx),
+                                     _stream(stream)))
 
 
 def moe_aux_loss(cfg, expert_count, prob_sum, loss, stream=None) -> None:

@@ -1,0 +1,209 @@
+// Backward of the combine and of the router: the derivative of the forward, with no gradient
+// through the selection, the capacity drops or the loss's counts, none for the selection bias or
+// the logit offsets, and the logits' fp32 rounding taken with derivative 1.
+//
+// combine_backward (Moonfrost expert card: a token's output sums its shared and top-k routed
+// experts): for every kept pair (t, j) with p = slot_pos[t, j] >= 0,
+//   dy_perm[p]     = topk_w[t, j] * dy[t]
+//   d_topk_w[t, j] = sum_c dy[t, c] * y_perm[p, c]     (0 for a dropped pair)
+// route_backward, per token:
+//   l = x W_r^T + off (fp32 FMAs), p = softmax(l) or sigmoid(l);
+//   dp from d_topk_w, through w_j = p_j / sum of the k selected p_j when norm_topk is set;
+//   the loss term dq_i = dL alpha E f_i / T, f_i = count_i / (T k) (Quartz research page,
+//   architecture table, row "Router": load-balancing weight 0.01), which for sigmoid scores
+//   enters through q = sigmoid / sum over all E;
+//   d_logits = p (dp + dq - <dp + dq, p>) (softmax) or dsigma sigma (1 - sigma) (sigmoid).
+// then d_w_router = d_logits^T x and dx = d_logits W_r, every sum in a fixed order.
+#pragma once
+#include "common.cuh"
+
+namespace moe {
+
+// four consecutive elements of a row, as fp32
+template <typename Ty> struct Bw4;
+template <> struct Bw4<float> {
+  static __device__ __forceinline__ float4 ld(const float *p) { return *(const float4 *)p; }
+  static __device__ __forceinline__ void st(float *p, float4 v) { *(float4 *)p = v; }
+};
+template <> struct Bw4<__nv_bfloat16> {
+  static __device__ __forceinline__ float4 ld(const __nv_bfloat16 *p) {
+    const uint2 u = *(const uint2 *)p;
+    const float2 a = __bfloat1622float2(*(const __nv_bfloat162 *)&u.x);
+    const float2 b = __bfloat1622float2(*(const __nv_bfloat162 *)&u.y);
+    return make_float4(a.x, a.y, b.x, b.y);
+  }
+  static __device__ __forceinline__ void st(__nv_bfloat16 *p, float4 v) {
+    const __nv_bfloat162 a = __floats2bfloat162_rn(v.x, v.y);
+    const __nv_bfloat162 b = __floats2bfloat162_rn(v.z, v.w);
+    uint2 u;
+    u.x = *(const uint32_t *)&a;
+    u.y = *(const uint32_t *)&b;
+    *(uint2 *)p = u;
+  }
+};
+
+// One warp per token; lane l takes the columns 4l, 4l + 128, ...; each of the k dot products is
+// reduced over the lanes in a fixed tree.
+template <typename Ty>
+__global__ void __launch_bounds__(256) combine_backward_kernel(
+    const float *__restrict__ dy, const Ty *__restrict__ y_perm,
+    const int32_t *__restrict__ slot_pos, const float *__restrict__ w, Ty *__restrict__ dy_perm,
+    float *__restrict__ d_w, int T, int k, int d) {
+  griddep_wait();
+  griddep_launch();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t = blockIdx.x * 8 + warp;
+  if (t >= T) return;
+  int pos[8];
+  float wj[8], dot[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    pos[j] = j < k ? slot_pos[(size_t)t * k + j] : -1;
+    wj[j] = j < k ? w[(size_t)t * k + j] : 0.0f;
+    dot[j] = 0.0f;
+  }
+#pragma unroll 1
+  for (int c = 4 * lane; c < d; c += 128) {
+    const float4 g = *(const float4 *)(dy + (size_t)t * d + c);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      if (pos[j] < 0) continue;
+      const float4 v = Bw4<Ty>::ld(y_perm + (size_t)pos[j] * d + c);
+      dot[j] = fmaf(g.x, v.x, dot[j]);
+      dot[j] = fmaf(g.y, v.y, dot[j]);
+      dot[j] = fmaf(g.z, v.z, dot[j]);
+      dot[j] = fmaf(g.w, v.w, dot[j]);
+      Bw4<Ty>::st(dy_perm + (size_t)pos[j] * d + c,
+                  make_float4(wj[j] * g.x, wj[j] * g.y, wj[j] * g.z, wj[j] * g.w));
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    if (j >= k) break;
+    const float s = warp_sum_f(dot[j]);
+    if (lane == 0) d_w[(size_t)t * k + j] = pos[j] >= 0 ? s : 0.0f;
+  }
+}
+
+struct RouteBwdArgs {
+  const void *x, *w_router;
+  const float *off;          // [E] or null
+  const int32_t *idx;        // [T, k]
+  const int32_t *count;      // [E] selections before capacity
+  const float *d_w;          // [T, k]
+  float *d_logits;           // [T, E]
+  int T, d, E, k, sigmoid, norm;
+  float alpha, dL;
+};
+
+// One warp per token; shared memory holds the warp's E logits (then probabilities) and dp.
+template <typename Tin>
+__global__ void __launch_bounds__(256) route_backward_kernel(RouteBwdArgs a) {
+  extern __shared__ float rb_smem[];
+  griddep_wait();
+  griddep_launch();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t = blockIdx.x * 8 + warp;
+  if (t >= a.T) return;  // no block-wide barrier below
+  const int E = a.E, d = a.d, k = a.k;
+  float *pr = rb_smem + (size_t)warp * 2 * E, *dp = pr + E;
+  const Tin *xr = (const Tin *)a.x + (size_t)t * d;
+  for (int e = 0; e < E; ++e) {
+    const Tin *we = (const Tin *)a.w_router + (size_t)e * d;
+    float s = 0.0f;
+    for (int c = 4 * lane; c < d; c += 128) {
+      const float4 u = Bw4<Tin>::ld(xr + c), v = Bw4<Tin>::ld(we + c);
+      s = fmaf(u.x, v.x, s);
+      s = fmaf(u.y, v.y, s);
+      s = fmaf(u.z, v.z, s);
+      s = fmaf(u.w, v.w, s);
+    }
+    s = warp_sum_f(s);
+    if (lane == 0) pr[e] = a.off ? s + a.off[e] : s;
+  }
+  __syncwarp();
+  float m = -INFINITY, ssum = 0.0f;
+  if (!a.sigmoid) {
+    for (int e = lane; e < E; e += 32) m = fmaxf(m, pr[e]);
+    m = warp_max_f(m);
+    for (int e = lane; e < E; e += 32) ssum += expf(pr[e] - m);
+  } else {
+    for (int e = lane; e < E; e += 32) ssum += 1.0f / (1.0f + expf(-pr[e]));
+  }
+  ssum = warp_sum_f(ssum);
+  __syncwarp();
+  for (int e = lane; e < E; e += 32) {
+    pr[e] = !a.sigmoid ? expf(pr[e] - m) / ssum : 1.0f / (1.0f + expf(-pr[e]));
+    dp[e] = 0.0f;
+  }
+  __syncwarp();
+  if (lane == 0) {  // the combine weights' gradient onto the selected probabilities
+    const int *ir = a.idx + (size_t)t * k;
+    const float *gw = a.d_w + (size_t)t * k;
+    if (a.norm) {
+      float S = 0.0f;
+      for (int j = 0; j < k; ++j) S += pr[ir[j]];
+      float inner = 0.0f;
+      for (int j = 0; j < k; ++j) inner = fmaf(gw[j], pr[ir[j]] / S, inner);
+      for (int j = 0; j < k; ++j) dp[ir[j]] += (gw[j] - inner) / S;
+    } else {
+      for (int j = 0; j < k; ++j) dp[ir[j]] += gw[j];
+    }
+  }
+  __syncwarp();
+  // loss term: dq_e = dL alpha E count_e / (T k T)
+  const float cq = a.dL * a.alpha * (float)E / ((float)a.T * (float)k * (float)a.T);
+  float *dl = a.d_logits + (size_t)t * E;
+  if (!a.sigmoid) {
+    float dot = 0.0f;
+    for (int e = lane; e < E; e += 32) dot = fmaf(dp[e] + cq * (float)a.count[e], pr[e], dot);
+    dot = warp_sum_f(dot);
+    for (int e = lane; e < E; e += 32) dl[e] = pr[e] * (dp[e] + cq * (float)a.count[e] - dot);
+  } else {
+    float qd = 0.0f;  // sum_j dq_j q_j
+    for (int e = lane; e < E; e += 32) qd = fmaf(cq * (float)a.count[e], pr[e] / ssum, qd);
+    qd = warp_sum_f(qd);
+    for (int e = lane; e < E; e += 32) {
+      const float ds = dp[e] + (cq * (float)a.count[e] - qd) / ssum;
+      dl[e] = ds * pr[e] * (1.0f - pr[e]);
+    }
+  }
+}
+
+template <typename Tin> __device__ __forceinline__ float bw_elem(const Tin *p, size_t i);
+template <> __device__ __forceinline__ float bw_elem<float>(const float *p, size_t i) { return p[i]; }
+template <> __device__ __forceinline__ float bw_elem<__nv_bfloat16>(const __nv_bfloat16 *p, size_t i) {
+  return __bfloat162float(p[i]);
+}
+
+// d_w_router[e, c] = sum over t (in order) of d_logits[t, e] x[t, c]; block (column tile, e).
+template <typename Tin>
+__global__ void __launch_bounds__(256) router_wgrad_kernel(const float *__restrict__ dl,
+                                                           const Tin *__restrict__ x, int T, int d,
+                                                           int E, float *__restrict__ dwr) {
+  griddep_wait();
+  griddep_launch();
+  const int e = blockIdx.y, c = blockIdx.x * 256 + threadIdx.x;
+  if (c >= d) return;
+  float acc = 0.0f;
+  for (int t = 0; t < T; ++t) acc = fmaf(dl[(size_t)t * E + e], bw_elem(x, (size_t)t * d + c), acc);
+  dwr[(size_t)e * d + c] = acc;
+}
+
+// dx[t, c] = sum over e (in order) of d_logits[t, e] W_r[e, c]; blocks stride over the tokens.
+template <typename Tin>
+__global__ void __launch_bounds__(256) router_dgrad_kernel(const float *__restrict__ dl,
+                                                           const Tin *__restrict__ wr, int T, int d,
+                                                           int E, float *__restrict__ dx) {
+  griddep_wait();
+  griddep_launch();
+  const int c = blockIdx.x * 256 + threadIdx.x;
+  if (c >= d) return;
+  for (int t = blockIdx.y; t < T; t += gridDim.y) {
+    float acc = 0.0f;
+    for (int e = 0; e < E; ++e) acc = fmaf(dl[(size_t)t * E + e], bw_elem(wr, (size_t)e * d + c), acc);
+    dx[(size_t)t * d + c] = acc;
+  }
+}
+
+}  // namespace moe

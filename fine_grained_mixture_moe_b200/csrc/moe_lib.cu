@@ -11,6 +11,7 @@
 #include <mutex>
 
 #include "../../include/moe.h"
+#include "backward.cuh"
 #include "combine.cuh"
 #include "common.cuh"
 #include "gemm_simt.cuh"
@@ -559,6 +560,23 @@ moe_status_t aux_impl(const moe_config_t *c, const int32_t *count, const float *
                     c->aux_alpha, loss);
 }
 
+// ------------------------------------------------------------------ backward of route and combine
+template <typename Tin>
+moe_status_t route_backward_impl(const moe_config_t *c, const RouteBwdArgs &a, float *d_w_router,
+                                 float *dx, cudaStream_t st) {
+  const size_t smem = (size_t)8 * 2 * c->E * sizeof(float);
+  if (smem > 48 * 1024 &&
+      cudaFuncSetAttribute(route_backward_kernel<Tin>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)smem) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  MOE_TRY(launch_pdl(route_backward_kernel<Tin>, dim3(ceil_div(c->T, 8)), dim3(256), smem, st, a));
+  MOE_TRY(launch_pdl(router_wgrad_kernel<Tin>, dim3(ceil_div(c->d, 256), c->E), dim3(256), 0, st,
+                     (const float *)a.d_logits, (const Tin *)a.x, c->T, c->d, c->E, d_w_router));
+  return launch_pdl(router_dgrad_kernel<Tin>, dim3(ceil_div(c->d, 256), std::min(c->T, 65535)),
+                    dim3(256), 0, st, (const float *)a.d_logits, (const Tin *)a.w_router, c->T,
+                    c->d, c->E, dx);
+}
+
 // ------------------------------------------------------------------ argument checks
 moe_status_t check_cfg(const moe_config_t *c) {
   if (!c) return MOE_ERR_INVALID_ARG;
@@ -652,6 +670,60 @@ moe_status_t moe_combine(const moe_config_t *cfg, const void *y_perm, const void
   MOE_REQUIRE(tok16(cfg, y_perm) && tok16(cfg, slot_pos) && tok16(cfg, topk_w) && tok16(cfg, y));
   MOE_REQUIRE(cfg->n_shared == 0 || tok16(cfg, y_shared));
   return combine_impl(cfg, y_perm, y_shared, slot_pos, topk_w, y, (cudaStream_t)stream, false);
+}
+
+moe_status_t moe_combine_backward(const moe_config_t *cfg, const float *dy, const void *y_perm,
+                                  const int32_t *slot_pos, const float *topk_w, void *dy_perm,
+                                  float *d_topk_w, void *stream) {
+  MOE_TRY(check_cfg(cfg));
+  MOE_REQUIRE(tok16(cfg, dy) && tok16(cfg, y_perm) && tok16(cfg, slot_pos) && tok16(cfg, topk_w) &&
+              tok16(cfg, dy_perm) && tok16(cfg, d_topk_w));
+  if (cfg->T == 0) return MOE_OK;
+  cudaStream_t st = (cudaStream_t)stream;
+  const dim3 grid(ceil_div(cfg->T, 8));
+  if (yperm_bf16(cfg))
+    return launch_pdl(combine_backward_kernel<__nv_bfloat16>, grid, dim3(256), 0, st, dy,
+                      (const __nv_bfloat16 *)y_perm, slot_pos, topk_w, (__nv_bfloat16 *)dy_perm,
+                      d_topk_w, cfg->T, cfg->top_k, cfg->d);
+  return launch_pdl(combine_backward_kernel<float>, grid, dim3(256), 0, st, dy,
+                    (const float *)y_perm, slot_pos, topk_w, (float *)dy_perm, d_topk_w, cfg->T,
+                    cfg->top_k, cfg->d);
+}
+
+moe_status_t moe_route_backward(const moe_config_t *cfg, const void *x, const moe_weights_t *w,
+                                const int32_t *topk_idx, const int32_t *expert_count,
+                                const float *d_topk_w, float d_loss, float *d_logits,
+                                float *d_w_router, float *dx, void *stream) {
+  MOE_TRY(check_cfg(cfg));
+  MOE_TRY(check_weights(cfg, w, true, false));
+  MOE_REQUIRE(std::isfinite(d_loss));
+  MOE_REQUIRE(tok16(cfg, x) && tok16(cfg, topk_idx) && aligned16(expert_count) &&
+              tok16(cfg, d_topk_w) && tok16(cfg, d_logits) && aligned16(d_w_router) &&
+              tok16(cfg, dx));
+  cudaStream_t st = (cudaStream_t)stream;
+  if (cfg->T == 0)
+    return cudaMemsetAsync(d_w_router, 0, (size_t)cfg->E * cfg->d * sizeof(float), st) == cudaSuccess
+               ? MOE_OK
+               : MOE_ERR_CUDA;
+  RouteBwdArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.x = x;
+  a.w_router = w->w_router;
+  a.off = w->logit_offset;
+  a.idx = topk_idx;
+  a.count = expert_count;
+  a.d_w = d_topk_w;
+  a.d_logits = d_logits;
+  a.T = cfg->T;
+  a.d = cfg->d;
+  a.E = cfg->E;
+  a.k = cfg->top_k;
+  a.sigmoid = cfg->score == MOE_SCORE_SIGMOID;
+  a.norm = cfg->norm_topk != 0;
+  a.alpha = cfg->aux_alpha;
+  a.dL = d_loss;
+  if (cfg->dtype == MOE_DTYPE_BF16) return route_backward_impl<__nv_bfloat16>(cfg, a, d_w_router, dx, st);
+  return route_backward_impl<float>(cfg, a, d_w_router, dx, st);
 }
 
 moe_status_t moe_aux_loss(const moe_config_t *cfg, const int32_t *expert_count,

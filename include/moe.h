@@ -153,6 +153,47 @@ moe_status_t moe_expert_forward(const moe_config_t *cfg, const void *x_perm,
 moe_status_t moe_combine(const moe_config_t *cfg, const void *y_perm, const void *y_shared,
                          const int32_t *slot_pos, const float *topk_w, void *y, void *stream);
 
+/* Backward pass, first steps. The pages train with this layer but do not write its backward
+ * out; it is the derivative of the forward, of J = sum(dy * y) + dL * loss, with no gradient
+ * through the selection (top-k, capacity drops, the loss's counts), none for the selection bias
+ * or the logit offsets, and each logit's fp32 rounding taken with derivative 1. The grouped
+ * expert GEMMs of the backward are not part of the library yet.
+ *
+ * Backward of moe_combine (Moonfrost expert card: a token's output sums its shared and top-k
+ * routed experts). For every kept pair (t, j), p = slot_pos[t, j] >= 0:
+ *   dy_perm[p]     = topk_w[t, j] * dy[t]
+ *   d_topk_w[t, j] = sum_c dy[t, c] * y_perm[p, c]      (0 for a dropped pair)
+ * dy: [T, d] fp32, the upstream gradient of y (the shared experts' upstream gradient is dy
+ * itself); y_perm, slot_pos, topk_w as the forward produced them; dy_perm: [offsets[E], d] in
+ * y_perm's dtype (bf16 for bf16 SwiGLU layers, else fp32), rows of dropped pairs do not exist;
+ * d_topk_w: [T, top_k] fp32. Sums over c in fp32, each reduced in a fixed order: bitwise
+ * reproducible. All buffers are the caller's device memory, 16-byte aligned (NULL only when
+ * T = 0). Asynchronous on `stream`; bad arguments return MOE_ERR_INVALID_ARG. */
+moe_status_t moe_combine_backward(const moe_config_t *cfg, const float *dy, const void *y_perm,
+                                  const int32_t *slot_pos, const float *topk_w, void *dy_perm,
+                                  float *d_topk_w, void *stream);
+
+/* Backward of moe_route and of the load-balancing loss (Quartz: architecture table, row
+ * "Router"; Sutra-1.3B, "48 + 1 experts" for sigmoid scores). Per token t, with the logits
+ * recomputed as l = x W_r^T + off in fp32 (not the forward's exact rounding: a difference of a
+ * few fp32 steps) and p = softmax(l) or sigmoid(l):
+ *   dp[e_j] gets d_topk_w[t, j], through w_j = p_j / (sum of the k selected p) when norm_topk
+ *   is set: dp[e_j] = (d_topk_w[t, j] - sum_i d_topk_w[t, i] w_i) / (that sum);
+ *   dq[e] = d_loss * aux_alpha * E * (expert_count[e] / (T top_k)) / T, the loss's term;
+ *   softmax: d_logits = p * (dp + dq - <dp + dq, p>);
+ *   sigmoid: d_logits = (dp + (dq - <dq, q>) / sum(p)) * p * (1 - p), q = p / sum(p).
+ * Then d_w_router = d_logits^T x ([E, d] fp32, the sum over t in token order) and
+ * dx = d_logits W_r ([T, d] fp32, the router's part of the input gradient, sum over e in order).
+ * x, w->w_router, w->logit_offset, topk_idx and expert_count (counts before capacity) as the
+ * forward took or returned them; d_topk_w from moe_combine_backward; d_logits: [T, E] fp32
+ * output. With T = 0 only d_w_router is written (zeros). All buffers are the caller's device
+ * memory, 16-byte aligned; d_loss must be finite. Asynchronous on `stream`; bad arguments return
+ * MOE_ERR_INVALID_ARG. */
+moe_status_t moe_route_backward(const moe_config_t *cfg, const void *x, const moe_weights_t *w,
+                                const int32_t *topk_idx, const int32_t *expert_count,
+                                const float *d_topk_w, float d_loss, float *d_logits,
+                                float *d_w_router, float *dx, void *stream);
+
 /* Load-balancing loss (Quartz: architecture table, row "Router", weight 0.01):
  *   loss = aux_alpha * E * sum_i (expert_count[i] / (T*top_k)) * (prob_sum[i] / T)
  * written to the device scalar `loss` (fp32); 0 when T = 0. */

@@ -1,7 +1,8 @@
 """Plain, slow CPU oracle of the backward pass of the fine-grained MoE FFN layer.
 
 TEST INFRASTRUCTURE, like ``moe_oracle``: imported only by the tests. It shares no code with the
-CUDA path, and no CUDA kernel computes this pass yet.
+CUDA path. CUDA kernels compute steps a and d-g below (the combine and the router); the expert
+steps b and c have none yet.
 
 The pages train whole models with this layer (research page, training setup: gradient
 accumulation and full gradient checkpointing), but none of them writes the backward out. Read
@@ -102,7 +103,8 @@ def layer_backward(cfg, inp: Dict[str, np.ndarray], dy: np.ndarray, dL: float = 
 
     Returns dx [T, d], d_w_router [E, d], the expert gradients under the weights' own names with
     a ``d_`` prefix (d_w_gate ... d_ws_down, or d_lr_V, d_lr_s, d_lr_U), and the intermediate
-    gradients d_logits [T, E] and d_w [T, k] (of the combine weights).
+    gradients d_logits [T, E], d_w [T, k] (of the combine weights), d_y_perm [N, d] (of the
+    grouped expert outputs) and dx_router [T, d] (the router's part of dx).
     """
     x = np.asarray(inp["x"], np.float64)
     T, d = x.shape
@@ -199,8 +201,10 @@ def layer_backward(cfg, inp: Dict[str, np.ndarray], dy: np.ndarray, dL: float = 
     # g. router
     Wr = np.asarray(inp["w_router"], np.float64)
     out["d_w_router"] = dlog.T @ x
-    dx += dlog @ Wr
+    out["dx_router"] = dlog @ Wr
+    dx += out["dx_router"]
     out["dx"] = dx
     out["d_logits"] = dlog
     out["d_w"] = dw
+    out["d_y_perm"] = dY
     return out

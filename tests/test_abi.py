@@ -137,6 +137,17 @@ def test_bad_pointers_and_workspace_are_rejected_on_the_host(lib):
     assert lib.moe_bias_update(P(cfg), None, 16, ctypes.c_float(0.1), None) == 1
     assert lib.moe_bias_update(P(cfg), 16, 20, ctypes.c_float(0.1), None) == 1
     assert lib.moe_bias_update(P(cfg), 16, 16, ctypes.c_float(float("nan")), None) == 1
+    # backward: misaligned or null buffers, non-finite loss gradient
+    assert lib.moe_combine_backward(P(cfg), 16, 16, 16, 16, 16, 8, None) == 1
+    assert lib.moe_combine_backward(P(cfg), None, 16, 16, 16, 16, 16, None) == 1
+    assert lib.moe_route_backward(P(cfg), 16, P(w), 16, 16, 16, ctypes.c_float(1.0), 16, 16,
+                                  24, None) == 1
+    assert lib.moe_route_backward(P(cfg), 16, P(w), 16, None, 16, ctypes.c_float(1.0), 16, 16,
+                                  16, None) == 1
+    assert lib.moe_route_backward(P(cfg), 16, P(w), 16, 16, 16, ctypes.c_float(float("inf")),
+                                  16, 16, 16, None) == 1
+    assert lib.moe_route_backward(P(cfg), 16, None, 16, 16, 16, ctypes.c_float(1.0), 16, 16, 16,
+                                  None) == 1
 
 
 def test_status_strings(lib):

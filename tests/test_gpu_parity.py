@@ -223,6 +223,62 @@ def test_near_ties_settled_exactly(name):
     assert (idx[:, 0] == 0).any() and (idx[:, 0] == 1).any()  # both orders occur
 
 
+# the backward of the combine and of the router, against the backward oracle: softmax and
+# sigmoid scores, norm_topk, capacity drops (heavy ones too), low-rank y_perm in fp32, fp32 layers
+BACKWARD = ["tiny_f32", "quartz_s", "capacity_s", "sigmoid_s", "lowrank_s", "norm_softmax",
+            "f32_sigmoid_cap", "heavy_drops"]
+
+
+@pytest.mark.parametrize("name", BACKWARD)
+def test_route_and_combine_backward(name):
+    from oracle import moe_backward as BW
+    c = SMALL[name] if name in SMALL else EDGE[name]
+    inp = make_inputs(c)
+    run = LayerOnGpu(c, inp)
+    o = run.steps()
+    T, d, k, E = run.cfg.T, run.cfg.d, run.cfg.top_k, run.cfg.E
+    dy = np.random.default_rng(11).standard_normal((T, d)).astype(np.float32)
+    dL = 1.7
+    ref = BW.layer_backward(c, inp, dy.astype(np.float64), dL)
+    dev = run.dev
+    dy_t = torch.as_tensor(dy).to(dev)
+    N = int(o["offsets"][-1])
+
+    # each step on the same inputs as the oracle's step: the combine on the forward's y_perm
+    # (whose error against the oracle is the forward's own), the router on the oracle's d_w
+    d_w_ref = torch.as_tensor(ref["d_w"].astype(np.float32)).to(dev)
+
+    def backward():
+        g = dict(dy_perm=torch.empty_like(o["y_perm"]),
+                 d_w=torch.empty((T, k), dtype=torch.float32, device=dev),
+                 d_logits=torch.empty((T, E), dtype=torch.float32, device=dev),
+                 d_w_router=torch.empty((E, d), dtype=torch.float32, device=dev),
+                 dx=torch.empty((T, d), dtype=torch.float32, device=dev))
+        B.moe_combine_backward(run.cfg, dy_t, o["y_perm"], o["slot_pos"], o["w"], g["dy_perm"],
+                               g["d_w"])
+        B.moe_route_backward(run.cfg, run.x, run.ws_struct, o["idx"], o["count"], d_w_ref, dL,
+                             g["d_logits"], g["d_w_router"], g["dx"])
+        torch.cuda.synchronize()
+        st, info = B.moe_get_device_error()
+        assert st == 0, (B.status_str(st), info)
+        return g
+
+    g = backward()
+    tol = tol_of(c)
+    ydt = "bf16" if g["dy_perm"].dtype == torch.bfloat16 else "f32"
+    assert rel_err_stored(np_(g["dy_perm"])[:N], ref["d_y_perm"], ydt) <= tol
+    assert rel_err(np_(g["d_w"]), ref["d_w"]) <= tol
+    assert rel_err(np_(g["d_logits"]), ref["d_logits"]) <= tol
+    assert rel_err(np_(g["d_w_router"]), ref["d_w_router"]) <= tol
+    assert rel_err(np_(g["dx"]), ref["dx_router"]) <= tol
+    # dropped pairs get a zero weight gradient; every sum has a fixed order
+    assert np.all(np_(g["d_w"])[np_(o["slot_pos"])[:T] < 0] == 0.0)
+    g2 = backward()
+    for key in g:
+        assert torch.equal(g[key][:N] if key == "dy_perm" else g[key],
+                           g2[key][:N] if key == "dy_perm" else g2[key]), key
+
+
 def test_bias_update_bitwise():
     """Loss-free balancing step on the routed counts of the sigmoid configuration, then the next
     routing call with the updated bias: the bias bit-exact against the oracle, the new routing
