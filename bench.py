@@ -399,6 +399,8 @@ def run_ours(args, rank, world, local_rank):
     d2h = y.numel() * y.element_size() + 4
 
     peaks, peak_src = load_peaks()
+    backward = backward_parts(c, cfg, layer, x, flush, stream, args.steps, peaks) \
+        if world == 1 else None
     table = roofline_table(c, n_kept, prof, args.steps, peaks, peak_src)
     dom = max(table, key=lambda n: table[n]["share"] or 0.0)
     dr = table[dom]
@@ -442,9 +444,85 @@ def run_ours(args, rank, world, local_rank):
         "gpu_launches": int(round(launches_per_step * args.steps)),
         "clocks": clk.summary(),
     }
+    if backward is not None:
+        result["backward_parts"] = backward
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(c, inp)
     return result
+
+
+def backward_parts(c, cfg, layer, x, flush, stream, K, peaks):
+    """The backward steps the library has so far (combine, router), each call timed alone with
+    CUDA events on the forward's resident outputs and a seeded upstream gradient, L2 flushed
+    between calls. Not part of the step above."""
+    import torch
+
+    from fine_grained_mixture_moe_b200 import binding as B
+    from fine_grained_mixture_moe_b200.layer import y_perm_dtype
+
+    dev = x.device
+    T, d, E, k = c.T, c.d, c.E, c.top_k
+    idx = torch.empty((T, k), dtype=torch.int32, device=dev)
+    wts = torch.empty((T, k), dtype=torch.float32, device=dev)
+    cnt = torch.empty(E, dtype=torch.int32, device=dev)
+    prob = torch.empty(E, dtype=torch.float32, device=dev)
+    offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
+    slot = torch.empty((T, k), dtype=torch.int32, device=dev)
+    src = torch.empty(T * k, dtype=torch.int32, device=dev)
+    xp = torch.empty((T * k, d), dtype=x.dtype, device=dev)
+    yp = torch.empty((T * k, d), dtype=y_perm_dtype(cfg), device=dev)
+    ysh = torch.empty((T, d), dtype=torch.float32, device=dev) if c.n_shared else None
+    B.moe_route(cfg, x, layer.wstruct, idx, wts, cnt, prob, layer.ws, layer.ws_bytes)
+    B.moe_permute(cfg, x, idx, offsets, slot, src, xp, layer.ws, layer.ws_bytes)
+    B.moe_expert_forward(cfg, xp, offsets, x, layer.wstruct, yp, ysh, layer.ws, layer.ws_bytes)
+    g = torch.Generator(device="cpu")
+    g.manual_seed(5)
+    dy = torch.randn((T, d), generator=g, dtype=torch.float32).to(dev)
+    dyp = torch.empty_like(yp)
+    d_w = torch.empty((T, k), dtype=torch.float32, device=dev)
+    d_logits = torch.empty((T, E), dtype=torch.float32, device=dev)
+    d_wr = torch.empty((E, d), dtype=torch.float32, device=dev)
+    dx = torch.empty((T, d), dtype=torch.float32, device=dev)
+    torch.cuda.synchronize()
+    N = int(offsets[-1])
+
+    def timed_call(fn):
+        for _ in range(3):
+            fn()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(K)]
+        torch.cuda.synchronize()
+        for i in range(K):
+            flush.fill_(i & 0xff)
+            ev[i][0].record(stream)
+            fn()
+            ev[i][1].record(stream)
+        torch.cuda.synchronize()
+        return statistics.fmean(a.elapsed_time(b) for a, b in ev) * 1e3
+
+    us_c = timed_call(lambda: B.moe_combine_backward(cfg, dy, yp, slot, wts, dyp, d_w))
+    us_r = timed_call(lambda: B.moe_route_backward(cfg, x, layer.wstruct, idx, cnt, d_w, 1.0,
+                                                   d_logits, d_wr, dx))
+    st, info = B.moe_get_device_error()
+    if st != 0:
+        raise RuntimeError(f"device error in the backward pass: {B.status_str(st)} info={info}")
+    by, bx = yp.element_size(), x.element_size()
+    # algorithmic bytes: every input read once, every output written once
+    bytes_c = T * d * 4 + 2 * N * d * by + T * k * 12
+    bytes_r = T * d * bx + E * d * bx + T * k * 8 + E * 4 + T * E * 4 + E * d * 4 + T * d * 4
+    flop_r = 6.0 * T * d * E  # logits again, then the two router products
+    hbm = peaks["hbm_gbs"]
+    fp32 = 148 * 128 * 2 * peaks.get("sm_max_mhz", 1965.0) * 1e6 / 1e12  # nominal, TFLOP/s
+    return {
+        "note": "each call timed alone (CUDA events, L2 flushed between calls); not in the step",
+        "combine_backward": {"avg_us": round(us_c, 2), "bound": "hbm", "bytes": bytes_c,
+                             "achieved_gbs": round(bytes_c / us_c / 1e3, 1),
+                             "frac": round(bytes_c / us_c / 1e3 / hbm, 4)},
+        "route_backward": {"avg_us": round(us_r, 2), "bound": "alu", "flop": flop_r,
+                           "achieved_tflops": round(flop_r / us_r / 1e6, 3),
+                           "frac": round(flop_r / us_r / 1e6 / fp32, 4), "bytes": bytes_r,
+                           "achieved_gbs": round(bytes_r / us_r / 1e3, 1)},
+    }
 
 
 def _threads():

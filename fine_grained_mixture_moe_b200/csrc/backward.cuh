@@ -13,7 +13,8 @@
 //   architecture table, row "Router": load-balancing weight 0.01), which for sigmoid scores
 //   enters through q = sigmoid / sum over all E;
 //   d_logits = p (dp + dq - <dp + dq, p>) (softmax) or dsigma sigma (1 - sigma) (sigmoid).
-// then d_w_router = d_logits^T x and dx = d_logits W_r, every sum in a fixed order.
+// then d_w_router = d_logits^T x and dx = d_logits W_r, every sum in a fixed order (the first
+// split over token ranges, the partial sums kept in dx until dx itself is written).
 #pragma once
 #include "common.cuh"
 
@@ -108,18 +109,29 @@ __global__ void __launch_bounds__(256) route_backward_kernel(RouteBwdArgs a) {
   const int E = a.E, d = a.d, k = a.k;
   float *pr = rb_smem + (size_t)warp * 2 * E, *dp = pr + E;
   const Tin *xr = (const Tin *)a.x + (size_t)t * d;
-  for (int e = 0; e < E; ++e) {
-    const Tin *we = (const Tin *)a.w_router + (size_t)e * d;
-    float s = 0.0f;
+  // logits, 8 experts per pass: each x vector feeds 8 independent chains
+  for (int e0 = 0; e0 < E; e0 += 8) {
+    float acc[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
     for (int c = 4 * lane; c < d; c += 128) {
-      const float4 u = Bw4<Tin>::ld(xr + c), v = Bw4<Tin>::ld(we + c);
-      s = fmaf(u.x, v.x, s);
-      s = fmaf(u.y, v.y, s);
-      s = fmaf(u.z, v.z, s);
-      s = fmaf(u.w, v.w, s);
+      const float4 u = Bw4<Tin>::ld(xr + c);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        if (e0 + i >= E) break;
+        const float4 v = Bw4<Tin>::ld((const Tin *)a.w_router + (size_t)(e0 + i) * d + c);
+        acc[i] = fmaf(u.x, v.x, acc[i]);
+        acc[i] = fmaf(u.y, v.y, acc[i]);
+        acc[i] = fmaf(u.z, v.z, acc[i]);
+        acc[i] = fmaf(u.w, v.w, acc[i]);
+      }
     }
-    s = warp_sum_f(s);
-    if (lane == 0) pr[e] = a.off ? s + a.off[e] : s;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      if (e0 + i >= E) break;
+      const float s = warp_sum_f(acc[i]);
+      if (lane == 0) pr[e0 + i] = a.off ? s + a.off[e0 + i] : s;
+    }
   }
   __syncwarp();
   float m = -INFINITY, ssum = 0.0f;
@@ -176,33 +188,67 @@ template <> __device__ __forceinline__ float bw_elem<__nv_bfloat16>(const __nv_b
   return __bfloat162float(p[i]);
 }
 
-// d_w_router[e, c] = sum over t (in order) of d_logits[t, e] x[t, c]; block (column tile, e).
+// d_w_router = d_logits^T x, split over the tokens: block (256 columns, 8 experts, split s)
+// sums tokens [s T / S, (s + 1) T / S) in order into part[s][e][c]; router_wgrad_sum adds the S
+// partial sums in split order (S = 1 writes the result directly).
 template <typename Tin>
 __global__ void __launch_bounds__(256) router_wgrad_kernel(const float *__restrict__ dl,
                                                            const Tin *__restrict__ x, int T, int d,
-                                                           int E, float *__restrict__ dwr) {
+                                                           int E, int S, float *__restrict__ part) {
   griddep_wait();
   griddep_launch();
-  const int e = blockIdx.y, c = blockIdx.x * 256 + threadIdx.x;
+  const int c = blockIdx.x * 256 + threadIdx.x, e0 = blockIdx.y * 8, s = blockIdx.z;
   if (c >= d) return;
-  float acc = 0.0f;
-  for (int t = 0; t < T; ++t) acc = fmaf(dl[(size_t)t * E + e], bw_elem(x, (size_t)t * d + c), acc);
-  dwr[(size_t)e * d + c] = acc;
+  const int t0 = (int)((long long)T * s / S), t1 = (int)((long long)T * (s + 1) / S);
+  float acc[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
+  for (int t = t0; t < t1; ++t) {
+    const float xv = bw_elem(x, (size_t)t * d + c);
+    const float *g = dl + (size_t)t * E + e0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      if (e0 + i < E) acc[i] = fmaf(g[i], xv, acc[i]);
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+    if (e0 + i < E) part[((size_t)s * E + e0 + i) * d + c] = acc[i];
 }
 
-// dx[t, c] = sum over e (in order) of d_logits[t, e] W_r[e, c]; blocks stride over the tokens.
+__global__ void __launch_bounds__(256) router_wgrad_sum_kernel(const float *__restrict__ part,
+                                                               int S, int E, int d,
+                                                               float *__restrict__ dwr) {
+  griddep_wait();
+  griddep_launch();
+  const size_t i = (size_t)blockIdx.x * 256 + threadIdx.x, n = (size_t)E * d;
+  if (i >= n) return;
+  float acc = part[i];
+  for (int s = 1; s < S; ++s) acc += part[(size_t)s * n + i];
+  dwr[i] = acc;
+}
+
+// dx[t, c..c+3] = sum over e (in order) of d_logits[t, e] W_r[e, c..c+3]; blocks stride over the
+// tokens.
 template <typename Tin>
 __global__ void __launch_bounds__(256) router_dgrad_kernel(const float *__restrict__ dl,
                                                            const Tin *__restrict__ wr, int T, int d,
                                                            int E, float *__restrict__ dx) {
   griddep_wait();
   griddep_launch();
-  const int c = blockIdx.x * 256 + threadIdx.x;
+  const int c = 4 * (blockIdx.x * 256 + threadIdx.x);
   if (c >= d) return;
   for (int t = blockIdx.y; t < T; t += gridDim.y) {
-    float acc = 0.0f;
-    for (int e = 0; e < E; ++e) acc = fmaf(dl[(size_t)t * E + e], bw_elem(wr, (size_t)e * d + c), acc);
-    dx[(size_t)t * d + c] = acc;
+    float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+    const float *g = dl + (size_t)t * E;
+    for (int e = 0; e < E; ++e) {
+      const float ge = g[e];
+      const float4 v = Bw4<Tin>::ld(wr + (size_t)e * d + c);
+      acc.x = fmaf(ge, v.x, acc.x);
+      acc.y = fmaf(ge, v.y, acc.y);
+      acc.z = fmaf(ge, v.z, acc.z);
+      acc.w = fmaf(ge, v.w, acc.w);
+    }
+    *(float4 *)(dx + (size_t)t * d + c) = acc;
   }
 }
 

@@ -570,9 +570,17 @@ moe_status_t route_backward_impl(const moe_config_t *c, const RouteBwdArgs &a, f
                            (int)smem) != cudaSuccess)
     return MOE_ERR_CUDA;
   MOE_TRY(launch_pdl(route_backward_kernel<Tin>, dim3(ceil_div(c->T, 8)), dim3(256), smem, st, a));
-  MOE_TRY(launch_pdl(router_wgrad_kernel<Tin>, dim3(ceil_div(c->d, 256), c->E), dim3(256), 0, st,
-                     (const float *)a.d_logits, (const Tin *)a.x, c->T, c->d, c->E, d_w_router));
-  return launch_pdl(router_dgrad_kernel<Tin>, dim3(ceil_div(c->d, 256), std::min(c->T, 65535)),
+  // d_w_router over S token ranges; their partial sums [S, E, d] live in dx (T x d floats,
+  // S E <= T) until the last kernel writes dx
+  const int S = std::max(1, std::min(32, c->T / c->E));
+  float *part = S > 1 ? dx : d_w_router;
+  MOE_TRY(launch_pdl(router_wgrad_kernel<Tin>, dim3(ceil_div(c->d, 256), ceil_div(c->E, 8), S),
+                     dim3(256), 0, st, (const float *)a.d_logits, (const Tin *)a.x, c->T, c->d,
+                     c->E, S, part));
+  if (S > 1)
+    MOE_TRY(launch_pdl(router_wgrad_sum_kernel, dim3(ceil_div((long long)c->E * c->d, 256)),
+                       dim3(256), 0, st, (const float *)part, S, c->E, c->d, d_w_router));
+  return launch_pdl(router_dgrad_kernel<Tin>, dim3(ceil_div(c->d, 1024), std::min(c->T, 65535)),
                     dim3(256), 0, st, (const float *)a.d_logits, (const Tin *)a.w_router, c->T,
                     c->d, c->E, dx);
 }

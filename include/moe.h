@@ -186,7 +186,8 @@ moe_status_t moe_combine_backward(const moe_config_t *cfg, const float *dy, cons
  * dx = d_logits W_r ([T, d] fp32, the router's part of the input gradient, sum over e in order).
  * x, w->w_router, w->logit_offset, topk_idx and expert_count (counts before capacity) as the
  * forward took or returned them; d_topk_w from moe_combine_backward; d_logits: [T, E] fp32
- * output. With T = 0 only d_w_router is written (zeros). All buffers are the caller's device
+ * output; dx also holds the weight gradient's partial sums (over token ranges) until the call
+ * writes it. With T = 0 only d_w_router is written (zeros). All buffers are the caller's device
  * memory, 16-byte aligned; d_loss must be finite. Asynchronous on `stream`; bad arguments return
  * MOE_ERR_INVALID_ARG. */
 moe_status_t moe_route_backward(const moe_config_t *cfg, const void *x, const moe_weights_t *w,
