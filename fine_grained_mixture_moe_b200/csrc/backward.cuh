@@ -109,29 +109,19 @@ __global__ void __launch_bounds__(256) route_backward_kernel(RouteBwdArgs a) {
   const int E = a.E, d = a.d, k = a.k;
   float *pr = rb_smem + (size_t)warp * 2 * E, *dp = pr + E;
   const Tin *xr = (const Tin *)a.x + (size_t)t * d;
-  // logits, 8 experts per pass: each x vector feeds 8 independent chains
-  for (int e0 = 0; e0 < E; e0 += 8) {
-    float acc[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
+  // logits, one expert per pass (on the Quartz shape 49 us, against 86 us with 8 chains per pass)
+  for (int e = 0; e < E; ++e) {
+    const Tin *we = (const Tin *)a.w_router + (size_t)e * d;
+    float s = 0.0f;
     for (int c = 4 * lane; c < d; c += 128) {
-      const float4 u = Bw4<Tin>::ld(xr + c);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        if (e0 + i >= E) break;
-        const float4 v = Bw4<Tin>::ld((const Tin *)a.w_router + (size_t)(e0 + i) * d + c);
-        acc[i] = fmaf(u.x, v.x, acc[i]);
-        acc[i] = fmaf(u.y, v.y, acc[i]);
-        acc[i] = fmaf(u.z, v.z, acc[i]);
-        acc[i] = fmaf(u.w, v.w, acc[i]);
-      }
+      const float4 u = Bw4<Tin>::ld(xr + c), v = Bw4<Tin>::ld(we + c);
+      s = fmaf(u.x, v.x, s);
+      s = fmaf(u.y, v.y, s);
+      s = fmaf(u.z, v.z, s);
+      s = fmaf(u.w, v.w, s);
     }
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      if (e0 + i >= E) break;
-      const float s = warp_sum_f(acc[i]);
-      if (lane == 0) pr[e0 + i] = a.off ? s + a.off[e0 + i] : s;
-    }
+    s = warp_sum_f(s);
+    if (lane == 0) pr[e] = a.off ? s + a.off[e] : s;
   }
   __syncwarp();
   float m = -INFINITY, ssum = 0.0f;
