@@ -53,3 +53,15 @@ def loss_config(cfg, world: int):
     ctypes.memmove(ctypes.addressof(g), ctypes.addressof(cfg), ctypes.sizeof(cfg))
     g.T = cfg.T * world
     return g
+
+
+def replica_loss_grad(d_loss: float, world: int) -> float:
+    """The d_loss to hand moe_route_backward on a replica whose loss is the global one.
+
+    The call forms the loss term dq_e = d_loss alpha E count_e / (T k T) with its own T =
+    T_local. The global loss has T_global = T_local * world in both places, so a replica passes
+    the all-reduced counts and d_loss / world^2; the ranks then sum d_w_router (and the expert
+    weight gradients) as usual for data parallelism.
+    """
+    return d_loss / float(world * world)
+

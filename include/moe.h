@@ -187,9 +187,11 @@ moe_status_t moe_combine_backward(const moe_config_t *cfg, const float *dy, cons
  * x, w->w_router, w->logit_offset, topk_idx and expert_count (counts before capacity) as the
  * forward took or returned them; d_topk_w from moe_combine_backward; d_logits: [T, E] fp32
  * output; dx also holds the weight gradient's partial sums (over token ranges) until the call
- * writes it. With T = 0 only d_w_router is written (zeros). All buffers are the caller's device
- * memory, 16-byte aligned; d_loss must be finite. Asynchronous on `stream`; bad arguments return
- * MOE_ERR_INVALID_ARG. */
+ * writes it. Data-parallel replicas whose loss is formed from the statistics summed over the
+ * ranks (T_global = world * T tokens) pass the summed counts and d_loss * (T / T_global)^2, then
+ * sum d_w_router over the ranks. With T = 0 only d_w_router is written (zeros). All buffers
+ * are the caller's device memory, 16-byte aligned; d_loss must be finite. Asynchronous on
+ * `stream`; bad arguments return MOE_ERR_INVALID_ARG. */
 moe_status_t moe_route_backward(const moe_config_t *cfg, const void *x, const moe_weights_t *w,
                                 const int32_t *topk_idx, const int32_t *expert_count,
                                 const float *d_topk_w, float d_loss, float *d_logits,

@@ -98,8 +98,13 @@ def lowrank_backward(X, V, s, U, dY) -> Dict[str, np.ndarray]:
     return dict(dX=dz @ V, dV=dz.T @ X, ds=(dzs * z).sum(axis=0), dU=dY.T @ zs)
 
 
-def layer_backward(cfg, inp: Dict[str, np.ndarray], dy: np.ndarray, dL: float = 1.0) -> Dict:
+def layer_backward(cfg, inp: Dict[str, np.ndarray], dy: np.ndarray, dL: float = 1.0,
+                   loss_count=None, loss_T=None) -> Dict:
     """Gradients of ``J = sum(dy * y) + dL * L`` for the layer of ``moe_oracle.layer_forward``.
+
+    ``loss_count`` [E] and ``loss_T`` are the statistics L is formed from when they are not this
+    call's own: data-parallel replicas form it from the counts summed over the ranks and the
+    global token count (module doc, step e). By default they are this call's counts and T.
 
     Returns dx [T, d], d_w_router [E, d], the expert gradients under the weights' own names with
     a ``d_`` prefix (d_w_gate ... d_ws_down, or d_lr_V, d_lr_s, d_lr_U), and the intermediate
@@ -186,8 +191,10 @@ def layer_backward(cfg, inp: Dict[str, np.ndarray], dy: np.ndarray, dL: float = 
                 dp[t, idx[t, j]] += dw[t, j]
 
     # e, f. load-balancing loss and the scores -> logits
-    f = np.asarray(r["count"], np.float64) / (T * k) if T else np.zeros(E)
-    dq = np.broadcast_to(dL * cfg.aux_alpha * E * f / T, (T, E)) if T else np.zeros((T, E))
+    cnt_L = np.asarray(r["count"] if loss_count is None else loss_count, np.float64)
+    T_L = T if loss_T is None else int(loss_T)
+    f = cnt_L / (T_L * k) if T_L else np.zeros(E)
+    dq = np.broadcast_to(dL * cfg.aux_alpha * E * f / T_L, (T, E)) if T_L else np.zeros((T, E))
     if cfg.score == "softmax":
         dp_all = dp + dq
         dlog = p * (dp_all - (dp_all * p).sum(axis=1, keepdims=True))

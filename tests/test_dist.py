@@ -60,6 +60,51 @@ def _rank_main(rank: int, port: int, force_int64: bool):
         dist.destroy_process_group()
 
 
+def _rank_backward(rank: int, port: int):
+    """Replica backward of the router: global counts, d_loss scaled for the call's own T, then a
+    sum of d_w_router over the ranks, against the single-process backward on the whole batch."""
+    from oracle import moe_backward as BW
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=WORLD,
+                            timeout=__import__("datetime").timedelta(seconds=60))
+    try:
+        c = CFG
+        inp = make_inputs(c)
+        Tl = c.T // WORLD
+        dy = np.random.default_rng(4).standard_normal((c.T, c.d))
+        dL = 1.3
+        full = BW.layer_backward(c, inp, dy, dL)
+        mine = dict(inp, x=inp["x"][rank * Tl:(rank + 1) * Tl])
+        cl = c.with_(T=Tl)
+        r = oracle.route(mine["x"], inp["w_router"], inp.get("logit_offset"),
+                         inp.get("select_bias"), c.score, c.top_k, c.norm_topk)
+        cnt = torch.as_tensor(np.asarray(r["count"], np.int32))
+        prob = torch.as_tensor(np.asarray(r["prob_sum"], np.float32))
+        gcnt, _ = D.allreduce_route_stats(cnt, prob, c.T * c.top_k)
+        dys = dy[rank * Tl:(rank + 1) * Tl]
+        # the form the device call computes: its own T, the global counts, d_loss scaled
+        g = BW.layer_backward(cl, mine, dys, D.replica_loss_grad(dL, WORLD),
+                              loss_count=gcnt.numpy())
+        # the same term written with the global T
+        g2 = BW.layer_backward(cl, mine, dys, dL, loss_count=gcnt.numpy(), loss_T=c.T)
+        np.testing.assert_allclose(g["d_logits"], g2["d_logits"], rtol=1e-12, atol=1e-15)
+        dwr = torch.as_tensor(g["d_w_router"])
+        dist.all_reduce(dwr)
+        np.testing.assert_allclose(dwr.numpy(), full["d_w_router"], rtol=1e-10, atol=1e-12)
+        np.testing.assert_allclose(g["dx_router"], full["dx_router"][rank * Tl:(rank + 1) * Tl],
+                                   rtol=1e-10, atol=1e-12)
+        # the replica's own statistics give a different gradient: the exchange is needed
+        own = BW.layer_backward(cl, mine, dys, dL)
+        assert np.abs(own["d_logits"] - g["d_logits"]).max() > 1e-9
+    finally:
+        dist.destroy_process_group()
+
+
+def test_replicas_reproduce_global_router_gradient():
+    mp.spawn(_rank_backward, args=(_free_port(),), nprocs=WORLD, join=True)
+
+
 @pytest.mark.parametrize("force_int64", [False, True])
 def test_replicas_reproduce_global_loss(force_int64):
     mp.spawn(_rank_main, args=(_free_port(), force_int64), nprocs=WORLD, join=True)
