@@ -224,9 +224,10 @@ def test_near_ties_settled_exactly(name):
 
 
 # the backward of the combine and of the router, against the backward oracle: softmax and
-# sigmoid scores, norm_topk, capacity drops (heavy ones too), low-rank y_perm in fp32, fp32 layers
+# sigmoid scores, norm_topk, capacity drops (heavy ones too), low-rank y_perm in fp32, fp32 layers;
+# T < 2E (one token range in the router's weight gradient: T1, k8_E97) and a single expert
 BACKWARD = ["tiny_f32", "quartz_s", "capacity_s", "sigmoid_s", "lowrank_s", "norm_softmax",
-            "f32_sigmoid_cap", "heavy_drops"]
+            "f32_sigmoid_cap", "heavy_drops", "T1", "k8_E97", "E1k1"]
 
 
 @pytest.mark.parametrize("name", BACKWARD)
