@@ -20,6 +20,9 @@
 
 namespace moe {
 
+// detail code (g_err_info) of a selected expert index outside [0, E) in the backward's input
+constexpr long long INFO_BAD_EXPERT_INDEX = 3;
+
 // four consecutive elements of a row, as fp32
 template <typename Ty> struct Bw4;
 template <> struct Bw4<float> {
@@ -142,7 +145,11 @@ __global__ void __launch_bounds__(256) route_backward_kernel(RouteBwdArgs a) {
   if (lane == 0) {  // the combine weights' gradient onto the selected probabilities
     const int *ir = a.idx + (size_t)t * k;
     const float *gw = a.d_w + (size_t)t * k;
-    if (a.norm) {
+    bool ok = true;
+    for (int j = 0; j < k; ++j) ok = ok && ir[j] >= 0 && ir[j] < E;
+    if (!ok) {
+      set_device_error(MOE_ERR_DEVICE_CHECK, INFO_BAD_EXPERT_INDEX);
+    } else if (a.norm) {
       float S = 0.0f;
       for (int j = 0; j < k; ++j) S += pr[ir[j]];
       float inner = 0.0f;
