@@ -247,7 +247,15 @@ moe_status_t moe_route_noalloc(const moe_config_t *cfg, const void *x, const moe
 const char *moe_status_str(moe_status_t s);
 
 /* Synchronises `stream`, then returns and clears the device error word of the current device
- * (MOE_OK if no device-side fault was recorded). *info (may be NULL) receives a detail code. */
+ * (MOE_OK if no device-side fault was recorded). *info (may be NULL) receives a detail code:
+ *   MOE_ERR_DEVICE_CHECK: 1 a sigmoid key that could not be resolved exactly; 2 an exact-sum
+ *     expansion that ran out of terms; 3 a selected expert index outside [0, E) given to
+ *     moe_route_backward; 100 + j an expert index outside [0, E) in slot j of moe_permute's
+ *     topk_idx.
+ *   MOE_ERR_TIMEOUT: the bounded wait that ran out: 10 operands (MMA waiting for TMA), 11 a
+ *     free stage (TMA waiting for the MMA), 12 a full accumulator, 13 a free accumulator, 14 the
+ *     drain of copies still in flight, 15 the router's token rows, 16 the scatter's token rows,
+ *     20 the timeout probe. */
 moe_status_t moe_get_device_error(void *stream, int64_t *info);
 
 /* Test and measurement controls (synchronous, current device):
