@@ -1,4 +1,5 @@
-"""B200-native forward pass of a DeepSeek-style fine-grained mixture-of-experts FFN layer.
+"""B200-native forward pass of a DeepSeek-style fine-grained mixture-of-experts FFN layer, and
+the first steps of its backward pass (the combine and the router).
 
 The compute path is the sm_100a CUDA library ``lib/libmoe.so`` behind the C ABI in
 ``include/moe.h``; :mod:`.binding` marshals arguments to it and :class:`MoELayer` holds device
@@ -7,7 +8,8 @@ the built library every call raises.
 """
 from .binding import (DEBUG_FORCE_EXACT, DEBUG_PROFILE, DEBUG_WAIT_LIMIT_NS, EXPORTED,  # noqa: F401
                       MoEConfig, MoEError, MoEWeights, load, make_config, make_weights,
-                      moe_aux_loss, moe_bias_update, moe_capacity, moe_combine, moe_debug_set,
+                      moe_aux_loss, moe_bias_update, moe_capacity, moe_combine,
+                      moe_combine_backward, moe_debug_set, moe_route_backward,
                       moe_debug_wait_timeout_probe, moe_expert_forward, moe_get_device_error,
                       moe_layer_forward, moe_permute, moe_profile_read, moe_route,
                       moe_route_noalloc, moe_workspace_size, status_str)
