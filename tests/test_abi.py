@@ -148,6 +148,14 @@ def test_bad_pointers_and_workspace_are_rejected_on_the_host(lib):
                                   16, 16, 16, None) == 1
     assert lib.moe_route_backward(P(cfg), 16, None, 16, 16, 16, ctypes.c_float(1.0), 16, 16, 16,
                                   None) == 1
+    assert lib.moe_route_backward(None, 16, P(w), 16, 16, 16, ctypes.c_float(1.0), 16, 16, 16,
+                                  None) == 1
+    assert lib.moe_combine_backward(None, 16, 16, 16, 16, 16, 16, None) == 1
+    # an unsupported shape is refused before any argument is touched
+    bad = B.make_config(T=16, d=100, E=8, top_k=2, ffn=64)
+    assert lib.moe_combine_backward(P(bad), 16, 16, 16, 16, 16, 16, None) == 2
+    assert lib.moe_route_backward(P(bad), 16, P(w), 16, 16, 16, ctypes.c_float(1.0), 16, 16,
+                                  16, None) == 2
 
 
 def test_status_strings(lib):
