@@ -905,28 +905,67 @@ extern "C" moe_status_t moe_debug_wait_timeout_probe(void *stream) {
 
 // ================================================================== moe_route_noalloc
 // The router's scratch (the per-CTA partial statistics) placed in a fixed array of the library's
-// own device memory instead of a caller workspace. Host code must not use the array's name as a device pointer: it is a host
-// stand-in for the symbol, so its device address is looked up once per device below.
+// own device memory instead of a caller workspace. Host code must not use the array's name as a
+// device pointer: it is a host stand-in for the symbol, so its device address is looked up per
+// device (and per context of that device) below.
 namespace {
 
 static __device__ __align__(256) unsigned char g_route_scratch[MOE_ROUTE_NOALLOC_SCRATCH_BYTES];
 
-void *g_route_scratch_dev[64];
+// Per device: the array's address and the id of the context it was looked up in. A context
+// made anew on the device (after cudaDeviceReset, for example) may load the module at another
+// address, so the address is looked up again whenever the current context's id differs.
+struct ScratchAddr {
+  void *ptr = nullptr;
+  unsigned long long ctx_id = 0;
+};
+ScratchAddr g_route_scratch_dev[64];
 std::mutex g_route_scratch_mu;
 
-// Device address of g_route_scratch on the current device (looked up on the first call there).
+// Unique id of the calling thread's current context (driver entry points, looked up once).
+moe_status_t current_context_id(unsigned long long *id) {
+  using GetCurrent = CUresult (*)(CUcontext *);
+  using GetId = CUresult (*)(CUcontext, unsigned long long *);
+  static GetCurrent get_current = nullptr;
+  static GetId get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    cudaDriverEntryPointQueryResult q;
+    void *f = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = (GetCurrent)f;
+    f = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = (GetId)f;
+  });
+  if (!get_current || !get_id) return MOE_ERR_CUDA;
+  CUcontext ctx = nullptr;
+  if (get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return MOE_ERR_CUDA;
+  return get_id(ctx, id) == CUDA_SUCCESS ? MOE_OK : MOE_ERR_CUDA;
+}
+
+// Device address of g_route_scratch on the current device, looked up (with that device current)
+// on the first call there and again when the device's context has been made anew.
 moe_status_t route_scratch_address(void **out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
   if (dev < 0 || dev >= 64) return MOE_ERR_UNSUPPORTED;
   std::lock_guard<std::mutex> lk(g_route_scratch_mu);
-  if (g_route_scratch_dev[dev] == nullptr) {
+  ScratchAddr &a = g_route_scratch_dev[dev];
+  unsigned long long ctx_id = 0;
+  const bool have_id = current_context_id(&ctx_id) == MOE_OK;  // false: no context yet
+  if (a.ptr == nullptr || !have_id || a.ctx_id != ctx_id) {
     void *p = nullptr;
+    // initialises the device's primary context when none is current on this thread
     const cudaError_t e = cudaGetSymbolAddress(&p, g_route_scratch);
     if (e != cudaSuccess || p == nullptr) return MOE_ERR_CUDA;
-    g_route_scratch_dev[dev] = p;
+    if (!have_id) MOE_TRY(current_context_id(&ctx_id));
+    a.ptr = p;
+    a.ctx_id = ctx_id;
   }
-  *out = g_route_scratch_dev[dev];
+  *out = a.ptr;
   return MOE_OK;
 }
 

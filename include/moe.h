@@ -125,7 +125,10 @@ moe_status_t moe_permute(const moe_config_t *cfg, const void *x, const int32_t *
                          int32_t *offsets, int32_t *slot_pos, int32_t *src_token,
                          void *x_perm, void *ws, size_t ws_bytes, void *stream);
 
-/* Grouped expert GEMMs on the grouped rows, and the shared experts on all tokens.
+/* Grouped expert GEMMs on the grouped rows, and the shared experts on all tokens
+ * (quartz-micro-preview-base card, "Architecture": routed SwiGLU experts of FFN width 640 and 2
+ * shared experts that every token passes through; Moonfrost expert card: the experts held as
+ * stacked (E, hidden, ffn) tensors; dormouse, "TSCT low-rank experts": experts U*diag(s)*V^T).
  *   SwiGLU expert e on row r (offsets[e] <= r < offsets[e+1]):
  *     y_perm[r] = W_down[e] (silu(W_gate[e] x_perm[r]) * (W_up[e] x_perm[r]))
  *   low-rank expert: y_perm[r] = U[e] (s[e] * (V[e] x_perm[r]))
@@ -145,7 +148,9 @@ moe_status_t moe_expert_forward(const moe_config_t *cfg, const void *x_perm,
                                 const moe_weights_t *w, void *y_perm, void *y_shared,
                                 void *ws, size_t ws_bytes, void *stream);
 
-/* Weighted un-permute: y[t] = y_shared[t] + sum_j [slot_pos[t,j] >= 0] topk_w[t,j] *
+/* Weighted un-permute (Moonfrost expert card: a token's output is the shared expert plus its
+ * top-k routed experts; Quartz architecture table: the 2 shared experts are always active):
+ * y[t] = y_shared[t] + sum_j [slot_pos[t,j] >= 0] topk_w[t,j] *
  * y_perm[slot_pos[t,j]], summed in fp32 in slot order. y_perm as moe_expert_forward writes it
  * (bf16 for bf16 SwiGLU layers, else fp32); y_shared and y are fp32 [.., d]: a bf16 rounding of
  * y itself would cost up to 2^-8 * max|y| / rms(y), the whole 2e-2 error budget of the layer.
@@ -216,7 +221,10 @@ moe_status_t moe_aux_loss(const moe_config_t *cfg, const int32_t *expert_count,
 moe_status_t moe_bias_update(const moe_config_t *cfg, const int32_t *expert_count,
                              float *select_bias, float u, void *stream);
 
-/* The whole layer: route -> permute -> experts -> combine -> loss, no host synchronisation.
+/* The whole layer: route -> permute -> experts -> combine -> loss, no host synchronisation
+ * (the layer of the Quartz architecture table: router, 24 routed experts top-6, 2 shared experts,
+ * load-balancing loss 0.01; the Moonfrost expert card's stacked experts under a capacity, whose
+ * per-expert host loop this call replaces: no count returns to the host).
  *   y [T, d] fp32; aux_loss: device fp32 scalar (may be NULL); expert_count: optional [E]
  *   int32 output of the router's per-expert selection counts (may be NULL). */
 moe_status_t moe_layer_forward(const moe_config_t *cfg, const void *x, const moe_weights_t *w,
@@ -235,7 +243,10 @@ moe_status_t moe_layer_forward(const moe_config_t *cfg, const void *x, const moe
  *   - Limit: the scratch needed is about 8*E*ceil(T/16) bytes; configurations that need
  *     more than MOE_ROUTE_NOALLOC_SCRATCH_BYTES return MOE_ERR_WORKSPACE with nothing enqueued.
  *   - Set-up: the first call on each device looks up the array's device address (with that
- *     device current); make that first call before any stream capture begins.
+ *     device current); make that first call before any stream capture begins. The address is
+ *     kept per device together with the id of the context it belongs to: if the device's
+ *     context is made anew (cudaDeviceReset, or another library that resets the device), the
+ *     next call looks it up again, and that call too must come before any stream capture.
  *   - Sharing: every call on a device uses the same array. Calls whose work overlaps on the GPU
  *     (other streams, other host threads) race on it and must be serialised by the caller. */
 #define MOE_ROUTE_NOALLOC_SCRATCH_BYTES (4u << 20)

@@ -158,6 +158,18 @@ def test_bad_pointers_and_workspace_are_rejected_on_the_host(lib):
                                   16, None) == 2
 
 
+def test_noalloc_route_refuses_one_token_past_its_scratch(lib):
+    """moe_route_noalloc keeps its scratch (two tables of E * ceil(T/16) int32 / fp32 partials,
+    each rounded up to 256 bytes) in a fixed 4 MiB array. With E = 1,024, T = 8,192 fills it
+    exactly (the GPU test runs that case); T = 8,193 needs 513 rows per table and must be
+    refused on the host with MOE_ERR_WORKSPACE before any device work, whatever the pointers."""
+    cfg = B.make_config(T=8193, d=1024, E=1024, top_k=2, rank=64, expert="lowrank")
+    w = B.MoEWeights()
+    w.w_router = 256
+    P = ctypes.byref
+    assert lib.moe_route_noalloc(P(cfg), 256, P(w), 256, 256, 256, 256, None) == 3
+
+
 def test_status_strings(lib):
     for s in range(7):
         assert B.status_str(s).startswith(B.STATUS_NAMES[s])

@@ -14,19 +14,26 @@ def _bench():
     return mod
 
 
-def _copy_tree(tmp_path):
+def _copy_tree(tmp_path, b):
+    """The kernel sources in a scratch tree, with a traffic file written for them (the committed
+    figures belong to the capture's sources, which later edits may have left behind)."""
     root = tmp_path / "repo"
     shutil.copytree(os.path.join(ROOT, "fine_grained_mixture_moe_b200", "csrc"),
                     root / "fine_grained_mixture_moe_b200" / "csrc")
-    shutil.copytree(os.path.join(ROOT, "profiles"), root / "profiles")
+    (root / "profiles").mkdir()
+    b.ROOT = str(root)
+    with open(root / "profiles" / "traffic_quartz.txt", "w") as fh:
+        fh.write("# test figures\n")
+        fh.write(f"sources_sha256 {b.kernel_sources_sha256()}\n")
+        fh.write("gemm_gateup 148840960\n")
     return root
 
 
 def test_traffic_follows_the_forward_sources(tmp_path):
     b = _bench()
-    b.ROOT = str(_copy_tree(tmp_path))
+    _copy_tree(tmp_path, b)
     got = b.captured_traffic("quartz", "gemm_gateup")
-    assert isinstance(got, int) and got > 0
+    assert got == 148840960
     assert b.captured_traffic("quartz", "no_such_kernel") is None
     assert b.captured_traffic("no_such_workload", "gemm_gateup") is None
     csrc = os.path.join(b.ROOT, "fine_grained_mixture_moe_b200", "csrc")

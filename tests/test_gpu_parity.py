@@ -34,6 +34,9 @@ SMALL = {
     "capacity_s": get_config("capacity", T=1037),
     "sigmoid_s": get_config("sigmoid", T=611),
     "lowrank_s": get_config("lowrank", T=1500, E=256),
+    # the full 1,024 experts with Zipf offsets: a 1,025-group tile list (the pair kernel's
+    # smaller operand ring), hundreds of empty experts and one large group
+    "lowrank_E1024": get_config("lowrank", T=3000),
 }
 
 EDGE = {
@@ -392,34 +395,49 @@ def test_bounded_wait_times_out_cleanly():
 # ------------------------------------------------------------------ full-size configurations
 @pytest.mark.parametrize("name", sorted(CONFIGS))
 def test_full_size(name):
-    """Every token's routing and permutation bit-exact; y on sampled tokens vs the per-token
-    definition; the loss. Launch configuration as the benchmark runs it (moe_layer_forward)."""
+    """Every token of the full-size configuration against the oracle, element by element, in
+    the launch configuration the benchmark times (moe_layer_forward, whose y must equal the
+    separate steps' y bit for bit): expert indices, counts, offsets, slot positions and source
+    tokens bit-exact; the combine weights and probability sums 1e-5; the grouped expert rows
+    y_perm (every kept row), the shared output and y (every token) within the stated tolerance;
+    the loss 1e-5. The 1,024-expert configuration reaches the 1,025-group tile list with its
+    997 empty experts and one group of about 22k rows. A small sample of tokens is also checked
+    against the per-token definition (oracle.token_output), which does not group the rows."""
     c = get_config(name)
     inp = make_inputs(c)
     run = LayerOnGpu(c, inp)
     o = run.steps()
-    ref = oracle.layer_forward(c, inp, with_outputs=False)
-    r, pm = ref["route"], ref["perm"]
+    y, aux, cnt = run.layer()
+    assert torch.equal(y, o["y"])
+    ref = oracle.layer_forward(c, inp, with_outputs=True)
+    r, pm, ef = ref["route"], ref["perm"], ref["experts"]
     assert np.array_equal(np_(o["idx"]), r["idx"])
     np.testing.assert_allclose(np_(o["w"]), r["w"], rtol=1e-5, atol=1e-7)
     assert np.array_equal(np_(o["count"]), r["count"])
+    assert np.array_equal(np_(cnt), r["count"])
     np.testing.assert_allclose(np_(o["prob"]), r["prob_sum"], rtol=1e-5, atol=1e-5)
     assert np.array_equal(np_(o["offsets"]), pm["offsets"])
     assert np.array_equal(np_(o["slot_pos"]), pm["slot_pos"])
     N = int(pm["offsets"][-1])
     assert np.array_equal(np_(o["src"])[:N], pm["src"])
     assert float(o["aux"]) == pytest.approx(ref["aux"], rel=1e-5)
-    y, aux, cnt = run.layer()
-    assert torch.equal(y, o["y"])
-    # a random sample fixes the rms; the 32 tokens with the largest outputs are added to the
-    # max, since the rounding errors grow with the magnitude of the summed rows
-    rng = np.random.default_rng(123)
-    rand = np.unique(np.concatenate([[0, c.T - 1], rng.choice(c.T, 126, replace=False)]))
+    assert float(aux) == float(o["aux"])
+    tol = tol_of(c)
+    ydt = "bf16" if o["y_perm"].dtype == torch.bfloat16 else "f32"
+    errs = {"y_perm": rel_err_stored(np_(o["y_perm"])[:N], ef["y_perm"], ydt)}
+    if c.n_shared:
+        errs["y_shared"] = rel_err(np_(o["y_shared"]), ef["y_shared"])
     yall = np_(y)
-    heavy = np.argsort(-np.abs(yall).max(axis=1))[:32]
-    sample = np.unique(np.concatenate([rand, heavy]))
-    yr = {int(t): oracle.token_output(c, inp, int(t), r["idx"][t], r["w"][t],
-                                      pm["slot_pos"][t] >= 0) for t in sample}
-    rms = np.sqrt(np.mean(np.stack([yr[int(t)] for t in rand]) ** 2))
-    err = max(float(np.max(np.abs(yall[t] - yr[int(t)]))) for t in sample)
-    assert err / rms <= tol_of(c), f"max|dy|/rms = {err / rms:.4f}" 
+    errs["y"] = rel_err(yall, ref["y"])
+    # the per-token definition on a sample: random tokens and the 16 with the largest outputs
+    rng = np.random.default_rng(123)
+    sample = np.unique(np.concatenate([[0, c.T - 1], rng.choice(c.T, 30, replace=False),
+                                       np.argsort(-np.abs(yall).max(axis=1))[:16]]))
+    rms = float(np.sqrt(np.mean(ref["y"] ** 2)))
+    errs["y_per_token"] = max(
+        float(np.max(np.abs(yall[t] - oracle.token_output(c, inp, int(t), r["idx"][t], r["w"][t],
+                                                            pm["slot_pos"][t] >= 0)))) / rms
+        for t in sample)
+    msg = f"{name}: worst max|d|/rms " + ", ".join(f"{k}={v:.3e}" for k, v in errs.items())
+    print(msg)
+    assert all(v <= tol for v in errs.values()), msg

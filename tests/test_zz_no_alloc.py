@@ -63,8 +63,17 @@ def test_noalloc_route_matches_workspace_route_twice_in_a_row():
         _same(ref, got)
 
 
+def test_noalloc_route_at_the_scratch_limit():
+    # 1,024 experts over 8,192 tokens: two 2 MiB tables of per-CTA partials (512 CTAs x 1,024
+    # experts x 4 bytes each), exactly the 4 MiB the library holds; one token more is refused
+    # (host-side test in test_abi.py)
+    ref, got = _route_both(get_config("lowrank", T=8192))
+    _same(ref, got)
+
+
 def test_noalloc_route_rejects_configurations_beyond_its_scratch():
-    c = get_config("lowrank")  # E = 1024 experts at d = 1024: ~8 MiB of scratch, over 4 MiB
+    # the full 1,024-expert configuration (T = 24,576) needs 8 E ceil(T/16) bytes = 12 MiB
+    c = get_config("lowrank")
     cfg = B.make_config(T=c.T, d=c.d, E=c.E, top_k=c.top_k, rank=c.rank, expert="lowrank")
     w = B.MoEWeights()
     w.w_router = 256
