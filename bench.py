@@ -189,7 +189,9 @@ def algorithmic(c, n_kept: int):
     # routed expert rows (bf16 for bf16 SwiGLU layers, else fp32), shared output and y in fp32
     ys = 2 if (c.dtype == "bf16" and c.expert == "swiglu") else 4
     out["combine"] = {"bytes": n_kept * d * ys + (T * d * 4.0 if S else 0) + 8.0 * T * k +
-                      T * d * 4.0}
+                      T * d * 4.0,
+                      "bytes_dtype_y": n_kept * d * ys + (T * d * es if S else 0) + 8.0 * T * k +
+                      T * d * es}
     return out
 
 
@@ -218,6 +220,11 @@ def roofline_table(c, n_kept, prof, steps, peaks, src):
             ach = a["bytes"] / (avg_ms * 1e-3) / 1e9
             row.update(bound="hbm", achieved=ach, peak=peaks["hbm_gbs"], unit="GB/s",
                        frac=ach / peaks["hbm_gbs"])
+            if "bytes_dtype_y" in a:
+                # the same launch against the byte count with y and the shared output in the
+                # layer's dtype (what a bf16 output would move), beside the fp32 figure above
+                ach2 = a["bytes_dtype_y"] / (avg_ms * 1e-3) / 1e9
+                row.update(achieved_dtype_y=ach2, frac_dtype_y=ach2 / peaks["hbm_gbs"])
         rows[name] = row
     tot = sum(ms for ms, n in prof.values())
     for name, (ms, n) in prof.items():
@@ -450,9 +457,88 @@ def run_ours(args, rank, world, local_rank):
     }
     if backward is not None:
         result["backward_parts"] = backward
+    if world == 1 and args.per_config != "none":
+        result["per_config"] = {
+            name: measure_config(name, args.steps, args.warmup, dev, flush, stream, peaks,
+                                 peak_src)
+            for name in args.per_config.split(",") if name and name != args.config}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(c, inp)
     return result
+
+
+def measure_config(name, K, W, dev, flush, stream, peaks, peak_src):
+    """One more configuration on this GPU, timed like the headline one: W warm-up layer calls,
+    then K calls each bracketed by CUDA events with the L2 flushed in between, then K calls with
+    the library's event profiler for the per-kernel table. Inputs resident, weights random-init
+    of the configuration's shapes."""
+    import torch
+
+    from fine_grained_mixture_moe_b200 import binding as B
+    from fine_grained_mixture_moe_b200.layer import MoELayer, upload_weights
+    from moe_synth import get_config, make_inputs
+
+    c = get_config(name)
+    inp = make_inputs(c)
+    cfg = B.make_config(T=c.T, d=c.d, E=c.E, top_k=c.top_k, n_shared=c.n_shared, ffn=c.ffn,
+                        ffn_shared=c.ffn_shared, rank=c.rank, score=c.score, expert=c.expert,
+                        dtype=c.dtype, norm_topk=c.norm_topk, capacity_factor=c.capacity_factor,
+                        aux_alpha=c.aux_alpha)
+    layer = MoELayer(cfg, upload_weights(cfg, inp, dev), dev)
+    x = torch.as_tensor(inp["x"]).to(layer.dtype).contiguous().to(dev)
+    y = torch.empty((c.T, c.d), dtype=torch.float32, device=dev)
+    aux = torch.empty((), dtype=torch.float32, device=dev)
+    cnt = torch.empty(c.E, dtype=torch.int32, device=dev)
+    for _ in range(W):
+        layer.forward(x, y, aux, cnt)
+    torch.cuda.synchronize()
+
+    def timed():
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(K)]
+        torch.cuda.synchronize()
+        for i in range(K):
+            flush.fill_(i & 0xff)
+            ev[i][0].record(stream)
+            layer.forward(x, y, aux, cnt)
+            ev[i][1].record(stream)
+        torch.cuda.synchronize()
+        return [a.elapsed_time(b) for a, b in ev]
+
+    ms = statistics.fmean(timed())
+    B.moe_debug_set(B.DEBUG_PROFILE, 1)
+    timed()
+    prof = B.moe_profile_read()
+    B.moe_debug_set(B.DEBUG_PROFILE, 0)
+    st, info = B.moe_get_device_error()
+    if st != 0:
+        raise RuntimeError(f"device error ({name}): {B.status_str(st)} info={info}")
+    # kept pairs from the permutation's offsets (capacity drops included)
+    idx = torch.empty((c.T, c.top_k), dtype=torch.int32, device=dev)
+    wts = torch.empty((c.T, c.top_k), dtype=torch.float32, device=dev)
+    prob = torch.empty(c.E, dtype=torch.float32, device=dev)
+    offs = torch.empty(c.E + 1, dtype=torch.int32, device=dev)
+    sl = torch.empty((c.T, c.top_k), dtype=torch.int32, device=dev)
+    sr = torch.empty(c.T * c.top_k, dtype=torch.int32, device=dev)
+    B.moe_route(cfg, x, layer.wstruct, idx, wts, cnt, prob, layer.ws, layer.ws_bytes)
+    B.moe_permute(cfg, x, idx, offs, sl, sr, None, layer.ws, layer.ws_bytes)
+    torch.cuda.synchronize()
+    n_kept = int(offs[-1])
+    counts = cnt.cpu().numpy()
+    table = roofline_table(c, n_kept, prof, K, peaks, peak_src)
+    out = {
+        "workload": workload_name(c),
+        "value": c.T / (ms * 1e-3), "unit": "tokens/s", "ms_per_step": ms, "steps": K,
+        "warmup": W, "dtype": c.dtype,
+        "kept_pairs": n_kept, "dropped_pairs": c.T * c.top_k - n_kept,
+        "expert_rows_min_max": [int(counts.min()), int(counts.max())],
+        "dead_experts": int((counts == 0).sum()),
+        "kernels": {k: {kk: (round(vv, 4) if isinstance(vv, float) else vv)
+                        for kk, vv in v.items()} for k, v in table.items()},
+    }
+    del layer, x, y
+    torch.cuda.empty_cache()
+    return out
 
 
 def backward_parts(c, cfg, layer, x, flush, stream, K, peaks):
@@ -529,28 +615,39 @@ def backward_parts(c, cfg, layer, x, flush, stream, K, peaks):
     }
 
 
-def _threads():
+def _cores() -> int:
     try:
-        from threadpoolctl import threadpool_info
-        n = [p.get("num_threads", 1) for p in threadpool_info()]
-        return max(n) if n else 1
-    except Exception:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
         return os.cpu_count() or 1
 
 
-def cpu_baseline(c, inp, T_sample=None):
-    """The oracle, as it stands, on a bounded token sample of the same workload."""
+def _oracle_seconds(c, inp, T, threads):
+    """Wall seconds of one oracle layer forward over the first T tokens with `threads` BLAS
+    threads (numpy's own loops are single-threaded)."""
     import oracle
-    T = c.T if T_sample is None else T_sample
+    from threadpoolctl import threadpool_limits
     sub = dict(inp)
     sub["x"] = inp["x"][:T]
     cs = c.with_(T=T)
-    t0 = time.perf_counter()
-    oracle.layer_forward(cs, sub)
-    dt = time.perf_counter() - t0
-    return {"value": T / dt, "unit": "tokens/s", "cores": _threads(), "kind": "oracle",
+    with threadpool_limits(limits=threads):
+        t0 = time.perf_counter()
+        oracle.layer_forward(cs, sub)
+        return time.perf_counter() - t0
+
+
+def cpu_baseline(c, inp, T_sample=None):
+    """The oracle, as it stands, on a bounded token sample of the same workload: once with
+    every core of the affinity mask, once on a single thread."""
+    T = min(c.T, T_sample or 2048)
+    cores = _cores()
+    dt_all = _oracle_seconds(c, inp, T, cores)
+    dt_one = _oracle_seconds(c, inp, T, 1)
+    return {"value": T / dt_all, "unit": "tokens/s", "cores": cores, "kind": "oracle",
             "sample": f"one layer forward over the first {T} tokens of the workload "
-                      f"({dt:.1f} s, fp64 numpy/OpenBLAS)"}
+                      f"({dt_all:.1f} s on {cores} cores, fp64 numpy/OpenBLAS)",
+            "single_thread": {"value": T / dt_one, "unit": "tokens/s", "cores": 1,
+                              "seconds": round(dt_one, 2)}}
 
 
 # ------------------------------------------------------------------ reference arm (oracle)
@@ -564,6 +661,8 @@ def run_reference(args):
     budget = 120.0 / max(args.steps + args.warmup, 1)
     T_s = int(max(32, min(c.T, budget / max(per_token_s, 1e-9))) // 32 * 32) or 32
     import oracle
+    from threadpoolctl import threadpool_limits
+    threadpool_limits(limits=_cores())
     sub = dict(inp)
     sub["x"] = inp["x"][:T_s]
     cs = c.with_(T=T_s)
@@ -581,7 +680,7 @@ def run_reference(args):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": workload_name(c), "tokens_per_step": T_s},
-        "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": _threads(), "kind": "oracle",
+        "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": _cores(), "kind": "oracle",
                          "sample": f"first {T_s} tokens of the workload per step"},
         "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -595,6 +694,9 @@ def main():
     ap.add_argument("--config", default="quartz")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--per-config", default="capacity,sigmoid,lowrank",
+                    help="further configurations timed on one GPU beside the headline one "
+                         "(comma-separated names, or 'none')")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

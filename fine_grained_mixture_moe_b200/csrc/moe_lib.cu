@@ -99,6 +99,7 @@ inline bool yperm_bf16(const moe_config_t *c) {
 struct Layout {
   size_t part_cnt, part_prob, chunk_base, kept;                 // route / statistics
   size_t chunk_count;                                           // moe_permute's own histogram
+  size_t lrank;                                                 // within-chunk ranks [T, k] u8
   size_t hidden, hidden_sh;                                     // experts
   size_t idx, wts, count, prob, offsets, slot_pos, src, x_perm, y_perm, y_shared, aux;  // layer
   size_t total;
@@ -119,6 +120,7 @@ Layout layout_of(const moe_config_t *c) {
   L.chunk_base = take(nch * E * 4);
   L.kept = take(E * 4);
   L.chunk_count = take(nch * E * 4);
+  L.lrank = take(T * k);
   L.hidden = take(T * k * width * es);
   L.hidden_sh = take(T * (size_t)c->n_shared * (size_t)c->ffn_shared * es);
   L.idx = take(T * k * 4);
@@ -381,7 +383,7 @@ moe_status_t launch_stats(const StatsArgs &sa, cudaStream_t st) {
 template <typename Tin>
 moe_status_t router_only(const moe_config_t *c, const void *x, const moe_weights_t *w,
                          int32_t *idx, float *wts, int32_t *part_cnt, float *part_prob,
-                         cudaStream_t st) {
+                         uint8_t *lrank, cudaStream_t st) {
   RouterArgs a;
   a.x = x;
   a.w = w->w_router;
@@ -391,6 +393,7 @@ moe_status_t router_only(const moe_config_t *c, const void *x, const moe_weights
   a.idx = idx; a.wts = wts;
   a.part_cnt = part_cnt;
   a.part_prob = part_prob;
+  a.lrank = lrank;
   return launch_router<Tin>(a, st);
 }
 
@@ -417,7 +420,7 @@ moe_status_t route_impl(const moe_config_t *c, const void *x, const moe_weights_
   }
   int32_t *pc = at<int32_t>(ws, L.part_cnt);
   float *pp = at<float>(ws, L.part_prob);
-  MOE_TRY(router_only<Tin>(c, x, w, idx, wts, pc, pp, st));
+  MOE_TRY(router_only<Tin>(c, x, w, idx, wts, pc, pp, nullptr, st));
   StatsArgs sa = stats_args(c, pc, pp);
   sa.count_out = count;
   sa.prob_out = prob;
@@ -426,21 +429,16 @@ moe_status_t route_impl(const moe_config_t *c, const void *x, const moe_weights_
 
 template <typename Tin>
 moe_status_t scatter_impl(const moe_config_t *c, const void *x, const int32_t *idx,
-                          const int32_t *chunk_base, const int32_t *kept, int32_t *offsets,
-                          int32_t *slot_pos, int32_t *src, void *x_perm, const int32_t *count,
-                          const float *prob, float *aux, cudaStream_t st) {
+                          const uint8_t *lrank, const int32_t *chunk_base, const int32_t *kept,
+                          int32_t *offsets, int32_t *slot_pos, int32_t *src, void *x_perm,
+                          const int32_t *count, const float *prob, float *aux, cudaStream_t st) {
   ProfScope ps(K_PERM_SCATTER, st);
-  // shared memory: the CTA's PM_TPC token rows, then per expert the lane mask, the chunk's
-  // base rank and the offset
-  const size_t smem = (size_t)PM_TPC * c->d * sizeof(Tin) + (size_t)c->E * 12;
-  if (smem > 48 * 1024 &&
-      cudaFuncSetAttribute(perm_scatter_kernel<Tin>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)smem) != cudaSuccess)
-    return MOE_ERR_CUDA;
-  return launch_pdl(perm_scatter_kernel<Tin>, dim3(ceil_div(c->T, PM_CHUNK) * PM_SPLIT), dim3(256),
-                    smem, st, idx, c->T, c->top_k, c->E, capacity_of(c), chunk_base, kept, offsets,
-                    slot_pos, src, (const Tin *)x, (Tin *)x_perm, c->d, count, prob, c->aux_alpha,
-                    aux);
+  const size_t smem = (size_t)c->E * sizeof(int);  // the expert offsets
+  const int grid = std::max(1, std::min(ceil_div(c->T, PM_THREADS / 32),
+                                        num_sms() * PM_CTAS_PER_SM));
+  return launch_pdl(perm_scatter_kernel<Tin>, dim3(grid), dim3(PM_THREADS), smem, st, idx, lrank,
+                    c->T, c->top_k, c->E, capacity_of(c), chunk_base, kept, offsets, slot_pos,
+                    src, (const Tin *)x, (Tin *)x_perm, c->d, count, prob, c->aux_alpha, aux);
 }
 
 template <typename Tin>
@@ -453,19 +451,20 @@ moe_status_t permute_impl(const moe_config_t *c, const void *x, const int32_t *i
   }
   const int nch = ceil_div(c->T, PM_CHUNK);
   int32_t *cc = at<int32_t>(ws, L.chunk_count), *cb = at<int32_t>(ws, L.chunk_base);
+  uint8_t *lr = at<uint8_t>(ws, L.lrank);
   {
     const size_t smem = (size_t)8 * c->E * 4;
     if (cudaFuncSetAttribute(perm_hist_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
       return MOE_ERR_CUDA;
     ProfScope ps(K_PERM_HIST, st);
     MOE_TRY(launch_pdl(perm_hist_kernel, dim3(ceil_div(nch, 8)), dim3(256), smem, st, idx, c->T,
-                       c->top_k, c->E, cc, nch));
+                       c->top_k, c->E, cc, lr, nch));
   }
   StatsArgs sa = stats_args(c, cc, nullptr);
   sa.chunk_base = cb;
   sa.kept = at<int32_t>(ws, L.kept);
   MOE_TRY(launch_stats(sa, st));
-  return scatter_impl<Tin>(c, x, idx, cb, sa.kept, offsets, slot_pos, src, x_perm, nullptr,
+  return scatter_impl<Tin>(c, x, idx, lr, cb, sa.kept, offsets, slot_pos, src, x_perm, nullptr,
                            nullptr, nullptr, st);
 }
 
@@ -779,10 +778,11 @@ moe_status_t moe_layer_forward(const moe_config_t *cfg, const void *x, const moe
   int32_t *pc = at<int32_t>(ws, L.part_cnt);
   float *pp = at<float>(ws, L.part_prob);
   int32_t *cb = at<int32_t>(ws, L.chunk_base);
+  uint8_t *lr = at<uint8_t>(ws, L.lrank);
   if (cfg->dtype == MOE_DTYPE_BF16)
-    MOE_TRY(router_only<__nv_bfloat16>(cfg, x, w, idx, wts, pc, pp, st));
+    MOE_TRY(router_only<__nv_bfloat16>(cfg, x, w, idx, wts, pc, pp, lr, st));
   else
-    MOE_TRY(router_only<float>(cfg, x, w, idx, wts, pc, pp, st));
+    MOE_TRY(router_only<float>(cfg, x, w, idx, wts, pc, pp, lr, st));
   StatsArgs sa = stats_args(cfg, pc, pp);
   sa.count_out = cnt;
   sa.prob_out = prob;
@@ -790,11 +790,11 @@ moe_status_t moe_layer_forward(const moe_config_t *cfg, const void *x, const moe
   sa.kept = at<int32_t>(ws, L.kept);
   MOE_TRY(launch_stats(sa, st));
   if (cfg->dtype == MOE_DTYPE_BF16)
-    MOE_TRY(scatter_impl<__nv_bfloat16>(cfg, x, idx, cb, sa.kept, offsets, slot_pos, src, x_perm,
-                                        cnt, prob, aux, st));
+    MOE_TRY(scatter_impl<__nv_bfloat16>(cfg, x, idx, lr, cb, sa.kept, offsets, slot_pos, src,
+                                        x_perm, cnt, prob, aux, st));
   else
-    MOE_TRY(scatter_impl<float>(cfg, x, idx, cb, sa.kept, offsets, slot_pos, src, x_perm, cnt,
-                                prob, aux, st));
+    MOE_TRY(scatter_impl<float>(cfg, x, idx, lr, cb, sa.kept, offsets, slot_pos, src, x_perm,
+                                cnt, prob, aux, st));
   // T > 0 here: the expert forward launched at least two kernels after the scatter
   MOE_TRY(experts_impl(cfg, x_perm, offsets, x, w, y_perm, y_sh, ws, st));
   return combine_impl(cfg, y_perm, y_sh, slot_pos, wts, y, st, true);
@@ -999,7 +999,7 @@ moe_status_t route_noalloc_impl(const moe_config_t *c, const void *x, const moe_
   // array by an earlier call is read
   int32_t *pc = (int32_t *)(scratch + L.part_cnt);
   float *pp = (float *)(scratch + L.part_prob);
-  MOE_TRY(router_only<Tin>(c, x, w, idx, wts, pc, pp, st));
+  MOE_TRY(router_only<Tin>(c, x, w, idx, wts, pc, pp, nullptr, st));
   StatsArgs sa = stats_args(c, pc, pp);
   sa.count_out = count;
   sa.prob_out = prob;

@@ -57,6 +57,8 @@ struct RouterArgs {
   float *part_prob;     // [nblk, E]
   int32_t *count_out;   // [E]
   float *prob_out;      // [E]
+  uint8_t *lrank;       // [T, k] or null: rank of pair (t, j) among the CTA's tokens routed to
+                        // the same expert (the permutation's within-chunk rank)
 };
 
 // Eight consecutive elements (bf16: 16 bytes; fp32: 32 bytes) and their pairs as fp32.
@@ -521,7 +523,7 @@ __device__ float finish_logit(double s, const Tin *xrow, const Tin *wrow, int d,
 // warp, fixed-order trees; the logits row becomes the probability basis of the load-balancing
 // statistics. One out-of-line copy serves the proven tokens and the settled ones.
 __device__ __noinline__ void finish_token(const RouterArgs &a, float *lrow, const int *br, int t,
-                                          int *cnt) {
+                                          int *cnt, int *sel) {
   const int lane = threadIdx.x & 31;
   const int E = a.E, k = a.k;
   const bool sigmoid = a.score == MOE_SCORE_SIGMOID;
@@ -548,6 +550,7 @@ __device__ __noinline__ void finish_token(const RouterArgs &a, float *lrow, cons
     a.idx[(size_t)t * k + lane] = ej;
     a.wts[(size_t)t * k + lane] = a.norm ? pj / psel : pj;
     atomicAdd(&cnt[ej], 1);
+    sel[lane] = ej;
   }
   __syncwarp();
 }
@@ -580,6 +583,7 @@ __global__ void __launch_bounds__(RT_THREADS, EPT == RT_EPT ? 2 : 1) router_kern
   int *cnt = (int *)(smem_raw + SL.cnt);
   double *xnorm = (double *)(smem_raw + SL.xnorm);
   unsigned *cmask = (unsigned *)(smem_raw + SL.cmask);  // [listed token][E/32]
+  int *s_sel = (int *)(smem_raw + SL.part);  // [RT_TM][8] selections; `part` is free after the screen
   __shared__ int s_nflag, s_flag[RT_TM];
   __shared__ unsigned long long s_wnmax;  // bits of nonnegative doubles / floats order as integers
   __shared__ int s_offmax, s_bmax;
@@ -829,7 +833,7 @@ __global__ void __launch_bounds__(RT_THREADS, EPT == RT_EPT ? 2 : 1) router_kern
     }
     const bool proven = __all_sync(0xffffffffu, ok) && !bad && !force && Bk < INFINITY;
     if (proven) {
-      finish_token(a, lrow, brw, t0 + tt, cnt);
+      finish_token(a, lrow, brw, t0 + tt, cnt, s_sel + tt * 8);
       continue;
     }
     // candidates: every expert whose key is not provably below the (k+1)-th approximate key
@@ -948,11 +952,21 @@ __global__ void __launch_bounds__(RT_THREADS, EPT == RT_EPT ? 2 : 1) router_kern
       const int tt = s_flag[f];
       warp_rank_into((sigmoid ? keys : lg) + tt * E, E, k, brw);
       __syncwarp();
-      finish_token(a, lg + tt * E, brw, t0 + tt, cnt);
+      finish_token(a, lg + tt * E, brw, t0 + tt, cnt, s_sel + tt * 8);
     }
   }
   __syncthreads();
 
+  // ---- within-chunk ranks: pair (tt, j) counts the earlier tokens of the CTA that selected the
+  // same expert (a token selects an expert at most once)
+  if (a.lrank && tid < ntok * k) {
+    const int tt = tid / k, j = tid - tt * k;
+    const int e = s_sel[tt * 8 + j];
+    int r = 0;
+    for (int u = 0; u < tt; ++u)
+      for (int jj = 0; jj < k; ++jj) r += s_sel[u * 8 + jj] == e ? 1 : 0;
+    a.lrank[(size_t)(t0 + tt) * k + j] = (uint8_t)r;
+  }
   // ---- per-CTA statistics (fixed token order), then the last CTA reduces in CTA order
   for (int e = tid; e < E; e += RT_THREADS) {
     float ps = 0.0f;
