@@ -195,8 +195,10 @@ def algorithmic(c, n_kept: int):
     return out
 
 
-def roofline_table(c, n_kept, prof, steps, peaks, src):
-    """Achieved vs peak per kernel kind from the profiler's per-launch averages."""
+def roofline_table(c, n_kept, prof, steps, peaks, src, in_step=None):
+    """Achieved vs peak per kernel kind from the profiler's per-launch averages (CUDA events
+    around each launch) and, when given, from the in-step durations (device timestamps, the
+    launches overlapped as in the step): `in_step_us` and `frac_in_step`."""
     alg = algorithmic(c, n_kept)
     # fp32 FMA on the CUDA cores: 148 SMs x 128 lanes x 2 flops at the maximum SM clock
     fp32_peak = 148 * 128 * 2 * peaks.get("sm_max_mhz", 1965.0) * 1e6 / 1e12  # TFLOP/s, nominal
@@ -225,6 +227,10 @@ def roofline_table(c, n_kept, prof, steps, peaks, src):
                 # layer's dtype (what a bf16 output would move), beside the fp32 figure above
                 ach2 = a["bytes_dtype_y"] / (avg_ms * 1e-3) / 1e9
                 row.update(achieved_dtype_y=ach2, frac_dtype_y=ach2 / peaks["hbm_gbs"])
+        if in_step and name in in_step and "frac" in row:
+            us = in_step[name]
+            row["in_step_us"] = us
+            row["frac_in_step"] = row["frac"] * row["avg_us"] / us
         rows[name] = row
     tot = sum(ms for ms, n in prof.values())
     for name, (ms, n) in prof.items():
@@ -351,11 +357,13 @@ def run_ours(args, rank, world, local_rank):
     if st != 0:
         raise RuntimeError(f"device error in the timed region: {B.status_str(st)} info={info}")
 
-    # pass 2: per-kernel durations (library event profiler, same steps)
+    # pass 2: per-kernel durations (library event profiler, same steps), then the same kernels'
+    # durations inside the step from the library's device timestamps
     B.moe_debug_set(B.DEBUG_PROFILE, 1)
     timed(args.steps)
     prof = B.moe_profile_read()
     B.moe_debug_set(B.DEBUG_PROFILE, 0)
+    in_step = in_step_durations(step, args.steps, flush) if world == 1 else None
 
     # pass 3: end to end through the public API with pinned host buffers. Each step copies its
     # tokens in, runs the layer and copies y and the loss out. Steps are double-buffered over
@@ -412,7 +420,7 @@ def run_ours(args, rank, world, local_rank):
     peaks, peak_src = load_peaks()
     backward = backward_parts(c, cfg, layer, x, flush, stream, args.steps, peaks) \
         if world == 1 else None
-    table = roofline_table(c, n_kept, prof, args.steps, peaks, peak_src)
+    table = roofline_table(c, n_kept, prof, args.steps, peaks, peak_src, in_step)
     dom = max(table, key=lambda n: table[n]["share"] or 0.0)
     dr = table[dom]
     launches_per_step = sum(n for _, n in prof.values()) / max(args.steps, 1)
@@ -467,6 +475,27 @@ def run_ours(args, rank, world, local_rank):
     return result
 
 
+def in_step_durations(step, K, flush):
+    """Per-kernel-kind durations inside the step from the library's device timestamps
+    (MOE_DEBUG_STAMP), averaged over K steps with the L2 flushed before each."""
+    import torch
+
+    from fine_grained_mixture_moe_b200 import binding as B
+    B.moe_debug_set(B.DEBUG_STAMP, 1)
+    acc = {}
+    try:
+        for i in range(K):
+            flush.fill_(i & 0xff)
+            torch.cuda.synchronize()
+            B.moe_stamp_read()  # clears the records of the flush's interval
+            step()
+            for n, us in B.moe_stamp_read().items():
+                acc.setdefault(n, []).append(us)
+    finally:
+        B.moe_debug_set(B.DEBUG_STAMP, 0)
+    return {n: statistics.fmean(v) for n, v in acc.items()}
+
+
 def measure_config(name, K, W, dev, flush, stream, peaks, peak_src):
     """One more configuration on this GPU, timed like the headline one: W warm-up layer calls,
     then K calls each bracketed by CUDA events with the L2 flushed in between, then K calls with
@@ -510,6 +539,7 @@ def measure_config(name, K, W, dev, flush, stream, peaks, peak_src):
     timed()
     prof = B.moe_profile_read()
     B.moe_debug_set(B.DEBUG_PROFILE, 0)
+    in_step = in_step_durations(lambda: layer.forward(x, y, aux, cnt), K, flush)
     st, info = B.moe_get_device_error()
     if st != 0:
         raise RuntimeError(f"device error ({name}): {B.status_str(st)} info={info}")
@@ -525,7 +555,7 @@ def measure_config(name, K, W, dev, flush, stream, peaks, peak_src):
     torch.cuda.synchronize()
     n_kept = int(offs[-1])
     counts = cnt.cpu().numpy()
-    table = roofline_table(c, n_kept, prof, K, peaks, peak_src)
+    table = roofline_table(c, n_kept, prof, K, peaks, peak_src, in_step)
     out = {
         "workload": workload_name(c),
         "value": c.T / (ms * 1e-3), "unit": "tokens/s", "ms_per_step": ms, "steps": K,

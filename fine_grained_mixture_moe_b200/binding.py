@@ -23,7 +23,7 @@ STATUS_NAMES = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED",
 SCORE = {"softmax": 0, "sigmoid": 1}
 EXPERT = {"swiglu": 0, "lowrank": 1}
 DTYPE = {"f32": 0, "bf16": 1}
-DEBUG_FORCE_EXACT, DEBUG_WAIT_LIMIT_NS, DEBUG_PROFILE = 1, 2, 3
+DEBUG_FORCE_EXACT, DEBUG_WAIT_LIMIT_NS, DEBUG_PROFILE, DEBUG_STAMP = 1, 2, 3, 4
 
 
 class MoEError(RuntimeError):
@@ -89,6 +89,7 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
         "moe_debug_set": (c_int32, [c_int32, c_int64]),
         "moe_profile_read": (c_int32, [P(ctypes.c_char_p), P(ctypes.c_double), P(c_int64),
                                        c_int32]),
+        "moe_stamp_read": (c_int32, [P(ctypes.c_char_p), P(ctypes.c_double), c_int32]),
         "moe_debug_wait_timeout_probe": (c_int32, [c_void_p]),
         "moe_route_noalloc": (c_int32, [P(MoEConfig), c_void_p, P(MoEWeights), c_void_p,
                                         c_void_p, c_void_p, c_void_p, c_void_p]),
@@ -106,7 +107,7 @@ EXPORTED = ("moe_workspace_size", "moe_capacity", "moe_route", "moe_permute",
             "moe_combine_backward", "moe_route_backward",
             "moe_layer_forward",
             "moe_status_str", "moe_get_device_error", "moe_debug_set", "moe_profile_read",
-            "moe_debug_wait_timeout_probe", "moe_route_noalloc")
+            "moe_stamp_read", "moe_debug_wait_timeout_probe", "moe_route_noalloc")
 
 
 def _ptr(t) -> Optional[int]:
@@ -244,6 +245,16 @@ def moe_profile_read(max_kinds: int = 32):
     n = (c_int64 * max_kinds)()
     cnt = load().moe_profile_read(names, ms, n, max_kinds)
     return {names[i].decode(): (ms[i], int(n[i])) for i in range(min(cnt, max_kinds))}
+
+
+def moe_stamp_read(max_kinds: int = 32):
+    """In-step kernel durations (microseconds) per kind since the last read (moe_stamp_read)."""
+    names = (ctypes.c_char_p * max_kinds)()
+    us = (ctypes.c_double * max_kinds)()
+    cnt = load().moe_stamp_read(names, us, max_kinds)
+    if cnt < 0:
+        raise MoEError("moe_stamp_read", 4)
+    return {names[i].decode(): us[i] for i in range(min(cnt, max_kinds))}
 
 
 def moe_debug_wait_timeout_probe(stream=None) -> None:

@@ -64,6 +64,7 @@ __global__ void __launch_bounds__(256, sizeof(Ty) == 2 ? 4 : 3) combine_kernel(c
   constexpr int V = YV::N;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t = blockIdx.x * 8 + warp;
+  const KernelStamp stamp(K_COMBINE);
   if (!early) griddep_wait();
   int pos_l = -1;
   float w_l = 0.0f;
@@ -72,6 +73,7 @@ __global__ void __launch_bounds__(256, sizeof(Ty) == 2 ? 4 : 3) combine_kernel(c
     w_l = __ldcg(w + (size_t)t * k + lane);
   }
   if (early) griddep_wait();
+  stamp.started();
   griddep_launch();
   if (t >= T) return;
   int pos[8];
@@ -109,7 +111,9 @@ __global__ void __launch_bounds__(256, sizeof(Ty) == 2 ? 4 : 3) combine_kernel(c
 
 __global__ void aux_loss_kernel(const int32_t *__restrict__ count, const float *__restrict__ prob,
                                 int E, int T, int k, float alpha, float *__restrict__ loss) {
+  const KernelStamp stamp(K_AUX);
   griddep_wait();
+  stamp.started();
   griddep_launch();
   double s = 0.0;
   for (int e = threadIdx.x; e < E; e += 32) s += (double)count[e] * (double)prob[e];

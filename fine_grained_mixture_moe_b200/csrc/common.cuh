@@ -40,6 +40,36 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
   return t;
 }
 
+// ------------------------------------------------------------------ kernel kinds and stamps
+// Kinds of the library's forward kernels (the host's profiler and the device stamps share them).
+enum KernelKind {
+  K_ROUTER, K_STATS, K_PERM_HIST, K_PERM_SCATTER, K_GEMM_GATEUP, K_GEMM_DOWN, K_GEMM_LR1,
+  K_GEMM_LR2, K_COMBINE, K_AUX, K_COUNT
+};
+
+// In-step timestamps. With stamping on (moe_debug_set(MOE_DEBUG_STAMP, 1)) a kernel records, per
+// kind, the global-timer time at which its first CTA passed griddep_wait (its inputs final) and
+// the time its last warp finished, as a min / max over 32 slots (CTA index mod 32) to spread the
+// atomics. Unlike CUDA events around each launch, this leaves programmatic dependent launch in
+// place, so a kernel is measured as it runs inside the layer call.
+constexpr int STAMP_SLOTS = 32;
+__device__ int g_stamp_on = 0;
+__device__ unsigned long long g_stamp[K_COUNT][STAMP_SLOTS][2];
+
+struct KernelStamp {
+  int kind;
+  bool on;
+  __device__ __forceinline__ explicit KernelStamp(int k) : kind(k), on(g_stamp_on != 0) {}
+  __device__ __forceinline__ void started() const {
+    if (on && threadIdx.x == 0)
+      atomicMin(&g_stamp[kind][blockIdx.x & (STAMP_SLOTS - 1)][0], globaltimer_ns());
+  }
+  __device__ __forceinline__ ~KernelStamp() {
+    if (on && (threadIdx.x & 31) == 0)
+      atomicMax(&g_stamp[kind][blockIdx.x & (STAMP_SLOTS - 1)][1], globaltimer_ns());
+  }
+};
+
 // ------------------------------------------------------------------ element conversion
 template <typename T> struct Elem;
 template <> struct Elem<float> {

@@ -17,7 +17,9 @@ __global__ void __launch_bounds__(256) gemm_simt_kernel(GroupedGemm p) {
   const int G = p.E + p.has_shared;
   int *prefix = sh_prefix;
   int *tmp = sh_prefix + G + 1;
+  const KernelStamp stamp(p.kind);
   griddep_wait();
+  stamp.started();
   griddep_launch();
   const int total = build_tile_prefix(p, SM_BM, SM_BN, prefix, tmp);
   const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;

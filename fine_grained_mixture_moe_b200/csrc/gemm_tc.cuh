@@ -181,7 +181,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1) gemm_tc_kernel(const __grid_con
     asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)&P.maps.a_r) : "memory");
     asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)&P.maps.b0_r) : "memory");
   }
+  const KernelStamp stamp(p.kind);
   griddep_wait();
+  stamp.started();
   griddep_launch();
   const int total = build_tile_prefix(p, TC_BM, BN, prefix, scan_tmp);  // contains __syncthreads
   tc_fence_before();

@@ -143,7 +143,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TC_THREADS, 1)
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
   }
+  const KernelStamp stamp(p.kind);
   griddep_wait();
+  stamp.started();
   griddep_launch();
   const int total = build_tile_prefix(p, TC2_BM, BN, prefix, scan_tmp);
   tc_fence_before();

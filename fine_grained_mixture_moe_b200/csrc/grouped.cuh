@@ -45,6 +45,7 @@ struct GroupedGemm {
   int b_rows_s;            // rows of the shared weight viewed as [b_rows_s, piece_k]
   void *out_s;
   int ldo_s;
+  int kind;                // KernelKind of the launch (in-step stamps)
 };
 
 // Tile counts per group and their exclusive prefix in shared memory (all threads call).

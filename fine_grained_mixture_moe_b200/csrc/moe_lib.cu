@@ -164,10 +164,6 @@ int num_sms() {
 }
 
 // ------------------------------------------------------------------ profiling (debug)
-enum KernelKind {
-  K_ROUTER, K_STATS, K_PERM_HIST, K_PERM_SCATTER, K_GEMM_GATEUP, K_GEMM_DOWN, K_GEMM_LR1,
-  K_GEMM_LR2, K_COMBINE, K_AUX, K_COUNT
-};
 const char *kKindName[K_COUNT] = {"router", "stats", "perm_hist", "perm_scatter", "gemm_gateup",
                                   "gemm_down", "gemm_lowrank_v", "gemm_lowrank_u", "combine",
                                   "aux_loss"};
@@ -196,6 +192,17 @@ struct ProfScope {
     if (slot >= 0) cudaEventRecord(g_prof.ev[2 * slot + 1], st);
   }
 };
+
+// Sets every in-step stamp slot to (no start, no end).
+moe_status_t stamp_reset() {
+  static unsigned long long h[K_COUNT][STAMP_SLOTS][2];
+  for (int k = 0; k < K_COUNT; ++k)
+    for (int sl = 0; sl < STAMP_SLOTS; ++sl) {
+      h[k][sl][0] = ~0ull;
+      h[k][sl][1] = 0ull;
+    }
+  return cudaMemcpyToSymbol(g_stamp, h, sizeof(h)) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
 
 moe_status_t last_launch_status() {
   const cudaError_t e = cudaGetLastError();
@@ -287,6 +294,7 @@ moe_status_t launch_tc(const GroupedGemm &g, cudaStream_t st, int kind) {
   TcParams P;
   std::memset(&P, 0, sizeof(P));
   P.p = g;
+  P.p.kind = kind;
   if (!build_maps(g, MODE == MODE_GATEUP, BN, &P.maps)) return MOE_ERR_CUDA;
   const int G = g.E + g.has_shared;
   const size_t smem = tc_smem_bytes<MODE, BN>(G);
@@ -307,6 +315,7 @@ moe_status_t launch_tc2(const GroupedGemm &g, cudaStream_t st, int kind) {
   TcParams P;
   std::memset(&P, 0, sizeof(P));
   P.p = g;
+  P.p.kind = kind;
   if (!build_maps(g, MODE == MODE_GATEUP, 128, &P.maps)) return MOE_ERR_CUDA;
   const int G = g.E + g.has_shared;
   static_assert(tc2_stages<MODE>(1024 + 1) >= 2, "tile list of 1024 experts leaves no room");
@@ -334,8 +343,10 @@ moe_status_t launch_simt(const GroupedGemm &g, cudaStream_t st, int kind) {
   const long long bound = tile_bound(g, SM_BM, SM_BN);
   if (bound == 0) return MOE_OK;
   const int grid = (int)std::min<long long>((long long)num_sms() * 8, bound);
+  GroupedGemm gk = g;
+  gk.kind = kind;
   ProfScope ps(kind, st);
-  return launch_pdl(kern, dim3(grid), dim3(256), smem, st, g);
+  return launch_pdl(kern, dim3(grid), dim3(256), smem, st, gk);
 }
 
 template <int MODE>
@@ -839,6 +850,11 @@ moe_status_t moe_debug_set(int32_t what, int64_t value) {
       const unsigned long long v = (unsigned long long)value;
       return cudaMemcpyToSymbol(g_wait_limit_ns, &v, sizeof(v)) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
     }
+    case MOE_DEBUG_STAMP: {
+      const int v = value != 0;
+      if (stamp_reset() != MOE_OK) return MOE_ERR_CUDA;
+      return cudaMemcpyToSymbol(g_stamp_on, &v, sizeof(int)) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+    }
     case MOE_DEBUG_PROFILE: {
       std::lock_guard<std::mutex> lk(g_prof_mu);
       if (value && !g_prof.created) {
@@ -852,6 +868,28 @@ moe_status_t moe_debug_set(int32_t what, int64_t value) {
     }
   }
   return MOE_ERR_INVALID_ARG;
+}
+
+int32_t moe_stamp_read(const char **names, double *us, int32_t max) {
+  if (cudaDeviceSynchronize() != cudaSuccess) return -1;
+  static unsigned long long h[K_COUNT][STAMP_SLOTS][2];
+  if (cudaMemcpyFromSymbol(h, g_stamp, sizeof(h)) != cudaSuccess) return -1;
+  if (stamp_reset() != MOE_OK) return -1;
+  int out = 0;
+  for (int k = 0; k < K_COUNT; ++k) {
+    unsigned long long t0 = ~0ull, t1 = 0ull;
+    for (int sl = 0; sl < STAMP_SLOTS; ++sl) {
+      t0 = std::min(t0, h[k][sl][0]);
+      t1 = std::max(t1, h[k][sl][1]);
+    }
+    if (t0 == ~0ull || t1 <= t0) continue;
+    if (out < max) {
+      if (names) names[out] = kKindName[k];
+      if (us) us[out] = (double)(t1 - t0) * 1e-3;
+    }
+    ++out;
+  }
+  return out;
 }
 
 int32_t moe_profile_read(const char **names, double *total_ms, int64_t *launches, int32_t max) {

@@ -31,7 +31,9 @@ __global__ void __launch_bounds__(256) perm_hist_kernel(const int32_t *__restric
                                                         int32_t *__restrict__ chunk_count,
                                                         uint8_t *__restrict__ lrank,
                                                         int nchunks) {
+  const KernelStamp stamp(K_PERM_HIST);
   griddep_wait();
+  stamp.started();
   griddep_launch();
   extern __shared__ unsigned sh_mask[];  // [8][E]
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -111,8 +113,10 @@ __global__ void __launch_bounds__(PM_THREADS, PM_CTAS_PER_SM) perm_scatter_kerne
       }
     }
   };
+  const KernelStamp stamp(K_PERM_SCATTER);
   if (t < T) load_token(t);
   griddep_wait();
+  stamp.started();
   griddep_launch();
   for (int e = tid; e < E; e += PM_THREADS) s_off[e] = kept[e];
   __syncthreads();

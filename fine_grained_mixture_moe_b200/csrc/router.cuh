@@ -41,8 +41,9 @@ constexpr int RT_TPT = 8;          // tokens per thread
 constexpr int RT_EPT = 3;          // experts per thread (6 in the wide form for many experts)
 constexpr int RT_EPT_WIDE = 6;
 constexpr int RT_WIDE_MIN_E = 97;  // the wide form from this many experts, when it fits
-constexpr int RT_SEL_THREAD_MAX_E = 64;  // ranking: up to this many experts each lane counts
-                                         // the rank of its own; above, iterative warp argmax
+constexpr int RT_SEL_THREAD_MAX_E = 64;  // ranking: up to this many experts a thread counts the
+                                         // rank of one (token, expert) pair; above, a warp per
+                                         // token takes the largest keys in turn
 constexpr int EXPANSION_MAX = 40;
 
 struct RouterArgs {
@@ -400,9 +401,23 @@ __device__ __forceinline__ float sigmoid_key(float l, float b, bool force) {
 // ------------------------------------------------------------------ kernel
 constexpr int RT_WD = 4;  // W chunks in flight per lane pair (cp.async ring)
 
+// The kernel's scalars in shared memory, kept in the dynamic allocation so that the host's size
+// check covers every byte the kernel uses.
+struct RouterMisc {
+  uint64_t xbar;                 // token-row copies
+  unsigned long long wnmax;      // max_e |W_e| bound (bits of a nonnegative double)
+  int nflag, offmax, bmax;       // listed tokens; max |offset|, max |bias| (bits of floats)
+  int xabort;
+  unsigned badtok, proven;       // bit tt: a non-finite logit; the order is proven
+  int flag[RT_TM];               // listed tokens
+  unsigned lmax[RT_TM];          // max |l| per token (bits of a nonnegative float)
+};
+constexpr int RT_MISC_BYTES = 256;
+static_assert(sizeof(RouterMisc) <= RT_MISC_BYTES, "router scalars");
+
 // Shared-memory layout of the router kernel (byte offsets), shared by host and device.
 struct RouterSmem {
-  size_t xs, xs_stride, ring, part, wsq, wn, off, lg, keys, byrank, cnt, xnorm, cmask, total;
+  size_t xs, xs_stride, ring, part, wsq, wn, off, lg, keys, cnt, xnorm, cmask, misc, total;
 };
 __host__ __device__ inline RouterSmem router_smem(int E, bool sigmoid, int d, int esize, int ept) {
   RouterSmem L;
@@ -421,10 +436,10 @@ __host__ __device__ inline RouterSmem router_smem(int E, bool sigmoid, int d, in
   L.off = take((size_t)E * sizeof(float));
   L.lg = take((size_t)RT_TM * E * sizeof(float));
   L.keys = take(sigmoid ? (size_t)RT_TM * E * sizeof(float) : 0);
-  L.byrank = take((size_t)RT_WARPS * 9 * sizeof(int));
   L.cnt = take((size_t)E * sizeof(int));
   L.xnorm = take(RT_TM * sizeof(double));
   L.cmask = take((size_t)RT_TM * ((E + 31) / 32) * sizeof(unsigned));  // candidates per listed token
+  L.misc = take(RT_MISC_BYTES);  // barrier and per-CTA scalars (RouterMisc)
   L.total = o;
   return L;
 }
@@ -479,31 +494,6 @@ __device__ __forceinline__ void warp_topn(const float *krow, int E, int n, int (
   }
 }
 
-// Experts of rank 0..n-1 of a row (descending key, NaN as -infinity, ties to the lower index)
-// into br[0..n), one warp. Up to 64 experts every lane counts the rank of its own experts.
-__device__ __noinline__ void warp_rank_into(const float *krow, int E, int n, int *br) {
-  const int lane = threadIdx.x & 31;
-  if (E <= RT_SEL_THREAD_MAX_E) {
-    for (int e = lane; e < E; e += 32) {
-      float v = krow[e];
-      if (v != v) v = -INFINITY;
-      int rank = 0;
-      for (int e2 = 0; e2 < E; ++e2) {
-        float v2 = krow[e2];
-        if (v2 != v2) v2 = -INFINITY;
-        rank += (v2 > v || (v2 == v && e2 < e)) ? 1 : 0;
-      }
-      if (rank < n) br[rank] = e;
-    }
-  } else {
-    int sel[9];
-    warp_topn(krow, E, n, sel);
-#pragma unroll
-    for (int j = 0; j < 9; ++j)
-      if (j < n && lane == 0) br[j] = sel[j];
-  }
-}
-
 // Canonical logit from the fp64 sum s of the exact products plus the offset (every lane holds
 // the same s): |s - S| <= gamma_{d+16} (sum |x_i W_i| + |off|) <= (d+16) 2^-52 (|x||W_e| + |off|).
 // When no fp32 rounding boundary lies within that distance, RN32(s) is the canonical logit;
@@ -517,42 +507,6 @@ __device__ float finish_logit(double s, const Tin *xrow, const Tin *wrow, int d,
   double mh, ml;
   if (force_level == 0 && rn32_certain(s, B, r, up, dn, mh, ml)) return r;
   return resolve_logit<Tin>(xrow, wrow, d, off, force_level);
-}
-
-// Probabilities, weights and outputs of token t (row lrow of logits, experts by rank in br), one
-// warp, fixed-order trees; the logits row becomes the probability basis of the load-balancing
-// statistics. One out-of-line copy serves the proven tokens and the settled ones.
-__device__ __noinline__ void finish_token(const RouterArgs &a, float *lrow, const int *br, int t,
-                                          int *cnt, int *sel) {
-  const int lane = threadIdx.x & 31;
-  const int E = a.E, k = a.k;
-  const bool sigmoid = a.score == MOE_SCORE_SIGMOID;
-  float m = -INFINITY, s = 0.0f;
-  if (!sigmoid) {
-    for (int e = lane; e < E; e += 32) m = fmaxf(m, lrow[e]);
-    m = warp_max_f(m);
-    for (int e = lane; e < E; e += 32) s += expf(lrow[e] - m);
-  } else {
-    for (int e = lane; e < E; e += 32) s += 1.0f / (1.0f + expf(-lrow[e]));
-  }
-  s = warp_sum_f(s);
-  int ej = 0;
-  float pj = 0.0f;
-  if (lane < k) {
-    ej = br[lane];
-    pj = !sigmoid ? expf(lrow[ej] - m) / s : 1.0f / (1.0f + expf(-lrow[ej]));
-  }
-  const float psel = warp_sum_f(pj);
-  __syncwarp();
-  for (int e = lane; e < E; e += 32)
-    lrow[e] = !sigmoid ? expf(lrow[e] - m) / s : (1.0f / (1.0f + expf(-lrow[e]))) / s;
-  if (lane < k) {
-    a.idx[(size_t)t * k + lane] = ej;
-    a.wts[(size_t)t * k + lane] = a.norm ? pj / psel : pj;
-    atomicAdd(&cnt[ej], 1);
-    sel[lane] = ej;
-  }
-  __syncwarp();
 }
 
 // EPT experts per thread (a round covers 8 EPT experts): 3 for up to 96 experts (two CTAs per SM),
@@ -579,24 +533,29 @@ __global__ void __launch_bounds__(RT_THREADS, EPT == RT_EPT ? 2 : 1) router_kern
   double *wn = (double *)(smem_raw + SL.wn);     // [E] upper bounds of |W_e|_2
   float *lg = (float *)(smem_raw + SL.lg);       // [RT_TM][E] logits, then probabilities
   float *keys = (float *)(smem_raw + SL.keys);   // [RT_TM][E] sigmoid keys
-  int *brw = (int *)(smem_raw + SL.byrank) + warp * 9;  // this warp's experts by rank
   int *cnt = (int *)(smem_raw + SL.cnt);
   double *xnorm = (double *)(smem_raw + SL.xnorm);
   unsigned *cmask = (unsigned *)(smem_raw + SL.cmask);  // [listed token][E/32]
-  int *s_sel = (int *)(smem_raw + SL.part);  // [RT_TM][8] selections; `part` is free after the screen
-  __shared__ int s_nflag, s_flag[RT_TM];
-  __shared__ unsigned long long s_wnmax;  // bits of nonnegative doubles / floats order as integers
-  __shared__ int s_offmax, s_bmax;
+  RouterMisc &M = *(RouterMisc *)(smem_raw + SL.misc);
+  int &s_nflag = M.nflag, *s_flag = M.flag;
+  unsigned long long &s_wnmax = M.wnmax;  // bits of nonnegative doubles / floats order as integers
+  int &s_offmax = M.offmax, &s_bmax = M.bmax;
+  unsigned &s_badtok = M.badtok, &s_proven = M.proven, *s_lmax = M.lmax;
+  // after the screen the per-warp partials are free: the selection's records live there
+  int *s_sel = (int *)(smem_raw + SL.part);                   // [RT_TM][8] final selections
+  int *s_by = s_sel + RT_TM * 8;                               // [RT_TM][9] experts by rank
+  double *s_bk = (double *)(smem_raw + SL.part + 1280);        // [RT_TM] key bounds
 
+  const KernelStamp stamp(K_ROUTER);
   griddep_wait();
+  stamp.started();
   griddep_launch();
   // ---- the CTA's token rows -> shared memory: one bulk copy per row, all in flight at once
   unsigned char *xs = smem_raw + SL.xs;
   const size_t xs_stride = SL.xs_stride;
   const uint32_t row_bytes = (uint32_t)d * (uint32_t)sizeof(Tin);
-  __shared__ __align__(8) uint64_t s_xbar;
-  __shared__ volatile int s_xabort;
-  const uint32_t xbar = smem_u32(&s_xbar);
+  volatile int &s_xabort = M.xabort;
+  const uint32_t xbar = smem_u32(&M.xbar);
   if (tid == 0) {
     mbar_init(xbar, 1);
     s_xabort = 0;
@@ -604,6 +563,11 @@ __global__ void __launch_bounds__(RT_THREADS, EPT == RT_EPT ? 2 : 1) router_kern
     s_offmax = 0;
     s_bmax = 0;
     s_nflag = 0;
+    s_badtok = 0u;
+    s_proven = 0u;
+  }
+  if (tid < RT_TM) {
+    s_lmax[tid] = 0u;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   __syncthreads();
@@ -793,55 +757,138 @@ __global__ void __launch_bounds__(RT_THREADS, EPT == RT_EPT ? 2 : 1) router_kern
     if (!sigmoid) return (double)l;
     return sigmoid64(l) + (a.bias ? (double)a.bias[e] : 0.0);
   };
-  // ---- selection, one warp per token. Tokens whose order the screen proves are finished here;
-  // the others are listed with their candidate experts, settled by the whole CTA below.
+  // Experts of rank 0..n-1 (descending key, NaN as -infinity, ties to the lower index) of the
+  // tokens in `tmask` into s_by[tt][0..n). Up to 64 experts a thread counts the rank of one
+  // (token, expert) pair; above, a warp per token takes the n largest in turn.
+  auto rank_tokens = [&](unsigned tmask, int n) {
+    const float *kb = sigmoid ? keys : lg;
+    if (E <= RT_SEL_THREAD_MAX_E) {
+      for (int q = tid; q < ntok * E; q += RT_THREADS) {
+        const int tt = q / E, e = q - tt * E;
+        if (!((tmask >> tt) & 1u)) continue;
+        const float *krow = kb + tt * E;
+        float v = krow[e];
+        if (v != v) v = -INFINITY;
+        int rank = 0;
+        for (int e2 = 0; e2 < E; ++e2) {
+          float v2 = krow[e2];
+          if (v2 != v2) v2 = -INFINITY;
+          rank += (v2 > v || (v2 == v && e2 < e)) ? 1 : 0;
+        }
+        if (rank < n) s_by[tt * 9 + rank] = e;
+      }
+    } else {
+      for (int tt = warp; tt < ntok; tt += RT_WARPS) {
+        if (!((tmask >> tt) & 1u)) continue;
+        int sel[9];
+        warp_topn(kb + tt * E, E, n, sel);
+#pragma unroll
+        for (int j = 0; j < 9; ++j)
+          if (j < n && lane == 0) s_by[tt * 9 + j] = sel[j];
+      }
+    }
+  };
+  // Probabilities, combine weights and outputs of every token, fixed-order trees; the logits row
+  // becomes the probability basis of the load-balancing statistics. Up to 64 experts 16 threads
+  // (a half-warp) take a token, all 16 tokens at once; above, a warp per token.
+  auto finish_tokens = [&]() {
+    const int G = E <= RT_SEL_THREAD_MAX_E ? 16 : 32;  // threads per token
+    const unsigned gmask = G == 16 ? 0xFFFFu << (lane & 16) : 0xFFFFFFFFu;
+    const int sub = tid & (G - 1);
+    for (int tt = tid / G; tt < ntok; tt += RT_THREADS / G) {  // whole groups
+      float *lrow = lg + tt * E;
+      float m = -INFINITY, sum = 0.0f;
+      if (!sigmoid) {
+        for (int e = sub; e < E; e += G) m = fmaxf(m, lrow[e]);
+        for (int o = G / 2; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(gmask, m, o));
+        for (int e = sub; e < E; e += G) sum += expf(lrow[e] - m);
+      } else {
+        for (int e = sub; e < E; e += G) sum += 1.0f / (1.0f + expf(-lrow[e]));
+      }
+      for (int o = G / 2; o > 0; o >>= 1) sum += __shfl_xor_sync(gmask, sum, o);
+      int ej = 0;
+      float pj = 0.0f;
+      if (sub < k) {
+        ej = s_by[tt * 9 + sub];
+        pj = !sigmoid ? expf(lrow[ej] - m) / sum : 1.0f / (1.0f + expf(-lrow[ej]));
+      }
+      float psel = pj;
+      for (int o = G / 2; o > 0; o >>= 1) psel += __shfl_xor_sync(gmask, psel, o);
+      __syncwarp(gmask);  // every read of the logits row precedes its overwrite
+      for (int e = sub; e < E; e += G)
+        lrow[e] = !sigmoid ? expf(lrow[e] - m) / sum : (1.0f / (1.0f + expf(-lrow[e]))) / sum;
+      if (sub < k) {
+        const size_t o = (size_t)(t0 + tt) * k + sub;
+        a.idx[o] = ej;
+        a.wts[o] = a.norm ? pj / psel : pj;
+        atomicAdd(&cnt[ej], 1);
+        s_sel[tt * 8 + sub] = ej;
+      }
+    }
+  };
+  // ---- selection in block-wide phases over the CTA's tokens (a token's order is proven from
+  // the screen, or its candidate experts are listed and settled exactly by the whole CTA below)
   const double mg = (double)(4 * ((nch + 15) / 16) + 10);  // roundings per term of the screen
   const double gam = mg * 0x1p-24 / (1.0 - mg * 0x1p-24);
   const double wmax = __longlong_as_double((long long)s_wnmax);
   const double omax = (double)__int_as_float(s_offmax), bmax = (double)__int_as_float(s_bmax);
   const int nmw = (E + 31) >> 5;  // candidate mask words per token
-  for (int tt = warp; tt < ntok; tt += RT_WARPS) {
-    float *lrow = lg + tt * E;
-    float *krow = sigmoid ? keys + tt * E : lrow;
-    bool bad = false;
-    float lmax = 0.0f;
-    for (int e = lane; e < E; e += 32) {
-      const float l = lrow[e];
-      bad |= !isfinite(l);
-      lmax = fmaxf(lmax, fabsf(l));
-      if (sigmoid) krow[e] = (float)key_of(tt, e);
+  // (a) sigmoid keys from the screened logits; per token: any non-finite logit, max |l|
+  for (int q = tid; q < ntok * E; q += RT_THREADS) {
+    const int tt = q / E, e = q - tt * E;
+    const float l = lg[q];
+    if (!isfinite(l)) atomicOr(&s_badtok, 1u << tt);
+    if (sigmoid) {
+      keys[q] = (float)key_of(tt, e);
+      atomicMax(&s_lmax[tt], __float_as_uint(fabsf(l)));
     }
-    bad = __any_sync(0xffffffffu, bad);
-    lmax = warp_max_f(lmax);
-    // Bound of the token's keys. Screen: |l~ - S| <= gamma_m (|x_t| max_e |W_e| + max |off|) for
-    // the exact sum S of every expert (m roundings per term, plus m 2^-149 for underflow).
-    // Sigmoid: the key comes from the canonical (rounded) logit, within that plus half an fp32
-    // step of l~; sigmoid is 1/4-Lipschitz, and its fp64 evaluation plus the bias add err by less
-    // than 2^-47 + 2^-51 |b|.
-    double Bk = gam * (xnorm[tt] * wmax + omax) * (1.0 + 0x1p-40) + mg * 0x1p-149;
-    if (sigmoid) Bk = 0.25 * (Bk + 0x1p-24 * ((double)lmax + Bk) + 0x1p-149) + 0x1p-47 + 0x1p-51 * bmax;
-    __syncwarp();
-    warp_rank_into(krow, E, min(k + 1, E), brw);
-    __syncwarp();
-    // the proof: each of the J gaps between consecutive approximate ranks exceeds twice the key
-    // bound plus two fp32 steps at that magnitude (lane j checks gap j)
-    const int J = min(k, E - 1);
+  }
+  __syncthreads();
+  // (b) experts of approximate ranks 0..k of every token
+  rank_tokens((1u << ntok) - 1u, min(k + 1, E));
+  __syncthreads();
+  // (c) the proof, 8 threads per token: each of the J gaps between consecutive approximate ranks
+  // must exceed twice the key bound plus two fp32 steps at that magnitude (thread j checks gap j)
+  if (tid < RT_TM * 8) {  // warps 0-3, whole
+    const int tt = tid >> 3, j = tid & 7;
     bool ok = true;
-    if (lane < J) {
-      const double prev = key_of(tt, brw[lane]), cur = key_of(tt, brw[lane + 1]);
-      ok = prev - cur > 2.0 * Bk + 0x1p-22 * (fmax(fabs(prev), fabs(cur)) + Bk) + 0x1p-148;
+    double Bk = 0.0;
+    if (tt < ntok) {
+      // Bound of the token's keys. Screen: |l~ - S| <= gamma_m (|x_t| max_e |W_e| + max |off|)
+      // for the exact sum S of every expert (m roundings per term, plus m 2^-149 for
+      // underflow). Sigmoid: the key comes from the canonical (rounded) logit, within that plus
+      // half an fp32 step of l~; sigmoid is 1/4-Lipschitz, and its fp64 evaluation plus the bias
+      // add err by less than 2^-47 + 2^-51 |b|.
+      Bk = gam * (xnorm[tt] * wmax + omax) * (1.0 + 0x1p-40) + mg * 0x1p-149;
+      if (sigmoid) {
+        const double lmax = (double)__uint_as_float(s_lmax[tt]);
+        Bk = 0.25 * (Bk + 0x1p-24 * (lmax + Bk) + 0x1p-149) + 0x1p-47 + 0x1p-51 * bmax;
+      }
+      if (j < min(k, E - 1)) {
+        const int *br = s_by + tt * 9;
+        const double prev = key_of(tt, br[j]), cur = key_of(tt, br[j + 1]);
+        ok = prev - cur > 2.0 * Bk + 0x1p-22 * (fmax(fabs(prev), fabs(cur)) + Bk) + 0x1p-148;
+      }
     }
-    const bool proven = __all_sync(0xffffffffu, ok) && !bad && !force && Bk < INFINITY;
-    if (proven) {
-      finish_token(a, lrow, brw, t0 + tt, cnt, s_sel + tt * 8);
-      continue;
+    const unsigned fails = __ballot_sync(0xffffffffu, !ok);
+    if (j == 0 && tt < ntok) {
+      s_bk[tt] = Bk;
+      const bool bad = (s_badtok >> tt) & 1u;
+      if (((fails >> (lane & 24)) & 0xFFu) == 0u && !bad && !force && Bk < INFINITY)
+        atomicOr(&s_proven, 1u << tt);
     }
-    // candidates: every expert whose key is not provably below the (k+1)-th approximate key
-    // (all of them when the bound is unusable or k = E)
+  }
+  __syncthreads();
+  // (d) the unproven tokens' candidates: every expert whose key is not provably below the
+  // (k+1)-th approximate key (all of them when the bound is unusable or k = E); a warp per token
+  for (int tt = warp; tt < ntok; tt += RT_WARPS) {
+    if ((s_proven >> tt) & 1u) continue;
+    const double Bk = s_bk[tt];
+    const bool bad = (s_badtok >> tt) & 1u;
     const bool all = force || bad || E <= k || !(Bk < INFINITY);
     double cut = -INFINITY;
     if (!all) {
-      const double vk = key_of(tt, brw[k]);
+      const double vk = key_of(tt, s_by[tt * 9 + k]);
       cut = vk - 2.0 * Bk - 0x1p-22 * (fabs(vk) + Bk) - 0x1p-148;
     }
     int f = 0;
@@ -947,14 +994,14 @@ __global__ void __launch_bounds__(RT_THREADS, EPT == RT_EPT ? 2 : 1) router_kern
       }
     }
     __syncthreads();
-    // the listed tokens, ranked again on their canonical candidate keys, then finished
-    for (int f = warp; f < nflag; f += RT_WARPS) {
-      const int tt = s_flag[f];
-      warp_rank_into((sigmoid ? keys : lg) + tt * E, E, k, brw);
-      __syncwarp();
-      finish_token(a, lg + tt * E, brw, t0 + tt, cnt, s_sel + tt * 8);
-    }
+    // the listed tokens, ranked again on their canonical candidate keys
+    unsigned fm = 0u;
+    for (int f = 0; f < nflag; ++f) fm |= 1u << s_flag[f];
+    rank_tokens(fm, k);
   }
+  __syncthreads();
+  // (e) probabilities, combine weights and outputs of every token, 16 threads per token
+  finish_tokens();
   __syncthreads();
 
   // ---- within-chunk ranks: pair (tt, j) counts the earlier tokens of the CTA that selected the

@@ -26,7 +26,9 @@ struct StatsArgs {
 };
 
 __global__ void __launch_bounds__(ST_THREADS) moe_stats_kernel(StatsArgs a) {
+  const KernelStamp stamp(K_STATS);
   griddep_wait();
+  stamp.started();
   griddep_launch();
   const int e = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int E = a.E;

@@ -275,15 +275,26 @@ moe_status_t moe_get_device_error(void *stream, int64_t *info);
  *     the floating-point expansion rather than the exact integer sum (for parity tests);
  *   MOE_DEBUG_WAIT_LIMIT_NS: upper bound on any device-side wait (default 2e9 ns);
  *   MOE_DEBUG_PROFILE: 1 = record a CUDA event pair around every kernel the library launches,
- *     per kernel kind, read with moe_profile_read(). */
-typedef enum { MOE_DEBUG_FORCE_EXACT = 1, MOE_DEBUG_WAIT_LIMIT_NS = 2, MOE_DEBUG_PROFILE = 3 }
-    moe_debug_t;
+ *     per kernel kind, read with moe_profile_read(). The events end the overlap of a kernel with
+ *     its predecessor's tail, so a short kernel reads longer than it runs inside a layer call;
+ *   MOE_DEBUG_STAMP: 1 = every forward kernel records, on the device's global timer, when its
+ *     first CTA's inputs became final and when its last warp finished, per kernel kind, read with
+ *     moe_stamp_read(); the launches stay overlapped as in normal operation. */
+typedef enum { MOE_DEBUG_FORCE_EXACT = 1, MOE_DEBUG_WAIT_LIMIT_NS = 2, MOE_DEBUG_PROFILE = 3,
+               MOE_DEBUG_STAMP = 4 } moe_debug_t;
 moe_status_t moe_debug_set(int32_t what, int64_t value);
 
 /* Kernel-level timing collected while MOE_DEBUG_PROFILE is on. Synchronises the device.
  * Fills up to `max` entries: names[i] (static strings), total_ms[i] and launches[i]; returns
  * the number of kernel kinds with at least one launch, and resets the accumulators. */
 int32_t moe_profile_read(const char **names, double *total_ms, int64_t *launches, int32_t max);
+
+/* In-step kernel durations recorded while MOE_DEBUG_STAMP is on: per kernel kind that ran since
+ * the last read, the time from its first CTA's inputs becoming final to its last warp's end, in
+ * microseconds (several launches of one kind in that interval count as one span). Synchronises
+ * the device, fills up to `max` entries of names[i] (static strings) and us[i], returns the
+ * number of kinds (or -1 on a CUDA error) and clears the records. */
+int32_t moe_stamp_read(const char **names, double *us, int32_t max);
 
 /* Test hook for failure detection: launches one tiny kernel that waits on a shared-memory
  * barrier nothing will complete, bounded by MOE_DEBUG_WAIT_LIMIT_NS; the kernel then records

@@ -377,6 +377,32 @@ def test_bitwise_determinism():
     assert torch.equal(y1, y2) and float(a1) == float(a2)
 
 
+def test_in_step_stamps():
+    """With MOE_DEBUG_STAMP on, one layer call leaves a positive duration for each forward kernel
+    kind it launched, each within the call's own event span; with it off nothing is recorded."""
+    c = SMALL["quartz_s"]
+    run = LayerOnGpu(c, make_inputs(c))
+    y_ref, _, _ = run.layer()
+    y_ref = y_ref.clone()
+    B.moe_debug_set(B.DEBUG_STAMP, 1)
+    try:
+        B.moe_stamp_read()
+        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ev0.record()
+        y, _, _ = run.layer()
+        ev1.record()
+        torch.cuda.synchronize()
+        span_us = ev0.elapsed_time(ev1) * 1e3
+        st = B.moe_stamp_read()
+    finally:
+        B.moe_debug_set(B.DEBUG_STAMP, 0)
+    assert torch.equal(y, y_ref)  # stamping changes no result
+    for n in ("router", "stats", "perm_scatter", "gemm_gateup", "gemm_down", "combine"):
+        assert n in st and 0.0 < st[n] <= span_us, (n, st, span_us)
+    run.layer()
+    assert B.moe_stamp_read() == {}
+
+
 def test_bounded_wait_times_out_cleanly():
     """A wait on a barrier that nothing completes ends with MOE_ERR_TIMEOUT; the context stays
     usable for the next call."""
