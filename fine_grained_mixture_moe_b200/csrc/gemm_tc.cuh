@@ -1,7 +1,7 @@
 // bf16 grouped expert GEMM on the 5th-generation tensor cores (sm_100a), single-SM form.
 //
-// It serves the low-rank V projection (SCALE) and down projections whose width is not a multiple
-// of 256 (PLAIN). The SwiGLU gate/up product and the other down projections run on CTA pairs
+// It serves the low-rank V projection (SCALE, N = rank); the PLAIN form is kept for narrow
+// outputs. The SwiGLU gate/up product and the down and low-rank U projections run on CTA pairs
 // (gemm_tc2.cuh), which share this file's PTX wrappers, tensor maps and epilogue conventions.
 //
 // One persistent CTA per SM walks a device-side tile list built from the group offsets

@@ -349,14 +349,15 @@ moe_status_t launch_simt(const GroupedGemm &g, cudaStream_t st, int kind) {
   return launch_pdl(kern, dim3(grid), dim3(256), smem, st, gk);
 }
 
+// bf16: gate/up and plain products on CTA pairs (256 x 256 tiles; an output width that is not a
+// multiple of 256 leaves the last column tile partly outside the expert, whose columns the
+// epilogue does not store), the low-rank projection on single SMs (N = rank).
 template <int MODE>
-moe_status_t launch_gemm(const moe_config_t *c, const GroupedGemm &g, int bn_hint,
-                         cudaStream_t st, int kind) {
+moe_status_t launch_gemm(const moe_config_t *c, const GroupedGemm &g, cudaStream_t st,
+                         int kind) {
   if (c->dtype == MOE_DTYPE_F32) return launch_simt<MODE>(g, st, kind);
-  if (MODE == MODE_GATEUP) return launch_tc2<MODE_GATEUP>(g, st, kind);
   if (MODE == MODE_SCALE) return launch_tc<MODE_SCALE, 64>(g, st, kind);
-  if (bn_hint == 256) return launch_tc2<MODE_PLAIN>(g, st, kind);
-  return launch_tc<MODE_PLAIN, 128>(g, st, kind);
+  return launch_tc2<MODE == MODE_GATEUP ? MODE_GATEUP : MODE_PLAIN>(g, st, kind);
 }
 
 // ------------------------------------------------------------------ steps
@@ -493,7 +494,6 @@ moe_status_t experts_impl(const moe_config_t *c, const void *x_perm, const int32
   g.T = T;
   g.rows_r = T * k;
   const bool sh = S > 0;
-  const int bn_down = (d % 256 == 0) ? 256 : 128;
   if (c->expert == MOE_EXPERT_SWIGLU) {
     const int f = c->ffn;
     GroupedGemm g1 = g;
@@ -505,7 +505,7 @@ moe_status_t experts_impl(const moe_config_t *c, const void *x_perm, const int32
       g1.N_s = S * fs; g1.K_s = d; g1.piece_k = d; g1.piece_rows = 0; g1.b_rows_s = S * fs;
       g1.out_s = Hs; g1.ldo_s = S * fs;
     }
-    MOE_TRY(launch_gemm<MODE_GATEUP>(c, g1, 128, st, K_GEMM_GATEUP));
+    MOE_TRY(launch_gemm<MODE_GATEUP>(c, g1, st, K_GEMM_GATEUP));
     GroupedGemm g2 = g;
     g2.E = E; g2.A_r = H; g2.lda_r = f; g2.B0_r = w->w_down; g2.N_r = d; g2.K_r = f;
     g2.out_r = y_perm; g2.ldo_r = d; g2.out_r_bf16 = yperm_bf16(c) ? 1 : 0;
@@ -514,7 +514,7 @@ moe_status_t experts_impl(const moe_config_t *c, const void *x_perm, const int32
       g2.A_s = Hs; g2.lda_s = S * fs; g2.B0_s = w->ws_down; g2.N_s = d; g2.K_s = S * fs;
       g2.piece_k = fs; g2.piece_rows = d; g2.b_rows_s = S * d; g2.out_s = y_shared; g2.ldo_s = d;
     }
-    return launch_gemm<MODE_PLAIN>(c, g2, bn_down, st, K_GEMM_DOWN);
+    return launch_gemm<MODE_PLAIN>(c, g2, st, K_GEMM_DOWN);
   }
   // low-rank experts: Z = (X V^T) * s, then Y = Z U^T. In bf16, Z is kept as two bf16 terms
   // [Z_hi | Z_lo] (Z_lo = the rounding residual), and the second product runs over K = 2r with
@@ -525,24 +525,24 @@ moe_status_t experts_impl(const moe_config_t *c, const void *x_perm, const int32
   GroupedGemm g1 = g;
   g1.E = E; g1.A_r = x_perm; g1.lda_r = d; g1.B0_r = w->lr_V; g1.N_r = r; g1.K_r = d;
   g1.out_r = H; g1.ldo_r = split ? 2 * r : r; g1.scale = w->lr_s; g1.lo_split = split ? r : 0;
-  MOE_TRY(launch_gemm<MODE_SCALE>(c, g1, 64, st, K_GEMM_LR1));
+  MOE_TRY(launch_gemm<MODE_SCALE>(c, g1, st, K_GEMM_LR1));
   GroupedGemm g2 = g;
   g2.E = E; g2.A_r = H; g2.lda_r = split ? 2 * r : r; g2.B0_r = w->lr_U; g2.N_r = d;
   g2.K_r = split ? 2 * r : r; g2.kb_r = split ? r : 0;
   g2.out_r = y_perm; g2.ldo_r = d; g2.out_r_bf16 = yperm_bf16(c) ? 1 : 0;
-  MOE_TRY(launch_gemm<MODE_PLAIN>(c, g2, bn_down, st, K_GEMM_LR2));
+  MOE_TRY(launch_gemm<MODE_PLAIN>(c, g2, st, K_GEMM_LR2));
   if (sh) {
     GroupedGemm g3 = g;
     g3.E = 0; g3.has_shared = 1;
     g3.A_s = x; g3.lda_s = d; g3.B0_s = w->ws_gate; g3.B1_s = w->ws_up;
     g3.N_s = S * fs; g3.K_s = d; g3.piece_k = d; g3.piece_rows = 0; g3.b_rows_s = S * fs;
     g3.out_s = Hs; g3.ldo_s = S * fs;
-    MOE_TRY(launch_gemm<MODE_GATEUP>(c, g3, 128, st, K_GEMM_GATEUP));
+    MOE_TRY(launch_gemm<MODE_GATEUP>(c, g3, st, K_GEMM_GATEUP));
     GroupedGemm g4 = g;
     g4.E = 0; g4.has_shared = 1;
     g4.A_s = Hs; g4.lda_s = S * fs; g4.B0_s = w->ws_down; g4.N_s = d; g4.K_s = S * fs;
     g4.piece_k = fs; g4.piece_rows = d; g4.b_rows_s = S * d; g4.out_s = y_shared; g4.ldo_s = d;
-    MOE_TRY(launch_gemm<MODE_PLAIN>(c, g4, bn_down, st, K_GEMM_DOWN));
+    MOE_TRY(launch_gemm<MODE_PLAIN>(c, g4, st, K_GEMM_DOWN));
   }
   return MOE_OK;
 }
