@@ -10,6 +10,7 @@ from .binding import (DEBUG_FORCE_EXACT, DEBUG_PROFILE, DEBUG_WAIT_LIMIT_NS, EXP
                       MoEConfig, MoEError, MoEWeights, load, make_config, make_weights,
                       moe_aux_loss, moe_bias_update, moe_capacity, moe_combine,
                       moe_combine_backward, moe_debug_set, moe_route_backward,
+                      moe_expert_backward, moe_backward_workspace_size, make_grads,
                       moe_debug_wait_timeout_probe, moe_expert_forward, moe_get_device_error,
                       moe_layer_forward, moe_permute, moe_profile_read, moe_route,
                       moe_route_noalloc, moe_workspace_size, status_str)

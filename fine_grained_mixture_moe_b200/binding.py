@@ -45,6 +45,20 @@ class MoEWeights(ctypes.Structure):
                                         "ws_up", "ws_down")]
 
 
+class MoEGrads(ctypes.Structure):
+    _fields_ = [(n, c_void_p) for n in ("d_w_gate", "d_w_up", "d_w_down", "d_lr_V", "d_lr_s",
+                                        "d_lr_U", "d_ws_gate", "d_ws_up", "d_ws_down")]
+
+
+def make_grads(tensors: Dict[str, object]) -> "MoEGrads":
+    """moe_grads_t from a dict name -> tensor (names of MoEGrads' fields; missing ones NULL)."""
+    g = MoEGrads()
+    for name, _ in MoEGrads._fields_:
+        if tensors.get(name) is not None:
+            setattr(g, name, _ptr(tensors[name]))
+    return g
+
+
 _lib: Optional[ctypes.CDLL] = None
 
 
@@ -90,6 +104,10 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
         "moe_profile_read": (c_int32, [P(ctypes.c_char_p), P(ctypes.c_double), P(c_int64),
                                        c_int32]),
         "moe_stamp_read": (c_int32, [P(ctypes.c_char_p), P(ctypes.c_double), c_int32]),
+        "moe_backward_workspace_size": (c_size_t, [P(MoEConfig)]),
+        "moe_expert_backward": (c_int32, [P(MoEConfig), c_void_p, c_void_p, c_void_p, c_void_p,
+                                          P(MoEWeights), c_void_p, c_void_p, c_void_p,
+                                          P(MoEGrads), c_void_p, c_size_t, c_void_p]),
         "moe_debug_wait_timeout_probe": (c_int32, [c_void_p]),
         "moe_route_noalloc": (c_int32, [P(MoEConfig), c_void_p, P(MoEWeights), c_void_p,
                                         c_void_p, c_void_p, c_void_p, c_void_p]),
@@ -104,7 +122,8 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
 
 EXPORTED = ("moe_workspace_size", "moe_capacity", "moe_route", "moe_permute",
             "moe_expert_forward", "moe_combine", "moe_aux_loss", "moe_bias_update",
-            "moe_combine_backward", "moe_route_backward",
+            "moe_combine_backward", "moe_route_backward", "moe_backward_workspace_size",
+            "moe_expert_backward",
             "moe_layer_forward",
             "moe_status_str", "moe_get_device_error", "moe_debug_set", "moe_profile_read",
             "moe_stamp_read", "moe_debug_wait_timeout_probe", "moe_route_noalloc")
@@ -245,6 +264,19 @@ def moe_profile_read(max_kinds: int = 32):
     n = (c_int64 * max_kinds)()
     cnt = load().moe_profile_read(names, ms, n, max_kinds)
     return {names[i].decode(): (ms[i], int(n[i])) for i in range(min(cnt, max_kinds))}
+
+
+def moe_backward_workspace_size(cfg) -> int:
+    return int(load().moe_backward_workspace_size(ctypes.byref(cfg)))
+
+
+def moe_expert_backward(cfg, x_perm, offsets, slot_pos, x, w: MoEWeights, dy_perm, dy, dx,
+                        grads: MoEGrads, ws, ws_bytes: int, stream=None) -> None:
+    _check("moe_expert_backward",
+           load().moe_expert_backward(ctypes.byref(cfg), _ptr(x_perm), _ptr(offsets),
+                                      _ptr(slot_pos), _ptr(x), ctypes.byref(w), _ptr(dy_perm),
+                                      _ptr(dy), _ptr(dx), ctypes.byref(grads), _ptr(ws),
+                                      ws_bytes, _stream(stream)))
 
 
 def moe_stamp_read(max_kinds: int = 32):

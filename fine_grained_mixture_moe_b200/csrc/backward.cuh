@@ -249,4 +249,137 @@ __global__ void __launch_bounds__(256) router_dgrad_kernel(const float *__restri
   }
 }
 
+
+// ------------------------------------------------------------------ expert steps of the backward
+// The weight gradients are products over a group's rows (dW_d[e] = dY_e^T h_e, dW_g[e] =
+// dg_e^T X_e, dW_u[e] = du_e^T X_e). The tensor cores take both operands K-major, so the grouped
+// activations are transposed first, each expert's rows padded with zeros to a multiple of 64 so
+// that no 64-wide k-block crosses into the next expert; the weights are transposed for the data
+// gradients (dh = dY W_d, dX = [dg | du] [W_g; W_u]) the same way.
+
+// koff[e] = sum over e' < e of the expert's row count rounded up to 64; koff[E] is the total.
+// Also the one-group tables of the shared experts' T rows: off_s = {0, T}, koff_s = {0, T
+// rounded up to 64}. One block; E <= 1024.
+__global__ void __launch_bounds__(1024) pad_offsets_kernel(const int32_t *__restrict__ offsets,
+                                                           int E, int32_t *__restrict__ koff,
+                                                           int T, int32_t *__restrict__ off_s,
+                                                           int32_t *__restrict__ koff_s) {
+  griddep_wait();
+  griddep_launch();
+  __shared__ int s[1024];
+  __shared__ int tmp[1024 / 32 + 1];
+  const int e = threadIdx.x;
+  s[e] = e < E ? ((offsets[e + 1] - offsets[e] + 63) & ~63) : 0;
+  __syncthreads();
+  const int total = block_excl_scan_inplace(s, 1024, tmp);
+  if (e < E) koff[e] = s[e];
+  if (e == 0) {
+    koff[E] = total;
+    off_s[0] = 0;
+    off_s[1] = T;
+    koff_s[0] = 0;
+    koff_s[1] = (T + 63) & ~63;
+  }
+}
+
+// Tiled transpose to bf16 through shared memory, 64 x 64 per CTA:
+//   grouped (in_offsets != null): group g's rows offsets[g] .. offsets[g+1] of the sources
+//     [rows, C] (row stride ldi) go to nseg segments of columns of out [C, ldo]: segment s
+//     spans columns nseg koff[g] + s P .. + P, P = koff[g+1] - koff[g] (the group's row count
+//     rounded up to 64), and holds the rows of source s, zeros past the group's rows
+//     (blockIdx.y runs over 64-column blocks of out, blockIdx.z = 0);
+//   dense: batch b = blockIdx.z, in0 + b * ibs is [R, C] (row stride ldi) and goes to
+//     out + b * obs + col0 as [C, R] with row stride ldo; blockIdx.y runs over 64-row blocks.
+template <typename Tin>
+__global__ void __launch_bounds__(256) transpose_bf16_kernel(
+    const Tin *__restrict__ in0, const Tin *__restrict__ in1, const Tin *__restrict__ in2,
+    int nseg, int C, int ldi, const int32_t *__restrict__ in_offsets,
+    const int32_t *__restrict__ koff, int G, int R, size_t ibs, __nv_bfloat16 *__restrict__ out,
+    int ldo, size_t obs, int col0) {
+  griddep_wait();
+  griddep_launch();
+  __shared__ float tile[64][65];
+  const int c0 = blockIdx.x * 64;
+  int r_in0, n_rows, o_col0;  // first input row, valid rows of the block, first output column
+  const Tin *src = in0;
+  __nv_bfloat16 *dst = out;
+  if (in_offsets) {
+    const int p0 = blockIdx.y * 64;  // column block of out
+    if (p0 >= nseg * koff[G]) return;
+    int lo = 0, hi = G - 1;          // group with nseg koff[g] <= p0 < nseg koff[g+1]
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (nseg * koff[mid] <= p0) lo = mid;
+      else hi = mid - 1;
+    }
+    const int P = koff[lo + 1] - koff[lo];
+    const int local = p0 - nseg * koff[lo];
+    const int seg = local / P, lr = local - seg * P;
+    src = seg == 0 ? in0 : (seg == 1 ? in1 : in2);
+    r_in0 = in_offsets[lo] + lr;
+    n_rows = max(0, min(64, in_offsets[lo + 1] - in_offsets[lo] - lr));
+    o_col0 = p0;
+  } else {
+    src += (size_t)blockIdx.z * ibs;
+    dst += (size_t)blockIdx.z * obs + col0;
+    r_in0 = blockIdx.y * 64;
+    n_rows = max(0, min(64, R - r_in0));
+    o_col0 = r_in0;
+  }
+  const int tx = threadIdx.x & 63, ty = threadIdx.x >> 6;  // 64 x 4
+  for (int r = ty; r < 64; r += 4) {
+    float v = 0.0f;
+    if (r < n_rows && c0 + tx < C) v = Elem<Tin>::to_f(src[(size_t)(r_in0 + r) * ldi + c0 + tx]);
+    tile[r][tx] = v;
+  }
+  __syncthreads();
+  const int n_out = in_offsets ? 64 : n_rows;  // grouped: the padding columns are written too
+  for (int c = ty; c < 64; c += 4)
+    if (c0 + c < C && tx < n_out)
+      dst[(size_t)(c0 + c) * ldo + o_col0 + tx] = __float2bfloat16_rn(tile[tx][c]);
+}
+
+// Rows of in [rows, d] (fp32) as two bf16 terms: out[r] = [hi (d) | lo (d)], hi = bf16(v),
+// lo = bf16(v - hi); d a multiple of 4.
+__global__ void __launch_bounds__(256) split_bf16_kernel(const float *__restrict__ in, int d,
+                                                         size_t rows, __nv_bfloat16 *__restrict__ out) {
+  griddep_wait();
+  griddep_launch();
+  const size_t n = rows * (size_t)d;
+  for (size_t i = ((size_t)blockIdx.x * 256 + threadIdx.x) * 4; i < n; i += (size_t)gridDim.x * 1024) {
+    const float4 v = *(const float4 *)(in + i);
+    const size_t r = i / d, c = i - r * d;
+    const __nv_bfloat162 a = __floats2bfloat162_rn(v.x, v.y), b = __floats2bfloat162_rn(v.z, v.w);
+    const float2 af = __bfloat1622float2(a), bf = __bfloat1622float2(b);
+    const __nv_bfloat162 al = __floats2bfloat162_rn(v.x - af.x, v.y - af.y);
+    const __nv_bfloat162 bl = __floats2bfloat162_rn(v.z - bf.x, v.w - bf.y);
+    uint2 hi, lo;
+    hi.x = *(const uint32_t *)&a;
+    hi.y = *(const uint32_t *)&b;
+    lo.x = *(const uint32_t *)&al;
+    lo.y = *(const uint32_t *)&bl;
+    *(uint2 *)(out + r * 2 * d + c) = hi;
+    *(uint2 *)(out + r * 2 * d + d + c) = lo;
+  }
+}
+
+// Zero the gradient slices of experts that received no rows (their weight-gradient products
+// have no tiles): up to three arrays with `per` floats per expert each.
+__global__ void __launch_bounds__(256) zero_empty_experts_kernel(
+    const int32_t *__restrict__ offsets, float *__restrict__ a, size_t pa, float *__restrict__ b,
+    size_t pb, float *__restrict__ c, size_t pc) {
+  griddep_wait();
+  griddep_launch();
+  const int e = blockIdx.x;
+  if (offsets[e + 1] != offsets[e]) return;
+  for (size_t i = (size_t)blockIdx.y * 256 + threadIdx.x; i < pa; i += (size_t)gridDim.y * 256)
+    a[(size_t)e * pa + i] = 0.0f;
+  if (b)
+    for (size_t i = (size_t)blockIdx.y * 256 + threadIdx.x; i < pb; i += (size_t)gridDim.y * 256)
+      b[(size_t)e * pb + i] = 0.0f;
+  if (c)
+    for (size_t i = (size_t)blockIdx.y * 256 + threadIdx.x; i < pc; i += (size_t)gridDim.y * 256)
+      c[(size_t)e * pc + i] = 0.0f;
+}
+
 }  // namespace moe

@@ -70,7 +70,7 @@ __global__ void __launch_bounds__(256, sizeof(Ty) == 2 ? 4 : 3) combine_kernel(c
   float w_l = 0.0f;
   if (t < T && lane < k) {
     pos_l = __ldcg(slot_pos + (size_t)t * k + lane);
-    w_l = __ldcg(w + (size_t)t * k + lane);
+    w_l = w ? __ldcg(w + (size_t)t * k + lane) : 1.0f;  // no weights: the plain sum (un-permute)
   }
   if (early) griddep_wait();
   stamp.started();

@@ -60,9 +60,16 @@ __device__ __forceinline__ void mbar_arrive_cta0(uint32_t bar_local) {
       : "memory");
 }
 
+// Modes whose B tile is two weights (gate rows in CTA 0, up rows in CTA 1).
+__host__ __device__ constexpr bool tc2_two_b(int mode) {
+  return mode == MODE_GATEUP || mode == MODE_GATEUP_RAW;
+}
+
 template <int MODE> struct Tc2Cfg {
-  static_assert(MODE == MODE_GATEUP || MODE == MODE_PLAIN, "pair kernel modes");
-  static constexpr int BN = MODE == MODE_GATEUP ? 128 : 256;  // output columns per tile
+  static_assert(MODE == MODE_GATEUP || MODE == MODE_PLAIN || MODE == MODE_GATEUP_RAW ||
+                    MODE == MODE_SWIGLU_BWD,
+                "pair kernel modes");
+  static constexpr int BN = tc2_two_b(MODE) ? 128 : 256;  // output columns per tile
   static constexpr int MMA_N = 256;                           // accumulator columns
   static constexpr int A_BYTES = 128 * TC_BK * 2;             // this CTA's 128 rows
   static constexpr int B_BYTES = 128 * TC_BK * 2;             // this CTA's half of B
@@ -167,7 +174,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TC_THREADS, 1)
         const TileInfo ti = decode_tile(p, tile, prefix, TC2_BM, BN);
         const bool routed = ti.g < p.E;
         const CUtensorMap *ma = routed ? &P.maps.a_r : &P.maps.a_s;
-        const CUtensorMap *mb = (MODE == MODE_GATEUP && rank == 1)
+        const CUtensorMap *mb = (tc2_two_b(MODE) && rank == 1)
                                     ? (routed ? &P.maps.b1_r : &P.maps.b1_s)
                                     : (routed ? &P.maps.b0_r : &P.maps.b0_s);
         const int a_row = ti.a_row0 + ti.m0 + (int)rank * 128;
@@ -177,7 +184,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TC_THREADS, 1)
         // the smaller byte count. Both CTAs decide it from the same tile record.
         const bool a1_void = ti.m0 + 128 >= ti.rows;
         const uint32_t stage_tx = 2 * C::STAGE_BYTES - (a1_void ? C::A_BYTES : 0);
-        const int n_off = MODE == MODE_GATEUP ? 0 : (int)rank * 128;
+        const int n_off = tc2_two_b(MODE) ? 0 : (int)rank * 128;
         const int nk = ti.K / TC_BK;
         for (int kb = 0; kb < nk; ++kb) {
           if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, limit, INFO_WAIT_MMA_EMPTY)) {
@@ -189,7 +196,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TC_THREADS, 1)
           if (rank == 0) mbar_expect_tx(full_bar(stage), stage_tx);
           const int kk = kb * TC_BK;
           int b_row, b_col;
-          if (routed) {
+          if (p.kgroup) {  // one A and one B for all groups, each group its own K columns
+            b_row = ti.n0 + n_off;
+            b_col = ti.kofs + kk;
+          } else if (routed) {
             b_row = ti.g * ti.N + ti.n0 + n_off;
             b_col = p.kb_r ? kk % p.kb_r : kk;
           } else {
@@ -197,7 +207,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TC_THREADS, 1)
             b_row = piece * p.piece_rows + ti.n0 + n_off;
             b_col = kk - piece * p.piece_k;
           }
-          if (rank == 0 || !a1_void) tma_load_2d_pair(sA, ma, kk, a_row, full_bar(stage));
+          if (rank == 0 || !a1_void) tma_load_2d_pair(sA, ma, ti.kofs + kk, a_row, full_bar(stage));
           tma_load_2d_pair(sB, mb, b_col, b_row, full_bar(stage));
           issued[stage] = true;
           issued_parity[stage] = (int)phase;
@@ -284,6 +294,82 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TC_THREADS, 1)
       const int cstop = rbase < ti.rows ? cend : cbeg;  // a warp of padding rows only: nothing to store
 #pragma unroll 1
       for (int c = cbeg; c < cstop; c += 32) {
+        if (MODE == MODE_GATEUP_RAW || MODE == MODE_SWIGLU_BWD) {
+          // backward epilogues, 32 columns of the lane's row at a time, each output written as
+          // 64 contiguous bytes of the row
+          const int col = ti.n0 + c;
+          const int hf = routed ? p.half_r : p.half_s;
+          uint32_t r0[32];
+          tmem_ld32(tbase + c, r0);
+          if (MODE == MODE_GATEUP_RAW) {
+            uint32_t r1[32];
+            tmem_ld32(tbase + BN + c, r1);
+            tmem_wait_ld();
+            if (row_ok && col < ti.N) {
+              float *o = (float *)out + (size_t)(ti.out_row0 + row) * ldo + col;
+#pragma unroll
+              for (int i = 0; i < 8; ++i) {
+                ((uint4 *)o)[i] = make_uint4(r0[4 * i], r0[4 * i + 1], r0[4 * i + 2], r0[4 * i + 3]);
+                ((uint4 *)(o + hf))[i] =
+                    make_uint4(r1[4 * i], r1[4 * i + 1], r1[4 * i + 2], r1[4 * i + 3]);
+              }
+            }
+          } else {
+            tmem_wait_ld();
+            if (row_ok && col < ti.N) {
+              const size_t arow = (size_t)(ti.out_row0 + row);
+              const float *gp = (const float *)(routed ? p.aux_r : p.aux_s) +
+                                arow * (routed ? p.ldaux_r : p.ldaux_s) + col;
+              __nv_bfloat16 *o = (__nv_bfloat16 *)out + arow * ldo + col;
+              __nv_bfloat16 *o2 = (__nv_bfloat16 *)(routed ? p.out2_r : p.out2_s) +
+                                  arow * (routed ? p.ld2_r : p.ld2_s) + col;
+              // 8 columns at a time: g, u in fp32; dg, du, h as hi + lo bf16 terms
+#pragma unroll
+              for (int q8 = 0; q8 < 4; ++q8) {
+                const float4 ga = ((const float4 *)gp)[2 * q8], gb = ((const float4 *)gp)[2 * q8 + 1];
+                const float4 ua = ((const float4 *)(gp + hf))[2 * q8],
+                             ub = ((const float4 *)(gp + hf))[2 * q8 + 1];
+                const float gv[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
+                const float uv[8] = {ua.x, ua.y, ua.z, ua.w, ub.x, ub.y, ub.z, ub.w};
+                uint32_t dgh[4], dgl[4], duh[4], dul[4], hh[4], hl[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                  float dgv[2], duv[2], hv[2];
+#pragma unroll
+                  for (int z = 0; z < 2; ++z) {
+                    const int e = 2 * i + z;
+                    const float g = gv[e], u = uv[e], dh = __uint_as_float(r0[8 * q8 + e]);
+                    const float sg = 1.0f / (1.0f + __expf(-g)), si = g * sg;
+                    dgv[z] = dh * u * sg * (1.0f + g * (1.0f - sg));
+                    duv[z] = dh * si;
+                    hv[z] = si * u;
+                  }
+                  const __nv_bfloat162 a = __floats2bfloat162_rn(dgv[0], dgv[1]);
+                  const __nv_bfloat162 b = __floats2bfloat162_rn(duv[0], duv[1]);
+                  const __nv_bfloat162 h = __floats2bfloat162_rn(hv[0], hv[1]);
+                  const float2 af = __bfloat1622float2(a), bfv = __bfloat1622float2(b),
+                               hf2 = __bfloat1622float2(h);
+                  const __nv_bfloat162 al = __floats2bfloat162_rn(dgv[0] - af.x, dgv[1] - af.y);
+                  const __nv_bfloat162 bl = __floats2bfloat162_rn(duv[0] - bfv.x, duv[1] - bfv.y);
+                  const __nv_bfloat162 hlo = __floats2bfloat162_rn(hv[0] - hf2.x, hv[1] - hf2.y);
+                  dgh[i] = *(const uint32_t *)&a;
+                  duh[i] = *(const uint32_t *)&b;
+                  hh[i] = *(const uint32_t *)&h;
+                  dgl[i] = *(const uint32_t *)&al;
+                  dul[i] = *(const uint32_t *)&bl;
+                  hl[i] = *(const uint32_t *)&hlo;
+                }
+                ((uint4 *)o)[q8] = make_uint4(dgh[0], dgh[1], dgh[2], dgh[3]);
+                ((uint4 *)(o + hf))[q8] = make_uint4(duh[0], duh[1], duh[2], duh[3]);
+                ((uint4 *)(o + 2 * hf))[q8] = make_uint4(dgl[0], dgl[1], dgl[2], dgl[3]);
+                ((uint4 *)(o + 3 * hf))[q8] = make_uint4(dul[0], dul[1], dul[2], dul[3]);
+                ((uint4 *)o2)[q8] = make_uint4(hh[0], hh[1], hh[2], hh[3]);
+                ((uint4 *)(o2 + hf))[q8] = make_uint4(hl[0], hl[1], hl[2], hl[3]);
+              }
+            }
+          }
+          continue;
+        }
         if (MODE == MODE_GATEUP) {
           // silu(gate) * up in bf16, 64 columns (128 bytes of each row) at a time: both 32-column
           // halves are packed, staged per warp and written as 32 coalesced 128-byte row stores
@@ -312,7 +398,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TC_THREADS, 1)
           const int col = ti.n0 + c;
           if (col < ti.N) {
             const int nrows = min(32, ti.rows - rbase);
-            unsigned char *obase = (unsigned char *)out + ((size_t)(ti.a_row0 + rbase) * ldo + col) * 2;
+            unsigned char *obase = (unsigned char *)out + ((size_t)(ti.out_row0 + rbase) * ldo + col) * 2;
             const size_t row_bytes = (size_t)ldo * 2;
             for (int rr = 0; rr < nrows; ++rr) {
               const uint32_t v = *(const uint32_t *)(stg + rr * 128 +
@@ -345,7 +431,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TC_THREADS, 1)
           const int col = ti.n0 + c;
           if (col < ti.N) {
             const int nrows = min(32, ti.rows - rbase);
-            unsigned char *obase = (unsigned char *)out + ((size_t)(ti.a_row0 + rbase) * ldo + col) * 2;
+            unsigned char *obase = (unsigned char *)out + ((size_t)(ti.out_row0 + rbase) * ldo + col) * 2;
             const size_t row_bytes = (size_t)ldo * 2;
             for (int rr = 0; rr < nrows; ++rr) {
               const uint32_t v = *(const uint32_t *)(stg + rr * 128 +
@@ -367,7 +453,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TC_THREADS, 1)
           const int col = ti.n0 + c;
           if (col < ti.N) {
             const int nrows = min(32, ti.rows - rbase);
-            unsigned char *obase = (unsigned char *)out + ((size_t)(ti.a_row0 + rbase) * ldo + col) * 4;
+            unsigned char *obase = (unsigned char *)out + ((size_t)(ti.out_row0 + rbase) * ldo + col) * 4;
             const size_t row_bytes = (size_t)ldo * 4;
             for (int rr = 0; rr < nrows; ++rr) {
               const uint32_t v = *(const uint32_t *)(stg + rr * 128 +

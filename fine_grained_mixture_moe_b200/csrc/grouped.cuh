@@ -9,7 +9,18 @@
 //                        This reads the shared down projections [S, d, fs] as one [d, S*fs]
 //                        matrix, so S shared experts of width fs act as one of width S*fs.
 // Epilogue modes: GATEUP out = silu(A B0^T) * (A B1^T) (SwiGLU, gate and up fused);
-//                 PLAIN  out = A B0^T;   SCALE out = (A B0^T) * scale[g][n] (low-rank s).
+//                 PLAIN  out = A B0^T;   SCALE out = (A B0^T) * scale[g][n] (low-rank s);
+//                 GATEUP_RAW (backward) g = A B0^T to out[., n], u = A B1^T to out[., half + n]
+//                   (fp32);
+//                 SWIGLU_BWD (backward) dh = A B0^T with fp32 g, u read from aux[., n] and
+//                   aux[., half + n]; dg = dh u silu'(g), du = dh silu(g) and h = silu(g) u, each
+//                   as two bf16 terms (v = hi + lo, hi = bf16(v), lo = bf16(v - hi)): out[., n] =
+//                   dg_hi, out[., half + n] = du_hi, out[., 2 half + n] = dg_lo,
+//                   out[., 3 half + n] = du_lo, out2[., n] = h_hi, out2[., half + n] = h_lo.
+// Groups along K (kgroup, backward weight gradients): group g is out rows [g M, g M + M) =
+// A[M, K_g] B[N, K_g]^T, where A and B are K-major [M or N][ld] and group g takes their columns
+// kseg koff[g] .. kseg koff[g+1] (koff padded to multiples of 64; kseg segments per group, so a
+// sum of split terms runs as one product); M is rows_r and ld is K_r.
 // Output types in the tensor-core (bf16) kernels: GATEUP and SCALE write bf16 (the next
 // product's operand, SCALE optionally as a hi + lo pair); PLAIN writes the routed groups' rows in
 // bf16 or fp32 (out_r_bf16) and the shared group's rows in fp32. The SIMT (fp32) kernels write
@@ -19,7 +30,8 @@
 
 namespace moe {
 
-enum GemmMode { MODE_GATEUP = 0, MODE_PLAIN = 1, MODE_SCALE = 2 };
+enum GemmMode { MODE_GATEUP = 0, MODE_PLAIN = 1, MODE_SCALE = 2, MODE_GATEUP_RAW = 3,
+                MODE_SWIGLU_BWD = 4 };
 
 struct GroupedGemm {
   const int32_t *offsets;  // [E+1] device
@@ -46,6 +58,17 @@ struct GroupedGemm {
   void *out_s;
   int ldo_s;
   int kind;                // KernelKind of the launch (in-step stamps)
+  // backward epilogues (GATEUP_RAW, SWIGLU_BWD): second half offset within a row of out / aux,
+  // the h output and the g, u input (bf16)
+  int half_r, half_s;
+  void *out2_r, *out2_s;
+  int ld2_r, ld2_s;
+  const void *aux_r, *aux_s;
+  int ldaux_r, ldaux_s;
+  // groups along K (backward weight gradients)
+  int kgroup;
+  const int32_t *koff;     // [E+1] device: padded K offsets of the groups
+  int kseg;                // K segments per group (kgroup)
 };
 
 // Tile counts per group and their exclusive prefix in shared memory (all threads call).
@@ -54,6 +77,11 @@ __device__ __forceinline__ int build_tile_prefix(const GroupedGemm &p, int BM, i
   const int G = p.E + p.has_shared;
   const int ntr = (p.N_r + BN - 1) / BN, nts = (p.N_s + BN - 1) / BN;
   for (int g = threadIdx.x; g < G; g += blockDim.x) {
+    if (p.kgroup) {
+      const int kg = p.kseg * (p.koff[g + 1] - p.koff[g]);
+      prefix[g] = kg > 0 ? ((p.rows_r + BM - 1) / BM) * ntr : 0;
+      continue;
+    }
     const int rows = g < p.E ? (p.offsets[g + 1] - p.offsets[g]) : p.T;
     prefix[g] = ((rows + BM - 1) / BM) * (g < p.E ? ntr : nts);
   }
@@ -66,7 +94,9 @@ __device__ __forceinline__ int build_tile_prefix(const GroupedGemm &p, int BM, i
 
 struct TileInfo {
   int g, rows, m0, n0, N, K;
-  int a_row0;  // first row of the group in A / out
+  int a_row0;    // first row of the group in A
+  int out_row0;  // first row of the group in out
+  int kofs;      // first column of the group in A and B (groups along K)
 };
 
 __device__ __forceinline__ TileInfo decode_tile(const GroupedGemm &p, int tile,
@@ -87,6 +117,15 @@ __device__ __forceinline__ TileInfo decode_tile(const GroupedGemm &p, int tile,
   const int local = tile - prefix[lo];
   ti.m0 = (local / nt) * BM;
   ti.n0 = (local % nt) * BN;
+  ti.kofs = 0;
+  if (p.kgroup) {
+    ti.a_row0 = 0;
+    ti.rows = p.rows_r;
+    ti.out_row0 = lo * p.rows_r;
+    ti.kofs = p.kseg * p.koff[lo];
+    ti.K = p.kseg * p.koff[lo + 1] - ti.kofs;
+    return ti;
+  }
   if (routed) {
     ti.a_row0 = p.offsets[lo];
     ti.rows = p.offsets[lo + 1] - ti.a_row0;
@@ -94,6 +133,7 @@ __device__ __forceinline__ TileInfo decode_tile(const GroupedGemm &p, int tile,
     ti.a_row0 = 0;
     ti.rows = p.T;
   }
+  ti.out_row0 = ti.a_row0;
   return ti;
 }
 

@@ -166,7 +166,7 @@ int num_sms() {
 // ------------------------------------------------------------------ profiling (debug)
 const char *kKindName[K_COUNT] = {"router", "stats", "perm_hist", "perm_scatter", "gemm_gateup",
                                   "gemm_down", "gemm_lowrank_v", "gemm_lowrank_u", "combine",
-                                  "aux_loss"};
+                                  "aux_loss", "backward_gemm"};
 constexpr int PROF_SLOTS = 8192;
 struct Prof {
   bool on = false;
@@ -263,6 +263,7 @@ bool make_map(CUtensorMap *m, const void *ptr, uint64_t rows, uint64_t cols, uin
 
 // ------------------------------------------------------------------ grouped GEMM launches
 long long tile_bound(const GroupedGemm &g, int BM, int BN) {
+  if (g.kgroup) return (long long)g.E * ceil_div(g.rows_r, BM) * ceil_div(g.N_r, BN);
   long long t = 0;
   if (g.E > 0) t += ((long long)ceil_div(g.rows_r, BM) + g.E) * ceil_div(g.N_r, BN);
   if (g.has_shared) t += (long long)ceil_div(g.T, BM) * ceil_div(g.N_s, BN);
@@ -276,10 +277,11 @@ bool build_maps(const GroupedGemm &g, bool two_b, uint32_t b_box, TcMaps *m) {
   bool ok = true;
   ok &= make_map(&m->a_r, g.E > 0 ? g.A_r : any, g.E > 0 ? g.rows_r : 1, g.E > 0 ? g.K_r : 64, 128);
   const int kb = g.kb_r ? g.kb_r : g.K_r;  // row length of the routed weights
-  ok &= make_map(&m->b0_r, g.E > 0 ? g.B0_r : any, g.E > 0 ? (uint64_t)g.E * g.N_r : 1,
+  // routed weights: E stacked [N_r, kb] matrices; groups along K: one [N_r, K_r] for all groups
+  const uint64_t b_rows = g.kgroup ? (uint64_t)g.N_r : (uint64_t)g.E * g.N_r;
+  ok &= make_map(&m->b0_r, g.E > 0 ? g.B0_r : any, g.E > 0 ? b_rows : 1, g.E > 0 ? kb : 64, b_box);
+  ok &= make_map(&m->b1_r, (g.E > 0 && two_b) ? g.B1_r : any, (g.E > 0 && two_b) ? b_rows : 1,
                  g.E > 0 ? kb : 64, b_box);
-  ok &= make_map(&m->b1_r, (g.E > 0 && two_b) ? g.B1_r : any,
-                 (g.E > 0 && two_b) ? (uint64_t)g.E * g.N_r : 1, g.E > 0 ? kb : 64, b_box);
   ok &= make_map(&m->a_s, g.has_shared ? g.A_s : any, g.has_shared ? g.T : 1,
                  g.has_shared ? g.K_s : 64, 128);
   ok &= make_map(&m->b0_s, g.has_shared ? g.B0_s : any, g.has_shared ? g.b_rows_s : 1,
@@ -316,7 +318,7 @@ moe_status_t launch_tc2(const GroupedGemm &g, cudaStream_t st, int kind) {
   std::memset(&P, 0, sizeof(P));
   P.p = g;
   P.p.kind = kind;
-  if (!build_maps(g, MODE == MODE_GATEUP, 128, &P.maps)) return MOE_ERR_CUDA;
+  if (!build_maps(g, tc2_two_b(MODE), 128, &P.maps)) return MOE_ERR_CUDA;
   const int G = g.E + g.has_shared;
   static_assert(tc2_stages<MODE>(1024 + 1) >= 2, "tile list of 1024 experts leaves no room");
   P.stages = tc2_stages<MODE>(G);
@@ -595,6 +597,220 @@ moe_status_t route_backward_impl(const moe_config_t *c, const RouteBwdArgs &a, f
                     c->d, c->E, dx);
 }
 
+// ------------------------------------------------------------------ backward of the experts
+// Workspace of moe_expert_backward (bf16 SwiGLU layers): g and u recomputed (fp32), [dg | du]
+// and h as hi + lo bf16 terms, the routed dX before the un-permute, the shared experts'
+// counterparts, dy as hi + lo terms, the transposed weights and the transposed, per-expert
+// zero-padded activations of the weight gradients (2 or 3 K segments per group).
+struct BwdLayout {
+  size_t koff, off_s, koff_s;
+  size_t gu, dgu, h, dxp, gu_s, dgu_s, h_s, dx_s, dy_b;
+  size_t wdt, wgut, wsdt, wsgut;
+  size_t ydt, ht, dgut, xpt, ydt_s, ht_s, dgut_s, xt_s;
+  size_t total;
+  int npad, tpad;
+};
+
+BwdLayout bwd_layout(const moe_config_t *c) {
+  BwdLayout L;
+  const size_t T = c->T, d = c->d, E = c->E, k = c->top_k, f = c->ffn;
+  const size_t sf = (size_t)c->n_shared * c->ffn_shared, N = T * k;
+  L.npad = (int)(((N + 64 * E) + 63) & ~(size_t)63);  // >= the sum of the padded group sizes
+  L.tpad = (int)((T + 63) & ~(size_t)63);
+  const size_t np = L.npad, tp = L.tpad;
+  size_t o = 0;
+  auto take = [&](size_t bytes) { size_t at = o; o = align256(o + std::max<size_t>(bytes, 1)); return at; };
+  L.koff = take((E + 1) * 4);
+  L.off_s = take(8);
+  L.koff_s = take(8);
+  L.gu = take(N * 2 * f * 4);
+  L.dgu = take(N * 4 * f * 2);
+  L.h = take(N * 2 * f * 2);
+  L.dxp = take(N * d * 4);
+  L.gu_s = take(T * 2 * sf * 4);
+  L.dgu_s = take(T * 4 * sf * 2);
+  L.h_s = take(T * 2 * sf * 2);
+  L.dx_s = take(T * d * 4);
+  L.dy_b = take(sf ? T * 2 * d * 2 : 0);
+  L.wdt = take(E * f * d * 2);
+  L.wgut = take(E * d * 2 * f * 2);
+  L.wsdt = take(sf * d * 2);
+  L.wsgut = take(d * 2 * sf * 2);
+  L.ydt = take(d * 2 * np * 2);
+  L.ht = take(f * 2 * np * 2);
+  L.dgut = take(2 * f * 2 * np * 2);
+  L.xpt = take(d * 2 * np * 2);
+  L.ydt_s = take(sf ? d * 3 * tp * 2 : 0);
+  L.ht_s = take(sf * 3 * tp * 2);
+  L.dgut_s = take(2 * sf * 2 * tp * 2);
+  L.xt_s = take(sf ? d * 2 * tp * 2 : 0);
+  L.total = o;
+  return L;
+}
+
+using bf16_t = __nv_bfloat16;
+
+// Transposes (transpose_bf16_kernel): grouped rows -> nseg padded column segments, or dense
+// batches.
+moe_status_t launch_transpose_grouped(int nseg, const bf16_t *s0, const bf16_t *s1,
+                                      const bf16_t *s2, int C, int ldi, const int32_t *offsets,
+                                      const int32_t *koff, int G, int ncolblocks, void *out,
+                                      int ldo, cudaStream_t st) {
+  return launch_pdl(transpose_bf16_kernel<bf16_t>, dim3(C / 64, ncolblocks, 1), dim3(256), 0, st,
+                    s0, s1, s2, nseg, C, ldi, offsets, koff, G, 0, (size_t)0, (bf16_t *)out, ldo,
+                    (size_t)0, 0);
+}
+moe_status_t launch_transpose_dense(const bf16_t *in, int R, int C, int batches, size_t ibs,
+                                    void *out, int ldo, size_t obs, int col0, cudaStream_t st) {
+  return launch_pdl(transpose_bf16_kernel<bf16_t>, dim3(C / 64, ceil_div(R, 64), batches),
+                    dim3(256), 0, st, in, (const bf16_t *)nullptr, (const bf16_t *)nullptr, 1, C,
+                    C, (const int32_t *)nullptr, (const int32_t *)nullptr, 0, R, ibs,
+                    (bf16_t *)out, ldo, obs, col0);
+}
+
+// One weight-gradient product with groups along K: out[g] (M x N, fp32, row-major) =
+// A[:, kseg koff[g] .. kseg koff[g+1]) B[:, same]^T, A [M, ld], B [N, ld] bf16.
+moe_status_t launch_wgrad(int G, const int32_t *koff, int kseg, const void *A, int M,
+                          const void *Bm, int N, int ld, float *out, cudaStream_t st) {
+  GroupedGemm g;
+  std::memset(&g, 0, sizeof(g));
+  g.kgroup = 1;
+  g.koff = koff;
+  g.kseg = kseg;
+  g.E = G;
+  g.A_r = A;
+  g.lda_r = ld;
+  g.rows_r = M;
+  g.B0_r = Bm;
+  g.N_r = N;
+  g.K_r = ld;
+  g.out_r = out;
+  g.ldo_r = N;
+  return launch_tc2<MODE_PLAIN>(g, st, K_BWD_GEMM);
+}
+
+moe_status_t expert_backward_impl(const moe_config_t *c, const void *x_perm,
+                                  const int32_t *offsets, const int32_t *slot_pos, const void *x,
+                                  const moe_weights_t *w, const void *dy_perm, const float *dy,
+                                  float *dx, const moe_grads_t *gr, void *ws, cudaStream_t st) {
+  const BwdLayout L = bwd_layout(c);
+  const int T = c->T, d = c->d, E = c->E, k = c->top_k, f = c->ffn;
+  const int S = c->n_shared, fs = c->ffn_shared, sf = S * fs;
+  const bool sh = S > 0;
+  using bf = bf16_t;
+  int32_t *koff = at<int32_t>(ws, L.koff), *off_s = at<int32_t>(ws, L.off_s),
+          *koff_s = at<int32_t>(ws, L.koff_s);
+  float *GU = at<float>(ws, L.gu), *GUs = at<float>(ws, L.gu_s);
+  bf *DGU = at<bf>(ws, L.dgu), *H = at<bf>(ws, L.h);
+  float *dXp = at<float>(ws, L.dxp), *dXs = at<float>(ws, L.dx_s);
+  bf *DGUs = at<bf>(ws, L.dgu_s), *Hs = at<bf>(ws, L.h_s), *dyb = at<bf>(ws, L.dy_b);
+  bf *Wdt = at<bf>(ws, L.wdt), *Wgut = at<bf>(ws, L.wgut), *Wsdt = at<bf>(ws, L.wsdt),
+     *Wsgut = at<bf>(ws, L.wsgut);
+  bf *Ydt = at<bf>(ws, L.ydt), *Ht = at<bf>(ws, L.ht), *DGUt = at<bf>(ws, L.dgut),
+     *Xpt = at<bf>(ws, L.xpt), *Ydts = at<bf>(ws, L.ydt_s), *Hts = at<bf>(ws, L.ht_s),
+     *DGUts = at<bf>(ws, L.dgut_s), *Xts = at<bf>(ws, L.xt_s);
+  const int np = L.npad, tp = L.tpad;
+  const bf *xp = (const bf *)x_perm, *xb = (const bf *)x, *dyp = (const bf *)dy_perm;
+
+  // padded group offsets of the weight gradients
+  MOE_TRY(launch_pdl(pad_offsets_kernel, dim3(1), dim3(1024), 0, st, offsets, E, koff, T, off_s,
+                     koff_s));
+  GroupedGemm base;
+  std::memset(&base, 0, sizeof(base));
+  base.offsets = offsets;
+  base.T = T;
+  base.rows_r = T * k;
+  base.E = E;
+  base.has_shared = sh;
+  // g and u (fp32) of the routed rows, and of every token for the shared experts
+  {
+    GroupedGemm g = base;
+    g.A_r = x_perm; g.lda_r = d; g.B0_r = w->w_gate; g.B1_r = w->w_up; g.N_r = f; g.K_r = d;
+    g.out_r = GU; g.ldo_r = 2 * f; g.half_r = f;
+    if (sh) {
+      g.A_s = x; g.lda_s = d; g.B0_s = w->ws_gate; g.B1_s = w->ws_up; g.N_s = sf; g.K_s = d;
+      g.piece_k = d; g.b_rows_s = sf; g.out_s = GUs; g.ldo_s = 2 * sf; g.half_s = sf;
+    }
+    MOE_TRY(launch_tc2<MODE_GATEUP_RAW>(g, st, K_BWD_GEMM));
+  }
+  // transposed weights: W_d [E][d][f] -> [E][f][d]; [W_g; W_u] -> [E][d][2f]; shared likewise
+  const bf *wg = (const bf *)w->w_gate, *wu = (const bf *)w->w_up, *wd = (const bf *)w->w_down;
+  MOE_TRY(launch_transpose_dense(wd, d, f, E, (size_t)d * f, Wdt, d, (size_t)f * d, 0, st));
+  MOE_TRY(launch_transpose_dense(wg, f, d, E, (size_t)f * d, Wgut, 2 * f, (size_t)d * 2 * f, 0, st));
+  MOE_TRY(launch_transpose_dense(wu, f, d, E, (size_t)f * d, Wgut, 2 * f, (size_t)d * 2 * f, f, st));
+  if (sh) {
+    const bf *sg = (const bf *)w->ws_gate, *su = (const bf *)w->ws_up, *sdn = (const bf *)w->ws_down;
+    MOE_TRY(launch_transpose_dense(sdn, d, fs, S, (size_t)d * fs, Wsdt, d, (size_t)fs * d, 0, st));
+    MOE_TRY(launch_transpose_dense(sg, sf, d, 1, 0, Wsgut, 2 * sf, 0, 0, st));
+    MOE_TRY(launch_transpose_dense(su, sf, d, 1, 0, Wsgut, 2 * sf, 0, sf, st));
+    // the shared experts' upstream gradient (fp32) as hi + lo bf16 terms
+    MOE_TRY(launch_pdl(split_bf16_kernel,
+                       dim3((unsigned)std::min<long long>(ceil_div((long long)T * d, 1024), 65535)),
+                       dim3(256), 0, st, dy, d, (size_t)T, dyb));
+  }
+  // dh = dY W_d with the SwiGLU backward in the epilogue: [dg | du] and h as hi + lo terms
+  {
+    GroupedGemm g = base;
+    g.A_r = dy_perm; g.lda_r = d; g.B0_r = Wdt; g.N_r = f; g.K_r = d;
+    g.out_r = DGU; g.ldo_r = 4 * f; g.half_r = f; g.out2_r = H; g.ld2_r = 2 * f;
+    g.aux_r = GU; g.ldaux_r = 2 * f;
+    if (sh) {  // A = [dy_hi | dy_lo], K = 2d, the weight's k wraps over its d columns
+      g.A_s = dyb; g.lda_s = 2 * d; g.B0_s = Wsdt; g.N_s = sf; g.K_s = 2 * d; g.piece_k = d;
+      g.piece_rows = 0; g.b_rows_s = sf; g.out_s = DGUs; g.ldo_s = 4 * sf; g.half_s = sf;
+      g.out2_s = Hs; g.ld2_s = 2 * sf; g.aux_s = GUs; g.ldaux_s = 2 * sf;
+    }
+    MOE_TRY(launch_tc2<MODE_SWIGLU_BWD>(g, st, K_BWD_GEMM));
+  }
+  // dX = [dg | du]_hi [W_g; W_u] + [dg | du]_lo [W_g; W_u] (fp32; K = 4 ffn, the weight's k
+  // wraps), then the un-permute: dx[t] = dX_s[t] + sum_j dX[pos(t, j)]
+  {
+    GroupedGemm g = base;
+    g.A_r = DGU; g.lda_r = 4 * f; g.B0_r = Wgut; g.N_r = d; g.K_r = 4 * f; g.kb_r = 2 * f;
+    g.out_r = dXp; g.ldo_r = d; g.out_r_bf16 = 0;
+    if (sh) {
+      g.A_s = DGUs; g.lda_s = 4 * sf; g.B0_s = Wsgut; g.N_s = d; g.K_s = 4 * sf;
+      g.piece_k = 2 * sf; g.piece_rows = 0; g.b_rows_s = d; g.out_s = dXs; g.ldo_s = d;
+    }
+    MOE_TRY(launch_tc2<MODE_PLAIN>(g, st, K_BWD_GEMM));
+  }
+  MOE_TRY(launch_pdl(combine_kernel<float>, dim3(ceil_div(T, 8)), dim3(256), 0, st,
+                     (const float *)dXp, sh ? (const float *)dXs : (const float *)nullptr,
+                     slot_pos, (const float *)nullptr, dx, T, k, d, false));
+  // weight gradients: one operand as hi + lo segments, the other repeated, so that each product
+  // sums both terms: dW_d = dY^T (h_hi + h_lo), dW_g = (dg_hi + dg_lo)^T X, dW_u likewise
+  const int nb2 = 2 * np / 64;
+  MOE_TRY(launch_transpose_grouped(2, dyp, dyp, nullptr, d, d, offsets, koff, E, nb2, Ydt, 2 * np, st));
+  MOE_TRY(launch_transpose_grouped(2, H, H + f, nullptr, f, 2 * f, offsets, koff, E, nb2, Ht, 2 * np, st));
+  MOE_TRY(launch_transpose_grouped(2, DGU, DGU + 2 * f, nullptr, 2 * f, 4 * f, offsets, koff, E,
+                                   nb2, DGUt, 2 * np, st));
+  MOE_TRY(launch_transpose_grouped(2, xp, xp, nullptr, d, d, offsets, koff, E, nb2, Xpt, 2 * np, st));
+  MOE_TRY(launch_wgrad(E, koff, 2, Ydt, d, Ht, f, 2 * np, gr->d_w_down, st));
+  MOE_TRY(launch_wgrad(E, koff, 2, DGUt, f, Xpt, d, 2 * np, gr->d_w_gate, st));
+  MOE_TRY(launch_wgrad(E, koff, 2, DGUt + (size_t)f * 2 * np, f, Xpt, d, 2 * np, gr->d_w_up, st));
+  MOE_TRY(launch_pdl(zero_empty_experts_kernel, dim3(E, 8), dim3(256), 0, st, offsets,
+                     gr->d_w_gate, (size_t)f * d, gr->d_w_up, (size_t)f * d, gr->d_w_down,
+                     (size_t)d * f));
+  if (sh) {
+    // dW_sg, dW_su: (dg_hi + dg_lo)^T x; dW_sd: (dy_hi + dy_lo)^T (h_hi + h_lo) less lo lo,
+    // three segments [hi hi | hi lo | lo hi]
+    MOE_TRY(launch_transpose_grouped(2, DGUs, DGUs + 2 * sf, nullptr, 2 * sf, 4 * sf, off_s,
+                                     koff_s, 1, 2 * tp / 64, DGUts, 2 * tp, st));
+    MOE_TRY(launch_transpose_grouped(2, xb, xb, nullptr, d, d, off_s, koff_s, 1, 2 * tp / 64, Xts,
+                                     2 * tp, st));
+    MOE_TRY(launch_transpose_grouped(3, dyb, dyb, dyb + d, d, 2 * d, off_s, koff_s, 1,
+                                     3 * tp / 64, Ydts, 3 * tp, st));
+    MOE_TRY(launch_transpose_grouped(3, Hs, Hs + sf, Hs, sf, 2 * sf, off_s, koff_s, 1,
+                                     3 * tp / 64, Hts, 3 * tp, st));
+    MOE_TRY(launch_wgrad(1, koff_s, 2, DGUts, sf, Xts, d, 2 * tp, gr->d_ws_gate, st));
+    MOE_TRY(launch_wgrad(1, koff_s, 2, DGUts + (size_t)sf * 2 * tp, sf, Xts, d, 2 * tp,
+                         gr->d_ws_up, st));
+    for (int s = 0; s < S; ++s)
+      MOE_TRY(launch_wgrad(1, koff_s, 3, Ydts, d, Hts + (size_t)s * fs * 3 * tp, fs, 3 * tp,
+                           gr->d_ws_down + (size_t)s * d * fs, st));
+  }
+  return MOE_OK;
+}
+
 // ------------------------------------------------------------------ argument checks
 moe_status_t check_cfg(const moe_config_t *c) {
   if (!c) return MOE_ERR_INVALID_ARG;
@@ -742,6 +958,43 @@ moe_status_t moe_route_backward(const moe_config_t *cfg, const void *x, const mo
   a.dL = d_loss;
   if (cfg->dtype == MOE_DTYPE_BF16) return route_backward_impl<__nv_bfloat16>(cfg, a, d_w_router, dx, st);
   return route_backward_impl<float>(cfg, a, d_w_router, dx, st);
+}
+
+size_t moe_backward_workspace_size(const moe_config_t *cfg) {
+  if (check_cfg(cfg) != MOE_OK) return 0;
+  return bwd_layout(cfg).total;
+}
+
+moe_status_t moe_expert_backward(const moe_config_t *cfg, const void *x_perm,
+                                 const int32_t *offsets, const int32_t *slot_pos, const void *x,
+                                 const moe_weights_t *w, const void *dy_perm, const float *dy,
+                                 float *dx, const moe_grads_t *g, void *ws, size_t ws_bytes,
+                                 void *stream) {
+  MOE_TRY(check_cfg(cfg));
+  if (cfg->dtype != MOE_DTYPE_BF16 || cfg->expert != MOE_EXPERT_SWIGLU) return MOE_ERR_UNSUPPORTED;
+  MOE_TRY(check_weights(cfg, w, false, true));
+  MOE_REQUIRE(g != nullptr);
+  MOE_REQUIRE(tok16(cfg, x_perm) && aligned16(offsets) && tok16(cfg, slot_pos) && tok16(cfg, x) &&
+              tok16(cfg, dy_perm) && tok16(cfg, dx));
+  MOE_REQUIRE(aligned16(g->d_w_gate) && aligned16(g->d_w_up) && aligned16(g->d_w_down));
+  MOE_REQUIRE(cfg->n_shared == 0 || (tok16(cfg, dy) && aligned16(g->d_ws_gate) &&
+                                     aligned16(g->d_ws_up) && aligned16(g->d_ws_down)));
+  MOE_REQUIRE(aligned16(ws));
+  if (ws_bytes < bwd_layout(cfg).total) return MOE_ERR_WORKSPACE;
+  cudaStream_t st = (cudaStream_t)stream;
+  if (cfg->T == 0) {  // no rows: every gradient is zero
+    const size_t E = cfg->E, f = cfg->ffn, d = cfg->d, sf = (size_t)cfg->n_shared * cfg->ffn_shared;
+    if (cudaMemsetAsync(g->d_w_gate, 0, E * f * d * 4, st) != cudaSuccess ||
+        cudaMemsetAsync(g->d_w_up, 0, E * f * d * 4, st) != cudaSuccess ||
+        cudaMemsetAsync(g->d_w_down, 0, E * f * d * 4, st) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    if (sf && (cudaMemsetAsync(g->d_ws_gate, 0, sf * d * 4, st) != cudaSuccess ||
+               cudaMemsetAsync(g->d_ws_up, 0, sf * d * 4, st) != cudaSuccess ||
+               cudaMemsetAsync(g->d_ws_down, 0, sf * d * 4, st) != cudaSuccess))
+      return MOE_ERR_CUDA;
+    return MOE_OK;
+  }
+  return expert_backward_impl(cfg, x_perm, offsets, slot_pos, x, w, dy_perm, dy, dx, g, ws, st);
 }
 
 moe_status_t moe_aux_loss(const moe_config_t *cfg, const int32_t *expert_count,

@@ -178,6 +178,45 @@ moe_status_t moe_combine_backward(const moe_config_t *cfg, const float *dy, cons
                                   const int32_t *slot_pos, const float *topk_w, void *dy_perm,
                                   float *d_topk_w, void *stream);
 
+/* Weight gradients of the experts: fp32 device buffers in the weights' own layouts. */
+typedef struct {
+  float *d_w_gate;   /* SwiGLU: [E, ffn, d] */
+  float *d_w_up;     /* SwiGLU: [E, ffn, d] */
+  float *d_w_down;   /* SwiGLU: [E, d, ffn] */
+  float *d_lr_V;     /* low-rank: [E, rank, d] */
+  float *d_lr_s;     /* low-rank: [E, rank] */
+  float *d_lr_U;     /* low-rank: [E, d, rank] */
+  float *d_ws_gate;  /* shared: [n_shared, ffn_shared, d] */
+  float *d_ws_up;    /* shared: [n_shared, ffn_shared, d] */
+  float *d_ws_down;  /* shared: [n_shared, d, ffn_shared] */
+} moe_grads_t;
+
+/* Bytes of workspace moe_expert_backward needs for `cfg` (0 for an invalid configuration). */
+size_t moe_backward_workspace_size(const moe_config_t *cfg);
+
+/* Backward of moe_expert_forward and of the un-permute (the derivative of the forward, the
+ * conventions of moe_combine_backward; Quartz architecture table and Moonfrost expert card: the
+ * routed SwiGLU experts on their grouped rows and the shared experts on every token). Per expert
+ * e on its grouped rows X_e with upstream gradient dY_e, g = X_e W_g^T, u = X_e W_u^T:
+ *   dh = dY_e W_d[e];  du = dh * silu(g);  dg = dh * u * silu'(g);  h = silu(g) * u
+ *   d_w_down[e] = dY_e^T h;  d_w_gate[e] = dg^T X_e;  d_w_up[e] = du^T X_e
+ *   dX_e = dg W_g[e] + du W_u[e]
+ * and likewise for the shared experts on all T tokens with upstream gradient dy. Then
+ *   dx[t] = dX_shared[t] + sum over the token's kept pairs (t, j) of dX[slot_pos[t, j]]
+ * (the experts' part of the input gradient; the router's part comes from moe_route_backward).
+ * x_perm, offsets, slot_pos: as moe_permute produced them; x: the layer input; dy_perm: [T*k, d]
+ * in y_perm's dtype, rows of kept pairs from moe_combine_backward; dy: [T, d] fp32 (used for the
+ * shared experts, may be NULL when n_shared = 0); dx: [T, d] fp32 output. g and u are recomputed
+ * in bf16 and dg, du, h rounded to bf16 (the next products' operands); every product accumulates
+ * in fp32 in a fixed order (bitwise reproducible). Experts with no rows get zero gradients.
+ * Supported: bf16 layers with SwiGLU experts; other configurations return MOE_ERR_UNSUPPORTED.
+ * ws: moe_backward_workspace_size(cfg) bytes of the caller's device memory. Asynchronous. */
+moe_status_t moe_expert_backward(const moe_config_t *cfg, const void *x_perm,
+                                 const int32_t *offsets, const int32_t *slot_pos, const void *x,
+                                 const moe_weights_t *w, const void *dy_perm, const float *dy,
+                                 float *dx, const moe_grads_t *g, void *ws, size_t ws_bytes,
+                                 void *stream);
+
 /* Backward of moe_route and of the load-balancing loss (Quartz: architecture table, row
  * "Router"; Sutra-1.3B, "48 + 1 experts" for sigmoid scores). Per token t, with the logits
  * recomputed as l = x W_r^T + off in fp32 (not the forward's exact rounding: a difference of a

@@ -283,6 +283,121 @@ def test_route_and_combine_backward(name):
                            g2[key][:N] if key == "dy_perm" else g2[key]), key
 
 
+# the backward's expert steps (moe_expert_backward): SwiGLU layers in bf16 with 0 to 3 shared
+# experts, norm_topk, capacity drops (heavy ones too), one token, one expert, k = E, wide and
+# narrow hidden sizes, widths that are not multiples of 256, and 97 experts (T < E: empty ones)
+EXPERT_BACKWARD = ["quartz_s", "capacity_s", "sigmoid_s", "norm_softmax", "heavy_drops",
+                   "three_shared", "T1", "T33", "k_eq_E", "E1k1", "k8_E97", "d4096"]
+
+
+def _expert_grads(c, run):
+    E, d, S = run.cfg.E, run.cfg.d, c.n_shared
+    f, fs, dev = c.ffn, c.ffn_shared, run.dev
+    g = dict(d_w_gate=torch.empty((E, f, d), dtype=torch.float32, device=dev),
+             d_w_up=torch.empty((E, f, d), dtype=torch.float32, device=dev),
+             d_w_down=torch.empty((E, d, f), dtype=torch.float32, device=dev))
+    if S:
+        g.update(d_ws_gate=torch.empty((S, fs, d), dtype=torch.float32, device=dev),
+                 d_ws_up=torch.empty((S, fs, d), dtype=torch.float32, device=dev),
+                 d_ws_down=torch.empty((S, d, fs), dtype=torch.float32, device=dev))
+    return g
+
+
+def _expert_step_reference(c, inp, dy_perm, dy):
+    """The oracle's expert step on this step's own inputs: the backward oracle's per-expert
+    SwiGLU backward (pinned by central differences) on the grouped rows with the device's
+    dy_perm (the combine backward's output, checked against the oracle's combine step in
+    test_route_and_combine_backward), the shared experts on dy, then the un-permute."""
+    from oracle import moe_backward as BW
+    pm = oracle.layer_forward(c, inp, with_outputs=False)["perm"]
+    offs, src = pm["offsets"], pm["src"]
+    N = int(offs[-1])
+    x = np.asarray(inp["x"], np.float64)
+    Xp = x[src]
+    dYp = np.asarray(dy_perm, np.float64)[:N]
+    out = {n: np.zeros(np.asarray(inp[n[2:]]).shape) for n in ("d_w_gate", "d_w_up", "d_w_down")}
+    dXp = np.zeros((N, x.shape[1]))
+    for e in range(c.E):
+        a, b = int(offs[e]), int(offs[e + 1])
+        if a == b:
+            continue
+        g = BW.swiglu_backward(Xp[a:b], inp["w_gate"][e], inp["w_up"][e], inp["w_down"][e],
+                               dYp[a:b])
+        out["d_w_gate"][e], out["d_w_up"][e], out["d_w_down"][e] = g["dWg"], g["dWu"], g["dWd"]
+        dXp[a:b] = g["dX"]
+    dx = np.zeros_like(x)
+    np.add.at(dx, src, dXp)
+    if c.n_shared:
+        for n in ("d_ws_gate", "d_ws_up", "d_ws_down"):
+            out[n] = np.zeros(np.asarray(inp[n[2:]]).shape)
+        for s_ in range(c.n_shared):
+            g = BW.swiglu_backward(x, inp["ws_gate"][s_], inp["ws_up"][s_], inp["ws_down"][s_],
+                                   np.asarray(dy, np.float64))
+            out["d_ws_gate"][s_], out["d_ws_up"][s_], out["d_ws_down"][s_] = (
+                g["dWg"], g["dWu"], g["dWd"])
+            dx += g["dX"]
+    out["dx"] = dx
+    return out
+
+
+@pytest.mark.parametrize("name", EXPERT_BACKWARD)
+def test_expert_backward(name):
+    """moe_expert_backward against the oracle's expert step on the same inputs: dx (the
+    experts' part) and every expert weight gradient within the bf16 tolerance of its rms;
+    bitwise equal on a second call. Its dy_perm comes from moe_combine_backward on the forward's
+    y_perm, as in a training step. (Against the whole-layer backward oracle instead, the weight
+    gradients also carry dy_perm's bf16 rounding: up to 0.08 of their rms on the Quartz shape,
+    a figure this step's own arithmetic does not set.)"""
+    c = SMALL[name] if name in SMALL else EDGE[name]
+    inp = make_inputs(c)
+    run = LayerOnGpu(c, inp)
+    o = run.steps()
+    T, d, k = run.cfg.T, run.cfg.d, run.cfg.top_k
+    dev = run.dev
+    dy = np.random.default_rng(11).standard_normal((T, d)).astype(np.float32)
+    dy_t = torch.as_tensor(dy).to(dev)
+    dyp = torch.empty_like(o["y_perm"])
+    d_w = torch.empty((T, k), dtype=torch.float32, device=dev)
+    B.moe_combine_backward(run.cfg, dy_t, o["y_perm"], o["slot_pos"], o["w"], dyp, d_w)
+    grads = _expert_grads(c, run)
+    ws_bytes = B.moe_backward_workspace_size(run.cfg)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    dx = torch.empty((T, d), dtype=torch.float32, device=dev)
+
+    def call():
+        B.moe_expert_backward(run.cfg, o["x_perm"], o["offsets"], o["slot_pos"], run.x,
+                              run.ws_struct, dyp, dy_t if c.n_shared else None, dx,
+                              B.make_grads(grads), ws, ws_bytes)
+        torch.cuda.synchronize()
+        st, info = B.moe_get_device_error()
+        assert st == 0, (B.status_str(st), info)
+
+    call()
+    ref = _expert_step_reference(c, inp, np_(dyp), dy)
+    tol = tol_of(c)
+    errs = {"dx": rel_err(np_(dx), ref["dx"])}
+    for n, t in grads.items():
+        errs[n] = rel_err(np_(t), ref[n])
+    msg = f"{name}: worst max|d|/rms " + ", ".join(f"{n}={v:.2e}" for n, v in errs.items())
+    print(msg)
+    assert all(v <= tol for v in errs.values()), msg
+    first = {n: t.clone() for n, t in grads.items()}
+    dx1 = dx.clone()
+    call()
+    assert torch.equal(dx, dx1) and all(torch.equal(grads[n], first[n]) for n in grads)
+
+
+def test_expert_backward_unsupported_configurations():
+    """fp32 layers and low-rank experts are refused on the host (MOE_ERR_UNSUPPORTED)."""
+    for c in (get_config("tiny_f32"), get_config("lowrank", T=64, E=16)):
+        cfg = B.make_config(T=c.T, d=c.d, E=c.E, top_k=c.top_k, n_shared=c.n_shared, ffn=c.ffn,
+                            ffn_shared=c.ffn_shared, rank=c.rank, expert=c.expert, dtype=c.dtype)
+        with pytest.raises(B.MoEError) as ei:
+            B.moe_expert_backward(cfg, 256, 256, 256, 256, B.MoEWeights(), 256, 256, 256,
+                                  B.MoEGrads(), 256, 1 << 20)
+        assert ei.value.status == 2
+
+
 def test_bias_update_bitwise():
     """Loss-free balancing step on the routed counts of the sigmoid configuration, then the next
     routing call with the updated bias: the bias bit-exact against the oracle, the new routing
