@@ -363,6 +363,67 @@ __global__ void __launch_bounds__(256) split_bf16_kernel(const float *__restrict
   }
 }
 
+// Low-rank experts: for the 64-row block b of the padded grouped rows (koff, as the transposes
+// use), with z = X V^T and dzs = dY U (fp32 [rows, r]) and the expert's s:
+//   dz = dzs s and zs = z s as bf16 hi + lo terms ([rows, 2r]: hi | lo);
+//   ds_part[b][j] = sum over the block's rows of dzs[., j] z[., j] (4 row groups in fixed order).
+__global__ void __launch_bounds__(256) lowrank_elem_kernel(
+    const float *__restrict__ z, const float *__restrict__ dzs, const float *__restrict__ s,
+    const int32_t *__restrict__ offsets, const int32_t *__restrict__ koff, int E, int r,
+    __nv_bfloat16 *__restrict__ dz2, __nv_bfloat16 *__restrict__ zs2,
+    float *__restrict__ ds_part) {
+  griddep_wait();
+  griddep_launch();
+  __shared__ float part[4][64];
+  const int p0 = blockIdx.x * 64;
+  if (p0 >= koff[E]) return;
+  int lo = 0, hi = E - 1;  // expert with koff[e] <= p0 < koff[e+1]
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (koff[mid] <= p0) lo = mid;
+    else hi = mid - 1;
+  }
+  const int local = p0 - koff[lo];
+  const int row0 = offsets[lo] + local, nrow = max(0, min(64, offsets[lo + 1] - offsets[lo] - local));
+  const int cl = threadIdx.x & 63, rg = threadIdx.x >> 6;
+  for (int j0 = 0; j0 < r; j0 += 64) {
+    const int j = j0 + cl;
+    const float sj = s[(size_t)lo * r + j];
+    float acc = 0.0f;
+    for (int i = rg; i < nrow; i += 4) {
+      const size_t row = (size_t)(row0 + i);
+      const float zv = z[row * r + j], dv = dzs[row * r + j];
+      acc = fmaf(dv, zv, acc);
+      const float a = dv * sj, b = zv * sj;
+      const __nv_bfloat16 ah = __float2bfloat16_rn(a), bh = __float2bfloat16_rn(b);
+      dz2[row * 2 * r + j] = ah;
+      dz2[row * 2 * r + r + j] = __float2bfloat16_rn(a - __bfloat162float(ah));
+      zs2[row * 2 * r + j] = bh;
+      zs2[row * 2 * r + r + j] = __float2bfloat16_rn(b - __bfloat162float(bh));
+    }
+    part[rg][cl] = acc;
+    __syncthreads();
+    if (rg == 0)
+      ds_part[(size_t)blockIdx.x * r + j] = ((part[0][cl] + part[1][cl]) + part[2][cl]) + part[3][cl];
+    __syncthreads();
+  }
+}
+
+// ds[e][j] = sum of the expert's block partials in block order (0 for an expert with no rows).
+__global__ void __launch_bounds__(256) lowrank_ds_kernel(const float *__restrict__ ds_part,
+                                                         const int32_t *__restrict__ koff, int r,
+                                                         float *__restrict__ ds) {
+  griddep_wait();
+  griddep_launch();
+  const int e = blockIdx.x;
+  const int b0 = koff[e] / 64, b1 = koff[e + 1] / 64;
+  for (int j = threadIdx.x; j < r; j += blockDim.x) {
+    float acc = 0.0f;
+    for (int b = b0; b < b1; ++b) acc += ds_part[(size_t)b * r + j];
+    ds[(size_t)e * r + j] = acc;
+  }
+}
+
 // Zero the gradient slices of experts that received no rows (their weight-gradient products
 // have no tiles): up to three arrays with `per` floats per expert each.
 __global__ void __launch_bounds__(256) zero_empty_experts_kernel(

@@ -607,13 +607,16 @@ struct BwdLayout {
   size_t gu, dgu, h, dxp, gu_s, dgu_s, h_s, dx_s, dy_b;
   size_t wdt, wgut, wsdt, wsgut;
   size_t ydt, ht, dgut, xpt, ydt_s, ht_s, dgut_s, xt_s;
+  size_t z, dzs, dys, dz2, zs2, ut, vt, dzt, zst, ds_part;  // low-rank experts
   size_t total;
   int npad, tpad;
 };
 
 BwdLayout bwd_layout(const moe_config_t *c) {
   BwdLayout L;
-  const size_t T = c->T, d = c->d, E = c->E, k = c->top_k, f = c->ffn;
+  const bool swi = c->expert == MOE_EXPERT_SWIGLU;
+  const size_t T = c->T, d = c->d, E = c->E, k = c->top_k;
+  const size_t f = swi ? c->ffn : 0, r = swi ? 0 : c->rank;
   const size_t sf = (size_t)c->n_shared * c->ffn_shared, N = T * k;
   L.npad = (int)(((N + 64 * E) + 63) & ~(size_t)63);  // >= the sum of the padded group sizes
   L.tpad = (int)((T + 63) & ~(size_t)63);
@@ -636,7 +639,7 @@ BwdLayout bwd_layout(const moe_config_t *c) {
   L.wgut = take(E * d * 2 * f * 2);
   L.wsdt = take(sf * d * 2);
   L.wsgut = take(d * 2 * sf * 2);
-  L.ydt = take(d * 2 * np * 2);
+  L.ydt = take(d * (swi ? 2 : 3) * np * 2);
   L.ht = take(f * 2 * np * 2);
   L.dgut = take(2 * f * 2 * np * 2);
   L.xpt = take(d * 2 * np * 2);
@@ -644,6 +647,16 @@ BwdLayout bwd_layout(const moe_config_t *c) {
   L.ht_s = take(sf * 3 * tp * 2);
   L.dgut_s = take(2 * sf * 2 * tp * 2);
   L.xt_s = take(sf ? d * 2 * tp * 2 : 0);
+  L.z = take(N * r * 4);
+  L.dzs = take(N * r * 4);
+  L.dys = take(r ? N * 2 * d * 2 : 0);
+  L.dz2 = take(N * 2 * r * 2);
+  L.zs2 = take(N * 2 * r * 2);
+  L.ut = take(E * r * d * 2);
+  L.vt = take(E * d * r * 2);
+  L.dzt = take(r * 2 * np * 2);
+  L.zst = take(r * 3 * np * 2);
+  L.ds_part = take((np / 64) * r * 4);
   L.total = o;
   return L;
 }
@@ -694,7 +707,9 @@ moe_status_t expert_backward_impl(const moe_config_t *c, const void *x_perm,
                                   const moe_weights_t *w, const void *dy_perm, const float *dy,
                                   float *dx, const moe_grads_t *gr, void *ws, cudaStream_t st) {
   const BwdLayout L = bwd_layout(c);
-  const int T = c->T, d = c->d, E = c->E, k = c->top_k, f = c->ffn;
+  const bool swi = c->expert == MOE_EXPERT_SWIGLU;
+  const int T = c->T, d = c->d, E = c->E, k = c->top_k, f = swi ? c->ffn : 0;
+  const int r = swi ? 0 : c->rank;
   const int S = c->n_shared, fs = c->ffn_shared, sf = S * fs;
   const bool sh = S > 0;
   using bf = bf16_t;
@@ -710,23 +725,27 @@ moe_status_t expert_backward_impl(const moe_config_t *c, const void *x_perm,
      *Xpt = at<bf>(ws, L.xpt), *Ydts = at<bf>(ws, L.ydt_s), *Hts = at<bf>(ws, L.ht_s),
      *DGUts = at<bf>(ws, L.dgut_s), *Xts = at<bf>(ws, L.xt_s);
   const int np = L.npad, tp = L.tpad;
-  const bf *xp = (const bf *)x_perm, *xb = (const bf *)x, *dyp = (const bf *)dy_perm;
+  const bf *xp = (const bf *)x_perm, *xb = (const bf *)x;
 
   // padded group offsets of the weight gradients
   MOE_TRY(launch_pdl(pad_offsets_kernel, dim3(1), dim3(1024), 0, st, offsets, E, koff, T, off_s,
                      koff_s));
+  // the SwiGLU launches carry the routed SwiGLU experts (E groups) and / or the shared experts
   GroupedGemm base;
   std::memset(&base, 0, sizeof(base));
   base.offsets = offsets;
   base.T = T;
   base.rows_r = T * k;
-  base.E = E;
+  base.E = swi ? E : 0;
   base.has_shared = sh;
+  const bool swiglu_launch = swi || sh;
   // g and u (fp32) of the routed rows, and of every token for the shared experts
-  {
+  if (swiglu_launch) {
     GroupedGemm g = base;
-    g.A_r = x_perm; g.lda_r = d; g.B0_r = w->w_gate; g.B1_r = w->w_up; g.N_r = f; g.K_r = d;
-    g.out_r = GU; g.ldo_r = 2 * f; g.half_r = f;
+    if (swi) {
+      g.A_r = x_perm; g.lda_r = d; g.B0_r = w->w_gate; g.B1_r = w->w_up; g.N_r = f; g.K_r = d;
+      g.out_r = GU; g.ldo_r = 2 * f; g.half_r = f;
+    }
     if (sh) {
       g.A_s = x; g.lda_s = d; g.B0_s = w->ws_gate; g.B1_s = w->ws_up; g.N_s = sf; g.K_s = d;
       g.piece_k = d; g.b_rows_s = sf; g.out_s = GUs; g.ldo_s = 2 * sf; g.half_s = sf;
@@ -734,10 +753,12 @@ moe_status_t expert_backward_impl(const moe_config_t *c, const void *x_perm,
     MOE_TRY(launch_tc2<MODE_GATEUP_RAW>(g, st, K_BWD_GEMM));
   }
   // transposed weights: W_d [E][d][f] -> [E][f][d]; [W_g; W_u] -> [E][d][2f]; shared likewise
-  const bf *wg = (const bf *)w->w_gate, *wu = (const bf *)w->w_up, *wd = (const bf *)w->w_down;
-  MOE_TRY(launch_transpose_dense(wd, d, f, E, (size_t)d * f, Wdt, d, (size_t)f * d, 0, st));
-  MOE_TRY(launch_transpose_dense(wg, f, d, E, (size_t)f * d, Wgut, 2 * f, (size_t)d * 2 * f, 0, st));
-  MOE_TRY(launch_transpose_dense(wu, f, d, E, (size_t)f * d, Wgut, 2 * f, (size_t)d * 2 * f, f, st));
+  if (swi) {
+    const bf *wg = (const bf *)w->w_gate, *wu = (const bf *)w->w_up, *wd = (const bf *)w->w_down;
+    MOE_TRY(launch_transpose_dense(wd, d, f, E, (size_t)d * f, Wdt, d, (size_t)f * d, 0, st));
+    MOE_TRY(launch_transpose_dense(wg, f, d, E, (size_t)f * d, Wgut, 2 * f, (size_t)d * 2 * f, 0, st));
+    MOE_TRY(launch_transpose_dense(wu, f, d, E, (size_t)f * d, Wgut, 2 * f, (size_t)d * 2 * f, f, st));
+  }
   if (sh) {
     const bf *sg = (const bf *)w->ws_gate, *su = (const bf *)w->ws_up, *sdn = (const bf *)w->ws_down;
     MOE_TRY(launch_transpose_dense(sdn, d, fs, S, (size_t)d * fs, Wsdt, d, (size_t)fs * d, 0, st));
@@ -749,11 +770,13 @@ moe_status_t expert_backward_impl(const moe_config_t *c, const void *x_perm,
                        dim3(256), 0, st, dy, d, (size_t)T, dyb));
   }
   // dh = dY W_d with the SwiGLU backward in the epilogue: [dg | du] and h as hi + lo terms
-  {
+  if (swiglu_launch) {
     GroupedGemm g = base;
-    g.A_r = dy_perm; g.lda_r = d; g.B0_r = Wdt; g.N_r = f; g.K_r = d;
-    g.out_r = DGU; g.ldo_r = 4 * f; g.half_r = f; g.out2_r = H; g.ld2_r = 2 * f;
-    g.aux_r = GU; g.ldaux_r = 2 * f;
+    if (swi) {
+      g.A_r = dy_perm; g.lda_r = d; g.B0_r = Wdt; g.N_r = f; g.K_r = d;
+      g.out_r = DGU; g.ldo_r = 4 * f; g.half_r = f; g.out2_r = H; g.ld2_r = 2 * f;
+      g.aux_r = GU; g.ldaux_r = 2 * f;
+    }
     if (sh) {  // A = [dy_hi | dy_lo], K = 2d, the weight's k wraps over its d columns
       g.A_s = dyb; g.lda_s = 2 * d; g.B0_s = Wsdt; g.N_s = sf; g.K_s = 2 * d; g.piece_k = d;
       g.piece_rows = 0; g.b_rows_s = sf; g.out_s = DGUs; g.ldo_s = 4 * sf; g.half_s = sf;
@@ -762,34 +785,94 @@ moe_status_t expert_backward_impl(const moe_config_t *c, const void *x_perm,
     MOE_TRY(launch_tc2<MODE_SWIGLU_BWD>(g, st, K_BWD_GEMM));
   }
   // dX = [dg | du]_hi [W_g; W_u] + [dg | du]_lo [W_g; W_u] (fp32; K = 4 ffn, the weight's k
-  // wraps), then the un-permute: dx[t] = dX_s[t] + sum_j dX[pos(t, j)]
-  {
+  // wraps); the shared experts' dX likewise
+  if (swiglu_launch) {
     GroupedGemm g = base;
-    g.A_r = DGU; g.lda_r = 4 * f; g.B0_r = Wgut; g.N_r = d; g.K_r = 4 * f; g.kb_r = 2 * f;
-    g.out_r = dXp; g.ldo_r = d; g.out_r_bf16 = 0;
+    if (swi) {
+      g.A_r = DGU; g.lda_r = 4 * f; g.B0_r = Wgut; g.N_r = d; g.K_r = 4 * f; g.kb_r = 2 * f;
+      g.out_r = dXp; g.ldo_r = d; g.out_r_bf16 = 0;
+    }
     if (sh) {
       g.A_s = DGUs; g.lda_s = 4 * sf; g.B0_s = Wsgut; g.N_s = d; g.K_s = 4 * sf;
       g.piece_k = 2 * sf; g.piece_rows = 0; g.b_rows_s = d; g.out_s = dXs; g.ldo_s = d;
     }
     MOE_TRY(launch_tc2<MODE_PLAIN>(g, st, K_BWD_GEMM));
   }
+  if (!swi) {
+    // low-rank experts, Y = (z s) U^T with z = X V^T: dzs = dY U, dz = dzs s, ds = sum dzs z,
+    // dX = dz V, dV = dz^T X, dU = dY^T (z s). dY (fp32) and dz, z s run as hi + lo terms.
+    float *Z = at<float>(ws, L.z), *dZS = at<float>(ws, L.dzs), *dsp = at<float>(ws, L.ds_part);
+    bf *dYs = at<bf>(ws, L.dys), *DZ2 = at<bf>(ws, L.dz2), *ZS2 = at<bf>(ws, L.zs2);
+    bf *Ut = at<bf>(ws, L.ut), *Vt = at<bf>(ws, L.vt), *DZt = at<bf>(ws, L.dzt),
+       *ZSt = at<bf>(ws, L.zst);
+    const bf *V = (const bf *)w->lr_V, *U = (const bf *)w->lr_U;
+    GroupedGemm lr;
+    std::memset(&lr, 0, sizeof(lr));
+    lr.offsets = offsets;
+    lr.T = T;
+    lr.rows_r = T * k;
+    lr.E = E;
+    {  // z = X V^T (fp32)
+      GroupedGemm g = lr;
+      g.A_r = x_perm; g.lda_r = d; g.B0_r = V; g.N_r = r; g.K_r = d; g.out_r = Z; g.ldo_r = r;
+      MOE_TRY(launch_tc2<MODE_PLAIN>(g, st, K_BWD_GEMM));
+    }
+    MOE_TRY(launch_transpose_dense(U, d, r, E, (size_t)d * r, Ut, d, (size_t)r * d, 0, st));
+    MOE_TRY(launch_transpose_dense(V, r, d, E, (size_t)r * d, Vt, r, (size_t)d * r, 0, st));
+    MOE_TRY(launch_pdl(split_bf16_kernel,
+                       dim3((unsigned)std::min<long long>(ceil_div((long long)T * k * d, 1024), 65535)),
+                       dim3(256), 0, st, (const float *)dy_perm, d, (size_t)T * k, dYs));
+    {  // dzs = [dY_hi | dY_lo] U (K = 2d, U^T's k wraps over its d columns)
+      GroupedGemm g = lr;
+      g.A_r = dYs; g.lda_r = 2 * d; g.B0_r = Ut; g.N_r = r; g.K_r = 2 * d; g.kb_r = d;
+      g.out_r = dZS; g.ldo_r = r;
+      MOE_TRY(launch_tc2<MODE_PLAIN>(g, st, K_BWD_GEMM));
+    }
+    MOE_TRY(launch_pdl(lowrank_elem_kernel, dim3(np / 64), dim3(256), 0, st, (const float *)Z,
+                       (const float *)dZS, w->lr_s, offsets, koff, E, r, DZ2, ZS2, dsp));
+    MOE_TRY(launch_pdl(lowrank_ds_kernel, dim3(E), dim3(256), 0, st, (const float *)dsp, koff, r,
+                       gr->d_lr_s));
+    {  // dX = [dz_hi | dz_lo] V (K = 2r, V^T's k wraps over its r columns)
+      GroupedGemm g = lr;
+      g.A_r = DZ2; g.lda_r = 2 * r; g.B0_r = Vt; g.N_r = d; g.K_r = 2 * r; g.kb_r = r;
+      g.out_r = dXp; g.ldo_r = d;
+      MOE_TRY(launch_tc2<MODE_PLAIN>(g, st, K_BWD_GEMM));
+    }
+    const int nb2 = 2 * np / 64, nb3 = 3 * np / 64;
+    MOE_TRY(launch_transpose_grouped(2, DZ2, DZ2 + r, nullptr, r, 2 * r, offsets, koff, E, nb2,
+                                     DZt, 2 * np, st));
+    MOE_TRY(launch_transpose_grouped(2, xp, xp, nullptr, d, d, offsets, koff, E, nb2, Xpt, 2 * np, st));
+    MOE_TRY(launch_transpose_grouped(3, dYs, dYs, dYs + d, d, 2 * d, offsets, koff, E, nb3, Ydt,
+                                     3 * np, st));
+    MOE_TRY(launch_transpose_grouped(3, ZS2, ZS2 + r, ZS2, r, 2 * r, offsets, koff, E, nb3, ZSt,
+                                     3 * np, st));
+    MOE_TRY(launch_wgrad(E, koff, 2, DZt, r, Xpt, d, 2 * np, gr->d_lr_V, st));
+    MOE_TRY(launch_wgrad(E, koff, 3, Ydt, d, ZSt, r, 3 * np, gr->d_lr_U, st));
+    MOE_TRY(launch_pdl(zero_empty_experts_kernel, dim3(E, 8), dim3(256), 0, st, offsets,
+                       gr->d_lr_V, (size_t)r * d, gr->d_lr_U, (size_t)d * r, (float *)nullptr,
+                       (size_t)0));
+  }
+  // the un-permute: dx[t] = dX_s[t] + sum_j dX[pos(t, j)]
   MOE_TRY(launch_pdl(combine_kernel<float>, dim3(ceil_div(T, 8)), dim3(256), 0, st,
                      (const float *)dXp, sh ? (const float *)dXs : (const float *)nullptr,
                      slot_pos, (const float *)nullptr, dx, T, k, d, false));
-  // weight gradients: one operand as hi + lo segments, the other repeated, so that each product
-  // sums both terms: dW_d = dY^T (h_hi + h_lo), dW_g = (dg_hi + dg_lo)^T X, dW_u likewise
-  const int nb2 = 2 * np / 64;
-  MOE_TRY(launch_transpose_grouped(2, dyp, dyp, nullptr, d, d, offsets, koff, E, nb2, Ydt, 2 * np, st));
-  MOE_TRY(launch_transpose_grouped(2, H, H + f, nullptr, f, 2 * f, offsets, koff, E, nb2, Ht, 2 * np, st));
-  MOE_TRY(launch_transpose_grouped(2, DGU, DGU + 2 * f, nullptr, 2 * f, 4 * f, offsets, koff, E,
-                                   nb2, DGUt, 2 * np, st));
-  MOE_TRY(launch_transpose_grouped(2, xp, xp, nullptr, d, d, offsets, koff, E, nb2, Xpt, 2 * np, st));
-  MOE_TRY(launch_wgrad(E, koff, 2, Ydt, d, Ht, f, 2 * np, gr->d_w_down, st));
-  MOE_TRY(launch_wgrad(E, koff, 2, DGUt, f, Xpt, d, 2 * np, gr->d_w_gate, st));
-  MOE_TRY(launch_wgrad(E, koff, 2, DGUt + (size_t)f * 2 * np, f, Xpt, d, 2 * np, gr->d_w_up, st));
-  MOE_TRY(launch_pdl(zero_empty_experts_kernel, dim3(E, 8), dim3(256), 0, st, offsets,
-                     gr->d_w_gate, (size_t)f * d, gr->d_w_up, (size_t)f * d, gr->d_w_down,
-                     (size_t)d * f));
+  if (swi) {
+    // weight gradients: one operand as hi + lo segments, the other repeated, so that each
+    // product sums both terms: dW_d = dY^T (h_hi + h_lo), dW_g = (dg_hi + dg_lo)^T X, dW_u
+    const bf *dyp = (const bf *)dy_perm;
+    const int nb2 = 2 * np / 64;
+    MOE_TRY(launch_transpose_grouped(2, dyp, dyp, nullptr, d, d, offsets, koff, E, nb2, Ydt, 2 * np, st));
+    MOE_TRY(launch_transpose_grouped(2, H, H + f, nullptr, f, 2 * f, offsets, koff, E, nb2, Ht, 2 * np, st));
+    MOE_TRY(launch_transpose_grouped(2, DGU, DGU + 2 * f, nullptr, 2 * f, 4 * f, offsets, koff, E,
+                                     nb2, DGUt, 2 * np, st));
+    MOE_TRY(launch_transpose_grouped(2, xp, xp, nullptr, d, d, offsets, koff, E, nb2, Xpt, 2 * np, st));
+    MOE_TRY(launch_wgrad(E, koff, 2, Ydt, d, Ht, f, 2 * np, gr->d_w_down, st));
+    MOE_TRY(launch_wgrad(E, koff, 2, DGUt, f, Xpt, d, 2 * np, gr->d_w_gate, st));
+    MOE_TRY(launch_wgrad(E, koff, 2, DGUt + (size_t)f * 2 * np, f, Xpt, d, 2 * np, gr->d_w_up, st));
+    MOE_TRY(launch_pdl(zero_empty_experts_kernel, dim3(E, 8), dim3(256), 0, st, offsets,
+                       gr->d_w_gate, (size_t)f * d, gr->d_w_up, (size_t)f * d, gr->d_w_down,
+                       (size_t)d * f));
+  }
   if (sh) {
     // dW_sg, dW_su: (dg_hi + dg_lo)^T x; dW_sd: (dy_hi + dy_lo)^T (h_hi + h_lo) less lo lo,
     // three segments [hi hi | hi lo | lo hi]
@@ -971,12 +1054,15 @@ moe_status_t moe_expert_backward(const moe_config_t *cfg, const void *x_perm,
                                  float *dx, const moe_grads_t *g, void *ws, size_t ws_bytes,
                                  void *stream) {
   MOE_TRY(check_cfg(cfg));
-  if (cfg->dtype != MOE_DTYPE_BF16 || cfg->expert != MOE_EXPERT_SWIGLU) return MOE_ERR_UNSUPPORTED;
+  if (cfg->dtype != MOE_DTYPE_BF16) return MOE_ERR_UNSUPPORTED;
   MOE_TRY(check_weights(cfg, w, false, true));
   MOE_REQUIRE(g != nullptr);
   MOE_REQUIRE(tok16(cfg, x_perm) && aligned16(offsets) && tok16(cfg, slot_pos) && tok16(cfg, x) &&
               tok16(cfg, dy_perm) && tok16(cfg, dx));
-  MOE_REQUIRE(aligned16(g->d_w_gate) && aligned16(g->d_w_up) && aligned16(g->d_w_down));
+  if (cfg->expert == MOE_EXPERT_SWIGLU)
+    MOE_REQUIRE(aligned16(g->d_w_gate) && aligned16(g->d_w_up) && aligned16(g->d_w_down));
+  else
+    MOE_REQUIRE(aligned16(g->d_lr_V) && aligned16(g->d_lr_s) && aligned16(g->d_lr_U));
   MOE_REQUIRE(cfg->n_shared == 0 || (tok16(cfg, dy) && aligned16(g->d_ws_gate) &&
                                      aligned16(g->d_ws_up) && aligned16(g->d_ws_down)));
   MOE_REQUIRE(aligned16(ws));
@@ -984,10 +1070,17 @@ moe_status_t moe_expert_backward(const moe_config_t *cfg, const void *x_perm,
   cudaStream_t st = (cudaStream_t)stream;
   if (cfg->T == 0) {  // no rows: every gradient is zero
     const size_t E = cfg->E, f = cfg->ffn, d = cfg->d, sf = (size_t)cfg->n_shared * cfg->ffn_shared;
-    if (cudaMemsetAsync(g->d_w_gate, 0, E * f * d * 4, st) != cudaSuccess ||
-        cudaMemsetAsync(g->d_w_up, 0, E * f * d * 4, st) != cudaSuccess ||
-        cudaMemsetAsync(g->d_w_down, 0, E * f * d * 4, st) != cudaSuccess)
+    const size_t r = cfg->rank;
+    if (cfg->expert == MOE_EXPERT_SWIGLU) {
+      if (cudaMemsetAsync(g->d_w_gate, 0, E * f * d * 4, st) != cudaSuccess ||
+          cudaMemsetAsync(g->d_w_up, 0, E * f * d * 4, st) != cudaSuccess ||
+          cudaMemsetAsync(g->d_w_down, 0, E * f * d * 4, st) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    } else if (cudaMemsetAsync(g->d_lr_V, 0, E * r * d * 4, st) != cudaSuccess ||
+               cudaMemsetAsync(g->d_lr_s, 0, E * r * 4, st) != cudaSuccess ||
+               cudaMemsetAsync(g->d_lr_U, 0, E * d * r * 4, st) != cudaSuccess) {
       return MOE_ERR_CUDA;
+    }
     if (sf && (cudaMemsetAsync(g->d_ws_gate, 0, sf * d * 4, st) != cudaSuccess ||
                cudaMemsetAsync(g->d_ws_up, 0, sf * d * 4, st) != cudaSuccess ||
                cudaMemsetAsync(g->d_ws_down, 0, sf * d * 4, st) != cudaSuccess))

@@ -201,15 +201,21 @@ size_t moe_backward_workspace_size(const moe_config_t *cfg);
  *   dh = dY_e W_d[e];  du = dh * silu(g);  dg = dh * u * silu'(g);  h = silu(g) * u
  *   d_w_down[e] = dY_e^T h;  d_w_gate[e] = dg^T X_e;  d_w_up[e] = du^T X_e
  *   dX_e = dg W_g[e] + du W_u[e]
+ * Low-rank expert (dormouse, "TSCT low-rank experts"), z = X_e V[e]^T, Y = (z * s) U[e]^T:
+ *   dzs = dY_e U[e];  d_lr_s[e] = sum over rows of dzs * z;  dz = dzs * s;
+ *   d_lr_V[e] = dz^T X_e;  d_lr_U[e] = dY_e^T (z * s);  dX_e = dz V[e]
  * and likewise for the shared experts on all T tokens with upstream gradient dy. Then
  *   dx[t] = dX_shared[t] + sum over the token's kept pairs (t, j) of dX[slot_pos[t, j]]
  * (the experts' part of the input gradient; the router's part comes from moe_route_backward).
  * x_perm, offsets, slot_pos: as moe_permute produced them; x: the layer input; dy_perm: [T*k, d]
- * in y_perm's dtype, rows of kept pairs from moe_combine_backward; dy: [T, d] fp32 (used for the
- * shared experts, may be NULL when n_shared = 0); dx: [T, d] fp32 output. g and u are recomputed
- * in bf16 and dg, du, h rounded to bf16 (the next products' operands); every product accumulates
- * in fp32 in a fixed order (bitwise reproducible). Experts with no rows get zero gradients.
- * Supported: bf16 layers with SwiGLU experts; other configurations return MOE_ERR_UNSUPPORTED.
+ * in y_perm's dtype (bf16 for SwiGLU, fp32 for low-rank layers), rows of kept pairs from
+ * moe_combine_backward; dy: [T, d] fp32 (used for the shared experts, may be NULL when
+ * n_shared = 0); dx: [T, d] fp32 output. g and u are recomputed in fp32; every product
+ * accumulates in fp32 in a fixed order (bitwise reproducible). Experts with no rows get zero gradients.
+ * Operands that are not exact bf16 values (g, u, dg, du, h, z, dz, z s, the fp32 dy and the
+ * low-rank layers' fp32 dy_perm) enter the tensor-core products as two bf16 terms, value and
+ * rounding residual, so each gradient carries no single bf16 rounding of its operands.
+ * Supported: bf16 layers (SwiGLU or low-rank experts); fp32 layers return MOE_ERR_UNSUPPORTED.
  * ws: moe_backward_workspace_size(cfg) bytes of the caller's device memory. Asynchronous. */
 moe_status_t moe_expert_backward(const moe_config_t *cfg, const void *x_perm,
                                  const int32_t *offsets, const int32_t *slot_pos, const void *x,

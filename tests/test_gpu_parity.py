@@ -287,15 +287,21 @@ def test_route_and_combine_backward(name):
 # experts, norm_topk, capacity drops (heavy ones too), one token, one expert, k = E, wide and
 # narrow hidden sizes, widths that are not multiples of 256, and 97 experts (T < E: empty ones)
 EXPERT_BACKWARD = ["quartz_s", "capacity_s", "sigmoid_s", "norm_softmax", "heavy_drops",
-                   "three_shared", "T1", "T33", "k_eq_E", "E1k1", "k8_E97", "d4096"]
+                   "three_shared", "T1", "T33", "k_eq_E", "E1k1", "k8_E97", "d4096",
+                   "lowrank_s", "lowrank_shared", "lowrank_E1024"]
 
 
 def _expert_grads(c, run):
     E, d, S = run.cfg.E, run.cfg.d, c.n_shared
-    f, fs, dev = c.ffn, c.ffn_shared, run.dev
-    g = dict(d_w_gate=torch.empty((E, f, d), dtype=torch.float32, device=dev),
-             d_w_up=torch.empty((E, f, d), dtype=torch.float32, device=dev),
-             d_w_down=torch.empty((E, d, f), dtype=torch.float32, device=dev))
+    f, fs, r, dev = c.ffn, c.ffn_shared, c.rank, run.dev
+    if c.expert == "swiglu":
+        g = dict(d_w_gate=torch.empty((E, f, d), dtype=torch.float32, device=dev),
+                 d_w_up=torch.empty((E, f, d), dtype=torch.float32, device=dev),
+                 d_w_down=torch.empty((E, d, f), dtype=torch.float32, device=dev))
+    else:
+        g = dict(d_lr_V=torch.empty((E, r, d), dtype=torch.float32, device=dev),
+                 d_lr_s=torch.empty((E, r), dtype=torch.float32, device=dev),
+                 d_lr_U=torch.empty((E, d, r), dtype=torch.float32, device=dev))
     if S:
         g.update(d_ws_gate=torch.empty((S, fs, d), dtype=torch.float32, device=dev),
                  d_ws_up=torch.empty((S, fs, d), dtype=torch.float32, device=dev),
@@ -315,15 +321,22 @@ def _expert_step_reference(c, inp, dy_perm, dy):
     x = np.asarray(inp["x"], np.float64)
     Xp = x[src]
     dYp = np.asarray(dy_perm, np.float64)[:N]
-    out = {n: np.zeros(np.asarray(inp[n[2:]]).shape) for n in ("d_w_gate", "d_w_up", "d_w_down")}
+    names = (("d_w_gate", "d_w_up", "d_w_down") if c.expert == "swiglu" else
+             ("d_lr_V", "d_lr_s", "d_lr_U"))
+    out = {n: np.zeros(np.asarray(inp[n[2:]]).shape) for n in names}
     dXp = np.zeros((N, x.shape[1]))
     for e in range(c.E):
         a, b = int(offs[e]), int(offs[e + 1])
         if a == b:
             continue
-        g = BW.swiglu_backward(Xp[a:b], inp["w_gate"][e], inp["w_up"][e], inp["w_down"][e],
-                               dYp[a:b])
-        out["d_w_gate"][e], out["d_w_up"][e], out["d_w_down"][e] = g["dWg"], g["dWu"], g["dWd"]
+        if c.expert == "swiglu":
+            g = BW.swiglu_backward(Xp[a:b], inp["w_gate"][e], inp["w_up"][e], inp["w_down"][e],
+                                   dYp[a:b])
+            out["d_w_gate"][e], out["d_w_up"][e], out["d_w_down"][e] = g["dWg"], g["dWu"], g["dWd"]
+        else:
+            g = BW.lowrank_backward(Xp[a:b], inp["lr_V"][e], inp["lr_s"][e], inp["lr_U"][e],
+                                    dYp[a:b])
+            out["d_lr_V"][e], out["d_lr_s"][e], out["d_lr_U"][e] = g["dV"], g["ds"], g["dU"]
         dXp[a:b] = g["dX"]
     dx = np.zeros_like(x)
     np.add.at(dx, src, dXp)
@@ -388,8 +401,8 @@ def test_expert_backward(name):
 
 
 def test_expert_backward_unsupported_configurations():
-    """fp32 layers and low-rank experts are refused on the host (MOE_ERR_UNSUPPORTED)."""
-    for c in (get_config("tiny_f32"), get_config("lowrank", T=64, E=16)):
+    """fp32 layers are refused on the host (MOE_ERR_UNSUPPORTED)."""
+    for c in (get_config("tiny_f32"), EDGE["f32_sigmoid_cap"]):
         cfg = B.make_config(T=c.T, d=c.d, E=c.E, top_k=c.top_k, n_shared=c.n_shared, ffn=c.ffn,
                             ffn_shared=c.ffn_shared, rank=c.rank, expert=c.expert, dtype=c.dtype)
         with pytest.raises(B.MoEError) as ei:
