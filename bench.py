@@ -572,9 +572,9 @@ def measure_config(name, K, W, dev, flush, stream, peaks, peak_src):
 
 
 def backward_parts(c, cfg, layer, x, flush, stream, K, peaks):
-    """The backward steps the library has so far (combine, router), each call timed alone with
-    CUDA events on the forward's resident outputs and a seeded upstream gradient, L2 flushed
-    between calls. Not part of the step above."""
+    """The backward's entry points (combine, experts, router), each call timed alone with CUDA
+    events on the forward's resident outputs and a seeded upstream gradient, L2 flushed between
+    calls. Not part of the step above."""
     import torch
 
     from fine_grained_mixture_moe_b200 import binding as B
@@ -623,6 +623,31 @@ def backward_parts(c, cfg, layer, x, flush, stream, K, peaks):
     us_c = timed_call(lambda: B.moe_combine_backward(cfg, dy, yp, slot, wts, dyp, d_w))
     us_r = timed_call(lambda: B.moe_route_backward(cfg, x, layer.wstruct, idx, cnt, d_w, 1.0,
                                                    d_logits, d_wr, dx))
+    # the experts' backward: data and weight gradients of every routed and shared expert
+    E_, f_, r_, S_, fs_ = c.E, c.ffn, c.rank, c.n_shared, c.ffn_shared
+    if c.expert == "swiglu":
+        gr = {"d_w_gate": torch.empty((E_, f_, d), dtype=torch.float32, device=dev),
+              "d_w_up": torch.empty((E_, f_, d), dtype=torch.float32, device=dev),
+              "d_w_down": torch.empty((E_, d, f_), dtype=torch.float32, device=dev)}
+        flop_e = 16.0 * d * f_ * N
+    else:
+        gr = {"d_lr_V": torch.empty((E_, r_, d), dtype=torch.float32, device=dev),
+              "d_lr_s": torch.empty((E_, r_), dtype=torch.float32, device=dev),
+              "d_lr_U": torch.empty((E_, d, r_), dtype=torch.float32, device=dev)}
+        flop_e = 10.0 * d * r_ * N
+    if S_:
+        gr.update(d_ws_gate=torch.empty((S_, fs_, d), dtype=torch.float32, device=dev),
+                  d_ws_up=torch.empty((S_, fs_, d), dtype=torch.float32, device=dev),
+                  d_ws_down=torch.empty((S_, d, fs_), dtype=torch.float32, device=dev))
+        flop_e += 16.0 * d * S_ * fs_ * T
+    bws = B.moe_backward_workspace_size(cfg)
+    bw_ws = torch.empty(bws, dtype=torch.uint8, device=dev)
+    dx_e = torch.empty((T, d), dtype=torch.float32, device=dev)
+    gstruct = B.make_grads(gr)
+    us_e = timed_call(lambda: B.moe_expert_backward(cfg, xp, offsets, slot, x, layer.wstruct, dyp,
+                                                    dy if S_ else None, dx_e, gstruct, bw_ws,
+                                                    bws))
+    del bw_ws
     st, info = B.moe_get_device_error()
     if st != 0:
         raise RuntimeError(f"device error in the backward pass: {B.status_str(st)} info={info}")
@@ -638,6 +663,12 @@ def backward_parts(c, cfg, layer, x, flush, stream, K, peaks):
         "combine_backward": {"avg_us": round(us_c, 2), "bound": "hbm", "bytes": bytes_c,
                              "achieved_gbs": round(bytes_c / us_c / 1e3, 1),
                              "frac": round(bytes_c / us_c / 1e3 / hbm, 4)},
+        "expert_backward": {"avg_us": round(us_e, 2), "bound": "tensor", "flop": flop_e,
+                            "achieved_tflops": round(flop_e / us_e / 1e6, 1),
+                            "frac": round(flop_e / us_e / 1e6 / peaks["bf16_tflops"], 4),
+                            "note": "algorithmic flops: g and u recomputed, dh, dX, the three "
+                                    "weight gradients (routed and shared); the kernels run "
+                                    "the non-bf16 operands as two bf16 terms"},
         "route_backward": {"avg_us": round(us_r, 2), "bound": "alu", "flop": flop_r,
                            "achieved_tflops": round(flop_r / us_r / 1e6, 3),
                            "frac": round(flop_r / us_r / 1e6 / fp32, 4), "bytes": bytes_r,

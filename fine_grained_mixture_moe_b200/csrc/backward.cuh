@@ -258,11 +258,13 @@ __global__ void __launch_bounds__(256) router_dgrad_kernel(const float *__restri
 // gradients (dh = dY W_d, dX = [dg | du] [W_g; W_u]) the same way.
 
 // koff[e] = sum over e' < e of the expert's row count rounded up to 64; koff[E] is the total.
-// Also the one-group tables of the shared experts' T rows: off_s = {0, T}, koff_s = {0, T
-// rounded up to 64}. One block; E <= 1024.
+// Also the group tables of the shared experts' T rows cut into nc chunks of ch rows (ch a
+// multiple of 64): off_s[i] = min(i ch, T), koff_s[i] = the same rounded up to 64. One block;
+// E <= 1024, nc <= 64.
 __global__ void __launch_bounds__(1024) pad_offsets_kernel(const int32_t *__restrict__ offsets,
                                                            int E, int32_t *__restrict__ koff,
-                                                           int T, int32_t *__restrict__ off_s,
+                                                           int T, int nc, int ch,
+                                                           int32_t *__restrict__ off_s,
                                                            int32_t *__restrict__ koff_s) {
   griddep_wait();
   griddep_launch();
@@ -273,35 +275,39 @@ __global__ void __launch_bounds__(1024) pad_offsets_kernel(const int32_t *__rest
   __syncthreads();
   const int total = block_excl_scan_inplace(s, 1024, tmp);
   if (e < E) koff[e] = s[e];
-  if (e == 0) {
-    koff[E] = total;
-    off_s[0] = 0;
-    off_s[1] = T;
-    koff_s[0] = 0;
-    koff_s[1] = (T + 63) & ~63;
+  if (e == 0) koff[E] = total;
+  if (e <= nc) {
+    const int v = min(e * ch, T);
+    off_s[e] = v;
+    koff_s[e] = (v + 63) & ~63;
   }
 }
 
-// Tiled transpose to bf16 through shared memory, 64 x 64 per CTA:
+// Tiled bf16 transpose through shared memory: a CTA moves 64 input rows x 128 input columns
+// (16 KB) with 16-byte loads and stores.
 //   grouped (in_offsets != null): group g's rows offsets[g] .. offsets[g+1] of the sources
 //     [rows, C] (row stride ldi) go to nseg segments of columns of out [C, ldo]: segment s
 //     spans columns nseg koff[g] + s P .. + P, P = koff[g+1] - koff[g] (the group's row count
 //     rounded up to 64), and holds the rows of source s, zeros past the group's rows
 //     (blockIdx.y runs over 64-column blocks of out, blockIdx.z = 0);
 //   dense: batch b = blockIdx.z, in0 + b * ibs is [R, C] (row stride ldi) and goes to
-//     out + b * obs + col0 as [C, R] with row stride ldo; blockIdx.y runs over 64-row blocks.
-template <typename Tin>
+//     out + b * obs + col0 as [C, R] with row stride ldo; blockIdx.y runs over 64-row blocks
+//     (R a multiple of 8).
+// C and ldi are multiples of 64, ldo of 8; pointers 16-byte aligned.
+constexpr int TR_COLS = 128;
 __global__ void __launch_bounds__(256) transpose_bf16_kernel(
-    const Tin *__restrict__ in0, const Tin *__restrict__ in1, const Tin *__restrict__ in2,
-    int nseg, int C, int ldi, const int32_t *__restrict__ in_offsets,
-    const int32_t *__restrict__ koff, int G, int R, size_t ibs, __nv_bfloat16 *__restrict__ out,
-    int ldo, size_t obs, int col0) {
+    const __nv_bfloat16 *__restrict__ in0, const __nv_bfloat16 *__restrict__ in1,
+    const __nv_bfloat16 *__restrict__ in2, int nseg, int C, int ldi,
+    const int32_t *__restrict__ in_offsets, const int32_t *__restrict__ koff, int G, int R,
+    size_t ibs, __nv_bfloat16 *__restrict__ out, int ldo, size_t obs, int col0) {
   griddep_wait();
   griddep_launch();
-  __shared__ float tile[64][65];
-  const int c0 = blockIdx.x * 64;
+  // [64][128] with the 16-byte chunk index of row r XORed with (r / 8) % 8: the store phase
+  // reads rows 8 apart, which then fall in different banks
+  __shared__ __align__(16) __nv_bfloat16 tile[64][TR_COLS];
+  const int c0 = blockIdx.x * TR_COLS;
   int r_in0, n_rows, o_col0;  // first input row, valid rows of the block, first output column
-  const Tin *src = in0;
+  const __nv_bfloat16 *src = in0;
   __nv_bfloat16 *dst = out;
   if (in_offsets) {
     const int p0 = blockIdx.y * 64;  // column block of out
@@ -326,17 +332,48 @@ __global__ void __launch_bounds__(256) transpose_bf16_kernel(
     n_rows = max(0, min(64, R - r_in0));
     o_col0 = r_in0;
   }
-  const int tx = threadIdx.x & 63, ty = threadIdx.x >> 6;  // 64 x 4
-  for (int r = ty; r < 64; r += 4) {
-    float v = 0.0f;
-    if (r < n_rows && c0 + tx < C) v = Elem<Tin>::to_f(src[(size_t)(r_in0 + r) * ldi + c0 + tx]);
-    tile[r][tx] = v;
+  const int ncols = min(TR_COLS, C - c0);  // 64 or 128
+  // load: 64 rows x 16 vectors of 8 columns, zeros past the valid rows
+  for (int q = threadIdx.x; q < 64 * (TR_COLS / 8); q += 256) {
+    const int r = q >> 4, v = q & 15;
+    uint4 val = make_uint4(0u, 0u, 0u, 0u);
+    if (r < n_rows && v * 8 < ncols)
+      val = *(const uint4 *)(src + (size_t)(r_in0 + r) * ldi + c0 + v * 8);
+    *(uint4 *)&tile[r][(v ^ ((r >> 3) & 7)) * 8] = val;
   }
   __syncthreads();
+  // store: output row c (an input column) takes 8 vectors of 8 input rows
   const int n_out = in_offsets ? 64 : n_rows;  // grouped: the padding columns are written too
-  for (int c = ty; c < 64; c += 4)
-    if (c0 + c < C && tx < n_out)
-      dst[(size_t)(c0 + c) * ldo + o_col0 + tx] = __float2bfloat16_rn(tile[tx][c]);
+  for (int q = threadIdx.x; q < TR_COLS * 8; q += 256) {
+    const int c = q >> 3, v = q & 7;
+    if (c >= ncols || v * 8 >= n_out) continue;
+    uint32_t w[4];
+    const int cx = (((c >> 3) ^ v) << 3) + (c & 7);  // rows v*8 .. v*8+7 share (r / 8) % 8 = v
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const __nv_bfloat16 a = tile[v * 8 + 2 * i][cx], b = tile[v * 8 + 2 * i + 1][cx];
+      w[i] = (uint32_t)__bfloat16_as_ushort(a) | ((uint32_t)__bfloat16_as_ushort(b) << 16);
+    }
+    *(uint4 *)(dst + (size_t)(c0 + c) * ldo + o_col0 + v * 8) = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+}
+
+// out[i] = sum over c < nc of part[c][i], in chunk order (partial weight gradients of chunks).
+__global__ void __launch_bounds__(256) sum_chunks_kernel(const float *__restrict__ part, int nc,
+                                                         size_t n, float *__restrict__ out) {
+  griddep_wait();
+  griddep_launch();
+  for (size_t i = ((size_t)blockIdx.x * 256 + threadIdx.x) * 4; i < n; i += (size_t)gridDim.x * 1024) {
+    float4 a = *(const float4 *)(part + i);
+    for (int c = 1; c < nc; ++c) {
+      const float4 b = *(const float4 *)(part + (size_t)c * n + i);
+      a.x += b.x;
+      a.y += b.y;
+      a.z += b.z;
+      a.w += b.w;
+    }
+    *(float4 *)(out + i) = a;
+  }
 }
 
 // Rows of in [rows, d] (fp32) as two bf16 terms: out[r] = [hi (d) | lo (d)], hi = bf16(v),

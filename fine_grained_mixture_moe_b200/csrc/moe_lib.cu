@@ -602,14 +602,18 @@ moe_status_t route_backward_impl(const moe_config_t *c, const RouteBwdArgs &a, f
 // and h as hi + lo bf16 terms, the routed dX before the un-permute, the shared experts'
 // counterparts, dy as hi + lo terms, the transposed weights and the transposed, per-expert
 // zero-padded activations of the weight gradients (2 or 3 K segments per group).
+constexpr int BWD_SHARED_CHUNKS = 8;
+
 struct BwdLayout {
   size_t koff, off_s, koff_s;
   size_t gu, dgu, h, dxp, gu_s, dgu_s, h_s, dx_s, dy_b;
   size_t wdt, wgut, wsdt, wsgut;
   size_t ydt, ht, dgut, xpt, ydt_s, ht_s, dgut_s, xt_s;
   size_t z, dzs, dys, dz2, zs2, ut, vt, dzt, zst, ds_part;  // low-rank experts
+  size_t part_s;  // the shared experts' weight gradients per token chunk
   size_t total;
   int npad, tpad;
+  int nc, ch;     // token chunks of the shared experts' weight gradients, rows per chunk
 };
 
 BwdLayout bwd_layout(const moe_config_t *c) {
@@ -619,13 +623,17 @@ BwdLayout bwd_layout(const moe_config_t *c) {
   const size_t f = swi ? c->ffn : 0, r = swi ? 0 : c->rank;
   const size_t sf = (size_t)c->n_shared * c->ffn_shared, N = T * k;
   L.npad = (int)(((N + 64 * E) + 63) & ~(size_t)63);  // >= the sum of the padded group sizes
-  L.tpad = (int)((T + 63) & ~(size_t)63);
+  // the shared experts' T rows in nc chunks of ch rows, so that their weight gradients (few
+  // output tiles, long K) fill the GPU; the chunks' partial sums are added in chunk order
+  L.nc = std::max(1, std::min(BWD_SHARED_CHUNKS, ceil_div((long long)T, 512)));
+  L.ch = (int)(((size_t)ceil_div((long long)std::max<size_t>(T, 1), L.nc) + 63) & ~(size_t)63);
+  L.tpad = (int)(((T + 63) & ~(size_t)63) + 64 * (size_t)L.nc);
   const size_t np = L.npad, tp = L.tpad;
   size_t o = 0;
   auto take = [&](size_t bytes) { size_t at = o; o = align256(o + std::max<size_t>(bytes, 1)); return at; };
   L.koff = take((E + 1) * 4);
-  L.off_s = take(8);
-  L.koff_s = take(8);
+  L.off_s = take((BWD_SHARED_CHUNKS + 1) * 4);
+  L.koff_s = take((BWD_SHARED_CHUNKS + 1) * 4);
   L.gu = take(N * 2 * f * 4);
   L.dgu = take(N * 4 * f * 2);
   L.h = take(N * 2 * f * 2);
@@ -657,6 +665,7 @@ BwdLayout bwd_layout(const moe_config_t *c) {
   L.dzt = take(r * 2 * np * 2);
   L.zst = take(r * 3 * np * 2);
   L.ds_part = take((np / 64) * r * 4);
+  L.part_s = take(sf ? (size_t)L.nc * std::max(sf * d, d * (size_t)c->ffn_shared) * 4 : 0);
   L.total = o;
   return L;
 }
@@ -669,13 +678,13 @@ moe_status_t launch_transpose_grouped(int nseg, const bf16_t *s0, const bf16_t *
                                       const bf16_t *s2, int C, int ldi, const int32_t *offsets,
                                       const int32_t *koff, int G, int ncolblocks, void *out,
                                       int ldo, cudaStream_t st) {
-  return launch_pdl(transpose_bf16_kernel<bf16_t>, dim3(C / 64, ncolblocks, 1), dim3(256), 0, st,
+  return launch_pdl(transpose_bf16_kernel, dim3(ceil_div(C, TR_COLS), ncolblocks, 1), dim3(256), 0, st,
                     s0, s1, s2, nseg, C, ldi, offsets, koff, G, 0, (size_t)0, (bf16_t *)out, ldo,
                     (size_t)0, 0);
 }
 moe_status_t launch_transpose_dense(const bf16_t *in, int R, int C, int batches, size_t ibs,
                                     void *out, int ldo, size_t obs, int col0, cudaStream_t st) {
-  return launch_pdl(transpose_bf16_kernel<bf16_t>, dim3(C / 64, ceil_div(R, 64), batches),
+  return launch_pdl(transpose_bf16_kernel, dim3(ceil_div(C, TR_COLS), ceil_div(R, 64), batches),
                     dim3(256), 0, st, in, (const bf16_t *)nullptr, (const bf16_t *)nullptr, 1, C,
                     C, (const int32_t *)nullptr, (const int32_t *)nullptr, 0, R, ibs,
                     (bf16_t *)out, ldo, obs, col0);
@@ -728,8 +737,8 @@ moe_status_t expert_backward_impl(const moe_config_t *c, const void *x_perm,
   const bf *xp = (const bf *)x_perm, *xb = (const bf *)x;
 
   // padded group offsets of the weight gradients
-  MOE_TRY(launch_pdl(pad_offsets_kernel, dim3(1), dim3(1024), 0, st, offsets, E, koff, T, off_s,
-                     koff_s));
+  MOE_TRY(launch_pdl(pad_offsets_kernel, dim3(1), dim3(1024), 0, st, offsets, E, koff, T, L.nc,
+                     L.ch, off_s, koff_s));
   // the SwiGLU launches carry the routed SwiGLU experts (E groups) and / or the shared experts
   GroupedGemm base;
   std::memset(&base, 0, sizeof(base));
@@ -875,21 +884,31 @@ moe_status_t expert_backward_impl(const moe_config_t *c, const void *x_perm,
   }
   if (sh) {
     // dW_sg, dW_su: (dg_hi + dg_lo)^T x; dW_sd: (dy_hi + dy_lo)^T (h_hi + h_lo) less lo lo,
-    // three segments [hi hi | hi lo | lo hi]
+    // three segments [hi hi | hi lo | lo hi]; each over the nc token chunks, then the chunks'
+    // partial sums added in order
+    const int nc = L.nc;
+    float *part = at<float>(ws, L.part_s);
+    auto sum_chunks = [&](size_t n, float *out) {
+      return launch_pdl(sum_chunks_kernel, dim3((unsigned)std::min<long long>(ceil_div((long long)n, 1024), 4096)),
+                        dim3(256), 0, st, (const float *)part, nc, n, out);
+    };
     MOE_TRY(launch_transpose_grouped(2, DGUs, DGUs + 2 * sf, nullptr, 2 * sf, 4 * sf, off_s,
-                                     koff_s, 1, 2 * tp / 64, DGUts, 2 * tp, st));
-    MOE_TRY(launch_transpose_grouped(2, xb, xb, nullptr, d, d, off_s, koff_s, 1, 2 * tp / 64, Xts,
+                                     koff_s, nc, 2 * tp / 64, DGUts, 2 * tp, st));
+    MOE_TRY(launch_transpose_grouped(2, xb, xb, nullptr, d, d, off_s, koff_s, nc, 2 * tp / 64, Xts,
                                      2 * tp, st));
-    MOE_TRY(launch_transpose_grouped(3, dyb, dyb, dyb + d, d, 2 * d, off_s, koff_s, 1,
+    MOE_TRY(launch_transpose_grouped(3, dyb, dyb, dyb + d, d, 2 * d, off_s, koff_s, nc,
                                      3 * tp / 64, Ydts, 3 * tp, st));
-    MOE_TRY(launch_transpose_grouped(3, Hs, Hs + sf, Hs, sf, 2 * sf, off_s, koff_s, 1,
+    MOE_TRY(launch_transpose_grouped(3, Hs, Hs + sf, Hs, sf, 2 * sf, off_s, koff_s, nc,
                                      3 * tp / 64, Hts, 3 * tp, st));
-    MOE_TRY(launch_wgrad(1, koff_s, 2, DGUts, sf, Xts, d, 2 * tp, gr->d_ws_gate, st));
-    MOE_TRY(launch_wgrad(1, koff_s, 2, DGUts + (size_t)sf * 2 * tp, sf, Xts, d, 2 * tp,
-                         gr->d_ws_up, st));
-    for (int s = 0; s < S; ++s)
-      MOE_TRY(launch_wgrad(1, koff_s, 3, Ydts, d, Hts + (size_t)s * fs * 3 * tp, fs, 3 * tp,
-                           gr->d_ws_down + (size_t)s * d * fs, st));
+    MOE_TRY(launch_wgrad(nc, koff_s, 2, DGUts, sf, Xts, d, 2 * tp, part, st));
+    MOE_TRY(sum_chunks((size_t)sf * d, gr->d_ws_gate));
+    MOE_TRY(launch_wgrad(nc, koff_s, 2, DGUts + (size_t)sf * 2 * tp, sf, Xts, d, 2 * tp, part, st));
+    MOE_TRY(sum_chunks((size_t)sf * d, gr->d_ws_up));
+    for (int s = 0; s < S; ++s) {
+      MOE_TRY(launch_wgrad(nc, koff_s, 3, Ydts, d, Hts + (size_t)s * fs * 3 * tp, fs, 3 * tp, part,
+                           st));
+      MOE_TRY(sum_chunks((size_t)d * fs, gr->d_ws_down + (size_t)s * d * fs));
+    }
   }
   return MOE_OK;
 }
