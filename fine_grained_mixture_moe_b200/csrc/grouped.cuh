@@ -71,19 +71,29 @@ struct GroupedGemm {
   int kseg;                // K segments per group (kgroup)
 };
 
-// Tile counts per group and their exclusive prefix in shared memory (all threads call).
+// Tile list order: the shared group (its K may be several experts' widths: the longest tiles)
+// first, then the routed groups, so that the last wave holds short tiles. Position o of the
+// order is group group_at(p, o).
+__device__ __forceinline__ int group_at(const GroupedGemm &p, int o) {
+  if (!p.has_shared) return o;
+  return o == 0 ? p.E : o - 1;
+}
+
+// Tile counts per group and their exclusive prefix (in tile-list order) in shared memory (all
+// threads call).
 __device__ __forceinline__ int build_tile_prefix(const GroupedGemm &p, int BM, int BN,
                                                  int *prefix, int *tmp) {
   const int G = p.E + p.has_shared;
   const int ntr = (p.N_r + BN - 1) / BN, nts = (p.N_s + BN - 1) / BN;
-  for (int g = threadIdx.x; g < G; g += blockDim.x) {
+  for (int o = threadIdx.x; o < G; o += blockDim.x) {
     if (p.kgroup) {
-      const int kg = p.kseg * (p.koff[g + 1] - p.koff[g]);
-      prefix[g] = kg > 0 ? ((p.rows_r + BM - 1) / BM) * ntr : 0;
+      const int kg = p.kseg * (p.koff[o + 1] - p.koff[o]);
+      prefix[o] = kg > 0 ? ((p.rows_r + BM - 1) / BM) * ntr : 0;
       continue;
     }
+    const int g = group_at(p, o);
     const int rows = g < p.E ? (p.offsets[g + 1] - p.offsets[g]) : p.T;
-    prefix[g] = ((rows + BM - 1) / BM) * (g < p.E ? ntr : nts);
+    prefix[o] = ((rows + BM - 1) / BM) * (g < p.E ? ntr : nts);
   }
   __syncthreads();
   const int total = block_excl_scan_inplace(prefix, G, tmp);
@@ -109,12 +119,13 @@ __device__ __forceinline__ TileInfo decode_tile(const GroupedGemm &p, int tile,
     else hi = mid - 1;
   }
   TileInfo ti;
+  const int local = tile - prefix[lo];
+  lo = p.kgroup ? lo : group_at(p, lo);  // list position -> group
   ti.g = lo;
   const bool routed = lo < p.E;
   ti.N = routed ? p.N_r : p.N_s;
   ti.K = routed ? p.K_r : p.K_s;
   const int nt = (ti.N + BN - 1) / BN;
-  const int local = tile - prefix[lo];
   ti.m0 = (local / nt) * BM;
   ti.n0 = (local % nt) * BN;
   ti.kofs = 0;
