@@ -302,17 +302,32 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TC_THREADS, 1)
           uint32_t r0[32];
           tmem_ld32(tbase + c, r0);
           if (MODE == MODE_GATEUP_RAW) {
+            // g then u (fp32), each staged per warp (32 rows x 32 columns) and written as 32
+            // coalesced 128-byte row pieces
             uint32_t r1[32];
             tmem_ld32(tbase + BN + c, r1);
             tmem_wait_ld();
-            if (row_ok && col < ti.N) {
-              float *o = (float *)out + (size_t)(ti.out_row0 + row) * ldo + col;
+            unsigned char *stg = stg_all + (warp - 2) * 4096;
+            const int nrows = min(32, ti.rows - rbase);
+#pragma unroll 1
+            for (int part = 0; part < 2; ++part) {
+              const uint32_t *rv = part ? r1 : r0;
 #pragma unroll
-              for (int i = 0; i < 8; ++i) {
-                ((uint4 *)o)[i] = make_uint4(r0[4 * i], r0[4 * i + 1], r0[4 * i + 2], r0[4 * i + 3]);
-                ((uint4 *)(o + hf))[i] =
-                    make_uint4(r1[4 * i], r1[4 * i + 1], r1[4 * i + 2], r1[4 * i + 3]);
+              for (int i = 0; i < 8; ++i)
+                *(uint4 *)(stg + lane * 128 + ((i ^ (lane & 7)) << 4)) =
+                    make_uint4(rv[4 * i], rv[4 * i + 1], rv[4 * i + 2], rv[4 * i + 3]);
+              __syncwarp();
+              if (col < ti.N) {
+                unsigned char *obase = (unsigned char *)out +
+                                       ((size_t)(ti.out_row0 + rbase) * ldo + col + part * hf) * 4;
+                const size_t row_bytes = (size_t)ldo * 4;
+                for (int rr = 0; rr < nrows; ++rr) {
+                  const uint32_t v = *(const uint32_t *)(stg + rr * 128 +
+                                                         (((lane >> 2) ^ (rr & 7)) << 4) + ((lane & 3) << 2));
+                  *(uint32_t *)(obase + rr * row_bytes + lane * 4) = v;
+                }
               }
+              __syncwarp();
             }
           } else {
             tmem_wait_ld();
@@ -323,12 +338,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TC_THREADS, 1)
               __nv_bfloat16 *o = (__nv_bfloat16 *)out + arow * ldo + col;
               __nv_bfloat16 *o2 = (__nv_bfloat16 *)(routed ? p.out2_r : p.out2_s) +
                                   arow * (routed ? p.ld2_r : p.ld2_s) + col;
-              // 8 columns at a time: g, u in fp32; dg, du, h as hi + lo bf16 terms
+              // the lane's 32 g and u (fp32), all requested before the first use
+              float4 gq[8], uq[8];
+#pragma unroll
+              for (int i = 0; i < 8; ++i) {
+                gq[i] = ((const float4 *)gp)[i];
+                uq[i] = ((const float4 *)(gp + hf))[i];
+              }
+              // 8 columns at a time: dg, du, h as hi + lo bf16 terms
 #pragma unroll
               for (int q8 = 0; q8 < 4; ++q8) {
-                const float4 ga = ((const float4 *)gp)[2 * q8], gb = ((const float4 *)gp)[2 * q8 + 1];
-                const float4 ua = ((const float4 *)(gp + hf))[2 * q8],
-                             ub = ((const float4 *)(gp + hf))[2 * q8 + 1];
+                const float4 ga = gq[2 * q8], gb = gq[2 * q8 + 1];
+                const float4 ua = uq[2 * q8], ub = uq[2 * q8 + 1];
                 const float gv[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
                 const float uv[8] = {ua.x, ua.y, ua.z, ua.w, ub.x, ub.y, ub.z, ub.w};
                 uint32_t dgh[4], dgl[4], duh[4], dul[4], hh[4], hl[4];
