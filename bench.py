@@ -53,12 +53,12 @@ def load_peaks():
 
 def kernel_sources_sha256() -> str:
     """sha256 of the sources the forward kernels are built from: every file of csrc in name
-    order except backward.cuh, whose kernels are not part of the step."""
+    order except the backward-only ones (backward*.cuh), whose code is not part of the step."""
     import glob
     import hashlib
     h = hashlib.sha256()
     for f in sorted(glob.glob(os.path.join(ROOT, "fine_grained_mixture_moe_b200", "csrc", "*"))):
-        if os.path.basename(f) == "backward.cuh":
+        if os.path.basename(f).startswith("backward"):
             continue
         with open(f, "rb") as fh:
             h.update(fh.read())

@@ -12,6 +12,7 @@
 // `acc_full` barriers; all sixteen epilogue warps arrive on the leader's `acc_empty`. No TMA
 // multicast is used. All waits are bounded as in gemm_tc.cuh.
 #pragma once
+#include "backward_epilogue.cuh"
 #include "gemm_tc.cuh"
 
 namespace moe {
@@ -74,7 +75,11 @@ template <int MODE> struct Tc2Cfg {
   static constexpr int A_BYTES = 128 * TC_BK * 2;             // this CTA's 128 rows
   static constexpr int B_BYTES = 128 * TC_BK * 2;             // this CTA's half of B
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;       // 32 KB
-  static constexpr int STG_BYTES = TC_EPI_WARPS * 4096;  // per-warp epilogue staging
+  // per-warp epilogue staging: 4 KB, or (SWIGLU_BWD) 8 KB for a g, u block pair and, after
+  // all warps' buffers, one mbarrier per warp for its bulk copies
+  static constexpr int STG_WARP = MODE == MODE_SWIGLU_BWD ? GU_PAIR_BYTES : 4096;
+  static constexpr int STG_BYTES =
+      TC_EPI_WARPS * STG_WARP + (MODE == MODE_SWIGLU_BWD ? TC_EPI_WARPS * 8 : 0);
   static constexpr int MAX_STAGES = 8;
   static constexpr int ACC_COLS = MMA_N;
   static constexpr int TMEM_COLS = 512;
@@ -139,6 +144,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TC_THREADS, 1)
       mbar_init(acce_bar(b), 2 * TC_EPI_WARPS);
     }
     mbar_init(drain_bar, 1);
+    if (MODE == MODE_SWIGLU_BWD)
+      for (int w = 0; w < TC_EPI_WARPS; ++w)
+        mbar_init(smem_u32(stg_all + TC_EPI_WARPS * C::STG_WARP + 8 * w), 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -275,120 +283,58 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TC_THREADS, 1)
     const int cbeg = half * (BN / 2), cend = cbeg + BN / 2;
     int acc = 0;
     uint32_t acc_phase = 0;
+    GuFeed feed;  // SWIGLU_BWD: this warp's g, u blocks
+    feed.buf = smem_u32(stg_all + (warp - 2) * C::STG_WARP);
+    feed.bar = smem_u32(stg_all + TC_EPI_WARPS * C::STG_WARP + 8 * (warp - 2));
+    feed.phase = 0;
+    feed.pending = false;
     for (int tile = pair; tile < total; tile += npairs) {
       const TileInfo ti = decode_tile(p, tile, prefix, TC2_BM, BN);
       const bool routed = ti.g < p.E;
+      const int rbase = ti.m0 + (int)rank * 128 + q * 32;  // first row of this warp's block
+      const int row = rbase + lane;
+      const bool row_ok = row < ti.rows;
+      // a warp of padding rows only, or columns past the group's width: nothing to store
+      const int cstop = rbase < ti.rows ? min(cend, ti.N - ti.n0) : cbeg;
+      if (MODE == MODE_SWIGLU_BWD && cstop > cbeg)
+        feed.issue(gu_pair_block(p, ti, routed, routed ? p.aux_r : p.aux_s, rbase, ti.n0 + cbeg),
+                   lane);
       bool ok = true;
       if (lane == 0)
         ok = mbar_wait(accf_bar(acc), acc_phase, abort_flag, limit, INFO_WAIT_ACC_FULL);
       ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
       if (!ok) break;
       tc_fence_after();
-      const int rbase = ti.m0 + (int)rank * 128 + q * 32;  // first row of this warp's block
-      const int row = rbase + lane;
-      const bool row_ok = row < ti.rows;
       void *out = routed ? p.out_r : p.out_s;
       const int ldo = routed ? p.ldo_r : p.ldo_s;
       const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * C::ACC_COLS);
-      unsigned char *stg = stg_all + (warp - 2) * 4096;
-      const int cstop = rbase < ti.rows ? cend : cbeg;  // a warp of padding rows only: nothing to store
+      unsigned char *stg = stg_all + (warp - 2) * C::STG_WARP;
 #pragma unroll 1
       for (int c = cbeg; c < cstop; c += 32) {
-        if (MODE == MODE_GATEUP_RAW || MODE == MODE_SWIGLU_BWD) {
-          // backward epilogues, 32 columns of the lane's row at a time, each output written as
-          // 64 contiguous bytes of the row
+        if (MODE == MODE_GATEUP_RAW) {
+          uint32_t r0[32], r1[32];
+          tmem_ld32(tbase + c, r0);
+          tmem_ld32(tbase + BN + c, r1);
+          tmem_wait_ld();
+          gateup_raw_chunk(r0, r1, stg, gu_pair_block(p, ti, routed, out, rbase, ti.n0 + c), lane);
+          continue;
+        }
+        if (MODE == MODE_SWIGLU_BWD) {
           const int col = ti.n0 + c;
           const int hf = routed ? p.half_r : p.half_s;
           uint32_t r0[32];
           tmem_ld32(tbase + c, r0);
-          if (MODE == MODE_GATEUP_RAW) {
-            // g then u (fp32), each staged per warp (32 rows x 32 columns) and written as 32
-            // coalesced 128-byte row pieces
-            uint32_t r1[32];
-            tmem_ld32(tbase + BN + c, r1);
-            tmem_wait_ld();
-            unsigned char *stg = stg_all + (warp - 2) * 4096;
-            const int nrows = min(32, ti.rows - rbase);
-#pragma unroll 1
-            for (int part = 0; part < 2; ++part) {
-              const uint32_t *rv = part ? r1 : r0;
-#pragma unroll
-              for (int i = 0; i < 8; ++i)
-                *(uint4 *)(stg + lane * 128 + ((i ^ (lane & 7)) << 4)) =
-                    make_uint4(rv[4 * i], rv[4 * i + 1], rv[4 * i + 2], rv[4 * i + 3]);
-              __syncwarp();
-              if (col < ti.N) {
-                unsigned char *obase = (unsigned char *)out +
-                                       ((size_t)(ti.out_row0 + rbase) * ldo + col + part * hf) * 4;
-                const size_t row_bytes = (size_t)ldo * 4;
-                for (int rr = 0; rr < nrows; ++rr) {
-                  const uint32_t v = *(const uint32_t *)(stg + rr * 128 +
-                                                         (((lane >> 2) ^ (rr & 7)) << 4) + ((lane & 3) << 2));
-                  *(uint32_t *)(obase + rr * row_bytes + lane * 4) = v;
-                }
-              }
-              __syncwarp();
-            }
-          } else {
-            tmem_wait_ld();
-            if (row_ok && col < ti.N) {
-              const size_t arow = (size_t)(ti.out_row0 + row);
-              const float *gp = (const float *)(routed ? p.aux_r : p.aux_s) +
-                                arow * (routed ? p.ldaux_r : p.ldaux_s) + col;
-              __nv_bfloat16 *o = (__nv_bfloat16 *)out + arow * ldo + col;
-              __nv_bfloat16 *o2 = (__nv_bfloat16 *)(routed ? p.out2_r : p.out2_s) +
-                                  arow * (routed ? p.ld2_r : p.ld2_s) + col;
-              // the lane's 32 g and u (fp32), all requested before the first use
-              float4 gq[8], uq[8];
-#pragma unroll
-              for (int i = 0; i < 8; ++i) {
-                gq[i] = ((const float4 *)gp)[i];
-                uq[i] = ((const float4 *)(gp + hf))[i];
-              }
-              // 8 columns at a time: dg, du, h as hi + lo bf16 terms
-#pragma unroll
-              for (int q8 = 0; q8 < 4; ++q8) {
-                const float4 ga = gq[2 * q8], gb = gq[2 * q8 + 1];
-                const float4 ua = uq[2 * q8], ub = uq[2 * q8 + 1];
-                const float gv[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
-                const float uv[8] = {ua.x, ua.y, ua.z, ua.w, ub.x, ub.y, ub.z, ub.w};
-                uint32_t dgh[4], dgl[4], duh[4], dul[4], hh[4], hl[4];
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                  float dgv[2], duv[2], hv[2];
-#pragma unroll
-                  for (int z = 0; z < 2; ++z) {
-                    const int e = 2 * i + z;
-                    const float g = gv[e], u = uv[e], dh = __uint_as_float(r0[8 * q8 + e]);
-                    const float sg = 1.0f / (1.0f + __expf(-g)), si = g * sg;
-                    dgv[z] = dh * u * sg * (1.0f + g * (1.0f - sg));
-                    duv[z] = dh * si;
-                    hv[z] = si * u;
-                  }
-                  const __nv_bfloat162 a = __floats2bfloat162_rn(dgv[0], dgv[1]);
-                  const __nv_bfloat162 b = __floats2bfloat162_rn(duv[0], duv[1]);
-                  const __nv_bfloat162 h = __floats2bfloat162_rn(hv[0], hv[1]);
-                  const float2 af = __bfloat1622float2(a), bfv = __bfloat1622float2(b),
-                               hf2 = __bfloat1622float2(h);
-                  const __nv_bfloat162 al = __floats2bfloat162_rn(dgv[0] - af.x, dgv[1] - af.y);
-                  const __nv_bfloat162 bl = __floats2bfloat162_rn(duv[0] - bfv.x, duv[1] - bfv.y);
-                  const __nv_bfloat162 hlo = __floats2bfloat162_rn(hv[0] - hf2.x, hv[1] - hf2.y);
-                  dgh[i] = *(const uint32_t *)&a;
-                  duh[i] = *(const uint32_t *)&b;
-                  hh[i] = *(const uint32_t *)&h;
-                  dgl[i] = *(const uint32_t *)&al;
-                  dul[i] = *(const uint32_t *)&bl;
-                  hl[i] = *(const uint32_t *)&hlo;
-                }
-                ((uint4 *)o)[q8] = make_uint4(dgh[0], dgh[1], dgh[2], dgh[3]);
-                ((uint4 *)(o + hf))[q8] = make_uint4(duh[0], duh[1], duh[2], duh[3]);
-                ((uint4 *)(o + 2 * hf))[q8] = make_uint4(dgl[0], dgl[1], dgl[2], dgl[3]);
-                ((uint4 *)(o + 3 * hf))[q8] = make_uint4(dul[0], dul[1], dul[2], dul[3]);
-                ((uint4 *)o2)[q8] = make_uint4(hh[0], hh[1], hh[2], hh[3]);
-                ((uint4 *)(o2 + hf))[q8] = make_uint4(hl[0], hl[1], hl[2], hl[3]);
-              }
-            }
-          }
+          tmem_wait_ld();
+          if (!feed.wait(abort_flag, limit)) { ok = false; break; }
+          const size_t arow = (size_t)(ti.out_row0 + row);
+          __nv_bfloat16 *o = (__nv_bfloat16 *)out + arow * ldo + col;
+          __nv_bfloat16 *o2 = (__nv_bfloat16 *)(routed ? p.out2_r : p.out2_s) +
+                              arow * (routed ? p.ld2_r : p.ld2_s) + col;
+          swiglu_bwd_chunk(r0, stg, lane, row_ok, o, o2, hf, [&] {
+            if (c + 32 < cstop)
+              feed.issue(gu_pair_block(p, ti, routed, routed ? p.aux_r : p.aux_s, rbase, col + 32),
+                         lane);
+          });
           continue;
         }
         if (MODE == MODE_GATEUP) {
@@ -485,11 +431,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TC_THREADS, 1)
           __syncwarp();
         }
       }
+      if (!ok) break;
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cta0(acce_bar(acc));
       if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
     }
+    if (MODE == MODE_SWIGLU_BWD) feed.drain(limit);
   }
 
   tc_fence_before();

@@ -10,10 +10,10 @@
 //                        matrix, so S shared experts of width fs act as one of width S*fs.
 // Epilogue modes: GATEUP out = silu(A B0^T) * (A B1^T) (SwiGLU, gate and up fused);
 //                 PLAIN  out = A B0^T;   SCALE out = (A B0^T) * scale[g][n] (low-rank s);
-//                 GATEUP_RAW (backward) g = A B0^T to out[., n], u = A B1^T to out[., half + n]
-//                   (fp32);
-//                 SWIGLU_BWD (backward) dh = A B0^T with fp32 g, u read from aux[., n] and
-//                   aux[., half + n]; dg = dh u silu'(g), du = dh silu(g) and h = silu(g) u, each
+//                 GATEUP_RAW (backward) g = A B0^T and u = A B1^T (fp32) to out, in the
+//                   blocked g, u layout of backward_epilogue.cuh (half = the width of g);
+//                 SWIGLU_BWD (backward) dh = A B0^T with fp32 g, u read from aux (the same
+//                   blocked layout); dg = dh u silu'(g), du = dh silu(g) and h = silu(g) u, each
 //                   as two bf16 terms (v = hi + lo, hi = bf16(v), lo = bf16(v - hi)): out[., n] =
 //                   dg_hi, out[., half + n] = du_hi, out[., 2 half + n] = dg_lo,
 //                   out[., 3 half + n] = du_lo, out2[., n] = h_hi, out2[., half + n] = h_lo.
@@ -64,7 +64,8 @@ struct GroupedGemm {
   void *out2_r, *out2_s;
   int ld2_r, ld2_s;
   const void *aux_r, *aux_s;
-  int ldaux_r, ldaux_s;
+  const int32_t *aux_row0;  // [E] device: first row of each routed group in the blocked g, u
+                            // buffer (group sizes rounded up to 64); the shared group starts at 0
   // groups along K (backward weight gradients)
   int kgroup;
   const int32_t *koff;     // [E+1] device: padded K offsets of the groups
