@@ -23,6 +23,7 @@ STATUS_NAMES = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED",
 SCORE = {"softmax": 0, "sigmoid": 1}
 EXPERT = {"swiglu": 0, "lowrank": 1}
 DTYPE = {"f32": 0, "bf16": 1}
+STORAGE = {"dtype": 0, "fp8": 1}
 DEBUG_FORCE_EXACT, DEBUG_WAIT_LIMIT_NS, DEBUG_PROFILE, DEBUG_STAMP = 1, 2, 3, 4
 
 
@@ -36,13 +37,15 @@ class MoEConfig(ctypes.Structure):
     _fields_ = [("T", c_int32), ("d", c_int32), ("E", c_int32), ("top_k", c_int32),
                 ("n_shared", c_int32), ("ffn", c_int32), ("ffn_shared", c_int32),
                 ("rank", c_int32), ("score", c_int32), ("expert", c_int32), ("dtype", c_int32),
-                ("norm_topk", c_int32), ("capacity_factor", c_float), ("aux_alpha", c_float)]
+                ("norm_topk", c_int32), ("capacity_factor", c_float), ("aux_alpha", c_float),
+                ("expert_storage", c_int32)]
 
 
 class MoEWeights(ctypes.Structure):
     _fields_ = [(n, c_void_p) for n in ("w_router", "logit_offset", "select_bias", "w_gate",
                                         "w_up", "w_down", "lr_V", "lr_U", "lr_s", "ws_gate",
-                                        "ws_up", "ws_down")]
+                                        "ws_up", "ws_down", "lr_V8", "lr_V_scale", "lr_U8",
+                                        "lr_U_scale")]
 
 
 class MoEGrads(ctypes.Structure):
@@ -111,6 +114,8 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
         "moe_debug_wait_timeout_probe": (c_int32, [c_void_p]),
         "moe_route_noalloc": (c_int32, [P(MoEConfig), c_void_p, P(MoEWeights), c_void_p,
                                         c_void_p, c_void_p, c_void_p, c_void_p]),
+        "moe_quantize_fp8": (c_int32, [c_void_p, c_int32, c_int64, c_int32, c_void_p, c_void_p,
+                                       c_void_p]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -126,7 +131,8 @@ EXPORTED = ("moe_workspace_size", "moe_capacity", "moe_route", "moe_permute",
             "moe_expert_backward",
             "moe_layer_forward",
             "moe_status_str", "moe_get_device_error", "moe_debug_set", "moe_profile_read",
-            "moe_stamp_read", "moe_debug_wait_timeout_probe", "moe_route_noalloc")
+            "moe_stamp_read", "moe_debug_wait_timeout_probe", "moe_route_noalloc",
+            "moe_quantize_fp8")
 
 
 def _ptr(t) -> Optional[int]:
@@ -161,10 +167,11 @@ def status_str(status: int) -> str:
 def make_config(T: int, d: int, E: int, top_k: int, n_shared: int = 0, ffn: int = 0,
                 ffn_shared: int = 0, rank: int = 0, score: str = "softmax",
                 expert: str = "swiglu", dtype: str = "bf16", norm_topk: bool = False,
-                capacity_factor: float = 0.0, aux_alpha: float = 0.01) -> MoEConfig:
+                capacity_factor: float = 0.0, aux_alpha: float = 0.01,
+                expert_storage: str = "dtype") -> MoEConfig:
     return MoEConfig(T, d, E, top_k, n_shared, ffn, ffn_shared, rank, SCORE[score],
                      EXPERT[expert], DTYPE[dtype], int(bool(norm_topk)), capacity_factor,
-                     aux_alpha)
+                     aux_alpha, STORAGE[expert_storage])
 
 
 def make_weights(tensors: Dict[str, object]) -> MoEWeights:
@@ -294,6 +301,14 @@ def moe_debug_wait_timeout_probe(stream=None) -> None:
 
 
 ROUTE_NOALLOC_SCRATCH_BYTES = 4 << 20
+
+
+def moe_quantize_fp8(x, rows: int, cols: int, q, scale, stream=None) -> None:
+    """Per-row E4M3 codes q [rows, cols] uint8 and fp32 scales [rows] of x (bf16 or fp32)."""
+    import torch
+    dt = DTYPE["bf16"] if x.dtype == torch.bfloat16 else DTYPE["f32"]
+    _check("moe_quantize_fp8", load().moe_quantize_fp8(_ptr(x), dt, rows, cols, _ptr(q),
+                                                       _ptr(scale), _stream(stream)))
 
 
 def moe_route_noalloc(cfg, x, w: MoEWeights, topk_idx, topk_w, expert_count, prob_sum,

@@ -40,13 +40,15 @@ struct TcParams {
 };
 
 template <int MODE, int BN> struct TcCfg {
-  static_assert(MODE == MODE_PLAIN || MODE == MODE_SCALE,
+  static_assert(MODE == MODE_PLAIN || MODE == MODE_SCALE || MODE == MODE_SCALE_FP8,
                 "single-SM form: down and low-rank products (gate/up runs on CTA pairs)");
   static constexpr int NB = 1;                                    // B tiles per stage
-  static constexpr int A_BYTES = TC_BM * TC_BK * 2;               // 16 KB
-  static constexpr int B_BYTES = BN * TC_BK * 2;
+  static constexpr int BK = mode_bk(MODE);                        // K elements per stage
+  static constexpr int A_BYTES = TC_BM * 128;                     // 16 KB: 128-byte rows
+  static constexpr int B_BYTES = BN * 128;
   static constexpr int STAGE_BYTES = A_BYTES + NB * B_BYTES;
-  static constexpr int STG_BYTES = MODE == MODE_PLAIN ? TC_EPI_WARPS * 4096 : 0;  // fp32 staging
+  static constexpr bool F32_OUT = MODE == MODE_PLAIN || MODE == MODE_SCALE_FP8;
+  static constexpr int STG_BYTES = F32_OUT ? TC_EPI_WARPS * 4096 : 0;  // fp32 staging
   static constexpr int STAGES = (200 * 1024 - STG_BYTES) / STAGE_BYTES > 8
                                     ? 8 : (200 * 1024 - STG_BYTES) / STAGE_BYTES;
   static constexpr int ACC_COLS = NB * BN;                        // fp32 columns per buffer
@@ -56,8 +58,9 @@ template <int MODE, int BN> struct TcCfg {
   static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "UMMA N for M=128, epilogue in 32s");
   static constexpr int MMA_N = NB * BN;
   static_assert(MMA_N <= 256, "UMMA N <= 256");
-  // instruction descriptor: D fp32, A/B bf16, both K-major, N>>3 at bit 17, M>>4 at bit 24
-  static constexpr uint32_t IDESC = (1u << 4) | (1u << 7) | (1u << 10) |
+  // instruction descriptor: D fp32, A/B bf16 (kind::f16) or E4M3 (kind::f8f6f4, format 0), both
+  // K-major, N>>3 at bit 17, M>>4 at bit 24
+  static constexpr uint32_t IDESC = (1u << 4) | (mode_fp8(MODE) ? 0u : (1u << 7) | (1u << 10)) |
                                     ((uint32_t)(MMA_N >> 3) << 17) | ((uint32_t)(TC_BM >> 4) << 24);
 };
 
@@ -86,6 +89,16 @@ __device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t
       "{\n\t.reg .pred p;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// The same with 8-bit operands (both E4M3 here): K = 32 elements (32 bytes) per instruction.
+__device__ __forceinline__ void tc_mma_f8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                          uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
       "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
@@ -207,7 +220,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) gemm_tc_kernel(const __grid_con
         const CUtensorMap *ma = routed ? &P.maps.a_r : &P.maps.a_s;
         const CUtensorMap *mb0 = routed ? &P.maps.b0_r : &P.maps.b0_s;
         const int a_row = ti.a_row0 + ti.m0;
-        const int nk = ti.K / TC_BK;
+        const int nk = (ti.K + C::BK - 1) / C::BK;
         for (int kb = 0; kb < nk; ++kb) {
           if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, limit, INFO_WAIT_MMA_EMPTY)) {
             ok = false;
@@ -216,7 +229,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) gemm_tc_kernel(const __grid_con
           const uint32_t sA = smem_u32(stages + (size_t)stage * C::STAGE_BYTES);
           const uint32_t sB0 = sA + C::A_BYTES;
           mbar_expect_tx(full_bar(stage), C::STAGE_BYTES);
-          const int kk = kb * TC_BK;
+          const int kk = kb * C::BK;
           int b_row, b_col;
           if (routed) {
             b_row = ti.g * ti.N + ti.n0;
@@ -253,7 +266,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) gemm_tc_kernel(const __grid_con
       bool ok = true, any = false;
       for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
         const TileInfo ti = decode_tile(p, tile, prefix, TC_BM, BN);
-        const int nk = ti.K / TC_BK;
+        const int nk = (ti.K + C::BK - 1) / C::BK;
         if (!mbar_wait(acce_bar(acc), acc_phase ^ 1u, abort_flag, limit, INFO_WAIT_ACC_EMPTY)) {
           ok = false;
           break;
@@ -269,11 +282,12 @@ __global__ void __launch_bounds__(TC_THREADS, 1) gemm_tc_kernel(const __grid_con
           const uint32_t sA = smem_u32(stages + (size_t)stage * C::STAGE_BYTES);
           const uint32_t sB0 = sA + C::A_BYTES;
 #pragma unroll
-          for (int k16 = 0; k16 < TC_BK / 16; ++k16) {
+          for (int k16 = 0; k16 < 4; ++k16) {  // 32 bytes of K per instruction
             const uint64_t ad = make_sdesc(sA + k16 * 32);
             const uint64_t bd0 = make_sdesc(sB0 + k16 * 32);
             const uint32_t accum = (kb > 0 || k16 > 0) ? 1u : 0u;
-            tc_mma(d0, ad, bd0, C::IDESC, accum);
+            if (mode_fp8(MODE)) tc_mma_f8(d0, ad, bd0, C::IDESC, accum);
+            else tc_mma(d0, ad, bd0, C::IDESC, accum);
           }
           any = true;
           tc_commit(empty_bar(stage));
@@ -317,7 +331,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) gemm_tc_kernel(const __grid_con
       // both the row-wise writes and the column-wise reads are conflict-free), then leave as 32
       // row stores of 128 contiguous bytes each instead of 32-row scattered 16-byte stores.
       unsigned char *stg = stg_all + (warp - 2) * 4096;
-      constexpr int SUB = (MODE == MODE_PLAIN) ? 1 : 2;  // 32-column TMEM loads per block
+      constexpr int SUB = C::F32_OUT ? 1 : 2;  // 32-column TMEM loads per block
 #pragma unroll 1
       for (int c = cbeg; c < cend; c += 32 * SUB) {
         if (MODE == MODE_SCALE) {
@@ -380,6 +394,16 @@ __global__ void __launch_bounds__(TC_THREADS, 1) gemm_tc_kernel(const __grid_con
           uint32_t r0[32];
           tmem_ld32(tbase + c, r0);
           tmem_wait_ld();
+          if (MODE == MODE_SCALE_FP8 && row_ok && ti.n0 + c < ti.N) {
+            // z = sum * (row scale) * (V row scale) * s, for columns col .. col + 31 (N is a
+            // multiple of 32)
+            const size_t cn = (size_t)ti.g * ti.N + ti.n0 + c;
+            const float rs = __ldg(p.row_scale + ti.a_row0 + row);
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              r0[i] = __float_as_uint(__uint_as_float(r0[i]) * rs * __ldg(p.col_scale + cn + i) *
+                                      __ldg(p.scale + cn + i));
+          }
 #pragma unroll
           for (int i = 0; i < 8; ++i)
             *(uint4 *)(stg + lane * 128 + ((i ^ (lane & 7)) << 4)) =

@@ -39,6 +39,15 @@ __device__ __forceinline__ void tc2_mma(uint32_t d_tmem, uint64_t adesc, uint64_
       "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
+__device__ __forceinline__ void tc2_mma_f8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                           uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
 // Arrive once on the barrier at this shared offset in both CTAs of the pair when all prior
 // tcgen05 operations of the issuing thread complete.
 __device__ __forceinline__ void tc2_commit_both(uint32_t bar) {
@@ -68,12 +77,13 @@ __host__ __device__ constexpr bool tc2_two_b(int mode) {
 
 template <int MODE> struct Tc2Cfg {
   static_assert(MODE == MODE_GATEUP || MODE == MODE_PLAIN || MODE == MODE_GATEUP_RAW ||
-                    MODE == MODE_SWIGLU_BWD,
+                    MODE == MODE_SWIGLU_BWD || MODE == MODE_PLAIN_FP8,
                 "pair kernel modes");
   static constexpr int BN = tc2_two_b(MODE) ? 128 : 256;  // output columns per tile
   static constexpr int MMA_N = 256;                           // accumulator columns
-  static constexpr int A_BYTES = 128 * TC_BK * 2;             // this CTA's 128 rows
-  static constexpr int B_BYTES = 128 * TC_BK * 2;             // this CTA's half of B
+  static constexpr int BK = mode_bk(MODE);                    // K elements per stage
+  static constexpr int A_BYTES = 128 * 128;                   // this CTA's 128 rows (128 B each)
+  static constexpr int B_BYTES = 128 * 128;                   // this CTA's half of B
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;       // 32 KB
   // per-warp epilogue staging: 4 KB, or (SWIGLU_BWD) 8 KB for a g, u block pair and, after
   // all warps' buffers, one mbarrier per warp for its bulk copies
@@ -83,7 +93,7 @@ template <int MODE> struct Tc2Cfg {
   static constexpr int MAX_STAGES = 8;
   static constexpr int ACC_COLS = MMA_N;
   static constexpr int TMEM_COLS = 512;
-  static constexpr uint32_t IDESC = (1u << 4) | (1u << 7) | (1u << 10) |
+  static constexpr uint32_t IDESC = (1u << 4) | (mode_fp8(MODE) ? 0u : (1u << 7) | (1u << 10)) |
                                     ((uint32_t)(MMA_N >> 3) << 17) |
                                     ((uint32_t)(TC2_BM >> 4) << 24);
 };
@@ -193,7 +203,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TC_THREADS, 1)
         const bool a1_void = ti.m0 + 128 >= ti.rows;
         const uint32_t stage_tx = 2 * C::STAGE_BYTES - (a1_void ? C::A_BYTES : 0);
         const int n_off = tc2_two_b(MODE) ? 0 : (int)rank * 128;
-        const int nk = ti.K / TC_BK;
+        const int nk = (ti.K + C::BK - 1) / C::BK;
         for (int kb = 0; kb < nk; ++kb) {
           if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, limit, INFO_WAIT_MMA_EMPTY)) {
             ok = false;
@@ -202,7 +212,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TC_THREADS, 1)
           const uint32_t sA = smem_u32(stages + (size_t)stage * C::STAGE_BYTES);
           const uint32_t sB = sA + C::A_BYTES;
           if (rank == 0) mbar_expect_tx(full_bar(stage), stage_tx);
-          const int kk = kb * TC_BK;
+          const int kk = kb * C::BK;
           int b_row, b_col;
           if (p.kgroup) {  // one A and one B for all groups, each group its own K columns
             b_row = ti.n0 + n_off;
@@ -241,7 +251,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TC_THREADS, 1)
       bool ok = true, any = false;
       for (int tile = pair; tile < total && ok; tile += npairs) {
         const TileInfo ti = decode_tile(p, tile, prefix, TC2_BM, BN);
-        const int nk = ti.K / TC_BK;
+        const int nk = (ti.K + C::BK - 1) / C::BK;
         if (!mbar_wait(acce_bar(acc), acc_phase ^ 1u, abort_flag, limit, INFO_WAIT_ACC_EMPTY)) {
           ok = false;
           break;
@@ -257,9 +267,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TC_THREADS, 1)
           const uint32_t sA = smem_u32(stages + (size_t)stage * C::STAGE_BYTES);
           const uint32_t sB = sA + C::A_BYTES;
 #pragma unroll
-          for (int k16 = 0; k16 < TC_BK / 16; ++k16) {
+          for (int k16 = 0; k16 < 4; ++k16) {  // 32 bytes of K per instruction
             const uint32_t accum = (kb > 0 || k16 > 0) ? 1u : 0u;
-            tc2_mma(d0, make_sdesc(sA + k16 * 32), make_sdesc(sB + k16 * 32), C::IDESC, accum);
+            if (mode_fp8(MODE))
+              tc2_mma_f8(d0, make_sdesc(sA + k16 * 32), make_sdesc(sB + k16 * 32), C::IDESC, accum);
+            else
+              tc2_mma(d0, make_sdesc(sA + k16 * 32), make_sdesc(sB + k16 * 32), C::IDESC, accum);
           }
           any = true;
           tc2_commit_both(empty_bar(stage));
@@ -412,6 +425,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TC_THREADS, 1)
           uint32_t r0[32];
           tmem_ld32(tbase + c, r0);
           tmem_wait_ld();
+          if (MODE == MODE_PLAIN_FP8 && routed && row_ok && ti.n0 + c < ti.N) {
+            // y = sum * (row scale) * (U row scale), columns col .. col + 31
+            const size_t cn = (size_t)ti.g * ti.N + ti.n0 + c;
+            const float rs = __ldg(p.row_scale + ti.a_row0 + row);
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              r0[i] = __float_as_uint(__uint_as_float(r0[i]) * rs * __ldg(p.col_scale + cn + i));
+          }
 #pragma unroll
           for (int i = 0; i < 8; ++i)
             *(uint4 *)(stg + lane * 128 + ((i ^ (lane & 7)) << 4)) =

@@ -17,6 +17,12 @@
 //                   as two bf16 terms (v = hi + lo, hi = bf16(v), lo = bf16(v - hi)): out[., n] =
 //                   dg_hi, out[., half + n] = du_hi, out[., 2 half + n] = dg_lo,
 //                   out[., 3 half + n] = du_lo, out2[., n] = h_hi, out2[., half + n] = h_lo.
+//                 SCALE_FP8 (E4M3 operands) z = (A B0^T) * row_scale[row] * col_scale[g][n]
+//                   * scale[g][n], fp32 out (the low-rank V projection with fp8 storage);
+//                 PLAIN_FP8 (E4M3 operands) out = (A B0^T) * row_scale[row] * col_scale[g][n],
+//                   fp32 out (the U projection). E4M3 operands have K-blocks of 128 elements
+//                   (128 bytes, as for bf16); a K that is not a multiple of 128 is completed with
+//                   the tensor map's zero fill.
 // Groups along K (kgroup, backward weight gradients): group g is out rows [g M, g M + M) =
 // A[M, K_g] B[N, K_g]^T, where A and B are K-major [M or N][ld] and group g takes their columns
 // kseg koff[g] .. kseg koff[g+1] (koff padded to multiples of 64; kseg segments per group, so a
@@ -31,7 +37,14 @@
 namespace moe {
 
 enum GemmMode { MODE_GATEUP = 0, MODE_PLAIN = 1, MODE_SCALE = 2, MODE_GATEUP_RAW = 3,
-                MODE_SWIGLU_BWD = 4 };
+                MODE_SWIGLU_BWD = 4, MODE_SCALE_FP8 = 5, MODE_PLAIN_FP8 = 6 };
+
+// Modes whose operands are E4M3 bytes (tcgen05 kind::f8f6f4) rather than bf16 (kind::f16).
+__host__ __device__ constexpr bool mode_fp8(int mode) {
+  return mode == MODE_SCALE_FP8 || mode == MODE_PLAIN_FP8;
+}
+// Elements of K per pipeline stage: one 128-byte swizzle row of either type.
+__host__ __device__ constexpr int mode_bk(int mode) { return mode_fp8(mode) ? 128 : 64; }
 
 struct GroupedGemm {
   const int32_t *offsets;  // [E+1] device
@@ -43,7 +56,9 @@ struct GroupedGemm {
   int N_r, K_r;
   void *out_r;
   int ldo_r;
-  const float *scale;  // [E, N_r] for MODE_SCALE
+  const float *scale;  // [E, N_r] for MODE_SCALE and MODE_SCALE_FP8
+  const float *row_scale;  // fp8 modes: [rows_r] scale of each A row (routed groups only)
+  const float *col_scale;  // fp8 modes: [E, N_r] scale of each B row
   int kb_r;            // row length of B_r when shorter than K_r: k wraps over B's columns
                        // (k-block at kk reads B columns kk % kb_r); 0 means K_r
   int lo_split;        // MODE_SCALE, bf16: > 0 stores v as hi = bf16(v) at column n and

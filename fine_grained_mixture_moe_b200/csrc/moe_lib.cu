@@ -14,6 +14,7 @@
 #include "backward.cuh"
 #include "combine.cuh"
 #include "common.cuh"
+#include "fp8.cuh"
 #include "gemm_simt.cuh"
 #include "gemm_tc.cuh"
 #include "gemm_tc2.cuh"
@@ -43,6 +44,11 @@ bool cfg_supported(const moe_config_t *c) {
     return false;
   }
   if (c->n_shared > 0 && (c->ffn_shared <= 0 || c->ffn_shared % 64)) return false;
+  if (c->expert_storage != MOE_STORAGE_DTYPE && c->expert_storage != MOE_STORAGE_FP8_E4M3)
+    return false;
+  if (c->expert_storage == MOE_STORAGE_FP8_E4M3 &&
+      (c->expert != MOE_EXPERT_LOWRANK || c->dtype != MOE_DTYPE_BF16))
+    return false;
   if (!std::isfinite(c->capacity_factor) || !std::isfinite(c->aux_alpha)) return false;
   // the router stages its 16 token rows and the logits in shared memory (227 KB per CTA)
   const bool sig = c->score == MOE_SCORE_SIGMOID;
@@ -102,8 +108,10 @@ struct Layout {
   size_t lrank;                                                 // within-chunk ranks [T, k] u8
   size_t hidden, hidden_sh;                                     // experts
   size_t idx, wts, count, prob, offsets, slot_pos, src, x_perm, y_perm, y_shared, aux;  // layer
+  size_t xq, sx, sx_perm, zq, sz;  // fp8 storage: E4M3 token rows and z rows, their scales
   size_t total;
 };
+inline bool fp8_experts(const moe_config_t *c) { return c->expert_storage == MOE_STORAGE_FP8_E4M3; }
 
 Layout layout_of(const moe_config_t *c) {
   Layout L;
@@ -134,6 +142,13 @@ Layout layout_of(const moe_config_t *c) {
   L.y_perm = take(T * k * d * (yperm_bf16(c) ? 2 : 4));
   L.y_shared = take(T * d * 4);
   L.aux = take(16);
+  // fp8 storage: the x_perm region holds the rows' E4M3 codes and `hidden` the fp32 z
+  const bool f8 = fp8_experts(c);
+  L.xq = take(f8 ? T * d : 0);
+  L.sx = take(f8 ? T * 4 : 0);
+  L.sx_perm = take(f8 ? T * k * 4 : 0);
+  L.zq = take(f8 ? T * k * (size_t)c->rank : 0);
+  L.sz = take(f8 ? T * k * 4 : 0);
   L.total = o;
   return L;
 }
@@ -244,18 +259,22 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// 2-D bf16 map over a row-major [rows, cols] matrix; box [box_rows, 64 columns], 128B swizzle.
-bool make_map(CUtensorMap *m, const void *ptr, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+// 2-D map over a row-major [rows, cols] matrix of bf16 (esz 2) or E4M3 bytes (esz 1); box
+// [box_rows, 128 bytes of columns], 128B swizzle. Columns past `cols` in a box read as zeros
+// (an E4M3 K of 64 fills half a box).
+bool make_map(CUtensorMap *m, const void *ptr, uint64_t rows, uint64_t cols, uint32_t box_rows,
+              int esz = 2) {
   auto fn = encode_fn();
   if (!fn) return false;
   if (rows == 0 || ptr == nullptr) {  // never dereferenced: map a dummy 1-row extent
     rows = 1;
   }
   cuuint64_t dims[2] = {cols, rows};
-  cuuint64_t strides[1] = {cols * 2};
-  cuuint32_t box[2] = {64, box_rows};
+  cuuint64_t strides[1] = {cols * (cuuint64_t)esz};
+  cuuint32_t box[2] = {(cuuint32_t)(128 / esz), box_rows};
   cuuint32_t estr[2] = {1, 1};
-  const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(ptr), dims, strides,
+  const CUresult r = fn(m, esz == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                        2, const_cast<void *>(ptr), dims, strides,
                         box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
@@ -272,16 +291,18 @@ long long tile_bound(const GroupedGemm &g, int BM, int BN) {
 
 // Tensor maps of one grouped launch: A boxes of 128 rows, B boxes of `b_box` rows.
 // routed operands: A [rows_r, K_r], B [E*N_r, K_r]; shared: A [T, K_s], B [b_rows_s, piece_k]
-bool build_maps(const GroupedGemm &g, bool two_b, uint32_t b_box, TcMaps *m) {
+bool build_maps(const GroupedGemm &g, bool two_b, uint32_t b_box, TcMaps *m, int esz = 2) {
   const void *any = g.E > 0 ? g.A_r : g.A_s;
   bool ok = true;
-  ok &= make_map(&m->a_r, g.E > 0 ? g.A_r : any, g.E > 0 ? g.rows_r : 1, g.E > 0 ? g.K_r : 64, 128);
+  ok &= make_map(&m->a_r, g.E > 0 ? g.A_r : any, g.E > 0 ? g.rows_r : 1, g.E > 0 ? g.K_r : 64, 128,
+                 esz);
   const int kb = g.kb_r ? g.kb_r : g.K_r;  // row length of the routed weights
   // routed weights: E stacked [N_r, kb] matrices; groups along K: one [N_r, K_r] for all groups
   const uint64_t b_rows = g.kgroup ? (uint64_t)g.N_r : (uint64_t)g.E * g.N_r;
-  ok &= make_map(&m->b0_r, g.E > 0 ? g.B0_r : any, g.E > 0 ? b_rows : 1, g.E > 0 ? kb : 64, b_box);
+  ok &= make_map(&m->b0_r, g.E > 0 ? g.B0_r : any, g.E > 0 ? b_rows : 1, g.E > 0 ? kb : 64, b_box,
+                 esz);
   ok &= make_map(&m->b1_r, (g.E > 0 && two_b) ? g.B1_r : any, (g.E > 0 && two_b) ? b_rows : 1,
-                 g.E > 0 ? kb : 64, b_box);
+                 g.E > 0 ? kb : 64, b_box, esz);
   ok &= make_map(&m->a_s, g.has_shared ? g.A_s : any, g.has_shared ? g.T : 1,
                  g.has_shared ? g.K_s : 64, 128);
   ok &= make_map(&m->b0_s, g.has_shared ? g.B0_s : any, g.has_shared ? g.b_rows_s : 1,
@@ -297,7 +318,7 @@ moe_status_t launch_tc(const GroupedGemm &g, cudaStream_t st, int kind) {
   std::memset(&P, 0, sizeof(P));
   P.p = g;
   P.p.kind = kind;
-  if (!build_maps(g, MODE == MODE_GATEUP, BN, &P.maps)) return MOE_ERR_CUDA;
+  if (!build_maps(g, MODE == MODE_GATEUP, BN, &P.maps, mode_fp8(MODE) ? 1 : 2)) return MOE_ERR_CUDA;
   const int G = g.E + g.has_shared;
   const size_t smem = tc_smem_bytes<MODE, BN>(G);
   auto kern = gemm_tc_kernel<MODE, BN>;
@@ -318,7 +339,7 @@ moe_status_t launch_tc2(const GroupedGemm &g, cudaStream_t st, int kind) {
   std::memset(&P, 0, sizeof(P));
   P.p = g;
   P.p.kind = kind;
-  if (!build_maps(g, tc2_two_b(MODE), 128, &P.maps)) return MOE_ERR_CUDA;
+  if (!build_maps(g, tc2_two_b(MODE), 128, &P.maps, mode_fp8(MODE) ? 1 : 2)) return MOE_ERR_CUDA;
   const int G = g.E + g.has_shared;
   static_assert(tc2_stages<MODE>(1024 + 1) >= 2, "tile list of 1024 experts leaves no room");
   P.stages = tc2_stages<MODE>(G);
@@ -445,14 +466,26 @@ template <typename Tin>
 moe_status_t scatter_impl(const moe_config_t *c, const void *x, const int32_t *idx,
                           const uint8_t *lrank, const int32_t *chunk_base, const int32_t *kept,
                           int32_t *offsets, int32_t *slot_pos, int32_t *src, void *x_perm,
-                          const int32_t *count, const float *prob, float *aux, cudaStream_t st) {
+                          const int32_t *count, const float *prob, float *aux, cudaStream_t st,
+                          const float *rs_in = nullptr, float *rs_out = nullptr) {
   ProfScope ps(K_PERM_SCATTER, st);
   const size_t smem = (size_t)c->E * sizeof(int);  // the expert offsets
   const int grid = std::max(1, std::min(ceil_div(c->T, PM_THREADS / 32),
                                         num_sms() * PM_CTAS_PER_SM));
   return launch_pdl(perm_scatter_kernel<Tin>, dim3(grid), dim3(PM_THREADS), smem, st, idx, lrank,
                     c->T, c->top_k, c->E, capacity_of(c), chunk_base, kept, offsets, slot_pos,
-                    src, (const Tin *)x, (Tin *)x_perm, c->d, count, prob, c->aux_alpha, aux);
+                    src, (const Tin *)x, (Tin *)x_perm, c->d, count, prob, c->aux_alpha, aux,
+                    rs_in, rs_out);
+}
+
+// Per-row E4M3 quantisation (fp8.cuh) of `rows` rows of `cols` elements.
+template <typename Tin>
+moe_status_t launch_quantize(const void *in, long long rows, int cols, uint8_t *q, float *scale,
+                             cudaStream_t st) {
+  if (rows == 0) return MOE_OK;
+  const int grid = (int)std::min<long long>((rows + 7) / 8, (long long)num_sms() * 16);
+  return launch_pdl(quantize_rows_kernel<Tin>, dim3(grid), dim3(256), 0, st, (const Tin *)in,
+                    rows, cols, q, scale);
 }
 
 template <typename Tin>
@@ -482,10 +515,68 @@ moe_status_t permute_impl(const moe_config_t *c, const void *x, const int32_t *i
                            nullptr, nullptr, st);
 }
 
+// The shared experts of a low-rank layer: SwiGLU gate/up then down over every token.
+moe_status_t lowrank_shared_impl(const moe_config_t *c, const GroupedGemm &g, const void *x,
+                                 const moe_weights_t *w, void *Hs, void *y_shared,
+                                 cudaStream_t st) {
+  const int d = c->d, S = c->n_shared, fs = c->ffn_shared;
+  GroupedGemm g3 = g;
+  g3.E = 0; g3.has_shared = 1;
+  g3.A_s = x; g3.lda_s = d; g3.B0_s = w->ws_gate; g3.B1_s = w->ws_up;
+  g3.N_s = S * fs; g3.K_s = d; g3.piece_k = d; g3.piece_rows = 0; g3.b_rows_s = S * fs;
+  g3.out_s = Hs; g3.ldo_s = S * fs;
+  MOE_TRY(launch_gemm<MODE_GATEUP>(c, g3, st, K_GEMM_GATEUP));
+  GroupedGemm g4 = g;
+  g4.E = 0; g4.has_shared = 1;
+  g4.A_s = Hs; g4.lda_s = S * fs; g4.B0_s = w->ws_down; g4.N_s = d; g4.K_s = S * fs;
+  g4.piece_k = fs; g4.piece_rows = d; g4.b_rows_s = S * d; g4.out_s = y_shared; g4.ldo_s = d;
+  return launch_gemm<MODE_PLAIN>(c, g4, st, K_GEMM_DOWN);
+}
+
+// Low-rank experts stored in E4M3 on their grouped rows (codes xq_perm, scales sx_perm):
+// z = (xq V8^T) * sx * V_scale * s (fp32, fp8 tensor cores) -> per-row E4M3 of z ->
+// y_perm = (zq U8^T) * sz * U_scale (fp32). The rank K = r of the second product is completed to
+// a 128-element stage by the tensor map's zero fill. Rows past the kept count are quantised too
+// (the host does not know the count); nothing reads them.
+moe_status_t experts_fp8_impl(const moe_config_t *c, const uint8_t *xq_perm, const float *sx_perm,
+                              const int32_t *offsets, const void *x, const moe_weights_t *w,
+                              void *y_perm, void *y_shared, void *ws, cudaStream_t st) {
+  const Layout L = layout_of(c);
+  const int T = c->T, d = c->d, E = c->E, k = c->top_k, r = c->rank;
+  float *Z = at<float>(ws, L.hidden);
+  uint8_t *zq = at<uint8_t>(ws, L.zq);
+  float *sz = at<float>(ws, L.sz);
+  GroupedGemm g;
+  std::memset(&g, 0, sizeof(g));
+  g.offsets = offsets;
+  g.T = T;
+  g.rows_r = T * k;
+  GroupedGemm g1 = g;
+  g1.E = E; g1.A_r = xq_perm; g1.lda_r = d; g1.B0_r = w->lr_V8; g1.N_r = r; g1.K_r = d;
+  g1.out_r = Z; g1.ldo_r = r; g1.scale = w->lr_s; g1.row_scale = sx_perm;
+  g1.col_scale = w->lr_V_scale;
+  MOE_TRY((launch_tc<MODE_SCALE_FP8, 64>(g1, st, K_GEMM_LR1)));
+  MOE_TRY(launch_quantize<float>(Z, (long long)T * k, r, zq, sz, st));
+  GroupedGemm g2 = g;
+  g2.E = E; g2.A_r = zq; g2.lda_r = r; g2.B0_r = w->lr_U8; g2.N_r = d; g2.K_r = r;
+  g2.out_r = y_perm; g2.ldo_r = d; g2.row_scale = sz; g2.col_scale = w->lr_U_scale;
+  MOE_TRY(launch_tc2<MODE_PLAIN_FP8>(g2, st, K_GEMM_LR2));
+  if (c->n_shared > 0)
+    MOE_TRY(lowrank_shared_impl(c, g, x, w, at<char>(ws, L.hidden_sh), y_shared, st));
+  return MOE_OK;
+}
+
 moe_status_t experts_impl(const moe_config_t *c, const void *x_perm, const int32_t *offsets,
                           const void *x, const moe_weights_t *w, void *y_perm, void *y_shared,
                           void *ws, cudaStream_t st) {
   if (c->T == 0) return MOE_OK;
+  if (fp8_experts(c)) {  // the bf16 rows quantised first, as the layer quantises its tokens
+    const Layout L = layout_of(c);
+    uint8_t *xq = at<uint8_t>(ws, L.x_perm);
+    float *sxp = at<float>(ws, L.sx_perm);
+    MOE_TRY(launch_quantize<__nv_bfloat16>(x_perm, (long long)c->T * c->top_k, c->d, xq, sxp, st));
+    return experts_fp8_impl(c, xq, sxp, offsets, x, w, y_perm, y_shared, ws, st);
+  }
   const Layout L = layout_of(c);
   const int T = c->T, d = c->d, E = c->E, k = c->top_k, S = c->n_shared, fs = c->ffn_shared;
   void *H = at<char>(ws, L.hidden);
@@ -533,19 +624,7 @@ moe_status_t experts_impl(const moe_config_t *c, const void *x_perm, const int32
   g2.K_r = split ? 2 * r : r; g2.kb_r = split ? r : 0;
   g2.out_r = y_perm; g2.ldo_r = d; g2.out_r_bf16 = yperm_bf16(c) ? 1 : 0;
   MOE_TRY(launch_gemm<MODE_PLAIN>(c, g2, st, K_GEMM_LR2));
-  if (sh) {
-    GroupedGemm g3 = g;
-    g3.E = 0; g3.has_shared = 1;
-    g3.A_s = x; g3.lda_s = d; g3.B0_s = w->ws_gate; g3.B1_s = w->ws_up;
-    g3.N_s = S * fs; g3.K_s = d; g3.piece_k = d; g3.piece_rows = 0; g3.b_rows_s = S * fs;
-    g3.out_s = Hs; g3.ldo_s = S * fs;
-    MOE_TRY(launch_gemm<MODE_GATEUP>(c, g3, st, K_GEMM_GATEUP));
-    GroupedGemm g4 = g;
-    g4.E = 0; g4.has_shared = 1;
-    g4.A_s = Hs; g4.lda_s = S * fs; g4.B0_s = w->ws_down; g4.N_s = d; g4.K_s = S * fs;
-    g4.piece_k = fs; g4.piece_rows = d; g4.b_rows_s = S * d; g4.out_s = y_shared; g4.ldo_s = d;
-    MOE_TRY(launch_gemm<MODE_PLAIN>(c, g4, st, K_GEMM_DOWN));
-  }
+  if (sh) MOE_TRY(lowrank_shared_impl(c, g, x, w, Hs, y_shared, st));
   return MOE_OK;
 }
 
@@ -593,6 +672,10 @@ moe_status_t check_weights(const moe_config_t *c, const moe_weights_t *w, bool r
   if (experts) {
     if (c->expert == MOE_EXPERT_SWIGLU) {
       if (!aligned16(w->w_gate) || !aligned16(w->w_up) || !aligned16(w->w_down)) return MOE_ERR_INVALID_ARG;
+    } else if (fp8_experts(c)) {
+      if (!aligned16(w->lr_V8) || !aligned16(w->lr_U8) || !aligned16(w->lr_s) ||
+          !aligned16(w->lr_V_scale) || !aligned16(w->lr_U_scale))
+        return MOE_ERR_INVALID_ARG;
     } else {
       if (!aligned16(w->lr_V) || !aligned16(w->lr_U) || !aligned16(w->lr_s)) return MOE_ERR_INVALID_ARG;
     }
@@ -818,6 +901,11 @@ moe_status_t moe_layer_forward(const moe_config_t *cfg, const void *x, const moe
   float *pp = at<float>(ws, L.part_prob);
   int32_t *cb = at<int32_t>(ws, L.chunk_base);
   uint8_t *lr = at<uint8_t>(ws, L.lrank);
+  const bool f8 = fp8_experts(cfg);
+  uint8_t *xq = at<uint8_t>(ws, L.xq);
+  float *sx = at<float>(ws, L.sx), *sxp = at<float>(ws, L.sx_perm);
+  // fp8 storage: every token row quantised once, before the routing (it needs x alone)
+  if (f8) MOE_TRY(launch_quantize<__nv_bfloat16>(x, cfg->T, cfg->d, xq, sx, st));
   if (cfg->dtype == MOE_DTYPE_BF16)
     MOE_TRY(router_only<__nv_bfloat16>(cfg, x, w, idx, wts, pc, pp, lr, st));
   else
@@ -828,15 +916,35 @@ moe_status_t moe_layer_forward(const moe_config_t *cfg, const void *x, const moe
   sa.chunk_base = cb;
   sa.kept = at<int32_t>(ws, L.kept);
   MOE_TRY(launch_stats(sa, st));
-  if (cfg->dtype == MOE_DTYPE_BF16)
+  if (f8)
+    MOE_TRY(scatter_impl<uint8_t>(cfg, xq, idx, lr, cb, sa.kept, offsets, slot_pos, src, x_perm,
+                                  cnt, prob, aux, st, sx, sxp));
+  else if (cfg->dtype == MOE_DTYPE_BF16)
     MOE_TRY(scatter_impl<__nv_bfloat16>(cfg, x, idx, lr, cb, sa.kept, offsets, slot_pos, src,
                                         x_perm, cnt, prob, aux, st));
   else
     MOE_TRY(scatter_impl<float>(cfg, x, idx, lr, cb, sa.kept, offsets, slot_pos, src, x_perm,
                                 cnt, prob, aux, st));
   // T > 0 here: the expert forward launched at least two kernels after the scatter
-  MOE_TRY(experts_impl(cfg, x_perm, offsets, x, w, y_perm, y_sh, ws, st));
+  if (f8)
+    MOE_TRY(experts_fp8_impl(cfg, (const uint8_t *)x_perm, sxp, offsets, x, w, y_perm, y_sh, ws,
+                             st));
+  else
+    MOE_TRY(experts_impl(cfg, x_perm, offsets, x, w, y_perm, y_sh, ws, st));
   return combine_impl(cfg, y_perm, y_sh, slot_pos, wts, y, st, true);
+}
+
+moe_status_t moe_quantize_fp8(const void *in, int32_t in_dtype, int64_t rows, int32_t cols,
+                              uint8_t *q, float *scale, void *stream) {
+  if (rows < 0 || cols <= 0) return MOE_ERR_INVALID_ARG;
+  if (cols % 16 || (in_dtype != MOE_DTYPE_BF16 && in_dtype != MOE_DTYPE_F32) ||
+      rows * (long long)cols >= (1ll << 40))
+    return MOE_ERR_UNSUPPORTED;
+  if (rows == 0) return MOE_OK;
+  MOE_REQUIRE(aligned16(in) && aligned16(q) && aligned16(scale));
+  cudaStream_t st = (cudaStream_t)stream;
+  if (in_dtype == MOE_DTYPE_BF16) return launch_quantize<__nv_bfloat16>(in, rows, cols, q, scale, st);
+  return launch_quantize<float>(in, rows, cols, q, scale, st);
 }
 
 const char *moe_status_str(moe_status_t s) {

@@ -74,6 +74,8 @@ __global__ void __launch_bounds__(256) perm_hist_kernel(const int32_t *__restric
 // memory; block 0 writes offsets[0..E] and, when `aux` is set, the load-balancing loss
 // alpha E sum_e (count_e / (T k)) (prob_e / T) (Quartz: weight 0.01), in the order of
 // aux_loss_kernel, so that the fused layer and the separate call agree bit for bit.
+// Rows of E4M3 codes (Tin = uint8_t) travel with their scales: rs_out[row] = rs_in[token] when
+// rs_out is set.
 // Before griddep_wait: this kernel always follows the statistics kernel, whose CTAs allow it to
 // start only after their own griddep_wait, i.e. once the kernel before the statistics (the
 // router or the histogram) has completed and flushed. So x, the routing and the within-chunk
@@ -85,7 +87,7 @@ __global__ void __launch_bounds__(PM_THREADS, PM_CTAS_PER_SM) perm_scatter_kerne
     int32_t *__restrict__ offsets, int32_t *__restrict__ slot_pos, int32_t *__restrict__ src,
     const Tin *__restrict__ x, Tin *__restrict__ x_perm, int d,
     const int32_t *__restrict__ count, const float *__restrict__ prob, float alpha,
-    float *__restrict__ aux) {
+    float *__restrict__ aux, const float *__restrict__ rs_in, float *__restrict__ rs_out) {
   extern __shared__ int s_off[];  // [E] expert offsets
   __shared__ int s_scan[PM_THREADS / 32 + 1];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -145,6 +147,7 @@ __global__ void __launch_bounds__(PM_THREADS, PM_CTAS_PER_SM) perm_scatter_kerne
         if (C < 0 || rank < C) pos = s_off[e] + rank;
         slot_pos[(size_t)t * k + lane] = pos;
         if (pos >= 0) src[pos] = t;
+        if (pos >= 0 && rs_out != nullptr) rs_out[pos] = __ldcg(rs_in + t);
       } else {
         slot_pos[(size_t)t * k + lane] = -1;
         set_device_error(MOE_ERR_DEVICE_CHECK, 100 + lane);

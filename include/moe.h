@@ -53,6 +53,12 @@ typedef enum {
 typedef enum { MOE_SCORE_SOFTMAX = 0, MOE_SCORE_SIGMOID = 1 } moe_score_t;
 typedef enum { MOE_EXPERT_SWIGLU = 0, MOE_EXPERT_LOWRANK = 1 } moe_expert_t;
 typedef enum { MOE_DTYPE_F32 = 0, MOE_DTYPE_BF16 = 1 } moe_dtype_t;
+/* Storage of the routed experts' weights. MOE_STORAGE_FP8_E4M3 is the fp8 rung of the storage
+ * ladder of the low-rank experts (dormouse, "TSCT low-rank experts": the U*diag(s)*V^T
+ * factorisation carries a storage ladder fp8 -> NVFP4 -> ternary): V and U as E4M3 rows with
+ * one fp32 scale per row (see moe_quantize_fp8), computed on the fp8 tensor cores. bf16 low-rank
+ * layers only. */
+typedef enum { MOE_STORAGE_DTYPE = 0, MOE_STORAGE_FP8_E4M3 = 1 } moe_storage_t;
 
 /* Problem statement of one layer call (the arguments the pages' architecture tables give:
  * hidden size, routed experts, top-k, shared experts, expert FFN width, scoring, capacity). */
@@ -71,6 +77,7 @@ typedef struct {
   int32_t norm_topk;    /* 1: divide the k selected weights by their sum */
   float capacity_factor;/* <= 0: dropless; else C = ceil(cf*T*top_k/E), exact on this fp32 */
   float aux_alpha;      /* load-balancing loss weight (0.01 on the Quartz pages) */
+  int32_t expert_storage; /* moe_storage_t of the routed experts' weights (0: dtype) */
 } moe_config_t;
 
 /* Weights, all device pointers in dtype unless noted; [a,b,c] = row-major shape. */
@@ -87,6 +94,12 @@ typedef struct {
   const void *ws_gate;       /* shared: [n_shared, ffn_shared, d] */
   const void *ws_up;         /* shared: [n_shared, ffn_shared, d] */
   const void *ws_down;       /* shared: [n_shared, d, ffn_shared] */
+  /* MOE_STORAGE_FP8_E4M3 only (then lr_V and lr_U are not read), as moe_quantize_fp8 writes
+   * them from V and U: */
+  const uint8_t *lr_V8;      /* [E, rank, d] E4M3 codes */
+  const float *lr_V_scale;   /* [E, rank] fp32 row scales */
+  const uint8_t *lr_U8;      /* [E, d, rank] E4M3 codes */
+  const float *lr_U_scale;   /* [E, d] fp32 row scales */
 } moe_weights_t;
 
 /* Bytes of workspace that every call below needs for `cfg` (the largest, moe_layer_forward).
@@ -142,7 +155,13 @@ moe_status_t moe_permute(const moe_config_t *cfg, const void *x, const int32_t *
  * averages its rounding; a low-rank layer's y can be a sum of as few as two rows with no shared
  * output, where one bf16 rounding alone exceeds the error budget.
  * y_shared: [T, d] fp32 (the S shared outputs summed in fp32), may be NULL when n_shared = 0;
- * it enters y alone, so it stays fp32. */
+ * it enters y alone, so it stays fp32.
+ * fp8 storage (expert_storage = MOE_STORAGE_FP8_E4M3): each x_perm row is quantised as
+ * moe_quantize_fp8 does (its E4M3 codes xq, scale sx), then per expert e, on the fp8 tensor
+ * cores with fp32 sums:
+ *   z = (xq V8[e]^T) * sx * V_scale[e] * s[e]  (per column);  zq, sz = the quantised rows of z;
+ *   y_perm[r] = (zq U8[e]^T) * sz * U_scale[e]  (fp32).
+ * The shared experts keep the layer's dtype. */
 moe_status_t moe_expert_forward(const moe_config_t *cfg, const void *x_perm,
                                 const int32_t *offsets, const void *x,
                                 const moe_weights_t *w, void *y_perm, void *y_shared,
@@ -158,11 +177,11 @@ moe_status_t moe_expert_forward(const moe_config_t *cfg, const void *x_perm,
 moe_status_t moe_combine(const moe_config_t *cfg, const void *y_perm, const void *y_shared,
                          const int32_t *slot_pos, const float *topk_w, void *y, void *stream);
 
-/* Backward pass, first steps. The pages train with this layer but do not write its backward
- * out; it is the derivative of the forward, of J = sum(dy * y) + dL * loss, with no gradient
- * through the selection (top-k, capacity drops, the loss's counts), none for the selection bias
- * or the logit offsets, and each logit's fp32 rounding taken with derivative 1. The grouped
- * expert GEMMs of the backward are not part of the library yet.
+/* Backward pass. The pages train with this layer but do not write its backward out; it is the
+ * derivative of the forward, of J = sum(dy * y) + dL * loss, with no gradient through the
+ * selection (top-k, capacity drops, the loss's counts), none for the selection bias or the logit
+ * offsets, and each logit's fp32 rounding taken with derivative 1. Three calls: this one, the
+ * experts' (moe_expert_backward) and the router's (moe_route_backward).
  *
  * Backward of moe_combine (Moonfrost expert card: a token's output sums its shared and top-k
  * routed experts). For every kept pair (t, j), p = slot_pos[t, j] >= 0:
@@ -298,6 +317,21 @@ moe_status_t moe_layer_forward(const moe_config_t *cfg, const void *x, const moe
 moe_status_t moe_route_noalloc(const moe_config_t *cfg, const void *x, const moe_weights_t *w,
                                int32_t *topk_idx, float *topk_w, int32_t *expert_count,
                                float *prob_sum, void *stream);
+
+/* Per-row E4M3 quantisation, the fp8 storage of moe_storage_t (dormouse, "TSCT low-rank
+ * experts": the storage ladder fp8 -> NVFP4 -> ternary of the U*diag(s)*V^T factorisation; the
+ * pages fix no scale granularity or rounding, so this is one scale per row and round to nearest).
+ * For every row v of `in` ([rows, cols], row-major; in_dtype MOE_DTYPE_BF16 or MOE_DTYPE_F32):
+ *   amax = max_i |v_i|;  scale[row] = RN32(amax / 448), or 1 for an all-zero row;
+ *   q[row, i] = E4M3 code of RN32(v_i / scale[row]), rounded to the nearest E4M3 value with ties
+ *   to the even code and magnitudes above 448 saturated (E4M3: 1 sign, 4 exponent bits of bias 7,
+ *   3 mantissa bits, largest finite 448; OCP FP8).
+ * q: [rows, cols] uint8; scale: [rows] fp32; cols a multiple of 16; inputs finite. The weights of
+ * an fp8 low-rank layer are lr_V8 / lr_V_scale = moe_quantize_fp8(V viewed as [E*rank, d]) and
+ * lr_U8 / lr_U_scale = moe_quantize_fp8(U viewed as [E*d, rank]). Asynchronous on `stream`; bad
+ * arguments return MOE_ERR_INVALID_ARG or MOE_ERR_UNSUPPORTED with nothing enqueued. */
+moe_status_t moe_quantize_fp8(const void *in, int32_t in_dtype, int64_t rows, int32_t cols,
+                              uint8_t *q, float *scale, void *stream);
 
 /* Human-readable name of a status. Never NULL. */
 const char *moe_status_str(moe_status_t s);

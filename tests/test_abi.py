@@ -50,6 +50,26 @@ def cfg_of(c, **kw):
     return B.make_config(**d)
 
 
+def test_fp8_storage_only_for_bf16_lowrank(lib):
+    """E4M3 expert storage is a rung of the low-rank experts' ladder, for bf16 layers only."""
+    assert B.moe_workspace_size(cfg_of(CONFIGS["lowrank"], expert_storage="fp8")) > 0
+    for name in ("quartz", "tiny_f32"):
+        assert B.moe_workspace_size(cfg_of(CONFIGS[name], expert_storage="fp8")) == 0
+    assert B.moe_workspace_size(cfg_of(CONFIGS["lowrank"], dtype="f32", expert_storage="fp8")) == 0
+    bad = cfg_of(CONFIGS["lowrank"])
+    bad.expert_storage = 7
+    assert B.moe_workspace_size(bad) == 0
+
+
+def test_quantize_fp8_host_refusals(lib):
+    # cols not a multiple of 16, a bad dtype, negative rows: refused before any device work
+    assert lib.moe_quantize_fp8(None, 1, 4, 24, None, None, None) == 2
+    assert lib.moe_quantize_fp8(None, 9, 4, 32, None, None, None) == 2
+    assert lib.moe_quantize_fp8(None, 1, -1, 32, None, None, None) == 1
+    assert lib.moe_quantize_fp8(None, 1, 0, 32, None, None, None) == B.MOE_OK
+    assert lib.moe_quantize_fp8(None, 1, 4, 32, None, None, None) == 1
+
+
 @pytest.mark.parametrize("name", sorted(CONFIGS))
 def test_workspace_size_and_capacity(lib, name):
     c = CONFIGS[name]
