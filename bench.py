@@ -82,12 +82,12 @@ def captured_traffic(config_name: str, kernel: str):
     return int(vals[kernel]) if kernel in vals else None
 
 
-def workload_name(c) -> str:
-    parts = [f"{c.name}: T={c.T} d={c.d} E={c.E} top-{c.top_k} {c.score}"]
+def workload_name(c, fp8: bool = False) -> str:
+    parts = [f"{c.name}{'_fp8' if fp8 else ''}: T={c.T} d={c.d} E={c.E} top-{c.top_k} {c.score}"]
     if c.expert == "swiglu":
         parts.append(f"SwiGLU ffn {c.ffn}")
     else:
-        parts.append(f"low-rank r={c.rank}")
+        parts.append(f"low-rank r={c.rank}" + (", U and V stored as E4M3 rows" if fp8 else ""))
     parts.append(f"{c.n_shared} shared" + (f" (ffn {c.ffn_shared})" if c.n_shared else ""))
     parts.append("dropless" if c.capacity_factor <= 0 else f"capacity factor {c.capacity_factor}")
     parts.append(c.dtype)
@@ -166,26 +166,45 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------ algorithmic work
-def algorithmic(c, n_kept: int):
+def algorithmic(c, n_kept: int, fp8: bool = False, active=None):
     """Per-launch algorithmic flops / bytes of each kernel kind (kept rows only, each input
-    read once, no tile padding)."""
-    T, d, E, k, S, fs = c.T, c.d, c.E, c.top_k, c.n_shared, c.ffn_shared
+    read once, each output written once, no tile padding). fp8: the low-rank experts' E4M3
+    storage (codes of 1 byte, fp32 z, the quantiser's two launches per step). `active`: the
+    experts that receive rows (only their weights are read); all E when not given."""
+    T, d, k, S, fs = c.T, c.d, c.top_k, c.n_shared, c.ffn_shared
+    E = c.E if active is None else active
+    N = n_kept
     es = 2 if c.dtype == "bf16" else 4
     out = {}
-    out["router"] = {"flops": 2.0 * T * d * E, "bytes": T * d * es + E * d * es + 8.0 * T * k}
-    perm_bytes = T * d * es + n_kept * d * es + 16.0 * T * k
-    out["perm_scatter"] = {"bytes": perm_bytes}
+    out["router"] = {"flops": 2.0 * T * d * c.E, "bytes": T * d * es + c.E * d * es + 8.0 * T * k}
+    # fp8: bf16 token rows in, their E4M3 codes and scales out
+    out["perm_scatter"] = {"bytes": T * d * es + N * d * (1 if fp8 else es) + 16.0 * T * k +
+                           (4.0 * N if fp8 else 0)}
+    sh_flops_gu, sh_flops_dn = 4.0 * d * S * fs * T, 2.0 * d * S * fs * T
+    sh_bytes_gu = (T * d + 2.0 * S * fs * d + T * S * fs) * es
+    sh_bytes_dn = (T * S * fs + S * fs * d) * es + T * d * 4.0
     if c.expert == "swiglu":
         f = c.ffn
-        out["gemm_gateup"] = {"flops": 4.0 * d * f * n_kept + 4.0 * d * S * fs * T}
-        out["gemm_down"] = {"flops": 2.0 * d * f * n_kept + 2.0 * d * S * fs * T}
+        ys = 2 if c.dtype == "bf16" else 4
+        out["gemm_gateup"] = {"flops": 4.0 * d * f * N + sh_flops_gu,
+                              "bytes": (N * d + 2.0 * E * f * d + N * f) * es + sh_bytes_gu}
+        out["gemm_down"] = {"flops": 2.0 * d * f * N + sh_flops_dn,
+                            "bytes": (N * f + E * d * f) * es + N * d * ys + sh_bytes_dn}
     else:
         r = c.rank
-        out["gemm_lowrank_v"] = {"flops": 2.0 * d * r * n_kept}
-        out["gemm_lowrank_u"] = {"flops": 2.0 * d * r * n_kept}
+        if fp8:  # codes of z and their scales written by the V product itself
+            out["gemm_lowrank_v"] = {"flops": 2.0 * d * r * N, "bytes": N * d + E * r * d +
+                                     N * r + 4.0 * (2 * N + 2 * E * r)}
+            out["gemm_lowrank_u"] = {"flops": 2.0 * d * r * N, "bytes": N * r + E * d * r +
+                                     N * d * 4.0 + 4.0 * (N + E * d)}
+        else:
+            out["gemm_lowrank_v"] = {"flops": 2.0 * d * r * N,
+                                     "bytes": (N * d + E * r * d + N * 2 * r) * es}
+            out["gemm_lowrank_u"] = {"flops": 2.0 * d * r * N,
+                                     "bytes": (N * 2 * r + E * d * r) * es + N * d * 4.0}
         if S:
-            out["gemm_gateup"] = {"flops": 4.0 * d * S * fs * T}
-            out["gemm_down"] = {"flops": 2.0 * d * S * fs * T}
+            out["gemm_gateup"] = {"flops": sh_flops_gu, "bytes": sh_bytes_gu}
+            out["gemm_down"] = {"flops": sh_flops_dn, "bytes": sh_bytes_dn}
     # routed expert rows (bf16 for bf16 SwiGLU layers, else fp32), shared output and y in fp32
     ys = 2 if (c.dtype == "bf16" and c.expert == "swiglu") else 4
     out["combine"] = {"bytes": n_kept * d * ys + (T * d * 4.0 if S else 0) + 8.0 * T * k +
@@ -195,11 +214,14 @@ def algorithmic(c, n_kept: int):
     return out
 
 
-def roofline_table(c, n_kept, prof, steps, peaks, src, in_step=None):
+def roofline_table(c, n_kept, prof, steps, peaks, src, in_step=None, fp8=False, active=None):
     """Achieved vs peak per kernel kind from the profiler's per-launch averages (CUDA events
     around each launch) and, when given, from the in-step durations (device timestamps, the
-    launches overlapped as in the step): `in_step_us` and `frac_in_step`."""
-    alg = algorithmic(c, n_kept)
+    launches overlapped as in the step): `in_step_us` and `frac_in_step`. A GEMM is held to the
+    tensor peak when its flops per byte exceed the machine's (peak flops / peak HBM bandwidth),
+    else to the HBM bandwidth (the low-rank products: K = rank); fp8 products take the measured
+    bf16 peak times the nominal fp8 / bf16 ratio of 2."""
+    alg = algorithmic(c, n_kept, fp8, active)
     # fp32 FMA on the CUDA cores: 148 SMs x 128 lanes x 2 flops at the maximum SM clock
     fp32_peak = 148 * 128 * 2 * peaks.get("sm_max_mhz", 1965.0) * 1e6 / 1e12  # TFLOP/s, nominal
     rows = {}
@@ -210,9 +232,16 @@ def roofline_table(c, n_kept, prof, steps, peaks, src, in_step=None):
         a = alg.get(name, {})
         row = {"launches": n, "avg_us": avg_ms * 1e3, "share": None}
         if name.startswith("gemm"):
-            ach = a["flops"] / (avg_ms * 1e-3) / 1e12
-            row.update(bound="tensor", achieved=ach, peak=peaks["bf16_tflops"], unit="TFLOP/s",
-                       frac=ach / peaks["bf16_tflops"])
+            tpeak = peaks["bf16_tflops"] * (2.0 if fp8 and "lowrank" in name else 1.0)
+            ridge = tpeak * 1e12 / (peaks["hbm_gbs"] * 1e9)
+            tflops = a["flops"] / (avg_ms * 1e-3) / 1e12
+            gbs = a["bytes"] / (avg_ms * 1e-3) / 1e9
+            if a["flops"] / a["bytes"] >= ridge:
+                row.update(bound="tensor", achieved=tflops, peak=tpeak, unit="TFLOP/s",
+                           frac=tflops / tpeak, hbm_gbs=gbs)
+            else:
+                row.update(bound="hbm", achieved=gbs, peak=peaks["hbm_gbs"], unit="GB/s",
+                           frac=gbs / peaks["hbm_gbs"], tflops=tflops)
         elif name == "router":
             ach = a["flops"] / (avg_ms * 1e-3) / 1e12
             row.update(bound="alu", achieved=ach, peak=fp32_peak, unit="TFLOP/s (fp32 FMA)",
@@ -507,12 +536,13 @@ def measure_config(name, K, W, dev, flush, stream, peaks, peak_src):
     from fine_grained_mixture_moe_b200.layer import MoELayer, upload_weights
     from moe_synth import get_config, make_inputs
 
-    c = get_config(name)
+    fp8 = name.endswith("_fp8")  # a configuration's low-rank experts stored as E4M3 rows
+    c = get_config(name[:-4] if fp8 else name)
     inp = make_inputs(c)
     cfg = B.make_config(T=c.T, d=c.d, E=c.E, top_k=c.top_k, n_shared=c.n_shared, ffn=c.ffn,
                         ffn_shared=c.ffn_shared, rank=c.rank, score=c.score, expert=c.expert,
                         dtype=c.dtype, norm_topk=c.norm_topk, capacity_factor=c.capacity_factor,
-                        aux_alpha=c.aux_alpha)
+                        aux_alpha=c.aux_alpha, expert_storage="fp8" if fp8 else "dtype")
     layer = MoELayer(cfg, upload_weights(cfg, inp, dev), dev)
     x = torch.as_tensor(inp["x"]).to(layer.dtype).contiguous().to(dev)
     y = torch.empty((c.T, c.d), dtype=torch.float32, device=dev)
@@ -555,9 +585,10 @@ def measure_config(name, K, W, dev, flush, stream, peaks, peak_src):
     torch.cuda.synchronize()
     n_kept = int(offs[-1])
     counts = cnt.cpu().numpy()
-    table = roofline_table(c, n_kept, prof, K, peaks, peak_src, in_step)
+    table = roofline_table(c, n_kept, prof, K, peaks, peak_src, in_step, fp8,
+                           int((counts > 0).sum()))
     out = {
-        "workload": workload_name(c),
+        "workload": workload_name(c, fp8),
         "value": c.T / (ms * 1e-3), "unit": "tokens/s", "ms_per_step": ms, "steps": K,
         "warmup": W, "dtype": c.dtype,
         "kept_pairs": n_kept, "dropped_pairs": c.T * c.top_k - n_kept,
@@ -755,7 +786,7 @@ def main():
     ap.add_argument("--config", default="quartz")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--per-config", default="capacity,sigmoid,lowrank",
+    ap.add_argument("--per-config", default="capacity,sigmoid,lowrank,lowrank_fp8",
                     help="further configurations timed on one GPU beside the headline one "
                          "(comma-separated names, or 'none')")
     args = ap.parse_args()

@@ -83,14 +83,6 @@ struct GuFeed {
   }
 };
 
-// 32 contiguous bytes to global memory in one store (dst 32-byte aligned): a whole L2 sector, so
-// the sector is never written in halves.
-__device__ __forceinline__ void st_global_32B(void *dst, const uint32_t (&v)[8]) {
-  asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(dst), "r"(v[0]),
-               "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
-               : "memory");
-}
-
 // SWIGLU_BWD: the lane's row of dh (r0, 32 columns) with g and u of the same row and columns
 // from the warp's block pair in shared memory; writes dg, du and h as hi + lo bf16 terms to
 // o[col..] (dg_hi), o + hf (du_hi), o + 2 hf (dg_lo), o + 3 hf (du_lo), o2 (h_hi), o2 + hf (h_lo),

@@ -44,7 +44,7 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
 // Kinds of the library's forward kernels (the host's profiler and the device stamps share them).
 enum KernelKind {
   K_ROUTER, K_STATS, K_PERM_HIST, K_PERM_SCATTER, K_GEMM_GATEUP, K_GEMM_DOWN, K_GEMM_LR1,
-  K_GEMM_LR2, K_COMBINE, K_AUX, K_BWD_GEMM, K_COUNT
+  K_GEMM_LR2, K_COMBINE, K_AUX, K_BWD_GEMM, K_QUANT, K_COUNT
 };
 
 // In-step timestamps. With stamping on (moe_debug_set(MOE_DEBUG_STAMP, 1)) a kernel records, per
@@ -173,6 +173,14 @@ template <typename T> __device__ __forceinline__ T *cluster_map(T *p, uint32_t r
 __device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void griddep_launch() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// 32 contiguous bytes to global memory in one store (dst 32-byte aligned): a whole L2 sector, so
+// the sector is never written in halves.
+__device__ __forceinline__ void st_global_32B(void *dst, const uint32_t (&v)[8]) {
+  asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(dst), "r"(v[0]),
+               "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
+               : "memory");
 }
 
 // ---------------------------------------------------------------- mbarriers (shared memory)

@@ -40,7 +40,9 @@ __global__ void __launch_bounds__(256) quantize_rows_kernel(const Tin *__restric
                                                             long long rows, int cols,
                                                             uint8_t *__restrict__ q,
                                                             float *__restrict__ scale) {
+  const KernelStamp stamp(K_QUANT);
   griddep_wait();
+  stamp.started();
   griddep_launch();
   const int lane = threadIdx.x & 31;
   const long long nwarps = (long long)gridDim.x * (blockDim.x >> 5);

@@ -20,6 +20,7 @@
 // it has in flight (again bounded), frees its TMEM and returns.
 #pragma once
 #include <cuda.h>
+#include "fp8.cuh"
 #include "grouped.cuh"
 
 namespace moe {
@@ -47,8 +48,11 @@ template <int MODE, int BN> struct TcCfg {
   static constexpr int A_BYTES = TC_BM * 128;                     // 16 KB: 128-byte rows
   static constexpr int B_BYTES = BN * 128;
   static constexpr int STAGE_BYTES = A_BYTES + NB * B_BYTES;
-  static constexpr bool F32_OUT = MODE == MODE_PLAIN || MODE == MODE_SCALE_FP8;
-  static constexpr int STG_BYTES = F32_OUT ? TC_EPI_WARPS * 4096 : 0;  // fp32 staging
+  static constexpr bool F32_OUT = MODE == MODE_PLAIN;
+  // PLAIN: per-warp fp32 staging; SCALE_FP8: the row maxima of the two column halves, per
+  // accumulator buffer [2][2][128]
+  static constexpr int STG_BYTES = F32_OUT ? TC_EPI_WARPS * 4096
+                                           : MODE == MODE_SCALE_FP8 ? 2 * 2 * TC_BM * 4 : 0;
   static constexpr int STAGES = (200 * 1024 - STG_BYTES) / STAGE_BYTES > 8
                                     ? 8 : (200 * 1024 - STG_BYTES) / STAGE_BYTES;
   static constexpr int ACC_COLS = NB * BN;                        // fp32 columns per buffer
@@ -331,9 +335,62 @@ __global__ void __launch_bounds__(TC_THREADS, 1) gemm_tc_kernel(const __grid_con
       // both the row-wise writes and the column-wise reads are conflict-free), then leave as 32
       // row stores of 128 contiguous bytes each instead of 32-row scattered 16-byte stores.
       unsigned char *stg = stg_all + (warp - 2) * 4096;
+      if (MODE == MODE_SCALE_FP8) {
+        // z = sum * (row scale) * (V row scale) * s, then the row's E4M3 codes and scale (the
+        // tile is the whole row: BN = N). Pass 1: each of the two warps of this lane quarter
+        // takes the maximum |z| over its half of the row; they meet at a named barrier (both
+        // passed the same accumulator wait, so both arrive); pass 2 recomputes z, converts and
+        // stores 32 codes per 32-byte store. rs = 0 on rows past the group: their z is not used.
+        float *s_am = (float *)stg_all;
+        const float rs = row_ok ? __ldg(p.row_scale + ti.a_row0 + row) : 0.0f;
+        const float4 *cs = (const float4 *)(p.col_scale + (size_t)ti.g * ti.N);
+        const float4 *ss = (const float4 *)(p.scale + (size_t)ti.g * ti.N);
+        auto zchunk = [&](int c, float (&z)[32]) {
+          uint32_t r0[32];
+          __syncwarp();  // the collective TMEM load runs converged
+          tmem_ld32(tbase + c, r0);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const float4 v = __ldg(cs + c / 4 + i), w = __ldg(ss + c / 4 + i);
+            z[4 * i] = __uint_as_float(r0[4 * i]) * rs * v.x * w.x;
+            z[4 * i + 1] = __uint_as_float(r0[4 * i + 1]) * rs * v.y * w.y;
+            z[4 * i + 2] = __uint_as_float(r0[4 * i + 2]) * rs * v.z * w.z;
+            z[4 * i + 3] = __uint_as_float(r0[4 * i + 3]) * rs * v.w * w.w;
+          }
+        };
+        float am = 0.0f;
+#pragma unroll 1
+        for (int c = cbeg; c < cend; c += 32) {
+          float z[32];
+          zchunk(c, z);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) am = fmaxf(am, fabsf(z[i]));
+        }
+        s_am[(acc * 2 + half) * TC_BM + q * 32 + lane] = am;
+        asm volatile("bar.sync %0, 64;" ::"r"(1 + q) : "memory");
+        am = fmaxf(s_am[(acc * 2) * TC_BM + q * 32 + lane], s_am[(acc * 2 + 1) * TC_BM + q * 32 + lane]);
+        const float sc = am > 0.0f ? __fdiv_rn(am, E4M3_MAX) : 1.0f;
+        if (half == 0 && row_ok) ((float *)p.out2_r)[ti.a_row0 + row] = sc;
+#pragma unroll 1
+        for (int c = cbeg; c < cend; c += 32) {  // warp-uniform: tcgen05.ld is collective
+          float z[32];
+          zchunk(c, z);
+          if (row_ok) {  // rows past the group: no conversion, no store
+            uint32_t w8[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              w8[i] = e4m3_code(__fdiv_rn(z[4 * i], sc)) |
+                      (e4m3_code(__fdiv_rn(z[4 * i + 1], sc)) << 8) |
+                      (e4m3_code(__fdiv_rn(z[4 * i + 2], sc)) << 16) |
+                      (e4m3_code(__fdiv_rn(z[4 * i + 3], sc)) << 24);
+            st_global_32B((uint8_t *)out + (size_t)(ti.a_row0 + row) * ldo + ti.n0 + c, w8);
+          }
+        }
+      }
       constexpr int SUB = C::F32_OUT ? 1 : 2;  // 32-column TMEM loads per block
 #pragma unroll 1
-      for (int c = cbeg; c < cend; c += 32 * SUB) {
+      for (int c = cbeg; c < (MODE == MODE_SCALE_FP8 ? cbeg : cend); c += 32 * SUB) {
         if (MODE == MODE_SCALE) {
           // bf16 low-rank projection: each lane already writes 64 contiguous bytes of its row, so
           // they go out directly
@@ -394,16 +451,6 @@ __global__ void __launch_bounds__(TC_THREADS, 1) gemm_tc_kernel(const __grid_con
           uint32_t r0[32];
           tmem_ld32(tbase + c, r0);
           tmem_wait_ld();
-          if (MODE == MODE_SCALE_FP8 && row_ok && ti.n0 + c < ti.N) {
-            // z = sum * (row scale) * (V row scale) * s, for columns col .. col + 31 (N is a
-            // multiple of 32)
-            const size_t cn = (size_t)ti.g * ti.N + ti.n0 + c;
-            const float rs = __ldg(p.row_scale + ti.a_row0 + row);
-#pragma unroll
-            for (int i = 0; i < 32; ++i)
-              r0[i] = __float_as_uint(__uint_as_float(r0[i]) * rs * __ldg(p.col_scale + cn + i) *
-                                      __ldg(p.scale + cn + i));
-          }
 #pragma unroll
           for (int i = 0; i < 8; ++i)
             *(uint4 *)(stg + lane * 128 + ((i ^ (lane & 7)) << 4)) =

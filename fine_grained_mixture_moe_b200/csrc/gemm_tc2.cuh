@@ -427,11 +427,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TC_THREADS, 1)
           tmem_wait_ld();
           if (MODE == MODE_PLAIN_FP8 && routed && row_ok && ti.n0 + c < ti.N) {
             // y = sum * (row scale) * (U row scale), columns col .. col + 31
-            const size_t cn = (size_t)ti.g * ti.N + ti.n0 + c;
+            const float4 *cs = (const float4 *)(p.col_scale + (size_t)ti.g * ti.N + ti.n0 + c);
             const float rs = __ldg(p.row_scale + ti.a_row0 + row);
 #pragma unroll
-            for (int i = 0; i < 32; ++i)
-              r0[i] = __float_as_uint(__uint_as_float(r0[i]) * rs * __ldg(p.col_scale + cn + i));
+            for (int i = 0; i < 8; ++i) {
+              const float4 v = __ldg(cs + i);
+              r0[4 * i] = __float_as_uint(__uint_as_float(r0[4 * i]) * rs * v.x);
+              r0[4 * i + 1] = __float_as_uint(__uint_as_float(r0[4 * i + 1]) * rs * v.y);
+              r0[4 * i + 2] = __float_as_uint(__uint_as_float(r0[4 * i + 2]) * rs * v.z);
+              r0[4 * i + 3] = __float_as_uint(__uint_as_float(r0[4 * i + 3]) * rs * v.w);
+            }
           }
 #pragma unroll
           for (int i = 0; i < 8; ++i)

@@ -18,7 +18,9 @@
 //                   dg_hi, out[., half + n] = du_hi, out[., 2 half + n] = dg_lo,
 //                   out[., 3 half + n] = du_lo, out2[., n] = h_hi, out2[., half + n] = h_lo.
 //                 SCALE_FP8 (E4M3 operands) z = (A B0^T) * row_scale[row] * col_scale[g][n]
-//                   * scale[g][n], fp32 out (the low-rank V projection with fp8 storage);
+//                   * scale[g][n] (the low-rank V projection with fp8 storage), stored as the
+//                   row's E4M3 codes to out (bytes) and its scale to out2 (fp32 per row), as
+//                   quantize_rows_kernel would make them from z; the tile is the whole row (N);
 //                 PLAIN_FP8 (E4M3 operands) out = (A B0^T) * row_scale[row] * col_scale[g][n],
 //                   fp32 out (the U projection). E4M3 operands have K-blocks of 128 elements
 //                   (128 bytes, as for bf16); a K that is not a multiple of 128 is completed with

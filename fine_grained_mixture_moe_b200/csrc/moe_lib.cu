@@ -46,8 +46,10 @@ bool cfg_supported(const moe_config_t *c) {
   if (c->n_shared > 0 && (c->ffn_shared <= 0 || c->ffn_shared % 64)) return false;
   if (c->expert_storage != MOE_STORAGE_DTYPE && c->expert_storage != MOE_STORAGE_FP8_E4M3)
     return false;
+  // fp8 storage: bf16 low-rank layers; the quantising scatter holds a row in registers
   if (c->expert_storage == MOE_STORAGE_FP8_E4M3 &&
-      (c->expert != MOE_EXPERT_LOWRANK || c->dtype != MOE_DTYPE_BF16))
+      (c->expert != MOE_EXPERT_LOWRANK || c->dtype != MOE_DTYPE_BF16 ||
+       c->d > 32 * PM_VEC * 8))
     return false;
   if (!std::isfinite(c->capacity_factor) || !std::isfinite(c->aux_alpha)) return false;
   // the router stages its 16 token rows and the logits in shared memory (227 KB per CTA)
@@ -108,7 +110,7 @@ struct Layout {
   size_t lrank;                                                 // within-chunk ranks [T, k] u8
   size_t hidden, hidden_sh;                                     // experts
   size_t idx, wts, count, prob, offsets, slot_pos, src, x_perm, y_perm, y_shared, aux;  // layer
-  size_t xq, sx, sx_perm, zq, sz;  // fp8 storage: E4M3 token rows and z rows, their scales
+  size_t sx_perm, zq, sz;  // fp8 storage: scales of the E4M3 token rows, z rows and scales
   size_t total;
 };
 inline bool fp8_experts(const moe_config_t *c) { return c->expert_storage == MOE_STORAGE_FP8_E4M3; }
@@ -117,10 +119,11 @@ Layout layout_of(const moe_config_t *c) {
   Layout L;
   const size_t T = c->T, d = c->d, E = c->E, k = c->top_k, es = esize(c);
   const size_t nch = std::max<size_t>(1, ceil_div(c->T, RT_TM));
-  // hidden rows: the SwiGLU activations, or the low-rank projection (bf16: hi and lo terms)
-  const size_t width = c->expert == MOE_EXPERT_SWIGLU
-                           ? (size_t)c->ffn
-                           : (size_t)c->rank * (c->dtype == MOE_DTYPE_BF16 ? 2 : 1);
+  // hidden rows: the SwiGLU activations, or the low-rank projection (bf16: hi and lo terms;
+  // fp8 storage: none, its E4M3 rows are `zq`)
+  const size_t width = c->expert == MOE_EXPERT_SWIGLU ? (size_t)c->ffn
+                       : fp8_experts(c)               ? 0
+                       : (size_t)c->rank * (c->dtype == MOE_DTYPE_BF16 ? 2 : 1);
   size_t o = 0;
   auto take = [&](size_t bytes) { size_t at = o; o = align256(o + std::max<size_t>(bytes, 1)); return at; };
   L.part_cnt = take(nch * E * 4);
@@ -142,10 +145,8 @@ Layout layout_of(const moe_config_t *c) {
   L.y_perm = take(T * k * d * (yperm_bf16(c) ? 2 : 4));
   L.y_shared = take(T * d * 4);
   L.aux = take(16);
-  // fp8 storage: the x_perm region holds the rows' E4M3 codes and `hidden` the fp32 z
+  // fp8 storage: the x_perm region holds the rows' E4M3 codes
   const bool f8 = fp8_experts(c);
-  L.xq = take(f8 ? T * d : 0);
-  L.sx = take(f8 ? T * 4 : 0);
   L.sx_perm = take(f8 ? T * k * 4 : 0);
   L.zq = take(f8 ? T * k * (size_t)c->rank : 0);
   L.sz = take(f8 ? T * k * 4 : 0);
@@ -181,7 +182,7 @@ int num_sms() {
 // ------------------------------------------------------------------ profiling (debug)
 const char *kKindName[K_COUNT] = {"router", "stats", "perm_hist", "perm_scatter", "gemm_gateup",
                                   "gemm_down", "gemm_lowrank_v", "gemm_lowrank_u", "combine",
-                                  "aux_loss", "backward_gemm"};
+                                  "aux_loss", "backward_gemm", "quantize_fp8"};
 constexpr int PROF_SLOTS = 8192;
 struct Prof {
   bool on = false;
@@ -466,16 +467,30 @@ template <typename Tin>
 moe_status_t scatter_impl(const moe_config_t *c, const void *x, const int32_t *idx,
                           const uint8_t *lrank, const int32_t *chunk_base, const int32_t *kept,
                           int32_t *offsets, int32_t *slot_pos, int32_t *src, void *x_perm,
-                          const int32_t *count, const float *prob, float *aux, cudaStream_t st,
-                          const float *rs_in = nullptr, float *rs_out = nullptr) {
+                          const int32_t *count, const float *prob, float *aux, cudaStream_t st) {
   ProfScope ps(K_PERM_SCATTER, st);
   const size_t smem = (size_t)c->E * sizeof(int);  // the expert offsets
   const int grid = std::max(1, std::min(ceil_div(c->T, PM_THREADS / 32),
                                         num_sms() * PM_CTAS_PER_SM));
   return launch_pdl(perm_scatter_kernel<Tin>, dim3(grid), dim3(PM_THREADS), smem, st, idx, lrank,
                     c->T, c->top_k, c->E, capacity_of(c), chunk_base, kept, offsets, slot_pos,
-                    src, (const Tin *)x, (Tin *)x_perm, c->d, count, prob, c->aux_alpha, aux,
-                    rs_in, rs_out);
+                    src, (const Tin *)x, (Tin *)x_perm, c->d, count, prob, c->aux_alpha, aux);
+}
+
+// The scatter of a layer with E4M3 experts: bf16 token rows in, their codes and scales out.
+moe_status_t scatter_q8_impl(const moe_config_t *c, const void *x, const int32_t *idx,
+                             const uint8_t *lrank, const int32_t *chunk_base, const int32_t *kept,
+                             int32_t *offsets, int32_t *slot_pos, int32_t *src, uint8_t *xq_perm,
+                             float *sx_perm, const int32_t *count, const float *prob, float *aux,
+                             cudaStream_t st) {
+  ProfScope ps(K_PERM_SCATTER, st);
+  const size_t smem = (size_t)c->E * sizeof(int);
+  const int grid = std::max(1, std::min(ceil_div(c->T, PM_THREADS / 32),
+                                        num_sms() * PM_CTAS_PER_SM));
+  return launch_pdl(perm_scatter_q8_kernel, dim3(grid), dim3(PM_THREADS), smem, st, idx, lrank,
+                    c->T, c->top_k, c->E, capacity_of(c), chunk_base, kept, offsets, slot_pos,
+                    src, (const __nv_bfloat16 *)x, xq_perm, sx_perm, c->d, count, prob,
+                    c->aux_alpha, aux);
 }
 
 // Per-row E4M3 quantisation (fp8.cuh) of `rows` rows of `cols` elements.
@@ -484,6 +499,7 @@ moe_status_t launch_quantize(const void *in, long long rows, int cols, uint8_t *
                              cudaStream_t st) {
   if (rows == 0) return MOE_OK;
   const int grid = (int)std::min<long long>((rows + 7) / 8, (long long)num_sms() * 16);
+  ProfScope ps(K_QUANT, st);
   return launch_pdl(quantize_rows_kernel<Tin>, dim3(grid), dim3(256), 0, st, (const Tin *)in,
                     rows, cols, q, scale);
 }
@@ -534,16 +550,15 @@ moe_status_t lowrank_shared_impl(const moe_config_t *c, const GroupedGemm &g, co
 }
 
 // Low-rank experts stored in E4M3 on their grouped rows (codes xq_perm, scales sx_perm):
-// z = (xq V8^T) * sx * V_scale * s (fp32, fp8 tensor cores) -> per-row E4M3 of z ->
+// z = (xq V8^T) * sx * V_scale * s (fp32 sums on the fp8 tensor cores), quantised per row in the
+// same kernel's epilogue (its tile is the whole row: BN = rank) -> zq, sz;
 // y_perm = (zq U8^T) * sz * U_scale (fp32). The rank K = r of the second product is completed to
-// a 128-element stage by the tensor map's zero fill. Rows past the kept count are quantised too
-// (the host does not know the count); nothing reads them.
+// a 128-element stage by the tensor map's zero fill.
 moe_status_t experts_fp8_impl(const moe_config_t *c, const uint8_t *xq_perm, const float *sx_perm,
                               const int32_t *offsets, const void *x, const moe_weights_t *w,
                               void *y_perm, void *y_shared, void *ws, cudaStream_t st) {
   const Layout L = layout_of(c);
   const int T = c->T, d = c->d, E = c->E, k = c->top_k, r = c->rank;
-  float *Z = at<float>(ws, L.hidden);
   uint8_t *zq = at<uint8_t>(ws, L.zq);
   float *sz = at<float>(ws, L.sz);
   GroupedGemm g;
@@ -553,10 +568,15 @@ moe_status_t experts_fp8_impl(const moe_config_t *c, const uint8_t *xq_perm, con
   g.rows_r = T * k;
   GroupedGemm g1 = g;
   g1.E = E; g1.A_r = xq_perm; g1.lda_r = d; g1.B0_r = w->lr_V8; g1.N_r = r; g1.K_r = d;
-  g1.out_r = Z; g1.ldo_r = r; g1.scale = w->lr_s; g1.row_scale = sx_perm;
+  g1.out_r = zq; g1.ldo_r = r; g1.out2_r = sz; g1.scale = w->lr_s; g1.row_scale = sx_perm;
   g1.col_scale = w->lr_V_scale;
-  MOE_TRY((launch_tc<MODE_SCALE_FP8, 64>(g1, st, K_GEMM_LR1)));
-  MOE_TRY(launch_quantize<float>(Z, (long long)T * k, r, zq, sz, st));
+  switch (r) {  // rank: a multiple of 64 up to 256
+    case 64: MOE_TRY((launch_tc<MODE_SCALE_FP8, 64>(g1, st, K_GEMM_LR1))); break;
+    case 128: MOE_TRY((launch_tc<MODE_SCALE_FP8, 128>(g1, st, K_GEMM_LR1))); break;
+    case 192: MOE_TRY((launch_tc<MODE_SCALE_FP8, 192>(g1, st, K_GEMM_LR1))); break;
+    case 256: MOE_TRY((launch_tc<MODE_SCALE_FP8, 256>(g1, st, K_GEMM_LR1))); break;
+    default: return MOE_ERR_UNSUPPORTED;
+  }
   GroupedGemm g2 = g;
   g2.E = E; g2.A_r = zq; g2.lda_r = r; g2.B0_r = w->lr_U8; g2.N_r = d; g2.K_r = r;
   g2.out_r = y_perm; g2.ldo_r = d; g2.row_scale = sz; g2.col_scale = w->lr_U_scale;
@@ -902,10 +922,7 @@ moe_status_t moe_layer_forward(const moe_config_t *cfg, const void *x, const moe
   int32_t *cb = at<int32_t>(ws, L.chunk_base);
   uint8_t *lr = at<uint8_t>(ws, L.lrank);
   const bool f8 = fp8_experts(cfg);
-  uint8_t *xq = at<uint8_t>(ws, L.xq);
-  float *sx = at<float>(ws, L.sx), *sxp = at<float>(ws, L.sx_perm);
-  // fp8 storage: every token row quantised once, before the routing (it needs x alone)
-  if (f8) MOE_TRY(launch_quantize<__nv_bfloat16>(x, cfg->T, cfg->d, xq, sx, st));
+  float *sxp = at<float>(ws, L.sx_perm);
   if (cfg->dtype == MOE_DTYPE_BF16)
     MOE_TRY(router_only<__nv_bfloat16>(cfg, x, w, idx, wts, pc, pp, lr, st));
   else
@@ -916,9 +933,9 @@ moe_status_t moe_layer_forward(const moe_config_t *cfg, const void *x, const moe
   sa.chunk_base = cb;
   sa.kept = at<int32_t>(ws, L.kept);
   MOE_TRY(launch_stats(sa, st));
-  if (f8)
-    MOE_TRY(scatter_impl<uint8_t>(cfg, xq, idx, lr, cb, sa.kept, offsets, slot_pos, src, x_perm,
-                                  cnt, prob, aux, st, sx, sxp));
+  if (f8)  // the token rows quantised on their way to the experts' rows
+    MOE_TRY(scatter_q8_impl(cfg, x, idx, lr, cb, sa.kept, offsets, slot_pos, src,
+                            (uint8_t *)x_perm, sxp, cnt, prob, aux, st));
   else if (cfg->dtype == MOE_DTYPE_BF16)
     MOE_TRY(scatter_impl<__nv_bfloat16>(cfg, x, idx, lr, cb, sa.kept, offsets, slot_pos, src,
                                         x_perm, cnt, prob, aux, st));

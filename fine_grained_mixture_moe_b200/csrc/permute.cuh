@@ -16,6 +16,7 @@
 //           x row, read once into registers, stored to its k rows of x_perm.
 #pragma once
 #include "common.cuh"
+#include "fp8.cuh"
 
 namespace moe {
 
@@ -74,8 +75,6 @@ __global__ void __launch_bounds__(256) perm_hist_kernel(const int32_t *__restric
 // memory; block 0 writes offsets[0..E] and, when `aux` is set, the load-balancing loss
 // alpha E sum_e (count_e / (T k)) (prob_e / T) (Quartz: weight 0.01), in the order of
 // aux_loss_kernel, so that the fused layer and the separate call agree bit for bit.
-// Rows of E4M3 codes (Tin = uint8_t) travel with their scales: rs_out[row] = rs_in[token] when
-// rs_out is set.
 // Before griddep_wait: this kernel always follows the statistics kernel, whose CTAs allow it to
 // start only after their own griddep_wait, i.e. once the kernel before the statistics (the
 // router or the histogram) has completed and flushed. So x, the routing and the within-chunk
@@ -87,7 +86,7 @@ __global__ void __launch_bounds__(PM_THREADS, PM_CTAS_PER_SM) perm_scatter_kerne
     int32_t *__restrict__ offsets, int32_t *__restrict__ slot_pos, int32_t *__restrict__ src,
     const Tin *__restrict__ x, Tin *__restrict__ x_perm, int d,
     const int32_t *__restrict__ count, const float *__restrict__ prob, float alpha,
-    float *__restrict__ aux, const float *__restrict__ rs_in, float *__restrict__ rs_out) {
+    float *__restrict__ aux) {
   extern __shared__ int s_off[];  // [E] expert offsets
   __shared__ int s_scan[PM_THREADS / 32 + 1];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -147,7 +146,6 @@ __global__ void __launch_bounds__(PM_THREADS, PM_CTAS_PER_SM) perm_scatter_kerne
         if (C < 0 || rank < C) pos = s_off[e] + rank;
         slot_pos[(size_t)t * k + lane] = pos;
         if (pos >= 0) src[pos] = t;
-        if (pos >= 0 && rs_out != nullptr) rs_out[pos] = __ldcg(rs_in + t);
       } else {
         slot_pos[(size_t)t * k + lane] = -1;
         set_device_error(MOE_ERR_DEVICE_CHECK, 100 + lane);
@@ -179,6 +177,125 @@ __global__ void __launch_bounds__(PM_THREADS, PM_CTAS_PER_SM) perm_scatter_kerne
             if (v < nvec) pv[(size_t)pj * nvec + v] = row[i];
           }
         }
+      }
+    }
+    if (t + nwarps < T) load_token(t + nwarps);
+  }
+}
+
+// The same scatter for a layer whose experts take E4M3 rows: each bf16 token row is quantised
+// on its way (per-row scale amax / 448, codes as quantize_rows_kernel makes them, bit for bit)
+// and its codes and scale are stored to every kept pair's row: xq_perm [rows, d] bytes,
+// sx_perm [rows]. The row is held in registers between its maximum and its conversion, so d is
+// at most 32 * PM_VEC * 8 elements (moe_config checks).
+__global__ void __launch_bounds__(PM_THREADS, PM_CTAS_PER_SM) perm_scatter_q8_kernel(
+    const int32_t *__restrict__ idx, const uint8_t *__restrict__ lrank, int T, int k, int E,
+    int C, const int32_t *__restrict__ chunk_base, const int32_t *__restrict__ kept,
+    int32_t *__restrict__ offsets, int32_t *__restrict__ slot_pos, int32_t *__restrict__ src,
+    const __nv_bfloat16 *__restrict__ x, uint8_t *__restrict__ xq_perm,
+    float *__restrict__ sx_perm, int d, const int32_t *__restrict__ count,
+    const float *__restrict__ prob, float alpha, float *__restrict__ aux) {
+  extern __shared__ int s_off[];  // [E] expert offsets
+  __shared__ int s_scan[PM_THREADS / 32 + 1];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int nwarps = gridDim.x * (PM_THREADS / 32);
+  const int gw = blockIdx.x * (PM_THREADS / 32) + warp;
+  const int nvec = d >> 3;  // 16-byte vectors (8 bf16) per row
+  const uint4 *xv = (const uint4 *)x;
+  uint2 *qv = (uint2 *)xq_perm;  // 8 codes per input vector
+
+  uint4 row[PM_VEC];
+  int e_l = -1, r_l = 0;
+  int t = gw;
+  auto load_token = [&](int tt) {
+    if (lane < k) {
+      e_l = __ldcg(idx + (size_t)tt * k + lane);
+      r_l = (int)__ldcg(lrank + (size_t)tt * k + lane);
+    }
+#pragma unroll
+    for (int i = 0; i < PM_VEC; ++i) {
+      const int v = lane + 32 * i;
+      if (v < nvec) row[i] = __ldcs(xv + (size_t)tt * nvec + v);
+    }
+  };
+  const KernelStamp stamp(K_PERM_SCATTER);
+  if (t < T) load_token(t);
+  griddep_wait();
+  stamp.started();
+  griddep_launch();
+  for (int e = tid; e < E; e += PM_THREADS) s_off[e] = kept[e];
+  __syncthreads();
+  const int n_kept = block_excl_scan_inplace(s_off, E, s_scan);
+  if (blockIdx.x == 0) {
+    for (int e = tid; e < E; e += PM_THREADS) offsets[e] = s_off[e];
+    if (tid == 0) offsets[E] = n_kept;
+    if (aux != nullptr && warp == 0) {
+      double sd = 0.0;
+      for (int e = lane; e < E; e += 32) sd += (double)count[e] * (double)prob[e];
+      sd = warp_sum_d(sd);
+      if (lane == 0) {
+        double L = 0.0;
+        if (T > 0) L = (double)alpha * (double)E * sd / ((double)T * (double)k * (double)T);
+        *aux = (float)L;
+      }
+    }
+  }
+  for (; t < T; t += nwarps) {
+    // the row's scale
+    float amax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < PM_VEC; ++i) {
+      if (lane + 32 * i < nvec) {
+        const __nv_bfloat162 *h = (const __nv_bfloat162 *)&row[i];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const float2 f = __bfloat1622float2(h[j]);
+          amax = fmaxf(amax, fmaxf(fabsf(f.x), fabsf(f.y)));
+        }
+      }
+    }
+    amax = warp_max_f(amax);
+    const float sc = amax > 0.0f ? __fdiv_rn(amax, E4M3_MAX) : 1.0f;
+    // the pair's row, as in perm_scatter_kernel
+    int pos = -1;
+    if (lane < k) {
+      const int e = e_l;
+      if (e >= 0 && e < E) {
+        const int rank = __ldcg(chunk_base + (size_t)(t / PM_CHUNK) * E + e) + r_l;
+        if (C < 0 || rank < C) pos = s_off[e] + rank;
+        slot_pos[(size_t)t * k + lane] = pos;
+        if (pos >= 0) {
+          src[pos] = t;
+          sx_perm[pos] = sc;
+        }
+      } else {
+        slot_pos[(size_t)t * k + lane] = -1;
+        set_device_error(MOE_ERR_DEVICE_CHECK, 100 + lane);
+      }
+    }
+    // the codes of vector i replace its first 8 bytes in place (vectors past the row hold no
+    // data: no division runs on them)
+#pragma unroll
+    for (int i = 0; i < PM_VEC; ++i) {
+      if (lane + 32 * i >= nvec) continue;
+      const __nv_bfloat162 *h = (const __nv_bfloat162 *)&row[i];
+      uint32_t w[2];
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        const float2 a = __bfloat1622float2(h[2 * j]), b = __bfloat1622float2(h[2 * j + 1]);
+        w[j] = e4m3_code(__fdiv_rn(a.x, sc)) | (e4m3_code(__fdiv_rn(a.y, sc)) << 8) |
+               (e4m3_code(__fdiv_rn(b.x, sc)) << 16) | (e4m3_code(__fdiv_rn(b.y, sc)) << 24);
+      }
+      row[i].x = w[0];
+      row[i].y = w[1];
+    }
+    for (int j = 0; j < k; ++j) {
+      const int pj = __shfl_sync(0xffffffffu, pos, j);
+      if (pj < 0) continue;
+#pragma unroll
+      for (int i = 0; i < PM_VEC; ++i) {
+        const int v = lane + 32 * i;
+        if (v < nvec) qv[(size_t)pj * nvec + v] = make_uint2(row[i].x, row[i].y);
       }
     }
     if (t + nwarps < T) load_token(t + nwarps);

@@ -43,12 +43,31 @@ def upload_weights(cfg: B.MoEConfig, host: Dict[str, object], device) -> Dict[st
     return out
 
 
+def quantize_lowrank_weights(cfg: B.MoEConfig, weights: Dict[str, torch.Tensor],
+                             stream=None) -> Dict[str, torch.Tensor]:
+    """The E4M3 rows and fp32 row scales of the low-rank experts' V [E, r, d] and U [E, d, r]
+    (moe_quantize_fp8 on the device), added to a copy of `weights` under the names of
+    moe_weights_t's fp8 fields."""
+    E, r, d = cfg.E, cfg.rank, cfg.d
+    out = dict(weights)
+    for name, rows, cols in (("lr_V", E * r, d), ("lr_U", E * d, r)):
+        src = weights[name]
+        q = torch.empty((rows, cols), dtype=torch.uint8, device=src.device)
+        sc = torch.empty(rows, dtype=torch.float32, device=src.device)
+        B.moe_quantize_fp8(src, rows, cols, q, sc, stream)
+        out[name + "8"] = q
+        out[name + "_scale"] = sc
+    return out
+
+
 class MoELayer:
     """Owns the device weights and the workspace of one MoE FFN layer configuration."""
 
     def __init__(self, cfg: B.MoEConfig, weights: Dict[str, torch.Tensor], device=None):
         self.cfg = cfg
         self.device = torch.device(device if device is not None else "cuda")
+        if cfg.expert_storage == B.STORAGE["fp8"] and "lr_V8" not in weights:
+            weights = quantize_lowrank_weights(cfg, weights)
         self.weights = weights
         self.wstruct = B.make_weights(weights)
         self.ws_bytes = B.moe_workspace_size(cfg)
