@@ -1,5 +1,5 @@
-"""B200-native forward pass of a DeepSeek-style fine-grained mixture-of-experts FFN layer, and
-the first steps of its backward pass (the combine and the router).
+"""B200-native forward and backward passes of a DeepSeek-style fine-grained mixture-of-experts
+FFN layer, with an fp8 (E4M3) storage of the low-rank experts.
 
 The compute path is the sm_100a CUDA library ``lib/libmoe.so`` behind the C ABI in
 ``include/moe.h``; :mod:`.binding` marshals arguments to it and :class:`MoELayer` holds device
@@ -12,6 +12,7 @@ from .binding import (DEBUG_FORCE_EXACT, DEBUG_PROFILE, DEBUG_WAIT_LIMIT_NS, EXP
                       moe_combine_backward, moe_debug_set, moe_route_backward,
                       moe_expert_backward, moe_backward_workspace_size, make_grads,
                       moe_debug_wait_timeout_probe, moe_expert_forward, moe_get_device_error,
-                      moe_layer_forward, moe_permute, moe_profile_read, moe_route,
-                      moe_route_noalloc, moe_workspace_size, status_str)
-from .layer import MoELayer, torch_dtype, upload_weights, y_perm_dtype  # noqa: F401
+                      moe_layer_forward, moe_permute, moe_profile_read, moe_quantize_fp8,
+                      moe_route, moe_route_noalloc, moe_workspace_size, status_str)
+from .layer import (MoELayer, quantize_lowrank_weights, torch_dtype, upload_weights,  # noqa: F401
+                    y_perm_dtype)

@@ -312,6 +312,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TC_THREADS, 1)
       if (MODE == MODE_SWIGLU_BWD && cstop > cbeg)
         feed.issue(gu_pair_block(p, ti, routed, routed ? p.aux_r : p.aux_s, rbase, ti.n0 + cbeg),
                    lane);
+      // PLAIN_FP8: the row's scale, read before the accumulator is ready
+      const float rs8 = (MODE == MODE_PLAIN_FP8 && routed && row_ok)
+                            ? __ldg(p.row_scale + ti.a_row0 + row) : 0.0f;
       bool ok = true;
       if (lane == 0)
         ok = mbar_wait(accf_bar(acc), acc_phase, abort_flag, limit, INFO_WAIT_ACC_FULL);
@@ -422,20 +425,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TC_THREADS, 1)
           __syncwarp();
         } else {
           // fp32 output, staged per warp and written as 128-byte rows
+          float4 cs8[8];  // PLAIN_FP8: the U rows' scales of columns col .. col + 31
+          if (MODE == MODE_PLAIN_FP8 && routed) {
+            const float4 *cs = (const float4 *)(p.col_scale + (size_t)ti.g * ti.N + ti.n0 + c);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) cs8[i] = __ldg(cs + i);
+          }
           uint32_t r0[32];
           tmem_ld32(tbase + c, r0);
           tmem_wait_ld();
-          if (MODE == MODE_PLAIN_FP8 && routed && row_ok && ti.n0 + c < ti.N) {
-            // y = sum * (row scale) * (U row scale), columns col .. col + 31
-            const float4 *cs = (const float4 *)(p.col_scale + (size_t)ti.g * ti.N + ti.n0 + c);
-            const float rs = __ldg(p.row_scale + ti.a_row0 + row);
+          if (MODE == MODE_PLAIN_FP8 && routed) {
+            // y = sum * (row scale) * (U row scale)
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
-              const float4 v = __ldg(cs + i);
-              r0[4 * i] = __float_as_uint(__uint_as_float(r0[4 * i]) * rs * v.x);
-              r0[4 * i + 1] = __float_as_uint(__uint_as_float(r0[4 * i + 1]) * rs * v.y);
-              r0[4 * i + 2] = __float_as_uint(__uint_as_float(r0[4 * i + 2]) * rs * v.z);
-              r0[4 * i + 3] = __float_as_uint(__uint_as_float(r0[4 * i + 3]) * rs * v.w);
+              r0[4 * i] = __float_as_uint(__uint_as_float(r0[4 * i]) * rs8 * cs8[i].x);
+              r0[4 * i + 1] = __float_as_uint(__uint_as_float(r0[4 * i + 1]) * rs8 * cs8[i].y);
+              r0[4 * i + 2] = __float_as_uint(__uint_as_float(r0[4 * i + 2]) * rs8 * cs8[i].z);
+              r0[4 * i + 3] = __float_as_uint(__uint_as_float(r0[4 * i + 3]) * rs8 * cs8[i].w);
             }
           }
 #pragma unroll

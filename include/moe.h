@@ -1,5 +1,5 @@
 /*
- * moe.h - C ABI of the B200 fine-grained mixture-of-experts FFN layer (forward pass).
+ * moe.h - C ABI of the B200 fine-grained mixture-of-experts FFN layer (forward and backward).
  *
  * The layer is the DeepSeek-style fine-grained MoE FFN that the source pages describe:
  *   - Vertex AGI research page / quartz-micro-preview-base model card, "Architecture":
