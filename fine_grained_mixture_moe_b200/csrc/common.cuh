@@ -44,7 +44,7 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
 // Kinds of the library's forward kernels (the host's profiler and the device stamps share them).
 enum KernelKind {
   K_ROUTER, K_STATS, K_PERM_HIST, K_PERM_SCATTER, K_GEMM_GATEUP, K_GEMM_DOWN, K_GEMM_LR1,
-  K_GEMM_LR2, K_COMBINE, K_AUX, K_BWD_GEMM, K_QUANT, K_COUNT
+  K_GEMM_LR2, K_COMBINE, K_AUX, K_BWD_GEMM, K_QUANT, K_SPLIT, K_COUNT
 };
 
 // In-step timestamps. With stamping on (moe_debug_set(MOE_DEBUG_STAMP, 1)) a kernel records, per

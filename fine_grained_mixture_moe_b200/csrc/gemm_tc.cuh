@@ -48,11 +48,11 @@ template <int MODE, int BN> struct TcCfg {
   static constexpr int A_BYTES = TC_BM * 128;                     // 16 KB: 128-byte rows
   static constexpr int B_BYTES = BN * 128;
   static constexpr int STAGE_BYTES = A_BYTES + NB * B_BYTES;
+  // PLAIN and SCALE: per-warp fp32 staging (SCALE stores fp32 z with out_f32); SCALE_FP8: the
+  // row maxima of the two column halves, per accumulator buffer [2][2][128]
   static constexpr bool F32_OUT = MODE == MODE_PLAIN;
-  // PLAIN: per-warp fp32 staging; SCALE_FP8: the row maxima of the two column halves, per
-  // accumulator buffer [2][2][128]
-  static constexpr int STG_BYTES = F32_OUT ? TC_EPI_WARPS * 4096
-                                           : MODE == MODE_SCALE_FP8 ? 2 * 2 * TC_BM * 4 : 0;
+  static constexpr int STG_BYTES = MODE == MODE_PLAIN || MODE == MODE_SCALE ? TC_EPI_WARPS * 4096
+                                   : MODE == MODE_SCALE_FP8 ? 2 * 2 * TC_BM * 4 : 0;
   static constexpr int STAGES = (200 * 1024 - STG_BYTES) / STAGE_BYTES > 8
                                     ? 8 : (200 * 1024 - STG_BYTES) / STAGE_BYTES;
   static constexpr int ACC_COLS = NB * BN;                        // fp32 columns per buffer
@@ -391,6 +391,41 @@ __global__ void __launch_bounds__(TC_THREADS, 1) gemm_tc_kernel(const __grid_con
       constexpr int SUB = C::F32_OUT ? 1 : 2;  // 32-column TMEM loads per block
 #pragma unroll 1
       for (int c = cbeg; c < (MODE == MODE_SCALE_FP8 ? cbeg : cend); c += 32 * SUB) {
+        if (MODE == MODE_SCALE && p.out_f32) {
+          // fp32 z = sum * s, SUB 32-column blocks, each staged per warp and written as 32
+          // coalesced 128-byte row stores
+#pragma unroll 1
+          for (int sub = 0; sub < SUB && c + 32 * sub < cend; ++sub) {  // this warp's columns only
+            uint32_t r0[32];
+            tmem_ld32(tbase + c + 32 * sub, r0);
+            tmem_wait_ld();
+            const int col = ti.n0 + c + 32 * sub;
+            if (col < ti.N) {
+              const float *sc = p.scale + (size_t)ti.g * ti.N + col;
+#pragma unroll
+              for (int i = 0; i < 32; ++i)
+                r0[i] = __float_as_uint(__uint_as_float(r0[i]) * __ldg(sc + i));
+            }
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              *(uint4 *)(stg + lane * 128 + ((i ^ (lane & 7)) << 4)) =
+                  make_uint4(r0[4 * i], r0[4 * i + 1], r0[4 * i + 2], r0[4 * i + 3]);
+            __syncwarp();
+            if (col < ti.N) {
+              const int rbase = ti.m0 + q * 32;
+              const int nrows = min(32, ti.rows - rbase);
+              unsigned char *obase = (unsigned char *)out + ((size_t)(ti.a_row0 + rbase) * ldo + col) * 4;
+              const size_t row_bytes = (size_t)ldo * 4;
+              for (int rr = 0; rr < nrows; ++rr) {
+                const uint32_t v = *(const uint32_t *)(stg + rr * 128 +
+                                                       (((lane >> 2) ^ (rr & 7)) << 4) + ((lane & 3) << 2));
+                *(uint32_t *)(obase + rr * row_bytes + lane * 4) = v;
+              }
+            }
+            __syncwarp();
+          }
+          continue;
+        }
         if (MODE == MODE_SCALE) {
           // bf16 low-rank projection: each lane already writes 64 contiguous bytes of its row, so
           // they go out directly

@@ -72,12 +72,12 @@ __device__ __forceinline__ void mbar_arrive_cta0(uint32_t bar_local) {
 
 // Modes whose B tile is two weights (gate rows in CTA 0, up rows in CTA 1).
 __host__ __device__ constexpr bool tc2_two_b(int mode) {
-  return mode == MODE_GATEUP || mode == MODE_GATEUP_RAW;
+  return mode == MODE_GATEUP || mode == MODE_GATEUP_RAW || mode == MODE_GATEUP_F32;
 }
 
 template <int MODE> struct Tc2Cfg {
   static_assert(MODE == MODE_GATEUP || MODE == MODE_PLAIN || MODE == MODE_GATEUP_RAW ||
-                    MODE == MODE_SWIGLU_BWD || MODE == MODE_PLAIN_FP8,
+                    MODE == MODE_SWIGLU_BWD || MODE == MODE_PLAIN_FP8 || MODE == MODE_GATEUP_F32,
                 "pair kernel modes");
   static constexpr int BN = tc2_two_b(MODE) ? 128 : 256;  // output columns per tile
   static constexpr int MMA_N = 256;                           // accumulator columns
@@ -351,6 +351,35 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TC_THREADS, 1)
               feed.issue(gu_pair_block(p, ti, routed, routed ? p.aux_r : p.aux_s, rbase, col + 32),
                          lane);
           });
+          continue;
+        }
+        if (MODE == MODE_GATEUP_F32) {
+          // silu(gate) * up in fp32 (IEEE exp and division), 32 columns (128 bytes of each row)
+          // at a time, staged per warp and written as 32 coalesced 128-byte row stores
+          uint32_t r0[32], r1[32];
+          tmem_ld32(tbase + c, r0);
+          tmem_ld32(tbase + BN + c, r1);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const float g = __uint_as_float(r0[i]);
+            r0[i] = __float_as_uint(g / (1.0f + expf(-g)) * __uint_as_float(r1[i]));
+          }
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            *(uint4 *)(stg + lane * 128 + ((i ^ (lane & 7)) << 4)) =
+                make_uint4(r0[4 * i], r0[4 * i + 1], r0[4 * i + 2], r0[4 * i + 3]);
+          __syncwarp();
+          const int col = ti.n0 + c;
+          const int nrows = min(32, ti.rows - rbase);
+          unsigned char *obase = (unsigned char *)out + ((size_t)(ti.out_row0 + rbase) * ldo + col) * 4;
+          const size_t row_bytes = (size_t)ldo * 4;
+          for (int rr = 0; rr < nrows; ++rr) {
+            const uint32_t v = *(const uint32_t *)(stg + rr * 128 +
+                                                   (((lane >> 2) ^ (rr & 7)) << 4) + ((lane & 3) << 2));
+            *(uint32_t *)(obase + rr * row_bytes + lane * 4) = v;
+          }
+          __syncwarp();
           continue;
         }
         if (MODE == MODE_GATEUP) {

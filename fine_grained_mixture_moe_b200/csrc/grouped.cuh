@@ -8,7 +8,8 @@
 //                        B*_s is at ((kk / piece_k) * piece_rows + n) * piece_k + kk % piece_k.
 //                        This reads the shared down projections [S, d, fs] as one [d, S*fs]
 //                        matrix, so S shared experts of width fs act as one of width S*fs.
-// Epilogue modes: GATEUP out = silu(A B0^T) * (A B1^T) (SwiGLU, gate and up fused);
+// Epilogue modes: GATEUP out = silu(A B0^T) * (A B1^T) (SwiGLU, gate and up fused; GATEUP_F32
+//                   the same stored as fp32);
 //                 PLAIN  out = A B0^T;   SCALE out = (A B0^T) * scale[g][n] (low-rank s);
 //                 GATEUP_RAW (backward) g = A B0^T and u = A B1^T (fp32) to out, in the
 //                   blocked g, u layout of backward_epilogue.cuh (half = the width of g);
@@ -29,17 +30,16 @@
 // A[M, K_g] B[N, K_g]^T, where A and B are K-major [M or N][ld] and group g takes their columns
 // kseg koff[g] .. kseg koff[g+1] (koff padded to multiples of 64; kseg segments per group, so a
 // sum of split terms runs as one product); M is rows_r and ld is K_r.
-// Output types in the tensor-core (bf16) kernels: GATEUP and SCALE write bf16 (the next
-// product's operand, SCALE optionally as a hi + lo pair); PLAIN writes the routed groups' rows in
-// bf16 or fp32 (out_r_bf16) and the shared group's rows in fp32. The SIMT (fp32) kernels write
-// fp32 throughout.
+// Output types in the tensor-core kernels: GATEUP and SCALE write bf16 (the next product's
+// operand, SCALE optionally as a hi + lo pair) or, with out_f32, fp32; PLAIN writes the routed
+// groups' rows in bf16 or fp32 (out_r_bf16) and the shared group's rows in fp32.
 #pragma once
 #include "common.cuh"
 
 namespace moe {
 
 enum GemmMode { MODE_GATEUP = 0, MODE_PLAIN = 1, MODE_SCALE = 2, MODE_GATEUP_RAW = 3,
-                MODE_SWIGLU_BWD = 4, MODE_SCALE_FP8 = 5, MODE_PLAIN_FP8 = 6 };
+                MODE_SWIGLU_BWD = 4, MODE_SCALE_FP8 = 5, MODE_PLAIN_FP8 = 6, MODE_GATEUP_F32 = 7 };
 
 // Modes whose operands are E4M3 bytes (tcgen05 kind::f8f6f4) rather than bf16 (kind::f16).
 __host__ __device__ constexpr bool mode_fp8(int mode) {
@@ -66,6 +66,8 @@ struct GroupedGemm {
   int lo_split;        // MODE_SCALE, bf16: > 0 stores v as hi = bf16(v) at column n and
                        // lo = bf16(v - hi) at column n + lo_split (a two-term bf16 split)
   int out_r_bf16;      // MODE_PLAIN, tensor-core kernels: routed rows stored as bf16 (else fp32)
+  int out_f32;         // MODE_SCALE (single SM): z stored as fp32 (the fp32 configuration, whose
+                       // operands are split bf16 terms; its gate/up is MODE_GATEUP_F32)
   int has_shared, T;
   const void *A_s;
   int lda_s;

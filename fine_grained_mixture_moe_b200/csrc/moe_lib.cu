@@ -14,8 +14,8 @@
 #include "backward.cuh"
 #include "combine.cuh"
 #include "common.cuh"
+#include "f32split.cuh"
 #include "fp8.cuh"
-#include "gemm_simt.cuh"
 #include "gemm_tc.cuh"
 #include "gemm_tc2.cuh"
 #include "permute.cuh"
@@ -111,6 +111,9 @@ struct Layout {
   size_t hidden, hidden_sh;                                     // experts
   size_t idx, wts, count, prob, offsets, slot_pos, src, x_perm, y_perm, y_shared, aux;  // layer
   size_t sx_perm, zq, sz;  // fp8 storage: scales of the E4M3 token rows, z rows and scales
+  // fp32 layers: operands as six bf16 K segments (f32split.cuh): token rows, hidden rows, the
+  // routed weights of both products, and the shared experts' counterparts
+  size_t s6_x, s6_h, s6_w1, s6_w1b, s6_w2, s6_xs, s6_hs, s6_sg, s6_su, s6_sd;
   size_t total;
 };
 inline bool fp8_experts(const moe_config_t *c) { return c->expert_storage == MOE_STORAGE_FP8_E4M3; }
@@ -150,6 +153,19 @@ Layout layout_of(const moe_config_t *c) {
   L.sx_perm = take(f8 ? T * k * 4 : 0);
   L.zq = take(f8 ? T * k * (size_t)c->rank : 0);
   L.sz = take(f8 ? T * k * 4 : 0);
+  const bool f32 = c->dtype == MOE_DTYPE_F32;
+  const size_t hw = c->expert == MOE_EXPERT_SWIGLU ? (size_t)c->ffn : (size_t)c->rank;
+  const size_t sfs = (size_t)c->n_shared * c->ffn_shared;
+  L.s6_x = take(f32 ? T * k * 6 * d * 2 : 0);
+  L.s6_h = take(f32 ? T * k * 6 * hw * 2 : 0);
+  L.s6_w1 = take(f32 ? E * hw * 6 * d * 2 : 0);
+  L.s6_w1b = take(f32 && c->expert == MOE_EXPERT_SWIGLU ? E * hw * 6 * d * 2 : 0);
+  L.s6_w2 = take(f32 ? E * d * 6 * hw * 2 : 0);
+  L.s6_xs = take(f32 ? T * 6 * d * 2 * (sfs > 0) : 0);
+  L.s6_hs = take(f32 ? T * 6 * sfs * 2 : 0);
+  L.s6_sg = take(f32 ? sfs * 6 * d * 2 : 0);
+  L.s6_su = take(f32 ? sfs * 6 * d * 2 : 0);
+  L.s6_sd = take(f32 ? d * 6 * sfs * 2 : 0);
   L.total = o;
   return L;
 }
@@ -182,7 +198,8 @@ int num_sms() {
 // ------------------------------------------------------------------ profiling (debug)
 const char *kKindName[K_COUNT] = {"router", "stats", "perm_hist", "perm_scatter", "gemm_gateup",
                                   "gemm_down", "gemm_lowrank_v", "gemm_lowrank_u", "combine",
-                                  "aux_loss", "backward_gemm", "quantize_fp8"};
+                                  "aux_loss", "backward_gemm", "quantize_fp8",
+                                  "split_f32"};
 constexpr int PROF_SLOTS = 8192;
 struct Prof {
   bool on = false;
@@ -356,30 +373,12 @@ moe_status_t launch_tc2(const GroupedGemm &g, cudaStream_t st, int kind) {
   return launch_pdl(kern, dim3(2 * pairs), dim3(TC_THREADS), smem, st, P);
 }
 
-template <int MODE>
-moe_status_t launch_simt(const GroupedGemm &g, cudaStream_t st, int kind) {
-  const int G = g.E + g.has_shared;
-  const size_t smem = (size_t)(G + 1 + 256 / 32 + 1) * sizeof(int);
-  auto kern = gemm_simt_kernel<float, float, MODE>;
-  if (smem > 48 * 1024 &&
-      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-    return MOE_ERR_CUDA;
-  const long long bound = tile_bound(g, SM_BM, SM_BN);
-  if (bound == 0) return MOE_OK;
-  const int grid = (int)std::min<long long>((long long)num_sms() * 8, bound);
-  GroupedGemm gk = g;
-  gk.kind = kind;
-  ProfScope ps(kind, st);
-  return launch_pdl(kern, dim3(grid), dim3(256), smem, st, gk);
-}
-
-// bf16: gate/up and plain products on CTA pairs (256 x 256 tiles; an output width that is not a
+// gate/up and plain products on CTA pairs (256 x 256 tiles; an output width that is not a
 // multiple of 256 leaves the last column tile partly outside the expert, whose columns the
 // epilogue does not store), the low-rank projection on single SMs (N = rank).
 template <int MODE>
 moe_status_t launch_gemm(const moe_config_t *c, const GroupedGemm &g, cudaStream_t st,
                          int kind) {
-  if (c->dtype == MOE_DTYPE_F32) return launch_simt<MODE>(g, st, kind);
   if (MODE == MODE_SCALE) return launch_tc<MODE_SCALE, 64>(g, st, kind);
   return launch_tc2<MODE == MODE_GATEUP ? MODE_GATEUP : MODE_PLAIN>(g, st, kind);
 }
@@ -586,10 +585,99 @@ moe_status_t experts_fp8_impl(const moe_config_t *c, const uint8_t *xq_perm, con
   return MOE_OK;
 }
 
+// fp32 operands as six bf16 K segments (f32split.cuh): rows x cols in, [rows, 6 cols] out.
+moe_status_t launch_split6(const void *in, long long rows, int cols, int piece, bool b_operand,
+                           void *out, cudaStream_t st) {
+  const long long n = rows * cols;
+  if (n == 0) return MOE_OK;
+  const int grid = (int)std::min<long long>((n + 255) / 256, (long long)num_sms() * 16);
+  ProfScope ps(K_SPLIT, st);
+  return launch_pdl(split6_bf16_kernel, dim3(grid), dim3(256), 0, st, (const float *)in, rows,
+                    cols, piece, b_operand ? 1 : 0, (__nv_bfloat16 *)out);
+}
+
+// The fp32 configuration on the tensor cores: every product's operands split into six bf16 K
+// segments (x_perm and x, the hidden rows, the weights, each call), the products run over
+// K' = 6 K on the bf16 kernels with fp32 hidden rows (gate/up) or z (low-rank) and fp32 outputs.
+moe_status_t experts_f32_impl(const moe_config_t *c, const void *x_perm, const int32_t *offsets,
+                              const void *x, const moe_weights_t *w, void *y_perm,
+                              void *y_shared, void *ws, cudaStream_t st) {
+  const Layout L = layout_of(c);
+  const int T = c->T, d = c->d, E = c->E, k = c->top_k, S = c->n_shared, fs = c->ffn_shared;
+  const int sf = S * fs;
+  const bool swi = c->expert == MOE_EXPERT_SWIGLU, sh = S > 0;
+  const int hw = swi ? c->ffn : c->rank;  // hidden width: ffn or rank
+  void *H = at<char>(ws, L.hidden), *Hs = at<char>(ws, L.hidden_sh);
+  void *x6 = at<char>(ws, L.s6_x), *h6 = at<char>(ws, L.s6_h), *w1 = at<char>(ws, L.s6_w1),
+       *w1b = at<char>(ws, L.s6_w1b), *w2 = at<char>(ws, L.s6_w2), *xs6 = at<char>(ws, L.s6_xs),
+       *hs6 = at<char>(ws, L.s6_hs), *sg6 = at<char>(ws, L.s6_sg), *su6 = at<char>(ws, L.s6_su),
+       *sd6 = at<char>(ws, L.s6_sd);
+  const long long N = (long long)T * k;
+  MOE_TRY(launch_split6(x_perm, N, d, d, false, x6, st));
+  if (swi) {
+    MOE_TRY(launch_split6(w->w_gate, (long long)E * hw, d, d, true, w1, st));
+    MOE_TRY(launch_split6(w->w_up, (long long)E * hw, d, d, true, w1b, st));
+    MOE_TRY(launch_split6(w->w_down, (long long)E * d, hw, hw, true, w2, st));
+  } else {
+    MOE_TRY(launch_split6(w->lr_V, (long long)E * hw, d, d, true, w1, st));
+    MOE_TRY(launch_split6(w->lr_U, (long long)E * d, hw, hw, true, w2, st));
+  }
+  if (sh) {
+    MOE_TRY(launch_split6(x, T, d, d, false, xs6, st));
+    MOE_TRY(launch_split6(w->ws_gate, sf, d, d, true, sg6, st));
+    MOE_TRY(launch_split6(w->ws_up, sf, d, d, true, su6, st));
+    MOE_TRY(launch_split6(w->ws_down, (long long)S * d, fs, fs, true, sd6, st));
+  }
+  GroupedGemm g;
+  std::memset(&g, 0, sizeof(g));
+  g.offsets = offsets;
+  g.T = T;
+  g.rows_r = T * k;
+  // first products: gate/up (h fp32) with the shared experts' in the same launch, or z = x V^T s
+  GroupedGemm g1 = g;
+  g1.E = E; g1.A_r = x6; g1.lda_r = 6 * d; g1.K_r = 6 * d; g1.B0_r = w1; g1.N_r = hw;
+  g1.out_r = H; g1.ldo_r = hw;
+  if (swi) {
+    g1.B1_r = w1b;
+    g1.has_shared = sh;
+    if (sh) {
+      g1.A_s = xs6; g1.lda_s = 6 * d; g1.B0_s = sg6; g1.B1_s = su6; g1.N_s = sf; g1.K_s = 6 * d;
+      g1.piece_k = 6 * d; g1.piece_rows = 0; g1.b_rows_s = sf; g1.out_s = Hs; g1.ldo_s = sf;
+    }
+    MOE_TRY(launch_tc2<MODE_GATEUP_F32>(g1, st, K_GEMM_GATEUP));
+  } else {
+    g1.scale = w->lr_s;
+    g1.out_f32 = 1;
+    MOE_TRY((launch_tc<MODE_SCALE, 64>(g1, st, K_GEMM_LR1)));
+    if (sh) {  // the shared experts' gate/up alone
+      GroupedGemm g3 = g;
+      g3.E = 0; g3.has_shared = 1;
+      g3.A_s = xs6; g3.lda_s = 6 * d; g3.B0_s = sg6; g3.B1_s = su6; g3.N_s = sf; g3.K_s = 6 * d;
+      g3.piece_k = 6 * d; g3.piece_rows = 0; g3.b_rows_s = sf; g3.out_s = Hs; g3.ldo_s = sf;
+      MOE_TRY(launch_tc2<MODE_GATEUP_F32>(g3, st, K_GEMM_GATEUP));
+    }
+  }
+  // second products: down (or U) over the split hidden rows, the shared down in the same launch
+  MOE_TRY(launch_split6(H, N, hw, hw, false, h6, st));
+  if (sh) MOE_TRY(launch_split6(Hs, T, sf, fs, false, hs6, st));
+  GroupedGemm g2 = g;
+  g2.E = E; g2.A_r = h6; g2.lda_r = 6 * hw; g2.K_r = 6 * hw; g2.B0_r = w2; g2.N_r = d;
+  g2.out_r = y_perm; g2.ldo_r = d; g2.out_r_bf16 = 0;
+  g2.has_shared = sh;
+  if (sh) {
+    g2.A_s = hs6; g2.lda_s = 6 * sf; g2.B0_s = sd6; g2.N_s = d; g2.K_s = 6 * sf;
+    g2.piece_k = 6 * fs; g2.piece_rows = d; g2.b_rows_s = S * d; g2.out_s = y_shared;
+    g2.ldo_s = d;
+  }
+  return launch_tc2<MODE_PLAIN>(g2, st, swi ? K_GEMM_DOWN : K_GEMM_LR2);
+}
+
 moe_status_t experts_impl(const moe_config_t *c, const void *x_perm, const int32_t *offsets,
                           const void *x, const moe_weights_t *w, void *y_perm, void *y_shared,
                           void *ws, cudaStream_t st) {
   if (c->T == 0) return MOE_OK;
+  if (c->dtype == MOE_DTYPE_F32)
+    return experts_f32_impl(c, x_perm, offsets, x, w, y_perm, y_shared, ws, st);
   if (fp8_experts(c)) {  // the bf16 rows quantised first, as the layer quantises its tokens
     const Layout L = layout_of(c);
     uint8_t *xq = at<uint8_t>(ws, L.x_perm);

@@ -27,6 +27,13 @@ CASES = {
     "lr_fp8_r192_shared": MoEConfig(name="lf8b", T=300, d=256, E=16, top_k=2, n_shared=1,
                                     ffn=0, ffn_shared=128, rank=192, expert="lowrank",
                                     offset=("normal", 0.5)),
+    # capacity drops (dropped pairs get no row), rank 256 (the largest tile), top-3
+    "lr_fp8_cap_r256": MoEConfig(name="lf8c", T=700, d=512, E=8, top_k=3, n_shared=0, ffn=0,
+                                 ffn_shared=0, rank=256, expert="lowrank", capacity_factor=0.6,
+                                 offset=("normal", 1.0)),
+    # one token
+    "lr_fp8_T1": MoEConfig(name="lf8d", T=1, d=128, E=4, top_k=2, n_shared=0, ffn=0,
+                           ffn_shared=0, rank=64, expert="lowrank"),
 }
 
 
@@ -102,3 +109,22 @@ def test_fp8_lowrank_layer(name):
     assert torch.equal(y, o["y"])
     print(f"{name}: max|dy|/rms layer {e_layer:.2e} y_perm {e_perm:.2e} steps {e_steps:.2e}")
     assert e_layer <= 2e-2 and e_perm <= 2e-2 and e_steps <= 2e-2
+
+
+def test_fp8_layer_no_tokens():
+    c = CASES["lr_fp8_s"]
+    cfg = B.make_config(T=0, d=c.d, E=c.E, top_k=c.top_k, rank=c.rank, expert="lowrank",
+                        dtype="bf16", expert_storage="fp8")
+    ws_bytes = B.moe_workspace_size(cfg)
+    assert ws_bytes > 0
+    dev = torch.device("cuda:0")
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    w = {n: torch.zeros(16, dtype=torch.uint8, device=dev) for n in
+         ("w_router", "lr_V8", "lr_U8", "lr_V_scale", "lr_U_scale", "lr_s")}
+    y = torch.empty((1, c.d), dtype=torch.float32, device=dev)
+    aux = torch.full((), 5.0, dtype=torch.float32, device=dev)
+    cnt = torch.full((c.E,), 7, dtype=torch.int32, device=dev)
+    B.moe_layer_forward(cfg, torch.empty((1, c.d), dtype=torch.bfloat16, device=dev),
+                        B.make_weights(w), y, aux, cnt, ws, ws_bytes)
+    torch.cuda.synchronize()
+    assert float(aux) == 0.0 and int(cnt.abs().sum()) == 0

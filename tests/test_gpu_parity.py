@@ -54,6 +54,13 @@ EDGE = {
     "f32_sigmoid_cap": MoEConfig(name="f32sc", T=130, d=128, E=8, top_k=3, n_shared=1, ffn=64,
                                  ffn_shared=64, dtype="f32", score="sigmoid", norm_topk=True,
                                  bias=("uniform", 0.1), capacity_factor=0.8),
+    # the fp32 configuration's low-rank path (z kept fp32 between the two split products) with a
+    # shared expert, and a ragged last column tile of gate/up (ffn 192)
+    "lowrank_f32_shared": MoEConfig(name="lrf32", T=210, d=128, E=8, top_k=2, n_shared=1, ffn=0,
+                                    ffn_shared=192, rank=128, expert="lowrank", dtype="f32",
+                                    offset=("normal", 0.5)),
+    "f32_ffn192": MoEConfig(name="f32f192", T=150, d=192, E=5, top_k=2, n_shared=2, ffn=192,
+                            ffn_shared=64, dtype="f32"),
     # the largest top_k, on both sides of the switch from per-pair rank selection (E <= 64) to
     # per-token warp selection
     "k8_E64": MoEConfig(name="k8e64", T=97, d=128, E=64, top_k=8, n_shared=1, ffn=64,
