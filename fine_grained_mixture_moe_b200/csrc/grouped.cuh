@@ -1,4 +1,4 @@
-// Grouped-GEMM problem description shared by the tensor-core (bf16) and SIMT (fp32) kernels.
+// Grouped-GEMM problem description of the tensor-core kernels (gemm_tc.cuh, gemm_tc2.cuh).
 //
 // A launch covers up to E routed groups plus one shared group:
 //   routed group g < E : rows offsets[g]..offsets[g+1] of A_r / out_r, weight B*_r + g*N_r*K_r
