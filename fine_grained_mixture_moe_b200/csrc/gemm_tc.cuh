@@ -38,6 +38,8 @@ struct TcParams {
   TcMaps maps;
   GroupedGemm p;
   int stages;  // CTA-pair kernel: operand pipeline depth chosen from the group count
+  int kpb;     // CTA-pair kernel: K-blocks per stage, 1 or 2 (2: 3-D tensor maps whose box spans
+               // two K-blocks, one A and one B copy per two K-blocks)
 };
 
 template <int MODE, int BN> struct TcCfg {

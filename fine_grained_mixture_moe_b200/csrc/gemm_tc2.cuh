@@ -30,6 +30,16 @@ __device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap
       "l"((uint64_t)map), "r"(c0), "r"(c1), "r"(bar0)
       : "memory");
 }
+// The same with a 3-D box {64 columns, rows, 2 K-blocks}: two K-blocks' tiles, one after the other.
+__device__ __forceinline__ void tma_load_3d_pair(uint32_t dst, const CUtensorMap *map, int c0,
+                                                 int c1, int c2, uint32_t bar_local) {
+  const uint32_t bar0 = bar_local & 0xFEFFFFFFu;
+  asm volatile(
+      "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
+      "l"((uint64_t)map), "r"(c0), "r"(c1), "r"(c2), "r"(bar0)
+      : "memory");
+}
 __device__ __forceinline__ void tc2_mma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
                                         uint32_t idesc, uint32_t accumulate) {
   asm volatile(
@@ -103,15 +113,17 @@ template <int MODE> constexpr size_t tc2_fixed_bytes(int G) {
   return 1024 + (size_t)Tc2Cfg<MODE>::STG_BYTES + 256 +
          (size_t)(G + 1 + TC_THREADS / 32 + 1) * sizeof(int);
 }
-// Operand stages that fit in the 227 KB a CTA may hold (at most MAX_STAGES; < 2 means the tile
-// list of G groups leaves no room for double buffering).
-template <int MODE> constexpr int tc2_stages(int G) {
+// Operand stages of kpb K-blocks that fit in the 227 KB a CTA may hold (at most MAX_STAGES K-blocks
+// in all; < 2 means the tile list of G groups leaves no room for double buffering).
+template <int MODE> constexpr int tc2_stages(int G, int kpb = 1) {
   const long long room = 227LL * 1024 - (long long)tc2_fixed_bytes<MODE>(G);
-  const long long n = room < 0 ? 0 : room / Tc2Cfg<MODE>::STAGE_BYTES;
-  return n > Tc2Cfg<MODE>::MAX_STAGES ? Tc2Cfg<MODE>::MAX_STAGES : (int)n;
+  const long long n = room < 0 ? 0 : room / ((long long)Tc2Cfg<MODE>::STAGE_BYTES * kpb);
+  const int cap = Tc2Cfg<MODE>::MAX_STAGES / kpb;
+  return n > cap ? cap : (int)n;
 }
-template <int MODE> constexpr size_t tc2_smem_bytes(int G) {
-  return tc2_fixed_bytes<MODE>(G) + (size_t)tc2_stages<MODE>(G) * Tc2Cfg<MODE>::STAGE_BYTES;
+template <int MODE> constexpr size_t tc2_smem_bytes(int G, int kpb = 1) {
+  return tc2_fixed_bytes<MODE>(G) +
+         (size_t)tc2_stages<MODE>(G, kpb) * Tc2Cfg<MODE>::STAGE_BYTES * kpb;
 }
 
 template <int MODE>
@@ -126,12 +138,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TC_THREADS, 1)
   const uint32_t rank = cluster_ctarank();
   const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
   const int NST = P.stages;  // operand stages (2..MAX_STAGES), fixed by the host from G
+  const int KPB = P.kpb;     // K-blocks per stage (1, or 2 with 3-D boxes)
+  const uint32_t stage_bytes = (uint32_t)C::STAGE_BYTES * KPB;
 
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t pad = ((raw + 1023u) & ~1023u) - raw;
   unsigned char *base = smem_raw + pad;
   unsigned char *stages = base;
-  unsigned char *stg_all = base + (size_t)NST * C::STAGE_BYTES;
+  unsigned char *stg_all = base + (size_t)NST * stage_bytes;
   uint64_t *bars = (uint64_t *)(stg_all + C::STG_BYTES);
   uint32_t *tmem_slot = (uint32_t *)(bars + 2 * NST + 5);
   volatile int *abort_flag = (volatile int *)(tmem_slot + 1);
@@ -201,16 +215,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TC_THREADS, 1)
         // what that stage last held there and the epilogue masks those rows; the leader expects
         // the smaller byte count. Both CTAs decide it from the same tile record.
         const bool a1_void = ti.m0 + 128 >= ti.rows;
-        const uint32_t stage_tx = 2 * C::STAGE_BYTES - (a1_void ? C::A_BYTES : 0);
+        const uint32_t stage_tx = KPB * (2 * C::STAGE_BYTES - (a1_void ? C::A_BYTES : 0));
         const int n_off = tc2_two_b(MODE) ? 0 : (int)rank * 128;
-        const int nk = (ti.K + C::BK - 1) / C::BK;
-        for (int kb = 0; kb < nk; ++kb) {
+        const int nk = (ti.K + C::BK - 1) / C::BK;  // a multiple of KPB (the host checks)
+        for (int kb = 0; kb < nk; kb += KPB) {
           if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, limit, INFO_WAIT_MMA_EMPTY)) {
             ok = false;
             break;
           }
-          const uint32_t sA = smem_u32(stages + (size_t)stage * C::STAGE_BYTES);
-          const uint32_t sB = sA + C::A_BYTES;
+          const uint32_t sA = smem_u32(stages + (size_t)stage * stage_bytes);
+          const uint32_t sB = sA + C::A_BYTES * KPB;
           if (rank == 0) mbar_expect_tx(full_bar(stage), stage_tx);
           const int kk = kb * C::BK;
           int b_row, b_col;
@@ -225,8 +239,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TC_THREADS, 1)
             b_row = piece * p.piece_rows + ti.n0 + n_off;
             b_col = kk - piece * p.piece_k;
           }
-          if (rank == 0 || !a1_void) tma_load_2d_pair(sA, ma, ti.kofs + kk, a_row, full_bar(stage));
-          tma_load_2d_pair(sB, mb, b_col, b_row, full_bar(stage));
+          if (KPB == 2) {  // boxes of two K-blocks: coordinates {column, row, K-block}
+            if (rank == 0 || !a1_void)
+              tma_load_3d_pair(sA, ma, 0, a_row, (ti.kofs + kk) / C::BK, full_bar(stage));
+            tma_load_3d_pair(sB, mb, 0, b_row, b_col / C::BK, full_bar(stage));
+          } else {
+            if (rank == 0 || !a1_void) tma_load_2d_pair(sA, ma, ti.kofs + kk, a_row, full_bar(stage));
+            tma_load_2d_pair(sB, mb, b_col, b_row, full_bar(stage));
+          }
           issued[stage] = true;
           issued_parity[stage] = (int)phase;
           if (++stage == NST) { stage = 0; phase ^= 1u; }
@@ -258,21 +278,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TC_THREADS, 1)
         }
         tc_fence_after();
         const uint32_t d0 = tmem_base + (uint32_t)(acc * C::ACC_COLS);
-        for (int kb = 0; kb < nk; ++kb) {
+        for (int kb = 0; kb < nk; kb += KPB) {
           if (!mbar_wait(full_bar(stage), phase, abort_flag, limit, INFO_WAIT_TMA_FULL)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t sA = smem_u32(stages + (size_t)stage * C::STAGE_BYTES);
-          const uint32_t sB = sA + C::A_BYTES;
+          const uint32_t sA0 = smem_u32(stages + (size_t)stage * stage_bytes);
+          const uint32_t sB0 = sA0 + C::A_BYTES * KPB;
+          for (int j = 0; j < KPB; ++j) {  // the stage's K-blocks, 16 KB tiles one after another
+            const uint32_t sA = sA0 + j * C::A_BYTES, sB = sB0 + j * C::B_BYTES;
 #pragma unroll
-          for (int k16 = 0; k16 < 4; ++k16) {  // 32 bytes of K per instruction
-            const uint32_t accum = (kb > 0 || k16 > 0) ? 1u : 0u;
-            if (mode_fp8(MODE))
-              tc2_mma_f8(d0, make_sdesc(sA + k16 * 32), make_sdesc(sB + k16 * 32), C::IDESC, accum);
-            else
-              tc2_mma(d0, make_sdesc(sA + k16 * 32), make_sdesc(sB + k16 * 32), C::IDESC, accum);
+            for (int k16 = 0; k16 < 4; ++k16) {  // 32 bytes of K per instruction
+              const uint32_t accum = (kb > 0 || j > 0 || k16 > 0) ? 1u : 0u;
+              if (mode_fp8(MODE))
+                tc2_mma_f8(d0, make_sdesc(sA + k16 * 32), make_sdesc(sB + k16 * 32), C::IDESC, accum);
+              else
+                tc2_mma(d0, make_sdesc(sA + k16 * 32), make_sdesc(sB + k16 * 32), C::IDESC, accum);
+            }
           }
           any = true;
           tc2_commit_both(empty_bar(stage));

@@ -298,6 +298,23 @@ bool make_map(CUtensorMap *m, const void *ptr, uint64_t rows, uint64_t cols, uin
   return r == CUDA_SUCCESS;
 }
 
+// 3-D bf16 map over a row-major [rows, cols] matrix seen as {64 columns, rows, cols / 64 K-blocks}
+// (strides: the row, then 128 bytes); box {64, box_rows, 2}: two K-blocks' [box_rows, 64] tiles,
+// one after the other, 128B swizzle. cols a multiple of 128.
+bool make_map3(CUtensorMap *m, const void *ptr, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  if (rows == 0 || ptr == nullptr) rows = 1;
+  cuuint64_t dims[3] = {64, rows, cols / 64};
+  cuuint64_t strides[2] = {cols * 2, 128};
+  cuuint32_t box[3] = {64, box_rows, 2};
+  cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr), dims,
+                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 // ------------------------------------------------------------------ grouped GEMM launches
 long long tile_bound(const GroupedGemm &g, int BM, int BN) {
   if (g.kgroup) return (long long)g.E * ceil_div(g.rows_r, BM) * ceil_div(g.N_r, BN);
@@ -309,8 +326,24 @@ long long tile_bound(const GroupedGemm &g, int BM, int BN) {
 
 // Tensor maps of one grouped launch: A boxes of 128 rows, B boxes of `b_box` rows.
 // routed operands: A [rows_r, K_r], B [E*N_r, K_r]; shared: A [T, K_s], B [b_rows_s, piece_k]
-bool build_maps(const GroupedGemm &g, bool two_b, uint32_t b_box, TcMaps *m, int esz = 2) {
+bool build_maps(const GroupedGemm &g, bool two_b, uint32_t b_box, TcMaps *m, int esz = 2,
+                bool kb2 = false) {
   const void *any = g.E > 0 ? g.A_r : g.A_s;
+  if (kb2) {  // bf16, every K and piece a multiple of 128 (pair_kb2)
+    const uint64_t b_rows = (uint64_t)g.E * g.N_r;
+    bool ok = true;
+    ok &= make_map3(&m->a_r, g.E > 0 ? g.A_r : any, g.E > 0 ? g.rows_r : 1, g.E > 0 ? g.K_r : 128, 128);
+    ok &= make_map3(&m->b0_r, g.E > 0 ? g.B0_r : any, g.E > 0 ? b_rows : 1, g.E > 0 ? g.K_r : 128, b_box);
+    ok &= make_map3(&m->b1_r, (g.E > 0 && two_b) ? g.B1_r : any, (g.E > 0 && two_b) ? b_rows : 1,
+                    g.E > 0 ? g.K_r : 128, b_box);
+    ok &= make_map3(&m->a_s, g.has_shared ? g.A_s : any, g.has_shared ? g.T : 1,
+                    g.has_shared ? g.K_s : 128, 128);
+    ok &= make_map3(&m->b0_s, g.has_shared ? g.B0_s : any, g.has_shared ? g.b_rows_s : 1,
+                    g.has_shared ? g.piece_k : 128, b_box);
+    ok &= make_map3(&m->b1_s, (g.has_shared && two_b) ? g.B1_s : any,
+                    (g.has_shared && two_b) ? g.b_rows_s : 1, g.has_shared ? g.piece_k : 128, b_box);
+    return ok;
+  }
   bool ok = true;
   ok &= make_map(&m->a_r, g.E > 0 ? g.A_r : any, g.E > 0 ? g.rows_r : 1, g.E > 0 ? g.K_r : 64, 128,
                  esz);
@@ -357,12 +390,19 @@ moe_status_t launch_tc2(const GroupedGemm &g, cudaStream_t st, int kind) {
   std::memset(&P, 0, sizeof(P));
   P.p = g;
   P.p.kind = kind;
-  if (!build_maps(g, tc2_two_b(MODE), 128, &P.maps, mode_fp8(MODE) ? 1 : 2)) return MOE_ERR_CUDA;
   const int G = g.E + g.has_shared;
+  // two K-blocks per stage (3-D boxes) for the forward bf16 products when every K splits into
+  // pairs of K-blocks and the ring keeps at least 2 stages of 2
+  const bool kb2 = (MODE == MODE_GATEUP || MODE == MODE_PLAIN) && !g.kgroup && g.kb_r == 0 &&
+                   (g.E == 0 || g.K_r % 128 == 0) &&
+                   (!g.has_shared || (g.K_s % 128 == 0 && g.piece_k % 128 == 0)) &&
+                   tc2_stages<MODE>(G, 2) >= 2;
+  P.kpb = kb2 ? 2 : 1;
+  if (!build_maps(g, tc2_two_b(MODE), 128, &P.maps, mode_fp8(MODE) ? 1 : 2, kb2)) return MOE_ERR_CUDA;
   static_assert(tc2_stages<MODE>(1024 + 1) >= 2, "tile list of 1024 experts leaves no room");
-  P.stages = tc2_stages<MODE>(G);
+  P.stages = tc2_stages<MODE>(G, P.kpb);
   if (P.stages < 2) return MOE_ERR_UNSUPPORTED;
-  const size_t smem = tc2_smem_bytes<MODE>(G);
+  const size_t smem = tc2_smem_bytes<MODE>(G, P.kpb);
   auto kern = gemm_tc2_kernel<MODE>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return MOE_ERR_CUDA;
