@@ -217,7 +217,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TC_THREADS, 1)
         const bool a1_void = ti.m0 + 128 >= ti.rows;
         const uint32_t stage_tx = KPB * (2 * C::STAGE_BYTES - (a1_void ? C::A_BYTES : 0));
         const int n_off = tc2_two_b(MODE) ? 0 : (int)rank * 128;
-        const int nk = (ti.K + C::BK - 1) / C::BK;  // a multiple of KPB (the host checks)
+        // with two K-blocks per stage an odd count leaves the last stage half used: its second
+        // tile (the next group's columns, or the map's zero fill) is loaded and not multiplied
+        const int nk = (ti.K + C::BK - 1) / C::BK;
         for (int kb = 0; kb < nk; kb += KPB) {
           if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, limit, INFO_WAIT_MMA_EMPTY)) {
             ok = false;
@@ -286,7 +288,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TC_THREADS, 1)
           tc_fence_after();
           const uint32_t sA0 = smem_u32(stages + (size_t)stage * stage_bytes);
           const uint32_t sB0 = sA0 + C::A_BYTES * KPB;
-          for (int j = 0; j < KPB; ++j) {  // the stage's K-blocks, 16 KB tiles one after another
+          for (int j = 0; j < KPB && kb + j < nk; ++j) {  // the stage's K-blocks, 16 KB tiles
             const uint32_t sA = sA0 + j * C::A_BYTES, sB = sB0 + j * C::B_BYTES;
 #pragma unroll
             for (int k16 = 0; k16 < 4; ++k16) {  // 32 bytes of K per instruction

@@ -300,7 +300,8 @@ bool make_map(CUtensorMap *m, const void *ptr, uint64_t rows, uint64_t cols, uin
 
 // 3-D bf16 map over a row-major [rows, cols] matrix seen as {64 columns, rows, cols / 64 K-blocks}
 // (strides: the row, then 128 bytes); box {64, box_rows, 2}: two K-blocks' [box_rows, 64] tiles,
-// one after the other, 128B swizzle. cols a multiple of 128.
+// one after the other, 128B swizzle. cols a multiple of 64; a box's K-block past the last reads
+// as zeros.
 bool make_map3(CUtensorMap *m, const void *ptr, uint64_t rows, uint64_t cols, uint32_t box_rows) {
   auto fn = encode_fn();
   if (!fn) return false;
@@ -329,13 +330,14 @@ long long tile_bound(const GroupedGemm &g, int BM, int BN) {
 bool build_maps(const GroupedGemm &g, bool two_b, uint32_t b_box, TcMaps *m, int esz = 2,
                 bool kb2 = false) {
   const void *any = g.E > 0 ? g.A_r : g.A_s;
-  if (kb2) {  // bf16, every K and piece a multiple of 128 (pair_kb2)
-    const uint64_t b_rows = (uint64_t)g.E * g.N_r;
+  if (kb2) {  // bf16; the same extents as the 2-D maps below
+    const int kb = g.kb_r ? g.kb_r : g.K_r;
+    const uint64_t b_rows = g.kgroup ? (uint64_t)g.N_r : (uint64_t)g.E * g.N_r;
     bool ok = true;
     ok &= make_map3(&m->a_r, g.E > 0 ? g.A_r : any, g.E > 0 ? g.rows_r : 1, g.E > 0 ? g.K_r : 128, 128);
-    ok &= make_map3(&m->b0_r, g.E > 0 ? g.B0_r : any, g.E > 0 ? b_rows : 1, g.E > 0 ? g.K_r : 128, b_box);
+    ok &= make_map3(&m->b0_r, g.E > 0 ? g.B0_r : any, g.E > 0 ? b_rows : 1, g.E > 0 ? kb : 128, b_box);
     ok &= make_map3(&m->b1_r, (g.E > 0 && two_b) ? g.B1_r : any, (g.E > 0 && two_b) ? b_rows : 1,
-                    g.E > 0 ? g.K_r : 128, b_box);
+                    g.E > 0 ? kb : 128, b_box);
     ok &= make_map3(&m->a_s, g.has_shared ? g.A_s : any, g.has_shared ? g.T : 1,
                     g.has_shared ? g.K_s : 128, 128);
     ok &= make_map3(&m->b0_s, g.has_shared ? g.B0_s : any, g.has_shared ? g.b_rows_s : 1,
@@ -391,12 +393,10 @@ moe_status_t launch_tc2(const GroupedGemm &g, cudaStream_t st, int kind) {
   P.p = g;
   P.p.kind = kind;
   const int G = g.E + g.has_shared;
-  // two K-blocks per stage (3-D boxes) for the forward bf16 products when every K splits into
-  // pairs of K-blocks and the ring keeps at least 2 stages of 2
-  const bool kb2 = (MODE == MODE_GATEUP || MODE == MODE_PLAIN) && !g.kgroup && g.kb_r == 0 &&
-                   (g.E == 0 || g.K_r % 128 == 0) &&
-                   (!g.has_shared || (g.K_s % 128 == 0 && g.piece_k % 128 == 0)) &&
-                   tc2_stages<MODE>(G, 2) >= 2;
+  // two K-blocks per stage (3-D boxes) for the bf16 products, when no stage can cross a wrap
+  // point of B's columns or a shared-expert piece, and the ring keeps at least 2 stages of 2
+  const bool kb2 = !mode_fp8(MODE) && (g.kb_r == 0 || g.kb_r % 128 == 0) &&
+                   (!g.has_shared || g.piece_k % 128 == 0) && tc2_stages<MODE>(G, 2) >= 2;
   P.kpb = kb2 ? 2 : 1;
   if (!build_maps(g, tc2_two_b(MODE), 128, &P.maps, mode_fp8(MODE) ? 1 : 2, kb2)) return MOE_ERR_CUDA;
   static_assert(tc2_stages<MODE>(1024 + 1) >= 2, "tile list of 1024 experts leaves no room");
