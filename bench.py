@@ -294,12 +294,13 @@ def run_ours(args, rank, world, local_rank):
     moe.load()
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
-    c = get_config(args.config)
+    fp8 = args.config.endswith("_fp8")  # low-rank experts stored as E4M3 rows
+    c = get_config(args.config[:-4] if fp8 else args.config)
     inp = make_inputs(c)
     cfg = B.make_config(T=c.T, d=c.d, E=c.E, top_k=c.top_k, n_shared=c.n_shared, ffn=c.ffn,
                         ffn_shared=c.ffn_shared, rank=c.rank, score=c.score, expert=c.expert,
                         dtype=c.dtype, norm_topk=c.norm_topk, capacity_factor=c.capacity_factor,
-                        aux_alpha=c.aux_alpha)
+                        aux_alpha=c.aux_alpha, expert_storage="fp8" if fp8 else "dtype")
     weights = upload_weights(cfg, inp, dev)
     layer = MoELayer(cfg, weights, dev)
     dt = layer.dtype
@@ -463,8 +464,9 @@ def run_ours(args, rank, world, local_rank):
 
     peaks, peak_src = load_peaks()
     backward = backward_parts(c, cfg, layer, x, flush, stream, args.steps, peaks) \
-        if world == 1 else None
-    table = roofline_table(c, n_kept, prof, args.steps, peaks, peak_src, in_step)
+        if world == 1 and not fp8 else None  # training stays bf16: no backward of fp8 storage
+    table = roofline_table(c, n_kept, prof, args.steps, peaks, peak_src, in_step, fp8,
+                           int((counts > 0).sum()))
     dom = max(table, key=lambda n: table[n]["share"] or 0.0)
     dr = table[dom]
     launches_per_step = sum(n for _, n in prof.values()) / max(args.steps, 1)
@@ -484,7 +486,7 @@ def run_ours(args, rank, world, local_rank):
         "data": "synthetic: seeded torch CPU generator, bf16-rounded N(0,1) tokens and "
                 "random-init weights of the configuration's shapes (no dataset, no checkpoint)",
         "config": {
-            "workload": workload_name(c),
+            "workload": workload_name(c, fp8),
             "tokens_per_gpu": c.T,
             "l2": "flushed between timed steps (256 MiB write outside the events)",
             "parallelism": f"dp{world} replicas" + (" + NCCL all-reduce of 2E expert stats"

@@ -965,7 +965,8 @@ moe_status_t moe_expert_backward(const moe_config_t *cfg, const void *x_perm,
                                  float *dx, const moe_grads_t *g, void *ws, size_t ws_bytes,
                                  void *stream) {
   MOE_TRY(check_cfg(cfg));
-  if (cfg->dtype != MOE_DTYPE_BF16) return MOE_ERR_UNSUPPORTED;
+  if (cfg->dtype != MOE_DTYPE_BF16 || cfg->expert_storage != MOE_STORAGE_DTYPE)
+    return MOE_ERR_UNSUPPORTED;
   MOE_TRY(check_weights(cfg, w, false, true));
   MOE_REQUIRE(g != nullptr);
   MOE_REQUIRE(tok16(cfg, x_perm) && aligned16(offsets) && tok16(cfg, slot_pos) && tok16(cfg, x) &&

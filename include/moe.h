@@ -234,7 +234,8 @@ size_t moe_backward_workspace_size(const moe_config_t *cfg);
  * Operands that are not exact bf16 values (g, u, dg, du, h, z, dz, z s, the fp32 dy and the
  * low-rank layers' fp32 dy_perm) enter the tensor-core products as two bf16 terms, value and
  * rounding residual, so each gradient carries no single bf16 rounding of its operands.
- * Supported: bf16 layers (SwiGLU or low-rank experts); fp32 layers return MOE_ERR_UNSUPPORTED.
+ * Supported: bf16 layers (SwiGLU or low-rank experts); fp32 layers and layers whose experts are
+ * stored in fp8 (training stays bf16) return MOE_ERR_UNSUPPORTED.
  * ws: moe_backward_workspace_size(cfg) bytes of the caller's device memory. Asynchronous. */
 moe_status_t moe_expert_backward(const moe_config_t *cfg, const void *x_perm,
                                  const int32_t *offsets, const int32_t *slot_pos, const void *x,

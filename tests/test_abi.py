@@ -61,6 +61,15 @@ def test_fp8_storage_only_for_bf16_lowrank(lib):
     assert B.moe_workspace_size(bad) == 0
 
 
+def test_expert_backward_refuses_fp8_storage(lib):
+    cfg = cfg_of(CONFIGS["lowrank"], T=64, expert_storage="fp8")
+    w = B.MoEWeights()
+    g = B.MoEGrads()
+    st = lib.moe_expert_backward(ctypes.byref(cfg), None, None, None, None, ctypes.byref(w), None,
+                                 None, None, ctypes.byref(g), None, 0, None)
+    assert st == 2  # MOE_ERR_UNSUPPORTED, before any pointer is looked at
+
+
 def test_quantize_fp8_host_refusals(lib):
     # cols not a multiple of 16, a bad dtype, negative rows: refused before any device work
     assert lib.moe_quantize_fp8(None, 1, 4, 24, None, None, None) == 2
