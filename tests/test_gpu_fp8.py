@@ -128,3 +128,12 @@ def test_fp8_layer_no_tokens():
                         B.make_weights(w), y, aux, cnt, ws, ws_bytes)
     torch.cuda.synchronize()
     assert float(aux) == 0.0 and int(cnt.abs().sum()) == 0
+
+
+def test_fp8_layer_bitwise_determinism():
+    c = CASES["lr_fp8_s"]
+    run = Fp8Layer(c, make_inputs(c))
+    y1, a1, _ = run.layer()
+    y1 = y1.clone()
+    y2, a2, _ = run.layer()
+    assert torch.equal(y1, y2) and float(a1) == float(a2)

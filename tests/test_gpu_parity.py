@@ -503,8 +503,11 @@ def test_back_to_back_calls_on_one_workspace():
         assert torch.equal(ya, yb) and aa == float(ab) and torch.equal(ca, cb)
 
 
-def test_bitwise_determinism():
-    c = SMALL["quartz_s"]
+@pytest.mark.parametrize("name", ["quartz_s", "tiny_f32", "lowrank_f32_shared", "sigmoid_s"])
+def test_bitwise_determinism(name):
+    """Two calls on the same inputs give the same bits (bf16 and fp32 layers; the fp32 one runs
+    its products on split bf16 terms)."""
+    c = SMALL[name] if name in SMALL else EDGE[name]
     run = LayerOnGpu(c, make_inputs(c))
     y1, a1, _ = run.layer()
     y1 = y1.clone()
