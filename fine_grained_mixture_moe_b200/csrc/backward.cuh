@@ -258,23 +258,35 @@ __global__ void __launch_bounds__(256) router_dgrad_kernel(const float *__restri
 // gradients (dh = dY W_d, dX = [dg | du] [W_g; W_u]) the same way.
 
 // koff[e] = sum over e' < e of the expert's row count rounded up to 64; koff[E] is the total.
+// korder: the experts by padded row count, largest first (ties: lower index first), the order in
+// which the weight-gradient products list their groups (each group's K is its row count, so
+// longest first balances the CTA pairs' round-robin share of the tiles).
 // Also the group tables of the shared experts' T rows cut into nc chunks of ch rows (ch a
 // multiple of 64): off_s[i] = min(i ch, T), koff_s[i] = the same rounded up to 64. One block;
 // E <= 1024, nc <= 64.
 __global__ void __launch_bounds__(1024) pad_offsets_kernel(const int32_t *__restrict__ offsets,
                                                            int E, int32_t *__restrict__ koff,
+                                                           int32_t *__restrict__ korder,
                                                            int T, int nc, int ch,
                                                            int32_t *__restrict__ off_s,
                                                            int32_t *__restrict__ koff_s) {
   griddep_wait();
   griddep_launch();
   __shared__ int s[1024];
+  __shared__ int sz[1024];
   __shared__ int tmp[1024 / 32 + 1];
   const int e = threadIdx.x;
   s[e] = e < E ? ((offsets[e + 1] - offsets[e] + 63) & ~63) : 0;
+  sz[e] = s[e];
   __syncthreads();
   const int total = block_excl_scan_inplace(s, 1024, tmp);
-  if (e < E) koff[e] = s[e];
+  if (e < E) {
+    koff[e] = s[e];
+    const int v = sz[e];
+    int r = 0;
+    for (int h = 0; h < E; ++h) r += (sz[h] > v || (sz[h] == v && h < e)) ? 1 : 0;
+    korder[r] = e;
+  }
   if (e == 0) koff[E] = total;
   if (e <= nc) {
     const int v = min(e * ch, T);

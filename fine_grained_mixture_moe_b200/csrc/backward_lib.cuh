@@ -36,7 +36,7 @@ moe_status_t route_backward_impl(const moe_config_t *c, const RouteBwdArgs &a, f
 constexpr int BWD_SHARED_CHUNKS = 8;
 
 struct BwdLayout {
-  size_t koff, off_s, koff_s;
+  size_t koff, korder, off_s, koff_s;
   size_t gu, dgu, h, dxp, gu_s, dgu_s, h_s, dx_s, dy_b;
   size_t wdt, wgut, wsdt, wsgut;
   size_t ydt, ht, dgut, xpt, ydt_s, ht_s, dgut_s, xt_s;
@@ -63,6 +63,7 @@ BwdLayout bwd_layout(const moe_config_t *c) {
   size_t o = 0;
   auto take = [&](size_t bytes) { size_t at = o; o = align256(o + std::max<size_t>(bytes, 1)); return at; };
   L.koff = take((E + 1) * 4);
+  L.korder = take(E * 4);
   L.off_s = take((BWD_SHARED_CHUNKS + 1) * 4);
   L.koff_s = take((BWD_SHARED_CHUNKS + 1) * 4);
   L.gu = take(np * 2 * f * 4);  // blocked g, u: each group's rows padded to 64
@@ -122,13 +123,16 @@ moe_status_t launch_transpose_dense(const bf16_t *in, int R, int C, int batches,
 }
 
 // One weight-gradient product with groups along K: out[g] (M x N, fp32, row-major) =
-// A[:, kseg koff[g] .. kseg koff[g+1]) B[:, same]^T, A [M, ld], B [N, ld] bf16.
-moe_status_t launch_wgrad(int G, const int32_t *koff, int kseg, const void *A, int M,
-                          const void *Bm, int N, int ld, float *out, cudaStream_t st) {
+// A[:, kseg koff[g] .. kseg koff[g+1]) B[:, same]^T, A [M, ld], B [N, ld] bf16. `order` (device,
+// or null for group order) lists the groups in the order their tiles are dealt to the CTA pairs.
+moe_status_t launch_wgrad(int G, const int32_t *koff, const int32_t *order, int kseg,
+                          const void *A, int M, const void *Bm, int N, int ld, float *out,
+                          cudaStream_t st) {
   GroupedGemm g;
   std::memset(&g, 0, sizeof(g));
   g.kgroup = 1;
   g.koff = koff;
+  g.gorder = order;
   g.kseg = kseg;
   g.E = G;
   g.A_r = A;
@@ -153,8 +157,8 @@ moe_status_t expert_backward_impl(const moe_config_t *c, const void *x_perm,
   const int S = c->n_shared, fs = c->ffn_shared, sf = S * fs;
   const bool sh = S > 0;
   using bf = bf16_t;
-  int32_t *koff = at<int32_t>(ws, L.koff), *off_s = at<int32_t>(ws, L.off_s),
-          *koff_s = at<int32_t>(ws, L.koff_s);
+  int32_t *koff = at<int32_t>(ws, L.koff), *korder = at<int32_t>(ws, L.korder),
+          *off_s = at<int32_t>(ws, L.off_s), *koff_s = at<int32_t>(ws, L.koff_s);
   float *GU = at<float>(ws, L.gu), *GUs = at<float>(ws, L.gu_s);
   bf *DGU = at<bf>(ws, L.dgu), *H = at<bf>(ws, L.h);
   float *dXp = at<float>(ws, L.dxp), *dXs = at<float>(ws, L.dx_s);
@@ -168,8 +172,8 @@ moe_status_t expert_backward_impl(const moe_config_t *c, const void *x_perm,
   const bf *xp = (const bf *)x_perm, *xb = (const bf *)x;
 
   // padded group offsets of the weight gradients
-  MOE_TRY(launch_pdl(pad_offsets_kernel, dim3(1), dim3(1024), 0, st, offsets, E, koff, T, L.nc,
-                     L.ch, off_s, koff_s));
+  MOE_TRY(launch_pdl(pad_offsets_kernel, dim3(1), dim3(1024), 0, st, offsets, E, koff, korder, T,
+                     L.nc, L.ch, off_s, koff_s));
   // the SwiGLU launches carry the routed SwiGLU experts (E groups) and / or the shared experts
   GroupedGemm base;
   std::memset(&base, 0, sizeof(base));
@@ -286,8 +290,8 @@ moe_status_t expert_backward_impl(const moe_config_t *c, const void *x_perm,
                                      3 * np, st));
     MOE_TRY(launch_transpose_grouped(3, ZS2, ZS2 + r, ZS2, r, 2 * r, offsets, koff, E, nb3, ZSt,
                                      3 * np, st));
-    MOE_TRY(launch_wgrad(E, koff, 2, DZt, r, Xpt, d, 2 * np, gr->d_lr_V, st));
-    MOE_TRY(launch_wgrad(E, koff, 3, Ydt, d, ZSt, r, 3 * np, gr->d_lr_U, st));
+    MOE_TRY(launch_wgrad(E, koff, korder, 2, DZt, r, Xpt, d, 2 * np, gr->d_lr_V, st));
+    MOE_TRY(launch_wgrad(E, koff, korder, 3, Ydt, d, ZSt, r, 3 * np, gr->d_lr_U, st));
     MOE_TRY(launch_pdl(zero_empty_experts_kernel, dim3(E, 8), dim3(256), 0, st, offsets,
                        gr->d_lr_V, (size_t)r * d, gr->d_lr_U, (size_t)d * r, (float *)nullptr,
                        (size_t)0));
@@ -306,9 +310,9 @@ moe_status_t expert_backward_impl(const moe_config_t *c, const void *x_perm,
     MOE_TRY(launch_transpose_grouped(2, DGU, DGU + 2 * f, nullptr, 2 * f, 4 * f, offsets, koff, E,
                                      nb2, DGUt, 2 * np, st));
     MOE_TRY(launch_transpose_grouped(2, xp, xp, nullptr, d, d, offsets, koff, E, nb2, Xpt, 2 * np, st));
-    MOE_TRY(launch_wgrad(E, koff, 2, Ydt, d, Ht, f, 2 * np, gr->d_w_down, st));
-    MOE_TRY(launch_wgrad(E, koff, 2, DGUt, f, Xpt, d, 2 * np, gr->d_w_gate, st));
-    MOE_TRY(launch_wgrad(E, koff, 2, DGUt + (size_t)f * 2 * np, f, Xpt, d, 2 * np, gr->d_w_up, st));
+    MOE_TRY(launch_wgrad(E, koff, korder, 2, Ydt, d, Ht, f, 2 * np, gr->d_w_down, st));
+    MOE_TRY(launch_wgrad(E, koff, korder, 2, DGUt, f, Xpt, d, 2 * np, gr->d_w_gate, st));
+    MOE_TRY(launch_wgrad(E, koff, korder, 2, DGUt + (size_t)f * 2 * np, f, Xpt, d, 2 * np, gr->d_w_up, st));
     MOE_TRY(launch_pdl(zero_empty_experts_kernel, dim3(E, 8), dim3(256), 0, st, offsets,
                        gr->d_w_gate, (size_t)f * d, gr->d_w_up, (size_t)f * d, gr->d_w_down,
                        (size_t)d * f));
@@ -331,12 +335,12 @@ moe_status_t expert_backward_impl(const moe_config_t *c, const void *x_perm,
                                      3 * tp / 64, Ydts, 3 * tp, st));
     MOE_TRY(launch_transpose_grouped(3, Hs, Hs + sf, Hs, sf, 2 * sf, off_s, koff_s, nc,
                                      3 * tp / 64, Hts, 3 * tp, st));
-    MOE_TRY(launch_wgrad(nc, koff_s, 2, DGUts, sf, Xts, d, 2 * tp, part, st));
+    MOE_TRY(launch_wgrad(nc, koff_s, nullptr, 2, DGUts, sf, Xts, d, 2 * tp, part, st));
     MOE_TRY(sum_chunks((size_t)sf * d, gr->d_ws_gate));
-    MOE_TRY(launch_wgrad(nc, koff_s, 2, DGUts + (size_t)sf * 2 * tp, sf, Xts, d, 2 * tp, part, st));
+    MOE_TRY(launch_wgrad(nc, koff_s, nullptr, 2, DGUts + (size_t)sf * 2 * tp, sf, Xts, d, 2 * tp, part, st));
     MOE_TRY(sum_chunks((size_t)sf * d, gr->d_ws_up));
     for (int s = 0; s < S; ++s) {
-      MOE_TRY(launch_wgrad(nc, koff_s, 3, Ydts, d, Hts + (size_t)s * fs * 3 * tp, fs, 3 * tp, part,
+      MOE_TRY(launch_wgrad(nc, koff_s, nullptr, 3, Ydts, d, Hts + (size_t)s * fs * 3 * tp, fs, 3 * tp, part,
                            st));
       MOE_TRY(sum_chunks((size_t)d * fs, gr->d_ws_down + (size_t)s * d * fs));
     }

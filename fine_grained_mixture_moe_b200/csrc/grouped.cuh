@@ -89,6 +89,8 @@ struct GroupedGemm {
   int kgroup;
   const int32_t *koff;     // [E+1] device: padded K offsets of the groups
   int kseg;                // K segments per group (kgroup)
+  const int32_t *gorder;   // kgroup: [E] device, the group at each position of the tile list
+                           // (longest K first); null: group order
 };
 
 // Tile list order: the shared group (its K may be several experts' widths: the longest tiles)
@@ -107,7 +109,8 @@ __device__ __forceinline__ int build_tile_prefix(const GroupedGemm &p, int BM, i
   const int ntr = (p.N_r + BN - 1) / BN, nts = (p.N_s + BN - 1) / BN;
   for (int o = threadIdx.x; o < G; o += blockDim.x) {
     if (p.kgroup) {
-      const int kg = p.kseg * (p.koff[o + 1] - p.koff[o]);
+      const int g = p.gorder ? p.gorder[o] : o;
+      const int kg = p.kseg * (p.koff[g + 1] - p.koff[g]);
       prefix[o] = kg > 0 ? ((p.rows_r + BM - 1) / BM) * ntr : 0;
       continue;
     }
@@ -140,7 +143,7 @@ __device__ __forceinline__ TileInfo decode_tile(const GroupedGemm &p, int tile,
   }
   TileInfo ti;
   const int local = tile - prefix[lo];
-  lo = p.kgroup ? lo : group_at(p, lo);  // list position -> group
+  lo = p.kgroup ? (p.gorder ? p.gorder[lo] : lo) : group_at(p, lo);  // list position -> group
   ti.g = lo;
   const bool routed = lo < p.E;
   ti.N = routed ? p.N_r : p.N_s;
