@@ -621,10 +621,10 @@ def measure_config(name, K, W, dev, flush, stream, peaks, peak_src):
     return out
 
 
-def backward_parts(c, cfg, layer, x, flush, stream, K, peaks):
-    """The backward's entry points (combine, experts, router), each call timed alone with CUDA
-    events on the forward's resident outputs and a seeded upstream gradient, L2 flushed between
-    calls. Not part of the step above."""
+def backward_calls(c, cfg, layer, x):
+    """The forward's outputs (route, permute, experts) on the device and the three backward
+    entry points as callables on them, with a seeded upstream gradient: (combine, route,
+    experts, info). Used by backward_parts and by --backward-launches."""
     import torch
 
     from fine_grained_mixture_moe_b200 import binding as B
@@ -655,24 +655,6 @@ def backward_parts(c, cfg, layer, x, flush, stream, K, peaks):
     dx = torch.empty((T, d), dtype=torch.float32, device=dev)
     torch.cuda.synchronize()
     N = int(offsets[-1])
-
-    def timed_call(fn):
-        for _ in range(3):
-            fn()
-        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-              for _ in range(K)]
-        torch.cuda.synchronize()
-        for i in range(K):
-            flush.fill_(i & 0xff)
-            ev[i][0].record(stream)
-            fn()
-            ev[i][1].record(stream)
-        torch.cuda.synchronize()
-        return statistics.fmean(a.elapsed_time(b) for a, b in ev) * 1e3
-
-    us_c = timed_call(lambda: B.moe_combine_backward(cfg, dy, yp, slot, wts, dyp, d_w))
-    us_r = timed_call(lambda: B.moe_route_backward(cfg, x, layer.wstruct, idx, cnt, d_w, 1.0,
-                                                   d_logits, d_wr, dx))
     # the experts' backward: data and weight gradients of every routed and shared expert
     E_, f_, r_, S_, fs_ = c.E, c.ffn, c.rank, c.n_shared, c.ffn_shared
     if c.expert == "swiglu":
@@ -694,14 +676,55 @@ def backward_parts(c, cfg, layer, x, flush, stream, K, peaks):
     bw_ws = torch.empty(bws, dtype=torch.uint8, device=dev)
     dx_e = torch.empty((T, d), dtype=torch.float32, device=dev)
     gstruct = B.make_grads(gr)
-    us_e = timed_call(lambda: B.moe_expert_backward(cfg, xp, offsets, slot, x, layer.wstruct, dyp,
-                                                    dy if S_ else None, dx_e, gstruct, bw_ws,
-                                                    bws))
-    del bw_ws
-    st, info = B.moe_get_device_error()
+
+    def combine():
+        B.moe_combine_backward(cfg, dy, yp, slot, wts, dyp, d_w)
+
+    def route():
+        B.moe_route_backward(cfg, x, layer.wstruct, idx, cnt, d_w, 1.0, d_logits, d_wr, dx)
+
+    def experts():
+        B.moe_expert_backward(cfg, xp, offsets, slot, x, layer.wstruct, dyp, dy if S_ else None,
+                              dx_e, gstruct, bw_ws, bws)
+
+    info = {"N": N, "flop_e": flop_e, "by": yp.element_size(), "bx": x.element_size(),
+            "keep": (gr, bw_ws)}
+    return combine, route, experts, info
+
+
+def backward_parts(c, cfg, layer, x, flush, stream, K, peaks):
+    """The backward's entry points (combine, experts, router), each call timed alone with CUDA
+    events on the forward's resident outputs and a seeded upstream gradient, L2 flushed between
+    calls. Not part of the step above."""
+    import torch
+
+    from fine_grained_mixture_moe_b200 import binding as B
+
+    T, d, E, k = c.T, c.d, c.E, c.top_k
+    combine, route, experts, info = backward_calls(c, cfg, layer, x)
+    N, flop_e = info["N"], info["flop_e"]
+
+    def timed_call(fn):
+        for _ in range(3):
+            fn()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(K)]
+        torch.cuda.synchronize()
+        for i in range(K):
+            flush.fill_(i & 0xff)
+            ev[i][0].record(stream)
+            fn()
+            ev[i][1].record(stream)
+        torch.cuda.synchronize()
+        return statistics.fmean(a.elapsed_time(b) for a, b in ev) * 1e3
+
+    us_c = timed_call(combine)
+    us_r = timed_call(route)
+    us_e = timed_call(experts)
+    st, info_err = B.moe_get_device_error()
     if st != 0:
-        raise RuntimeError(f"device error in the backward pass: {B.status_str(st)} info={info}")
-    by, bx = yp.element_size(), x.element_size()
+        raise RuntimeError(f"device error in the backward pass: {B.status_str(st)} info={info_err}")
+    by, bx = info["by"], info["bx"]
     # algorithmic bytes: every input read once, every output written once
     bytes_c = T * d * 4 + 2 * N * d * by + T * k * 12
     bytes_r = T * d * bx + E * d * bx + T * k * 8 + E * 4 + T * E * 4 + E * d * 4 + T * d * 4
@@ -797,6 +820,41 @@ def run_reference(args):
     }
 
 
+def run_backward_launches(args):
+    """--backward-launches: the backward entry points of one configuration, twice each, untimed
+    (a short program for a profiler's launch list; prints one line)."""
+    import torch
+
+    import fine_grained_mixture_moe_b200 as moe
+    from fine_grained_mixture_moe_b200 import binding as B
+    from fine_grained_mixture_moe_b200 import build as _b
+    from fine_grained_mixture_moe_b200.layer import MoELayer, upload_weights
+    from moe_synth import get_config, make_inputs
+
+    _b.build()
+    moe.load()
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    c = get_config(args.config)
+    inp = make_inputs(c)
+    cfg = B.make_config(T=c.T, d=c.d, E=c.E, top_k=c.top_k, n_shared=c.n_shared, ffn=c.ffn,
+                        ffn_shared=c.ffn_shared, rank=c.rank, score=c.score, expert=c.expert,
+                        dtype=c.dtype, norm_topk=c.norm_topk, capacity_factor=c.capacity_factor,
+                        aux_alpha=c.aux_alpha)
+    layer = MoELayer(cfg, upload_weights(cfg, inp, dev), dev)
+    x = torch.as_tensor(inp["x"]).to(layer.dtype).contiguous().to(dev)
+    combine, route, experts, _ = backward_calls(c, cfg, layer, x)
+    for _ in range(2):
+        combine()
+        route()
+        experts()
+    torch.cuda.synchronize()
+    st, info = B.moe_get_device_error()
+    if st != 0:
+        raise RuntimeError(f"device error in the backward pass: {B.status_str(st)} info={info}")
+    return {"backward_launches": c.name, "passes": 2}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -808,7 +866,12 @@ def main():
     ap.add_argument("--per-config", default="capacity,sigmoid,lowrank,lowrank_fp8",
                     help="further configurations timed on one GPU beside the headline one "
                          "(comma-separated names, or 'none')")
+    ap.add_argument("--backward-launches", action="store_true",
+                    help="run the backward entry points of --config twice, untimed, and exit")
     args = ap.parse_args()
+    if args.backward_launches:
+        print(json.dumps(run_backward_launches(args)), flush=True)
+        return
     if args.warmup < 3:
         args.warmup = 3
     world = int(os.environ.get("WORLD_SIZE", "1"))

@@ -46,46 +46,110 @@ template <> struct Bw4<__nv_bfloat16> {
   }
 };
 
-// One warp per token; lane l takes the columns 4l, 4l + 128, ...; each of the k dot products is
-// reduced over the lanes in a fixed tree.
+// eight consecutive elements of a row: loaded raw (one 16-byte access for bf16, two for fp32),
+// then widened to fp32
+template <typename Ty> struct Bw8;
+template <> struct Bw8<float> {
+  struct Raw { float4 a, b; };
+  static __device__ __forceinline__ Raw ld(const float *p) {
+    return Raw{((const float4 *)p)[0], ((const float4 *)p)[1]};
+  }
+  static __device__ __forceinline__ void unpack(const Raw &r, float (&v)[8]) {
+    v[0] = r.a.x; v[1] = r.a.y; v[2] = r.a.z; v[3] = r.a.w;
+    v[4] = r.b.x; v[5] = r.b.y; v[6] = r.b.z; v[7] = r.b.w;
+  }
+  static __device__ __forceinline__ void st(float *p, const float (&v)[8]) {
+    ((float4 *)p)[0] = make_float4(v[0], v[1], v[2], v[3]);
+    ((float4 *)p)[1] = make_float4(v[4], v[5], v[6], v[7]);
+  }
+};
+template <> struct Bw8<__nv_bfloat16> {
+  using Raw = uint4;
+  static __device__ __forceinline__ Raw ld(const __nv_bfloat16 *p) { return *(const uint4 *)p; }
+  static __device__ __forceinline__ void unpack(const Raw &r, float (&v)[8]) {
+    const uint32_t u[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 f = __bfloat1622float2(*(const __nv_bfloat162 *)&u[i]);
+      v[2 * i] = f.x;
+      v[2 * i + 1] = f.y;
+    }
+  }
+  static __device__ __forceinline__ void st(__nv_bfloat16 *p, const float (&v)[8]) {
+    uint32_t u[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const __nv_bfloat162 b = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
+      u[i] = *(const uint32_t *)&b;
+    }
+    *(uint4 *)p = make_uint4(u[0], u[1], u[2], u[3]);
+  }
+};
+
+// A block of 8 warps takes tpb tokens (tpb in {1, 2, 4, 8}), 8 / tpb warps per token; a warp takes
+// the token's 256-column slices w, w + 8 / tpb, ... with eight columns per lane, and issues the
+// loads of all k rows of a slice before it uses them. Each dot product is summed per lane over
+// its columns, over the lanes in a fixed tree, then over the token's warps in order.
 template <typename Ty>
-__global__ void __launch_bounds__(256) combine_backward_kernel(
+__global__ void __launch_bounds__(256, sizeof(Ty) == 2 ? 3 : 2) combine_backward_kernel(
     const float *__restrict__ dy, const Ty *__restrict__ y_perm,
     const int32_t *__restrict__ slot_pos, const float *__restrict__ w, Ty *__restrict__ dy_perm,
-    float *__restrict__ d_w, int T, int k, int d) {
+    float *__restrict__ d_w, int T, int k, int d, int tpb) {
+  __shared__ float part[8][8];  // [warp][slot]
   griddep_wait();
   griddep_launch();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int t = blockIdx.x * 8 + warp;
-  if (t >= T) return;
-  int pos[8];
-  float wj[8], dot[8];
+  const int wpt = 8 / tpb;
+  const int tl = warp / wpt;
+  const int t = blockIdx.x * tpb + tl;
+  float dot[8];
 #pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    pos[j] = j < k ? slot_pos[(size_t)t * k + j] : -1;
-    wj[j] = j < k ? w[(size_t)t * k + j] : 0.0f;
-    dot[j] = 0.0f;
-  }
-#pragma unroll 1
-  for (int c = 4 * lane; c < d; c += 128) {
-    const float4 g = *(const float4 *)(dy + (size_t)t * d + c);
+  for (int j = 0; j < 8; ++j) dot[j] = 0.0f;
+  if (t < T) {
+    int pos[8];
+    float wj[8];
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
-      if (pos[j] < 0) continue;
-      const float4 v = Bw4<Ty>::ld(y_perm + (size_t)pos[j] * d + c);
-      dot[j] = fmaf(g.x, v.x, dot[j]);
-      dot[j] = fmaf(g.y, v.y, dot[j]);
-      dot[j] = fmaf(g.z, v.z, dot[j]);
-      dot[j] = fmaf(g.w, v.w, dot[j]);
-      Bw4<Ty>::st(dy_perm + (size_t)pos[j] * d + c,
-                  make_float4(wj[j] * g.x, wj[j] * g.y, wj[j] * g.z, wj[j] * g.w));
+      pos[j] = j < k ? slot_pos[(size_t)t * k + j] : -1;
+      wj[j] = j < k ? w[(size_t)t * k + j] : 0.0f;
+    }
+    for (int c = ((warp - tl * wpt) * 32 + lane) * 8; c < d; c += wpt * 256) {
+      typename Bw8<Ty>::Raw r[8];
+      const Bw8<float>::Raw gr = Bw8<float>::ld(dy + (size_t)t * d + c);
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        if (pos[j] >= 0) r[j] = Bw8<Ty>::ld(y_perm + (size_t)pos[j] * d + c);
+      float g[8];
+      Bw8<float>::unpack(gr, g);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        if (pos[j] < 0) continue;
+        float v[8], o[8];
+        Bw8<Ty>::unpack(r[j], v);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          dot[j] = fmaf(g[i], v[i], dot[j]);
+          o[i] = wj[j] * g[i];
+        }
+        Bw8<Ty>::st(dy_perm + (size_t)pos[j] * d + c, o);
+      }
     }
   }
 #pragma unroll
   for (int j = 0; j < 8; ++j) {
     if (j >= k) break;
     const float s = warp_sum_f(dot[j]);
-    if (lane == 0) d_w[(size_t)t * k + j] = pos[j] >= 0 ? s : 0.0f;
+    if (lane == 0) part[warp][j] = s;
+  }
+  __syncthreads();
+  if ((int)threadIdx.x < tpb * k) {
+    const int tt = threadIdx.x / k, j = threadIdx.x - tt * k;
+    const int t2 = blockIdx.x * tpb + tt;
+    if (t2 < T) {
+      float s = 0.0f;
+      for (int q = 0; q < wpt; ++q) s += part[tt * wpt + q][j];
+      d_w[(size_t)t2 * k + j] = slot_pos[(size_t)t2 * k + j] >= 0 ? s : 0.0f;
+    }
   }
 }
 
@@ -100,33 +164,39 @@ struct RouteBwdArgs {
   float alpha, dL;
 };
 
-// One warp per token; shared memory holds the warp's E logits (then probabilities) and dp.
-template <typename Tin>
-__global__ void __launch_bounds__(256) route_backward_kernel(RouteBwdArgs a) {
-  extern __shared__ float rb_smem[];
-  griddep_wait();
-  griddep_launch();
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int t = blockIdx.x * 8 + warp;
-  if (t >= a.T) return;  // no block-wide barrier below
-  const int E = a.E, d = a.d, k = a.k;
-  float *pr = rb_smem + (size_t)warp * 2 * E, *dp = pr + E;
-  const Tin *xr = (const Tin *)a.x + (size_t)t * d;
-  // logits, one expert per pass (on the Quartz shape 49 us, against 86 us with 8 chains per pass)
-  for (int e = 0; e < E; ++e) {
-    const Tin *we = (const Tin *)a.w_router + (size_t)e * d;
-    float s = 0.0f;
-    for (int c = 4 * lane; c < d; c += 128) {
-      const float4 u = Bw4<Tin>::ld(xr + c), v = Bw4<Tin>::ld(we + c);
-      s = fmaf(u.x, v.x, s);
-      s = fmaf(u.y, v.y, s);
-      s = fmaf(u.z, v.z, s);
-      s = fmaf(u.w, v.w, s);
-    }
-    s = warp_sum_f(s);
-    if (lane == 0) pr[e] = a.off ? s + a.off[e] : s;
+// Logit tiling of route_backward: a block of 8 warps takes RB_TM tokens; lane = tg + 4 eg holds
+// tokens 4 tg .. 4 tg + 3 and experts 3 eg .. 3 eg + 2 of a round of 24 experts, warp w the
+// columns [w d / 8, (w + 1) d / 8) in chunks of eight. The warps' partial sums are added in warp
+// order.
+constexpr int RB_TM = 16;
+constexpr int RB_ROUND = 24;
+
+template <typename Tin> struct Ld8;  // eight consecutive inputs as fp32 (zeros when !ok)
+template <> struct Ld8<float> {
+  static __device__ __forceinline__ void ld(const float *p, bool ok, float (&v)[8]) {
+    float4 a = make_float4(0.f, 0.f, 0.f, 0.f), b = a;
+    if (ok) { a = __ldg((const float4 *)p); b = __ldg((const float4 *)p + 1); }
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
   }
-  __syncwarp();
+};
+template <> struct Ld8<__nv_bfloat16> {
+  static __device__ __forceinline__ void ld(const __nv_bfloat16 *p, bool ok, float (&v)[8]) {
+    const uint4 r = ok ? __ldg((const uint4 *)p) : make_uint4(0u, 0u, 0u, 0u);
+    Bw8<__nv_bfloat16>::unpack(r, v);
+  }
+};
+
+// Shared memory of route_backward_kernel (floats): the warps' partial sums of a round, the
+// block's logits (then probabilities) [RB_TM][E] and one dp row [E] per warp.
+__host__ __device__ constexpr size_t route_bwd_smem_floats(int E) {
+  return (size_t)8 * RB_TM * RB_ROUND + (size_t)RB_TM * E + (size_t)8 * E;
+}
+
+// Everything after the logits for token t, by one warp: probabilities, dp from d_topk_w, the
+// loss term and d_logits. pr holds the token's E logits (replaced by its probabilities).
+__device__ __forceinline__ void route_bwd_token(const RouteBwdArgs &a, int t, float *pr,
+                                                float *dp, int lane) {
+  const int E = a.E, k = a.k;
   float m = -INFINITY, ssum = 0.0f;
   if (!a.sigmoid) {
     for (int e = lane; e < E; e += 32) m = fmaxf(m, pr[e]);
@@ -177,6 +247,73 @@ __global__ void __launch_bounds__(256) route_backward_kernel(RouteBwdArgs a) {
       dl[e] = ds * pr[e] * (1.0f - pr[e]);
     }
   }
+  __syncwarp();
+}
+
+template <typename Tin>
+__global__ void __launch_bounds__(256) route_backward_kernel(RouteBwdArgs a) {
+  extern __shared__ float rb_smem[];
+  griddep_wait();
+  griddep_launch();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tg = lane & 3, eg = lane >> 2;
+  const int E = a.E, d = a.d;
+  const int t0 = blockIdx.x * RB_TM;
+  float *part = rb_smem;                          // [8][RB_TM][RB_ROUND]
+  float *lg = part + 8 * RB_TM * RB_ROUND;        // [RB_TM][E]
+  float *dpw = lg + (size_t)RB_TM * E;            // [8][E]
+  const int cs = d / 8;                           // columns per warp (a multiple of 8)
+  const int c0 = warp * cs;
+  const Tin *xb = (const Tin *)a.x, *wb = (const Tin *)a.w_router;
+  bool tok_ok[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) tok_ok[i] = t0 + 4 * tg + i < a.T;
+  for (int e0 = 0; e0 < E; e0 += RB_ROUND) {
+    float acc[4][3];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 3; ++j) acc[i][j] = 0.0f;
+    bool ex_ok[3];
+#pragma unroll
+    for (int j = 0; j < 3; ++j) ex_ok[j] = e0 + 3 * eg + j < E;
+    for (int c = c0; c < c0 + cs; c += 8) {
+      float xv[4][8], wv[3][8];
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        Ld8<Tin>::ld(xb + (size_t)(t0 + 4 * tg + i) * d + c, tok_ok[i], xv[i]);
+#pragma unroll
+      for (int j = 0; j < 3; ++j)
+        Ld8<Tin>::ld(wb + (size_t)(e0 + 3 * eg + j) * d + c, ex_ok[j], wv[j]);
+#pragma unroll
+      for (int q = 0; q < 8; ++q)
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+          for (int j = 0; j < 3; ++j) acc[i][j] = fmaf(xv[i][q], wv[j][q], acc[i][j]);
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 3; ++j)
+        part[(warp * RB_TM + 4 * tg + i) * RB_ROUND + 3 * eg + j] = acc[i][j];
+    __syncthreads();
+    for (int o = threadIdx.x; o < RB_TM * RB_ROUND; o += 256) {
+      const int tt = o / RB_ROUND, e = e0 + (o - tt * RB_ROUND);
+      if (e < E) {
+        float s = 0.0f;
+#pragma unroll
+        for (int w = 0; w < 8; ++w) s += part[w * RB_TM * RB_ROUND + o];
+        lg[(size_t)tt * E + e] = a.off ? s + a.off[e] : s;
+      }
+    }
+    __syncthreads();
+  }
+  // each warp finishes two of the block's tokens
+  for (int tt = warp; tt < RB_TM; tt += 8) {
+    const int t = t0 + tt;
+    if (t < a.T) route_bwd_token(a, t, lg + (size_t)tt * E, dpw + (size_t)warp * E, lane);
+  }
 }
 
 template <typename Tin> __device__ __forceinline__ float bw_elem(const Tin *p, size_t i);
@@ -185,31 +322,66 @@ template <> __device__ __forceinline__ float bw_elem<__nv_bfloat16>(const __nv_b
   return __bfloat162float(p[i]);
 }
 
-// d_w_router = d_logits^T x, split over the tokens: block (256 columns, 8 experts, split s)
-// sums tokens [s T / S, (s + 1) T / S) in order into part[s][e][c]; router_wgrad_sum adds the S
+// Two consecutive inputs as fp32.
+template <typename Tin> __device__ __forceinline__ float2 ld2(const Tin *p);
+template <> __device__ __forceinline__ float2 ld2<float>(const float *p) {
+  return __ldg((const float2 *)p);
+}
+template <> __device__ __forceinline__ float2 ld2<__nv_bfloat16>(const __nv_bfloat16 *p) {
+  const uint32_t u = __ldg((const unsigned int *)p);
+  return __bfloat1622float2(*(const __nv_bfloat162 *)&u);
+}
+
+// d_w_router = d_logits^T x, split over the tokens: block (512 columns, 8 experts, split s) sums
+// tokens [s T / S, (s + 1) T / S) in order into part[s][e][c], a thread two columns of eight
+// experts; the split's d_logits rows pass through shared memory 64 tokens at a time, and each
+// thread loads the x values of eight tokens before it uses them. router_wgrad_sum adds the S
 // partial sums in split order (S = 1 writes the result directly).
 template <typename Tin>
 __global__ void __launch_bounds__(256) router_wgrad_kernel(const float *__restrict__ dl,
                                                            const Tin *__restrict__ x, int T, int d,
                                                            int E, int S, float *__restrict__ part) {
+  __shared__ __align__(16) float g_s[64][8];
   griddep_wait();
   griddep_launch();
-  const int c = blockIdx.x * 256 + threadIdx.x, e0 = blockIdx.y * 8, s = blockIdx.z;
-  if (c >= d) return;
+  const int c = 2 * (blockIdx.x * 256 + threadIdx.x), e0 = blockIdx.y * 8, s = blockIdx.z;
   const int t0 = (int)((long long)T * s / S), t1 = (int)((long long)T * (s + 1) / S);
-  float acc[8];
+  float acc[8][2];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
-  for (int t = t0; t < t1; ++t) {
-    const float xv = bw_elem(x, (size_t)t * d + c);
-    const float *g = dl + (size_t)t * E + e0;
+  for (int i = 0; i < 8; ++i) acc[i][0] = acc[i][1] = 0.0f;
+  for (int tb = t0; tb < t1; tb += 64) {
+    const int n = min(64, t1 - tb);
+    __syncthreads();
+    for (int o = threadIdx.x; o < 64 * 8; o += 256) {
+      const int tt = o >> 3, i = o & 7;
+      g_s[tt][i] = (tt < n && e0 + i < E) ? dl[(size_t)(tb + tt) * E + e0 + i] : 0.0f;
+    }
+    __syncthreads();
+    if (c < d) {
+      for (int tt = 0; tt < n; tt += 8) {
+        float2 xv[8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i)
-      if (e0 + i < E) acc[i] = fmaf(g[i], xv, acc[i]);
+        for (int u = 0; u < 8; ++u)
+          xv[u] = tt + u < n ? ld2(x + (size_t)(tb + tt + u) * d + c) : make_float2(0.0f, 0.0f);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const float4 ga = *(const float4 *)&g_s[tt + u][0];
+          const float4 gb = *(const float4 *)&g_s[tt + u][4];
+          const float g[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            acc[i][0] = fmaf(g[i], xv[u].x, acc[i][0]);
+            acc[i][1] = fmaf(g[i], xv[u].y, acc[i][1]);
+          }
+        }
+      }
+    }
   }
+  if (c >= d) return;
 #pragma unroll
   for (int i = 0; i < 8; ++i)
-    if (e0 + i < E) part[((size_t)s * E + e0 + i) * d + c] = acc[i];
+    if (e0 + i < E)
+      *(float2 *)(part + ((size_t)s * E + e0 + i) * d + c) = make_float2(acc[i][0], acc[i][1]);
 }
 
 __global__ void __launch_bounds__(256) router_wgrad_sum_kernel(const float *__restrict__ part,
@@ -220,32 +392,66 @@ __global__ void __launch_bounds__(256) router_wgrad_sum_kernel(const float *__re
   const size_t i = (size_t)blockIdx.x * 256 + threadIdx.x, n = (size_t)E * d;
   if (i >= n) return;
   float acc = part[i];
-  for (int s = 1; s < S; ++s) acc += part[(size_t)s * n + i];
+  int s = 1;
+  for (; s + 8 <= S; s += 8) {  // eight loads in flight, added in split order
+    float v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) v[u] = part[(size_t)(s + u) * n + i];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) acc += v[u];
+  }
+  for (; s < S; ++s) acc += part[(size_t)s * n + i];
   dwr[i] = acc;
 }
 
-// dx[t, c..c+3] = sum over e (in order) of d_logits[t, e] W_r[e, c..c+3]; blocks stride over the
-// tokens.
+// dx[t, c..c+3] = sum over e (in order) of d_logits[t, e] W_r[e, c..c+3]: a block takes 16 tokens
+// at a time (blocks stride over the token blocks) and 1024 columns, a thread four columns of the
+// 16 tokens; the tokens' d_logits pass through shared memory (expert-major) 64 experts at a time.
 template <typename Tin>
 __global__ void __launch_bounds__(256) router_dgrad_kernel(const float *__restrict__ dl,
                                                            const Tin *__restrict__ wr, int T, int d,
                                                            int E, float *__restrict__ dx) {
+  __shared__ __align__(16) float g_s[64][16];
   griddep_wait();
   griddep_launch();
   const int c = 4 * (blockIdx.x * 256 + threadIdx.x);
-  if (c >= d) return;
-  for (int t = blockIdx.y; t < T; t += gridDim.y) {
-    float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-    const float *g = dl + (size_t)t * E;
-    for (int e = 0; e < E; ++e) {
-      const float ge = g[e];
-      const float4 v = Bw4<Tin>::ld(wr + (size_t)e * d + c);
-      acc.x = fmaf(ge, v.x, acc.x);
-      acc.y = fmaf(ge, v.y, acc.y);
-      acc.z = fmaf(ge, v.z, acc.z);
-      acc.w = fmaf(ge, v.w, acc.w);
+  for (int t0 = blockIdx.y * 16; t0 < T; t0 += gridDim.y * 16) {
+  float4 acc[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) acc[i] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+  for (int eb = 0; eb < E; eb += 64) {
+    const int n = min(64, E - eb);
+    __syncthreads();
+    for (int o = threadIdx.x; o < 64 * 16; o += 256) {
+      const int e = o >> 4, tt = o & 15;
+      g_s[e][tt] = (e < n && t0 + tt < T) ? dl[(size_t)(t0 + tt) * E + eb + e] : 0.0f;
     }
-    *(float4 *)(dx + (size_t)t * d + c) = acc;
+    __syncthreads();
+    if (c < d) {
+#pragma unroll 4
+      for (int e = 0; e < n; ++e) {
+        const float4 v = Bw4<Tin>::ld(wr + (size_t)(eb + e) * d + c);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float4 g = *(const float4 *)&g_s[e][4 * q];
+          const float gg[4] = {g.x, g.y, g.z, g.w};
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            float4 &r = acc[4 * q + u];
+            r.x = fmaf(gg[u], v.x, r.x);
+            r.y = fmaf(gg[u], v.y, r.y);
+            r.z = fmaf(gg[u], v.z, r.z);
+            r.w = fmaf(gg[u], v.w, r.w);
+          }
+        }
+      }
+    }
+  }
+  if (c < d) {
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+      if (t0 + i < T) *(float4 *)(dx + (size_t)(t0 + i) * d + c) = acc[i];
+  }
   }
 }
 
@@ -258,6 +464,9 @@ __global__ void __launch_bounds__(256) router_dgrad_kernel(const float *__restri
 // gradients (dh = dY W_d, dX = [dg | du] [W_g; W_u]) the same way.
 
 // koff[e] = sum over e' < e of the expert's row count rounded up to 64; koff[E] is the total.
+// kstart[e] = offsets[e+1] - (koff[e+1] - koff[e]): the row of the grouped activations at which
+// the expert's padded row range starts when it is aligned to the expert's last row (the rows
+// before offsets[e] belong to earlier experts, or lie before row 0).
 // korder: the experts by padded row count, largest first (ties: lower index first), the order in
 // which the weight-gradient products list their groups (each group's K is its row count, so
 // longest first balances the CTA pairs' round-robin share of the tiles).
@@ -267,6 +476,7 @@ __global__ void __launch_bounds__(256) router_dgrad_kernel(const float *__restri
 __global__ void __launch_bounds__(1024) pad_offsets_kernel(const int32_t *__restrict__ offsets,
                                                            int E, int32_t *__restrict__ koff,
                                                            int32_t *__restrict__ korder,
+                                                           int32_t *__restrict__ kstart,
                                                            int T, int nc, int ch,
                                                            int32_t *__restrict__ off_s,
                                                            int32_t *__restrict__ koff_s) {
@@ -282,6 +492,7 @@ __global__ void __launch_bounds__(1024) pad_offsets_kernel(const int32_t *__rest
   const int total = block_excl_scan_inplace(s, 1024, tmp);
   if (e < E) {
     koff[e] = s[e];
+    kstart[e] = offsets[e + 1] - sz[e];
     const int v = sz[e];
     int r = 0;
     for (int h = 0; h < E; ++h) r += (sz[h] > v || (sz[h] == v && h < e)) ? 1 : 0;

@@ -11,14 +11,18 @@ moe_status_t moe_combine_backward(const moe_config_t *cfg, const float *dy, cons
               tok16(cfg, dy_perm) && tok16(cfg, d_topk_w));
   if (cfg->T == 0) return MOE_OK;
   cudaStream_t st = (cudaStream_t)stream;
-  const dim3 grid(ceil_div(cfg->T, 8));
+  // tokens per block: as many as leave each token's 256-column slices a warp each (8 warps)
+  const int slices = ceil_div(cfg->d, 256);
+  int tpb = 8;
+  while (tpb > 1 && tpb * slices > 8) tpb >>= 1;
+  const dim3 grid(ceil_div(cfg->T, tpb));
   if (yperm_bf16(cfg))
     return launch_pdl(combine_backward_kernel<__nv_bfloat16>, grid, dim3(256), 0, st, dy,
                       (const __nv_bfloat16 *)y_perm, slot_pos, topk_w, (__nv_bfloat16 *)dy_perm,
-                      d_topk_w, cfg->T, cfg->top_k, cfg->d);
+                      d_topk_w, cfg->T, cfg->top_k, cfg->d, tpb);
   return launch_pdl(combine_backward_kernel<float>, grid, dim3(256), 0, st, dy,
                     (const float *)y_perm, slot_pos, topk_w, (float *)dy_perm, d_topk_w, cfg->T,
-                    cfg->top_k, cfg->d);
+                    cfg->top_k, cfg->d, tpb);
 }
 
 moe_status_t moe_route_backward(const moe_config_t *cfg, const void *x, const moe_weights_t *w,

@@ -88,11 +88,13 @@ struct GuFeed {
 // o[col..] (dg_hi), o + hf (du_hi), o + 2 hf (dg_lo), o + 3 hf (du_lo), o2 (h_hi), o2 + hf (h_lo),
 // 16 columns (32 bytes, one sector) per store. The caller has waited for the block pair; the
 // shared memory is released (the next pair may be issued) once g and u are in registers.
-// o, o2 and 2 hf bytes are multiples of 32 bytes.
+// o, o2 and 2 hf bytes are multiples of 32 bytes. A row past the group (!row_ok) stores nothing,
+// or zeros in all six outputs when zero_row is set (the padding rows of a padded layout).
 template <typename Issue>
 __device__ __forceinline__ void swiglu_bwd_chunk(const uint32_t (&r0)[32], const unsigned char *buf,
-                                                 int lane, bool row_ok, __nv_bfloat16 *o,
-                                                 __nv_bfloat16 *o2, int hf, Issue issue_next) {
+                                                 int lane, bool row_ok, bool zero_row,
+                                                 __nv_bfloat16 *o, __nv_bfloat16 *o2, int hf,
+                                                 Issue issue_next) {
   float4 gq[8], uq[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
@@ -104,7 +106,19 @@ __device__ __forceinline__ void swiglu_bwd_chunk(const uint32_t (&r0)[32], const
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   __syncwarp();
   issue_next();
-  if (!row_ok) return;
+  if (!row_ok) {
+    if (zero_row) {
+      const uint32_t z[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+#pragma unroll
+      for (int h16 = 0; h16 < 2; ++h16) {
+#pragma unroll
+        for (int s4 = 0; s4 < 4; ++s4) st_global_32B(o + s4 * hf + 16 * h16, z);
+        st_global_32B(o2 + 16 * h16, z);
+        st_global_32B(o2 + hf + 16 * h16, z);
+      }
+    }
+    return;
+  }
 #pragma unroll
   for (int h16 = 0; h16 < 2; ++h16) {
     uint32_t dgh[8], dgl[8], duh[8], dul[8], hh[8], hl[8];

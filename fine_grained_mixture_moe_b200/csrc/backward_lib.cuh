@@ -7,43 +7,46 @@
 template <typename Tin>
 moe_status_t route_backward_impl(const moe_config_t *c, const RouteBwdArgs &a, float *d_w_router,
                                  float *dx, cudaStream_t st) {
-  const size_t smem = (size_t)8 * 2 * c->E * sizeof(float);
+  const size_t smem = route_bwd_smem_floats(c->E) * sizeof(float);
   if (smem > 48 * 1024 &&
       cudaFuncSetAttribute(route_backward_kernel<Tin>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)smem) != cudaSuccess)
     return MOE_ERR_CUDA;
-  MOE_TRY(launch_pdl(route_backward_kernel<Tin>, dim3(ceil_div(c->T, 8)), dim3(256), smem, st, a));
-  // d_w_router over S token ranges; their partial sums [S, E, d] live in dx (T x d floats,
-  // S E <= T) until the last kernel writes dx
-  const int S = std::max(1, std::min(32, c->T / c->E));
+  MOE_TRY(launch_pdl(route_backward_kernel<Tin>, dim3(ceil_div(c->T, RB_TM)), dim3(256), smem, st,
+                     a));
+  // d_w_router over S token ranges (about two blocks per SM); their partial sums [S, E, d] live
+  // in dx (T x d floats, S E <= T) until the last kernel writes dx
+  const int per_split = ceil_div(c->d, 512) * ceil_div(c->E, 8);
+  const int S = std::max(1, std::min({64, c->T / c->E, ceil_div(2 * 148, per_split)}));
   float *part = S > 1 ? dx : d_w_router;
-  MOE_TRY(launch_pdl(router_wgrad_kernel<Tin>, dim3(ceil_div(c->d, 256), ceil_div(c->E, 8), S),
+  MOE_TRY(launch_pdl(router_wgrad_kernel<Tin>, dim3(ceil_div(c->d, 512), ceil_div(c->E, 8), S),
                      dim3(256), 0, st, (const float *)a.d_logits, (const Tin *)a.x, c->T, c->d,
                      c->E, S, part));
   if (S > 1)
     MOE_TRY(launch_pdl(router_wgrad_sum_kernel, dim3(ceil_div((long long)c->E * c->d, 256)),
                        dim3(256), 0, st, (const float *)part, S, c->E, c->d, d_w_router));
-  return launch_pdl(router_dgrad_kernel<Tin>, dim3(ceil_div(c->d, 1024), std::min(c->T, 65535)),
+  return launch_pdl(router_dgrad_kernel<Tin>, dim3(ceil_div(c->d, 1024), std::min(ceil_div(c->T, 16), 65535)),
                     dim3(256), 0, st, (const float *)a.d_logits, (const Tin *)a.w_router, c->T,
                     c->d, c->E, dx);
 }
 
 // ------------------------------------------------------------------ backward of the experts
-// Workspace of moe_expert_backward (bf16 SwiGLU layers): g and u recomputed (fp32), [dg | du]
-// and h as hi + lo bf16 terms, the routed dX before the un-permute, the shared experts'
-// counterparts, dy as hi + lo terms, the transposed weights and the transposed, per-expert
-// zero-padded activations of the weight gradients (2 or 3 K segments per group).
+// Workspace of moe_expert_backward (bf16 layers): g and u recomputed (fp32), [dg | du] and h as
+// hi + lo bf16 terms (routed rows at the padded positions koff, zero padding rows first), the routed dX
+// before the un-permute, the shared experts' counterparts, dy as hi + lo terms and the transposed
+// weights. The SwiGLU weight gradients read the activations in place (MN-major operands); the
+// low-rank ones still use transposed, per-expert zero-padded copies (2 or 3 K segments).
 constexpr int BWD_SHARED_CHUNKS = 8;
 
 struct BwdLayout {
-  size_t koff, korder, off_s, koff_s;
+  size_t koff, korder, kstart, off_s, koff_s;
   size_t gu, dgu, h, dxp, gu_s, dgu_s, h_s, dx_s, dy_b;
   size_t wdt, wgut, wsdt, wsgut;
-  size_t ydt, ht, dgut, xpt, ydt_s, ht_s, dgut_s, xt_s;
+  size_t ydt, xpt;
   size_t z, dzs, dys, dz2, zs2, ut, vt, dzt, zst, ds_part;  // low-rank experts
   size_t part_s;  // the shared experts' weight gradients per token chunk
   size_t total;
-  int npad, tpad;
+  int npad;
   int nc, ch;     // token chunks of the shared experts' weight gradients, rows per chunk
 };
 
@@ -58,17 +61,17 @@ BwdLayout bwd_layout(const moe_config_t *c) {
   // output tiles, long K) fill the GPU; the chunks' partial sums are added in chunk order
   L.nc = std::max(1, std::min(BWD_SHARED_CHUNKS, ceil_div((long long)T, 512)));
   L.ch = (int)(((size_t)ceil_div((long long)std::max<size_t>(T, 1), L.nc) + 63) & ~(size_t)63);
-  L.tpad = (int)(((T + 63) & ~(size_t)63) + 64 * (size_t)L.nc);
-  const size_t np = L.npad, tp = L.tpad;
+  const size_t np = L.npad;
   size_t o = 0;
   auto take = [&](size_t bytes) { size_t at = o; o = align256(o + std::max<size_t>(bytes, 1)); return at; };
   L.koff = take((E + 1) * 4);
   L.korder = take(E * 4);
+  L.kstart = take(E * 4);
   L.off_s = take((BWD_SHARED_CHUNKS + 1) * 4);
   L.koff_s = take((BWD_SHARED_CHUNKS + 1) * 4);
   L.gu = take(np * 2 * f * 4);  // blocked g, u: each group's rows padded to 64
-  L.dgu = take(N * 4 * f * 2);
-  L.h = take(N * 2 * f * 2);
+  L.dgu = take(np * 4 * f * 2);
+  L.h = take(np * 2 * f * 2);
   L.dxp = take(N * d * 4);
   L.gu_s = take(((T + 63) & ~(size_t)63) * 2 * sf * 4);
   L.dgu_s = take(T * 4 * sf * 2);
@@ -79,14 +82,8 @@ BwdLayout bwd_layout(const moe_config_t *c) {
   L.wgut = take(E * d * 2 * f * 2);
   L.wsdt = take(sf * d * 2);
   L.wsgut = take(d * 2 * sf * 2);
-  L.ydt = take(d * (swi ? 2 : 3) * np * 2);
-  L.ht = take(f * 2 * np * 2);
-  L.dgut = take(2 * f * 2 * np * 2);
-  L.xpt = take(d * 2 * np * 2);
-  L.ydt_s = take(sf ? d * 3 * tp * 2 : 0);
-  L.ht_s = take(sf * 3 * tp * 2);
-  L.dgut_s = take(2 * sf * 2 * tp * 2);
-  L.xt_s = take(sf ? d * 2 * tp * 2 : 0);
+  L.ydt = take(swi ? 0 : d * 3 * np * 2);
+  L.xpt = take(swi ? 0 : d * 2 * np * 2);
   L.z = take(N * r * 4);
   L.dzs = take(N * r * 4);
   L.dys = take(r ? N * 2 * d * 2 : 0);
@@ -146,6 +143,47 @@ moe_status_t launch_wgrad(int G, const int32_t *koff, const int32_t *order, int 
   return launch_tc2<MODE_PLAIN>(g, st, K_BWD_GEMM);
 }
 
+// One weight-gradient product with groups along K whose operands are read in place (MN-major):
+// out[g] (M x N, fp32, row-major) = sum over segments s < kseg of A[ra, col_a[s] + m] B[rb,
+// col_b[s] + n] over k < koff[g+1] - koff[g], ra = row_a[g] + k, rb = row_b[g] + k. A [rows_a,
+// lda] and B [rows_b, ldb] bf16 row-major; past a group's last row one of the two operands holds
+// zeros (a padded layout, or the end of the matrix).
+struct MnOperand {
+  const void *ptr;
+  int ld, rows;
+  const int32_t *row0;  // [G] device
+  int col[3];
+};
+moe_status_t launch_wgrad_mn(int G, const int32_t *koff, const int32_t *order, int kseg,
+                             const MnOperand &A, int M, const MnOperand &Bm, int N, float *out,
+                             cudaStream_t st) {
+  GroupedGemm g;
+  std::memset(&g, 0, sizeof(g));
+  g.kgroup = 1;
+  g.mn = 1;
+  g.koff = koff;
+  g.gorder = order;
+  g.kseg = kseg;
+  g.E = G;
+  g.A_r = A.ptr;
+  g.B0_r = Bm.ptr;
+  g.rows_r = M;
+  g.N_r = N;
+  g.mn_lda = A.ld;
+  g.mn_ldb = Bm.ld;
+  g.mn_rows_a = A.rows;
+  g.mn_rows_b = Bm.rows;
+  g.mn_row_a = A.row0;
+  g.mn_row_b = Bm.row0;
+  for (int s = 0; s < kseg; ++s) {
+    g.mn_col_a[s] = A.col[s];
+    g.mn_col_b[s] = Bm.col[s];
+  }
+  g.out_r = out;
+  g.ldo_r = N;
+  return launch_tc2<MODE_PLAIN>(g, st, K_BWD_GEMM);
+}
+
 moe_status_t expert_backward_impl(const moe_config_t *c, const void *x_perm,
                                   const int32_t *offsets, const int32_t *slot_pos, const void *x,
                                   const moe_weights_t *w, const void *dy_perm, const float *dy,
@@ -158,6 +196,7 @@ moe_status_t expert_backward_impl(const moe_config_t *c, const void *x_perm,
   const bool sh = S > 0;
   using bf = bf16_t;
   int32_t *koff = at<int32_t>(ws, L.koff), *korder = at<int32_t>(ws, L.korder),
+          *kstart = at<int32_t>(ws, L.kstart),
           *off_s = at<int32_t>(ws, L.off_s), *koff_s = at<int32_t>(ws, L.koff_s);
   float *GU = at<float>(ws, L.gu), *GUs = at<float>(ws, L.gu_s);
   bf *DGU = at<bf>(ws, L.dgu), *H = at<bf>(ws, L.h);
@@ -165,15 +204,13 @@ moe_status_t expert_backward_impl(const moe_config_t *c, const void *x_perm,
   bf *DGUs = at<bf>(ws, L.dgu_s), *Hs = at<bf>(ws, L.h_s), *dyb = at<bf>(ws, L.dy_b);
   bf *Wdt = at<bf>(ws, L.wdt), *Wgut = at<bf>(ws, L.wgut), *Wsdt = at<bf>(ws, L.wsdt),
      *Wsgut = at<bf>(ws, L.wsgut);
-  bf *Ydt = at<bf>(ws, L.ydt), *Ht = at<bf>(ws, L.ht), *DGUt = at<bf>(ws, L.dgut),
-     *Xpt = at<bf>(ws, L.xpt), *Ydts = at<bf>(ws, L.ydt_s), *Hts = at<bf>(ws, L.ht_s),
-     *DGUts = at<bf>(ws, L.dgut_s), *Xts = at<bf>(ws, L.xt_s);
-  const int np = L.npad, tp = L.tpad;
-  const bf *xp = (const bf *)x_perm, *xb = (const bf *)x;
+  bf *Ydt = at<bf>(ws, L.ydt), *Xpt = at<bf>(ws, L.xpt);
+  const int np = L.npad;
+  const bf *xp = (const bf *)x_perm;
 
   // padded group offsets of the weight gradients
-  MOE_TRY(launch_pdl(pad_offsets_kernel, dim3(1), dim3(1024), 0, st, offsets, E, koff, korder, T,
-                     L.nc, L.ch, off_s, koff_s));
+  MOE_TRY(launch_pdl(pad_offsets_kernel, dim3(1), dim3(1024), 0, st, offsets, E, koff, korder,
+                     kstart, T, L.nc, L.ch, off_s, koff_s));
   // the SwiGLU launches carry the routed SwiGLU experts (E groups) and / or the shared experts
   GroupedGemm base;
   std::memset(&base, 0, sizeof(base));
@@ -219,7 +256,7 @@ moe_status_t expert_backward_impl(const moe_config_t *c, const void *x_perm,
     if (swi) {
       g.A_r = dy_perm; g.lda_r = d; g.B0_r = Wdt; g.N_r = f; g.K_r = d;
       g.out_r = DGU; g.ldo_r = 4 * f; g.half_r = f; g.out2_r = H; g.ld2_r = 2 * f;
-      g.aux_r = GU; g.aux_row0 = koff;
+      g.aux_r = GU; g.aux_row0 = koff; g.pad_out = 1;
     }
     if (sh) {  // A = [dy_hi | dy_lo], K = 2d, the weight's k wraps over its d columns
       g.A_s = dyb; g.lda_s = 2 * d; g.B0_s = Wsdt; g.N_s = sf; g.K_s = 2 * d; g.piece_k = d;
@@ -235,6 +272,7 @@ moe_status_t expert_backward_impl(const moe_config_t *c, const void *x_perm,
     if (swi) {
       g.A_r = DGU; g.lda_r = 4 * f; g.B0_r = Wgut; g.N_r = d; g.K_r = 4 * f; g.kb_r = 2 * f;
       g.out_r = dXp; g.ldo_r = d; g.out_r_bf16 = 0;
+      g.a_row_end = koff; g.rows_r = np;  // [dg | du] rows at the padded positions
     }
     if (sh) {
       g.A_s = DGUs; g.lda_s = 4 * sf; g.B0_s = Wsgut; g.N_s = d; g.K_s = 4 * sf;
@@ -302,46 +340,44 @@ moe_status_t expert_backward_impl(const moe_config_t *c, const void *x_perm,
                      slot_pos, (const float *)nullptr, dx, T, k, d, false));
   if (swi) {
     // weight gradients: one operand as hi + lo segments, the other repeated, so that each
-    // product sums both terms: dW_d = dY^T (h_hi + h_lo), dW_g = (dg_hi + dg_lo)^T X, dW_u
-    const bf *dyp = (const bf *)dy_perm;
-    const int nb2 = 2 * np / 64;
-    MOE_TRY(launch_transpose_grouped(2, dyp, dyp, nullptr, d, d, offsets, koff, E, nb2, Ydt, 2 * np, st));
-    MOE_TRY(launch_transpose_grouped(2, H, H + f, nullptr, f, 2 * f, offsets, koff, E, nb2, Ht, 2 * np, st));
-    MOE_TRY(launch_transpose_grouped(2, DGU, DGU + 2 * f, nullptr, 2 * f, 4 * f, offsets, koff, E,
-                                     nb2, DGUt, 2 * np, st));
-    MOE_TRY(launch_transpose_grouped(2, xp, xp, nullptr, d, d, offsets, koff, E, nb2, Xpt, 2 * np, st));
-    MOE_TRY(launch_wgrad(E, koff, korder, 2, Ydt, d, Ht, f, 2 * np, gr->d_w_down, st));
-    MOE_TRY(launch_wgrad(E, koff, korder, 2, DGUt, f, Xpt, d, 2 * np, gr->d_w_gate, st));
-    MOE_TRY(launch_wgrad(E, koff, korder, 2, DGUt + (size_t)f * 2 * np, f, Xpt, d, 2 * np, gr->d_w_up, st));
+    // product sums both terms: dW_d = dY^T (h_hi + h_lo), dW_g = (dg_hi + dg_lo)^T X, dW_u.
+    // h and [dg | du] rows from koff (zeros first, then the group's rows); dY and X rows from
+    // kstart, so that the group's rows meet its rows and the rows before them meet zeros
+    // (the rows past the last kept pair, which no kernel writes, are never read).
+    const int N = T * k;
+    const MnOperand dyo{dy_perm, d, N, kstart, {0, 0, 0}};
+    const MnOperand ho{H, 2 * f, np, koff, {0, f, 0}};
+    const MnOperand xo{x_perm, d, N, kstart, {0, 0, 0}};
+    const MnOperand dgo{DGU, 4 * f, np, koff, {0, 2 * f, 0}};
+    const MnOperand duo{DGU, 4 * f, np, koff, {f, 3 * f, 0}};
+    MOE_TRY(launch_wgrad_mn(E, koff, korder, 2, dyo, d, ho, f, gr->d_w_down, st));
+    MOE_TRY(launch_wgrad_mn(E, koff, korder, 2, dgo, f, xo, d, gr->d_w_gate, st));
+    MOE_TRY(launch_wgrad_mn(E, koff, korder, 2, duo, f, xo, d, gr->d_w_up, st));
     MOE_TRY(launch_pdl(zero_empty_experts_kernel, dim3(E, 8), dim3(256), 0, st, offsets,
                        gr->d_w_gate, (size_t)f * d, gr->d_w_up, (size_t)f * d, gr->d_w_down,
                        (size_t)d * f));
   }
   if (sh) {
     // dW_sg, dW_su: (dg_hi + dg_lo)^T x; dW_sd: (dy_hi + dy_lo)^T (h_hi + h_lo) less lo lo,
-    // three segments [hi hi | hi lo | lo hi]; each over the nc token chunks, then the chunks'
-    // partial sums added in order
+    // three segments [hi hi | hi lo | lo hi]; each over the nc token chunks (64-aligned; rows
+    // past T read as zeros), then the chunks' partial sums added in order
     const int nc = L.nc;
     float *part = at<float>(ws, L.part_s);
     auto sum_chunks = [&](size_t n, float *out) {
       return launch_pdl(sum_chunks_kernel, dim3((unsigned)std::min<long long>(ceil_div((long long)n, 1024), 4096)),
                         dim3(256), 0, st, (const float *)part, nc, n, out);
     };
-    MOE_TRY(launch_transpose_grouped(2, DGUs, DGUs + 2 * sf, nullptr, 2 * sf, 4 * sf, off_s,
-                                     koff_s, nc, 2 * tp / 64, DGUts, 2 * tp, st));
-    MOE_TRY(launch_transpose_grouped(2, xb, xb, nullptr, d, d, off_s, koff_s, nc, 2 * tp / 64, Xts,
-                                     2 * tp, st));
-    MOE_TRY(launch_transpose_grouped(3, dyb, dyb, dyb + d, d, 2 * d, off_s, koff_s, nc,
-                                     3 * tp / 64, Ydts, 3 * tp, st));
-    MOE_TRY(launch_transpose_grouped(3, Hs, Hs + sf, Hs, sf, 2 * sf, off_s, koff_s, nc,
-                                     3 * tp / 64, Hts, 3 * tp, st));
-    MOE_TRY(launch_wgrad(nc, koff_s, nullptr, 2, DGUts, sf, Xts, d, 2 * tp, part, st));
+    const MnOperand xo{x, d, T, off_s, {0, 0, 0}};
+    const MnOperand dgo{DGUs, 4 * sf, T, off_s, {0, 2 * sf, 0}};
+    const MnOperand duo{DGUs, 4 * sf, T, off_s, {sf, 3 * sf, 0}};
+    const MnOperand dyo{dyb, 2 * d, T, off_s, {0, 0, d}};
+    MOE_TRY(launch_wgrad_mn(nc, koff_s, nullptr, 2, dgo, sf, xo, d, part, st));
     MOE_TRY(sum_chunks((size_t)sf * d, gr->d_ws_gate));
-    MOE_TRY(launch_wgrad(nc, koff_s, nullptr, 2, DGUts + (size_t)sf * 2 * tp, sf, Xts, d, 2 * tp, part, st));
+    MOE_TRY(launch_wgrad_mn(nc, koff_s, nullptr, 2, duo, sf, xo, d, part, st));
     MOE_TRY(sum_chunks((size_t)sf * d, gr->d_ws_up));
     for (int s = 0; s < S; ++s) {
-      MOE_TRY(launch_wgrad(nc, koff_s, nullptr, 3, Ydts, d, Hts + (size_t)s * fs * 3 * tp, fs, 3 * tp, part,
-                           st));
+      const MnOperand ho{Hs, 2 * sf, T, off_s, {s * fs, sf + s * fs, s * fs}};
+      MOE_TRY(launch_wgrad_mn(nc, koff_s, nullptr, 3, dyo, d, ho, fs, part, st));
       MOE_TRY(sum_chunks((size_t)d * fs, gr->d_ws_down + (size_t)s * d * fs));
     }
   }

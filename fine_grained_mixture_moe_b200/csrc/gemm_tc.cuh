@@ -117,6 +117,19 @@ __device__ __forceinline__ uint64_t make_sdesc(uint32_t saddr) {
   d |= (uint64_t)2 << 61;             // SWIZZLE_128B
   return d;
 }
+// The same for an MN-major operand (rows of the tile are K): 64 M (or N) elements per 128-byte
+// row, K rows in 8-row groups of 1024 bytes (stride byte offset), and the next 64 elements of M
+// `lbo` bytes further (leading byte offset).
+__device__ __forceinline__ uint64_t make_sdesc_mn(uint32_t saddr, uint32_t lbo) {
+  uint64_t d = (uint64_t)((saddr & 0x3FFFFu) >> 4);
+  d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;  // leading byte offset: the next 64 of M / N
+  d |= (uint64_t)(1024 >> 4) << 32;             // stride byte offset: the next 8 rows of K
+  d |= (uint64_t)1 << 46;                       // descriptor version (sm_100)
+  d |= (uint64_t)2 << 61;                       // SWIZZLE_128B
+  return d;
+}
+// Instruction-descriptor bits of MN-major A and B (kind::f16).
+constexpr uint32_t IDESC_MN_MAJOR = (1u << 15) | (1u << 16);
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,"

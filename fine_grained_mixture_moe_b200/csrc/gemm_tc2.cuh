@@ -218,8 +218,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TC_THREADS, 1)
         const uint32_t stage_tx = KPB * (2 * C::STAGE_BYTES - (a1_void ? C::A_BYTES : 0));
         const int n_off = tc2_two_b(MODE) ? 0 : (int)rank * 128;
         // with two K-blocks per stage an odd count leaves the last stage half used: its second
-        // tile (the next group's columns, or the map's zero fill) is loaded and not multiplied
-        const int nk = (ti.K + C::BK - 1) / C::BK;
+        // tile (the next group's columns, or the map's zero fill) is loaded and not multiplied.
+        // MN-major: each segment's nbg K-blocks start a stage (nbg rounded up to KPB)
+        const int nbg = p.mn ? ti.K / (p.kseg * C::BK) : 0;
+        const int nbg_pad = (nbg + KPB - 1) / KPB * KPB;
+        const int nk = p.mn ? p.kseg * nbg_pad : (ti.K + C::BK - 1) / C::BK;
         for (int kb = 0; kb < nk; kb += KPB) {
           if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, limit, INFO_WAIT_MMA_EMPTY)) {
             ok = false;
@@ -241,7 +244,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TC_THREADS, 1)
             b_row = piece * p.piece_rows + ti.n0 + n_off;
             b_col = kk - piece * p.piece_k;
           }
-          if (KPB == 2) {  // boxes of two K-blocks: coordinates {column, row, K-block}
+          if (p.mn) {  // MN-major: 64 KPB rows of K, two 64-column blocks of M (N) per operand
+            const int seg = kb / nbg_pad, j0 = kb - seg * nbg_pad;
+            const int acb = (ti.m0 + (int)rank * 128 + p.mn_col_a[seg]) >> 6;
+            const int bcb = (ti.n0 + n_off + p.mn_col_b[seg]) >> 6;
+            if (rank == 0 || !a1_void)
+              tma_load_3d_pair(sA, ma, 0, p.mn_row_a[ti.g] + j0 * C::BK, acb, full_bar(stage));
+            tma_load_3d_pair(sB, mb, 0, p.mn_row_b[ti.g] + j0 * C::BK, bcb, full_bar(stage));
+          } else if (KPB == 2) {  // boxes of two K-blocks: coordinates {column, row, K-block}
             if (rank == 0 || !a1_void)
               tma_load_3d_pair(sA, ma, 0, a_row, (ti.kofs + kk) / C::BK, full_bar(stage));
             tma_load_3d_pair(sB, mb, 0, b_row, b_col / C::BK, full_bar(stage));
@@ -273,7 +283,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TC_THREADS, 1)
       bool ok = true, any = false;
       for (int tile = pair; tile < total && ok; tile += npairs) {
         const TileInfo ti = decode_tile(p, tile, prefix, TC2_BM, BN);
-        const int nk = (ti.K + C::BK - 1) / C::BK;
+        const int nbg = p.mn ? ti.K / (p.kseg * C::BK) : 0;  // as in the producer
+        const int nbg_pad = (nbg + KPB - 1) / KPB * KPB;
+        const int nk = p.mn ? p.kseg * nbg_pad : (ti.K + C::BK - 1) / C::BK;
         if (!mbar_wait(acce_bar(acc), acc_phase ^ 1u, abort_flag, limit, INFO_WAIT_ACC_EMPTY)) {
           ok = false;
           break;
@@ -288,8 +300,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TC_THREADS, 1)
           tc_fence_after();
           const uint32_t sA0 = smem_u32(stages + (size_t)stage * stage_bytes);
           const uint32_t sB0 = sA0 + C::A_BYTES * KPB;
-          for (int j = 0; j < KPB && kb + j < nk; ++j) {  // the stage's K-blocks, 16 KB tiles
+          const int j0 = p.mn ? kb % nbg_pad : 0;  // MN-major: first K-block of the segment
+          for (int j = 0; j < KPB && (p.mn ? j0 + j < nbg : kb + j < nk); ++j) {
             const uint32_t sA = sA0 + j * C::A_BYTES, sB = sB0 + j * C::B_BYTES;
+            if (!mode_fp8(MODE) && p.mn) {
+              // each operand: two 64-column blocks of 64 KPB rows; K-block j at 64 j rows, 16
+              // rows of K (2 KB) per instruction
+              const uint32_t lbo = 8192u * KPB;
+#pragma unroll
+              for (int k16 = 0; k16 < 4; ++k16)
+                tc2_mma(d0, make_sdesc_mn(sA0 + j * 8192 + k16 * 2048, lbo),
+                        make_sdesc_mn(sB0 + j * 8192 + k16 * 2048, lbo), C::IDESC | IDESC_MN_MAJOR,
+                        (kb > 0 || j > 0 || k16 > 0) ? 1u : 0u);
+              continue;
+            }
 #pragma unroll
             for (int k16 = 0; k16 < 4; ++k16) {  // 32 bytes of K per instruction
               const uint32_t accum = (kb > 0 || j > 0 || k16 > 0) ? 1u : 0u;
@@ -332,8 +356,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TC_THREADS, 1)
       const int rbase = ti.m0 + (int)rank * 128 + q * 32;  // first row of this warp's block
       const int row = rbase + lane;
       const bool row_ok = row < ti.rows;
+      // SWIGLU_BWD with padded outputs: the group's rows up to the next multiple of 64 are
+      // written, row i < rows at aux_row0[g+1] - rows + i and the padding ones (as zeros) in
+      // front of them
+      const bool pad = MODE == MODE_SWIGLU_BWD && p.pad_out && routed;
+      const int rows_w = pad ? ((ti.rows + 63) & ~63) : ti.rows;
       // a warp of padding rows only, or columns past the group's width: nothing to store
-      const int cstop = rbase < ti.rows ? min(cend, ti.N - ti.n0) : cbeg;
+      const int cstop = rbase < rows_w ? min(cend, ti.N - ti.n0) : cbeg;
       if (MODE == MODE_SWIGLU_BWD && cstop > cbeg)
         feed.issue(gu_pair_block(p, ti, routed, routed ? p.aux_r : p.aux_s, rbase, ti.n0 + cbeg),
                    lane);
@@ -367,11 +396,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TC_THREADS, 1)
           tmem_ld32(tbase + c, r0);
           tmem_wait_ld();
           if (!feed.wait(abort_flag, limit)) { ok = false; break; }
-          const size_t arow = (size_t)(ti.out_row0 + row);
+          const size_t arow = pad ? (size_t)(p.aux_row0[ti.g] + (row_ok ? row + rows_w - ti.rows
+                                                                         : row - ti.rows))
+                                  : (size_t)(ti.out_row0 + row);
           __nv_bfloat16 *o = (__nv_bfloat16 *)out + arow * ldo + col;
           __nv_bfloat16 *o2 = (__nv_bfloat16 *)(routed ? p.out2_r : p.out2_s) +
                               arow * (routed ? p.ld2_r : p.ld2_s) + col;
-          swiglu_bwd_chunk(r0, stg, lane, row_ok, o, o2, hf, [&] {
+          swiglu_bwd_chunk(r0, stg, lane, row_ok, !row_ok && row < rows_w, o, o2, hf, [&] {
             if (c + 32 < cstop)
               feed.issue(gu_pair_block(p, ti, routed, routed ? p.aux_r : p.aux_s, rbase, col + 32),
                          lane);

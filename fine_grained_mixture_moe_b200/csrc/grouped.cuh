@@ -29,7 +29,8 @@
 // Groups along K (kgroup, backward weight gradients): group g is out rows [g M, g M + M) =
 // A[M, K_g] B[N, K_g]^T, where A and B are K-major [M or N][ld] and group g takes their columns
 // kseg koff[g] .. kseg koff[g+1] (koff padded to multiples of 64; kseg segments per group, so a
-// sum of split terms runs as one product); M is rows_r and ld is K_r.
+// sum of split terms runs as one product); M is rows_r and ld is K_r. With mn set, A and B are
+// instead read MN-major from the row-major activations themselves (fields below).
 // Output types in the tensor-core kernels: GATEUP and SCALE write bf16 (the next product's
 // operand, SCALE optionally as a hi + lo pair) or, with out_f32, fp32; PLAIN writes the routed
 // groups' rows in bf16 or fp32 (out_r_bf16) and the shared group's rows in fp32.
@@ -91,6 +92,23 @@ struct GroupedGemm {
   int kseg;                // K segments per group (kgroup)
   const int32_t *gorder;   // kgroup: [E] device, the group at each position of the tile list
                            // (longest K first); null: group order
+  // kgroup with MN-major operands (mn != 0): A and B are row-major [rows, ld] matrices whose
+  // rows are K; group g takes rows mn_row_a[g] + k of A and mn_row_b[g] + k of B for k < its
+  // padded row count (koff[g+1] - koff[g]), once per segment s < kseg, segment s reading the
+  // columns mn_col_a[s] + m of A and mn_col_b[s] + n of B (multiples of 64). The leading rows
+  // beyond a group's own are zeros in one operand (the padded layout below) and, in the other,
+  // rows of earlier groups or rows before row 0 (which the tensor map reads as zeros).
+  int mn;
+  const int32_t *mn_row_a, *mn_row_b;  // [E] device
+  int mn_col_a[3], mn_col_b[3];
+  int mn_lda, mn_ldb;                  // row lengths (elements)
+  int mn_rows_a, mn_rows_b;            // row extents of the tensor maps
+  // routed rows at padded positions, padding first: group g owns rows [aux_row0[g],
+  // aux_row0[g+1]) (its row count rounded up to 64), zeros in the leading ones and its rows in
+  // the trailing ones. SWIGLU_BWD (pad_out) writes out and out2 that way; a_row_end (non-null,
+  // [E+1]) makes group g's A rows start at a_row_end[g+1] - rows (out rows stay at offsets[g])
+  int pad_out;
+  const int32_t *a_row_end;
 };
 
 // Tile list order: the shared group (its K may be several experts' widths: the longest tiles)
@@ -161,13 +179,14 @@ __device__ __forceinline__ TileInfo decode_tile(const GroupedGemm &p, int tile,
     return ti;
   }
   if (routed) {
-    ti.a_row0 = p.offsets[lo];
-    ti.rows = p.offsets[lo + 1] - ti.a_row0;
+    ti.out_row0 = p.offsets[lo];
+    ti.rows = p.offsets[lo + 1] - ti.out_row0;
+    ti.a_row0 = p.a_row_end ? p.a_row_end[lo + 1] - ti.rows : ti.out_row0;
   } else {
     ti.a_row0 = 0;
     ti.rows = p.T;
+    ti.out_row0 = 0;
   }
-  ti.out_row0 = ti.a_row0;
   return ti;
 }
 

@@ -316,6 +316,23 @@ bool make_map3(CUtensorMap *m, const void *ptr, uint64_t rows, uint64_t cols, ui
   return r == CUDA_SUCCESS;
 }
 
+// MN-major operand: the same 3-D view of a row-major [rows, cols] matrix (cols a multiple of
+// 64), box {64, box_rows, 2}: box_rows rows (K) of two consecutive 64-column blocks (M or N),
+// block after block; rows before 0 or past the end read as zeros.
+bool make_map_mn(CUtensorMap *m, const void *ptr, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  if (rows == 0 || ptr == nullptr) rows = 1;
+  cuuint64_t dims[3] = {64, rows, cols / 64};
+  cuuint64_t strides[2] = {cols * 2, 128};
+  cuuint32_t box[3] = {64, box_rows, 2};
+  cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr), dims,
+                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 // ------------------------------------------------------------------ grouped GEMM launches
 long long tile_bound(const GroupedGemm &g, int BM, int BN) {
   if (g.kgroup) return (long long)g.E * ceil_div(g.rows_r, BM) * ceil_div(g.N_r, BN);
@@ -330,6 +347,15 @@ long long tile_bound(const GroupedGemm &g, int BM, int BN) {
 bool build_maps(const GroupedGemm &g, bool two_b, uint32_t b_box, TcMaps *m, int esz = 2,
                 bool kb2 = false) {
   const void *any = g.E > 0 ? g.A_r : g.A_s;
+  if (g.mn) {  // groups along K, both operands MN-major (the other maps are unused)
+    const uint32_t box_rows = kb2 ? 128 : 64;
+    bool ok = make_map_mn(&m->a_r, g.A_r, g.mn_rows_a, g.mn_lda, box_rows);
+    ok &= make_map_mn(&m->b0_r, g.B0_r, g.mn_rows_b, g.mn_ldb, box_rows);
+    m->b1_r = m->b0_r;
+    m->a_s = m->a_r;
+    m->b0_s = m->b1_s = m->b0_r;
+    return ok;
+  }
   if (kb2) {  // bf16; the same extents as the 2-D maps below
     const int kb = g.kb_r ? g.kb_r : g.K_r;
     const uint64_t b_rows = g.kgroup ? (uint64_t)g.N_r : (uint64_t)g.E * g.N_r;
@@ -395,8 +421,11 @@ moe_status_t launch_tc2(const GroupedGemm &g, cudaStream_t st, int kind) {
   const int G = g.E + g.has_shared;
   // two K-blocks per stage (3-D boxes) for the bf16 products, when no stage can cross a wrap
   // point of B's columns or a shared-expert piece, and the ring keeps at least 2 stages of 2
-  const bool kb2 = !mode_fp8(MODE) && (g.kb_r == 0 || g.kb_r % 128 == 0) &&
-                   (!g.has_shared || g.piece_k % 128 == 0) && tc2_stages<MODE>(G, 2) >= 2;
+  // (MN-major operands: every segment's K-blocks start a stage, so no stage crosses one)
+  const bool kb2 = !mode_fp8(MODE) && tc2_stages<MODE>(G, 2) >= 2 &&
+                   (g.mn || ((g.kb_r == 0 || g.kb_r % 128 == 0) &&
+                             (!g.has_shared || g.piece_k % 128 == 0)));
+  if (g.mn && (mode_fp8(MODE) || !g.kgroup || g.kseg < 1 || g.kseg > 3)) return MOE_ERR_UNSUPPORTED;
   P.kpb = kb2 ? 2 : 1;
   if (!build_maps(g, tc2_two_b(MODE), 128, &P.maps, mode_fp8(MODE) ? 1 : 2, kb2)) return MOE_ERR_CUDA;
   static_assert(tc2_stages<MODE>(1024 + 1) >= 2, "tile list of 1024 experts leaves no room");

@@ -236,6 +236,10 @@ size_t moe_backward_workspace_size(const moe_config_t *cfg);
  * rounding residual, so each gradient carries no single bf16 rounding of its operands.
  * Supported: bf16 layers (SwiGLU or low-rank experts); fp32 layers and layers whose experts are
  * stored in fp8 (training stays bf16) return MOE_ERR_UNSUPPORTED.
+ * SwiGLU weight gradients read x_perm and dy_perm in place, in 64-row blocks aligned to each
+ * expert's last row: up to 63 rows before an expert's first row (earlier experts' rows) are
+ * multiplied by zeros, so rows of x_perm and dy_perm past offsets[E] are never read, but a
+ * non-finite value in one expert's rows can make the next expert's weight gradients non-finite.
  * ws: moe_backward_workspace_size(cfg) bytes of the caller's device memory. Asynchronous. */
 moe_status_t moe_expert_backward(const moe_config_t *cfg, const void *x_perm,
                                  const int32_t *offsets, const int32_t *slot_pos, const void *x,
