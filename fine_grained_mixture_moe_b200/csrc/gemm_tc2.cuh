@@ -220,9 +220,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TC_THREADS, 1)
         // with two K-blocks per stage an odd count leaves the last stage half used: its second
         // tile (the next group's columns, or the map's zero fill) is loaded and not multiplied.
         // MN-major: each segment's nbg K-blocks start a stage (nbg rounded up to KPB)
-        const int nbg = p.mn ? ti.K / (p.kseg * C::BK) : 0;
-        const int nbg_pad = (nbg + KPB - 1) / KPB * KPB;
-        const int nk = p.mn ? p.kseg * nbg_pad : (ti.K + C::BK - 1) / C::BK;
+        int nbg_pad = 0, nk;
+        if (p.mn) {
+          nbg_pad = (ti.K / (p.kseg * C::BK) + KPB - 1) / KPB * KPB;
+          nk = p.kseg * nbg_pad;
+        } else {
+          nk = (ti.K + C::BK - 1) / C::BK;
+        }
         for (int kb = 0; kb < nk; kb += KPB) {
           if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, limit, INFO_WAIT_MMA_EMPTY)) {
             ok = false;
@@ -283,9 +287,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TC_THREADS, 1)
       bool ok = true, any = false;
       for (int tile = pair; tile < total && ok; tile += npairs) {
         const TileInfo ti = decode_tile(p, tile, prefix, TC2_BM, BN);
-        const int nbg = p.mn ? ti.K / (p.kseg * C::BK) : 0;  // as in the producer
-        const int nbg_pad = (nbg + KPB - 1) / KPB * KPB;
-        const int nk = p.mn ? p.kseg * nbg_pad : (ti.K + C::BK - 1) / C::BK;
+        int nbg = 0, nbg_pad = 0, nk;  // as in the producer
+        if (p.mn) {
+          nbg = ti.K / (p.kseg * C::BK);
+          nbg_pad = (nbg + KPB - 1) / KPB * KPB;
+          nk = p.kseg * nbg_pad;
+        } else {
+          nk = (ti.K + C::BK - 1) / C::BK;
+        }
         if (!mbar_wait(acce_bar(acc), acc_phase ^ 1u, abort_flag, limit, INFO_WAIT_ACC_EMPTY)) {
           ok = false;
           break;
@@ -300,27 +309,30 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(TC_THREADS, 1)
           tc_fence_after();
           const uint32_t sA0 = smem_u32(stages + (size_t)stage * stage_bytes);
           const uint32_t sB0 = sA0 + C::A_BYTES * KPB;
-          const int j0 = p.mn ? kb % nbg_pad : 0;  // MN-major: first K-block of the segment
-          for (int j = 0; j < KPB && (p.mn ? j0 + j < nbg : kb + j < nk); ++j) {
-            const uint32_t sA = sA0 + j * C::A_BYTES, sB = sB0 + j * C::B_BYTES;
-            if (!mode_fp8(MODE) && p.mn) {
-              // each operand: two 64-column blocks of 64 KPB rows; K-block j at 64 j rows, 16
-              // rows of K (2 KB) per instruction
-              const uint32_t lbo = 8192u * KPB;
+          if (!mode_fp8(MODE) && p.mn) {
+            // MN-major: each operand two 64-column blocks of 64 KPB rows; the stage's K-blocks
+            // that lie in the segment (nbg >= 1 for every listed tile), 16 rows of K (2 KB)
+            // per instruction
+            const int j0 = kb % nbg_pad;
+            const uint32_t lbo = 8192u * KPB;
+            for (int j = 0; j < KPB && j0 + j < nbg; ++j) {
 #pragma unroll
               for (int k16 = 0; k16 < 4; ++k16)
                 tc2_mma(d0, make_sdesc_mn(sA0 + j * 8192 + k16 * 2048, lbo),
                         make_sdesc_mn(sB0 + j * 8192 + k16 * 2048, lbo), C::IDESC | IDESC_MN_MAJOR,
                         (kb > 0 || j > 0 || k16 > 0) ? 1u : 0u);
-              continue;
             }
+          } else {
+            for (int j = 0; j < KPB && kb + j < nk; ++j) {  // the stage's K-blocks, 16 KB tiles
+              const uint32_t sA = sA0 + j * C::A_BYTES, sB = sB0 + j * C::B_BYTES;
 #pragma unroll
-            for (int k16 = 0; k16 < 4; ++k16) {  // 32 bytes of K per instruction
-              const uint32_t accum = (kb > 0 || j > 0 || k16 > 0) ? 1u : 0u;
-              if (mode_fp8(MODE))
-                tc2_mma_f8(d0, make_sdesc(sA + k16 * 32), make_sdesc(sB + k16 * 32), C::IDESC, accum);
-              else
-                tc2_mma(d0, make_sdesc(sA + k16 * 32), make_sdesc(sB + k16 * 32), C::IDESC, accum);
+              for (int k16 = 0; k16 < 4; ++k16) {  // 32 bytes of K per instruction
+                const uint32_t accum = (kb > 0 || j > 0 || k16 > 0) ? 1u : 0u;
+                if (mode_fp8(MODE))
+                  tc2_mma_f8(d0, make_sdesc(sA + k16 * 32), make_sdesc(sB + k16 * 32), C::IDESC, accum);
+                else
+                  tc2_mma(d0, make_sdesc(sA + k16 * 32), make_sdesc(sB + k16 * 32), C::IDESC, accum);
+              }
             }
           }
           any = true;
