@@ -407,6 +407,46 @@ def test_expert_backward(name):
     assert torch.equal(dx, dx1) and all(torch.equal(grads[n], first[n]) for n in grads)
 
 
+@pytest.mark.parametrize("name", ["capacity_s", "heavy_drops"])
+def test_expert_backward_never_reads_rows_past_the_kept_pairs(name):
+    """Under a capacity limit x_perm and dy_perm hold rows past offsets[E] that no kernel
+    writes. The weight gradients read both in place in 64-row blocks aligned to each expert's
+    last row, so those rows must never be read: with NaN planted there, every output stays
+    finite and within the tolerance of the oracle's expert step."""
+    c = SMALL[name] if name in SMALL else EDGE[name]
+    inp = make_inputs(c)
+    run = LayerOnGpu(c, inp)
+    o = run.steps()
+    T, d, k = run.cfg.T, run.cfg.d, run.cfg.top_k
+    dev = run.dev
+    N = int(o["offsets"][-1])
+    assert N < T * k, "the configuration drops no pair"
+    dy = np.random.default_rng(13).standard_normal((T, d)).astype(np.float32)
+    dy_t = torch.as_tensor(dy).to(dev)
+    dyp = torch.empty_like(o["y_perm"])
+    d_w = torch.empty((T, k), dtype=torch.float32, device=dev)
+    B.moe_combine_backward(run.cfg, dy_t, o["y_perm"], o["slot_pos"], o["w"], dyp, d_w)
+    xp = o["x_perm"].clone()
+    xp[N:] = float("nan")
+    dyp[N:] = float("nan")
+    grads = _expert_grads(c, run)
+    ws_bytes = B.moe_backward_workspace_size(run.cfg)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    dx = torch.empty((T, d), dtype=torch.float32, device=dev)
+    B.moe_expert_backward(run.cfg, xp, o["offsets"], o["slot_pos"], run.x, run.ws_struct, dyp,
+                          dy_t if c.n_shared else None, dx, B.make_grads(grads), ws, ws_bytes)
+    torch.cuda.synchronize()
+    st, info = B.moe_get_device_error()
+    assert st == 0, (B.status_str(st), info)
+    ref = _expert_step_reference(c, inp, np_(dyp), dy)
+    tol = tol_of(c)
+    outs = dict(grads, dx=dx)
+    for n, t in outs.items():
+        a = np_(t)
+        assert np.isfinite(a).all(), n
+        assert rel_err(a, ref[n]) <= tol, n
+
+
 def test_expert_backward_unsupported_configurations():
     """fp32 layers are refused on the host (MOE_ERR_UNSUPPORTED)."""
     for c in (get_config("tiny_f32"), EDGE["f32_sigmoid_cap"]):
