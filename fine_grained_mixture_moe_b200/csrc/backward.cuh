@@ -458,10 +458,13 @@ __global__ void __launch_bounds__(256) router_dgrad_kernel(const float *__restri
 
 // ------------------------------------------------------------------ expert steps of the backward
 // The weight gradients are products over a group's rows (dW_d[e] = dY_e^T h_e, dW_g[e] =
-// dg_e^T X_e, dW_u[e] = du_e^T X_e). The tensor cores take both operands K-major, so the grouped
-// activations are transposed first, each expert's rows padded with zeros to a multiple of 64 so
-// that no 64-wide k-block crosses into the next expert; the weights are transposed for the data
-// gradients (dh = dY W_d, dX = [dg | du] [W_g; W_u]) the same way.
+// dg_e^T X_e, dW_u[e] = du_e^T X_e). For SwiGLU layers the tensor cores read both operands
+// MN-major from the row-major activations, in 64-row K-blocks aligned to each expert's last row
+// (kstart below); h and [dg | du] are written with zero rows in front of each expert's rows, so
+// the rows a block reads before the expert's first row contribute nothing. The low-rank layers'
+// activations are still transposed into K-major copies, each expert's rows padded with zeros to a
+// multiple of 64; the weights are transposed for the data gradients (dh = dY W_d,
+// dX = [dg | du] [W_g; W_u]) the same way.
 
 // koff[e] = sum over e' < e of the expert's row count rounded up to 64; koff[E] is the total.
 // kstart[e] = offsets[e+1] - (koff[e+1] - koff[e]): the row of the grouped activations at which
